@@ -1,0 +1,455 @@
+"""Benchmark of the FP8 MoE quantisation + grouped-GEMM hot path on B200.
+
+One step = one pass of the whole path over the dense Llama3-8B FFN
+up-projection workload (one expert group, X [8192, 4096] bf16, W [14336,
+4096] bf16): rowwise quantisation of X (one scale per token), rowwise
+quantisation of W (one scale per output channel), FP8 scaled grouped GEMM
+(fp32 out).  ``value`` is the step's throughput in GEMM-equivalent TFLOP/s
+(2*M*N*K per step divided by the whole step time, quantisation included);
+the per-kernel figures (quantisation GB/s, GEMM TFLOP/s, fractions of the
+measured peaks) sit beside it.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+Multi-GPU (torchrun, one process per GPU): every rank runs its own replica of
+the workload (the path has no exchange step; weak scaling); the timed region
+is bracketed by a barrier and a device synchronise, and the time is the max
+over ranks.  ``--impl reference`` times the CPU oracle (single thread) on a
+bounded sample of the same workload, on rank 0 only.
+"""
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from quantization_grouped_gemm_b200 import workloads as wl  # noqa: E402
+
+METRIC = "fused FP8 quant GB/s (% HBM peak); FP8 grouped GEMM TFLOP/s (% peak)"
+L2_BYTES = 126 * 1024 * 1024
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return dict(hbm_gbs=float(p["hbm_gbs"]), bf16=float(p["bf16_tflops"]),
+                    bf16_sustained=float(p.get("bf16_tflops_sustained", p["bf16_tflops"])),
+                    source="measured")
+    except Exception:
+        return dict(hbm_gbs=6650.0, bf16=1590.0, bf16_sustained=1400.0, source="fallback")
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason sampling during the timed region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            time.sleep(0.15)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        if self.proc is None or not self.path:
+            return None
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    rows.append(dict(sm=float(parts[1]), smax=float(parts[2]),
+                                     power=float(parts[3]) if parts[3] not in ("", "[N/A]") else 0.0,
+                                     hw=parts[5], hwt=parts[6], swt=parts[7], pcap=parts[8]))
+                except ValueError:
+                    continue
+        os.unlink(self.path)
+        if not rows:
+            return None
+        loaded = [r for r in rows if r["power"] > 200.0] or rows
+        reasons = set()
+        for r in loaded:
+            for key, name in (("hw", "hw_slowdown"), ("hwt", "hw_thermal_slowdown"),
+                              ("swt", "sw_thermal_slowdown"), ("pcap", "sw_power_cap")):
+                if r[key].lower() == "active":
+                    reasons.add(name)
+        return dict(sm_mhz=statistics.median(r["sm"] for r in loaded),
+                    sm_max_mhz=max(r["smax"] for r in loaded), reasons=sorted(reasons),
+                    samples=len(loaded))
+
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1 and not torch.distributed.is_initialized():
+        import datetime
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+        torch.distributed.init_process_group(backend=backend,
+                                             timeout=datetime.timedelta(seconds=120))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def max_over_ranks(v, world):
+    if world == 1:
+        return v
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    t = torch.tensor([v], dtype=torch.float64, device=dev)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ----------------------------------------------------------------------------- CPU oracle
+def oracle_sample(w, rows_x, rows_w, n_elem, seed=0):
+    """Times the oracle on a bounded sample: rowwise quantisation of rows_x rows
+    of X and rows_w rows of W, and n_elem GEMM outputs built from them.
+    Returns (seconds for the sample, seconds extrapolated to one full step)."""
+    import oracle as orc
+    m, k = w.x.shape
+    n = w.w.shape[1]
+    g = np.random.default_rng(seed)
+    xr = np.sort(g.choice(m, rows_x, replace=False))
+    wr = np.sort(g.choice(n, rows_w, replace=False))
+    xb = wl.bf16_bits(w.x)[xr]
+    wb = wl.bf16_bits(w.w.reshape(n, k))[wr]
+    t0 = time.perf_counter()
+    qa, sa, _ = orc.quant_rowwise(xb)
+    t1 = time.perf_counter()
+    qb, sb, _ = orc.quant_rowwise(wb)
+    t2 = time.perf_counter()
+    ri = g.integers(0, rows_x, n_elem)
+    ci = g.integers(0, rows_w, n_elem)
+    orc.gemm_m_jagged_sample(qa, sa, qb[None], sb[None], np.array([rows_x], np.int32), ri, ci)
+    t3 = time.perf_counter()
+    full = (t1 - t0) * m / rows_x + (t2 - t1) * n / rows_w + (t3 - t2) * (m * n) / n_elem
+    return t3 - t0, full, dict(rows_x=rows_x, rows_w=rows_w, gemm_outputs=n_elem)
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return 0
+    w = wl.llama3_8b_up_proj()
+    m, k = w.x.shape
+    n = w.w.shape[1]
+    flops = 2.0 * m * n * k
+    rows_x, rows_w, n_elem = 128, 128, 1500
+    for _ in range(args.warmup):
+        oracle_sample(w, rows_x, rows_w, n_elem)
+    fulls = []
+    t_sample = 0.0
+    for i in range(args.steps):
+        s, full, desc = oracle_sample(w, rows_x, rows_w, n_elem, seed=i + 1)
+        t_sample += s
+        fulls.append(full)
+    t_step = statistics.mean(fulls)
+    value = flops / t_step / 1e12
+    sample = (f"per step: oracle rowwise quantisation of {rows_x} X rows and {rows_w} W rows, "
+              f"{n_elem} fp64 GEMM outputs; time extrapolated to the full step by rows and "
+              f"outputs")
+    line = dict(metric=METRIC, value=value, unit="TFLOP/s", n_gpus=args.gpus, steps=args.steps,
+                warmup=args.warmup, ms_per_step=t_step * 1e3, higher_is_better=True,
+                scaling="weak", vs_baseline=None, dtype="f32 quantisation / f64 GEMM",
+                data="synthetic", impl="reference", config=config_dict(w),
+                cpu_baseline=dict(value=value, unit="TFLOP/s", cores=1, kind="oracle",
+                                  sample=sample),
+                e2e=dict(value=value, unit="TFLOP/s", h2d_bytes_per_step=0,
+                         d2h_bytes_per_step=0))
+    print(json.dumps(line))
+    return 0
+
+
+def config_dict(w, Step=None):
+    m, k = w.x.shape
+    d = dict(workload=w.name, M=m, K=k, E=w.num_groups, fmt="e4m3fn", gemm_out="fp32")
+    if w.grad_out is not None and Step is not None and Step.__name__ == "BackwardDwStep":
+        d.update(N=w.grad_out.shape[1],
+                 step=("jagged column-wise quant + transpose of grad_out and of X + "
+                       "contraction-jagged FP8 grouped GEMM (dW)"))
+    else:
+        d.update(N=w.w.shape[1],
+                 step=("rowwise quant X + rowwise quant W (per expert output channel) + "
+                       "token-jagged FP8 grouped GEMM"))
+    d["l2"] = ("no explicit flush: each step reads and writes more than the 126 MB L2 "
+               "(bf16 inputs plus fp32 output)")
+    return d
+
+
+# ----------------------------------------------------------------------------- GPU arm
+class ForwardStep:
+    """Token-jagged forward: rowwise X, rowwise W viewed [E*N, K] (one scale per
+    expert output channel), FP8 grouped GEMM (fp32 out)."""
+
+    def __init__(self, w):
+        import quantization_grouped_gemm_b200 as qgg
+        self.qgg = qgg
+        self.w = w
+        m, k = w.x.shape
+        e, n = w.w.shape[0], w.w.shape[1]
+        self.m, self.n, self.k, self.e = m, n, k, e
+        self.x = w.x.cuda()
+        self.wt = w.w.reshape(e * n, k).cuda()
+        self.off = torch.from_numpy(w.offsets).cuda()
+        self.qa = torch.empty((m, k), dtype=torch.uint8, device="cuda")
+        self.sa = torch.empty((m,), dtype=torch.float32, device="cuda")
+        self.qb = torch.empty((e * n, k), dtype=torch.uint8, device="cuda")
+        self.sb = torch.empty((e * n,), dtype=torch.float32, device="cuda")
+        self.out = torch.empty((m, n), dtype=torch.float32, device="cuda")
+        rows = int(np.asarray(w.offsets)[-1]) if len(w.offsets) else 0
+        self.flops = 2.0 * rows * n * k
+        self.names = ["quant_rowwise_x", "quant_rowwise_w", "grouped_gemm"]
+        self.bytes = [m * k * 3 + m * 4, e * n * k * 3 + e * n * 4, None]
+        self.host_inputs = [(self.x, w.x), (self.wt, w.w.reshape(e * n, k))]
+        self.result = self.out
+
+    def kernels(self):
+        q = self.qgg
+        e, n, k = self.e, self.n, self.k
+        return [
+            lambda: q.fp8_quant_rowwise(self.x, q=self.qa, scales=self.sa),
+            lambda: q.fp8_quant_rowwise(self.wt, q=self.qb, scales=self.sb),
+            lambda: q.fp8_scaled_grouped_gemm(q.M_JAGGED, self.qa, self.sa,
+                                              self.qb.view(e, n, k), self.sb.view(e, n),
+                                              self.off, out=self.out),
+        ]
+
+
+class BackwardDwStep:
+    """Contraction-jagged weight gradient: jagged column-wise quantisation with
+    fused transpose of grad_out [M, N] and of X [M, K], then dW_e = dH_e^T X_e."""
+
+    def __init__(self, w):
+        import quantization_grouped_gemm_b200 as qgg
+        self.qgg = qgg
+        self.w = w
+        m, k = w.x.shape
+        n = w.grad_out.shape[1]
+        e = w.num_groups
+        self.m, self.n, self.k, self.e = m, n, k, e
+        self.g = w.grad_out.cuda()
+        self.x = w.x.cuda()
+        self.off = torch.from_numpy(w.offsets).cuda()
+        ld = (m + 15) // 16 * 16
+        self.qg = torch.empty((n, ld), dtype=torch.uint8, device="cuda")
+        self.qx = torch.empty((k, ld), dtype=torch.uint8, device="cuda")
+        self.sg = torch.empty((e, n), dtype=torch.float32, device="cuda")
+        self.sx = torch.empty((e, k), dtype=torch.float32, device="cuda")
+        self.wsg = torch.empty(qgg.colwise_workspace_bytes(m, n, e), dtype=torch.uint8,
+                               device="cuda")
+        self.wsx = torch.empty(qgg.colwise_workspace_bytes(m, k, e), dtype=torch.uint8,
+                               device="cuda")
+        self.out = torch.empty((e, n, k), dtype=torch.float32, device="cuda")
+        self.flops = 2.0 * m * n * k
+        self.names = ["quant_colwise_t_grad_out", "quant_colwise_t_x", "grouped_gemm"]
+        self.bytes = [m * n * 3 + e * n * 4 + e * 4, m * k * 3 + e * k * 4 + e * 4, None]
+        self.host_inputs = [(self.g, w.grad_out), (self.x, w.x)]
+        self.result = self.out
+
+    def kernels(self):
+        q = self.qgg
+        T = q.LAYOUT_TRANSPOSED
+        return [
+            lambda: q.fp8_quant_colwise_jagged(self.g, self.off, T, q=self.qg, scales=self.sg,
+                                               workspace=self.wsg),
+            lambda: q.fp8_quant_colwise_jagged(self.x, self.off, T, q=self.qx, scales=self.sx,
+                                               workspace=self.wsx),
+            lambda: q.fp8_scaled_grouped_gemm(q.K_JAGGED, self.qg, self.sg, self.qx, self.sx,
+                                              self.off, m_total=self.m, out=self.out),
+        ]
+
+
+WORKLOADS = {
+    "llama3_8b_up_proj": (lambda: wl.llama3_8b_up_proj(), ForwardStep),
+    "tiny_moe": (lambda: wl.tiny_moe(), ForwardStep),
+    "deepseek_moe16b_bwd": (lambda: wl.deepseek_moe_16b_backward(), BackwardDwStep),
+    "deepseek_v3_fwd": (lambda: wl.deepseek_v3_local_experts(), ForwardStep),
+    "llama4_m8192_zipf": (lambda: wl.llama4_sweep(8192, "zipf"), ForwardStep),
+    "llama4_m131072_uniform": (lambda: wl.llama4_sweep(131072, "uniform"), ForwardStep),
+}
+
+
+def run_gpu(args, world, rank, local):
+    pk = peaks()
+    make, Step = WORKLOADS[args.workload]
+    w = make()
+    st = Step(w)
+    ks = st.kernels()
+    nk = len(ks)
+
+    def step(ev=None):
+        for i, f in enumerate(ks):
+            if ev is not None:
+                ev[i].record()
+            f()
+        if ev is not None:
+            ev[nk].record()
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nk + 1)]
+           for _ in range(args.steps)]
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        t_start.record()
+        for i in range(args.steps):
+            step(evs[i])
+        t_end.record()
+        torch.cuda.synchronize()
+    barrier(world)
+    total_ms = max_over_ranks(t_start.elapsed_time(t_end), world)
+    ms_step = total_ms / args.steps
+    k_ms = [statistics.mean(e[i].elapsed_time(e[i + 1]) for e in evs) for i in range(nk)]
+    clocks = clk.summary()
+
+    # end to end through the public API with host buffers: pinned H2D of the
+    # step's inputs, the step's calls, D2H of the result, every step
+    pinned = [(d, h.contiguous().pin_memory()) for d, h in st.host_inputs]
+    hout = torch.empty(st.result.shape, dtype=st.result.dtype).pin_memory()
+    e2e_steps = max(2, min(args.steps, 5))
+
+    def e2e_step():
+        for d, h in pinned:
+            d.copy_(h.view(d.shape), non_blocking=True)
+        step()
+        hout.copy_(st.result, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    barrier(world)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record()
+    torch.cuda.synchronize()
+    barrier(world)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world) / e2e_steps
+
+    flops = st.flops
+    value = flops * world / (ms_step * 1e-3) / 1e12
+    gm_ms = k_ms[-1]
+    gemm_tflops = flops / (gm_ms * 1e-3) / 1e12
+    fp8_peak = 2.0 * pk["bf16"]
+    q_bytes = sum(b for b in st.bytes if b)
+    q_ms = sum(k_ms[:-1])
+    quant_gbs = q_bytes / (q_ms * 1e-3) / 1e9
+    kern = {}
+    for name, b, t in zip(st.names, st.bytes, k_ms):
+        if b:
+            gbs = b / (t * 1e-3) / 1e9
+            kern[name] = dict(us=t * 1e3, gbs=gbs, frac_hbm=gbs / pk["hbm_gbs"],
+                              algorithmic_bytes=b)
+        else:
+            kern[name] = dict(us=t * 1e3, tflops=gemm_tflops, frac_fp8=gemm_tflops / fp8_peak,
+                              flops=flops)
+    kern.update(quant_gbs=quant_gbs, quant_frac_hbm=quant_gbs / pk["hbm_gbs"],
+                hbm_peak_gbs=pk["hbm_gbs"], fp8_peak_tflops=fp8_peak)
+    line = dict(
+        metric=METRIC, value=value, unit="TFLOP/s", n_gpus=world, steps=args.steps,
+        warmup=args.warmup, ms_per_step=ms_step, higher_is_better=True, scaling="weak",
+        vs_baseline=None, dtype="fp8_e4m3", data="synthetic", config=config_dict(w, Step),
+        roofline=dict(bound="tensor", achieved=gemm_tflops, peak=fp8_peak, unit="TFLOP/s",
+                      frac=gemm_tflops / fp8_peak, traffic=TRAFFIC.get(args.workload),
+                      peak_note=(f"{pk['source']} bf16 burst {pk['bf16']} TFLOP/s x 2 "
+                                 "(nominal fp8:bf16 dense ratio)")),
+        kernels=kern,
+        e2e=dict(value=flops * world / (e2e_ms * 1e-3) / 1e12, unit="TFLOP/s",
+                 h2d_bytes_per_step=int(sum(h.numel() * h.element_size() for _, h in pinned)),
+                 d2h_bytes_per_step=int(hout.numel() * hout.element_size()), ms_per_step=e2e_ms),
+        gpu_launches=nk * args.steps,
+        clocks=clocks,
+    )
+    if rank == 0 and world == 1 and Step is ForwardStep and not args.no_cpu_baseline:
+        _, full, desc = oracle_sample(w, min(8192, st.m), min(8192, st.e * st.n), 120000)
+        cpu_v = flops / full / 1e12
+        line["cpu_baseline"] = dict(
+            value=cpu_v, unit="TFLOP/s", cores=1, kind="oracle",
+            sample=(f"oracle (1 thread) rowwise quantisation of {desc['rows_x']} X rows and "
+                    f"{desc['rows_w']} W rows plus {desc['gemm_outputs']} fp64 GEMM outputs, "
+                    "extrapolated to one full step"))
+    if rank == 0:
+        print(json.dumps(line))
+    return 0
+
+
+# DRAM bytes per launch of the grouped GEMM from an ncu capture of the same
+# command (dram__bytes_read.sum + dram__bytes_write.sum); None until captured
+# for the current kernel.
+TRAFFIC = {}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="llama3_8b_up_proj", choices=sorted(WORKLOADS))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.impl == "reference":
+        # the CPU oracle runs on rank 0 alone; no process group is needed
+        rank = int(os.environ.get("RANK", "0"))
+        return run_reference(args, int(os.environ.get("WORLD_SIZE", "1")), rank)
+    world, rank, local = dist_setup(args)
+    try:
+        if True:
+            if not torch.cuda.is_available():
+                raise RuntimeError("bench.py needs a CUDA device for the GPU arm")
+            rc = run_gpu(args, world, rank, local)
+    finally:
+        if world > 1 and torch.distributed.is_initialized():
+            torch.distributed.destroy_process_group()
+    return rc
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,212 @@
+/*
+ * fp8qgg — FP8 training quantisation for MoE expert GEMMs and the FP8 scaled
+ * grouped GEMM that consumes it, for NVIDIA B200 (sm_100a).
+ *
+ * C ABI.  Every tensor argument is a DEVICE pointer owned by the caller; the
+ * library keeps no state between calls and every call is enqueued on `stream`
+ * (a cudaStream_t passed as void*; NULL = the legacy default stream) with no
+ * implicit synchronisation.  Unless a function says otherwise it allocates no
+ * device memory.
+ *
+ * Sources, cited by page title and section:
+ *  [AIR] "FP8 su GPU AMD: i guadagni di TorchTitan e TorchAO ora sono nel
+ *        mainline PyTorch" (ai-radar.it)
+ *  [ABP] "AMD Boosts PyTorch FP8 Training on Instinct GPUs" (latestnews.news)
+ *  [PRI] "AMD Primus adds FP8/MXFP8 kernels, megakernel fusion and DeepSeek-V3
+ *        training at 1024 GPUs" (fosswire.org)
+ *
+ * Conventions shared by every entry point
+ *  - Formats: FP8QGG_E4M3FN (largest finite 448, signed zero, NaN S.1111.111)
+ *    is the default; FP8QGG_E4M3FNUZ (largest finite 240, single zero, only
+ *    NaN 0x80) is the format of [AIR] section "La correttezza del formato viene
+ *    prima del tuning" and [ABP] third paragraph.  Scaling against the wrong
+ *    maximum clips silently; `scale_max` reproduces that case on purpose and
+ *    `sat_count` makes it observable.
+ *  - Quantisation chain ([AIR] section "Il guadagno vero è nel movimento dei
+ *    dati", first paragraph), all in one pass over HBM:
+ *        amax = max |x|                       (exact)
+ *        s    = fp32(Fmax / max(amax, 1e-12)) (IEEE round to nearest)
+ *        y    = clamp(fp32(x * s), -Fmax, Fmax)
+ *        q    = e4m3(y)   round to nearest, ties to even, one rounding from
+ *                         fp32, saturating; e4m3fnuz maps every zero to 0x00.
+ *    Fmax = scale_max when scale_max > 0, else the format's largest finite.
+ *    The stored scale is s (dequantise with decode(q) / s).
+ *  - Offsets ([AIR] introduction, second paragraph: an offsets tensor routes
+ *    tokens to experts): int32[num_groups] of CUMULATIVE group ends, no
+ *    leading zero, device memory.  Group e spans rows [start_e, end_e) with
+ *    start_0 = 0, start_e = end_{e-1}, end_e = clamp(offsets[e], start_e,
+ *    rows_total).  Malformed offsets (decreasing, negative, beyond rows_total)
+ *    are clamped that way on the device, so no access leaves the buffers, and
+ *    FP8QGG_STATUS_BAD_OFFSETS is OR-ed into *dev_status when it is given.
+ *    Rows past the last end belong to no group and are not written.
+ *  - sat_count (nullable, device uint64): the kernel ADDS the number of
+ *    elements whose pre-clamp |y| is more than one fp32 ulp above the
+ *    encoding's largest finite value.  Zero it before the call.
+ *  - dev_status (nullable, device int32): the kernel ORs FP8QGG_STATUS_* bits.
+ *    Zero it before the call; read it after the stream has synchronised.
+ *  - Return value: FP8QGG_OK or one of the negative FP8QGG_ERR_* codes below.
+ *    Argument errors are detected on the host before anything is enqueued.
+ */
+#ifndef FP8QGG_H
+#define FP8QGG_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* return codes */
+#define FP8QGG_OK 0
+#define FP8QGG_ERR_NULL (-1)        /* a required pointer is NULL */
+#define FP8QGG_ERR_SHAPE (-2)       /* bad size, leading dimension or group count */
+#define FP8QGG_ERR_ALIGN (-3)       /* base pointer or leading dimension misaligned */
+#define FP8QGG_ERR_UNSUPPORTED (-4) /* bad flag or unsupported combination */
+#define FP8QGG_ERR_CUDA (-5)        /* a CUDA runtime/driver call failed */
+
+/* formats */
+#define FP8QGG_E4M3FN 0
+#define FP8QGG_E4M3FNUZ 1
+
+/* output layouts of the jagged column-wise quantisation */
+#define FP8QGG_LAYOUT_SAME 0
+#define FP8QGG_LAYOUT_TRANSPOSED 1
+
+/* grouped GEMM modes */
+#define FP8QGG_M_JAGGED 0 /* groups split the rows of A and of the output */
+#define FP8QGG_K_JAGGED 1 /* groups split the contraction axis */
+
+/* grouped GEMM output types */
+#define FP8QGG_OUT_F32 0
+#define FP8QGG_OUT_BF16 1
+
+/* bits OR-ed into *dev_status */
+#define FP8QGG_STATUS_BAD_OFFSETS 1  /* offsets had to be clamped */
+#define FP8QGG_STATUS_TIMEOUT 2      /* a bounded device-side wait gave up */
+#define FP8QGG_STATUS_GROUP_TOO_TALL 4 /* a group exceeded the single-pass limit */
+
+/* The FP8 variant this device's tensor cores consume.  The pages add
+ * automatic detection of the format because the wrong maximum corrupts
+ * results silently ([AIR] "La correttezza del formato viene prima del
+ * tuning"); on sm_100 the answer is always FP8QGG_E4M3FN. */
+int fp8_native_format(void);
+
+/* Short English text for a return code. */
+const char *fp8qgg_error_string(int code);
+
+/*
+ * Encode step alone: q[i] = e4m3(y[i]), round to nearest, ties to even, one
+ * rounding from fp32, saturating at the format's largest finite magnitude
+ * (no scaling, no clamp).  It is the cast at the end of the chain of [AIR]
+ * "Il guadagno vero è nel movimento dei dati", exposed for callers that bring
+ * their own scales and for exhaustive checks of the device encoder.  NaN
+ * inputs give unspecified codes.
+ *   y fp32 [n] (4-byte aligned), q uint8 [n]; n >= 0 (0 is a no-op).
+ */
+int fp8_cast_f32(const float *y, int64_t n, uint8_t *q, int fmt, void *stream);
+
+/*
+ * Rowwise quantisation: one scale per row ([AIR] introduction: activations
+ * take one scale per row).  Also the per-output-channel scale of a weight
+ * stored [N, K] (rows = output channels).
+ *   x      bf16 [rows, ld_x], row-major, read only.
+ *   q      uint8 e4m3 codes [rows, ld_q], written for columns [0, cols).
+ *   scales fp32 [rows], written.
+ * Requirements: rows >= 0; cols in [1, 32768] and a multiple of 8;
+ * ld_x >= cols and ld_x % 8 == 0; ld_q >= cols and ld_q % 8 == 0;
+ * x and q 16-byte aligned, scales 4-byte aligned.  rows == 0 is a no-op.
+ */
+int fp8_quant_rowwise(const void *x, int64_t rows, int64_t cols, int64_t ld_x,
+                      uint8_t *q, int64_t ld_q, float *scales,
+                      int fmt, float scale_max, uint64_t *sat_count, void *stream);
+
+/*
+ * Bytes of device workspace fp8_quant_colwise_jagged needs for this problem
+ * (cross-block absmax partials and arrival counters for groups taller than
+ * one block's on-chip chunk).  Always > 0.
+ */
+size_t fp8_quant_colwise_jagged_workspace_size(int64_t rows_total, int64_t cols,
+                                               int32_t num_groups);
+
+/*
+ * Jagged column-wise quantisation: for every expert group e and column c the
+ * absmax runs over the group's rows only, giving one scale per (e, c)
+ * ([AIR] introduction: one scale per column of each expert's weights; the
+ * backward applies the same per-group column scaling to gradients,
+ * [AIR] "Il guadagno vero è nel movimento dei dati", second paragraph).
+ *   x        bf16 [rows_total, ld_x], row-major, read once from HBM.
+ *   offsets  int32 [num_groups] cumulative group ends (device).
+ *   layout   FP8QGG_LAYOUT_SAME:       q[r * ld_q + c], ld_q >= cols, ld_q % 8 == 0.
+ *            FP8QGG_LAYOUT_TRANSPOSED: q[c * ld_q + r], ld_q >= rows_total,
+ *            ld_q % 16 == 0.  Group e occupies columns [start_e, end_e) of
+ *            every output row: the contraction axis of the weight-gradient
+ *            GEMM comes out contiguous, with no separate transposed copy
+ *            (the pages remove a .t().contiguous().t() round trip).
+ *   scales   fp32 [num_groups, cols]; an empty group gets Fmax / 1e-12 in
+ *            every column and no codes.
+ *   workspace, workspace_bytes: device scratch of at least
+ *            fp8_quant_colwise_jagged_workspace_size(...) bytes, 16-byte
+ *            aligned, owned by the caller; its contents on entry do not
+ *            matter (the call clears what it uses, on `stream`).  Calls that
+ *            share one workspace must be ordered on the device.
+ * Requirements: rows_total >= 0; cols in [1, 2^31) and a multiple of 8;
+ * num_groups in [1, 1024]; ld_x >= cols, ld_x % 8 == 0; x, q and workspace
+ * 16-byte aligned.  One group may hold at most (resident blocks) x 512 rows
+ * (about 150k rows on a B200); a taller group sets
+ * FP8QGG_STATUS_GROUP_TOO_TALL and its codes are not valid.
+ */
+int fp8_quant_colwise_jagged(const void *x, int64_t rows_total, int64_t cols, int64_t ld_x,
+                             const int32_t *offsets, int32_t num_groups,
+                             uint8_t *q, int64_t ld_q, int layout, float *scales,
+                             int fmt, float scale_max, uint64_t *sat_count,
+                             int32_t *dev_status, void *workspace, size_t workspace_bytes,
+                             void *stream);
+
+/*
+ * FP8 scaled grouped GEMM on the 5th-generation tensor cores (the pages run
+ * the expert GEMMs as one grouped GEMM over FP8 operands: [ABP] third
+ * paragraph; [PRI] "What Primus adds").  e4m3fn operands, fp32 accumulation.
+ * Group boundaries are read from `offsets` ON THE DEVICE: no host
+ * synchronisation on routing results.
+ *
+ * mode FP8QGG_M_JAGGED (forward, input gradient): rows of A and of the output
+ * are split into groups; group e multiplies with its own B_e.
+ *   out[m, n] = (sum_k A[m,k] * B_e[n,k]) / scale_a[m] / scale_b[e*sbs + n]
+ *   a        e4m3 [m_total, ld_a]            (K contiguous)
+ *   b        e4m3, B_e[n, k] at b[e*b_group_stride + n*ld_b + k]
+ *   scale_a  fp32 [m_total]                  (scale_a_group_stride unused)
+ *   scale_b  fp32, scale_b_group_stride (sbs) >= n
+ *   out      [m_total, ld_out] of out_dtype; rows outside every group are
+ *            not written (out_group_stride unused).
+ * mode FP8QGG_K_JAGGED (weight gradient): the contraction axis (tokens) is
+ * split into groups; one output matrix per group.
+ *   out[e, i, j] = (sum_{t in group e} A[i,t] * B[j,t]) / scale_a[e*sas + i] / scale_b[e*sbs + j]
+ *   a        e4m3 [n, ld_a], b e4m3 [k, ld_b]: the TRANSPOSED outputs of
+ *            fp8_quant_colwise_jagged (tokens contiguous), m_total tokens.
+ *   scale_a  fp32, group stride sas >= n;  scale_b fp32, group stride sbs >= k
+ *   out      [num_groups, n, ld_out] with group stride out_group_stride
+ *            (>= n * ld_out); an empty group's matrix is written as zeros.
+ *   b_group_stride unused.
+ * Requirements: fmt == FP8QGG_E4M3FN (the tensor cores have no e4m3fnuz
+ * input); m_total >= 0, n >= 1, k >= 1; num_groups in [1, 1024];
+ * a, b 16-byte aligned; ld_a, ld_b, b_group_stride multiples of 16;
+ * out 16-byte aligned; FP32 output needs n (M_JAGGED) or k (K_JAGGED) and
+ * ld_out multiples of 4, BF16 output multiples of 8.  The call returns
+ * FP8QGG_ERR_ALIGN or FP8QGG_ERR_SHAPE otherwise.
+ */
+int fp8_scaled_grouped_gemm(int mode,
+                            const uint8_t *a, int64_t ld_a, const float *scale_a,
+                            int64_t scale_a_group_stride,
+                            const uint8_t *b, int64_t ld_b, int64_t b_group_stride,
+                            const float *scale_b, int64_t scale_b_group_stride,
+                            const int32_t *offsets, int32_t num_groups,
+                            int64_t m_total, int64_t n, int64_t k,
+                            void *out, int64_t ld_out, int64_t out_group_stride, int out_dtype,
+                            int fmt, int32_t *dev_status, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FP8QGG_H */

@@ -37,6 +37,8 @@ def lib():
         L.oracle_fp8_decode.argtypes = [ctypes.c_uint8, ci]
         L.oracle_fp8_encode.restype = ctypes.c_uint8
         L.oracle_fp8_encode.argtypes = [f32, ci]
+        L.oracle_fp8_encode_array.restype = None
+        L.oracle_fp8_encode_array.argtypes = [P, i64, P, ci]
         L.oracle_fp8_max.restype = ctypes.c_double
         L.oracle_fp8_max.argtypes = [ci]
         L.oracle_group_bounds.restype = None
@@ -83,12 +85,10 @@ def encode(y: float, fmt: int) -> int:
 
 
 def encode_array(y, fmt: int) -> np.ndarray:
-    """Encode every element of an fp32 array (small inputs: one C call each)."""
-    flat = np.asarray(y, dtype=np.float32).ravel()
+    """Encode every element of an fp32 array (the C encoder in a plain loop)."""
+    flat = np.ascontiguousarray(np.asarray(y, dtype=np.float32).ravel())
     out = np.empty(flat.shape, dtype=np.uint8)
-    f = lib().oracle_fp8_encode
-    for i, v in enumerate(flat.tolist()):
-        out[i] = f(v, fmt)
+    lib().oracle_fp8_encode_array(_p(flat), flat.size, _p(out), fmt)
     return out.reshape(np.shape(y))
 
 

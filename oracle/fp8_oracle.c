@@ -300,3 +300,9 @@ void oracle_gemm_k_jagged_sample(const uint8_t *qa, int64_t ld_a, const float *s
         bound[s] = 1e-3 * mag;
     }
 }
+
+/* The encoder applied to every element of an fp32 array (plain loop). */
+void oracle_fp8_encode_array(const float *y, int64_t n, uint8_t *q, int fmt)
+{
+    for (int64_t i = 0; i < n; ++i) q[i] = oracle_fp8_encode(y[i], fmt);
+}

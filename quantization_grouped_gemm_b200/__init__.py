@@ -1,1 +1,228 @@
-"""B200-native FP8 quantisation and FP8 scaled grouped GEMM for MoE training."""
+"""B200-native FP8 quantisation and FP8 scaled grouped GEMM for MoE training.
+
+Thin Python binding over the C ABI in ``include/fp8qgg.h`` (``libfp8qgg.so``,
+built in-tree for sm_100a).  This module only marshals arguments: it turns
+torch CUDA tensors into device pointers, allocates outputs with torch and
+passes torch's current stream.  Every step of the computation runs in the
+library's CUDA kernels; there is no CPU or PyTorch fallback.  A missing or
+unloadable library raises ``RuntimeError``.
+"""
+import ctypes
+import os
+import threading
+
+import torch
+
+E4M3FN = 0
+E4M3FNUZ = 1
+LAYOUT_SAME = 0
+LAYOUT_TRANSPOSED = 1
+M_JAGGED = 0
+K_JAGGED = 1
+OUT_F32 = 0
+OUT_BF16 = 1
+STATUS_BAD_OFFSETS = 1
+STATUS_TIMEOUT = 2
+STATUS_GROUP_TOO_TALL = 4
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libfp8qgg.so")
+_lib = None
+_lock = threading.Lock()
+
+_P = ctypes.c_void_p
+_I64 = ctypes.c_int64
+_I32 = ctypes.c_int32
+_INT = ctypes.c_int
+_F32 = ctypes.c_float
+_SZ = ctypes.c_size_t
+
+_SIGNATURES = {
+    "fp8_native_format": (_INT, []),
+    "fp8qgg_error_string": (ctypes.c_char_p, [_INT]),
+    "fp8_quant_rowwise": (_INT, [_P, _I64, _I64, _I64, _P, _I64, _P, _INT, _F32, _P, _P]),
+    "fp8_quant_colwise_jagged_workspace_size": (_SZ, [_I64, _I64, _I32]),
+    "fp8_quant_colwise_jagged": (_INT, [_P, _I64, _I64, _I64, _P, _I32, _P, _I64, _INT, _P,
+                                        _INT, _F32, _P, _P, _P, _SZ, _P]),
+    "fp8_scaled_grouped_gemm": (_INT, [_INT, _P, _I64, _P, _I64, _P, _I64, _I64, _P, _I64, _P,
+                                       _I32, _I64, _I64, _I64, _P, _I64, _I64, _INT, _INT, _P,
+                                       _P]),
+    "fp8_cast_f32": (_INT, [_P, _I64, _P, _INT, _P]),
+}
+
+
+def lib():
+    """The loaded C library (built in-tree on first use if absent)."""
+    global _lib
+    if _lib is None:
+        with _lock:
+            if _lib is None:
+                if not os.path.exists(LIB_PATH):
+                    from . import build as _build
+                    _build.build()
+                try:
+                    L = ctypes.CDLL(LIB_PATH)
+                except OSError as e:
+                    raise RuntimeError(f"fp8qgg CUDA library could not be loaded: {e}") from e
+                for name, (res, args) in _SIGNATURES.items():
+                    f = getattr(L, name)
+                    f.restype = res
+                    f.argtypes = args
+                _lib = L
+    return _lib
+
+
+class Fp8qggError(RuntimeError):
+    pass
+
+
+def _check(rc: int, what: str):
+    if rc != 0:
+        msg = lib().fp8qgg_error_string(rc).decode()
+        raise Fp8qggError(f"{what} failed with status {rc}: {msg}")
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _ld(t):
+    """Leading dimension (elements between rows) of a row-major 2-D tensor; for a
+    tensor with at most one row the row stride is irrelevant and the width is used."""
+    if t.shape[0] <= 1:
+        return t.shape[1]
+    assert t.stride(1) == 1 or t.shape[1] <= 1, "rows must be contiguous"
+    return t.stride(0)
+
+
+def _need_cuda(*ts):
+    for t in ts:
+        if t is not None and not t.is_cuda:
+            raise ValueError("fp8qgg operates on CUDA tensors only")
+
+
+def native_format() -> int:
+    return lib().fp8_native_format()
+
+
+def fp8_quant_rowwise(x, fmt=E4M3FN, scale_max=0.0, q=None, scales=None, sat_count=None,
+                      stream=None):
+    """Rowwise quantisation of a bf16 [rows, cols] CUDA tensor (row stride may exceed cols).
+
+    Returns (q uint8 [rows, cols], scales fp32 [rows])."""
+    _need_cuda(x)
+    assert x.dtype == torch.bfloat16 and x.dim() == 2
+    rows, cols = x.shape
+    if q is None:
+        q = torch.empty((rows, cols), dtype=torch.uint8, device=x.device)
+    if scales is None:
+        scales = torch.empty((rows,), dtype=torch.float32, device=x.device)
+    _need_cuda(q, scales, sat_count)
+    rc = lib().fp8_quant_rowwise(_ptr(x), rows, cols, _ld(x), _ptr(q), _ld(q),
+                                 _ptr(scales), fmt, float(scale_max), _ptr(sat_count),
+                                 _stream(stream))
+    _check(rc, "fp8_quant_rowwise")
+    return q, scales
+
+
+def colwise_workspace_bytes(rows_total, cols, num_groups) -> int:
+    return int(lib().fp8_quant_colwise_jagged_workspace_size(rows_total, cols, num_groups))
+
+
+def fp8_quant_colwise_jagged(x, offsets, layout=LAYOUT_SAME, fmt=E4M3FN, scale_max=0.0,
+                             q=None, ld_q=None, scales=None, workspace=None, sat_count=None,
+                             status=None, stream=None):
+    """Per-(group, column) quantisation of a bf16 [rows_total, cols] CUDA tensor.
+
+    offsets: int32 CUDA tensor of cumulative group ends.  Returns (q, scales)
+    with q [rows_total, cols] (SAME) or [cols, ld_q] (TRANSPOSED), scales
+    fp32 [num_groups, cols]."""
+    _need_cuda(x, offsets)
+    assert x.dtype == torch.bfloat16 and x.dim() == 2
+    assert offsets.dtype == torch.int32
+    rows, cols = x.shape
+    e = offsets.numel()
+    if q is None:
+        if layout == LAYOUT_TRANSPOSED:
+            ld = ld_q if ld_q is not None else (rows + 15) // 16 * 16
+            q = torch.empty((cols, ld), dtype=torch.uint8, device=x.device)
+        else:
+            q = torch.empty((rows, cols), dtype=torch.uint8, device=x.device)
+    if scales is None:
+        scales = torch.empty((e, cols), dtype=torch.float32, device=x.device)
+    if workspace is None:
+        workspace = torch.empty(colwise_workspace_bytes(rows, cols, e), dtype=torch.uint8,
+                                device=x.device)
+    _need_cuda(q, scales, workspace, sat_count, status)
+    rc = lib().fp8_quant_colwise_jagged(
+        _ptr(x), rows, cols, _ld(x), _ptr(offsets), e, _ptr(q), _ld(q), layout,
+        _ptr(scales), fmt, float(scale_max), _ptr(sat_count), _ptr(status), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(rc, "fp8_quant_colwise_jagged")
+    return q, scales
+
+
+def fp8_scaled_grouped_gemm(mode, a, scale_a, b, scale_b, offsets, m_total=None, n=None, k=None,
+                            out=None, out_dtype=torch.float32, status=None, b_group_stride=None,
+                            stream=None):
+    """FP8 scaled grouped GEMM (see the C header for the two modes).
+
+    M_JAGGED: a uint8 [m_total, K], scale_a [m_total], b uint8 [E, N, K] (or any
+    layout with b_group_stride), scale_b [E, N] -> out [m_total, N].
+    K_JAGGED: a uint8 [N, ld_a], b uint8 [K, ld_b] (token axis contiguous),
+    scale_a [E, N], scale_b [E, K], m_total tokens -> out [E, N, K]."""
+    _need_cuda(a, scale_a, b, scale_b, offsets)
+    assert a.dtype == torch.uint8 and b.dtype == torch.uint8 and offsets.dtype == torch.int32
+    e = offsets.numel()
+    if out is not None:
+        out_dtype = out.dtype
+    assert out_dtype in (torch.float32, torch.bfloat16)
+    odt = OUT_F32 if out_dtype == torch.float32 else OUT_BF16
+    if mode == M_JAGGED:
+        m_total = a.shape[0] if m_total is None else m_total
+        k = a.shape[1] if k is None else k
+        if b.dim() == 3:
+            n = b.shape[1] if n is None else n
+            ld_b = b.stride(1)
+            bgs = b.stride(0) if b_group_stride is None else b_group_stride
+        else:
+            n = b.shape[0] // e if n is None else n
+            ld_b = b.stride(0)
+            bgs = n * ld_b if b_group_stride is None else b_group_stride
+        sbs = scale_b.shape[-1] if scale_b.dim() == 2 else n
+        if out is None:
+            out = torch.empty((m_total, n), dtype=out_dtype, device=a.device)
+        ld_out, ogs, sas, ld_a = _ld(out), 0, 0, _ld(a)
+    else:
+        n = a.shape[0] if n is None else n
+        k = b.shape[0] if k is None else k
+        assert m_total is not None
+        ld_a, ld_b, bgs = _ld(a), _ld(b), 0
+        sas = scale_a.shape[-1]
+        sbs = scale_b.shape[-1]
+        if out is None:
+            out = torch.empty((e, n, k), dtype=out_dtype, device=a.device)
+        ld_out, ogs = out.stride(-2), out.stride(0)
+    _need_cuda(out, status)
+    rc = lib().fp8_scaled_grouped_gemm(
+        mode, _ptr(a), ld_a, _ptr(scale_a), sas, _ptr(b), ld_b, bgs, _ptr(scale_b), sbs,
+        _ptr(offsets), e, m_total, n, k, _ptr(out), ld_out, ogs, odt, E4M3FN, _ptr(status),
+        _stream(stream))
+    _check(rc, "fp8_scaled_grouped_gemm")
+    return out
+
+
+def fp8_cast_f32(y, fmt=E4M3FN, q=None, sat_count=None, stream=None):
+    """Round-to-nearest-even saturating cast of an fp32 CUDA tensor to e4m3 codes."""
+    _need_cuda(y)
+    assert y.dtype == torch.float32 and y.is_contiguous()
+    if q is None:
+        q = torch.empty(y.shape, dtype=torch.uint8, device=y.device)
+    rc = lib().fp8_cast_f32(_ptr(y), y.numel(), _ptr(q), fmt, _stream(stream))
+    _check(rc, "fp8_cast_f32")
+    return q

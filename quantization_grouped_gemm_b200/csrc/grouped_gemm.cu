@@ -1,0 +1,541 @@
+// FP8 scaled grouped GEMM on the B200 5th-generation tensor cores.
+//
+// The pages run the MoE expert GEMMs as one grouped GEMM over FP8 operands
+// whose groups come from the token offsets ("AMD Boosts PyTorch FP8 Training
+// on Instinct GPUs", third paragraph; "AMD Primus adds FP8/MXFP8 kernels ...",
+// "What Primus adds for MoE training on MI355X": FP8 grouped GEMM and
+// sync-free MoE execution).  This kernel reads the offsets on the device and
+// never synchronises with the host.
+//
+// Structure (one persistent CTA per SM, 6 warps):
+//   warp 0      TMA producer: A and B tiles, 128 bytes of K per row, 128-byte
+//               swizzle, into a 4-stage shared-memory ring (mbarrier full /
+//               empty pairs).
+//   warp 1      allocates 512 TMEM columns (two 128 x 256 fp32 accumulators)
+//               and issues tcgen05.mma kind::f8f6f4 (M128 N256 K32) from one
+//               lane; tcgen05.commit frees ring stages and publishes finished
+//               accumulators.  In the contraction-jagged mode it also zeroes,
+//               in shared memory, the token columns of a tile that fall
+//               outside the group (group edges need not be 16-aligned, TMA
+//               coordinates must be).
+//   warps 2-5   epilogue: tcgen05.ld of their 32 TMEM lanes, multiply by
+//               1/scale_a (row) and 1/scale_b (column), masked stores.  With
+//               two accumulators the epilogue of tile i overlaps the
+//               mainloop of tile i+1.
+// Tiles are enumerated group by group; in the token-jagged mode the N tiles
+// of one M tile are consecutive so that concurrent CTAs share the A rows in
+// L2 and the whole B_e stays L2-resident across the group.
+#include <algorithm>
+
+#include "device_common.cuh"
+#include "host_common.h"
+
+namespace fp8qgg {
+
+constexpr int BM = 128;
+constexpr int BN = 256;
+constexpr int BK = 128;  // bytes of K per stage row = one 128-byte swizzle atom
+constexpr int kStages = 4;
+constexpr int kGemmThreads = 192;
+constexpr int kEpiThreads = 128;
+constexpr int kMaxGemmGroups = 1024;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kStageBytes = (BM + BN) * BK;
+constexpr uint32_t kIdesc = idesc_e4m3_f32(BM, BN);
+
+struct GemmSmem {
+  uint8_t a[kStages][BM * BK];  // 16 KB each, 1024-aligned (swizzle atoms)
+  uint8_t b[kStages][BN * BK];  // 32 KB each
+  float inv_sb[2][BN];
+  int32_t end[kMaxGemmGroups];
+  int32_t tile_prefix[kMaxGemmGroups + 1];
+  uint64_t full[kStages];
+  uint64_t empty[kStages];
+  uint64_t tfull[2];
+  uint64_t tempty[2];
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort;
+};
+
+struct GemmParams {
+  const float *scale_a;
+  int64_t sas;  // scale_a group stride (contraction-jagged mode)
+  const float *scale_b;
+  int64_t sbs;  // scale_b group stride
+  const int32_t *offsets;
+  int num_groups;
+  int64_t m_total, n, k;
+  void *out;
+  int64_t ld_out;
+  int64_t out_gs;  // output group stride (contraction-jagged mode)
+  int32_t *status;
+};
+
+struct TileInfo {
+  int e;       // group
+  int tm, tn;  // tile coordinates inside the group
+  int32_t gstart, gend;
+  int nk;  // k blocks
+};
+
+template <int MODE>
+__device__ __forceinline__ TileInfo decode_tile(const GemmSmem &sm, const GemmParams &p,
+                                                int32_t t) {
+  int lo = 0, hi = p.num_groups - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (sm.tile_prefix[mid] <= t) lo = mid; else hi = mid - 1;
+  }
+  TileInfo ti;
+  ti.e = lo;
+  ti.gstart = lo ? sm.end[lo - 1] : 0;
+  ti.gend = sm.end[lo];
+  const int32_t local = t - sm.tile_prefix[lo];
+  if constexpr (MODE == FP8QGG_M_JAGGED) {
+    const int nt = static_cast<int>((p.n + BN - 1) / BN);
+    ti.tm = local / nt;
+    ti.tn = local % nt;
+    ti.nk = static_cast<int>((p.k + BK - 1) / BK);
+  } else {
+    const int nt = static_cast<int>((p.k + BN - 1) / BN);
+    ti.tm = local / nt;
+    ti.tn = local % nt;
+    ti.nk = ti.gend > ti.gstart ? (ti.gend - (ti.gstart & ~15) + BK - 1) / BK : 0;
+  }
+  return ti;
+}
+
+// Clamped group ends and cumulative tile counts, warp-parallel (one warp).
+template <int MODE>
+__device__ void build_tile_table(GemmSmem &sm, const GemmParams &p, int lane) {
+  const int32_t R = static_cast<int32_t>(p.m_total);
+  const int32_t nt_m = static_cast<int32_t>((p.n + BN - 1) / BN);
+  const int32_t tiles_k_mode =
+      static_cast<int32_t>(((p.n + BM - 1) / BM) * ((p.k + BN - 1) / BN));
+  int32_t carry_end = 0, carry_tiles = 0;
+  bool bad = false;
+  for (int base = 0; base < p.num_groups; base += 32) {
+    const int e = base + lane;
+    const int32_t raw = e < p.num_groups ? __ldg(p.offsets + e) : INT32_MIN;
+    int32_t run = max(raw, 0);
+    for (int d = 1; d < 32; d <<= 1) {
+      const int32_t o = __shfl_up_sync(0xFFFFFFFFu, run, d);
+      if (lane >= d) run = max(run, o);
+    }
+    const int32_t endv = min(R, max(carry_end, run));
+    int32_t prev = __shfl_up_sync(0xFFFFFFFFu, endv, 1);
+    if (lane == 0) prev = carry_end;
+    if (e < p.num_groups && (raw < prev || raw > R)) bad = true;
+    int32_t tiles = 0;
+    if (e < p.num_groups) {
+      if constexpr (MODE == FP8QGG_M_JAGGED)
+        tiles = ((endv - prev + BM - 1) / BM) * nt_m;
+      else
+        tiles = tiles_k_mode;
+    }
+    for (int d = 1; d < 32; d <<= 1) {
+      const int32_t o = __shfl_up_sync(0xFFFFFFFFu, tiles, d);
+      if (lane >= d) tiles += o;
+    }
+    if (e < p.num_groups) {
+      sm.end[e] = endv;
+      sm.tile_prefix[e + 1] = carry_tiles + tiles;
+    }
+    carry_end = __shfl_sync(0xFFFFFFFFu, endv, 31);
+    carry_tiles += __shfl_sync(0xFFFFFFFFu, tiles, 31);
+  }
+  if (lane == 0) sm.tile_prefix[0] = 0;
+  bad = __any_sync(0xFFFFFFFFu, bad);
+  if (bad && lane == 0 && blockIdx.x == 0) status_or(p.status, FP8QGG_STATUS_BAD_OFFSETS);
+}
+
+// Zero the K columns outside [lo, hi) of a K-major tile written by TMA with
+// 128-byte swizzle (logical 16-byte chunk j of row r sits at chunk j ^ (r & 7)).
+__device__ __forceinline__ void mask_k_tile(uint8_t *tile, int rows, int lo, int hi, int lane) {
+  for (int r = lane; r < rows; r += 32) {
+    uint8_t *row = tile + r * BK;
+#pragma unroll
+    for (int j = 0; j < BK / 16; ++j) {
+      const int k0 = 16 * j;
+      if (k0 >= lo && k0 + 16 <= hi) continue;
+      uint4 *ptr = reinterpret_cast<uint4 *>(row + ((j ^ (r & 7)) << 4));
+      if (k0 + 16 <= lo || k0 >= hi) {
+        *ptr = make_uint4(0u, 0u, 0u, 0u);
+        continue;
+      }
+      uint4 v = *ptr;
+      uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int b = 0; b < 16; ++b) {
+        const int kk = k0 + b;
+        if (kk < lo || kk >= hi) w[b >> 2] &= ~(0xFFu << (8 * (b & 3)));
+      }
+      *ptr = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+  }
+}
+
+// Barrier over the 128 epilogue threads that also ANDs a flag across them,
+// so that an abort is always decided by all of them together.
+__device__ __forceinline__ bool epi_bar_and(bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 q, %1, 0;\n\t"
+      "bar.red.and.pred p, 1, %2, q;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(r)
+      : "r"(static_cast<uint32_t>(v)), "n"(kEpiThreads)
+      : "memory");
+  return r != 0;
+}
+
+template <int OUT>
+__device__ __forceinline__ void store_chunk(void *out_row, int64_t col0, int64_t ncols,
+                                            const uint32_t (&r)[32], float inv_a,
+                                            const float *inv_b) {
+  if constexpr (OUT == FP8QGG_OUT_F32) {
+    float *o = static_cast<float *>(out_row) + col0;
+#pragma unroll
+    for (int v = 0; v < 8; ++v) {
+      if (col0 + 4 * v >= ncols) break;
+      float4 f;
+      f.x = __fmul_rn(__fmul_rn(__uint_as_float(r[4 * v + 0]), inv_a), inv_b[4 * v + 0]);
+      f.y = __fmul_rn(__fmul_rn(__uint_as_float(r[4 * v + 1]), inv_a), inv_b[4 * v + 1]);
+      f.z = __fmul_rn(__fmul_rn(__uint_as_float(r[4 * v + 2]), inv_a), inv_b[4 * v + 2]);
+      f.w = __fmul_rn(__fmul_rn(__uint_as_float(r[4 * v + 3]), inv_a), inv_b[4 * v + 3]);
+      *reinterpret_cast<float4 *>(o + 4 * v) = f;
+    }
+  } else {
+    __nv_bfloat16 *o = static_cast<__nv_bfloat16 *>(out_row) + col0;
+#pragma unroll
+    for (int v = 0; v < 4; ++v) {
+      if (col0 + 8 * v >= ncols) break;
+      uint32_t w[4];
+#pragma unroll
+      for (int h = 0; h < 4; ++h) {
+        const int c = 8 * v + 2 * h;
+        const float f0 = __fmul_rn(__fmul_rn(__uint_as_float(r[c]), inv_a), inv_b[c]);
+        const float f1 = __fmul_rn(__fmul_rn(__uint_as_float(r[c + 1]), inv_a), inv_b[c + 1]);
+        __nv_bfloat162 b2 = __floats2bfloat162_rn(f0, f1);
+        w[h] = *reinterpret_cast<uint32_t *>(&b2);
+      }
+      *reinterpret_cast<uint4 *>(o + 8 * v) = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+  }
+}
+
+template <int MODE, int OUT>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    grouped_gemm_kernel(const __grid_constant__ CUtensorMap amap,
+                        const __grid_constant__ CUtensorMap bmap, const GemmParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  GemmSmem &sm = *reinterpret_cast<GemmSmem *>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (warp == 0 && lane == 0) {
+    prefetch_tensormap(&amap);
+    prefetch_tensormap(&bmap);
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&sm.full[s], 1);
+      mbar_init(&sm.empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&sm.tfull[b], 1);
+      mbar_init(&sm.tempty[b], kEpiThreads);
+    }
+    mbar_init(&sm.drain, 1);
+    sm.abort = 0;
+    fence_mbarrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&sm.tmem_base, kTmemCols);
+    tmem_relinquish();
+  }
+  if (warp == 2) build_tile_table<MODE>(sm, p, lane);
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+
+  const int32_t total = sm.tile_prefix[p.num_groups];
+  volatile int *abort = &sm.abort;
+  const uint32_t tmem_base = sm.tmem_base;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      uint32_t stage = 0, phase = 0;
+      uint32_t armed = 0;  // stages with a load issued
+      uint32_t last_par[kStages] = {0, 0, 0, 0};
+      bool ok = true;
+      for (int32_t t = blockIdx.x; t < total && ok; t += gridDim.x) {
+        const TileInfo ti = decode_tile<MODE>(sm, p, t);
+        for (int kb = 0; kb < ti.nk; ++kb) {
+          if (!mbar_wait(&sm.empty[stage], phase ^ 1, abort)) { ok = false; break; }
+          mbar_arrive_expect_tx(&sm.full[stage], kStageBytes);
+          if constexpr (MODE == FP8QGG_M_JAGGED) {
+            tma_load_2d(sm.a[stage], &amap, &sm.full[stage], kb * BK, ti.gstart + ti.tm * BM);
+            tma_load_3d(sm.b[stage], &bmap, &sm.full[stage], kb * BK, ti.tn * BN, ti.e);
+          } else {
+            const int32_t kx = (ti.gstart & ~15) + kb * BK;
+            tma_load_2d(sm.a[stage], &amap, &sm.full[stage], kx, ti.tm * BM);
+            tma_load_2d(sm.b[stage], &bmap, &sm.full[stage], kx, ti.tn * BN);
+          }
+          armed |= 1u << stage;
+          last_par[stage] = phase;
+          if (++stage == kStages) { stage = 0; phase ^= 1; }
+        }
+      }
+      if (!ok) {
+        *abort = 1;
+        status_or(p.status, FP8QGG_STATUS_TIMEOUT);
+        // let copies already in flight land before the CTA can exit
+        volatile int never = 0;
+        for (int s = 0; s < kStages; ++s)
+          if (armed & (1u << s)) (void)mbar_wait(&sm.full[s], last_par[s], &never);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    uint32_t stage = 0, phase = 0, acc = 0, acc_phase = 0;
+    bool ok = true;
+    for (int32_t t = blockIdx.x; t < total && ok; t += gridDim.x) {
+      const TileInfo ti = decode_tile<MODE>(sm, p, t);
+      if (!__all_sync(0xFFFFFFFFu, mbar_wait(&sm.tempty[acc], acc_phase ^ 1, abort))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after_sync();
+      const uint32_t d_tmem = tmem_base + acc * BN;
+      for (int kb = 0; kb < ti.nk; ++kb) {
+        if (!__all_sync(0xFFFFFFFFu, mbar_wait(&sm.full[stage], phase, abort))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after_sync();
+        if constexpr (MODE == FP8QGG_K_JAGGED) {
+          const int32_t kx = (ti.gstart & ~15) + kb * BK;
+          const int lo = max(0, ti.gstart - kx);
+          const int hi = min(BK, ti.gend - kx);
+          if (lo > 0 || hi < BK) {
+            mask_k_tile(sm.a[stage], BM, lo, hi, lane);
+            mask_k_tile(sm.b[stage], BN, lo, hi, lane);
+            fence_proxy_async_smem();
+            __syncwarp();
+          }
+        }
+        if (lane == 0) {
+          const uint64_t adesc = smem_desc_k_sw128(smem_addr(sm.a[stage]));
+          const uint64_t bdesc = smem_desc_k_sw128(smem_addr(sm.b[stage]));
+#pragma unroll
+          for (int kk = 0; kk < BK / 32; ++kk)
+            mma_f8f6f4(d_tmem, adesc + 2 * kk, bdesc + 2 * kk, kIdesc, (kb | kk) != 0);
+          mma_commit(&sm.empty[stage]);
+        }
+        __syncwarp();
+        if (++stage == kStages) { stage = 0; phase ^= 1; }
+      }
+      if (!ok) break;
+      if (lane == 0) {
+        if (ti.nk > 0) mma_commit(&sm.tfull[acc]); else mbar_arrive(&sm.tfull[acc]);
+      }
+      __syncwarp();
+      if (++acc == 2) { acc = 0; acc_phase ^= 1; }
+    }
+    if (!ok && lane == 0) {
+      *abort = 1;
+      status_or(p.status, FP8QGG_STATUS_TIMEOUT);
+    }
+    // every MMA this thread issued has completed before TMEM is released
+    if (lane == 0) {
+      mma_commit(&sm.drain);
+      volatile int never = 0;
+      (void)mbar_wait(&sm.drain, 0, &never);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int et = threadIdx.x - 64;  // 0..127
+    const int quarter = warp & 3;     // TMEM lanes [32*quarter, 32*quarter + 32)
+    const int row = 32 * quarter + lane;
+    uint32_t acc = 0, acc_phase = 0;
+    for (int32_t t = blockIdx.x; t < total; t += gridDim.x) {
+      const TileInfo ti = decode_tile<MODE>(sm, p, t);
+      const int64_t ncols = MODE == FP8QGG_M_JAGGED ? p.n : p.k;
+      // column reciprocal scales of this tile
+      for (int h = 0; h < 2; ++h) {
+        const int c = 2 * et + h;
+        const int64_t col = static_cast<int64_t>(ti.tn) * BN + c;
+        float inv = 0.0f;
+        if (col < ncols) inv = __frcp_rn(__ldg(p.scale_b + ti.e * p.sbs + col));
+        sm.inv_sb[acc][c] = inv;
+      }
+      int64_t orow;
+      bool valid;
+      float inv_a = 0.0f;
+      char *out_row;
+      if constexpr (MODE == FP8QGG_M_JAGGED) {
+        orow = static_cast<int64_t>(ti.gstart) + static_cast<int64_t>(ti.tm) * BM + row;
+        valid = orow < ti.gend;
+        if (valid) inv_a = __frcp_rn(__ldg(p.scale_a + orow));
+        out_row = static_cast<char *>(p.out) +
+                  orow * p.ld_out * (OUT == FP8QGG_OUT_F32 ? 4 : 2);
+      } else {
+        orow = static_cast<int64_t>(ti.tm) * BM + row;
+        valid = orow < p.n;
+        if (valid) inv_a = __frcp_rn(__ldg(p.scale_a + ti.e * p.sas + orow));
+        out_row = static_cast<char *>(p.out) +
+                  (ti.e * p.out_gs + orow * p.ld_out) * (OUT == FP8QGG_OUT_F32 ? 4 : 2);
+      }
+      const bool got = mbar_wait(&sm.tfull[acc], acc_phase, abort);
+      if (!epi_bar_and(got)) {
+        *abort = 1;
+        if (et == 0) status_or(p.status, FP8QGG_STATUS_TIMEOUT);
+        break;
+      }
+      tc_fence_after_sync();
+      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(32 * quarter) << 16) + acc * BN;
+#pragma unroll 1
+      for (int c = 0; c < BN / 32; ++c) {
+        uint32_t r[32];
+        if (ti.nk > 0) {
+          tmem_ld_32x32b_x32(taddr + 32 * c, r);
+          tmem_ld_wait();
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) r[i] = 0u;
+        }
+        const int64_t col0 = static_cast<int64_t>(ti.tn) * BN + 32 * c;
+        if (valid && col0 < ncols)
+          store_chunk<OUT>(out_row, col0, ncols, r, inv_a, &sm.inv_sb[acc][32 * c]);
+      }
+      tc_fence_before_sync();
+      mbar_arrive(&sm.tempty[acc]);
+      if (++acc == 2) { acc = 0; acc_phase ^= 1; }
+    }
+  }
+
+  tc_fence_before_sync();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after_sync();
+    tmem_dealloc(tmem_base, kTmemCols);
+  }
+}
+
+namespace {
+using GemmKernel = void (*)(const CUtensorMap, const CUtensorMap, const GemmParams);
+
+GemmKernel gemm_kernel(int mode, int out_dtype) {
+  if (mode == FP8QGG_M_JAGGED)
+    return out_dtype == FP8QGG_OUT_F32 ? grouped_gemm_kernel<FP8QGG_M_JAGGED, FP8QGG_OUT_F32>
+                                       : grouped_gemm_kernel<FP8QGG_M_JAGGED, FP8QGG_OUT_BF16>;
+  return out_dtype == FP8QGG_OUT_F32 ? grouped_gemm_kernel<FP8QGG_K_JAGGED, FP8QGG_OUT_F32>
+                                     : grouped_gemm_kernel<FP8QGG_K_JAGGED, FP8QGG_OUT_BF16>;
+}
+}  // namespace
+
+}  // namespace fp8qgg
+
+using namespace fp8qgg;
+
+extern "C" int fp8_scaled_grouped_gemm(int mode, const uint8_t *a, int64_t ld_a,
+                                       const float *scale_a, int64_t scale_a_group_stride,
+                                       const uint8_t *b, int64_t ld_b, int64_t b_group_stride,
+                                       const float *scale_b, int64_t scale_b_group_stride,
+                                       const int32_t *offsets, int32_t num_groups,
+                                       int64_t m_total, int64_t n, int64_t k, void *out,
+                                       int64_t ld_out, int64_t out_group_stride, int out_dtype,
+                                       int fmt, int32_t *dev_status, void *stream) {
+  if (mode != FP8QGG_M_JAGGED && mode != FP8QGG_K_JAGGED) return FP8QGG_ERR_UNSUPPORTED;
+  if (out_dtype != FP8QGG_OUT_F32 && out_dtype != FP8QGG_OUT_BF16) return FP8QGG_ERR_UNSUPPORTED;
+  if (fmt != FP8QGG_E4M3FN) return FP8QGG_ERR_UNSUPPORTED;
+  if (num_groups < 1 || num_groups > kMaxGemmGroups) return FP8QGG_ERR_SHAPE;
+  if (m_total < 0 || m_total > INT32_MAX - 2 * BK || n < 1 || k < 1) return FP8QGG_ERR_SHAPE;
+  if (n > INT32_MAX / 2 || k > INT32_MAX / 2) return FP8QGG_ERR_SHAPE;
+  const int64_t ocols = mode == FP8QGG_M_JAGGED ? n : k;
+  const int vec = out_dtype == FP8QGG_OUT_F32 ? 4 : 8;
+  if (mode == FP8QGG_M_JAGGED) {
+    if (ld_a < k || ld_b < k || ld_out < n || scale_b_group_stride < n) return FP8QGG_ERR_SHAPE;
+    if (num_groups > 1 && b_group_stride < n * ld_b) return FP8QGG_ERR_SHAPE;
+  } else {
+    if (ld_a < m_total || ld_b < m_total || ld_out < k) return FP8QGG_ERR_SHAPE;
+    if (scale_a_group_stride < n || scale_b_group_stride < k) return FP8QGG_ERR_SHAPE;
+    if (num_groups > 1 && out_group_stride < n * ld_out) return FP8QGG_ERR_SHAPE;
+  }
+  if (!a || !b || !scale_a || !scale_b || !offsets || !out) return FP8QGG_ERR_NULL;
+  if (!aligned(a, 16) || !aligned(b, 16) || !aligned(out, 16)) return FP8QGG_ERR_ALIGN;
+  if (!aligned(scale_a, 4) || !aligned(scale_b, 4) || !aligned(offsets, 4))
+    return FP8QGG_ERR_ALIGN;
+  if (dev_status && !aligned(dev_status, 4)) return FP8QGG_ERR_ALIGN;
+  if (ld_a % 16 || ld_b % 16) return FP8QGG_ERR_ALIGN;
+  if (mode == FP8QGG_M_JAGGED && b_group_stride % 16) return FP8QGG_ERR_ALIGN;
+  if (ocols % vec || ld_out % vec) return FP8QGG_ERR_ALIGN;
+  if (mode == FP8QGG_K_JAGGED && num_groups > 1 && out_group_stride % vec) return FP8QGG_ERR_ALIGN;
+
+  CUtensorMap amap, bmap;
+  const uint32_t abox[2] = {BK, BM};
+  if (mode == FP8QGG_M_JAGGED) {
+    const uint64_t adims[2] = {static_cast<uint64_t>(k),
+                               static_cast<uint64_t>(std::max<int64_t>(m_total, 1))};
+    const uint64_t astr[1] = {static_cast<uint64_t>(ld_a)};
+    const uint64_t bdims[3] = {static_cast<uint64_t>(k), static_cast<uint64_t>(n),
+                               static_cast<uint64_t>(num_groups)};
+    const uint64_t bstr[2] = {static_cast<uint64_t>(ld_b),
+                              static_cast<uint64_t>(num_groups > 1 ? b_group_stride
+                                                                   : n * ld_b)};
+    const uint32_t bbox[3] = {BK, BN, 1};
+    if (!encode_tensor_map(&amap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t *>(a),
+                           adims, astr, abox, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !encode_tensor_map(&bmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<uint8_t *>(b),
+                           bdims, bstr, bbox, CU_TENSOR_MAP_SWIZZLE_128B))
+      return FP8QGG_ERR_CUDA;
+  } else {
+    const uint64_t mt = static_cast<uint64_t>(std::max<int64_t>(m_total, 1));
+    const uint64_t adims[2] = {mt, static_cast<uint64_t>(n)};
+    const uint64_t astr[1] = {static_cast<uint64_t>(ld_a)};
+    const uint64_t bdims[2] = {mt, static_cast<uint64_t>(k)};
+    const uint64_t bstr[1] = {static_cast<uint64_t>(ld_b)};
+    const uint32_t bbox[2] = {BK, BN};
+    if (!encode_tensor_map(&amap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t *>(a),
+                           adims, astr, abox, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !encode_tensor_map(&bmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t *>(b),
+                           bdims, bstr, bbox, CU_TENSOR_MAP_SWIZZLE_128B))
+      return FP8QGG_ERR_CUDA;
+  }
+
+  DeviceInfo dev;
+  if (!device_info(&dev)) return FP8QGG_ERR_CUDA;
+  GemmKernel kern = gemm_kernel(mode, out_dtype);
+  const int smem = static_cast<int>(sizeof(GemmSmem)) + 1024;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+      cudaSuccess)
+    return FP8QGG_ERR_CUDA;
+  int64_t max_tiles;
+  if (mode == FP8QGG_M_JAGGED)
+    max_tiles = ((m_total + BM - 1) / BM + num_groups) * ((n + BN - 1) / BN);
+  else
+    max_tiles = int64_t(num_groups) * ((n + BM - 1) / BM) * ((k + BN - 1) / BN);
+  if (max_tiles > INT32_MAX) return FP8QGG_ERR_SHAPE;
+  const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(max_tiles, dev.sm_count)));
+
+  GemmParams prm;
+  prm.scale_a = scale_a;
+  prm.sas = scale_a_group_stride;
+  prm.scale_b = scale_b;
+  prm.sbs = scale_b_group_stride;
+  prm.offsets = offsets;
+  prm.num_groups = num_groups;
+  prm.m_total = m_total;
+  prm.n = n;
+  prm.k = k;
+  prm.out = out;
+  prm.ld_out = ld_out;
+  prm.out_gs = out_group_stride;
+  prm.status = dev_status;
+  kern<<<grid, kGemmThreads, smem, static_cast<cudaStream_t>(stream)>>>(amap, bmap, prm);
+  return cudaGetLastError() == cudaSuccess ? FP8QGG_OK : FP8QGG_ERR_CUDA;
+}

@@ -1,0 +1,135 @@
+"""Host-side checks of the C ABI that need no GPU: the library builds and loads,
+exports every entry point the header declares, and rejects bad arguments on
+the host before anything is enqueued."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import quantization_grouped_gemm_b200 as qgg
+from quantization_grouped_gemm_b200 import build as qbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "fp8qgg.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = re.findall(r"^\s*(?:const\s+)?[A-Za-z_][\w ]*?[\s\*]+(\w+)\s*\(", text, flags=re.M)
+    return sorted(set(n for n in names if n not in ("defined",)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    qbuild.build()
+    return qgg.lib()
+
+
+def test_header_declares_the_three_entry_points():
+    names = declared_functions()
+    for n in ("fp8_quant_rowwise", "fp8_quant_colwise_jagged", "fp8_scaled_grouped_gemm"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    names = declared_functions()
+    assert len(names) >= 7
+    for n in names:
+        assert hasattr(lib, n), n
+    # and the binding knows the signature of each
+    assert set(names) <= set(qgg._SIGNATURES)
+
+
+def test_library_is_built_for_sm100a():
+    qbuild.build()
+    assert "arch=compute_100a,code=sm_100a" in qbuild.ARCH
+    with open(qbuild.LIB, "rb") as f:
+        blob = f.read()
+    assert b"sm_100a" in blob
+
+
+def test_native_format_and_error_strings(lib):
+    assert lib.fp8_native_format() == qgg.E4M3FN
+    for rc in (0, -1, -2, -3, -4, -5):
+        assert lib.fp8qgg_error_string(rc)
+    assert lib.fp8qgg_error_string(-99) == b"unknown error"
+
+
+FAKE = ctypes.c_void_p(1 << 20)  # 16-byte-aligned non-null value, never dereferenced on these paths
+ODD = ctypes.c_void_p((1 << 20) + 4)
+
+
+def test_rowwise_argument_checks(lib):
+    f = lib.fp8_quant_rowwise
+    assert f(None, 4, 64, 64, FAKE, 64, FAKE, 0, 0.0, None, None) == -1
+    assert f(FAKE, 4, 0, 64, FAKE, 64, FAKE, 0, 0.0, None, None) == -2
+    assert f(FAKE, 4, 64, 32, FAKE, 64, FAKE, 0, 0.0, None, None) == -2
+    assert f(FAKE, 4, 40000, 40000, FAKE, 40000, FAKE, 0, 0.0, None, None) == -2
+    assert f(FAKE, 4, 60, 64, FAKE, 64, FAKE, 0, 0.0, None, None) == -3
+    assert f(ODD, 4, 64, 64, FAKE, 64, FAKE, 0, 0.0, None, None) == -3
+    assert f(FAKE, 4, 64, 64, FAKE, 64, FAKE, 7, 0.0, None, None) == -4
+    assert f(FAKE, 4, 64, 64, FAKE, 64, FAKE, 0, -1.0, None, None) == -4
+    assert f(FAKE, 0, 64, 64, FAKE, 64, FAKE, 0, 0.0, None, None) == 0  # empty: no-op
+
+
+def test_colwise_argument_checks(lib):
+    f = lib.fp8_quant_colwise_jagged
+    ws = lib.fp8_quant_colwise_jagged_workspace_size(100, 64, 4)
+    assert ws >= 4 * 64 * 4 and ws % 256 == 0
+
+    def call(**kw):
+        a = dict(x=FAKE, rows=100, cols=64, ld_x=64, off=FAKE, e=4, q=FAKE, ld_q=64, layout=0,
+                 s=FAKE, fmt=0, smax=0.0, sat=None, st=None, ws=FAKE, wsb=ws)
+        a.update(kw)
+        return f(a["x"], a["rows"], a["cols"], a["ld_x"], a["off"], a["e"], a["q"], a["ld_q"],
+                 a["layout"], a["s"], a["fmt"], a["smax"], a["sat"], a["st"], a["ws"], a["wsb"],
+                 None)
+
+    assert call(x=None) == -1
+    assert call(off=None) == -1
+    assert call(ws=None) == -1
+    assert call(e=0) == -2
+    assert call(e=2000) == -2
+    assert call(wsb=ws - 1) == -2
+    assert call(layout=1, ld_q=64) == -2       # transposed needs ld_q >= rows_total
+    assert call(layout=1, ld_q=104) == -3      # and ld_q % 16 == 0
+    assert call(cols=60, ld_x=64) == -3
+    assert call(layout=5) == -4
+    assert call(fmt=3) == -4
+
+
+def test_gemm_argument_checks(lib):
+    f = lib.fp8_scaled_grouped_gemm
+
+    def call(**kw):
+        a = dict(mode=0, a=FAKE, lda=64, sa=FAKE, sas=0, b=FAKE, ldb=64, bgs=64 * 32, sb=FAKE,
+                 sbs=32, off=FAKE, e=2, m=100, n=32, k=64, out=FAKE, ldo=32, ogs=0, odt=0, fmt=0)
+        a.update(kw)
+        return f(a["mode"], a["a"], a["lda"], a["sa"], a["sas"], a["b"], a["ldb"], a["bgs"],
+                 a["sb"], a["sbs"], a["off"], a["e"], a["m"], a["n"], a["k"], a["out"], a["ldo"],
+                 a["ogs"], a["odt"], a["fmt"], None, None)
+
+    assert call(fmt=1) == -4           # no e4m3fnuz input on the tensor cores
+    assert call(mode=2) == -4
+    assert call(odt=3) == -4
+    assert call(e=0) == -2
+    assert call(e=1025) == -2
+    assert call(lda=32) == -2
+    assert call(bgs=64) == -2          # groups of B overlap
+    assert call(a=None) == -1
+    assert call(lda=72) == -3          # leading dimension not a multiple of 16
+    assert call(n=30, ldo=32, sbs=32) == -3
+    assert call(a=ODD) == -3
+    # K-jagged: token axis is the leading dimension of both operands
+    assert call(mode=1, lda=64, ldb=64, m=100, sas=32, sbs=64, ldo=64, ogs=32 * 64) == -2
+    assert call(mode=1, lda=112, ldb=112, m=100, sas=32, sbs=64, ldo=64, ogs=16) == -2
+
+
+def test_cast_argument_checks(lib):
+    f = lib.fp8_cast_f32
+    assert f(FAKE, -1, FAKE, 0, None) == -2
+    assert f(FAKE, 4, FAKE, 2, None) == -4
+    assert f(None, 4, FAKE, 0, None) == -1
+    assert f(FAKE, 0, FAKE, 0, None) == 0

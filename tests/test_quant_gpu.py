@@ -1,0 +1,257 @@
+"""GPU parity of the quantisation kernels against the CPU oracle.
+
+Codes, scales and saturation counts must be bit-exact.  Every call goes
+through the C ABI (via the thin binding); expected values come only from the
+oracle."""
+import numpy as np
+import pytest
+import torch
+
+import oracle as orc
+import quantization_grouped_gemm_b200 as qgg
+from quantization_grouped_gemm_b200 import workloads as wl
+
+pytestmark = pytest.mark.gpu
+FMTS = [qgg.E4M3FN, qgg.E4M3FNUZ]
+
+
+def dev(t):
+    return t.cuda()
+
+
+def bits(t):
+    return wl.bf16_bits(t.cpu())
+
+
+def rand_bf16(seed, rows, cols, outliers=0.01, zero_rows=(), zero_cols=()):
+    g = np.random.default_rng(seed)
+    a = g.standard_normal((rows, cols)).astype(np.float32)
+    if outliers and a.size:
+        idx = g.integers(0, a.size, max(1, int(a.size * outliers)))
+        a.reshape(-1)[idx] *= 100
+    for r in zero_rows:
+        a[r, :] = 0
+    for c in zero_cols:
+        a[:, c] = 0
+    return wl.to_bf16(a)
+
+
+# ----------------------------------------------------------------- encoder sweep
+@pytest.mark.parametrize("fmt", FMTS)
+def test_device_encoder_exhaustive_over_the_active_binades(fmt):
+    """Every fp32 bit pattern whose magnitude lies in [2^-12, 2^9) (both signs),
+    through fp8_cast_f32, equals the oracle's encode; a sample of the rest too."""
+    mant = torch.arange(1 << 23, dtype=torch.int32, device="cuda")
+    for exp_field in range(127 - 12, 127 + 9):
+        for sign in (0, 1):
+            pat = mant | ((sign << 31) | (exp_field << 23))
+            y = pat.view(torch.float32)
+            q = qgg.fp8_cast_f32(y, fmt).cpu().numpy()
+            ref = orc.encode_array(y.cpu().numpy(), fmt)
+            bad = np.nonzero(q != ref)[0]
+            assert bad.size == 0, (exp_field, sign, [(hex(int(pat[i])), hex(q[i]), hex(ref[i]))
+                                                     for i in bad[:5]])
+    g = np.random.default_rng(5)
+    pats = g.integers(0, 1 << 32, 1 << 22, dtype=np.uint64).astype(np.uint32)
+    pats = pats[(pats & 0x7F800000) != 0x7F800000]  # no NaN/Inf
+    y = pats.view(np.float32)
+    q = qgg.fp8_cast_f32(torch.from_numpy(y).cuda(), fmt).cpu().numpy()
+    assert (q == orc.encode_array(y, fmt)).all()
+    special = np.array([0.0, -0.0, np.inf, -np.inf, 448.0, -448.0, 240.0, 232.0, -232.0, 464.0],
+                       np.float32)
+    q = qgg.fp8_cast_f32(torch.from_numpy(special).cuda(), fmt).cpu().numpy()
+    assert (q == orc.encode_array(special, fmt)).all()
+
+
+@pytest.mark.parametrize("n", [1, 7, 8, 9, 1000, 4099])
+def test_cast_ragged_lengths(n):
+    g = np.random.default_rng(n)
+    y = (g.standard_normal(n) * 50).astype(np.float32)
+    for fmt in FMTS:
+        q = qgg.fp8_cast_f32(torch.from_numpy(y).cuda(), fmt).cpu().numpy()
+        assert (q == orc.encode_array(y, fmt)).all()
+
+
+# ----------------------------------------------------------------- rowwise
+ROW_SHAPES = [(1, 8), (3, 256), (17, 1408), (64, 4096), (33, 7168), (5, 5120), (2, 32768),
+              (300, 72), (1000, 2048), (9, 16384)]
+
+
+@pytest.mark.parametrize("rows,cols", ROW_SHAPES)
+@pytest.mark.parametrize("fmt", FMTS)
+def test_rowwise_parity(rows, cols, fmt):
+    x = rand_bf16(rows * 7 + cols, rows, cols, zero_rows=[0] if rows > 2 else [])
+    xb = bits(x)
+    q_ref, s_ref, sat_ref = orc.quant_rowwise(xb, fmt)
+    sat = torch.zeros(1, dtype=torch.int64, device="cuda")
+    q, s = qgg.fp8_quant_rowwise(dev(x), fmt, sat_count=sat)
+    torch.cuda.synchronize()
+    assert (q.cpu().numpy() == q_ref).all()
+    assert (s.cpu().numpy().view(np.uint32) == s_ref.view(np.uint32)).all()
+    assert int(sat.item()) == sat_ref == 0
+
+
+def test_rowwise_strided_input_and_output_leave_padding_untouched():
+    rows, cols, ldx, ldq = 37, 1408, 1408 + 64, 1408 + 24
+    full = rand_bf16(3, rows, ldx)
+    x = dev(full)[:, :cols]
+    qbuf = torch.full((rows, ldq), 0xAB, dtype=torch.uint8, device="cuda")
+    q, s = qgg.fp8_quant_rowwise(x, q=qbuf[:, :cols],
+                                 scales=torch.empty(rows, device="cuda"))
+    q_ref, s_ref, _ = orc.quant_rowwise(bits(full)[:, :cols])
+    qb = qbuf.cpu().numpy()
+    assert (qb[:, :cols] == q_ref).all()
+    assert (qb[:, cols:] == 0xAB).all()
+    assert (s.cpu().numpy() == s_ref).all()
+
+
+@pytest.mark.parametrize("fmt", FMTS)
+def test_rowwise_every_bf16_value_at_unit_scale(fmt):
+    """All finite bf16 values within +-fmax, with fmax itself in every row so that
+    s = fmax / fmax = 1: the codes are the encoder applied to x."""
+    fmax = orc.fp8_max(fmt)
+    pats = np.arange(65536, dtype=np.uint32)
+    vals = (pats << 16).view(np.float32)
+    keep = np.isfinite(vals) & (np.abs(vals) <= fmax)
+    p16 = pats[keep].astype(np.uint16)
+    per = 255
+    nrows = (p16.size + per - 1) // per
+    grid = np.full((nrows, per + 1), 0, np.uint16)
+    body = np.zeros(nrows * per, np.uint16)
+    body[: p16.size] = p16
+    grid[:, :per] = body.reshape(nrows, per)
+    grid[:, per] = (np.array([fmax], np.float32).view(np.uint32) >> 16).astype(np.uint16)
+    x = torch.from_numpy(grid.view(np.int16)).view(torch.bfloat16)
+    q_ref, s_ref, _ = orc.quant_rowwise(grid, fmt)
+    assert (s_ref == 1.0).all()
+    q, s = qgg.fp8_quant_rowwise(dev(x), fmt)
+    assert (q.cpu().numpy() == q_ref).all()
+    assert (s.cpu().numpy() == 1.0).all()
+
+
+@pytest.mark.parametrize("fmt,smax", [(qgg.E4M3FNUZ, 448.0), (qgg.E4M3FN, 240.0)])
+def test_rowwise_format_mismatch_is_counted_like_the_oracle(fmt, smax):
+    x = rand_bf16(77, 64, 512, outliers=0.0)
+    q_ref, s_ref, sat_ref = orc.quant_rowwise(bits(x), fmt, scale_max=smax)
+    sat = torch.zeros(1, dtype=torch.int64, device="cuda")
+    q, s = qgg.fp8_quant_rowwise(dev(x), fmt, scale_max=smax, sat_count=sat)
+    assert (q.cpu().numpy() == q_ref).all()
+    assert (s.cpu().numpy() == s_ref).all()
+    assert int(sat.item()) == sat_ref
+    if fmt == qgg.E4M3FNUZ:
+        assert sat_ref > 0
+    else:
+        assert sat_ref == 0
+
+
+def test_rowwise_zero_rows_is_a_no_op():
+    x = torch.empty((0, 64), dtype=torch.bfloat16, device="cuda")
+    q, s = qgg.fp8_quant_rowwise(x)
+    assert q.shape == (0, 64) and s.shape == (0,)
+
+
+# ----------------------------------------------------------------- jagged colwise
+COL_CASES = [
+    ([5, 0, 19, 8], 16),
+    ([0, 1, 15, 17, 0, 33], 72),
+    ([511, 512, 513], 64),
+    ([1500, 0, 3], 200),
+    ([2000], 8),
+    ([0, 0, 0], 64),
+    ([1, 1, 1, 1, 1, 1, 1, 1, 1, 1, 1, 1, 1, 1, 1, 1, 1], 128),
+    ([3000, 70, 700], 1408),
+]
+
+
+@pytest.mark.parametrize("sizes,cols", COL_CASES)
+@pytest.mark.parametrize("fmt", FMTS)
+@pytest.mark.parametrize("layout", [qgg.LAYOUT_SAME, qgg.LAYOUT_TRANSPOSED])
+def test_colwise_parity(sizes, cols, fmt, layout):
+    m = int(sum(sizes))
+    x = rand_bf16(m + cols + len(sizes), m, cols, zero_cols=[cols // 2] if cols > 2 else [])
+    off = wl.offsets_from_sizes(sizes)
+    ld = (m + 16 + 15) // 16 * 16 if layout == qgg.LAYOUT_TRANSPOSED else cols
+    q_ref, s_ref, sat_ref = orc.quant_colwise_jagged(bits(x), off, layout, fmt, ld_q=ld,
+                                                     fill=0xAB)
+    if layout == qgg.LAYOUT_TRANSPOSED:
+        qbuf = torch.full((cols, ld), 0xAB, dtype=torch.uint8, device="cuda")
+    else:
+        qbuf = torch.full((m, cols), 0xAB, dtype=torch.uint8, device="cuda")
+    sat = torch.zeros(1, dtype=torch.int64, device="cuda")
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    q, s = qgg.fp8_quant_colwise_jagged(dev(x), torch.from_numpy(off).cuda(), layout, fmt,
+                                        q=qbuf, sat_count=sat, status=st)
+    torch.cuda.synchronize()
+    qn = q.cpu().numpy()
+    bad = np.argwhere(qn != q_ref)
+    assert bad.size == 0, bad[:10]
+    assert (s.cpu().numpy().view(np.uint32) == s_ref.view(np.uint32)).all()
+    assert int(sat.item()) == sat_ref == 0
+    assert int(st.item()) == 0
+
+
+def test_colwise_transposed_equals_transpose_of_same_layout():
+    sizes = [700, 1, 0, 1200, 45]
+    m, cols = sum(sizes), 136
+    x = dev(rand_bf16(9, m, cols))
+    off = torch.from_numpy(wl.offsets_from_sizes(sizes)).cuda()
+    q1, s1 = qgg.fp8_quant_colwise_jagged(x, off, qgg.LAYOUT_SAME)
+    q2, s2 = qgg.fp8_quant_colwise_jagged(x, off, qgg.LAYOUT_TRANSPOSED)
+    assert torch.equal(q2[:, :m], q1.t())
+    assert torch.equal(s1, s2)
+
+
+def test_colwise_malformed_offsets_are_clamped_and_reported():
+    m, cols = 100, 64
+    x = rand_bf16(11, m, cols)
+    off = np.array([5, 3, 200, -1], np.int32)
+    q_ref, s_ref, _ = orc.quant_colwise_jagged(bits(x), off, orc.SAME)
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    q, s = qgg.fp8_quant_colwise_jagged(dev(x), torch.from_numpy(off).cuda(), status=st)
+    assert (q.cpu().numpy() == q_ref).all()
+    assert (s.cpu().numpy() == s_ref).all()
+    assert int(st.item()) & qgg.STATUS_BAD_OFFSETS
+
+
+def test_colwise_rows_past_last_offset_are_not_written():
+    m, cols = 300, 64
+    x = rand_bf16(12, m, cols)
+    off = np.array([100, 250], np.int32)
+    qbuf = torch.full((m, cols), 0xAB, dtype=torch.uint8, device="cuda")
+    q, _ = qgg.fp8_quant_colwise_jagged(dev(x), torch.from_numpy(off).cuda(), q=qbuf)
+    q_ref, _, _ = orc.quant_colwise_jagged(bits(x), off, orc.SAME, fill=0xAB)
+    assert (q.cpu().numpy() == q_ref).all()
+    assert (q.cpu().numpy()[250:] == 0xAB).all()
+
+
+def test_colwise_workspace_is_reusable_across_calls():
+    sizes = [2500, 10, 1800]
+    m, cols = sum(sizes), 256
+    off = torch.from_numpy(wl.offsets_from_sizes(sizes)).cuda()
+    ws = torch.full((qgg.colwise_workspace_bytes(m, cols, 3),), 0x7F, dtype=torch.uint8,
+                    device="cuda")
+    outs = []
+    for seed in (1, 2, 1):
+        x = dev(rand_bf16(seed, m, cols))
+        outs.append(qgg.fp8_quant_colwise_jagged(x, off, qgg.LAYOUT_TRANSPOSED, workspace=ws))
+    assert torch.equal(outs[0][0], outs[2][0]) and torch.equal(outs[0][1], outs[2][1])
+    x = rand_bf16(2, m, cols)
+    q_ref, s_ref, _ = orc.quant_colwise_jagged(bits(x), off.cpu().numpy(), orc.TRANSPOSED,
+                                               ld_q=outs[1][0].shape[1])
+    assert (outs[1][0].cpu().numpy()[:, :m] == q_ref[:, :m]).all()
+    assert (outs[1][1].cpu().numpy() == s_ref).all()
+
+
+@pytest.mark.parametrize("fmt,smax", [(qgg.E4M3FNUZ, 448.0), (qgg.E4M3FN, 240.0)])
+def test_colwise_format_mismatch_is_counted_like_the_oracle(fmt, smax):
+    sizes = [600, 0, 90]
+    x = rand_bf16(13, sum(sizes), 64, outliers=0.0)
+    off = wl.offsets_from_sizes(sizes)
+    q_ref, s_ref, sat_ref = orc.quant_colwise_jagged(bits(x), off, orc.SAME, fmt,
+                                                     scale_max=smax)
+    sat = torch.zeros(1, dtype=torch.int64, device="cuda")
+    q, s = qgg.fp8_quant_colwise_jagged(dev(x), torch.from_numpy(off).cuda(), fmt=fmt,
+                                        scale_max=smax, sat_count=sat)
+    assert (q.cpu().numpy() == q_ref).all()
+    assert (s.cpu().numpy() == s_ref).all()
+    assert int(sat.item()) == sat_ref
