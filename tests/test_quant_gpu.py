@@ -234,7 +234,8 @@ def test_colwise_workspace_is_reusable_across_calls():
     for seed in (1, 2, 1):
         x = dev(rand_bf16(seed, m, cols))
         outs.append(qgg.fp8_quant_colwise_jagged(x, off, qgg.LAYOUT_TRANSPOSED, workspace=ws))
-    assert torch.equal(outs[0][0], outs[2][0]) and torch.equal(outs[0][1], outs[2][1])
+    assert torch.equal(outs[0][0][:, :m], outs[2][0][:, :m])
+    assert torch.equal(outs[0][1], outs[2][1])
     x = rand_bf16(2, m, cols)
     q_ref, s_ref, _ = orc.quant_colwise_jagged(bits(x), off.cpu().numpy(), orc.TRANSPOSED,
                                                ld_q=outs[1][0].shape[1])
