@@ -39,6 +39,7 @@ constexpr int kStages = 4;
 constexpr int kGemmThreads = 192;
 constexpr int kEpiThreads = 128;
 constexpr int kMaxGemmGroups = 1024;
+constexpr int kBand = 16;  // M tiles per raster band (token-jagged mode)
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kStageBytes = (BM + BN) * BK;
 constexpr uint32_t kIdesc = idesc_e4m3_f32(BM, BN);
@@ -46,6 +47,7 @@ constexpr uint32_t kIdesc = idesc_e4m3_f32(BM, BN);
 struct GemmSmem {
   uint8_t a[kStages][BM * BK];  // 16 KB each, 1024-aligned (swizzle atoms)
   uint8_t b[kStages][BN * BK];  // 32 KB each
+  float stg[kEpiThreads / 32][32 * 32];  // per epilogue warp: 32 rows x 32 fp32, swizzled
   float inv_sb[2][BN];
   int32_t end[kMaxGemmGroups];
   int32_t tile_prefix[kMaxGemmGroups + 1];
@@ -93,9 +95,16 @@ __device__ __forceinline__ TileInfo decode_tile(const GemmSmem &sm, const GemmPa
   ti.gend = sm.end[lo];
   const int32_t local = t - sm.tile_prefix[lo];
   if constexpr (MODE == FP8QGG_M_JAGGED) {
+    // Bands of kBand M tiles: consecutive tiles walk down a band before moving
+    // to the next N tile, so the tiles in flight at once share a few A rows
+    // and a few B rows in L2.
     const int nt = static_cast<int>((p.n + BN - 1) / BN);
-    ti.tm = local / nt;
-    ti.tn = local % nt;
+    const int mt = (ti.gend - ti.gstart + BM - 1) / BM;
+    const int band = local / (kBand * nt);
+    const int rem = local - band * kBand * nt;
+    const int bm = min(kBand, mt - band * kBand);
+    ti.tm = band * kBand + rem % bm;
+    ti.tn = rem / bm;
     ti.nk = static_cast<int>((p.k + BK - 1) / BK);
   } else {
     const int nt = static_cast<int>((p.k + BN - 1) / BN);
@@ -191,38 +200,68 @@ __device__ __forceinline__ bool epi_bar_and(bool v) {
   return r != 0;
 }
 
+// Epilogue of one 32-column chunk for the warp's 32 rows: scale in registers,
+// write the chunk to the warp's shared-memory tile (16-byte pieces swizzled by
+// row so that both the row-wise writes and the column-wise reads are free of
+// bank conflicts), then store whole row segments: 8 lanes cover 128
+// consecutive bytes of one output row.  Streaming stores keep the output from
+// evicting the operands from L2.
 template <int OUT>
-__device__ __forceinline__ void store_chunk(void *out_row, int64_t col0, int64_t ncols,
+__device__ __forceinline__ void store_chunk(float *stg, char *out_base, int64_t row_stride_bytes,
+                                            int valid_rows, int64_t col0, int64_t ncols,
                                             const uint32_t (&r)[32], float inv_a,
-                                            const float *inv_b) {
+                                            const float *inv_b, int lane) {
   if constexpr (OUT == FP8QGG_OUT_F32) {
-    float *o = static_cast<float *>(out_row) + col0;
 #pragma unroll
-    for (int v = 0; v < 8; ++v) {
-      if (col0 + 4 * v >= ncols) break;
+    for (int j = 0; j < 8; ++j) {
       float4 f;
-      f.x = __fmul_rn(__fmul_rn(__uint_as_float(r[4 * v + 0]), inv_a), inv_b[4 * v + 0]);
-      f.y = __fmul_rn(__fmul_rn(__uint_as_float(r[4 * v + 1]), inv_a), inv_b[4 * v + 1]);
-      f.z = __fmul_rn(__fmul_rn(__uint_as_float(r[4 * v + 2]), inv_a), inv_b[4 * v + 2]);
-      f.w = __fmul_rn(__fmul_rn(__uint_as_float(r[4 * v + 3]), inv_a), inv_b[4 * v + 3]);
-      *reinterpret_cast<float4 *>(o + 4 * v) = f;
+      f.x = __fmul_rn(__fmul_rn(__uint_as_float(r[4 * j + 0]), inv_a), inv_b[4 * j + 0]);
+      f.y = __fmul_rn(__fmul_rn(__uint_as_float(r[4 * j + 1]), inv_a), inv_b[4 * j + 1]);
+      f.z = __fmul_rn(__fmul_rn(__uint_as_float(r[4 * j + 2]), inv_a), inv_b[4 * j + 2]);
+      f.w = __fmul_rn(__fmul_rn(__uint_as_float(r[4 * j + 3]), inv_a), inv_b[4 * j + 3]);
+      *reinterpret_cast<float4 *>(stg + lane * 32 + 4 * (j ^ (lane & 7))) = f;
     }
-  } else {
-    __nv_bfloat16 *o = static_cast<__nv_bfloat16 *>(out_row) + col0;
+    __syncwarp();
 #pragma unroll
-    for (int v = 0; v < 4; ++v) {
-      if (col0 + 8 * v >= ncols) break;
+    for (int pss = 0; pss < 4; ++pss) {
+      const int lr = pss * 4 + (lane >> 3) + 0;
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        const int row = lr + 16 * half;
+        const int j = lane & 7;
+        const float4 v = *reinterpret_cast<const float4 *>(stg + row * 32 + 4 * (j ^ (row & 7)));
+        if (row < valid_rows && col0 + 4 * j < ncols)
+          __stcs(reinterpret_cast<float4 *>(out_base + row * row_stride_bytes) + (col0 / 4 + j),
+                 v);
+      }
+    }
+    __syncwarp();
+  } else {
+    uint32_t *sw = reinterpret_cast<uint32_t *>(stg);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
       uint32_t w[4];
 #pragma unroll
       for (int h = 0; h < 4; ++h) {
-        const int c = 8 * v + 2 * h;
+        const int c = 8 * j + 2 * h;
         const float f0 = __fmul_rn(__fmul_rn(__uint_as_float(r[c]), inv_a), inv_b[c]);
         const float f1 = __fmul_rn(__fmul_rn(__uint_as_float(r[c + 1]), inv_a), inv_b[c + 1]);
         __nv_bfloat162 b2 = __floats2bfloat162_rn(f0, f1);
         w[h] = *reinterpret_cast<uint32_t *>(&b2);
       }
-      *reinterpret_cast<uint4 *>(o + 8 * v) = make_uint4(w[0], w[1], w[2], w[3]);
+      *reinterpret_cast<uint4 *>(sw + lane * 16 + 4 * (j ^ ((lane >> 1) & 3))) =
+          make_uint4(w[0], w[1], w[2], w[3]);
     }
+    __syncwarp();
+#pragma unroll
+    for (int pss = 0; pss < 4; ++pss) {
+      const int row = pss * 8 + (lane >> 2);
+      const int j = lane & 3;
+      const uint4 v = *reinterpret_cast<const uint4 *>(sw + row * 16 + 4 * (j ^ ((row >> 1) & 3)));
+      if (row < valid_rows && col0 + 8 * j < ncols)
+        __stcs(reinterpret_cast<uint4 *>(out_base + row * row_stride_bytes) + (col0 / 8 + j), v);
+    }
+    __syncwarp();
   }
 }
 
@@ -360,7 +399,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     // ------------------------------------------------------------ epilogue
     const int et = threadIdx.x - 64;  // 0..127
     const int quarter = warp & 3;     // TMEM lanes [32*quarter, 32*quarter + 32)
-    const int row = 32 * quarter + lane;
+    float *stg = sm.stg[quarter];
+    constexpr int kOutBytes = OUT == FP8QGG_OUT_F32 ? 4 : 2;
+    const int64_t row_stride = p.ld_out * kOutBytes;
     uint32_t acc = 0, acc_phase = 0;
     for (int32_t t = blockIdx.x; t < total; t += gridDim.x) {
       const TileInfo ti = decode_tile<MODE>(sm, p, t);
@@ -373,22 +414,22 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         if (col < ncols) inv = __frcp_rn(__ldg(p.scale_b + ti.e * p.sbs + col));
         sm.inv_sb[acc][c] = inv;
       }
-      int64_t orow;
-      bool valid;
+      // this thread's accumulator row, and the warp's 32-row output window
+      int64_t row0;   // first output row of the warp's window
+      int valid_rows;  // rows of the window inside the group / matrix
+      char *out_base;
       float inv_a = 0.0f;
-      char *out_row;
       if constexpr (MODE == FP8QGG_M_JAGGED) {
-        orow = static_cast<int64_t>(ti.gstart) + static_cast<int64_t>(ti.tm) * BM + row;
-        valid = orow < ti.gend;
-        if (valid) inv_a = __frcp_rn(__ldg(p.scale_a + orow));
-        out_row = static_cast<char *>(p.out) +
-                  orow * p.ld_out * (OUT == FP8QGG_OUT_F32 ? 4 : 2);
+        row0 = static_cast<int64_t>(ti.gstart) + static_cast<int64_t>(ti.tm) * BM + 32 * quarter;
+        valid_rows = static_cast<int>(
+            ::max(int64_t(0), ::min(int64_t(32), static_cast<int64_t>(ti.gend) - row0)));
+        if (lane < valid_rows) inv_a = __frcp_rn(__ldg(p.scale_a + row0 + lane));
+        out_base = static_cast<char *>(p.out) + row0 * row_stride;
       } else {
-        orow = static_cast<int64_t>(ti.tm) * BM + row;
-        valid = orow < p.n;
-        if (valid) inv_a = __frcp_rn(__ldg(p.scale_a + ti.e * p.sas + orow));
-        out_row = static_cast<char *>(p.out) +
-                  (ti.e * p.out_gs + orow * p.ld_out) * (OUT == FP8QGG_OUT_F32 ? 4 : 2);
+        row0 = static_cast<int64_t>(ti.tm) * BM + 32 * quarter;
+        valid_rows = static_cast<int>(::max(int64_t(0), ::min(int64_t(32), p.n - row0)));
+        if (lane < valid_rows) inv_a = __frcp_rn(__ldg(p.scale_a + ti.e * p.sas + row0 + lane));
+        out_base = static_cast<char *>(p.out) + ti.e * p.out_gs * kOutBytes + row0 * row_stride;
       }
       const bool got = mbar_wait(&sm.tfull[acc], acc_phase, abort);
       if (!epi_bar_and(got)) {
@@ -400,6 +441,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(32 * quarter) << 16) + acc * BN;
 #pragma unroll 1
       for (int c = 0; c < BN / 32; ++c) {
+        const int64_t col0 = static_cast<int64_t>(ti.tn) * BN + 32 * c;
         uint32_t r[32];
         if (ti.nk > 0) {
           tmem_ld_32x32b_x32(taddr + 32 * c, r);
@@ -408,9 +450,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
           for (int i = 0; i < 32; ++i) r[i] = 0u;
         }
-        const int64_t col0 = static_cast<int64_t>(ti.tn) * BN + 32 * c;
-        if (valid && col0 < ncols)
-          store_chunk<OUT>(out_row, col0, ncols, r, inv_a, &sm.inv_sb[acc][32 * c]);
+        if (valid_rows > 0 && col0 < ncols)
+          store_chunk<OUT>(stg, out_base, row_stride, valid_rows, col0, ncols, r, inv_a,
+                           &sm.inv_sb[acc][32 * c], lane);
       }
       tc_fence_before_sync();
       mbar_arrive(&sm.tempty[acc]);

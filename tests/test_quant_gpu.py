@@ -256,3 +256,24 @@ def test_colwise_format_mismatch_is_counted_like_the_oracle(fmt, smax):
     assert (q.cpu().numpy() == q_ref).all()
     assert (s.cpu().numpy() == s_ref).all()
     assert int(sat.item()) == sat_ref
+
+
+@pytest.mark.parametrize("layout", [qgg.LAYOUT_SAME, qgg.LAYOUT_TRANSPOSED])
+def test_colwise_tall_groups_split_over_many_blocks(layout):
+    """Groups of 20k and 9k rows: 53 and 24 chunks per column tile combine their
+    partial absmax across blocks."""
+    sizes = [20011, 3, 9000, 0, 385]
+    m, cols = sum(sizes), 136
+    x = rand_bf16(31, m, cols, outliers=0.001)
+    off = wl.offsets_from_sizes(sizes)
+    ld = (m + 15) // 16 * 16
+    q_ref, s_ref, _ = orc.quant_colwise_jagged(bits(x), off, layout, ld_q=ld if layout else None)
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    q, s = qgg.fp8_quant_colwise_jagged(dev(x), torch.from_numpy(off).cuda(), layout,
+                                        ld_q=ld, status=st)
+    qn = q.cpu().numpy()
+    if layout == qgg.LAYOUT_TRANSPOSED:
+        qn, q_ref = qn[:, :m], q_ref[:, :m]
+    assert (qn == q_ref).all()
+    assert (s.cpu().numpy().view(np.uint32) == s_ref.view(np.uint32)).all()
+    assert int(st.item()) == 0
