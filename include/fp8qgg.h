@@ -164,6 +164,37 @@ int fp8_quant_colwise_jagged(const void *x, int64_t rows_total, int64_t cols, in
                              void *stream);
 
 /*
+ * Same computation as fp8_quant_colwise_jagged, for callers that cannot
+ * allocate device memory or supply a workspace (for example a runtime that
+ * fixes its memory budget at start-up and forbids cudaMalloc later, or a
+ * plugin interface that passes tensors but no scratch buffer).  The pages
+ * have no counterpart to this entry point; it exists only for such callers.
+ *
+ * It calls no cudaMalloc/cudaFree and no allocating routine.  Its scratch is a
+ * fixed device array of FP8QGG_NOALLOC_SCRATCH_BYTES inside the library, held
+ * by every GPU that loads the library until the process exits.
+ *  - Size limit: problems whose fp8_quant_colwise_jagged_workspace_size(...)
+ *    exceeds FP8QGG_NOALLOC_SCRATCH_BYTES are rejected with FP8QGG_ERR_SHAPE
+ *    before anything is enqueued (with 64-column tiles that is num_groups *
+ *    cols * 4 bytes plus a small counter area; e.g. 64 groups x 7168 columns
+ *    fits).
+ *  - Set-up: the first call on each device looks up the array's device
+ *    address with that device current (cudaGetSymbolAddress).  Make that
+ *    first call before any stream capture on the device.
+ *  - Sharing: every call uses the same array and clears the part it needs on
+ *    `stream` first.  Calls on one device whose executions could overlap on
+ *    the GPU race; order them (one stream, or events).
+ * Arguments, layouts, requirements and errors are otherwise those of
+ * fp8_quant_colwise_jagged without the workspace pair.
+ */
+#define FP8QGG_NOALLOC_SCRATCH_BYTES (2u * 1024u * 1024u)
+int fp8_quant_colwise_jagged_noalloc(const void *x, int64_t rows_total, int64_t cols,
+                                     int64_t ld_x, const int32_t *offsets, int32_t num_groups,
+                                     uint8_t *q, int64_t ld_q, int layout, float *scales,
+                                     int fmt, float scale_max, uint64_t *sat_count,
+                                     int32_t *dev_status, void *stream);
+
+/*
  * FP8 scaled grouped GEMM on the 5th-generation tensor cores (the pages run
  * the expert GEMMs as one grouped GEMM over FP8 operands: [ABP] third
  * paragraph; [PRI] "What Primus adds").  e4m3fn operands, fp32 accumulation.

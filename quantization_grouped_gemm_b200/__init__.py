@@ -48,6 +48,8 @@ _SIGNATURES = {
                                        _I32, _I64, _I64, _I64, _P, _I64, _I64, _INT, _INT, _P,
                                        _P]),
     "fp8_cast_f32": (_INT, [_P, _I64, _P, _INT, _P]),
+    "fp8_quant_colwise_jagged_noalloc": (_INT, [_P, _I64, _I64, _I64, _P, _I32, _P, _I64, _INT,
+                                                _P, _INT, _F32, _P, _P, _P]),
 }
 
 

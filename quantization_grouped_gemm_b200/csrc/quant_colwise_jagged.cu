@@ -29,6 +29,7 @@
 //      consecutive addresses.
 #include <algorithm>
 #include <cstring>
+#include <mutex>
 
 #include "device_common.cuh"
 #include "host_common.h"
@@ -452,6 +453,72 @@ extern "C" int fp8_quant_colwise_jagged(const void *x, int64_t rows_total, int64
   if (cudaMemsetAsync(workspace, 0, need, s) != cudaSuccess) return FP8QGG_ERR_CUDA;
   uint32_t *ws_amax = static_cast<uint32_t *>(workspace);
   uint32_t *ws_cnt = reinterpret_cast<uint32_t *>(static_cast<uint8_t *>(workspace) +
+                                                  colwise_amax_bytes(cols, num_groups));
+  return colwise_launch(x, rows_total, cols, ld_x, offsets, num_groups, q, ld_q, layout, scales,
+                        fmt, scale_max, sat_count, dev_status, ws_amax, ws_cnt, s);
+}
+
+// ---------------------------------------------------------------------------
+// Entry point for callers that must not allocate device memory.
+//
+// Some callers cannot hand this library a workspace: runtimes that plan their
+// whole device-memory budget up front and forbid cudaMalloc afterwards (an
+// allocation can synchronise the device and fragments the plan), or plugin
+// interfaces that pass tensors but no scratch buffer.  For them the scratch
+// lives in a fixed array in this library's device image instead.  Each GPU that
+// loads the library holds this array (kNoAllocScratchBytes) until the process
+// exits.  All calls share it, so calls on one device that could overlap in time
+// on the GPU race with each other; order them on one stream (or with events).
+
+namespace fp8qgg {
+
+constexpr size_t kNoAllocScratchBytes = FP8QGG_NOALLOC_SCRATCH_BYTES;
+static_assert(kNoAllocScratchBytes % 256 == 0, "scratch must keep 256-byte granules");
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+namespace {
+constexpr int kMaxScratchDevices = 64;
+void *g_scratch_addr[kMaxScratchDevices];
+std::mutex g_scratch_mutex;
+}  // namespace
+
+// Device address of the fixed scratch array on the current device.  In host
+// code `g_noalloc_scratch` only names a host-side stand-in, so the address is
+// looked up once per device (with that device current) and cached.
+static bool noalloc_scratch(void **out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxScratchDevices) return false;
+  std::lock_guard<std::mutex> lock(g_scratch_mutex);
+  if (!g_scratch_addr[dev]) {
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return false;
+    g_scratch_addr[dev] = p;
+  }
+  *out = g_scratch_addr[dev];
+  return true;
+}
+
+}  // namespace fp8qgg
+
+extern "C" int fp8_quant_colwise_jagged_noalloc(const void *x, int64_t rows_total, int64_t cols,
+                                                int64_t ld_x, const int32_t *offsets,
+                                                int32_t num_groups, uint8_t *q, int64_t ld_q,
+                                                int layout, float *scales, int fmt,
+                                                float scale_max, uint64_t *sat_count,
+                                                int32_t *dev_status, void *stream) {
+  int rc = colwise_check(x, rows_total, cols, ld_x, offsets, num_groups, q, ld_q, layout, scales,
+                         fmt, scale_max, sat_count, dev_status);
+  if (rc != FP8QGG_OK) return rc;
+  const size_t need = fp8_quant_colwise_jagged_workspace_size(rows_total, cols, num_groups);
+  if (need > kNoAllocScratchBytes) return FP8QGG_ERR_SHAPE;
+  void *scratch = nullptr;
+  if (!noalloc_scratch(&scratch)) return FP8QGG_ERR_CUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // the previous call's partial maxima and counters must not leak into this one
+  if (cudaMemsetAsync(scratch, 0, need, s) != cudaSuccess) return FP8QGG_ERR_CUDA;
+  uint32_t *ws_amax = static_cast<uint32_t *>(scratch);
+  uint32_t *ws_cnt = reinterpret_cast<uint32_t *>(static_cast<uint8_t *>(scratch) +
                                                   colwise_amax_bytes(cols, num_groups));
   return colwise_launch(x, rows_total, cols, ld_x, offsets, num_groups, q, ld_q, layout, scales,
                         fmt, scale_max, sat_count, dev_status, ws_amax, ws_cnt, s);

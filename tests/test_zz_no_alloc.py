@@ -1,0 +1,88 @@
+"""The no-allocation variant of the jagged column-wise quantisation.
+
+Callers such as runtimes that fix their device-memory budget at start-up (and
+forbid cudaMalloc afterwards) or plugin interfaces that hand over tensors but
+no scratch buffer cannot pass a workspace.  fp8_quant_colwise_jagged_noalloc
+serves them from a fixed scratch array inside the library.  These checks call
+it through the C ABI and require the same codes and scales as the regular
+entry point, on two calls in a row (the second call must not see the first
+call's leftovers in the shared scratch).
+
+The file name sorts last so that a run stopping at the first failure has
+already run every other test.
+"""
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+import quantization_grouped_gemm_b200 as qgg
+from quantization_grouped_gemm_b200 import workloads as wl
+
+pytestmark = pytest.mark.gpu
+
+
+def _p(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else None
+
+
+def call_noalloc(x, off, layout, q, scales, fmt=qgg.E4M3FN, status=None):
+    lib = qgg.lib()
+    rows, cols = x.shape
+    ld_q = q.stride(0) if q.shape[0] > 1 else q.shape[1]
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    return lib.fp8_quant_colwise_jagged_noalloc(
+        _p(x), rows, cols, x.stride(0), _p(off), off.numel(), _p(q), ld_q, layout, _p(scales),
+        fmt, 0.0, None, _p(status), stream)
+
+
+def make_case(seed, sizes, cols):
+    m = int(sum(sizes))
+    g = np.random.default_rng(seed)
+    a = g.standard_normal((m, cols)).astype(np.float32)
+    a.reshape(-1)[g.integers(0, a.size, max(1, a.size // 500))] *= 50
+    x = wl.to_bf16(a).cuda()
+    off = torch.from_numpy(wl.offsets_from_sizes(sizes)).cuda()
+    return x, off
+
+
+@pytest.mark.parametrize("layout", [qgg.LAYOUT_SAME, qgg.LAYOUT_TRANSPOSED])
+def test_noalloc_matches_regular_entry_point_on_two_calls_in_a_row(layout):
+    # two different problems back to back: both use the shared scratch for
+    # groups taller than one block's chunk
+    cases = [make_case(1, [2500, 0, 17, 1300, 5], 200), make_case(2, [700, 4100, 3], 136)]
+    outs = []
+    for x, off in cases:
+        m, cols = x.shape
+        ld = (m + 15) // 16 * 16
+        shape = (cols, ld) if layout == qgg.LAYOUT_TRANSPOSED else (m, cols)
+        q = torch.full(shape, 0xAB, dtype=torch.uint8, device="cuda")
+        s = torch.full((off.numel(), cols), -1.0, device="cuda")
+        st = torch.zeros(1, dtype=torch.int32, device="cuda")
+        assert call_noalloc(x, off, layout, q, s, status=st) == 0
+        outs.append((q, s, st))
+    torch.cuda.synchronize()
+    for (x, off), (q, s, st) in zip(cases, outs):
+        m = x.shape[0]
+        q_ref, s_ref = qgg.fp8_quant_colwise_jagged(x, off, layout,
+                                                    ld_q=q.shape[1] if layout else None)
+        torch.cuda.synchronize()
+        if layout == qgg.LAYOUT_TRANSPOSED:
+            assert torch.equal(q[:, :m], q_ref[:, :m])
+        else:
+            assert torch.equal(q, q_ref)
+        assert torch.equal(s, s_ref)
+        assert int(st.item()) == 0
+
+
+def test_noalloc_rejects_problems_beyond_its_scratch():
+    lib = qgg.lib()
+    groups, cols = 1024, 1024  # needs 4 MiB of partial maxima: above the fixed scratch
+    assert qgg.colwise_workspace_bytes(100, cols, groups) > 2 * 1024 * 1024
+    x = torch.zeros((100, cols), dtype=torch.bfloat16, device="cuda")
+    off = torch.full((groups,), 100, dtype=torch.int32, device="cuda")
+    q = torch.empty((100, cols), dtype=torch.uint8, device="cuda")
+    s = torch.empty((groups, cols), device="cuda")
+    rc = call_noalloc(x, off, qgg.LAYOUT_SAME, q, s)
+    assert rc == -2, lib.fp8qgg_error_string(rc)
