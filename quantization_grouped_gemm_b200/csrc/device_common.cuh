@@ -245,6 +245,30 @@ __device__ __forceinline__ uint32_t quant_pair(uint32_t packed, float s, float s
   return cvt_x2<FMT>(y0, y1);
 }
 
+// Fast form of quant_pair for the common case: no saturation count, and no
+// clamp because the scaling maximum is at least the format's largest finite
+// value.  Then clamping to +-smax before the saturating encode changes no code
+// (a value beyond the format maximum saturates to it either way), so the two
+// products go straight to the encoder.  Both products come from one packed
+// instruction (two IEEE round-to-nearest fp32 multiplies).
+template <int FMT>
+__device__ __forceinline__ uint32_t quant_pair_fast(uint32_t packed, uint64_t s2) {
+  const float x0 = __uint_as_float(packed << 16);
+  const float x1 = __uint_as_float(packed & 0xFFFF0000u);
+  uint64_t xx, yy;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(xx) : "f"(x0), "f"(x1));
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(yy) : "l"(xx), "l"(s2));
+  float y0, y1;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(y0), "=f"(y1) : "l"(yy));
+  return cvt_x2<FMT>(y0, y1);
+}
+
+__device__ __forceinline__ uint64_t pack_f32x2(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+
 // Per-halfword unsigned max of |bf16| bit patterns: the absolute value of a
 // finite bf16 compares like its 15-bit magnitude pattern.
 __device__ __forceinline__ uint32_t abs_max_bf16x2(uint32_t acc, uint32_t packed) {

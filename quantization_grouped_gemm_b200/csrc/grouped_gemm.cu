@@ -439,20 +439,29 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       }
       tc_fence_after_sync();
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(32 * quarter) << 16) + acc * BN;
+      // two 32-column TMEM loads per wait: the second load's latency hides
+      // behind the first's
 #pragma unroll 1
-      for (int c = 0; c < BN / 32; ++c) {
-        const int64_t col0 = static_cast<int64_t>(ti.tn) * BN + 32 * c;
-        uint32_t r[32];
+      for (int c = 0; c < BN / 32; c += 2) {
+        uint32_t r0[32], r1[32];
         if (ti.nk > 0) {
-          tmem_ld_32x32b_x32(taddr + 32 * c, r);
+          tmem_ld_32x32b_x32(taddr + 32 * c, r0);
+          tmem_ld_32x32b_x32(taddr + 32 * (c + 1), r1);
           tmem_ld_wait();
         } else {
 #pragma unroll
-          for (int i = 0; i < 32; ++i) r[i] = 0u;
+          for (int i = 0; i < 32; ++i) {
+            r0[i] = 0u;
+            r1[i] = 0u;
+          }
         }
+        const int64_t col0 = static_cast<int64_t>(ti.tn) * BN + 32 * c;
         if (valid_rows > 0 && col0 < ncols)
-          store_chunk<OUT>(stg, out_base, row_stride, valid_rows, col0, ncols, r, inv_a,
+          store_chunk<OUT>(stg, out_base, row_stride, valid_rows, col0, ncols, r0, inv_a,
                            &sm.inv_sb[acc][32 * c], lane);
+        if (valid_rows > 0 && col0 + 32 < ncols)
+          store_chunk<OUT>(stg, out_base, row_stride, valid_rows, col0 + 32, ncols, r1, inv_a,
+                           &sm.inv_sb[acc][32 * (c + 1)], lane);
       }
       tc_fence_before_sync();
       mbar_arrive(&sm.tempty[acc]);

@@ -127,7 +127,7 @@ __device__ __forceinline__ uint32_t quant_pair2(uint32_t packed, float s0, float
   return cvt_x2<FMT>(y0, y1);
 }
 
-template <int FMT, int LAYOUT>
+template <int FMT, int LAYOUT, bool FAST>
 __global__ void __launch_bounds__(kColThreads, 2)
     quant_colwise_jagged_kernel(const __grid_constant__ CUtensorMap xmap, int64_t rows_total,
                                 int cols, const int32_t *__restrict__ offsets, int num_groups,
@@ -252,15 +252,23 @@ __global__ void __launch_bounds__(kColThreads, 2)
         const uint4 v = *reinterpret_cast<const uint4 *>(&sm.tile[rr * 32 + 4 * j]);
         const float *s = &sm.scale[8 * j];
         uint2 o;
-        o.x = quant_pair2<FMT>(v.x, s[0], s[1], smax, sat_thr, sat) |
-              (quant_pair2<FMT>(v.y, s[2], s[3], smax, sat_thr, sat) << 16);
-        o.y = quant_pair2<FMT>(v.z, s[4], s[5], smax, sat_thr, sat) |
-              (quant_pair2<FMT>(v.w, s[6], s[7], smax, sat_thr, sat) << 16);
+        if constexpr (FAST) {
+          o.x = quant_pair_fast<FMT>(v.x, pack_f32x2(s[0], s[1])) |
+                (quant_pair_fast<FMT>(v.y, pack_f32x2(s[2], s[3])) << 16);
+          o.y = quant_pair_fast<FMT>(v.z, pack_f32x2(s[4], s[5])) |
+                (quant_pair_fast<FMT>(v.w, pack_f32x2(s[6], s[7])) << 16);
+        } else {
+          o.x = quant_pair2<FMT>(v.x, s[0], s[1], smax, sat_thr, sat) |
+                (quant_pair2<FMT>(v.y, s[2], s[3], smax, sat_thr, sat) << 16);
+          o.y = quant_pair2<FMT>(v.z, s[4], s[5], smax, sat_thr, sat) |
+                (quant_pair2<FMT>(v.w, s[6], s[7], smax, sat_thr, sat) << 16);
+        }
         *reinterpret_cast<uint2 *>(q + static_cast<int64_t>(r0 + rr) * ld_q + c0 + 8 * j) = o;
       }
     } else {
       const float s0 = sm.scale[2 * lane];
       const float s1 = sm.scale[2 * lane + 1];
+      const uint64_t s01 = pack_f32x2(s0, s1);
       for (int32_t A = r0 & ~15; A < r1; A += kStgRows) {
         // cast: warp w covers tokens [A + 16w, A + 16w + 16) of column pair `lane`
         const int32_t gb = A + 16 * warp;
@@ -271,7 +279,11 @@ __global__ void __launch_bounds__(kColThreads, 2)
           for (int i = 0; i < 16; ++i) {
             const int32_t g = gb + i;
             const uint32_t wv = (g >= r0 && g < r1) ? sm.tile[(g - r0) * 32 + lane] : 0u;
-            const uint32_t c2 = quant_pair2<FMT>(wv, s0, s1, smax, sat_thr, sat);
+            uint32_t c2;
+            if constexpr (FAST)
+              c2 = quant_pair_fast<FMT>(wv, s01);
+            else
+              c2 = quant_pair2<FMT>(wv, s0, s1, smax, sat_thr, sat);
             lo4[i >> 2] |= (c2 & 0xFFu) << (8 * (i & 3));
             hi4[i >> 2] |= (c2 >> 8) << (8 * (i & 3));
           }
@@ -305,7 +317,7 @@ __global__ void __launch_bounds__(kColThreads, 2)
     __syncthreads();
   }
 
-  if (sat_count) {
+  if (!FAST && sat_count) {
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) sat += __shfl_xor_sync(0xFFFFFFFFu, sat, off);
     if (lane == 0 && sat) atomicAdd(sat_count, static_cast<unsigned long long>(sat));
@@ -318,14 +330,20 @@ using ColKernel = void (*)(const CUtensorMap, int64_t, int, const int32_t *, int
                            int64_t, float *, float, float, unsigned long long *, int32_t *,
                            uint32_t *, uint32_t *);
 
-ColKernel col_kernel(int fmt, int layout) {
-  if (fmt == FP8QGG_E4M3FN)
-    return layout == FP8QGG_LAYOUT_SAME
-               ? quant_colwise_jagged_kernel<FP8QGG_E4M3FN, FP8QGG_LAYOUT_SAME>
-               : quant_colwise_jagged_kernel<FP8QGG_E4M3FN, FP8QGG_LAYOUT_TRANSPOSED>;
+template <int FMT, bool FAST>
+ColKernel col_kernel_fmt(int layout) {
   return layout == FP8QGG_LAYOUT_SAME
-             ? quant_colwise_jagged_kernel<FP8QGG_E4M3FNUZ, FP8QGG_LAYOUT_SAME>
-             : quant_colwise_jagged_kernel<FP8QGG_E4M3FNUZ, FP8QGG_LAYOUT_TRANSPOSED>;
+             ? quant_colwise_jagged_kernel<FMT, FP8QGG_LAYOUT_SAME, FAST>
+             : quant_colwise_jagged_kernel<FMT, FP8QGG_LAYOUT_TRANSPOSED, FAST>;
+}
+
+// The fast kernels skip the clamp and the saturation count (see quant_pair_fast).
+ColKernel col_kernel(int fmt, int layout, bool fast) {
+  if (fmt == FP8QGG_E4M3FN)
+    return fast ? col_kernel_fmt<FP8QGG_E4M3FN, true>(layout)
+                : col_kernel_fmt<FP8QGG_E4M3FN, false>(layout);
+  return fast ? col_kernel_fmt<FP8QGG_E4M3FNUZ, true>(layout)
+              : col_kernel_fmt<FP8QGG_E4M3FNUZ, false>(layout);
 }
 
 size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
@@ -392,7 +410,9 @@ int colwise_launch(const void *x, int64_t rows_total, int64_t cols, int64_t ld_x
 
   DeviceInfo dev;
   if (!device_info(&dev)) return FP8QGG_ERR_CUDA;
-  ColKernel kern = col_kernel(fmt, layout);
+  const float smax_eff = effective_scale_max(fmt, scale_max);
+  ColKernel kern =
+      col_kernel(fmt, layout, sat_count == nullptr && smax_eff >= format_max(fmt));
   const int smem = static_cast<int>(sizeof(ColSmem)) + 1024;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
       cudaSuccess)

@@ -25,7 +25,7 @@ __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
-template <int VPL, int G, int FMT>
+template <int VPL, int G, int FMT, bool FAST>
 __global__ void __launch_bounds__(kRowThreads)
     quant_rowwise_kernel(const uint4 *__restrict__ x, int64_t rows, int nvec, int64_t ld_x_vec,
                          uint8_t *__restrict__ q, int64_t ld_q, float *__restrict__ scales,
@@ -79,15 +79,21 @@ __global__ void __launch_bounds__(kRowThreads)
       const int idx = (i * G + wt) * 32 + lane;
       if (idx < nvec) {
         uint2 o;
-        o.x = quant_pair<FMT>(v[i].x, s, smax, sat_thr, sat) |
-              (quant_pair<FMT>(v[i].y, s, smax, sat_thr, sat) << 16);
-        o.y = quant_pair<FMT>(v[i].z, s, smax, sat_thr, sat) |
-              (quant_pair<FMT>(v[i].w, s, smax, sat_thr, sat) << 16);
+        if constexpr (FAST) {
+          const uint64_t s2 = pack_f32x2(s, s);
+          o.x = quant_pair_fast<FMT>(v[i].x, s2) | (quant_pair_fast<FMT>(v[i].y, s2) << 16);
+          o.y = quant_pair_fast<FMT>(v[i].z, s2) | (quant_pair_fast<FMT>(v[i].w, s2) << 16);
+        } else {
+          o.x = quant_pair<FMT>(v[i].x, s, smax, sat_thr, sat) |
+                (quant_pair<FMT>(v[i].y, s, smax, sat_thr, sat) << 16);
+          o.y = quant_pair<FMT>(v[i].z, s, smax, sat_thr, sat) |
+                (quant_pair<FMT>(v[i].w, s, smax, sat_thr, sat) << 16);
+        }
         *reinterpret_cast<uint2 *>(qr + static_cast<int64_t>(idx) * 8) = o;
       }
     }
   }
-  if (sat_count) {
+  if (!FAST && sat_count) {
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) sat += __shfl_xor_sync(0xFFFFFFFFu, sat, off);
     if (lane == 0 && sat) atomicAdd(sat_count, static_cast<unsigned long long>(sat));
@@ -104,29 +110,32 @@ constexpr int kNumVpl = sizeof(kVplChoices) / sizeof(kVplChoices[0]);
 constexpr int kGChoices[] = {1, 2, 4, 8};
 constexpr int kNumG = 4;
 
-template <int FMT, int GI, int VI>
+template <int FMT, bool FAST, int GI, int VI>
 RowKernel row_kernel_at() {
-  return quant_rowwise_kernel<kVplChoices[VI], kGChoices[GI], FMT>;
+  return quant_rowwise_kernel<kVplChoices[VI], kGChoices[GI], FMT, FAST>;
 }
 
-template <int FMT, int GI, int... VIs>
+template <int FMT, bool FAST, int GI, int... VIs>
 void fill_row(RowKernel *t, std::integer_sequence<int, VIs...>) {
-  ((t[GI * kNumVpl + VIs] = row_kernel_at<FMT, GI, VIs>()), ...);
+  ((t[GI * kNumVpl + VIs] = row_kernel_at<FMT, FAST, GI, VIs>()), ...);
 }
 
-template <int FMT>
+template <int FMT, bool FAST>
 void fill_table(RowKernel *t) {
-  fill_row<FMT, 0>(t, std::make_integer_sequence<int, kNumVpl>{});
-  fill_row<FMT, 1>(t, std::make_integer_sequence<int, kNumVpl>{});
-  fill_row<FMT, 2>(t, std::make_integer_sequence<int, kNumVpl>{});
-  fill_row<FMT, 3>(t, std::make_integer_sequence<int, kNumVpl>{});
+  fill_row<FMT, FAST, 0>(t, std::make_integer_sequence<int, kNumVpl>{});
+  fill_row<FMT, FAST, 1>(t, std::make_integer_sequence<int, kNumVpl>{});
+  fill_row<FMT, FAST, 2>(t, std::make_integer_sequence<int, kNumVpl>{});
+  fill_row<FMT, FAST, 3>(t, std::make_integer_sequence<int, kNumVpl>{});
 }
 
+// [format][fast]: the fast kernels skip the clamp and the saturation count
 struct RowTable {
-  RowKernel k[2][kNumG * kNumVpl];
+  RowKernel k[2][2][kNumG * kNumVpl];
   RowTable() {
-    fill_table<FP8QGG_E4M3FN>(k[0]);
-    fill_table<FP8QGG_E4M3FNUZ>(k[1]);
+    fill_table<FP8QGG_E4M3FN, false>(k[0][0]);
+    fill_table<FP8QGG_E4M3FN, true>(k[0][1]);
+    fill_table<FP8QGG_E4M3FNUZ, false>(k[1][0]);
+    fill_table<FP8QGG_E4M3FNUZ, true>(k[1][1]);
   }
 };
 
@@ -172,7 +181,10 @@ extern "C" int fp8_quant_rowwise(const void *x, int64_t rows, int64_t cols, int6
 
   int gi = 0, vi = 0;
   if (!rowwise_plan(cols / 8, &gi, &vi)) return FP8QGG_ERR_SHAPE;
-  RowKernel kern = row_table().k[fmt][gi * kNumVpl + vi];
+  const float smax = effective_scale_max(fmt, scale_max);
+  const float sat_thr = saturation_threshold(fmt);
+  const bool fast = sat_count == nullptr && smax >= format_max(fmt);
+  RowKernel kern = row_table().k[fmt][fast ? 1 : 0][gi * kNumVpl + vi];
 
   DeviceInfo dev;
   if (!device_info(&dev)) return FP8QGG_ERR_CUDA;
@@ -185,8 +197,6 @@ extern "C" int fp8_quant_rowwise(const void *x, int64_t rows, int64_t cols, int6
   const int64_t want = (rows + teams - 1) / teams;
   const int grid = static_cast<int>(std::min<int64_t>(want, int64_t(per_sm) * dev.sm_count));
 
-  const float smax = effective_scale_max(fmt, scale_max);
-  const float sat_thr = saturation_threshold(fmt);
   kern<<<grid, kRowThreads, 0, static_cast<cudaStream_t>(stream)>>>(
       static_cast<const uint4 *>(x), rows, static_cast<int>(cols / 8), ld_x / 8, q, ld_q, scales,
       smax, sat_thr, reinterpret_cast<unsigned long long *>(sat_count));
