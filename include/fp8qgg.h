@@ -84,7 +84,7 @@ extern "C" {
 /* bits OR-ed into *dev_status */
 #define FP8QGG_STATUS_BAD_OFFSETS 1  /* offsets had to be clamped */
 #define FP8QGG_STATUS_TIMEOUT 2      /* a bounded device-side wait gave up */
-#define FP8QGG_STATUS_GROUP_TOO_TALL 4 /* a group exceeded the single-pass limit */
+#define FP8QGG_STATUS_GROUP_TOO_TALL 4 /* reserved (no current kernel sets it) */
 
 /* The FP8 variant this device's tensor cores consume.  The pages add
  * automatic detection of the format because the wrong maximum corrupts
@@ -122,9 +122,8 @@ int fp8_quant_rowwise(const void *x, int64_t rows, int64_t cols, int64_t ld_x,
                       int fmt, float scale_max, uint64_t *sat_count, void *stream);
 
 /*
- * Bytes of device workspace fp8_quant_colwise_jagged needs for this problem
- * (cross-block absmax partials and arrival counters for groups taller than
- * one block's on-chip chunk).  Always > 0.
+ * Bytes of device workspace fp8_quant_colwise_jagged needs (a work counter
+ * shared by the blocks; 256 bytes whatever the problem).  Always > 0.
  */
 size_t fp8_quant_colwise_jagged_workspace_size(int64_t rows_total, int64_t cols,
                                                int32_t num_groups);
@@ -152,9 +151,9 @@ size_t fp8_quant_colwise_jagged_workspace_size(int64_t rows_total, int64_t cols,
  *            share one workspace must be ordered on the device.
  * Requirements: rows_total >= 0; cols in [1, 2^31) and a multiple of 8;
  * num_groups in [1, 1024]; ld_x >= cols, ld_x % 8 == 0; x, q and workspace
- * 16-byte aligned.  One group may hold at most (resident blocks) x 512 rows
- * (about 150k rows on a B200); a taller group sets
- * FP8QGG_STATUS_GROUP_TOO_TALL and its codes are not valid.
+ * 16-byte aligned.  Groups of any height are handled: up to 3072 rows a
+ * (group, 32-column) block of x is read from HBM once; a taller group's block
+ * is read a second time for the cast, while it is still in L2.
  */
 int fp8_quant_colwise_jagged(const void *x, int64_t rows_total, int64_t cols, int64_t ld_x,
                              const int32_t *offsets, int32_t num_groups,
@@ -175,9 +174,8 @@ int fp8_quant_colwise_jagged(const void *x, int64_t rows_total, int64_t cols, in
  * by every GPU that loads the library until the process exits.
  *  - Size limit: problems whose fp8_quant_colwise_jagged_workspace_size(...)
  *    exceeds FP8QGG_NOALLOC_SCRATCH_BYTES are rejected with FP8QGG_ERR_SHAPE
- *    before anything is enqueued (with 64-column tiles that is num_groups *
- *    cols * 4 bytes plus a small counter area; e.g. 64 groups x 7168 columns
- *    fits).
+ *    before anything is enqueued (the current kernel needs 256 bytes for any
+ *    problem, so every valid problem fits).
  *  - Set-up: the first call on each device looks up the array's device
  *    address with that device current (cudaGetSymbolAddress).  Make that
  *    first call before any stream capture on the device.

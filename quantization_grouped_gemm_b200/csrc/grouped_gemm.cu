@@ -51,6 +51,7 @@ struct GemmSmem {
   float inv_sb[2][BN];
   int32_t end[kMaxGemmGroups];
   int32_t tile_prefix[kMaxGemmGroups + 1];
+  int32_t order[kMaxGemmGroups];  // contraction-jagged mode: groups, largest first
   uint64_t full[kStages];
   uint64_t empty[kStages];
   uint64_t tfull[2];
@@ -113,6 +114,47 @@ __device__ __forceinline__ TileInfo decode_tile(const GemmSmem &sm, const GemmPa
     ti.nk = ti.gend > ti.gstart ? (ti.gend - (ti.gstart & ~15) + BK - 1) / BK : 0;
   }
   return ti;
+}
+
+// Contraction-jagged mode: every group has the same number of tiles, but a
+// tile's cost grows with the group's token count.  Position `pos` of the list
+// sorted by group size (largest first) maps to group order[pos / tpg].
+__device__ __forceinline__ TileInfo decode_tile_sorted(const GemmSmem &sm, const GemmParams &p,
+                                                       int32_t pos) {
+  const int32_t tpg = sm.tile_prefix[1] - sm.tile_prefix[0];
+  const int e = sm.order[pos / tpg];
+  const int32_t local = pos - (pos / tpg) * tpg;
+  TileInfo ti;
+  ti.e = e;
+  ti.gstart = e ? sm.end[e - 1] : 0;
+  ti.gend = sm.end[e];
+  const int nt = static_cast<int>((p.k + BN - 1) / BN);
+  ti.tm = local / nt;
+  ti.tn = local % nt;
+  ti.nk = ti.gend > ti.gstart ? (ti.gend - (ti.gstart & ~15) + BK - 1) / BK : 0;
+  return ti;
+}
+
+// The i-th tile of this CTA.  Token-jagged mode: plain grid stride (tiles
+// cost the same).  Contraction-jagged mode: rounds of gridDim.x tiles taken in
+// alternating directions over the size-sorted list, so that every CTA gets a
+// similar mix of long and short tiles.  Returns a position >= total when the
+// CTA has no i-th tile.
+template <int MODE>
+__device__ __forceinline__ int32_t tile_position(int32_t i) {
+  const int32_t G = static_cast<int32_t>(gridDim.x);
+  const int32_t b = static_cast<int32_t>(blockIdx.x);
+  if constexpr (MODE == FP8QGG_M_JAGGED) return b + i * G;
+  return i * G + ((i & 1) ? (G - 1 - b) : b);
+}
+
+template <int MODE>
+__device__ __forceinline__ TileInfo tile_at(const GemmSmem &sm, const GemmParams &p,
+                                            int32_t pos) {
+  if constexpr (MODE == FP8QGG_M_JAGGED)
+    return decode_tile<MODE>(sm, p, pos);
+  else
+    return decode_tile_sorted(sm, p, pos);
 }
 
 // Clamped group ends and cumulative tile counts, warp-parallel (one warp).
@@ -298,6 +340,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   tc_fence_before_sync();
   __syncthreads();
   tc_fence_after_sync();
+  if constexpr (MODE == FP8QGG_K_JAGGED) {
+    // rank of each group by token count (ties by index): order[rank] = group
+    for (int e = threadIdx.x; e < p.num_groups; e += kGemmThreads) {
+      const int32_t se = sm.end[e] - (e ? sm.end[e - 1] : 0);
+      int rank = 0;
+      for (int f = 0; f < p.num_groups; ++f) {
+        const int32_t sf = sm.end[f] - (f ? sm.end[f - 1] : 0);
+        rank += (sf > se) || (sf == se && f < e);
+      }
+      sm.order[rank] = e;
+    }
+    __syncthreads();
+  }
 
   const int32_t total = sm.tile_prefix[p.num_groups];
   volatile int *abort = &sm.abort;
@@ -310,8 +365,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       uint32_t armed = 0;  // stages with a load issued
       uint32_t last_par[kStages] = {0, 0, 0, 0};
       bool ok = true;
-      for (int32_t t = blockIdx.x; t < total && ok; t += gridDim.x) {
-        const TileInfo ti = decode_tile<MODE>(sm, p, t);
+      for (int32_t i = 0, t = tile_position<MODE>(0); t < total && ok;
+           t = tile_position<MODE>(++i)) {
+        const TileInfo ti = tile_at<MODE>(sm, p, t);
         for (int kb = 0; kb < ti.nk; ++kb) {
           if (!mbar_wait(&sm.empty[stage], phase ^ 1, abort)) { ok = false; break; }
           mbar_arrive_expect_tx(&sm.full[stage], kStageBytes);
@@ -341,8 +397,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     // ------------------------------------------------------------ MMA issuer
     uint32_t stage = 0, phase = 0, acc = 0, acc_phase = 0;
     bool ok = true;
-    for (int32_t t = blockIdx.x; t < total && ok; t += gridDim.x) {
-      const TileInfo ti = decode_tile<MODE>(sm, p, t);
+    for (int32_t i = 0, t = tile_position<MODE>(0); t < total && ok;
+         t = tile_position<MODE>(++i)) {
+      const TileInfo ti = tile_at<MODE>(sm, p, t);
       if (!__all_sync(0xFFFFFFFFu, mbar_wait(&sm.tempty[acc], acc_phase ^ 1, abort))) {
         ok = false;
         break;
@@ -403,8 +460,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     constexpr int kOutBytes = OUT == FP8QGG_OUT_F32 ? 4 : 2;
     const int64_t row_stride = p.ld_out * kOutBytes;
     uint32_t acc = 0, acc_phase = 0;
-    for (int32_t t = blockIdx.x; t < total; t += gridDim.x) {
-      const TileInfo ti = decode_tile<MODE>(sm, p, t);
+    for (int32_t i = 0, t = tile_position<MODE>(0); t < total; t = tile_position<MODE>(++i)) {
+      const TileInfo ti = tile_at<MODE>(sm, p, t);
       const int64_t ncols = MODE == FP8QGG_M_JAGGED ? p.n : p.k;
       // column reciprocal scales of this tile
       for (int h = 0; h < 2; ++h) {

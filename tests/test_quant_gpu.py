@@ -277,3 +277,19 @@ def test_colwise_tall_groups_split_over_many_blocks(layout):
     assert (qn == q_ref).all()
     assert (s.cpu().numpy().view(np.uint32) == s_ref.view(np.uint32)).all()
     assert int(st.item()) == 0
+
+
+@pytest.mark.parametrize("layout", [qgg.LAYOUT_SAME, qgg.LAYOUT_TRANSPOSED])
+def test_colwise_single_group_of_seventy_thousand_rows(layout):
+    """No group-height limit: one 70,003-row group (two passes per column tile)."""
+    m, cols = 70003, 40
+    x = rand_bf16(41, m, cols, outliers=0.0005)
+    off = np.array([m], np.int32)
+    ld = (m + 15) // 16 * 16
+    q_ref, s_ref, _ = orc.quant_colwise_jagged(bits(x), off, layout, ld_q=ld if layout else None)
+    q, s = qgg.fp8_quant_colwise_jagged(dev(x), torch.from_numpy(off).cuda(), layout, ld_q=ld)
+    qn = q.cpu().numpy()
+    if layout == qgg.LAYOUT_TRANSPOSED:
+        qn, q_ref = qn[:, :m], q_ref[:, :m]
+    assert (qn == q_ref).all()
+    assert (s.cpu().numpy().view(np.uint32) == s_ref.view(np.uint32)).all()

@@ -76,13 +76,9 @@ def test_noalloc_matches_regular_entry_point_on_two_calls_in_a_row(layout):
         assert int(st.item()) == 0
 
 
-def test_noalloc_rejects_problems_beyond_its_scratch():
-    lib = qgg.lib()
-    groups, cols = 1024, 1024  # needs 4 MiB of partial maxima: above the fixed scratch
-    assert qgg.colwise_workspace_bytes(100, cols, groups) > 2 * 1024 * 1024
-    x = torch.zeros((100, cols), dtype=torch.bfloat16, device="cuda")
-    off = torch.full((groups,), 100, dtype=torch.int32, device="cuda")
-    q = torch.empty((100, cols), dtype=torch.uint8, device="cuda")
-    s = torch.empty((groups, cols), device="cuda")
-    rc = call_noalloc(x, off, qgg.LAYOUT_SAME, q, s)
-    assert rc == -2, lib.fp8qgg_error_string(rc)
+def test_noalloc_scratch_covers_the_problems_it_accepts():
+    """Every problem the regular entry point accepts needs no more scratch than
+    the fixed array holds, so the no-allocation entry point accepts it too."""
+    limit = 2 * 1024 * 1024
+    for rows, cols, groups in [(1, 8, 1), (98304, 2048, 64), (131072, 8192, 1024)]:
+        assert 0 < qgg.colwise_workspace_bytes(rows, cols, groups) <= limit
