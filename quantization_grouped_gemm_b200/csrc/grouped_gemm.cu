@@ -307,10 +307,58 @@ __device__ __forceinline__ void store_chunk(float *stg, char *out_base, int64_t 
   }
 }
 
+// Bulk-store path of the epilogue.  A store unit is 32 rows x 64 bytes (16
+// fp32 or 32 bf16 columns), written to one of two 2 KB shared-memory buffers
+// of the warp in the 64-byte swizzle layout (16-byte piece j of row r at piece
+// j ^ ((r >> 1) & 3): conflict-free row-wise writes) and sent to global memory
+// by one bulk tensor store, which clips at the edges of the output tensor.
+// The other buffer's store is still allowed in flight while this one fills.
+template <int MODE, int OUT>
+__device__ __forceinline__ void store_unit_tma(float *buf, const CUtensorMap *omap,
+                                               const uint32_t *r, float inv_a,
+                                               const float *inv_b, int32_t x, int32_t y,
+                                               int32_t e, int lane) {
+  if (lane == 0) bulk_wait_read<1>();
+  __syncwarp();
+  uint32_t *bw = reinterpret_cast<uint32_t *>(buf);
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    uint4 v;
+    if constexpr (OUT == FP8QGG_OUT_F32) {
+      v.x = __float_as_uint(__fmul_rn(__fmul_rn(__uint_as_float(r[4 * j + 0]), inv_a), inv_b[4 * j + 0]));
+      v.y = __float_as_uint(__fmul_rn(__fmul_rn(__uint_as_float(r[4 * j + 1]), inv_a), inv_b[4 * j + 1]));
+      v.z = __float_as_uint(__fmul_rn(__fmul_rn(__uint_as_float(r[4 * j + 2]), inv_a), inv_b[4 * j + 2]));
+      v.w = __float_as_uint(__fmul_rn(__fmul_rn(__uint_as_float(r[4 * j + 3]), inv_a), inv_b[4 * j + 3]));
+    } else {
+      uint32_t w[4];
+#pragma unroll
+      for (int h = 0; h < 4; ++h) {
+        const int c = 8 * j + 2 * h;
+        const float f0 = __fmul_rn(__fmul_rn(__uint_as_float(r[c]), inv_a), inv_b[c]);
+        const float f1 = __fmul_rn(__fmul_rn(__uint_as_float(r[c + 1]), inv_a), inv_b[c + 1]);
+        __nv_bfloat162 b2 = __floats2bfloat162_rn(f0, f1);
+        w[h] = *reinterpret_cast<uint32_t *>(&b2);
+      }
+      v = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+    *reinterpret_cast<uint4 *>(bw + lane * 16 + 4 * (j ^ ((lane >> 1) & 3))) = v;
+  }
+  fence_proxy_async_smem();
+  __syncwarp();
+  if (lane == 0) {
+    if constexpr (MODE == FP8QGG_M_JAGGED)
+      tma_store_2d(omap, buf, x, y);
+    else
+      tma_store_3d(omap, buf, x, y, e);
+    bulk_commit();
+  }
+}
+
 template <int MODE, int OUT>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap amap,
-                        const __grid_constant__ CUtensorMap bmap, const GemmParams p) {
+                        const __grid_constant__ CUtensorMap bmap,
+                        const __grid_constant__ CUtensorMap omap, const GemmParams p) {
   extern __shared__ uint8_t smem_raw[];
   GemmSmem &sm = *reinterpret_cast<GemmSmem *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -320,6 +368,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   if (warp == 0 && lane == 0) {
     prefetch_tensormap(&amap);
     prefetch_tensormap(&bmap);
+    prefetch_tensormap(&omap);
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&sm.full[s], 1);
       mbar_init(&sm.empty[s], 1);
@@ -460,6 +509,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     constexpr int kOutBytes = OUT == FP8QGG_OUT_F32 ? 4 : 2;
     const int64_t row_stride = p.ld_out * kOutBytes;
     uint32_t acc = 0, acc_phase = 0;
+    uint32_t nunit = 0;  // bulk store units issued by this warp (buffer = nunit & 1)
     for (int32_t i = 0, t = tile_position<MODE>(0); t < total; t = tile_position<MODE>(++i)) {
       const TileInfo ti = tile_at<MODE>(sm, p, t);
       const int64_t ncols = MODE == FP8QGG_M_JAGGED ? p.n : p.k;
@@ -497,7 +547,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       tc_fence_after_sync();
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(32 * quarter) << 16) + acc * BN;
       // two 32-column TMEM loads per wait: the second load's latency hides
-      // behind the first's
+      // behind the first's.  Whole 32-row windows go out through bulk tensor
+      // stores; a token-jagged window that crosses the group's end (its last
+      // rows belong to the next group) is stored row by row instead.
+      const bool use_tma = MODE == FP8QGG_K_JAGGED || valid_rows == 32;
+      if (!use_tma && valid_rows > 0) {
+        if (lane == 0) bulk_wait_read<0>();
+        __syncwarp();
+      }
 #pragma unroll 1
       for (int c = 0; c < BN / 32; c += 2) {
         uint32_t r0[32], r1[32];
@@ -507,23 +564,52 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           tmem_ld_wait();
         } else {
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            r0[i] = 0u;
-            r1[i] = 0u;
+          for (int i2 = 0; i2 < 32; ++i2) {
+            r0[i2] = 0u;
+            r1[i2] = 0u;
           }
         }
         const int64_t col0 = static_cast<int64_t>(ti.tn) * BN + 32 * c;
-        if (valid_rows > 0 && col0 < ncols)
-          store_chunk<OUT>(stg, out_base, row_stride, valid_rows, col0, ncols, r0, inv_a,
-                           &sm.inv_sb[acc][32 * c], lane);
-        if (valid_rows > 0 && col0 + 32 < ncols)
-          store_chunk<OUT>(stg, out_base, row_stride, valid_rows, col0 + 32, ncols, r1, inv_a,
-                           &sm.inv_sb[acc][32 * (c + 1)], lane);
+        if (valid_rows <= 0) continue;
+        if (use_tma) {
+          const int32_t y = static_cast<int32_t>(row0);
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const uint32_t *rr = h ? r1 : r0;
+            const int64_t cc = col0 + 32 * h;
+            if (cc >= ncols) break;
+            if constexpr (OUT == FP8QGG_OUT_F32) {
+              store_unit_tma<MODE, OUT>(stg + 512 * (nunit & 1), &omap, rr, inv_a,
+                                        &sm.inv_sb[acc][32 * (c + h)], static_cast<int32_t>(cc),
+                                        y, ti.e, lane);
+              ++nunit;
+              store_unit_tma<MODE, OUT>(stg + 512 * (nunit & 1), &omap, rr + 16, inv_a,
+                                        &sm.inv_sb[acc][32 * (c + h) + 16],
+                                        static_cast<int32_t>(cc + 16), y, ti.e, lane);
+              ++nunit;
+            } else {
+              store_unit_tma<MODE, OUT>(stg + 512 * (nunit & 1), &omap, rr, inv_a,
+                                        &sm.inv_sb[acc][32 * (c + h)], static_cast<int32_t>(cc),
+                                        y, ti.e, lane);
+              ++nunit;
+            }
+          }
+        } else {
+          if (col0 < ncols)
+            store_chunk<OUT>(stg, out_base, row_stride, valid_rows, col0, ncols, r0, inv_a,
+                             &sm.inv_sb[acc][32 * c], lane);
+          if (col0 + 32 < ncols)
+            store_chunk<OUT>(stg, out_base, row_stride, valid_rows, col0 + 32, ncols, r1, inv_a,
+                             &sm.inv_sb[acc][32 * (c + 1)], lane);
+        }
       }
       tc_fence_before_sync();
       mbar_arrive(&sm.tempty[acc]);
       if (++acc == 2) { acc = 0; acc_phase ^= 1; }
     }
+    // every bulk store has completed before the block exits
+    if (lane == 0) bulk_wait_all();
+    __syncwarp();
   }
 
   tc_fence_before_sync();
@@ -535,7 +621,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 }
 
 namespace {
-using GemmKernel = void (*)(const CUtensorMap, const CUtensorMap, const GemmParams);
+using GemmKernel = void (*)(const CUtensorMap, const CUtensorMap, const CUtensorMap,
+                           const GemmParams);
 
 GemmKernel gemm_kernel(int mode, int out_dtype) {
   if (mode == FP8QGG_M_JAGGED)
@@ -615,6 +702,32 @@ extern "C" int fp8_scaled_grouped_gemm(int mode, const uint8_t *a, int64_t ld_a,
       return FP8QGG_ERR_CUDA;
   }
 
+  // output map for the bulk stores: boxes of 32 rows x 64 bytes, 64-byte swizzle
+  CUtensorMap omap;
+  {
+    const CUtensorMapDataType odt = out_dtype == FP8QGG_OUT_F32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
+                                                                : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    const uint64_t esz = out_dtype == FP8QGG_OUT_F32 ? 4 : 2;
+    const uint32_t box_x = static_cast<uint32_t>(64 / esz);
+    if (mode == FP8QGG_M_JAGGED) {
+      const uint64_t dims[2] = {static_cast<uint64_t>(n),
+                                static_cast<uint64_t>(std::max<int64_t>(m_total, 1))};
+      const uint64_t str[1] = {static_cast<uint64_t>(ld_out) * esz};
+      const uint32_t box[2] = {box_x, 32};
+      if (!encode_tensor_map(&omap, odt, 2, out, dims, str, box, CU_TENSOR_MAP_SWIZZLE_64B))
+        return FP8QGG_ERR_CUDA;
+    } else {
+      const uint64_t dims[3] = {static_cast<uint64_t>(k), static_cast<uint64_t>(n),
+                                static_cast<uint64_t>(num_groups)};
+      const uint64_t gs = num_groups > 1 ? static_cast<uint64_t>(out_group_stride)
+                                         : static_cast<uint64_t>(n * ld_out);
+      const uint64_t str[2] = {static_cast<uint64_t>(ld_out) * esz, gs * esz};
+      const uint32_t box[3] = {box_x, 32, 1};
+      if (!encode_tensor_map(&omap, odt, 3, out, dims, str, box, CU_TENSOR_MAP_SWIZZLE_64B))
+        return FP8QGG_ERR_CUDA;
+    }
+  }
+
   DeviceInfo dev;
   if (!device_info(&dev)) return FP8QGG_ERR_CUDA;
   GemmKernel kern = gemm_kernel(mode, out_dtype);
@@ -644,6 +757,6 @@ extern "C" int fp8_scaled_grouped_gemm(int mode, const uint8_t *a, int64_t ld_a,
   prm.ld_out = ld_out;
   prm.out_gs = out_group_stride;
   prm.status = dev_status;
-  kern<<<grid, kGemmThreads, smem, static_cast<cudaStream_t>(stream)>>>(amap, bmap, prm);
+  kern<<<grid, kGemmThreads, smem, static_cast<cudaStream_t>(stream)>>>(amap, bmap, omap, prm);
   return cudaGetLastError() == cudaSuccess ? FP8QGG_OK : FP8QGG_ERR_CUDA;
 }
