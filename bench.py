@@ -421,9 +421,12 @@ def run_gpu(args, world, rank, local):
 
 
 # DRAM bytes per launch of the grouped GEMM from an ncu capture of the same
-# command (dram__bytes_read.sum + dram__bytes_write.sum); None until captured
-# for the current kernel.
-TRAFFIC = {}
+# command (dram__bytes_read.sum + dram__bytes_write.sum, profiles/); a workload
+# is absent until the current kernel has been captured on it.
+TRAFFIC = {
+    "llama3_8b_up_proj": 268084992 + 420487424,
+    "deepseek_moe16b_bwd": 412315648 + 680423680,
+}
 
 
 def main():
