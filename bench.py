@@ -424,7 +424,6 @@ def run_gpu(args, world, rank, local):
 # command (dram__bytes_read.sum + dram__bytes_write.sum, profiles/); a workload
 # is absent until the current kernel has been captured on it.
 TRAFFIC = {
-    "llama3_8b_up_proj": 268084992 + 420487424,
     "deepseek_moe16b_bwd": 412315648 + 680423680,
 }
 

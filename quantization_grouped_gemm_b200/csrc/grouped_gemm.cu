@@ -39,7 +39,7 @@ constexpr int kStages = 4;
 constexpr int kGemmThreads = 192;
 constexpr int kEpiThreads = 128;
 constexpr int kMaxGemmGroups = 1024;
-constexpr int kBand = 16;  // M tiles per raster band (token-jagged mode)
+constexpr int kBandRows = 2048;  // rows per raster band of tiles (token-jagged mode)
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kStageBytes = (BM + BN) * BK;
 constexpr uint32_t kIdesc = idesc_e4m3_f32(BM, BN);
@@ -82,9 +82,8 @@ struct TileInfo {
   int nk;  // k blocks
 };
 
-template <int MODE>
-__device__ __forceinline__ TileInfo decode_tile(const GemmSmem &sm, const GemmParams &p,
-                                                int32_t t) {
+template <int MODE, int ROWS = BM, class Smem = GemmSmem>
+__device__ __forceinline__ TileInfo decode_tile(const Smem &sm, const GemmParams &p, int32_t t) {
   int lo = 0, hi = p.num_groups - 1;
   while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;
@@ -99,12 +98,13 @@ __device__ __forceinline__ TileInfo decode_tile(const GemmSmem &sm, const GemmPa
     // Bands of kBand M tiles: consecutive tiles walk down a band before moving
     // to the next N tile, so the tiles in flight at once share a few A rows
     // and a few B rows in L2.
+    constexpr int kB = kBandRows / ROWS;
     const int nt = static_cast<int>((p.n + BN - 1) / BN);
-    const int mt = (ti.gend - ti.gstart + BM - 1) / BM;
-    const int band = local / (kBand * nt);
-    const int rem = local - band * kBand * nt;
-    const int bm = min(kBand, mt - band * kBand);
-    ti.tm = band * kBand + rem % bm;
+    const int mt = (ti.gend - ti.gstart + ROWS - 1) / ROWS;
+    const int band = local / (kB * nt);
+    const int rem = local - band * kB * nt;
+    const int bm = min(kB, mt - band * kB);
+    ti.tm = band * kB + rem % bm;
     ti.tn = rem / bm;
     ti.nk = static_cast<int>((p.k + BK - 1) / BK);
   } else {
@@ -158,8 +158,8 @@ __device__ __forceinline__ TileInfo tile_at(const GemmSmem &sm, const GemmParams
 }
 
 // Clamped group ends and cumulative tile counts, warp-parallel (one warp).
-template <int MODE>
-__device__ void build_tile_table(GemmSmem &sm, const GemmParams &p, int lane) {
+template <int MODE, int ROWS = BM, class Smem = GemmSmem>
+__device__ void build_tile_table(Smem &sm, const GemmParams &p, int lane) {
   const int32_t R = static_cast<int32_t>(p.m_total);
   const int32_t nt_m = static_cast<int32_t>((p.n + BN - 1) / BN);
   const int32_t tiles_k_mode =
@@ -181,7 +181,7 @@ __device__ void build_tile_table(GemmSmem &sm, const GemmParams &p, int lane) {
     int32_t tiles = 0;
     if (e < p.num_groups) {
       if constexpr (MODE == FP8QGG_M_JAGGED)
-        tiles = ((endv - prev + BM - 1) / BM) * nt_m;
+        tiles = ((endv - prev + ROWS - 1) / ROWS) * nt_m;
       else
         tiles = tiles_k_mode;
     }
@@ -620,6 +620,259 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   }
 }
 
+// ---------------------------------------------------------------------------
+// Token-jagged mode on SM pairs (cta_group::2).  A cluster of two CTAs owns a
+// 256 x 256 output tile: each CTA loads 128 rows of A and 128 rows of B (its
+// half of the tile's N) per k-block, the first CTA of the pair issues
+// tcgen05.mma.cta_group::2 (M256 N256 K32) reading both CTAs' shared memory,
+// and each CTA's TMEM receives its 128 rows of the accumulator.  Per SM the
+// operand stream is 32 KB per 128-deep k-block instead of 48 KB, and the ring
+// has 6 stages.  Both CTAs' copies complete on the first CTA's full barriers;
+// its commits are multicast to both CTAs' empty and accumulator-full
+// barriers; both epilogues release the first CTA's accumulator-empty barrier.
+constexpr int kPairRows = 256;
+constexpr int kStages2 = 6;
+constexpr uint32_t kStage2Bytes = 2u * (128 + 128) * BK;  // both CTAs' copies
+constexpr uint32_t kIdesc2 = idesc_e4m3_f32(256, BN);
+
+struct Gemm2Smem {
+  uint8_t a[kStages2][128 * BK];
+  uint8_t b[kStages2][128 * BK];
+  float stg[kEpiThreads / 32][32 * 32];
+  float inv_sb[2][BN];
+  int32_t end[kMaxGemmGroups];
+  int32_t tile_prefix[kMaxGemmGroups + 1];
+  uint64_t full[kStages2];
+  uint64_t empty[kStages2];
+  uint64_t tfull[2];
+  uint64_t tempty[2];
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort;
+};
+
+template <int OUT>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
+    grouped_gemm_2sm_kernel(const __grid_constant__ CUtensorMap amap,
+                            const __grid_constant__ CUtensorMap bmap,
+                            const __grid_constant__ CUtensorMap omap, const GemmParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  Gemm2Smem &sm = *reinterpret_cast<Gemm2Smem *>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool first = rank == 0;
+  constexpr int MODE = FP8QGG_M_JAGGED;
+
+  if (warp == 0 && lane == 0) {
+    prefetch_tensormap(&amap);
+    prefetch_tensormap(&bmap);
+    prefetch_tensormap(&omap);
+    for (int s2 = 0; s2 < kStages2; ++s2) {
+      mbar_init(&sm.full[s2], 1);
+      mbar_init(&sm.empty[s2], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&sm.tfull[b], 1);
+      mbar_init(&sm.tempty[b], 2 * kEpiThreads);
+    }
+    mbar_init(&sm.drain, 1);
+    sm.abort = 0;
+    fence_mbarrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc_2sm(&sm.tmem_base, kTmemCols);
+    tmem_relinquish_2sm();
+  }
+  if (warp == 2) build_tile_table<MODE, kPairRows>(sm, p, lane);
+  tc_fence_before_sync();
+  __syncthreads();
+  cluster_sync();  // both CTAs' barriers exist before any copy or arrive crosses the pair
+  tc_fence_after_sync();
+
+  const int32_t total = sm.tile_prefix[p.num_groups];
+  const int32_t cid = static_cast<int32_t>(blockIdx.x) >> 1;
+  const int32_t ncl = static_cast<int32_t>(gridDim.x) >> 1;
+  volatile int *abort = &sm.abort;
+  const uint32_t tmem_base = sm.tmem_base;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer (both CTAs)
+    if (lane == 0) {
+      uint32_t stage = 0, phase = 0;
+      uint32_t armed = 0;
+      uint32_t last_par[kStages2];
+      bool ok = true;
+      for (int32_t t = cid; t < total && ok; t += ncl) {
+        const TileInfo ti = decode_tile<MODE, kPairRows>(sm, p, t);
+        const int32_t arow = ti.gstart + ti.tm * kPairRows + 128 * static_cast<int32_t>(rank);
+        const int32_t brow = ti.tn * BN + 128 * static_cast<int32_t>(rank);
+        for (int kb = 0; kb < ti.nk; ++kb) {
+          if (!mbar_wait(&sm.empty[stage], phase ^ 1, abort)) { ok = false; break; }
+          const uint32_t full0 = mapa_shared(smem_addr(&sm.full[stage]), 0);
+          if (first) {
+            mbar_arrive_expect_tx(&sm.full[stage], kStage2Bytes);
+            armed |= 1u << stage;
+            last_par[stage] = phase;
+          }
+          tma_load_2d_2sm(sm.a[stage], &amap, full0, kb * BK, arow);
+          tma_load_3d_2sm(sm.b[stage], &bmap, full0, kb * BK, brow, ti.e);
+          if (++stage == kStages2) { stage = 0; phase ^= 1; }
+        }
+      }
+      if (!ok) {
+        *abort = 1;
+        status_or(p.status, FP8QGG_STATUS_TIMEOUT);
+        volatile int never = 0;
+        for (int s2 = 0; s2 < kStages2; ++s2)
+          if (armed & (1u << s2)) (void)mbar_wait(&sm.full[s2], last_par[s2], &never);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer (first CTA)
+    if (first) {
+      uint32_t stage = 0, phase = 0, acc = 0, acc_phase = 0;
+      bool ok = true;
+      for (int32_t t = cid; t < total && ok; t += ncl) {
+        const TileInfo ti = decode_tile<MODE, kPairRows>(sm, p, t);
+        if (!__all_sync(0xFFFFFFFFu, mbar_wait(&sm.tempty[acc], acc_phase ^ 1, abort))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after_sync();
+        const uint32_t d_tmem = tmem_base + acc * BN;
+        for (int kb = 0; kb < ti.nk; ++kb) {
+          if (!__all_sync(0xFFFFFFFFu, mbar_wait(&sm.full[stage], phase, abort))) {
+            ok = false;
+            break;
+          }
+          tc_fence_after_sync();
+          if (lane == 0) {
+            const uint64_t adesc = smem_desc_k_sw128(smem_addr(sm.a[stage]));
+            const uint64_t bdesc = smem_desc_k_sw128(smem_addr(sm.b[stage]));
+#pragma unroll
+            for (int kk = 0; kk < BK / 32; ++kk)
+              mma_f8f6f4_2sm(d_tmem, adesc + 2 * kk, bdesc + 2 * kk, kIdesc2, (kb | kk) != 0);
+            mma_commit_2sm_mc(&sm.empty[stage], 0x3);
+          }
+          __syncwarp();
+          if (++stage == kStages2) { stage = 0; phase ^= 1; }
+        }
+        if (!ok) break;
+        if (lane == 0) mma_commit_2sm_mc(&sm.tfull[acc], 0x3);
+        __syncwarp();
+        if (++acc == 2) { acc = 0; acc_phase ^= 1; }
+      }
+      if (!ok && lane == 0) {
+        *abort = 1;
+        status_or(p.status, FP8QGG_STATUS_TIMEOUT);
+      }
+      if (lane == 0) {
+        mma_commit_2sm(&sm.drain);
+        volatile int never = 0;
+        (void)mbar_wait(&sm.drain, 0, &never);
+      }
+      __syncwarp();
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue (both CTAs)
+    const int et = threadIdx.x - 64;
+    const int quarter = warp & 3;
+    float *stg = sm.stg[quarter];
+    constexpr int kOutBytes = OUT == FP8QGG_OUT_F32 ? 4 : 2;
+    const int64_t row_stride = p.ld_out * kOutBytes;
+    uint32_t tempty0[2];
+    for (int b = 0; b < 2; ++b) tempty0[b] = mapa_shared(smem_addr(&sm.tempty[b]), 0);
+    uint32_t acc = 0, acc_phase = 0;
+    uint32_t nunit = 0;
+    for (int32_t t = cid; t < total; t += ncl) {
+      const TileInfo ti = decode_tile<MODE, kPairRows>(sm, p, t);
+      const int64_t ncols = p.n;
+      for (int h = 0; h < 2; ++h) {
+        const int c = 2 * et + h;
+        const int64_t col = static_cast<int64_t>(ti.tn) * BN + c;
+        float inv = 0.0f;
+        if (col < ncols) inv = __frcp_rn(__ldg(p.scale_b + ti.e * p.sbs + col));
+        sm.inv_sb[acc][c] = inv;
+      }
+      const int64_t row0 = static_cast<int64_t>(ti.gstart) + static_cast<int64_t>(ti.tm) * kPairRows +
+                           128 * static_cast<int64_t>(rank) + 32 * quarter;
+      const int valid_rows = static_cast<int>(
+          ::max(int64_t(0), ::min(int64_t(32), static_cast<int64_t>(ti.gend) - row0)));
+      float inv_a = 0.0f;
+      if (lane < valid_rows) inv_a = __frcp_rn(__ldg(p.scale_a + row0 + lane));
+      char *out_base = static_cast<char *>(p.out) + row0 * row_stride;
+      const bool got = mbar_wait(&sm.tfull[acc], acc_phase, abort);
+      if (!epi_bar_and(got)) {
+        *abort = 1;
+        if (et == 0) status_or(p.status, FP8QGG_STATUS_TIMEOUT);
+        break;
+      }
+      tc_fence_after_sync();
+      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(32 * quarter) << 16) + acc * BN;
+      const bool use_tma = valid_rows == 32;
+      if (!use_tma && valid_rows > 0) {
+        if (lane == 0) bulk_wait_read<0>();
+        __syncwarp();
+      }
+#pragma unroll 1
+      for (int c = 0; c < BN / 32; c += 2) {
+        uint32_t r0[32], r1[32];
+        tmem_ld_32x32b_x32(taddr + 32 * c, r0);
+        tmem_ld_32x32b_x32(taddr + 32 * (c + 1), r1);
+        tmem_ld_wait();
+        const int64_t col0 = static_cast<int64_t>(ti.tn) * BN + 32 * c;
+        if (valid_rows <= 0) continue;
+        if (use_tma) {
+          const int32_t y = static_cast<int32_t>(row0);
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const uint32_t *rr = h ? r1 : r0;
+            const int64_t cc = col0 + 32 * h;
+            if (cc >= ncols) break;
+            if constexpr (OUT == FP8QGG_OUT_F32) {
+              store_unit_tma<MODE, OUT>(stg + 512 * (nunit & 1), &omap, rr, inv_a,
+                                        &sm.inv_sb[acc][32 * (c + h)], static_cast<int32_t>(cc),
+                                        y, ti.e, lane);
+              ++nunit;
+              store_unit_tma<MODE, OUT>(stg + 512 * (nunit & 1), &omap, rr + 16, inv_a,
+                                        &sm.inv_sb[acc][32 * (c + h) + 16],
+                                        static_cast<int32_t>(cc + 16), y, ti.e, lane);
+              ++nunit;
+            } else {
+              store_unit_tma<MODE, OUT>(stg + 512 * (nunit & 1), &omap, rr, inv_a,
+                                        &sm.inv_sb[acc][32 * (c + h)], static_cast<int32_t>(cc),
+                                        y, ti.e, lane);
+              ++nunit;
+            }
+          }
+        } else {
+          if (col0 < ncols)
+            store_chunk<OUT>(stg, out_base, row_stride, valid_rows, col0, ncols, r0, inv_a,
+                             &sm.inv_sb[acc][32 * c], lane);
+          if (col0 + 32 < ncols)
+            store_chunk<OUT>(stg, out_base, row_stride, valid_rows, col0 + 32, ncols, r1, inv_a,
+                             &sm.inv_sb[acc][32 * (c + 1)], lane);
+        }
+      }
+      tc_fence_before_sync();
+      mbar_arrive_cluster(tempty0[acc]);
+      if (++acc == 2) { acc = 0; acc_phase ^= 1; }
+    }
+    if (lane == 0) bulk_wait_all();
+    __syncwarp();
+  }
+
+  tc_fence_before_sync();
+  __syncthreads();
+  cluster_sync();  // the pair's MMAs are drained and no peer access is pending
+  if (warp == 1) {
+    tc_fence_after_sync();
+    tmem_dealloc_2sm(tmem_base, kTmemCols);
+  }
+}
+
 namespace {
 using GemmKernel = void (*)(const CUtensorMap, const CUtensorMap, const CUtensorMap,
                            const GemmParams);
@@ -730,18 +983,6 @@ extern "C" int fp8_scaled_grouped_gemm(int mode, const uint8_t *a, int64_t ld_a,
 
   DeviceInfo dev;
   if (!device_info(&dev)) return FP8QGG_ERR_CUDA;
-  GemmKernel kern = gemm_kernel(mode, out_dtype);
-  const int smem = static_cast<int>(sizeof(GemmSmem)) + 1024;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
-      cudaSuccess)
-    return FP8QGG_ERR_CUDA;
-  int64_t max_tiles;
-  if (mode == FP8QGG_M_JAGGED)
-    max_tiles = ((m_total + BM - 1) / BM + num_groups) * ((n + BN - 1) / BN);
-  else
-    max_tiles = int64_t(num_groups) * ((n + BM - 1) / BM) * ((k + BN - 1) / BN);
-  if (max_tiles > INT32_MAX) return FP8QGG_ERR_SHAPE;
-  const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(max_tiles, dev.sm_count)));
 
   GemmParams prm;
   prm.scale_a = scale_a;
@@ -757,6 +998,48 @@ extern "C" int fp8_scaled_grouped_gemm(int mode, const uint8_t *a, int64_t ld_a,
   prm.ld_out = ld_out;
   prm.out_gs = out_group_stride;
   prm.status = dev_status;
+
+  // Token-jagged problems whose groups average at least one 256-row pair
+  // tile run on SM pairs (half the operand stream per SM); smaller groups
+  // keep 128-row tiles so that little tensor work is spent on padding.
+  if (mode == FP8QGG_M_JAGGED && m_total >= int64_t(kPairRows) * num_groups && dev.sm_count >= 2) {
+    CUtensorMap bmap2;
+    const uint64_t bdims[3] = {static_cast<uint64_t>(k), static_cast<uint64_t>(n),
+                               static_cast<uint64_t>(num_groups)};
+    const uint64_t bstr[2] = {static_cast<uint64_t>(ld_b),
+                              static_cast<uint64_t>(num_groups > 1 ? b_group_stride : n * ld_b)};
+    const uint32_t bbox[3] = {BK, 128, 1};
+    if (!encode_tensor_map(&bmap2, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<uint8_t *>(b),
+                           bdims, bstr, bbox, CU_TENSOR_MAP_SWIZZLE_128B))
+      return FP8QGG_ERR_CUDA;
+    auto kern2 = out_dtype == FP8QGG_OUT_F32 ? grouped_gemm_2sm_kernel<FP8QGG_OUT_F32>
+                                             : grouped_gemm_2sm_kernel<FP8QGG_OUT_BF16>;
+    const int smem2 = static_cast<int>(sizeof(Gemm2Smem)) + 1024;
+    if (cudaFuncSetAttribute(kern2, cudaFuncAttributeMaxDynamicSharedMemorySize, smem2) !=
+        cudaSuccess)
+      return FP8QGG_ERR_CUDA;
+    const int64_t pair_tiles =
+        ((m_total + kPairRows - 1) / kPairRows + num_groups) * ((n + BN - 1) / BN);
+    const int clusters =
+        static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(pair_tiles, dev.sm_count / 2)));
+    kern2<<<2 * clusters, kGemmThreads, smem2, static_cast<cudaStream_t>(stream)>>>(amap, bmap2,
+                                                                                  omap, prm);
+    return cudaGetLastError() == cudaSuccess ? FP8QGG_OK : FP8QGG_ERR_CUDA;
+  }
+
+  GemmKernel kern = gemm_kernel(mode, out_dtype);
+  const int smem = static_cast<int>(sizeof(GemmSmem)) + 1024;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+      cudaSuccess)
+    return FP8QGG_ERR_CUDA;
+  int64_t max_tiles;
+  if (mode == FP8QGG_M_JAGGED)
+    max_tiles = ((m_total + BM - 1) / BM + num_groups) * ((n + BN - 1) / BN);
+  else
+    max_tiles = int64_t(num_groups) * ((n + BM - 1) / BM) * ((k + BN - 1) / BN);
+  if (max_tiles > INT32_MAX) return FP8QGG_ERR_SHAPE;
+  const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(max_tiles, dev.sm_count)));
+
   kern<<<grid, kGemmThreads, smem, static_cast<cudaStream_t>(stream)>>>(amap, bmap, omap, prm);
   return cudaGetLastError() == cudaSuccess ? FP8QGG_OK : FP8QGG_ERR_CUDA;
 }

@@ -102,6 +102,47 @@ def test_m_jagged_many_tiles_persistent_wraparound():
     check_all(out, ref, rows=rows)
 
 
+# groups averaging >= 256 rows run on SM pairs (cta_group::2, 256-row tiles)
+@pytest.mark.parametrize("sizes,n,k", [
+    ([600, 900, 0, 1200], 384, 320),
+    ([256, 512, 257, 255, 1], 256, 128),
+    ([4096], 528, 1040),
+    ([3000, 17, 700], 96, 256),
+])
+def test_m_jagged_pair_tiles_every_element(sizes, n, k):
+    out, ref = m_jagged_case(sum(sizes) + 3 * n + k, sizes, n, k)
+    check_all(out, ref)
+
+
+def test_m_jagged_pair_tiles_bf16_and_rows_past_last_offset():
+    out, ref = m_jagged_case(77, [700, 500], 256, 512, out_dtype=torch.bfloat16, m_total=1300,
+                             offsets=[700, 1200])
+    check_all(out, ref, extra_rel=2.0 ** -8)
+    assert np.isnan(out[1200:]).all()
+
+
+def test_m_jagged_pair_tiles_exact_small_k_with_unit_scales():
+    g = np.random.default_rng(19)
+    m, n, k = 1100, 272, 16
+    sizes = [520, 0, 580]
+    table = orc.decode_table(orc.E4M3FN)
+    allowed = np.array([c for c in range(256) if np.isfinite(table[c]) and
+                        1.0 <= abs(table[c]) < 16.0], np.uint8)
+    qa = allowed[g.integers(0, allowed.size, (m, k))]
+    qb = allowed[g.integers(0, allowed.size, (3, n, k))]
+    ones_a = np.ones(m, np.float32)
+    ones_b = np.ones((3, n), np.float32)
+    off = wl.offsets_from_sizes(sizes)
+    out = qgg.fp8_scaled_grouped_gemm(qgg.M_JAGGED, torch.from_numpy(qa).cuda(),
+                                      torch.from_numpy(ones_a).cuda(),
+                                      torch.from_numpy(qb).cuda(),
+                                      torch.from_numpy(ones_b).cuda(),
+                                      torch.from_numpy(off).cuda()).cpu().numpy()
+    rr, cc = np.meshgrid(np.arange(m), np.arange(n), indexing="ij")
+    c, _ = orc.gemm_m_jagged_sample(qa, ones_a, qb, ones_b, off, rr.ravel(), cc.ravel())
+    assert (out.ravel() == c).all()
+
+
 def test_m_jagged_exact_small_k_with_unit_scales():
     """Codes with exponents in [1, 16) and unit scales: products and sums of up to
     16 terms are exact in fp32, so the tensor cores must match fp64 exactly."""
