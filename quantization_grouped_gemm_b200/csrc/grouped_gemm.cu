@@ -36,8 +36,9 @@ constexpr int BM = 128;
 constexpr int BN = 256;
 constexpr int BK = 128;  // bytes of K per stage row = one 128-byte swizzle atom
 constexpr int kStages = 4;
-constexpr int kGemmThreads = 192;
-constexpr int kEpiThreads = 128;
+constexpr int kEpiWarps = 8;  // two per TMEM lane quarter: one per 128-column half
+constexpr int kEpiThreads = 32 * kEpiWarps;
+constexpr int kGemmThreads = 64 + kEpiThreads;
 constexpr int kMaxGemmGroups = 1024;
 constexpr int kBandRows = 2048;  // rows per raster band of tiles (token-jagged mode)
 constexpr uint32_t kTmemCols = 512;
@@ -47,7 +48,7 @@ constexpr uint32_t kIdesc = idesc_e4m3_f32(BM, BN);
 struct GemmSmem {
   uint8_t a[kStages][BM * BK];  // 16 KB each, 1024-aligned (swizzle atoms)
   uint8_t b[kStages][BN * BK];  // 32 KB each
-  float stg[kEpiThreads / 32][32 * 32];  // per epilogue warp: 32 rows x 32 fp32, swizzled
+  float stg[kEpiWarps][512];  // per epilogue warp: one 32-row x 64-byte output unit
   float inv_sb[2][BN];
   int32_t end[kMaxGemmGroups];
   int32_t tile_prefix[kMaxGemmGroups + 1];
@@ -201,28 +202,51 @@ __device__ void build_tile_table(Smem &sm, const GemmParams &p, int lane) {
   if (bad && lane == 0 && blockIdx.x == 0) status_or(p.status, FP8QGG_STATUS_BAD_OFFSETS);
 }
 
+// Byte mask keeping the bytes [lo, hi) of a 16-byte piece (lo, hi in 0..16).
+__device__ __forceinline__ uint4 keep_mask16(int lo, int hi) {
+  uint32_t w[4];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    uint32_t m = 0;
+#pragma unroll
+    for (int b = 0; b < 4; ++b) {
+      const int k = 4 * q + b;
+      if (k >= lo && k < hi) m |= 0xFFu << (8 * b);
+    }
+    w[q] = m;
+  }
+  return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
 // Zero the K columns outside [lo, hi) of a K-major tile written by TMA with
-// 128-byte swizzle (logical 16-byte chunk j of row r sits at chunk j ^ (r & 7)).
+// 128-byte swizzle (logical 16-byte piece j of row r sits at piece j ^ (r & 7)).
+// Only the pieces that cross lo or hi are read back; pieces wholly outside are
+// overwritten with zeros; the byte masks are built once per call.
 __device__ __forceinline__ void mask_k_tile(uint8_t *tile, int rows, int lo, int hi, int lane) {
+  const int j_lo = lo >> 4;             // piece holding column lo
+  const int j_hi = (hi + 15) >> 4;      // first piece wholly at or after hi
+  const bool part_lo = (lo & 15) != 0;
+  const bool part_hi = (hi & 15) != 0;
+  const int j_hp = hi >> 4;             // piece holding column hi (when partial)
+  const uint4 m_lo = keep_mask16(lo & 15, (j_lo == j_hp && part_hi) ? (hi & 15) : 16);
+  const uint4 m_hi = keep_mask16(0, hi & 15);
+  const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
   for (int r = lane; r < rows; r += 32) {
     uint8_t *row = tile + r * BK;
-#pragma unroll
-    for (int j = 0; j < BK / 16; ++j) {
-      const int k0 = 16 * j;
-      if (k0 >= lo && k0 + 16 <= hi) continue;
-      uint4 *ptr = reinterpret_cast<uint4 *>(row + ((j ^ (r & 7)) << 4));
-      if (k0 + 16 <= lo || k0 >= hi) {
-        *ptr = make_uint4(0u, 0u, 0u, 0u);
-        continue;
-      }
+    const int sw = r & 7;
+    for (int j = 0; j < j_lo; ++j) *reinterpret_cast<uint4 *>(row + ((j ^ sw) << 4)) = zero;
+    for (int j = j_hi; j < BK / 16; ++j) *reinterpret_cast<uint4 *>(row + ((j ^ sw) << 4)) = zero;
+    if (part_lo) {
+      uint4 *ptr = reinterpret_cast<uint4 *>(row + ((j_lo ^ sw) << 4));
       uint4 v = *ptr;
-      uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-      for (int b = 0; b < 16; ++b) {
-        const int kk = k0 + b;
-        if (kk < lo || kk >= hi) w[b >> 2] &= ~(0xFFu << (8 * (b & 3)));
-      }
-      *ptr = make_uint4(w[0], w[1], w[2], w[3]);
+      v.x &= m_lo.x; v.y &= m_lo.y; v.z &= m_lo.z; v.w &= m_lo.w;
+      *ptr = v;
+    }
+    if (part_hi && !(part_lo && j_hp == j_lo)) {
+      uint4 *ptr = reinterpret_cast<uint4 *>(row + ((j_hp ^ sw) << 4));
+      uint4 v = *ptr;
+      v.x &= m_hi.x; v.y &= m_hi.y; v.z &= m_hi.z; v.w &= m_hi.w;
+      *ptr = v;
     }
   }
 }
@@ -242,83 +266,22 @@ __device__ __forceinline__ bool epi_bar_and(bool v) {
   return r != 0;
 }
 
-// Epilogue of one 32-column chunk for the warp's 32 rows: scale in registers,
-// write the chunk to the warp's shared-memory tile (16-byte pieces swizzled by
-// row so that both the row-wise writes and the column-wise reads are free of
-// bank conflicts), then store whole row segments: 8 lanes cover 128
-// consecutive bytes of one output row.  Streaming stores keep the output from
-// evicting the operands from L2.
-template <int OUT>
-__device__ __forceinline__ void store_chunk(float *stg, char *out_base, int64_t row_stride_bytes,
-                                            int valid_rows, int64_t col0, int64_t ncols,
-                                            const uint32_t (&r)[32], float inv_a,
-                                            const float *inv_b, int lane) {
-  if constexpr (OUT == FP8QGG_OUT_F32) {
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      float4 f;
-      f.x = __fmul_rn(__fmul_rn(__uint_as_float(r[4 * j + 0]), inv_a), inv_b[4 * j + 0]);
-      f.y = __fmul_rn(__fmul_rn(__uint_as_float(r[4 * j + 1]), inv_a), inv_b[4 * j + 1]);
-      f.z = __fmul_rn(__fmul_rn(__uint_as_float(r[4 * j + 2]), inv_a), inv_b[4 * j + 2]);
-      f.w = __fmul_rn(__fmul_rn(__uint_as_float(r[4 * j + 3]), inv_a), inv_b[4 * j + 3]);
-      *reinterpret_cast<float4 *>(stg + lane * 32 + 4 * (j ^ (lane & 7))) = f;
-    }
-    __syncwarp();
-#pragma unroll
-    for (int pss = 0; pss < 4; ++pss) {
-      const int lr = pss * 4 + (lane >> 3) + 0;
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        const int row = lr + 16 * half;
-        const int j = lane & 7;
-        const float4 v = *reinterpret_cast<const float4 *>(stg + row * 32 + 4 * (j ^ (row & 7)));
-        if (row < valid_rows && col0 + 4 * j < ncols)
-          __stcs(reinterpret_cast<float4 *>(out_base + row * row_stride_bytes) + (col0 / 4 + j),
-                 v);
-      }
-    }
-    __syncwarp();
-  } else {
-    uint32_t *sw = reinterpret_cast<uint32_t *>(stg);
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      uint32_t w[4];
-#pragma unroll
-      for (int h = 0; h < 4; ++h) {
-        const int c = 8 * j + 2 * h;
-        const float f0 = __fmul_rn(__fmul_rn(__uint_as_float(r[c]), inv_a), inv_b[c]);
-        const float f1 = __fmul_rn(__fmul_rn(__uint_as_float(r[c + 1]), inv_a), inv_b[c + 1]);
-        __nv_bfloat162 b2 = __floats2bfloat162_rn(f0, f1);
-        w[h] = *reinterpret_cast<uint32_t *>(&b2);
-      }
-      *reinterpret_cast<uint4 *>(sw + lane * 16 + 4 * (j ^ ((lane >> 1) & 3))) =
-          make_uint4(w[0], w[1], w[2], w[3]);
-    }
-    __syncwarp();
-#pragma unroll
-    for (int pss = 0; pss < 4; ++pss) {
-      const int row = pss * 8 + (lane >> 2);
-      const int j = lane & 3;
-      const uint4 v = *reinterpret_cast<const uint4 *>(sw + row * 16 + 4 * (j ^ ((row >> 1) & 3)));
-      if (row < valid_rows && col0 + 8 * j < ncols)
-        __stcs(reinterpret_cast<uint4 *>(out_base + row * row_stride_bytes) + (col0 / 8 + j), v);
-    }
-    __syncwarp();
-  }
-}
-
-// Bulk-store path of the epilogue.  A store unit is 32 rows x 64 bytes (16
-// fp32 or 32 bf16 columns), written to one of two 2 KB shared-memory buffers
-// of the warp in the 64-byte swizzle layout (16-byte piece j of row r at piece
-// j ^ ((r >> 1) & 3): conflict-free row-wise writes) and sent to global memory
-// by one bulk tensor store, which clips at the edges of the output tensor.
-// The other buffer's store is still allowed in flight while this one fills.
+// One output unit of an epilogue warp: its 32 rows x 64 bytes (16 fp32 or 32
+// bf16 columns starting at column x).  The values are scaled in registers and
+// written to the warp's 2 KB buffer in the 64-byte swizzle layout (16-byte
+// piece j of row r at piece j ^ ((r >> 1) & 3): conflict-free row-wise
+// writes).  Then either one bulk tensor store sends the buffer out (clipped at
+// the edges of the output tensor), or, for a window that crosses the end of
+// its group, lanes write the valid rows back as coalesced 16-byte pieces.
+// Streaming stores keep the output from evicting the operands from L2.
 template <int MODE, int OUT>
-__device__ __forceinline__ void store_unit_tma(float *buf, const CUtensorMap *omap,
-                                               const uint32_t *r, float inv_a,
-                                               const float *inv_b, int32_t x, int32_t y,
-                                               int32_t e, int lane) {
-  if (lane == 0) bulk_wait_read<1>();
+__device__ __forceinline__ void emit_unit(float *buf, const CUtensorMap *omap, const uint32_t *r,
+                                          float inv_a, const float *inv_b, int32_t x, int32_t y,
+                                          int32_t e, bool tma, char *out_base,
+                                          int64_t row_stride, int valid_rows, int64_t ncols,
+                                          int lane) {
+  constexpr int kOutBytes = OUT == FP8QGG_OUT_F32 ? 4 : 2;
+  if (lane == 0) bulk_wait_read<0>();
   __syncwarp();
   uint32_t *bw = reinterpret_cast<uint32_t *>(buf);
 #pragma unroll
@@ -343,14 +306,81 @@ __device__ __forceinline__ void store_unit_tma(float *buf, const CUtensorMap *om
     }
     *reinterpret_cast<uint4 *>(bw + lane * 16 + 4 * (j ^ ((lane >> 1) & 3))) = v;
   }
-  fence_proxy_async_smem();
-  __syncwarp();
-  if (lane == 0) {
-    if constexpr (MODE == FP8QGG_M_JAGGED)
-      tma_store_2d(omap, buf, x, y);
-    else
-      tma_store_3d(omap, buf, x, y, e);
-    bulk_commit();
+  if (tma) {
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+      if constexpr (MODE == FP8QGG_M_JAGGED)
+        tma_store_2d(omap, buf, x, y);
+      else
+        tma_store_3d(omap, buf, x, y, e);
+      bulk_commit();
+    }
+  } else {
+    __syncwarp();
+    constexpr int kColsPerPiece = 16 / kOutBytes;
+#pragma unroll
+    for (int pss = 0; pss < 4; ++pss) {
+      const int row = pss * 8 + (lane >> 2);
+      const int j = lane & 3;
+      const uint4 v = *reinterpret_cast<const uint4 *>(bw + row * 16 + 4 * (j ^ ((row >> 1) & 3)));
+      const int64_t col = static_cast<int64_t>(x) + kColsPerPiece * j;
+      if (row < valid_rows && col < ncols)
+        __stcs(reinterpret_cast<uint4 *>(out_base + row * row_stride + col * kOutBytes), v);
+    }
+    __syncwarp();
+  }
+}
+
+// Epilogue of one tile for one warp: TMEM lanes [32*quarter, +32) (the rows
+// row0 .. row0+31 of the output), columns [128*chalf, +128) of the tile.
+// Two 32-column TMEM loads share one wait.
+template <int MODE, int OUT>
+__device__ __forceinline__ void epilogue_tile(float *stg, const CUtensorMap *omap,
+                                              const GemmParams &p, const TileInfo &ti,
+                                              uint32_t taddr, int chalf, int64_t row0,
+                                              int valid_rows, float inv_a, const float *inv_sb,
+                                              int lane) {
+  constexpr int kOutBytes = OUT == FP8QGG_OUT_F32 ? 4 : 2;
+  const int64_t ncols = MODE == FP8QGG_M_JAGGED ? p.n : p.k;
+  const int64_t row_stride = p.ld_out * kOutBytes;
+  char *out_base = static_cast<char *>(p.out) +
+                   (MODE == FP8QGG_K_JAGGED ? ti.e * p.out_gs * kOutBytes : 0) + row0 * row_stride;
+  // token-jagged windows that cross the group's end are stored row by row
+  const bool tma = MODE == FP8QGG_K_JAGGED || valid_rows == 32;
+  const int32_t y = static_cast<int32_t>(row0);
+#pragma unroll 1
+  for (int cp = 0; cp < 2; ++cp) {
+    uint32_t r0[32], r1[32];
+    const uint32_t ta = taddr + 128 * chalf + 64 * cp;
+    if (ti.nk > 0) {
+      tmem_ld_32x32b_x32(ta, r0);
+      tmem_ld_32x32b_x32(ta + 32, r1);
+      tmem_ld_wait();
+    } else {
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        r0[i] = 0u;
+        r1[i] = 0u;
+      }
+    }
+    if (valid_rows <= 0) continue;
+    const int64_t col0 = static_cast<int64_t>(ti.tn) * BN + 128 * chalf + 64 * cp;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int64_t cc = col0 + 32 * h;
+      if (cc >= ncols) break;
+      const uint32_t *rr = h ? r1 : r0;
+      const float *ib = inv_sb + 128 * chalf + 64 * cp + 32 * h;
+      emit_unit<MODE, OUT>(stg, omap, rr, inv_a, ib, static_cast<int32_t>(cc), y, ti.e, tma,
+                           out_base, row_stride, valid_rows, ncols, lane);
+      if constexpr (OUT == FP8QGG_OUT_F32) {
+        if (cc + 16 < ncols)
+          emit_unit<MODE, OUT>(stg, omap, rr + 16, inv_a, ib + 16,
+                               static_cast<int32_t>(cc + 16), y, ti.e, tma, out_base, row_stride,
+                               valid_rows, ncols, lane);
+      }
+    }
   }
 }
 
@@ -503,40 +533,31 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     __syncwarp();
   } else {
     // ------------------------------------------------------------ epilogue
-    const int et = threadIdx.x - 64;  // 0..127
-    const int quarter = warp & 3;     // TMEM lanes [32*quarter, 32*quarter + 32)
-    float *stg = sm.stg[quarter];
-    constexpr int kOutBytes = OUT == FP8QGG_OUT_F32 ? 4 : 2;
-    const int64_t row_stride = p.ld_out * kOutBytes;
+    const int et = threadIdx.x - 64;    // 0..255
+    const int ew = warp - 2;            // epilogue warp 0..7
+    const int quarter = warp & 3;       // TMEM lanes [32*quarter, 32*quarter + 32)
+    const int chalf = ew >> 2;          // columns [128*chalf, 128*chalf + 128) of the tile
+    float *stg = sm.stg[ew];
     uint32_t acc = 0, acc_phase = 0;
-    uint32_t nunit = 0;  // bulk store units issued by this warp (buffer = nunit & 1)
     for (int32_t i = 0, t = tile_position<MODE>(0); t < total; t = tile_position<MODE>(++i)) {
       const TileInfo ti = tile_at<MODE>(sm, p, t);
       const int64_t ncols = MODE == FP8QGG_M_JAGGED ? p.n : p.k;
-      // column reciprocal scales of this tile
-      for (int h = 0; h < 2; ++h) {
-        const int c = 2 * et + h;
-        const int64_t col = static_cast<int64_t>(ti.tn) * BN + c;
-        float inv = 0.0f;
-        if (col < ncols) inv = __frcp_rn(__ldg(p.scale_b + ti.e * p.sbs + col));
-        sm.inv_sb[acc][c] = inv;
+      {  // column reciprocal scales of this tile, one column per thread
+        const int64_t col = static_cast<int64_t>(ti.tn) * BN + et;
+        sm.inv_sb[acc][et] = col < ncols ? __frcp_rn(__ldg(p.scale_b + ti.e * p.sbs + col)) : 0.0f;
       }
-      // this thread's accumulator row, and the warp's 32-row output window
-      int64_t row0;   // first output row of the warp's window
+      int64_t row0;    // first output row of the warp's 32-row window
       int valid_rows;  // rows of the window inside the group / matrix
-      char *out_base;
       float inv_a = 0.0f;
       if constexpr (MODE == FP8QGG_M_JAGGED) {
         row0 = static_cast<int64_t>(ti.gstart) + static_cast<int64_t>(ti.tm) * BM + 32 * quarter;
         valid_rows = static_cast<int>(
             ::max(int64_t(0), ::min(int64_t(32), static_cast<int64_t>(ti.gend) - row0)));
         if (lane < valid_rows) inv_a = __frcp_rn(__ldg(p.scale_a + row0 + lane));
-        out_base = static_cast<char *>(p.out) + row0 * row_stride;
       } else {
         row0 = static_cast<int64_t>(ti.tm) * BM + 32 * quarter;
         valid_rows = static_cast<int>(::max(int64_t(0), ::min(int64_t(32), p.n - row0)));
         if (lane < valid_rows) inv_a = __frcp_rn(__ldg(p.scale_a + ti.e * p.sas + row0 + lane));
-        out_base = static_cast<char *>(p.out) + ti.e * p.out_gs * kOutBytes + row0 * row_stride;
       }
       const bool got = mbar_wait(&sm.tfull[acc], acc_phase, abort);
       if (!epi_bar_and(got)) {
@@ -545,64 +566,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         break;
       }
       tc_fence_after_sync();
-      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(32 * quarter) << 16) + acc * BN;
-      // two 32-column TMEM loads per wait: the second load's latency hides
-      // behind the first's.  Whole 32-row windows go out through bulk tensor
-      // stores; a token-jagged window that crosses the group's end (its last
-      // rows belong to the next group) is stored row by row instead.
-      const bool use_tma = MODE == FP8QGG_K_JAGGED || valid_rows == 32;
-      if (!use_tma && valid_rows > 0) {
-        if (lane == 0) bulk_wait_read<0>();
-        __syncwarp();
-      }
-#pragma unroll 1
-      for (int c = 0; c < BN / 32; c += 2) {
-        uint32_t r0[32], r1[32];
-        if (ti.nk > 0) {
-          tmem_ld_32x32b_x32(taddr + 32 * c, r0);
-          tmem_ld_32x32b_x32(taddr + 32 * (c + 1), r1);
-          tmem_ld_wait();
-        } else {
-#pragma unroll
-          for (int i2 = 0; i2 < 32; ++i2) {
-            r0[i2] = 0u;
-            r1[i2] = 0u;
-          }
-        }
-        const int64_t col0 = static_cast<int64_t>(ti.tn) * BN + 32 * c;
-        if (valid_rows <= 0) continue;
-        if (use_tma) {
-          const int32_t y = static_cast<int32_t>(row0);
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const uint32_t *rr = h ? r1 : r0;
-            const int64_t cc = col0 + 32 * h;
-            if (cc >= ncols) break;
-            if constexpr (OUT == FP8QGG_OUT_F32) {
-              store_unit_tma<MODE, OUT>(stg + 512 * (nunit & 1), &omap, rr, inv_a,
-                                        &sm.inv_sb[acc][32 * (c + h)], static_cast<int32_t>(cc),
-                                        y, ti.e, lane);
-              ++nunit;
-              store_unit_tma<MODE, OUT>(stg + 512 * (nunit & 1), &omap, rr + 16, inv_a,
-                                        &sm.inv_sb[acc][32 * (c + h) + 16],
-                                        static_cast<int32_t>(cc + 16), y, ti.e, lane);
-              ++nunit;
-            } else {
-              store_unit_tma<MODE, OUT>(stg + 512 * (nunit & 1), &omap, rr, inv_a,
-                                        &sm.inv_sb[acc][32 * (c + h)], static_cast<int32_t>(cc),
-                                        y, ti.e, lane);
-              ++nunit;
-            }
-          }
-        } else {
-          if (col0 < ncols)
-            store_chunk<OUT>(stg, out_base, row_stride, valid_rows, col0, ncols, r0, inv_a,
-                             &sm.inv_sb[acc][32 * c], lane);
-          if (col0 + 32 < ncols)
-            store_chunk<OUT>(stg, out_base, row_stride, valid_rows, col0 + 32, ncols, r1, inv_a,
-                             &sm.inv_sb[acc][32 * (c + 1)], lane);
-        }
-      }
+      epilogue_tile<MODE, OUT>(stg, &omap, p, ti,
+                               tmem_base + (static_cast<uint32_t>(32 * quarter) << 16) + acc * BN,
+                               chalf, row0, valid_rows, inv_a, sm.inv_sb[acc], lane);
       tc_fence_before_sync();
       mbar_arrive(&sm.tempty[acc]);
       if (++acc == 2) { acc = 0; acc_phase ^= 1; }
@@ -638,7 +604,7 @@ constexpr uint32_t kIdesc2 = idesc_e4m3_f32(256, BN);
 struct Gemm2Smem {
   uint8_t a[kStages2][128 * BK];
   uint8_t b[kStages2][128 * BK];
-  float stg[kEpiThreads / 32][32 * 32];
+  float stg[kEpiWarps][512];
   float inv_sb[2][BN];
   int32_t end[kMaxGemmGroups];
   int32_t tile_prefix[kMaxGemmGroups + 1];
@@ -778,23 +744,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   } else {
     // ------------------------------------------------------------ epilogue (both CTAs)
     const int et = threadIdx.x - 64;
+    const int ew = warp - 2;
     const int quarter = warp & 3;
-    float *stg = sm.stg[quarter];
-    constexpr int kOutBytes = OUT == FP8QGG_OUT_F32 ? 4 : 2;
-    const int64_t row_stride = p.ld_out * kOutBytes;
+    const int chalf = ew >> 2;
+    float *stg = sm.stg[ew];
     uint32_t tempty0[2];
     for (int b = 0; b < 2; ++b) tempty0[b] = mapa_shared(smem_addr(&sm.tempty[b]), 0);
     uint32_t acc = 0, acc_phase = 0;
-    uint32_t nunit = 0;
     for (int32_t t = cid; t < total; t += ncl) {
       const TileInfo ti = decode_tile<MODE, kPairRows>(sm, p, t);
-      const int64_t ncols = p.n;
-      for (int h = 0; h < 2; ++h) {
-        const int c = 2 * et + h;
-        const int64_t col = static_cast<int64_t>(ti.tn) * BN + c;
-        float inv = 0.0f;
-        if (col < ncols) inv = __frcp_rn(__ldg(p.scale_b + ti.e * p.sbs + col));
-        sm.inv_sb[acc][c] = inv;
+      {
+        const int64_t col = static_cast<int64_t>(ti.tn) * BN + et;
+        sm.inv_sb[acc][et] = col < p.n ? __frcp_rn(__ldg(p.scale_b + ti.e * p.sbs + col)) : 0.0f;
       }
       const int64_t row0 = static_cast<int64_t>(ti.gstart) + static_cast<int64_t>(ti.tm) * kPairRows +
                            128 * static_cast<int64_t>(rank) + 32 * quarter;
@@ -802,7 +763,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
           ::max(int64_t(0), ::min(int64_t(32), static_cast<int64_t>(ti.gend) - row0)));
       float inv_a = 0.0f;
       if (lane < valid_rows) inv_a = __frcp_rn(__ldg(p.scale_a + row0 + lane));
-      char *out_base = static_cast<char *>(p.out) + row0 * row_stride;
       const bool got = mbar_wait(&sm.tfull[acc], acc_phase, abort);
       if (!epi_bar_and(got)) {
         *abort = 1;
@@ -810,52 +770,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         break;
       }
       tc_fence_after_sync();
-      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(32 * quarter) << 16) + acc * BN;
-      const bool use_tma = valid_rows == 32;
-      if (!use_tma && valid_rows > 0) {
-        if (lane == 0) bulk_wait_read<0>();
-        __syncwarp();
-      }
-#pragma unroll 1
-      for (int c = 0; c < BN / 32; c += 2) {
-        uint32_t r0[32], r1[32];
-        tmem_ld_32x32b_x32(taddr + 32 * c, r0);
-        tmem_ld_32x32b_x32(taddr + 32 * (c + 1), r1);
-        tmem_ld_wait();
-        const int64_t col0 = static_cast<int64_t>(ti.tn) * BN + 32 * c;
-        if (valid_rows <= 0) continue;
-        if (use_tma) {
-          const int32_t y = static_cast<int32_t>(row0);
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const uint32_t *rr = h ? r1 : r0;
-            const int64_t cc = col0 + 32 * h;
-            if (cc >= ncols) break;
-            if constexpr (OUT == FP8QGG_OUT_F32) {
-              store_unit_tma<MODE, OUT>(stg + 512 * (nunit & 1), &omap, rr, inv_a,
-                                        &sm.inv_sb[acc][32 * (c + h)], static_cast<int32_t>(cc),
-                                        y, ti.e, lane);
-              ++nunit;
-              store_unit_tma<MODE, OUT>(stg + 512 * (nunit & 1), &omap, rr + 16, inv_a,
-                                        &sm.inv_sb[acc][32 * (c + h) + 16],
-                                        static_cast<int32_t>(cc + 16), y, ti.e, lane);
-              ++nunit;
-            } else {
-              store_unit_tma<MODE, OUT>(stg + 512 * (nunit & 1), &omap, rr, inv_a,
-                                        &sm.inv_sb[acc][32 * (c + h)], static_cast<int32_t>(cc),
-                                        y, ti.e, lane);
-              ++nunit;
-            }
-          }
-        } else {
-          if (col0 < ncols)
-            store_chunk<OUT>(stg, out_base, row_stride, valid_rows, col0, ncols, r0, inv_a,
-                             &sm.inv_sb[acc][32 * c], lane);
-          if (col0 + 32 < ncols)
-            store_chunk<OUT>(stg, out_base, row_stride, valid_rows, col0 + 32, ncols, r1, inv_a,
-                             &sm.inv_sb[acc][32 * (c + 1)], lane);
-        }
-      }
+      epilogue_tile<MODE, OUT>(stg, &omap, p, ti,
+                               tmem_base + (static_cast<uint32_t>(32 * quarter) << 16) + acc * BN,
+                               chalf, row0, valid_rows, inv_a, sm.inv_sb[acc], lane);
       tc_fence_before_sync();
       mbar_arrive_cluster(tempty0[acc]);
       if (++acc == 2) { acc = 0; acc_phase ^= 1; }
