@@ -122,8 +122,11 @@ int fp8_quant_rowwise(const void *x, int64_t rows, int64_t cols, int64_t ld_x,
                       int fmt, float scale_max, uint64_t *sat_count, void *stream);
 
 /*
- * Bytes of device workspace fp8_quant_colwise_jagged needs (a work counter
- * shared by the blocks; 256 bytes whatever the problem).  Always > 0.
+ * Bytes of device workspace fp8_quant_colwise_jagged needs: a work counter
+ * shared by the blocks (256 bytes), plus, for every (group, 64-column) unit
+ * that may be taller than 448 rows, an arrival counter and 64 absmax words
+ * (260 bytes per unit; at most min(num_groups, rows_total / 432) groups can be
+ * that tall).  Always > 0 and a multiple of 256.
  */
 size_t fp8_quant_colwise_jagged_workspace_size(int64_t rows_total, int64_t cols,
                                                int32_t num_groups);
@@ -151,9 +154,11 @@ size_t fp8_quant_colwise_jagged_workspace_size(int64_t rows_total, int64_t cols,
  *            share one workspace must be ordered on the device.
  * Requirements: rows_total >= 0; cols in [1, 2^31) and a multiple of 8;
  * num_groups in [1, 1024]; ld_x >= cols, ld_x % 8 == 0; x, q and workspace
- * 16-byte aligned.  Groups of any height are handled: up to 3072 rows a
- * (group, 32-column) block of x is read from HBM once; a taller group's block
- * is read a second time for the cast, while it is still in L2.
+ * 16-byte aligned.  Groups of any height are handled: up to 448 rows a
+ * (group, 64-column) block of x is read from HBM once and stays on chip for
+ * the cast; a taller block is cut into chunks of at most 448 rows spread over
+ * the SMs, whose absmax merge in the workspace, and each chunk is read a
+ * second time for the cast, while it is still in L2.
  */
 int fp8_quant_colwise_jagged(const void *x, int64_t rows_total, int64_t cols, int64_t ld_x,
                              const int32_t *offsets, int32_t num_groups,
@@ -174,8 +179,10 @@ int fp8_quant_colwise_jagged(const void *x, int64_t rows_total, int64_t cols, in
  * by every GPU that loads the library until the process exits.
  *  - Size limit: problems whose fp8_quant_colwise_jagged_workspace_size(...)
  *    exceeds FP8QGG_NOALLOC_SCRATCH_BYTES are rejected with FP8QGG_ERR_SHAPE
- *    before anything is enqueued (the current kernel needs 256 bytes for any
- *    problem, so every valid problem fits).
+ *    before anything is enqueued.  2 MiB covers, for instance, 64 groups of
+ *    a 98304 x 2048 tensor (532,736 bytes) or 1024 groups of a 131072 x 1408
+ *    tensor (1,733,632 bytes); it does not cover 64 groups of a 98304 x 8192
+ *    tensor (2,130,176 bytes).
  *  - Set-up: the first call on each device looks up the array's device
  *    address with that device current (cudaGetSymbolAddress).  Make that
  *    first call before any stream capture on the device.

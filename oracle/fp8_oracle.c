@@ -27,7 +27,11 @@
  *  - e4m3fn (OCP): bias 7, largest finite 448, NaN = S.1111.111, has -0.
  *  - e4m3fnuz: bias 8, largest finite 240 (0x7F), NaN only 0x80, no -0.
  *  - encode = round to nearest, ties to even mantissa, in ONE rounding from
- *    the fp32 value, saturating at the largest finite value.
+ *    the fp32 value, saturating at the largest finite value (infinities
+ *    included); NaN encodes as a NaN code: 0x7F for e4m3fn (0xFF, the other
+ *    e4m3fn NaN, is an equally valid result), 0x80 for e4m3fnuz.
+ *  - absmax = the largest |x| over the values that are not NaN (a NaN
+ *    compares false and is skipped).
  *  - scale s = fp32(fmax / max(amax, 1e-12f)) with IEEE round-to-nearest;
  *    y = fp32(x * s); y is clamped to [-fmax, fmax]; q = encode(y).
  *    The quantisation scale s is what is stored (x ~ decode(q) / s).
@@ -82,6 +86,10 @@ double oracle_fp8_decode(uint8_t code, int fmt)
  * spacing is a power of two. */
 uint8_t oracle_fp8_encode(float y, int fmt)
 {
+    /* NaN (the pages never meet one) goes to a NaN code: 0x7F for e4m3fn
+     * (0xFF is NaN too; the sign of a NaN is not portable), 0x80, the only
+     * NaN, for e4m3fnuz */
+    if (isnan(y)) return (uint8_t)(fmt == ORC_FMT_E4M3FNUZ ? 0x80 : 0x7F);
     int bias = fmt_bias(fmt);
     double maxv = fmt_max(fmt);
     int neg = signbit(y) ? 1 : 0;

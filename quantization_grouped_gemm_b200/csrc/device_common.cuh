@@ -23,6 +23,16 @@ __device__ __forceinline__ uint32_t smem_addr(const void *p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
+// The first 1024-byte aligned address inside a dynamic shared-memory buffer,
+// reached by pointer arithmetic on the buffer itself (a detour through an
+// integer would hide from the compiler that the result is shared memory, and
+// every access through it would become a generic one).
+template <class T>
+__device__ __forceinline__ T *align_smem_1024(uint8_t *raw) {
+  const uint32_t a = static_cast<uint32_t>(__cvta_generic_to_shared(raw));
+  return reinterpret_cast<T *>(raw + ((1024u - (a & 1023u)) & 1023u));
+}
+
 __device__ __forceinline__ uint64_t global_timer_ns() {
   uint64_t t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
@@ -338,6 +348,7 @@ __device__ __forceinline__ uint32_t cvt_e4m3fn_x2(float lo, float hi) {
 // when |y| lies above the midpoint 232 between 224 and 240, and the e4m3fn
 // negative zero 0x80 (the e4m3fnuz NaN) becomes the single zero 0x00.
 __device__ __forceinline__ uint32_t fnuz_fix(uint32_t code, float y) {
+  if (y != y) return 0x80u;  // NaN: the format's only NaN code
   if (fabsf(y) > 232.0f) return (y < 0.0f ? 0x80u : 0u) | 0x7Fu;
   return code == 0x80u ? 0u : code;
 }
@@ -355,6 +366,12 @@ __device__ __forceinline__ uint32_t cvt_x2(float lo, float hi) {
     return cvt_e4m3fn_x2(lo, hi);
 }
 
+// Clamp to [-smax, smax] that lets a NaN through (to be encoded as NaN), the
+// way two comparisons would; fminf/fmaxf would turn it into -smax.
+__device__ __forceinline__ float clamp_keep_nan(float y, float smax) {
+  return fabsf(y) > smax ? copysignf(smax, y) : y;
+}
+
 // Scale, clamp and encode one pair of bf16 values packed in a 32-bit word.
 // Counts saturated elements (pre-clamp |y| above sat_thr) into *sat.
 template <int FMT>
@@ -365,8 +382,8 @@ __device__ __forceinline__ uint32_t quant_pair(uint32_t packed, float s, float s
   float y0 = __fmul_rn(x0, s);
   float y1 = __fmul_rn(x1, s);
   sat += (fabsf(y0) > sat_thr) + (fabsf(y1) > sat_thr);
-  y0 = fminf(fmaxf(y0, -smax), smax);
-  y1 = fminf(fmaxf(y1, -smax), smax);
+  y0 = clamp_keep_nan(y0, smax);
+  y1 = clamp_keep_nan(y1, smax);
   return cvt_x2<FMT>(y0, y1);
 }
 
@@ -394,11 +411,20 @@ __device__ __forceinline__ uint64_t pack_f32x2(float lo, float hi) {
   return r;
 }
 
-// Per-halfword unsigned max of |bf16| bit patterns: the absolute value of a
-// finite bf16 compares like its 15-bit magnitude pattern.
-__device__ __forceinline__ uint32_t abs_max_bf16x2(uint32_t acc, uint32_t packed) {
-  return __vmaxu2(acc, packed & 0x7FFF7FFFu);
+// Running absmax of bf16 pairs: one packed IEEE max of magnitudes per pair
+// (max.xorsign.abs: |result| = max(|acc|, |x|); its sign bit carries no
+// meaning and is cleared by absmax_bits).  A NaN operand is ignored, as an
+// IEEE maxNum does, so a NaN input never decides a scale; the accumulator,
+// which starts at zero, never becomes NaN.  Subnormals are kept.
+__device__ __forceinline__ uint32_t absmax_acc(uint32_t acc, uint32_t x) {
+  uint32_t r;
+  asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(acc), "r"(x));
+  return r;
 }
+
+// Magnitude bit patterns of a running absmax: for non-NaN bf16 they compare
+// like the magnitudes themselves, so halves can be merged with integer max.
+__device__ __forceinline__ uint32_t absmax_bits(uint32_t acc) { return acc & 0x7FFF7FFFu; }
 
 __device__ __forceinline__ float bf16_bits_to_float(uint32_t bits16) {
   return __uint_as_float(bits16 << 16);

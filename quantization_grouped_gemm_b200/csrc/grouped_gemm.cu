@@ -390,8 +390,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                         const __grid_constant__ CUtensorMap bmap,
                         const __grid_constant__ CUtensorMap omap, const GemmParams p) {
   extern __shared__ uint8_t smem_raw[];
-  GemmSmem &sm = *reinterpret_cast<GemmSmem *>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  GemmSmem &sm = *align_smem_1024<GemmSmem>(smem_raw);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
@@ -623,8 +622,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
                             const __grid_constant__ CUtensorMap bmap,
                             const __grid_constant__ CUtensorMap omap, const GemmParams p) {
   extern __shared__ uint8_t smem_raw[];
-  Gemm2Smem &sm = *reinterpret_cast<Gemm2Smem *>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  Gemm2Smem &sm = *align_smem_1024<Gemm2Smem>(smem_raw);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();

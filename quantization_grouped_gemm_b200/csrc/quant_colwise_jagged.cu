@@ -9,17 +9,30 @@
 // of the column-scales kernel transposed on chip so that stores coalesce).
 // "AMD Boosts PyTorch FP8 Training on Instinct GPUs", third paragraph.
 //
-// B200 design.  A unit of work is one (group, 32-column tile): all of the
-// group's rows for 32 columns.  One block per SM takes units from an atomic
-// counter, largest groups first.  Inside a block one producer warp streams the
-// unit's rows with TMA, 256-row boxes, into a 12-slot shared-memory ring; eight
-// consumer warps take the column absmax box by box, derive the 32 scales and
-// cast.  A unit of at most 12 boxes (3072 rows) stays in the ring between the
-// absmax and the cast: one HBM read.  A taller unit is streamed a second time
-// for the cast; the units in flight at once belong to the same few groups, so
-// the second read is served by L2.  No block ever waits for another block.
-// TRANSPOSED output goes through a shared-memory [column][token] tile and is
-// written as 16-byte runs along the tokens.
+// B200 design.  A unit is one (group, 64-column tile): 128-byte row segments.
+// One block per SM; one producer warp streams rows with TMA into a ring of six
+// 240-row slots (30 KB); each of fifteen consumer warps owns 16 rows of every
+// slot and works on them alone (absmax, cast, store straight from registers),
+// meeting the other warps only once per unit to combine the column absmax.
+//
+// Work is a list of tasks taken from an atomic counter:
+//  - a unit whose rows fit in three slots (720 rows) is one "whole" task:
+//    every lane keeps its part of the rows in registers between the absmax and
+//    the cast (one HBM read) and frees each slot at once, so the ring keeps
+//    streaming;
+//  - a taller unit is cut into chunks of equal height (at most three slots),
+//    and every chunk gives two tasks:
+//    an "amax" task (column absmax of the chunk, merged into the unit's
+//    absmax in global memory with atomic max, then counted in the unit's
+//    arrival counter) and a "cast" task (waits for the unit's count, derives
+//    the scales, re-reads the chunk and casts it).  A cast task is placed in
+//    the list after every amax task of its unit and about two grid-widths of
+//    tasks later, so the chunk it re-reads is still in L2 and the wait is
+//    short.  Chunks of one tall group are spread over many SMs, so a skewed
+//    routing (one expert with many tokens) keeps every SM busy.
+// Tall units come first, largest group first, then whole units largest first.
+// A task only ever waits for tasks that were handed out before it, each held
+// by a running block, so the blocks need not be co-resident.
 #include <algorithm>
 #include <cstring>
 #include <mutex>
@@ -29,38 +42,75 @@
 
 namespace fp8qgg {
 
-constexpr int kCW = 32;                   // columns per unit: 64 bytes of bf16 per row
-constexpr int kWords = kCW / 2;           // 32-bit words (column pairs) per row
-constexpr int kBoxRows = 256;             // rows per TMA box (16 KB)
-constexpr int kSlots = 12;                // ring depth = boxes a unit may keep on chip
-constexpr int kConsumerWarps = 8;
-constexpr int kConsumers = 32 * kConsumerWarps;
-constexpr int kColThreads = kConsumers + 32;  // + one producer warp
-constexpr int kMaxGroups = 1024;
-constexpr int kStgPitch = kBoxRows + 16;  // [column][token] staging row, bytes
-constexpr uint32_t kBoxBytes = kBoxRows * kCW * 2;
+#ifndef FP8QGG_COLWISE_CHUNK_BOXES
+#define FP8QGG_COLWISE_CHUNK_BOXES 4
+#endif
+#ifndef FP8QGG_COLWISE_CONSUMER_WARPS
+#define FP8QGG_COLWISE_CONSUMER_WARPS 7
+#endif
+#ifndef FP8QGG_COLWISE_BLOCKS_PER_SM
+#define FP8QGG_COLWISE_BLOCKS_PER_SM 2
+#endif
+#ifndef FP8QGG_COLWISE_LAG_HALF_GRIDS
+#define FP8QGG_COLWISE_LAG_HALF_GRIDS 3
+#endif
 
-enum : int16_t { kLastBox = 1, kResident = 2 };
+constexpr int kCW = 64;                 // columns per unit: 128 bytes of bf16 per row
+constexpr int kWords = kCW / 2;         // 32-bit words (column pairs) per row
+constexpr int kSubRows = 16;            // rows of a slot owned by one consumer warp
+constexpr int kLaneRows = kSubRows / 4; // rows of a lane's block
+constexpr int kConsumerWarps = FP8QGG_COLWISE_CONSUMER_WARPS;  // + the producer warp
+constexpr int kBlocksPerSM = FP8QGG_COLWISE_BLOCKS_PER_SM;
+constexpr int kBoxRows = kSubRows * kConsumerWarps;  // rows per ring slot (112: 14 KB)
+constexpr int kSlots = 6;
+constexpr int kChunkBoxes = FP8QGG_COLWISE_CHUNK_BOXES;
+constexpr int kChunkRows = kChunkBoxes * kBoxRows;   // rows of a whole unit / of a chunk
+constexpr int kConsumers = 32 * kConsumerWarps;
+constexpr int kColThreads = kConsumers + 32;         // + one producer warp
+constexpr int kMaxGroups = 1024;
+constexpr uint32_t kSubBytes = kSubRows * kCW * 2;
+constexpr uint32_t kBoxBytes = kBoxRows * kCW * 2;
+constexpr int kUnitAmaxWords = kCW;     // global absmax of a tall unit: one word per column
+constexpr int kRedBufs = kSlots + 1;
+static_assert(kChunkBoxes <= kSlots, "a task's slots must fit the ring");
+static_assert(kChunkRows % 16 == 0 && kBoxRows % 16 == 0, "boxes and chunks keep 16-row alignment");
+static_assert(kLaneRows == 4 || kLaneRows == 8, "a lane's block is 4 or 8 rows");
+
+enum : int8_t { kTaskWhole = 0, kTaskAmax = 1, kTaskCast = 2, kTaskEnd = 3 };
+enum : int8_t { kFirstBox = 1, kLastBox = 2, kWriteScales = 4 };
 
 struct SlotMeta {
-  int32_t unit;  // position in the size-sorted unit list; -1 ends the stream
-  int32_t y;     // first row of the box (16-aligned)
-  int16_t pass;  // 1: absmax, 2: cast of a unit that did not stay on chip
-  int16_t flags;
+  int32_t y;       // first row of the slot
+  int32_t v0, v1;  // rows [v0, v1) of the slot belong to the task
+  int32_t c0;      // first column of the unit
+  int32_t e;       // group
+  int32_t tu;      // tall unit (amax and cast tasks)
+  int32_t target;  // chunk arrivals that complete the tall unit's absmax
+  int8_t kind;
+  int8_t flags;
+  int16_t nbox;    // slots of the task
 };
+static_assert(sizeof(SlotMeta) == 32, "slot metadata is two 16-byte words");
 
 struct ColSmem {
-  uint32_t ring[kSlots][kBoxRows * kWords];  // [row][16 words]; word = 2 bf16 columns
-  uint8_t stg[kCW * kStgPitch];
-  SlotMeta meta[kSlots];
-  uint32_t red[kConsumers / kWords][kWords];
-  float scale[kCW];
+  uint32_t ring[kSlots][kBoxRows * kWords];  // [row][32 words]; word = 2 bf16 columns
+  // per-warp column absmax of a whole or amax task, one buffer per task that
+  // can be in flight: a warp runs at most kSlots slots (so kSlots tasks)
+  // ahead of another, which may still be reading its buffer
+  alignas(16) uint32_t red[kRedBufs][kConsumerWarps][kWords];
+  alignas(16) SlotMeta meta[kSlots];
+  alignas(16) uint32_t samax[kSlots][kUnitAmaxWords];  // cast tasks: the unit's absmax words
   int32_t end[kMaxGroups];
-  int32_t order[kMaxGroups];
+  int32_t order[kMaxGroups];                 // groups by row span, largest first
+  int32_t prefix[kMaxGroups];                // tall groups: first amax task of the group
   uint64_t full[kSlots];
   uint64_t empty[kSlots];
+  uint64_t red_bar[kRedBufs];
+  int32_t n_tall, na, lag, total;
   int abort;
 };
+static_assert(offsetof(ColSmem, red) % 16 == 0 && offsetof(ColSmem, ring) % 1024 == 0,
+              "16-byte shared-memory accesses and TMA destinations stay aligned");
 
 // Clamped group ends (warp 0): end_e = min(R, max(0, max_{j<=e} offsets[j]))
 // is the closed form of "start_e = end_{e-1}, end_e = clamp(offsets[e],
@@ -91,176 +141,326 @@ __device__ void build_group_ends(ColSmem &sm, const int32_t *offsets, int num_gr
   if (bad && lane == 0 && blockIdx.x == 0) status_or(status, FP8QGG_STATUS_BAD_OFFSETS);
 }
 
-struct Unit {
-  int e, ct;
-  int32_t gstart, gend;
+__device__ __forceinline__ int32_t group_start(const ColSmem &sm, int e) {
+  return e ? sm.end[e - 1] : 0;
+}
+
+// Rows a group's units cover: from the 16-aligned row at or below its first
+// row to its end (0 for an empty group).
+__device__ __forceinline__ int32_t group_span(const ColSmem &sm, int e) {
+  const int32_t s = group_start(sm, e);
+  const int32_t g = sm.end[e];
+  return g > s ? g - (s & ~15) : 0;
+}
+
+struct Task {
+  int16_t kind;
+  int32_t e, ct, k, C, tu;
+  int32_t gstart, r0, r1;  // group's first row; the task's rows [r0, r1)
 };
 
-__device__ __forceinline__ Unit decode_unit(const ColSmem &sm, int32_t u, int n_ct) {
-  Unit r;
-  r.e = sm.order[u / n_ct];
-  r.ct = u - (u / n_ct) * n_ct;
-  r.gstart = r.e ? sm.end[r.e - 1] : 0;
-  r.gend = sm.end[r.e];
+// Task t of the list.  Tall units' amax tasks form stream A, their cast tasks
+// stream B (same order); the list opens with L = min(lag, |A|) tasks of A,
+// then alternates A, B, and ends with the rest of B, so cast task j follows
+// amax task j + L.  Whole units follow.
+__device__ Task decode_task(const ColSmem &sm, int32_t t, int n_ct) {
+  Task r;
+  const int32_t NA = sm.na;
+  if (t < 2 * NA) {
+    const int32_t L = min(sm.lag, NA);
+    bool is_amax;
+    int32_t j;
+    if (t < L) {
+      is_amax = true;
+      j = t;
+    } else if (t < L + 2 * (NA - L)) {
+      const int32_t o = t - L;
+      is_amax = !(o & 1);
+      j = is_amax ? L + (o >> 1) : (o >> 1);
+    } else {
+      is_amax = false;
+      j = (NA - L) + (t - L - 2 * (NA - L));
+    }
+    int lo = 0, hi = sm.n_tall - 1;  // the tall group holding task j
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (sm.prefix[mid] <= j) lo = mid; else hi = mid - 1;
+    }
+    r.e = sm.order[lo];
+    r.gstart = group_start(sm, r.e);
+    const int32_t gend = sm.end[r.e];
+    const int32_t a = r.gstart & ~15;
+    r.C = (gend - a + kChunkRows - 1) / kChunkRows;
+    // chunks of equal height (a multiple of 16, at most kChunkRows)
+    const int32_t ch = ((gend - a + r.C - 1) / r.C + 15) & ~15;
+    const int32_t rr = j - sm.prefix[lo];
+    r.ct = rr / r.C;
+    r.k = rr - r.ct * r.C;
+    r.tu = lo * n_ct + r.ct;
+    r.r0 = a + r.k * ch;
+    r.r1 = min(gend, r.r0 + ch);
+    r.kind = is_amax ? kTaskAmax : kTaskCast;
+  } else {
+    const int32_t s = t - 2 * NA;
+    const int i = sm.n_tall + s / n_ct;
+    r.ct = s - (s / n_ct) * n_ct;
+    r.e = sm.order[i];
+    r.gstart = group_start(sm, r.e);
+    const int32_t gend = sm.end[r.e];
+    r.r0 = r.gstart & ~15;
+    r.r1 = gend > r.gstart ? gend : r.r0;
+    r.k = 0;
+    r.C = 1;
+    r.tu = -1;
+    r.kind = kTaskWhole;
+  }
   return r;
 }
 
-__device__ __forceinline__ void consumer_bar() {
-  asm volatile("bar.sync 1, %0;" ::"n"(kConsumers) : "memory");
-}
+// Every consumer lane owns a kLaneRows x 8 block of its warp's part of a
+// slot: rows kLaneRows * rq + k (rq = lane / 8) and columns 8c8 .. 8c8 + 7
+// (c8 = lane % 8), one 16-byte shared-memory load per row.
+struct Block {
+  uint4 d[kLaneRows];  // row k: columns 8c8 .. 8c8 + 7 as four bf16 pairs
+};
 
-// Barrier over the consumer warps that ANDs a flag across them, so that a
-// wait that gives up is given up by all consumers together.
-__device__ __forceinline__ bool consumer_bar_and(bool v) {
-  uint32_t r;
-  asm volatile(
-      "{\n\t.reg .pred p, q;\n\t"
-      "setp.ne.u32 q, %1, 0;\n\t"
-      "bar.red.and.pred p, 1, %2, q;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(r)
-      : "r"(static_cast<uint32_t>(v)), "n"(kConsumers)
-      : "memory");
-  return r != 0;
-}
-
-// Scale and encode two bf16 values that sit in one 32-bit word but belong to
-// two different columns (two different scales).
-template <int FMT>
-__device__ __forceinline__ uint32_t quant_pair2(uint32_t packed, float s0, float s1, float smax,
-                                                float sat_thr, uint32_t &sat) {
-  const float x0 = __uint_as_float(packed << 16);
-  const float x1 = __uint_as_float(packed & 0xFFFF0000u);
-  float y0 = __fmul_rn(x0, s0);
-  float y1 = __fmul_rn(x1, s1);
-  sat += (fabsf(y0) > sat_thr) + (fabsf(y1) > sat_thr);
-  y0 = fminf(fmaxf(y0, -smax), smax);
-  y1 = fminf(fmaxf(y1, -smax), smax);
-  return cvt_x2<FMT>(y0, y1);
-}
-
-template <int FMT, bool FAST>
-__device__ __forceinline__ uint32_t quant_word(uint32_t w, uint64_t s2, float s0, float s1,
-                                               float smax, float sat_thr, uint32_t &sat) {
-  if constexpr (FAST)
-    return quant_pair_fast<FMT>(w, s2);
-  else
-    return quant_pair2<FMT>(w, s0, s1, smax, sat_thr, sat);
-}
-
-// Cast one box (rows [y, y + 256) of which [v0, v1) belong to the unit) with
-// the unit's scales and store it.  Called by the 256 consumer threads.
-template <int FMT, int LAYOUT, bool FAST>
-__device__ __forceinline__ void cast_box(ColSmem &sm, const uint32_t *box, int32_t y,
-                                         int32_t v0, int32_t v1, int c0, int cols,
-                                         uint8_t *__restrict__ q, int64_t ld_q, float smax,
-                                         float sat_thr, uint32_t &sat) {
-  const int tid = threadIdx.x;
-  if constexpr (LAYOUT == FP8QGG_LAYOUT_SAME) {
+// Loads the lane's block of rows [r0, r1) (other rows read as zero).
+__device__ __forceinline__ void load_block(Block &b, const uint32_t *sub, int32_t ys, int32_t r0,
+                                           int32_t r1, int lane) {
+  const int rq = lane >> 3, c8 = lane & 7;
+  const uint4 *src = reinterpret_cast<const uint4 *>(sub + kLaneRows * rq * kWords + 4 * c8);
+  if (r0 == ys && r1 == ys + kSubRows) {  // the warp's rows all belong to the task
 #pragma unroll
-    for (int k = 0; k < (kBoxRows * kCW / 8) / kConsumers; ++k) {
-      const int idx = tid + k * kConsumers;
-      const int rr = idx >> 2;   // row in box
-      const int j = idx & 3;     // 8-column vector
-      const int32_t row = y + rr;
-      if (row < v0 || row >= v1 || c0 + 8 * j >= cols) continue;
-      const uint4 v = *reinterpret_cast<const uint4 *>(&box[rr * kWords + 4 * j]);
-      const float *sc = &sm.scale[8 * j];
-      uint2 o;
-      o.x = quant_word<FMT, FAST>(v.x, pack_f32x2(sc[0], sc[1]), sc[0], sc[1], smax, sat_thr, sat) |
-            (quant_word<FMT, FAST>(v.y, pack_f32x2(sc[2], sc[3]), sc[2], sc[3], smax, sat_thr,
-                                   sat) << 16);
-      o.y = quant_word<FMT, FAST>(v.z, pack_f32x2(sc[4], sc[5]), sc[4], sc[5], smax, sat_thr, sat) |
-            (quant_word<FMT, FAST>(v.w, pack_f32x2(sc[6], sc[7]), sc[6], sc[7], smax, sat_thr,
-                                   sat) << 16);
-      *reinterpret_cast<uint2 *>(q + static_cast<int64_t>(row) * ld_q + c0 + 8 * j) = o;
-    }
+    for (int k = 0; k < kLaneRows; ++k) b.d[k] = src[k * (kWords / 4)];
   } else {
-    // cast: thread -> column pair cp, 16-row group g
-    const int cp = tid & (kWords - 1);
-    const int g = tid / kWords;
-    const float s0 = sm.scale[2 * cp];
-    const float s1 = sm.scale[2 * cp + 1];
-    const uint64_t s01 = pack_f32x2(s0, s1);
-    uint32_t lo4[4] = {0u, 0u, 0u, 0u};
-    uint32_t hi4[4] = {0u, 0u, 0u, 0u};
-    const int32_t gb = y + 16 * g;
-    if (gb < v1 && gb + 16 > v0) {
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        const int32_t row = gb + i;
-        const uint32_t w = (row >= v0 && row < v1) ? box[(16 * g + i) * kWords + cp] : 0u;
-        const uint32_t c2 = quant_word<FMT, FAST>(w, s01, s0, s1, smax, sat_thr, sat);
-        lo4[i >> 2] |= (c2 & 0xFFu) << (8 * (i & 3));
-        hi4[i >> 2] |= (c2 >> 8) << (8 * (i & 3));
-      }
+    for (int k = 0; k < kLaneRows; ++k) {
+      const int32_t row = ys + kLaneRows * rq + k;
+      b.d[k] = (row >= r0 && row < r1) ? src[k * (kWords / 4)] : make_uint4(0u, 0u, 0u, 0u);
     }
-    *reinterpret_cast<uint4 *>(&sm.stg[(2 * cp) * kStgPitch + 16 * g]) =
-        make_uint4(lo4[0], lo4[1], lo4[2], lo4[3]);
-    *reinterpret_cast<uint4 *>(&sm.stg[(2 * cp + 1) * kStgPitch + 16 * g]) =
-        make_uint4(hi4[0], hi4[1], hi4[2], hi4[3]);
-    consumer_bar();
-    // store: 16 consecutive threads write the 256 tokens of one output row
-#pragma unroll
-    for (int k = 0; k < (kCW * kBoxRows / 16) / kConsumers; ++k) {
-      const int idx = tid + k * kConsumers;
-      const int c = idx / (kBoxRows / 16);
-      const int sgi = idx % (kBoxRows / 16);
-      const int32_t g0 = y + 16 * sgi;
-      if (c0 + c >= cols || g0 >= v1 || g0 + 16 <= v0) continue;
-      uint8_t *dst = q + static_cast<int64_t>(c0 + c) * ld_q + g0;
-      const uint8_t *src = &sm.stg[c * kStgPitch + 16 * sgi];
-      if (g0 >= v0 && g0 + 16 <= v1) {
-        *reinterpret_cast<uint4 *>(dst) = *reinterpret_cast<const uint4 *>(src);
-      } else {
-        for (int b = 0; b < 16; ++b)
-          if (g0 + b >= v0 && g0 + b < v1) dst[b] = src[b];
-      }
-    }
-    consumer_bar();
   }
 }
 
+__device__ __forceinline__ void amax_block(uint4 &am, const Block &b) {
+#pragma unroll
+  for (int k = 0; k < kLaneRows; ++k) {
+    am.x = absmax_acc(am.x, b.d[k].x);
+    am.y = absmax_acc(am.y, b.d[k].y);
+    am.z = absmax_acc(am.z, b.d[k].z);
+    am.w = absmax_acc(am.w, b.d[k].w);
+  }
+}
+
+// Magnitude bit patterns of a running absmax (comparable as unsigned halves).
+__device__ __forceinline__ uint4 finish_amax(uint4 am) {
+  return make_uint4(absmax_bits(am.x), absmax_bits(am.y), absmax_bits(am.z), absmax_bits(am.w));
+}
+
+// The lane's 8 column scales: s[j] for column 8c8 + j.  The paired
+// multiplies take them as (s[2p], s[2p + 1]) (SAME: adjacent columns, which
+// are adjacent registers) or (s[j], s[j]) (TRANSPOSED: one column, two rows).
+template <int LAYOUT>
+struct ColScales {
+  float s[8];
+};
+
+template <int LAYOUT>
+__device__ __forceinline__ void scales_from_bits(ColScales<LAYOUT> &sc, const uint32_t (&a)[8],
+                                                 float smax) {
+#pragma unroll
+  for (int i = 0; i < 8; ++i) sc.s[i] = scale_from_amax(bf16_bits_to_float(a[i]), smax);
+}
+
+template <int LAYOUT>
+__device__ __forceinline__ void write_scales(const ColScales<LAYOUT> &sc, float *scales, int e,
+                                             int c0, int cols, int lane) {
+  const int c = c0 + 8 * lane;
+  if (lane < 8 && c < cols) {
+    float4 *dst = reinterpret_cast<float4 *>(scales + static_cast<int64_t>(e) * cols + c);
+    if ((reinterpret_cast<uintptr_t>(dst) & 15) == 0) {
+      dst[0] = make_float4(sc.s[0], sc.s[1], sc.s[2], sc.s[3]);
+      dst[1] = make_float4(sc.s[4], sc.s[5], sc.s[6], sc.s[7]);
+    } else {
+      float *d = scales + static_cast<int64_t>(e) * cols + c;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) d[i] = sc.s[i];
+    }
+  }
+}
+
+// Scale, clamp and encode two values (each with its own scale); the first
+// goes to the low byte.  FAST: one packed multiply, no clamp, no count (see
+// quant_pair_fast).
+template <int FMT, bool FAST>
+__device__ __forceinline__ uint32_t enc2(float x0, float x1, uint64_t s01, float s0, float s1,
+                                         float smax, float sat_thr, uint32_t &sat) {
+  if constexpr (FAST) {
+    uint64_t xx, yy;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(xx) : "f"(x0), "f"(x1));
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(yy) : "l"(xx), "l"(s01));
+    float y0, y1;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(y0), "=f"(y1) : "l"(yy));
+    return cvt_x2<FMT>(y0, y1);
+  } else {
+    float y0 = __fmul_rn(x0, s0);
+    float y1 = __fmul_rn(x1, s1);
+    sat += (fabsf(y0) > sat_thr) + (fabsf(y1) > sat_thr);
+    y0 = clamp_keep_nan(y0, smax);
+    y1 = clamp_keep_nan(y1, smax);
+    return cvt_x2<FMT>(y0, y1);
+  }
+}
+
+__device__ __forceinline__ uint32_t word_at(const uint4 &v, int p) {
+  return p == 0 ? v.x : p == 1 ? v.y : p == 2 ? v.z : v.w;
+}
+
+// Casts the lane's block (rows [r0, r1) of the warp part starting at row ys)
+// and stores the codes; rows outside [r0, r1) belong to other groups and are
+// never written.  SAME: one 8-byte store per row (columns 8c8 .. 8c8 + 7).
+// TRANSPOSED: adjacent rows of one column are encoded together, and one store
+// per column holds the lane's kLaneRows tokens; the four lanes with the same
+// c8 write 4 * kLaneRows consecutive tokens of that column.
 template <int FMT, int LAYOUT, bool FAST>
-__global__ void __launch_bounds__(kColThreads, 1)
-    quant_colwise_jagged_kernel(const __grid_constant__ CUtensorMap xmap, int64_t rows_total,
+__device__ __forceinline__ void cast_block(const Block &b, int32_t ys, int32_t r0, int32_t r1,
+                                           int c0, int cols, uint8_t *__restrict__ q,
+                                           int64_t ld_q, const ColScales<LAYOUT> &sc, float smax,
+                                           float sat_thr, uint32_t &sat, int lane) {
+  const int rq = lane >> 3, c8 = lane & 7;
+  const int32_t rb = ys + kLaneRows * rq;  // the block's first row
+  if (r0 >= r1 || rb >= r1 || rb + kLaneRows <= r0 || c0 + 8 * c8 >= cols) return;
+  if constexpr (LAYOUT == FP8QGG_LAYOUT_SAME) {
+#pragma unroll
+    for (int k = 0; k < kLaneRows; ++k) {
+      const int32_t row = rb + k;
+      if (row < r0 || row >= r1) continue;
+      uint32_t c[4];
+#pragma unroll
+      for (int p = 0; p < 4; ++p) {
+        const uint32_t w = word_at(b.d[k], p);
+        c[p] = enc2<FMT, FAST>(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u),
+                               pack_f32x2(sc.s[2 * p], sc.s[2 * p + 1]), sc.s[2 * p],
+                               sc.s[2 * p + 1], smax, sat_thr, sat);
+      }
+      *reinterpret_cast<uint2 *>(q + static_cast<int64_t>(row) * ld_q + c0 + 8 * c8) =
+          make_uint2(c[0] | (c[1] << 16), c[2] | (c[3] << 16));
+    }
+  } else {
+    const bool full = rb >= r0 && rb + kLaneRows <= r1;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int p = j >> 1;
+      uint32_t c[kLaneRows / 2];
+#pragma unroll
+      for (int m = 0; m < kLaneRows / 2; ++m) {
+        const uint32_t w0 = word_at(b.d[2 * m], p);
+        const uint32_t w1 = word_at(b.d[2 * m + 1], p);
+        const float x0 = __uint_as_float((j & 1) ? (w0 & 0xFFFF0000u) : (w0 << 16));
+        const float x1 = __uint_as_float((j & 1) ? (w1 & 0xFFFF0000u) : (w1 << 16));
+        c[m] = enc2<FMT, FAST>(x0, x1, pack_f32x2(sc.s[j], sc.s[j]), sc.s[j], sc.s[j], smax,
+                               sat_thr, sat);
+      }
+      uint32_t tok[kLaneRows / 4];  // the lane's tokens of column 8c8 + j
+#pragma unroll
+      for (int i = 0; i < kLaneRows / 4; ++i) tok[i] = c[2 * i] | (c[2 * i + 1] << 16);
+      uint8_t *dst = q + static_cast<int64_t>(c0 + 8 * c8 + j) * ld_q + rb;
+      if (full) {
+        if constexpr (kLaneRows == 8)
+          *reinterpret_cast<uint2 *>(dst) = make_uint2(tok[0], tok[kLaneRows / 4 - 1]);
+        else
+          *reinterpret_cast<uint32_t *>(dst) = tok[0];
+      } else {
+#pragma unroll
+        for (int k = 0; k < kLaneRows; ++k)
+          if (rb + k >= r0 && rb + k < r1)
+            dst[k] = static_cast<uint8_t>(tok[k >> 2] >> (8 * (k & 3)));
+      }
+    }
+  }
+}
+
+__device__ __forceinline__ void split_bits(uint32_t (&a)[8], const uint4 &m) {
+  a[0] = m.x & 0xFFFFu; a[1] = m.x >> 16; a[2] = m.y & 0xFFFFu; a[3] = m.y >> 16;
+  a[4] = m.z & 0xFFFFu; a[5] = m.z >> 16; a[6] = m.w & 0xFFFFu; a[7] = m.w >> 16;
+}
+
+template <int FMT, int LAYOUT, bool FAST>
+__global__ void __launch_bounds__(kColThreads, kBlocksPerSM)
+    quant_colwise_jagged_kernel(const __grid_constant__ CUtensorMap xmap_box,
+                                const __grid_constant__ CUtensorMap xmap_sub, int64_t rows_total,
                                 int cols, const int32_t *__restrict__ offsets, int num_groups,
                                 uint8_t *__restrict__ q, int64_t ld_q,
                                 float *__restrict__ scales, float smax, float sat_thr,
                                 unsigned long long *sat_count, int32_t *status,
-                                uint32_t *__restrict__ work_counter) {
+                                uint32_t *__restrict__ work_counter, uint32_t *__restrict__ arrive,
+                                uint32_t *__restrict__ unit_amax, int32_t units_cap) {
   extern __shared__ uint8_t smem_raw[];
-  ColSmem &sm = *reinterpret_cast<ColSmem *>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  ColSmem &sm = *align_smem_1024<ColSmem>(smem_raw);
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
   const int lane = tid & 31;
   const int n_ct = (cols + kCW - 1) / kCW;
 
   if (tid == kConsumers) {
-    prefetch_tensormap(&xmap);
+    prefetch_tensormap(&xmap_box);
+    prefetch_tensormap(&xmap_sub);
     for (int s = 0; s < kSlots; ++s) {
-      mbar_init(&sm.full[s], 1);
+      mbar_init(&sm.full[s], 2);  // the copy's bytes + two producer arrivals
       mbar_init(&sm.empty[s], kConsumerWarps);
     }
+    for (int b = 0; b < kRedBufs; ++b) mbar_init(&sm.red_bar[b], kConsumerWarps);
     sm.abort = 0;
     fence_mbarrier_init();
   }
   build_group_ends(sm, offsets, num_groups, rows_total, status);
   __syncthreads();
-  // groups ranked by row count, largest first (ties by index)
+  // groups ranked by row span, largest first (ties by index)
   for (int e = tid; e < num_groups; e += kColThreads) {
-    const int32_t se = sm.end[e] - (e ? sm.end[e - 1] : 0);
+    const int32_t se = group_span(sm, e);
     int rank = 0;
     for (int f = 0; f < num_groups; ++f) {
-      const int32_t sf = sm.end[f] - (f ? sm.end[f - 1] : 0);
+      const int32_t sf = group_span(sm, f);
       rank += (sf > se) || (sf == se && f < e);
     }
     sm.order[rank] = e;
   }
   __syncthreads();
+  // tall groups (span above one chunk) are a prefix of the order; prefix sums
+  // of their amax-task counts (n_ct units x chunks each)
+  if (warp == 0) {
+    int32_t carry = 0;
+    int n_tall = 0;
+    for (int base = 0; base < num_groups; base += 32) {
+      const int i = base + lane;
+      int32_t c = 0;
+      if (i < num_groups) {
+        const int32_t sp = group_span(sm, sm.order[i]);
+        if (sp > kChunkRows) c = n_ct * ((sp + kChunkRows - 1) / kChunkRows);
+      }
+      int32_t incl = c;
+      for (int d = 1; d < 32; d <<= 1) {
+        const int32_t o = __shfl_up_sync(0xFFFFFFFFu, incl, d);
+        if (lane >= d) incl += o;
+      }
+      if (i < num_groups) sm.prefix[i] = carry + incl - c;
+      n_tall += __popc(__ballot_sync(0xFFFFFFFFu, c > 0));
+      carry += __shfl_sync(0xFFFFFFFFu, incl, 31);
+    }
+    if (lane == 0) {
+      sm.n_tall = n_tall;
+      sm.na = carry;
+      const int32_t c_max =
+          n_tall ? (group_span(sm, sm.order[0]) + kChunkRows - 1) / kChunkRows : 0;
+      sm.lag = max(FP8QGG_COLWISE_LAG_HALF_GRIDS * static_cast<int32_t>(gridDim.x) / 2, c_max);
+      sm.total = 2 * carry + (num_groups - n_tall) * n_ct;
+    }
+  }
+  __syncthreads();
+  if (sm.n_tall * n_ct > units_cap) {  // cannot happen for clamped ends; guards the workspace
+    if (tid == 0 && blockIdx.x == 0) status_or(status, FP8QGG_STATUS_BAD_OFFSETS);
+    return;
+  }
 
-  const int32_t total_units = num_groups * n_ct;
   volatile int *abort = &sm.abort;
 
   if (warp == kConsumerWarps) {
@@ -270,42 +470,95 @@ __global__ void __launch_bounds__(kColThreads, 1)
       uint32_t armed = 0;  // slots whose latest phase carries a copy
       uint32_t armed_par[kSlots];
       bool ok = true;
-      auto push = [&](int32_t unit, int32_t y, int16_t pass, int16_t flags, bool load,
-                      int c0) -> bool {
+      // A cast task's first slot also carries the unit's absmax: the producer
+      // waits (bounded) until every chunk of the unit has been counted, then
+      // copies the 64 absmax words into the slot before its second arrival.
+      auto fetch_unit_amax = [&](const SlotMeta &m, uint32_t *dst) -> bool {
+        const uint32_t *cnt = arrive + m.tu;
+        uint32_t v;
+        asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(cnt) : "memory");
+        if (v < static_cast<uint32_t>(m.target)) {
+          const uint64_t t0 = global_timer_ns();
+          while (true) {
+            __nanosleep(256);
+            asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(cnt) : "memory");
+            if (v >= static_cast<uint32_t>(m.target)) break;
+            if (*abort || global_timer_ns() - t0 > kWaitLimitNs) return false;
+          }
+        }
+        const uint4 *src =
+            reinterpret_cast<const uint4 *>(unit_amax + static_cast<int64_t>(m.tu) * kUnitAmaxWords);
+        uint4 words[kUnitAmaxWords / 4];
+#pragma unroll
+        for (int i = 0; i < kUnitAmaxWords / 4; ++i) words[i] = __ldcg(src + i);
+#pragma unroll
+        for (int i = 0; i < kUnitAmaxWords / 4; ++i) reinterpret_cast<uint4 *>(dst)[i] = words[i];
+        return true;
+      };
+      auto push = [&](const SlotMeta &m, int j0, int j1, bool load) -> bool {
         if (!mbar_wait(&sm.empty[slot], phase ^ 1, abort)) return false;
-        sm.meta[slot] = SlotMeta{unit, y, pass, flags};
+        sm.meta[slot] = m;
         if (load) {
-          mbar_arrive_expect_tx(&sm.full[slot], kBoxBytes);
-          tma_load_2d(sm.ring[slot], &xmap, &sm.full[slot], c0, y);
+          if (j0 == 0 && j1 == kConsumerWarps - 1) {
+            mbar_arrive_expect_tx(&sm.full[slot], kBoxBytes);
+            tma_load_2d(sm.ring[slot], &xmap_box, &sm.full[slot], m.c0, m.y);
+          } else {
+            mbar_arrive_expect_tx(&sm.full[slot], (j1 - j0 + 1) * kSubBytes);
+            for (int j = j0; j <= j1; ++j)
+              tma_load_2d(sm.ring[slot] + j * kSubRows * kWords, &xmap_sub, &sm.full[slot], m.c0,
+                          m.y + j * kSubRows);
+          }
           armed |= 1u << slot;
           armed_par[slot] = phase;
         } else {
           mbar_arrive(&sm.full[slot]);
           armed &= ~(1u << slot);
         }
+        bool fetched = true;
+        if (m.kind == kTaskCast && (m.flags & kFirstBox))
+          fetched = fetch_unit_amax(m, sm.samax[slot]);
+        // the second arrival comes even after a failed fetch, so that the
+        // phase still ends when the copy lands
+        mbar_arrive(&sm.full[slot]);
         if (++slot == kSlots) { slot = 0; phase ^= 1; }
-        return true;
+        return fetched;
       };
-      int32_t u = static_cast<int32_t>(atomicAdd(work_counter, 1u));
-      while (ok && u < total_units) {
+      const int32_t total = sm.total;
+      int32_t t = static_cast<int32_t>(atomicAdd(work_counter, 1u));
+      while (ok && t < total) {
         const int32_t next = static_cast<int32_t>(atomicAdd(work_counter, 1u));
-        const Unit un = decode_unit(sm, u, n_ct);
-        const int c0 = un.ct * kCW;
-        if (un.gend <= un.gstart) {
-          ok = push(u, un.gstart & ~15, 1, kLastBox | kResident, false, c0);
+        const Task tk = decode_task(sm, t, n_ct);
+        SlotMeta m;
+        m.c0 = tk.ct * kCW;
+        m.e = tk.e;
+        m.tu = tk.tu;
+        m.target = tk.C;
+        m.kind = tk.kind;
+        if (tk.r1 <= tk.r0) {  // empty group: scales only
+          m.y = tk.r0;
+          m.v0 = m.v1 = tk.r0;
+          m.flags = kFirstBox | kLastBox;
+          m.nbox = 1;
+          ok = push(m, 0, 0, false);
         } else {
-          const int32_t A = un.gstart & ~15;
-          const int nbox = (un.gend - A + kBoxRows - 1) / kBoxRows;
-          const int16_t res = nbox <= kSlots ? kResident : 0;
-          for (int b = 0; ok && b < nbox; ++b)
-            ok = push(u, A + b * kBoxRows, 1, (b == nbox - 1 ? kLastBox : 0) | res, true, c0);
-          if (!res)
-            for (int b = 0; ok && b < nbox; ++b)
-              ok = push(u, A + b * kBoxRows, 2, b == nbox - 1 ? kLastBox : 0, true, c0);
+          const int nb = (tk.r1 - tk.r0 + kBoxRows - 1) / kBoxRows;
+          m.nbox = static_cast<int16_t>(nb);
+          for (int b = 0; ok && b < nb; ++b) {
+            m.y = tk.r0 + b * kBoxRows;
+            m.v0 = max(tk.gstart, m.y);
+            m.v1 = min(tk.r1, m.y + kBoxRows);
+            m.flags = (b == 0 ? kFirstBox : 0) | (b == nb - 1 ? kLastBox : 0) |
+                      (tk.kind == kTaskCast && tk.k == 0 ? kWriteScales : 0);
+            ok = push(m, (m.v0 - m.y) / kSubRows, (m.v1 - 1 - m.y) / kSubRows, true);
+          }
         }
-        u = next;
+        t = next;
       }
-      if (ok) ok = push(-1, 0, 0, 0, false, 0);
+      if (ok) {
+        SlotMeta m{};
+        m.kind = kTaskEnd;
+        ok = push(m, 0, 0, false);
+      }
       if (!ok) {
         *abort = 1;
         status_or(status, FP8QGG_STATUS_TIMEOUT);
@@ -317,77 +570,153 @@ __global__ void __launch_bounds__(kColThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ consumers
+    const int w = warp;
+    const int c8 = lane & 7;
     uint32_t slot = 0, phase = 0;
     uint32_t sat = 0;
-    const int cp = tid & (kWords - 1);     // absmax: column pair
-    const int rp = tid / kWords;           // absmax: row phase (0..15)
-    constexpr int kPhases = kConsumers / kWords;
-    uint32_t am = 0;
-    uint32_t res_slot = 0, res_phase = 0;  // first ring slot of an on-chip unit
-    int res_count = 0;
-    while (true) {
-      const bool got = mbar_wait(&sm.full[slot], phase, abort);
-      if (!consumer_bar_and(got)) {
-        *abort = 1;
-        if (tid == 0) status_or(status, FP8QGG_STATUS_TIMEOUT);
-        break;
-      }
-      const SlotMeta m = sm.meta[slot];
-      if (m.unit < 0) break;
-      const Unit un = decode_unit(sm, m.unit, n_ct);
-      const int c0 = un.ct * kCW;
-      const int32_t v0 = max(un.gstart, m.y);
-      const int32_t v1 = min(un.gend, m.y + kBoxRows);
-      const uint32_t *box = sm.ring[slot];
-      if (m.pass == 1) {
-        for (int32_t rr = max(v0 - m.y, 0) + ((rp - max(v0 - m.y, 0)) % kPhases + kPhases) % kPhases;
-             rr < v1 - m.y; rr += kPhases)
-          am = abs_max_bf16x2(am, box[rr * kWords + cp]);
-        if (m.flags & kResident) {
-          if (res_count == 0) { res_slot = slot; res_phase = phase; }
-          ++res_count;
-        } else {
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&sm.empty[slot]);
-        }
-        if (m.flags & kLastBox) {
-          // column absmax over the row phases -> the unit's 32 scales
-          sm.red[rp][cp] = am;
-          consumer_bar();
-          if (tid < kWords) {
-            uint32_t mm = 0;
-#pragma unroll
-            for (int ph = 0; ph < kPhases; ++ph) mm = __vmaxu2(mm, sm.red[ph][tid]);
-            const float sa = scale_from_amax(__uint_as_float((mm & 0xFFFFu) << 16), smax);
-            const float sb = scale_from_amax(__uint_as_float(mm & 0xFFFF0000u), smax);
-            sm.scale[2 * tid] = sa;
-            sm.scale[2 * tid + 1] = sb;
-            const int64_t base = static_cast<int64_t>(un.e) * cols + c0 + 2 * tid;
-            if (c0 + 2 * tid < cols) scales[base] = sa;
-            if (c0 + 2 * tid + 1 < cols) scales[base + 1] = sb;
-          }
-          consumer_bar();
-          am = 0;
-          // a unit that stayed on chip is cast now, box by box, from the ring
-          uint32_t s2 = res_slot;
-          for (int i = 0; i < res_count; ++i) {
-            const SlotMeta mi = sm.meta[s2];
-            cast_box<FMT, LAYOUT, FAST>(sm, sm.ring[s2], mi.y, max(un.gstart, mi.y),
-                                        min(un.gend, mi.y + kBoxRows), c0, cols, q, ld_q, smax,
-                                        sat_thr, sat);
-            consumer_bar();
-            if (lane == 0) mbar_arrive(&sm.empty[s2]);
-            if (++s2 == kSlots) s2 = 0;
-          }
-          res_count = 0;
-          (void)res_phase;
-        }
-      } else {
-        cast_box<FMT, LAYOUT, FAST>(sm, box, m.y, v0, v1, c0, cols, q, ld_q, smax, sat_thr, sat);
-        consumer_bar();
-        if (lane == 0) mbar_arrive(&sm.empty[slot]);
-      }
+    int rbuf = 0;
+    uint32_t rpar = 0;  // bit b: parity of the next phase of red_bar[b]
+    static_assert(kRedBufs <= 32, "parity bits fit one word");
+    ColScales<LAYOUT> sc;
+    uint4 chunk_am = make_uint4(0u, 0u, 0u, 0u);  // amax tasks: absmax over the chunk so far
+    uint32_t pub_turn = 0;  // the warp that publishes the next amax task
+    bool failed = false;
+    auto advance = [&]() {
       if (++slot == kSlots) { slot = 0; phase ^= 1; }
+    };
+    auto release = [&]() {
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.empty[slot]);
+    };
+    while (!failed) {
+      if (!mbar_wait(&sm.full[slot], phase, abort)) { failed = true; break; }
+      SlotMeta m = sm.meta[slot];
+      if (m.kind == kTaskEnd) break;
+      if (m.kind == kTaskWhole) {
+        // up to kChunkBoxes slots; the lane keeps its blocks in registers and
+        // frees each slot at once, so the ring keeps streaming
+        Block blk[kChunkBoxes];
+        int32_t ysb[kChunkBoxes], r0b[kChunkBoxes], r1b[kChunkBoxes];
+        uint4 am = make_uint4(0u, 0u, 0u, 0u);
+        const int nb = m.nbox;
+#pragma unroll
+        for (int b = 0; b < kChunkBoxes; ++b) {
+          ysb[b] = 0;
+          r0b[b] = r1b[b] = 0;
+          if (b < nb && !failed) {
+            if (b > 0) {
+              advance();
+              if (!mbar_wait(&sm.full[slot], phase, abort)) { failed = true; continue; }
+              m = sm.meta[slot];
+            }
+            ysb[b] = m.y + w * kSubRows;
+            r0b[b] = max(m.v0, ysb[b]);
+            r1b[b] = min(m.v1, ysb[b] + kSubRows);
+            load_block(blk[b], sm.ring[slot] + w * kSubRows * kWords, ysb[b], r0b[b], r1b[b],
+                       lane);
+            release();
+            amax_block(am, blk[b]);
+          }
+        }
+        if (failed) break;
+        // the warp's column absmax (rows meet by shuffles), then the warps'
+        // meet in shared memory
+        am = finish_amax(am);
+#pragma unroll
+        for (int d = 8; d < 32; d <<= 1) {
+          am.x = __vmaxu2(am.x, __shfl_xor_sync(0xFFFFFFFFu, am.x, d));
+          am.y = __vmaxu2(am.y, __shfl_xor_sync(0xFFFFFFFFu, am.y, d));
+          am.z = __vmaxu2(am.z, __shfl_xor_sync(0xFFFFFFFFu, am.z, d));
+          am.w = __vmaxu2(am.w, __shfl_xor_sync(0xFFFFFFFFu, am.w, d));
+        }
+        if (lane < 8) *reinterpret_cast<uint4 *>(&sm.red[rbuf][w][4 * c8]) = am;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.red_bar[rbuf]);
+        if (!mbar_wait(&sm.red_bar[rbuf], (rpar >> rbuf) & 1u, abort)) { failed = true; break; }
+        rpar ^= 1u << rbuf;
+        uint4 mm = make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+        for (int wp = 0; wp < kConsumerWarps; ++wp) {
+          const uint4 v = *reinterpret_cast<const uint4 *>(&sm.red[rbuf][wp][4 * c8]);
+          mm.x = __vmaxu2(mm.x, v.x);
+          mm.y = __vmaxu2(mm.y, v.y);
+          mm.z = __vmaxu2(mm.z, v.z);
+          mm.w = __vmaxu2(mm.w, v.w);
+        }
+        if (++rbuf == kRedBufs) rbuf = 0;
+        uint32_t a[8];
+        split_bits(a, mm);
+        scales_from_bits<LAYOUT>(sc, a, smax);
+        if (w == 0) write_scales<LAYOUT>(sc, scales, m.e, m.c0, cols, lane);
+#pragma unroll
+        for (int b = 0; b < kChunkBoxes; ++b)
+          if (b < nb)
+            cast_block<FMT, LAYOUT, FAST>(blk[b], ysb[b], r0b[b], r1b[b], m.c0, cols, q, ld_q, sc,
+                                          smax, sat_thr, sat, lane);
+      } else {
+        const int32_t ys = m.y + w * kSubRows;
+        const int32_t r0 = max(m.v0, ys);
+        const int32_t r1 = min(m.v1, ys + kSubRows);
+        if (m.kind == kTaskCast && (m.flags & kFirstBox)) {
+          // the unit's absmax words came with the slot (read before it is freed)
+          const uint4 x0 = *reinterpret_cast<const uint4 *>(&sm.samax[slot][8 * c8]);
+          const uint4 x1 = *reinterpret_cast<const uint4 *>(&sm.samax[slot][8 * c8 + 4]);
+          const uint32_t a[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+          scales_from_bits<LAYOUT>(sc, a, smax);
+        }
+        Block blk;
+        load_block(blk, sm.ring[slot] + w * kSubRows * kWords, ys, r0, r1, lane);
+        release();
+        if (m.kind == kTaskCast) {
+          if ((m.flags & kFirstBox) && (m.flags & kWriteScales) && w == 0)
+            write_scales<LAYOUT>(sc, scales, m.e, m.c0, cols, lane);
+          cast_block<FMT, LAYOUT, FAST>(blk, ys, r0, r1, m.c0, cols, q, ld_q, sc, smax, sat_thr,
+                                        sat, lane);
+        } else {
+          uint4 &am = chunk_am;
+          amax_block(am, blk);
+          if (m.flags & kLastBox) {
+            am = finish_amax(am);
+#pragma unroll
+            for (int d = 8; d < 32; d <<= 1) {
+              am.x = __vmaxu2(am.x, __shfl_xor_sync(0xFFFFFFFFu, am.x, d));
+              am.y = __vmaxu2(am.y, __shfl_xor_sync(0xFFFFFFFFu, am.y, d));
+              am.z = __vmaxu2(am.z, __shfl_xor_sync(0xFFFFFFFFu, am.z, d));
+              am.w = __vmaxu2(am.w, __shfl_xor_sync(0xFFFFFFFFu, am.w, d));
+            }
+            // the warps' partials meet in shared memory; one warp (turn by
+            // turn) merges the chunk's absmax into the unit's words in global
+            // memory and counts the chunk, the others go on at once
+            if (lane < 8) *reinterpret_cast<uint4 *>(&sm.red[rbuf][w][4 * c8]) = am;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm.red_bar[rbuf]);
+            if (w == static_cast<int>(pub_turn)) {
+              if (!mbar_wait(&sm.red_bar[rbuf], (rpar >> rbuf) & 1u, abort)) {
+                failed = true;
+                break;
+              }
+              uint32_t mm = 0;
+#pragma unroll
+              for (int wp = 0; wp < kConsumerWarps; ++wp) mm = __vmaxu2(mm, sm.red[rbuf][wp][lane]);
+              uint32_t *ua = unit_amax + static_cast<int64_t>(m.tu) * kUnitAmaxWords + 2 * lane;
+              atomicMax(ua, mm & 0xFFFFu);
+              atomicMax(ua + 1, mm >> 16);
+              __threadfence();  // every lane's merges are visible before the count
+              __syncwarp();
+              if (lane == 0) atomicAdd(arrive + m.tu, 1u);
+            }
+            rpar ^= 1u << rbuf;
+            if (++rbuf == kRedBufs) rbuf = 0;
+            if (++pub_turn == kConsumerWarps) pub_turn = 0;
+            am = make_uint4(0u, 0u, 0u, 0u);
+          }
+        }
+      }
+      advance();
+    }
+    if (failed) {
+      *abort = 1;
+      if (lane == 0) status_or(status, FP8QGG_STATUS_TIMEOUT);
     }
     if (!FAST && sat_count) {
 #pragma unroll
@@ -399,9 +728,9 @@ __global__ void __launch_bounds__(kColThreads, 1)
 
 namespace {
 
-using ColKernel = void (*)(const CUtensorMap, int64_t, int, const int32_t *, int, uint8_t *,
-                           int64_t, float *, float, float, unsigned long long *, int32_t *,
-                           uint32_t *);
+using ColKernel = void (*)(const CUtensorMap, const CUtensorMap, int64_t, int, const int32_t *,
+                           int, uint8_t *, int64_t, float *, float, float, unsigned long long *,
+                           int32_t *, uint32_t *, uint32_t *, uint32_t *, int32_t);
 
 template <int FMT, bool FAST>
 ColKernel col_kernel_fmt(int layout) {
@@ -419,10 +748,28 @@ ColKernel col_kernel(int fmt, int layout, bool fast) {
               : col_kernel_fmt<FP8QGG_E4M3FNUZ, false>(layout);
 }
 
-}  // namespace
+// Scratch layout: [0, 256) the work counter; then one arrival counter per
+// tall unit (rounded up to 256 bytes); then 64 absmax words per tall unit.
+// A tall group has at least kChunkRows - 14 rows, so at most
+// rows_total / (kChunkRows - 16) groups are tall.
+struct ColScratch {
+  int64_t units_cap;
+  size_t arrive_off, amax_off, bytes;
+};
 
-// Bytes of scratch the kernel needs: one work counter, rounded to 256.
-constexpr size_t kColwiseScratchBytes = 256;
+ColScratch colwise_scratch(int64_t rows_total, int64_t cols, int32_t num_groups) {
+  ColScratch s;
+  const int64_t n_ct = (std::max<int64_t>(cols, 1) + kCW - 1) / kCW;
+  const int64_t tall = std::min<int64_t>(std::max<int32_t>(num_groups, 0),
+                                         std::max<int64_t>(rows_total, 0) / (kChunkRows - 16));
+  s.units_cap = tall * n_ct;
+  s.arrive_off = 256;
+  s.amax_off = s.arrive_off + (static_cast<size_t>(s.units_cap) * 4 + 255) / 256 * 256;
+  s.bytes = s.amax_off + static_cast<size_t>(s.units_cap) * kUnitAmaxWords * 4;
+  return s;
+}
+
+}  // namespace
 
 // Validates the arguments of a jagged column-wise call; returns FP8QGG_OK or
 // the error code.
@@ -430,7 +777,7 @@ int colwise_check(const void *x, int64_t rows_total, int64_t cols, int64_t ld_x,
                   const int32_t *offsets, int32_t num_groups, uint8_t *q, int64_t ld_q,
                   int layout, float *scales, int fmt, float scale_max, uint64_t *sat_count,
                   int32_t *dev_status) {
-  if (rows_total < 0 || rows_total > INT32_MAX - 2 * kBoxRows) return FP8QGG_ERR_SHAPE;
+  if (rows_total < 0 || rows_total > INT32_MAX - 4 * kChunkRows) return FP8QGG_ERR_SHAPE;
   if (cols < 1 || cols > INT32_MAX / 2 || ld_x < cols) return FP8QGG_ERR_SHAPE;
   if (num_groups < 1 || num_groups > kMaxGroups) return FP8QGG_ERR_SHAPE;
   if (fmt != FP8QGG_E4M3FN && fmt != FP8QGG_E4M3FNUZ) return FP8QGG_ERR_UNSUPPORTED;
@@ -449,25 +796,33 @@ int colwise_check(const void *x, int64_t rows_total, int64_t cols, int64_t ld_x,
     return FP8QGG_ERR_ALIGN;
   if (sat_count && !aligned(sat_count, 8)) return FP8QGG_ERR_ALIGN;
   if (dev_status && !aligned(dev_status, 4)) return FP8QGG_ERR_ALIGN;
+  // the task list must stay within int32: amax + cast tasks of the tall
+  // units (each group's span is its rows plus at most 15) and whole units
   const int64_t n_ct = (cols + kCW - 1) / kCW;
-  if (int64_t(num_groups) * n_ct > INT32_MAX / 2) return FP8QGG_ERR_SHAPE;
+  const int64_t chunks = (rows_total + 16 * int64_t(num_groups)) / kChunkRows + num_groups;
+  if (n_ct * (2 * chunks + num_groups) > INT32_MAX / 2) return FP8QGG_ERR_SHAPE;
   return FP8QGG_OK;
 }
 
-// Enqueues the kernel.  *work_counter must already be zero on `stream`.
+// Enqueues the kernel.  The first colwise_scratch(...).bytes of `scratch`
+// must already be zero on `stream`.
 int colwise_launch(const void *x, int64_t rows_total, int64_t cols, int64_t ld_x,
                    const int32_t *offsets, int32_t num_groups, uint8_t *q, int64_t ld_q,
                    int layout, float *scales, int fmt, float scale_max, uint64_t *sat_count,
-                   int32_t *dev_status, uint32_t *work_counter, cudaStream_t stream) {
-  // With no rows no copy is ever issued, so the map may stay empty.
-  CUtensorMap xmap;
-  memset(&xmap, 0, sizeof xmap);
+                   int32_t *dev_status, void *scratch, cudaStream_t stream) {
+  // With no rows no copy is ever issued, so the maps may stay empty.
+  CUtensorMap xmap_box, xmap_sub;
+  memset(&xmap_box, 0, sizeof xmap_box);
+  memset(&xmap_sub, 0, sizeof xmap_sub);
   if (rows_total > 0) {
     const uint64_t dims[2] = {static_cast<uint64_t>(cols), static_cast<uint64_t>(rows_total)};
     const uint64_t strides[1] = {static_cast<uint64_t>(ld_x) * 2};
     const uint32_t box[2] = {kCW, kBoxRows};
-    if (!encode_tensor_map(&xmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(x),
-                           dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE))
+    const uint32_t subbox[2] = {kCW, kSubRows};
+    if (!encode_tensor_map(&xmap_box, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(x),
+                           dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+        !encode_tensor_map(&xmap_sub, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(x),
+                           dims, strides, subbox, CU_TENSOR_MAP_SWIZZLE_NONE))
       return FP8QGG_ERR_CUDA;
   }
 
@@ -479,15 +834,21 @@ int colwise_launch(const void *x, int64_t rows_total, int64_t cols, int64_t ld_x
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
       cudaSuccess)
     return FP8QGG_ERR_CUDA;
+  // at most this many tasks: the grid never exceeds the work
   const int64_t n_ct = (cols + kCW - 1) / kCW;
-  const int64_t units = int64_t(num_groups) * n_ct;
-  const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(units, dev.sm_count)));
+  const int64_t tasks_max =
+      n_ct * (2 * ((rows_total + 16 * int64_t(num_groups)) / kChunkRows + num_groups) + num_groups);
+  const int grid = static_cast<int>(
+      std::max<int64_t>(1, std::min<int64_t>(tasks_max, int64_t(dev.sm_count) * kBlocksPerSM)));
   const float sat_thr = saturation_threshold(fmt);
-  kern<<<grid, kColThreads, smem, stream>>>(xmap, rows_total, static_cast<int>(cols), offsets,
-                                            static_cast<int>(num_groups), q, ld_q, scales, smax,
-                                            sat_thr,
-                                            reinterpret_cast<unsigned long long *>(sat_count),
-                                            dev_status, work_counter);
+  const ColScratch sl = colwise_scratch(rows_total, cols, num_groups);
+  uint8_t *base = static_cast<uint8_t *>(scratch);
+  kern<<<grid, kColThreads, smem, stream>>>(
+      xmap_box, xmap_sub, rows_total, static_cast<int>(cols), offsets,
+      static_cast<int>(num_groups), q, ld_q, scales, smax, sat_thr,
+      reinterpret_cast<unsigned long long *>(sat_count), dev_status,
+      reinterpret_cast<uint32_t *>(base), reinterpret_cast<uint32_t *>(base + sl.arrive_off),
+      reinterpret_cast<uint32_t *>(base + sl.amax_off), static_cast<int32_t>(sl.units_cap));
   return cudaGetLastError() == cudaSuccess ? FP8QGG_OK : FP8QGG_ERR_CUDA;
 }
 
@@ -497,10 +858,7 @@ using namespace fp8qgg;
 
 extern "C" size_t fp8_quant_colwise_jagged_workspace_size(int64_t rows_total, int64_t cols,
                                                           int32_t num_groups) {
-  (void)rows_total;
-  (void)cols;
-  (void)num_groups;
-  return kColwiseScratchBytes;
+  return colwise_scratch(rows_total, cols, num_groups).bytes;
 }
 
 extern "C" int fp8_quant_colwise_jagged(const void *x, int64_t rows_total, int64_t cols,
@@ -519,8 +877,7 @@ extern "C" int fp8_quant_colwise_jagged(const void *x, int64_t rows_total, int64
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (cudaMemsetAsync(workspace, 0, need, s) != cudaSuccess) return FP8QGG_ERR_CUDA;
   return colwise_launch(x, rows_total, cols, ld_x, offsets, num_groups, q, ld_q, layout, scales,
-                        fmt, scale_max, sat_count, dev_status, static_cast<uint32_t *>(workspace),
-                        s);
+                        fmt, scale_max, sat_count, dev_status, workspace, s);
 }
 
 // ---------------------------------------------------------------------------
@@ -580,9 +937,8 @@ extern "C" int fp8_quant_colwise_jagged_noalloc(const void *x, int64_t rows_tota
   void *scratch = nullptr;
   if (!noalloc_scratch(&scratch)) return FP8QGG_ERR_CUDA;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  // the previous call's work counter must not leak into this one
+  // the previous call's counters and absmax words must not leak into this one
   if (cudaMemsetAsync(scratch, 0, need, s) != cudaSuccess) return FP8QGG_ERR_CUDA;
   return colwise_launch(x, rows_total, cols, ld_x, offsets, num_groups, q, ld_q, layout, scales,
-                        fmt, scale_max, sat_count, dev_status, static_cast<uint32_t *>(scratch),
-                        s);
+                        fmt, scale_max, sat_count, dev_status, scratch, s);
 }

@@ -54,11 +54,12 @@ __global__ void __launch_bounds__(kRowThreads)
     }
 #pragma unroll
     for (int i = 0; i < VPL; ++i) {
-      am = abs_max_bf16x2(am, v[i].x);
-      am = abs_max_bf16x2(am, v[i].y);
-      am = abs_max_bf16x2(am, v[i].z);
-      am = abs_max_bf16x2(am, v[i].w);
+      am = absmax_acc(am, v[i].x);
+      am = absmax_acc(am, v[i].y);
+      am = absmax_acc(am, v[i].z);
+      am = absmax_acc(am, v[i].w);
     }
+    am = absmax_bits(am);
     uint32_t m = max(am & 0xFFFFu, am >> 16);
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, off));

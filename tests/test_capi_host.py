@@ -74,10 +74,26 @@ def test_rowwise_argument_checks(lib):
     assert f(FAKE, 0, 64, 64, FAKE, 64, FAKE, 0, 0.0, None, None) == 0  # empty: no-op
 
 
+def test_colwise_noalloc_refuses_problems_beyond_its_scratch(lib):
+    # the size check runs on the host before any device access
+    f = lib.fp8_quant_colwise_jagged_noalloc
+    big = (98304, 8192, 64)
+    assert lib.fp8_quant_colwise_jagged_workspace_size(*big) > 2 * 1024 * 1024
+    assert f(FAKE, big[0], big[1], big[1], FAKE, big[2], FAKE, big[1], 0, FAKE, 0, 0.0, None,
+             None, None) == -2
+
+
 def test_colwise_argument_checks(lib):
     f = lib.fp8_quant_colwise_jagged
     ws = lib.fp8_quant_colwise_jagged_workspace_size(100, 64, 4)
     assert ws > 0 and ws % 256 == 0
+    # tall units (over 448 rows) each need an arrival counter and 64 absmax
+    # words; at most min(groups, rows / 432) groups can be that tall
+    g = lib.fp8_quant_colwise_jagged_workspace_size
+    assert g(431, 64, 4) == 256
+    assert g(432, 64, 4) == 256 + 256 + 256
+    assert g(98304, 2048, 64) == 256 + 2048 * 4 + 2048 * 256
+    assert g(98304, 2048, 1000) == g(98304, 2048, 227) > g(98304, 2048, 64)
 
     def call(**kw):
         a = dict(x=FAKE, rows=100, cols=64, ld_x=64, off=FAKE, e=4, q=FAKE, ld_q=64, layout=0,

@@ -208,6 +208,46 @@ def test_rowwise_scale_is_ieee_fp32_division():
         assert (s.view(np.uint32) == expect.astype(np.float32).view(np.uint32)).all()
 
 
+@pytest.mark.parametrize("fmt", [FN, FNUZ])
+def test_encode_nan_gives_a_nan_code_and_infinity_saturates(fmt):
+    """A NaN of either sign and any payload goes to a code that decodes to NaN
+    (for a positive NaN the very code torch's float8 cast gives); an infinity
+    saturates at the largest finite value like every magnitude above it (the
+    saturating-encode reading)."""
+    nans = (np.array([0x7FC00000, 0xFFC00000, 0x7F800001, 0x7FFFFFFF, 0xFF800001], np.uint32)
+            .view(np.float32))
+    for y in nans:
+        assert np.isnan(orc.decode(orc.encode(float(y), fmt), fmt))
+    pos = nans[~np.signbit(nans)]
+    assert (orc.encode_array(pos, fmt) == torch_encode(pos, fmt)).all()
+    t = orc.decode_table(fmt)
+    top = int(np.nanargmax(np.where(np.isfinite(t), t, -np.inf)))
+    low = int(np.nanargmin(np.where(np.isfinite(t), t, np.inf)))
+    assert orc.encode(float("inf"), fmt) == top and t[top] == orc.fp8_max(fmt)
+    assert orc.encode(float("-inf"), fmt) == low and t[low] == -orc.fp8_max(fmt)
+
+
+def test_absmax_skips_nan_and_keeps_infinity():
+    """A NaN in a row never decides its scale: [NaN, 2, -1] scales like [2, -1];
+    an infinite absmax gives scale fmax / inf = 0, and x * 0 of the infinity is
+    NaN, encoded as NaN."""
+    nan, inf = float("nan"), float("inf")
+    for fmt in (FN, FNUZ):
+        fmax = np.float32(orc.fp8_max(fmt))
+        _, s, _ = orc.quant_rowwise(bits_of([[nan, 2.0, -1.0, nan]]), fmt)
+        assert s[0] == fmax / np.float32(2.0)
+        _, s2, _ = orc.quant_rowwise(bits_of([[nan, nan]]), fmt)
+        assert s2[0] == fmax / np.float32(1e-12)
+        q3, s3, _ = orc.quant_rowwise(bits_of([[inf, 3.0, -5.0]]), fmt)
+        assert s3[0] == 0.0
+        nan_code = 0x80 if fmt == FNUZ else 0x7F
+        zero_neg = 0x00 if fmt == FNUZ else 0x80
+        assert list(q3[0]) == [nan_code, 0x00, zero_neg]
+        qc, sc, _ = orc.quant_colwise_jagged(bits_of([[nan, 1.0], [4.0, nan], [-8.0, 2.0]]),
+                                             np.array([3], np.int32), orc.SAME, fmt)
+        assert sc[0, 0] == fmax / np.float32(8.0) and sc[0, 1] == fmax / np.float32(2.0)
+
+
 def test_rowwise_codes_match_torch_cast_of_clamped_product():
     """Codes equal torch's cast of clamp(fp32(x * s)) (single rounding from fp32)."""
     xb = _random_rows(13, 128, 64)

@@ -19,6 +19,15 @@ def dev(t):
     return t.cuda()
 
 
+def canon(codes, fmt):
+    """Codes with the two e4m3fn NaN codes (0x7F, 0xFF) made one: the sign of a
+    NaN is not defined, so either is a correct result where the oracle has 0x7F."""
+    c = np.asarray(codes).copy()
+    if fmt == qgg.E4M3FN:
+        c[c == 0xFF] = 0x7F
+    return c
+
+
 def bits(t):
     return wl.bf16_bits(t.cpu())
 
@@ -57,10 +66,12 @@ def test_device_encoder_exhaustive_over_the_active_binades(fmt):
     y = pats.view(np.float32)
     q = qgg.fp8_cast_f32(torch.from_numpy(y).cuda(), fmt).cpu().numpy()
     assert (q == orc.encode_array(y, fmt)).all()
-    special = np.array([0.0, -0.0, np.inf, -np.inf, 448.0, -448.0, 240.0, 232.0, -232.0, 464.0],
-                       np.float32)
+    special = np.array([0.0, -0.0, np.inf, -np.inf, 448.0, -448.0, 240.0, 232.0, -232.0, 464.0,
+                        np.nan, -np.nan], np.float32)
+    special = np.concatenate([special, np.array([0x7F800001, 0xFFC00001], np.uint32)
+                              .view(np.float32)])
     q = qgg.fp8_cast_f32(torch.from_numpy(special).cuda(), fmt).cpu().numpy()
-    assert (q == orc.encode_array(special, fmt)).all()
+    assert (canon(q, fmt) == orc.encode_array(special, fmt)).all()
 
 
 @pytest.mark.parametrize("n", [1, 7, 8, 9, 1000, 4099])
@@ -129,6 +140,35 @@ def test_rowwise_every_bf16_value_at_unit_scale(fmt):
     assert (s.cpu().numpy() == 1.0).all()
 
 
+@pytest.mark.parametrize("fmt", FMTS)
+def test_rowwise_special_values_match_the_oracle(fmt):
+    """Rows holding NaNs (ignored by the absmax, like the oracle's comparison),
+    all-NaN rows, infinities (scale 0), signed zeros and subnormal-only rows."""
+    rows, cols = 12, 1408
+    g = np.random.default_rng(21 + fmt)
+    a = wl.bf16_bits(rand_bf16(6, rows, cols)).copy()
+    a[0, ::97] = 0x7FC1
+    a[1, 5::89] = 0xFFC0
+    a[2, :] = 0x7F81                                   # all NaN
+    a[3, 17] = 0x7F80                                  # +inf
+    a[4, 99] = 0xFF80                                  # -inf
+    a[5, :] = 0x8000                                   # -0
+    a[6, :] = g.integers(1, 0x80, cols).astype(np.uint16)          # subnormals
+    a[7, :] = g.integers(1, 0x80, cols).astype(np.uint16) | 0x8000
+    a[8, :] = 0x0001
+    a[9, ::2] = 0x7FC0
+    a[9, 1::2] = 0x0003
+    x = torch.from_numpy(a.view(np.int16)).view(torch.bfloat16)
+    q_ref, s_ref, _ = orc.quant_rowwise(a, fmt)
+    q, s = qgg.fp8_quant_rowwise(dev(x), fmt)
+    assert (canon(q.cpu().numpy(), fmt) == q_ref).all()
+    assert (s.cpu().numpy().view(np.uint32) == s_ref.view(np.uint32)).all()
+    sat = torch.zeros(1, dtype=torch.int64, device="cuda")  # the clamping (slow) kernel too
+    q2, s2 = qgg.fp8_quant_rowwise(dev(x), fmt, sat_count=sat)
+    assert (canon(q2.cpu().numpy(), fmt) == q_ref).all()
+    assert (s2.cpu().numpy().view(np.uint32) == s_ref.view(np.uint32)).all()
+
+
 @pytest.mark.parametrize("fmt,smax", [(qgg.E4M3FNUZ, 448.0), (qgg.E4M3FN, 240.0)])
 def test_rowwise_format_mismatch_is_counted_like_the_oracle(fmt, smax):
     x = rand_bf16(77, 64, 512, outliers=0.0)
@@ -188,6 +228,43 @@ def test_colwise_parity(sizes, cols, fmt, layout):
     assert (s.cpu().numpy().view(np.uint32) == s_ref.view(np.uint32)).all()
     assert int(sat.item()) == sat_ref == 0
     assert int(st.item()) == 0
+
+
+@pytest.mark.parametrize("fmt", FMTS)
+@pytest.mark.parametrize("layout", [qgg.LAYOUT_SAME, qgg.LAYOUT_TRANSPOSED])
+@pytest.mark.parametrize("sizes", [[100, 0, 150, 50], [900, 20]])
+def test_colwise_special_values_match_the_oracle(sizes, layout, fmt):
+    """Columns whose group absmax is a subnormal, signed zeros, infinities and
+    NaNs with several payloads: the absmax and the codes follow the oracle
+    bit for bit (the second size list takes the path that merges chunks)."""
+    m, cols = sum(sizes), 64
+    g = np.random.default_rng(sum(sizes) + layout + 7 * fmt)
+    a = wl.bf16_bits(rand_bf16(5, m, cols)).copy()
+    sub = g.integers(1, 0x80, (m, 8)).astype(np.uint16)           # positive subnormals
+    a[:, 0:8] = sub | (g.integers(0, 2, (m, 8)).astype(np.uint16) << 15)
+    a[:, 8] = 0x8000                                                # -0 everywhere
+    a[:, 9] = 0x0000
+    a[::37, 10] = 0x7F80                                            # +inf
+    a[5::41, 11] = 0xFF80                                           # -inf
+    a[::53, 12] = 0x7FC1                                            # NaN payloads
+    a[7::59, 13] = 0xFFC0
+    a[3::61, 14] = 0x7F81
+    a[:, 15] = 0x7F7F                                               # largest finite
+    a[1::2, 15] = 0x0001
+    x = torch.from_numpy(a.view(np.int16)).view(torch.bfloat16)
+    off = wl.offsets_from_sizes(sizes)
+    ld = (m + 15) // 16 * 16 if layout == qgg.LAYOUT_TRANSPOSED else cols
+    q_ref, s_ref, _ = orc.quant_colwise_jagged(a, off, layout, fmt, ld_q=ld, fill=0xAB)
+    shape = (cols, ld) if layout == qgg.LAYOUT_TRANSPOSED else (m, cols)
+    qbuf = torch.full(shape, 0xAB, dtype=torch.uint8, device="cuda")
+    for sat in (None, torch.zeros(1, dtype=torch.int64, device="cuda")):
+        qbuf.fill_(0xAB)
+        q, s = qgg.fp8_quant_colwise_jagged(dev(x), torch.from_numpy(off).cuda(), layout, fmt,
+                                            q=qbuf, sat_count=sat)
+        torch.cuda.synchronize()
+        bad = np.argwhere(canon(q.cpu().numpy(), fmt) != q_ref)
+        assert bad.size == 0, bad[:10]
+        assert (s.cpu().numpy().view(np.uint32) == s_ref.view(np.uint32)).all()
 
 
 def test_colwise_transposed_equals_transpose_of_same_layout():

@@ -76,9 +76,26 @@ def test_noalloc_matches_regular_entry_point_on_two_calls_in_a_row(layout):
         assert int(st.item()) == 0
 
 
-def test_noalloc_scratch_covers_the_problems_it_accepts():
-    """Every problem the regular entry point accepts needs no more scratch than
-    the fixed array holds, so the no-allocation entry point accepts it too."""
+def test_noalloc_rejects_problems_beyond_its_scratch_and_accepts_the_rest():
+    """Problems whose workspace exceeds the fixed array are refused with
+    FP8QGG_ERR_SHAPE before anything runs; one just inside the limit runs."""
     limit = 2 * 1024 * 1024
-    for rows, cols, groups in [(1, 8, 1), (98304, 2048, 64), (131072, 8192, 1024)]:
-        assert 0 < qgg.colwise_workspace_bytes(rows, cols, groups) <= limit
+    big = (98304, 8192, 64)
+    assert qgg.colwise_workspace_bytes(*big) > limit
+    assert 0 < qgg.colwise_workspace_bytes(98304, 2048, 64) <= limit
+    # a small stand-in with the big problem's sizes is enough for the check,
+    # which happens on the host before any device access
+    x, off = make_case(3, [800, 900], 64)
+    q = torch.empty((1700, 64), dtype=torch.uint8, device="cuda")
+    s = torch.empty((2, 64), device="cuda")
+    lib = qgg.lib()
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    rc = lib.fp8_quant_colwise_jagged_noalloc(
+        _p(x), big[0], big[1], big[1], _p(off), big[2], _p(q), big[1], qgg.LAYOUT_SAME, _p(s),
+        qgg.E4M3FN, 0.0, None, None, stream)
+    assert rc == -2
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    assert call_noalloc(x, off, qgg.LAYOUT_SAME, q, s, status=st) == 0
+    q_ref, s_ref = qgg.fp8_quant_colwise_jagged(x, off, qgg.LAYOUT_SAME)
+    torch.cuda.synchronize()
+    assert torch.equal(q, q_ref) and torch.equal(s, s_ref) and int(st.item()) == 0
