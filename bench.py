@@ -272,7 +272,7 @@ class BackwardDwStep:
         self.g = w.grad_out.cuda()
         self.x = w.x.cuda()
         self.off = torch.from_numpy(w.offsets).cuda()
-        ld = (m + 15) // 16 * 16
+        ld = (m + 127) // 128 * 128  # 128-token aligned rows for the GEMM's copies
         self.qg = torch.empty((n, ld), dtype=torch.uint8, device="cuda")
         self.qx = torch.empty((k, ld), dtype=torch.uint8, device="cuda")
         self.sg = torch.empty((e, n), dtype=torch.float32, device="cuda")

@@ -151,7 +151,9 @@ def fp8_quant_colwise_jagged(x, offsets, layout=LAYOUT_SAME, fmt=E4M3FN, scale_m
     e = offsets.numel()
     if q is None:
         if layout == LAYOUT_TRANSPOSED:
-            ld = ld_q if ld_q is not None else (rows + 15) // 16 * 16
+            # default row pitch: a multiple of 128 tokens, so that every
+            # 128-token block the contraction-jagged GEMM copies is aligned
+            ld = ld_q if ld_q is not None else (rows + 127) // 128 * 128
             q = torch.empty((cols, ld), dtype=torch.uint8, device=x.device)
         else:
             q = torch.empty((rows, cols), dtype=torch.uint8, device=x.device)

@@ -39,6 +39,10 @@ constexpr int kStages = 4;
 constexpr int kEpiWarps = 8;  // two per TMEM lane quarter: one per 128-column half
 constexpr int kEpiThreads = 32 * kEpiWarps;
 constexpr int kGemmThreads = 64 + kEpiThreads;
+// the one-CTA kernel adds a warp that masks the edge blocks of the
+// contraction-jagged mode, off the MMA warp's path
+constexpr int kMaskWarp = kGemmThreads / 32;
+constexpr int kGemm1Threads = kGemmThreads + 32;
 constexpr int kMaxGemmGroups = 1024;
 constexpr int kBandRows = 2048;  // rows per raster band of tiles (token-jagged mode)
 constexpr uint32_t kTmemCols = 512;
@@ -55,6 +59,7 @@ struct GemmSmem {
   int32_t order[kMaxGemmGroups];  // contraction-jagged mode: groups, largest first
   uint64_t full[kStages];
   uint64_t empty[kStages];
+  uint64_t ready[kStages];  // contraction-jagged mode: edge block masked
   uint64_t tfull[2];
   uint64_t tempty[2];
   uint64_t drain;
@@ -112,7 +117,7 @@ __device__ __forceinline__ TileInfo decode_tile(const Smem &sm, const GemmParams
     const int nt = static_cast<int>((p.k + BN - 1) / BN);
     ti.tm = local / nt;
     ti.tn = local % nt;
-    ti.nk = ti.gend > ti.gstart ? (ti.gend - (ti.gstart & ~15) + BK - 1) / BK : 0;
+    ti.nk = ti.gend > ti.gstart ? (ti.gend - (ti.gstart & ~(BK - 1)) + BK - 1) / BK : 0;
   }
   return ti;
 }
@@ -132,7 +137,7 @@ __device__ __forceinline__ TileInfo decode_tile_sorted(const GemmSmem &sm, const
   const int nt = static_cast<int>((p.k + BN - 1) / BN);
   ti.tm = local / nt;
   ti.tn = local % nt;
-  ti.nk = ti.gend > ti.gstart ? (ti.gend - (ti.gstart & ~15) + BK - 1) / BK : 0;
+  ti.nk = ti.gend > ti.gstart ? (ti.gend - (ti.gstart & ~(BK - 1)) + BK - 1) / BK : 0;
   return ti;
 }
 
@@ -219,36 +224,63 @@ __device__ __forceinline__ uint4 keep_mask16(int lo, int hi) {
 }
 
 // Zero the K columns outside [lo, hi) of a K-major tile written by TMA with
-// 128-byte swizzle (logical 16-byte piece j of row r sits at piece j ^ (r & 7)).
-// Only the pieces that cross lo or hi are read back; pieces wholly outside are
-// overwritten with zeros; the byte masks are built once per call.
-__device__ __forceinline__ void mask_k_tile(uint8_t *tile, int rows, int lo, int hi, int lane) {
-  const int j_lo = lo >> 4;             // piece holding column lo
-  const int j_hi = (hi + 15) >> 4;      // first piece wholly at or after hi
-  const bool part_lo = (lo & 15) != 0;
-  const bool part_hi = (hi & 15) != 0;
-  const int j_hp = hi >> 4;             // piece holding column hi (when partial)
-  const uint4 m_lo = keep_mask16(lo & 15, (j_lo == j_hp && part_hi) ? (hi & 15) : 16);
-  const uint4 m_hi = keep_mask16(0, hi & 15);
-  const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
-  for (int r = lane; r < rows; r += 32) {
-    uint8_t *row = tile + r * BK;
-    const int sw = r & 7;
-    for (int j = 0; j < j_lo; ++j) *reinterpret_cast<uint4 *>(row + ((j ^ sw) << 4)) = zero;
-    for (int j = j_hi; j < BK / 16; ++j) *reinterpret_cast<uint4 *>(row + ((j ^ sw) << 4)) = zero;
-    if (part_lo) {
-      uint4 *ptr = reinterpret_cast<uint4 *>(row + ((j_lo ^ sw) << 4));
-      uint4 v = *ptr;
-      v.x &= m_lo.x; v.y &= m_lo.y; v.z &= m_lo.z; v.w &= m_lo.w;
-      *ptr = v;
-    }
-    if (part_hi && !(part_lo && j_hp == j_lo)) {
-      uint4 *ptr = reinterpret_cast<uint4 *>(row + ((j_hp ^ sw) << 4));
-      uint4 v = *ptr;
-      v.x &= m_hi.x; v.y &= m_hi.y; v.z &= m_hi.z; v.w &= m_hi.w;
-      *ptr = v;
+// 128-byte swizzle (logical 16-byte piece j of row r sits at piece j ^ (r & 7)),
+// within the 32-column MMA steps that will be issued: those that hold a column
+// of [lo, hi), i.e. steps lo / 32 .. ceil(hi / 32) - 1.  So at most four
+// pieces per row are touched (two around lo, two around hi).  The piece masks
+// are built once per call.
+template <int ROWS>
+__device__ __forceinline__ void mask_k_edges(uint8_t *tile, int lo, int hi, int lane) {
+  // the two pieces of the step holding lo and the two of the step holding
+  // hi - 1 (the same two when lo and hi share a step: applying a piece's mask
+  // twice changes nothing)
+  const int s0 = lo >> 5, s1 = (hi - 1) >> 5;
+  int pj[4];
+  uint4 pm[4];
+  bool act[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    pj[i] = 2 * (i < 2 ? s0 : s1) + (i & 1);
+    const int a = max(lo - 16 * pj[i], 0), b = min(hi - 16 * pj[i], 16);
+    act[i] = !(a == 0 && b == 16);
+    pm[i] = b > a ? keep_mask16(a, b) : make_uint4(0u, 0u, 0u, 0u);
+  }
+  // all reads first, then all writes: the lane's ROWS / 32 rows are
+  // independent, so their shared-memory latencies overlap
+  const int sw = lane & 7;  // rows lane, lane + 32, ... share the swizzle phase
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    if (act[i]) {
+      uint4 v[ROWS / 32];
+      uint4 *ptr[ROWS / 32];
+#pragma unroll
+      for (int rr = 0; rr < ROWS / 32; ++rr) {
+        ptr[rr] = reinterpret_cast<uint4 *>(tile + (lane + 32 * rr) * BK + ((pj[i] ^ sw) << 4));
+        v[rr] = *ptr[rr];
+      }
+#pragma unroll
+      for (int rr = 0; rr < ROWS / 32; ++rr) {
+        v[rr].x &= pm[i].x; v[rr].y &= pm[i].y; v[rr].z &= pm[i].z; v[rr].w &= pm[i].w;
+        *ptr[rr] = v[rr];
+      }
     }
   }
+}
+
+// The group's columns [lo, hi) of k-block kb of a contraction-jagged tile
+// (blocks start on 128-token boundaries) and whether the block needs masking.
+struct KEdge {
+  int lo, hi;
+  bool masked;
+};
+
+__device__ __forceinline__ KEdge k_edge(const TileInfo &ti, int kb) {
+  const int32_t kx = (ti.gstart & ~(BK - 1)) + kb * BK;
+  KEdge e;
+  e.lo = max(0, ti.gstart - kx);
+  e.hi = min(BK, ti.gend - kx);
+  e.masked = (e.lo & 31) != 0 || (e.hi & 31) != 0;
+  return e;
 }
 
 // Barrier over the 128 epilogue threads that also ANDs a flag across them,
@@ -385,7 +417,7 @@ __device__ __forceinline__ void epilogue_tile(float *stg, const CUtensorMap *oma
 }
 
 template <int MODE, int OUT>
-__global__ void __launch_bounds__(kGemmThreads, 1)
+__global__ void __launch_bounds__(kGemm1Threads, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap amap,
                         const __grid_constant__ CUtensorMap bmap,
                         const __grid_constant__ CUtensorMap omap, const GemmParams p) {
@@ -400,7 +432,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     prefetch_tensormap(&omap);
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&sm.full[s], 1);
-      mbar_init(&sm.empty[s], 1);
+      // contraction-jagged mode: a stage is free once the MMAs are done AND
+      // the mask warp has passed it, so the mask warp never falls a phase
+      // behind a stage
+      mbar_init(&sm.empty[s], MODE == FP8QGG_K_JAGGED ? 2 : 1);
+      mbar_init(&sm.ready[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&sm.tfull[b], 1);
@@ -420,7 +456,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   tc_fence_after_sync();
   if constexpr (MODE == FP8QGG_K_JAGGED) {
     // rank of each group by token count (ties by index): order[rank] = group
-    for (int e = threadIdx.x; e < p.num_groups; e += kGemmThreads) {
+    for (int e = threadIdx.x; e < p.num_groups; e += kGemm1Threads) {
       const int32_t se = sm.end[e] - (e ? sm.end[e - 1] : 0);
       int rank = 0;
       for (int f = 0; f < p.num_groups; ++f) {
@@ -453,7 +489,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             tma_load_2d(sm.a[stage], &amap, &sm.full[stage], kb * BK, ti.gstart + ti.tm * BM);
             tma_load_3d(sm.b[stage], &bmap, &sm.full[stage], kb * BK, ti.tn * BN, ti.e);
           } else {
-            const int32_t kx = (ti.gstart & ~15) + kb * BK;
+            const int32_t kx = (ti.gstart & ~(BK - 1)) + kb * BK;
             tma_load_2d(sm.a[stage], &amap, &sm.full[stage], kx, ti.tm * BM);
             tma_load_2d(sm.b[stage], &bmap, &sm.full[stage], kx, ti.tn * BN);
           }
@@ -474,6 +510,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     uint32_t stage = 0, phase = 0, acc = 0, acc_phase = 0;
+    uint32_t rpar = 0;  // bit s: parity of the next phase of ready[s]
     bool ok = true;
     for (int32_t i = 0, t = tile_position<MODE>(0); t < total && ok;
          t = tile_position<MODE>(++i)) {
@@ -485,28 +522,33 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       tc_fence_after_sync();
       const uint32_t d_tmem = tmem_base + acc * BN;
       for (int kb = 0; kb < ti.nk; ++kb) {
-        if (!__all_sync(0xFFFFFFFFu, mbar_wait(&sm.full[stage], phase, abort))) {
+        int k0 = 0, k1 = BK / 32;  // 32-column MMA steps [k0, k1) of this block
+        bool masked = false;
+        if constexpr (MODE == FP8QGG_K_JAGGED) {
+          // blocks start on 128-token boundaries (aligned copies); the
+          // group's columns of this block are [lo, hi): steps wholly outside
+          // are not issued, and the mask warp zeroes the columns of the
+          // issued steps that lie outside the group
+          const KEdge ed = k_edge(ti, kb);
+          k0 = ed.lo >> 5;
+          k1 = (ed.hi + 31) >> 5;
+          masked = ed.masked;
+        }
+        const bool got = masked ? mbar_wait(&sm.ready[stage], (rpar >> stage) & 1u, abort)
+                                : mbar_wait(&sm.full[stage], phase, abort);
+        if (!__all_sync(0xFFFFFFFFu, got)) {
           ok = false;
           break;
         }
+        if (masked) rpar ^= 1u << stage;
         tc_fence_after_sync();
-        if constexpr (MODE == FP8QGG_K_JAGGED) {
-          const int32_t kx = (ti.gstart & ~15) + kb * BK;
-          const int lo = max(0, ti.gstart - kx);
-          const int hi = min(BK, ti.gend - kx);
-          if (lo > 0 || hi < BK) {
-            mask_k_tile(sm.a[stage], BM, lo, hi, lane);
-            mask_k_tile(sm.b[stage], BN, lo, hi, lane);
-            fence_proxy_async_smem();
-            __syncwarp();
-          }
-        }
         if (lane == 0) {
           const uint64_t adesc = smem_desc_k_sw128(smem_addr(sm.a[stage]));
           const uint64_t bdesc = smem_desc_k_sw128(smem_addr(sm.b[stage]));
 #pragma unroll
           for (int kk = 0; kk < BK / 32; ++kk)
-            mma_f8f6f4(d_tmem, adesc + 2 * kk, bdesc + 2 * kk, kIdesc, (kb | kk) != 0);
+            if (kk >= k0 && kk < k1)
+              mma_f8f6f4(d_tmem, adesc + 2 * kk, bdesc + 2 * kk, kIdesc, kb != 0 || kk != k0);
           mma_commit(&sm.empty[stage]);
         }
         __syncwarp();
@@ -530,6 +572,41 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       (void)mbar_wait(&sm.drain, 0, &never);
     }
     __syncwarp();
+  } else if (warp == kMaskWarp) {
+    // ------------------------------------------------------------ edge masks
+    // Follows every stage in order, and for each edge block of the
+    // contraction-jagged mode zeroes the columns outside the group once the
+    // copy has landed, then releases the block to the MMA warp.  It waits for
+    // every stage's copy and counts in every stage's release, so it is never
+    // more than one phase ahead of or behind a stage.
+    if constexpr (MODE == FP8QGG_K_JAGGED) {
+      uint32_t stage = 0, phase = 0;
+      bool ok = true;
+      for (int32_t i = 0, t = tile_position<MODE>(0); t < total && ok;
+           t = tile_position<MODE>(++i)) {
+        const TileInfo ti = tile_at<MODE>(sm, p, t);
+        for (int kb = 0; kb < ti.nk; ++kb) {
+          if (!__all_sync(0xFFFFFFFFu, mbar_wait(&sm.full[stage], phase, abort))) {
+            ok = false;
+            break;
+          }
+          const KEdge ed = k_edge(ti, kb);
+          if (ed.masked) {
+            mask_k_edges<BM>(sm.a[stage], ed.lo, ed.hi, lane);
+            mask_k_edges<BN>(sm.b[stage], ed.lo, ed.hi, lane);
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm.ready[stage]);
+          }
+          if (lane == 0) mbar_arrive(&sm.empty[stage]);
+          if (++stage == kStages) { stage = 0; phase ^= 1; }
+        }
+      }
+      if (!ok && lane == 0) {
+        *abort = 1;
+        status_or(p.status, FP8QGG_STATUS_TIMEOUT);
+      }
+    }
   } else {
     // ------------------------------------------------------------ epilogue
     const int et = threadIdx.x - 64;    // 0..255
@@ -955,6 +1032,6 @@ extern "C" int fp8_scaled_grouped_gemm(int mode, const uint8_t *a, int64_t ld_a,
   if (max_tiles > INT32_MAX) return FP8QGG_ERR_SHAPE;
   const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(max_tiles, dev.sm_count)));
 
-  kern<<<grid, kGemmThreads, smem, static_cast<cudaStream_t>(stream)>>>(amap, bmap, omap, prm);
+  kern<<<grid, kGemm1Threads, smem, static_cast<cudaStream_t>(stream)>>>(amap, bmap, omap, prm);
   return cudaGetLastError() == cudaSuccess ? FP8QGG_OK : FP8QGG_ERR_CUDA;
 }

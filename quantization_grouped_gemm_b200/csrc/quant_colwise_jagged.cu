@@ -469,6 +469,7 @@ __global__ void __launch_bounds__(kColThreads, kBlocksPerSM)
       uint32_t slot = 0, phase = 0;
       uint32_t armed = 0;  // slots whose latest phase carries a copy
       uint32_t armed_par[kSlots];
+      int pending = -1;  // cast task slot still owed its second arrival
       bool ok = true;
       // A cast task's first slot also carries the unit's absmax: the producer
       // waits (bounded) until every chunk of the unit has been counted, then
@@ -514,19 +515,32 @@ __global__ void __launch_bounds__(kColThreads, kBlocksPerSM)
           mbar_arrive(&sm.full[slot]);
           armed &= ~(1u << slot);
         }
-        bool fetched = true;
+        // A cast task's first slot waits for its second arrival until the
+        // unit's absmax is in the slot; the task's other slots are issued
+        // first, so the fetch overlaps their copies.  (They never need the
+        // first slot back: a task has fewer slots than the ring.)
         if (m.kind == kTaskCast && (m.flags & kFirstBox))
-          fetched = fetch_unit_amax(m, sm.samax[slot]);
-        // the second arrival comes even after a failed fetch, so that the
-        // phase still ends when the copy lands
-        mbar_arrive(&sm.full[slot]);
+          pending = static_cast<int>(slot);
+        else
+          mbar_arrive(&sm.full[slot]);
         if (++slot == kSlots) { slot = 0; phase ^= 1; }
+        return true;
+      };
+      // the deferred second arrival comes even after a failed fetch, so that
+      // the phase still ends when the copy lands
+      auto finish_pending = [&](const SlotMeta &m) -> bool {
+        if (pending < 0) return true;
+        const bool fetched = fetch_unit_amax(m, sm.samax[pending]);
+        mbar_arrive(&sm.full[pending]);
+        pending = -1;
         return fetched;
       };
       const int32_t total = sm.total;
+      // task indices are taken two ahead, hiding the counter's round trip
       int32_t t = static_cast<int32_t>(atomicAdd(work_counter, 1u));
+      int32_t next = static_cast<int32_t>(atomicAdd(work_counter, 1u));
       while (ok && t < total) {
-        const int32_t next = static_cast<int32_t>(atomicAdd(work_counter, 1u));
+        const int32_t next2 = static_cast<int32_t>(atomicAdd(work_counter, 1u));
         const Task tk = decode_task(sm, t, n_ct);
         SlotMeta m;
         m.c0 = tk.ct * kCW;
@@ -551,8 +565,10 @@ __global__ void __launch_bounds__(kColThreads, kBlocksPerSM)
                       (tk.kind == kTaskCast && tk.k == 0 ? kWriteScales : 0);
             ok = push(m, (m.v0 - m.y) / kSubRows, (m.v1 - 1 - m.y) / kSubRows, true);
           }
+          if (ok) ok = finish_pending(m);
         }
         t = next;
+        next = next2;
       }
       if (ok) {
         SlotMeta m{};
@@ -562,6 +578,7 @@ __global__ void __launch_bounds__(kColThreads, kBlocksPerSM)
       if (!ok) {
         *abort = 1;
         status_or(status, FP8QGG_STATUS_TIMEOUT);
+        if (pending >= 0) mbar_arrive(&sm.full[pending]);
         // copies already issued land before the block may exit
         volatile int never = 0;
         for (int s2 = 0; s2 < kSlots; ++s2)
