@@ -423,7 +423,10 @@ def run_gpu(args, world, rank, local):
 # DRAM bytes per launch of the grouped GEMM from an ncu capture of the same
 # command (dram__bytes_read.sum + dram__bytes_write.sum, profiles/); a workload
 # is absent until the current kernel has been captured on it.
-TRAFFIC = {}
+TRAFFIC = {
+    "llama3_8b_up_proj": 269102336 + 422105344,     # grouped_gemm_2sm_kernel<0>
+    "deepseek_moe16b_bwd": 400662528 + 680892928,   # grouped_gemm_kernel<1, 0>
+}
 
 
 def main():

@@ -57,22 +57,31 @@ namespace fp8qgg {
 
 constexpr int kCW = 64;                 // columns per unit: 128 bytes of bf16 per row
 constexpr int kWords = kCW / 2;         // 32-bit words (column pairs) per row
-constexpr int kSubRows = 16;            // rows of a slot owned by one consumer warp
+#ifndef FP8QGG_COLWISE_SUB_ROWS
+#define FP8QGG_COLWISE_SUB_ROWS 16
+#endif
+#ifndef FP8QGG_COLWISE_SLOTS
+#define FP8QGG_COLWISE_SLOTS 6
+#endif
+constexpr int kSubRows = FP8QGG_COLWISE_SUB_ROWS;  // rows of a slot owned by one consumer warp
 constexpr int kLaneRows = kSubRows / 4; // rows of a lane's block
 constexpr int kConsumerWarps = FP8QGG_COLWISE_CONSUMER_WARPS;  // + the producer warp
 constexpr int kBlocksPerSM = FP8QGG_COLWISE_BLOCKS_PER_SM;
 constexpr int kBoxRows = kSubRows * kConsumerWarps;  // rows per ring slot (112: 14 KB)
-constexpr int kSlots = 6;
+constexpr int kSlots = FP8QGG_COLWISE_SLOTS;
 constexpr int kChunkBoxes = FP8QGG_COLWISE_CHUNK_BOXES;
 constexpr int kChunkRows = kChunkBoxes * kBoxRows;   // rows of a whole unit / of a chunk
 constexpr int kConsumers = 32 * kConsumerWarps;
 constexpr int kColThreads = kConsumers + 32;         // + one producer warp
-constexpr int kMaxGroups = 1024;
+#ifndef FP8QGG_COLWISE_MAX_GROUPS
+#define FP8QGG_COLWISE_MAX_GROUPS 1024
+#endif
+constexpr int kMaxGroups = FP8QGG_COLWISE_MAX_GROUPS;
 constexpr uint32_t kSubBytes = kSubRows * kCW * 2;
 constexpr uint32_t kBoxBytes = kBoxRows * kCW * 2;
 constexpr int kUnitAmaxWords = kCW;     // global absmax of a tall unit: one word per column
 constexpr int kRedBufs = kSlots + 1;
-static_assert(kChunkBoxes <= kSlots, "a task's slots must fit the ring");
+static_assert(kChunkBoxes < kSlots, "a task leaves a ring slot free (its first slot may wait for the producer while the others are issued)");
 static_assert(kChunkRows % 16 == 0 && kBoxRows % 16 == 0, "boxes and chunks keep 16-row alignment");
 static_assert(kLaneRows == 4 || kLaneRows == 8, "a lane's block is 4 or 8 rows");
 
@@ -264,11 +273,23 @@ struct ColScales {
   float s[8];
 };
 
+// The four lanes that share columns 8c8 .. 8c8 + 7 (rq = 0..3) divide for two
+// of them each (columns 8c8 + 2rq, 8c8 + 2rq + 1) and swap the results, so
+// each IEEE division runs once per warp and column.  Called by all 32 lanes.
 template <int LAYOUT>
 __device__ __forceinline__ void scales_from_bits(ColScales<LAYOUT> &sc, const uint32_t (&a)[8],
-                                                 float smax) {
+                                                 float smax, int lane) {
+  const int rq = lane >> 3;
+  const uint32_t b0 = rq == 0 ? a[0] : rq == 1 ? a[2] : rq == 2 ? a[4] : a[6];
+  const uint32_t b1 = rq == 0 ? a[1] : rq == 1 ? a[3] : rq == 2 ? a[5] : a[7];
+  const float s0 = scale_from_amax(bf16_bits_to_float(b0), smax);
+  const float s1 = scale_from_amax(bf16_bits_to_float(b1), smax);
 #pragma unroll
-  for (int i = 0; i < 8; ++i) sc.s[i] = scale_from_amax(bf16_bits_to_float(a[i]), smax);
+  for (int pq = 0; pq < 4; ++pq) {
+    const int src = (lane & 7) | (pq << 3);
+    sc.s[2 * pq] = __shfl_sync(0xFFFFFFFFu, s0, src);
+    sc.s[2 * pq + 1] = __shfl_sync(0xFFFFFFFFu, s1, src);
+  }
 }
 
 template <int LAYOUT>
@@ -606,7 +627,8 @@ __global__ void __launch_bounds__(kColThreads, kBlocksPerSM)
       if (lane == 0) mbar_arrive(&sm.empty[slot]);
     };
     while (!failed) {
-      if (!mbar_wait(&sm.full[slot], phase, abort)) { failed = true; break; }
+      // every wait is decided for the whole warp, so that its lanes never part
+      if (!__all_sync(0xFFFFFFFFu, mbar_wait(&sm.full[slot], phase, abort))) { failed = true; break; }
       SlotMeta m = sm.meta[slot];
       if (m.kind == kTaskEnd) break;
       if (m.kind == kTaskWhole) {
@@ -623,7 +645,10 @@ __global__ void __launch_bounds__(kColThreads, kBlocksPerSM)
           if (b < nb && !failed) {
             if (b > 0) {
               advance();
-              if (!mbar_wait(&sm.full[slot], phase, abort)) { failed = true; continue; }
+              if (!__all_sync(0xFFFFFFFFu, mbar_wait(&sm.full[slot], phase, abort))) {
+                failed = true;
+                continue;
+              }
               m = sm.meta[slot];
             }
             ysb[b] = m.y + w * kSubRows;
@@ -649,7 +674,10 @@ __global__ void __launch_bounds__(kColThreads, kBlocksPerSM)
         if (lane < 8) *reinterpret_cast<uint4 *>(&sm.red[rbuf][w][4 * c8]) = am;
         __syncwarp();
         if (lane == 0) mbar_arrive(&sm.red_bar[rbuf]);
-        if (!mbar_wait(&sm.red_bar[rbuf], (rpar >> rbuf) & 1u, abort)) { failed = true; break; }
+        if (!__all_sync(0xFFFFFFFFu, mbar_wait(&sm.red_bar[rbuf], (rpar >> rbuf) & 1u, abort))) {
+          failed = true;
+          break;
+        }
         rpar ^= 1u << rbuf;
         uint4 mm = make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
@@ -663,7 +691,7 @@ __global__ void __launch_bounds__(kColThreads, kBlocksPerSM)
         if (++rbuf == kRedBufs) rbuf = 0;
         uint32_t a[8];
         split_bits(a, mm);
-        scales_from_bits<LAYOUT>(sc, a, smax);
+        scales_from_bits<LAYOUT>(sc, a, smax, lane);
         if (w == 0) write_scales<LAYOUT>(sc, scales, m.e, m.c0, cols, lane);
 #pragma unroll
         for (int b = 0; b < kChunkBoxes; ++b)
@@ -679,7 +707,7 @@ __global__ void __launch_bounds__(kColThreads, kBlocksPerSM)
           const uint4 x0 = *reinterpret_cast<const uint4 *>(&sm.samax[slot][8 * c8]);
           const uint4 x1 = *reinterpret_cast<const uint4 *>(&sm.samax[slot][8 * c8 + 4]);
           const uint32_t a[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
-          scales_from_bits<LAYOUT>(sc, a, smax);
+          scales_from_bits<LAYOUT>(sc, a, smax, lane);
         }
         Block blk;
         load_block(blk, sm.ring[slot] + w * kSubRows * kWords, ys, r0, r1, lane);
@@ -708,7 +736,8 @@ __global__ void __launch_bounds__(kColThreads, kBlocksPerSM)
             __syncwarp();
             if (lane == 0) mbar_arrive(&sm.red_bar[rbuf]);
             if (w == static_cast<int>(pub_turn)) {
-              if (!mbar_wait(&sm.red_bar[rbuf], (rpar >> rbuf) & 1u, abort)) {
+              if (!__all_sync(0xFFFFFFFFu,
+                              mbar_wait(&sm.red_bar[rbuf], (rpar >> rbuf) & 1u, abort))) {
                 failed = true;
                 break;
               }

@@ -337,8 +337,8 @@ def test_colwise_format_mismatch_is_counted_like_the_oracle(fmt, smax):
 
 @pytest.mark.parametrize("layout", [qgg.LAYOUT_SAME, qgg.LAYOUT_TRANSPOSED])
 def test_colwise_tall_groups_split_over_many_blocks(layout):
-    """Groups of 20k and 9k rows: 53 and 24 chunks per column tile combine their
-    partial absmax across blocks."""
+    """Groups of 20k and 9k rows: cut into 45 and 21 chunks per 64-column tile,
+    spread over the blocks, which merge their partial absmax in the workspace."""
     sizes = [20011, 3, 9000, 0, 385]
     m, cols = sum(sizes), 136
     x = rand_bf16(31, m, cols, outliers=0.001)
@@ -358,7 +358,8 @@ def test_colwise_tall_groups_split_over_many_blocks(layout):
 
 @pytest.mark.parametrize("layout", [qgg.LAYOUT_SAME, qgg.LAYOUT_TRANSPOSED])
 def test_colwise_single_group_of_seventy_thousand_rows(layout):
-    """No group-height limit: one 70,003-row group (two passes per column tile)."""
+    """No group-height limit: one 70,003-row group (157 chunks per column tile,
+    each read once for its absmax and once, from L2, for its cast)."""
     m, cols = 70003, 40
     x = rand_bf16(41, m, cols, outliers=0.0005)
     off = np.array([m], np.int32)
