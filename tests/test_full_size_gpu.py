@@ -1,0 +1,133 @@
+"""Parity at the full sizes of the benchmarked workloads, in the launch
+configuration the benchmark times (its step classes and arguments).
+
+The oracle cannot redo a whole step in seconds, so outputs are sampled where
+the method makes samples independent:
+  - rowwise: sampled rows (a row's scale and codes depend on that row only);
+  - jagged colwise: sampled columns over all rows (a column's scales and codes
+    depend on that column only), with the same offsets;
+  - grouped GEMM: sampled outputs, computed by the oracle from its OWN
+    quantisation of the rows and columns they need (never from the kernels'
+    codes), within the bound 1e-3 * sum |a||b| per element.
+Inputs are the seeded synthetic workloads the benchmark uses.
+"""
+import os
+import sys
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as orc
+from quantization_grouped_gemm_b200 import workloads as wl
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+import bench  # noqa: E402  (the step classes the benchmark times)
+
+pytestmark = pytest.mark.gpu
+
+
+def run_step(step):
+    for f in step.kernels():
+        f()
+    torch.cuda.synchronize()
+
+
+def sample(g, n, count, must=()):
+    return np.unique(np.concatenate([np.asarray(must, np.int64),
+                                     g.integers(0, n, count)])).astype(np.int64)
+
+
+def check_forward(w, seed, n_rows=40, n_cols=40, n_out=2000):
+    """Rowwise X and W on sampled rows, and the token-jagged GEMM on sampled
+    outputs, for a ForwardStep run at full size."""
+    st = bench.ForwardStep(w)
+    run_step(st)
+    g = np.random.default_rng(seed)
+    m, k = w.x.shape
+    e, n = w.w.shape[0], w.w.shape[1]
+    off = np.asarray(w.offsets, np.int64)
+    end = int(off[-1])
+    # activations: sampled rows inside the groups (group starts and ends included)
+    starts = np.concatenate([[0], off[:-1]])
+    edges = np.concatenate([starts[off > starts], off[off > starts] - 1])
+    rows = sample(g, end, n_rows, must=edges[:8])
+    qa_ref, sa_ref, _ = orc.quant_rowwise(wl.bf16_bits(w.x[torch.from_numpy(rows)]))
+    assert (st.qa[torch.from_numpy(rows).cuda()].cpu().numpy() == qa_ref).all()
+    assert (st.sa.cpu().numpy()[rows].view(np.uint32) == sa_ref.view(np.uint32)).all()
+    # weights: every expert's sampled output channels (quantised as [E*N, K] rows)
+    cols = sample(g, n, n_cols, must=[0, n - 1])
+    wsel = w.w[:, torch.from_numpy(cols), :].reshape(e * len(cols), k)
+    qb_ref, sb_ref, _ = orc.quant_rowwise(wl.bf16_bits(wsel))
+    qb = st.qb.view(e, n, k)[:, torch.from_numpy(cols).cuda(), :].reshape(e * len(cols), k)
+    assert (qb.cpu().numpy() == qb_ref).all()
+    sb = st.sb.view(e, n)[:, torch.from_numpy(cols).cuda()].reshape(-1)
+    assert (sb.cpu().numpy().view(np.uint32) == sb_ref.view(np.uint32)).all()
+    # GEMM: outputs (rows[i], cols[j]) from the oracle's operands, with the
+    # sampled rows regrouped into compact offsets (a row keeps its group)
+    grp = np.searchsorted(off, rows, side="right")
+    off_c = np.array([(grp <= ge).sum() for ge in range(e)], np.int32)
+    li = g.integers(0, len(rows), n_out)
+    lj = g.integers(0, len(cols), n_out)
+    c, b = orc.gemm_m_jagged_sample(qa_ref, sa_ref, qb_ref.reshape(e, len(cols), k),
+                                    sb_ref.reshape(e, len(cols)), off_c, li, lj)
+    out = st.out[torch.from_numpy(rows[li]).cuda(), torch.from_numpy(cols[lj]).cuda()]
+    got = out.cpu().numpy().astype(np.float64)
+    bad = np.nonzero(~(np.abs(got - c) <= b))[0]
+    assert bad.size == 0, (bad.size, got[bad[:4]], c[bad[:4]], b[bad[:4]])
+
+
+def test_llama3_8b_up_projection_full_size_sampled():
+    check_forward(wl.llama3_8b_up_proj(), 11)
+
+
+def test_deepseek_v3_local_experts_full_size_sampled():
+    check_forward(wl.deepseek_v3_local_experts(), 12)
+
+
+@pytest.mark.parametrize("m,loads", [(131072, "uniform"), (8192, "zipf")])
+def test_llama4_sweep_full_size_sampled(m, loads):
+    w = wl.llama4_sweep(m, loads)
+    check_forward(w, 13 + m)
+    # the sweep also runs under e4m3fnuz (240): rowwise of the same X, sampled rows
+    import quantization_grouped_gemm_b200 as qgg
+    q, s = qgg.fp8_quant_rowwise(w.x.cuda(), qgg.E4M3FNUZ)
+    g = np.random.default_rng(m)
+    rows = sample(g, m, 40, must=[0, m - 1])
+    q_ref, s_ref, _ = orc.quant_rowwise(wl.bf16_bits(w.x[torch.from_numpy(rows)]), orc.E4M3FNUZ)
+    assert (q[torch.from_numpy(rows).cuda()].cpu().numpy() == q_ref).all()
+    assert (s.cpu().numpy()[rows].view(np.uint32) == s_ref.view(np.uint32)).all()
+
+
+def test_deepseek_moe16b_backward_full_size_sampled():
+    """Jagged colwise + transpose of grad_out and X on sampled columns (all
+    98304 rows, 64 Zipf groups), then the contraction-jagged dW on sampled
+    (expert, row, column) outputs."""
+    w = wl.deepseek_moe_16b_backward()
+    st = bench.BackwardDwStep(w)
+    run_step(st)
+    g = np.random.default_rng(14)
+    m = st.m
+    ld = st.qg.shape[1]
+    checked = []
+    for src, q_dev, s_dev in ((w.grad_out, st.qg, st.sg), (w.x, st.qx, st.sx)):
+        cols = sample(g, src.shape[1], 24, must=[0, src.shape[1] - 1])
+        xb = wl.bf16_bits(src[:, torch.from_numpy(cols)])
+        q_ref, s_ref, _ = orc.quant_colwise_jagged(xb, w.offsets, orc.TRANSPOSED, ld_q=ld)
+        got_q = q_dev[torch.from_numpy(cols).cuda(), :m].cpu().numpy()
+        assert (got_q == q_ref[:, :m]).all()
+        got_s = s_dev[:, torch.from_numpy(cols).cuda()].cpu().numpy()
+        assert (got_s.view(np.uint32) == s_ref.view(np.uint32)).all()
+        checked.append((cols, q_ref, s_ref))
+    (ci, qa_t, sa), (cj, qb_t, sb) = checked
+    ns = 3000
+    grp = g.integers(0, st.e, ns)
+    li = g.integers(0, len(ci), ns)
+    lj = g.integers(0, len(cj), ns)
+    c, b = orc.gemm_k_jagged_sample(qa_t, sa, qb_t, sb, w.offsets, m, grp, li, lj)
+    out = st.out[torch.from_numpy(grp).cuda(), torch.from_numpy(ci[li]).cuda(),
+                 torch.from_numpy(cj[lj]).cuda()]
+    got = out.cpu().numpy().astype(np.float64)
+    bad = np.nonzero(~(np.abs(got - c) <= b))[0]
+    assert bad.size == 0, (bad.size, got[bad[:4]], c[bad[:4]], b[bad[:4]])

@@ -209,3 +209,17 @@ def test_k_jagged_every_element(sizes, n, k):
     for e, sz in enumerate(sizes):
         if sz == 0:
             assert (out[e] == 0).all()
+
+
+def test_k_jagged_group_starts_at_every_residue_of_a_block():
+    """Groups whose starts fall at every position inside a 128-token block (and
+    whose ends too), so that every pattern of skipped 32-token steps and
+    masked pieces at both edges of a block is met."""
+    g = np.random.default_rng(128)
+    sizes = [int(v) for v in g.integers(1, 300, 60)]
+    sizes[3:6] = [0, 128, 1]
+    m = sum(sizes)
+    starts = np.cumsum([0] + sizes[:-1]) % 128
+    assert len(set(starts.tolist())) > 40
+    out, ref = k_jagged_case(4242, sizes, 40, 72, ld_pad=100)
+    check_k_all(out, ref)
