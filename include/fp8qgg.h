@@ -24,13 +24,16 @@
  *    `sat_count` makes it observable.
  *  - Quantisation chain ([AIR] section "Il guadagno vero è nel movimento dei
  *    dati", first paragraph), all in one pass over HBM:
- *        amax = max |x|                       (exact)
+ *        amax = max |x|                       (exact; NaN inputs are skipped)
  *        s    = fp32(Fmax / max(amax, 1e-12)) (IEEE round to nearest)
  *        y    = clamp(fp32(x * s), -Fmax, Fmax)
  *        q    = e4m3(y)   round to nearest, ties to even, one rounding from
  *                         fp32, saturating; e4m3fnuz maps every zero to 0x00.
  *    Fmax = scale_max when scale_max > 0, else the format's largest finite.
- *    The stored scale is s (dequantise with decode(q) / s).
+ *    The stored scale is s (dequantise with decode(q) / s).  Special inputs
+ *    (the pages never meet them): an infinity saturates like any magnitude
+ *    above Fmax, an infinite amax gives s = 0, and a NaN (also inf * 0)
+ *    encodes to a NaN code (e4m3fn 0x7F or 0xFF, e4m3fnuz 0x80).
  *  - Offsets ([AIR] introduction, second paragraph: an offsets tensor routes
  *    tokens to experts): int32[num_groups] of CUMULATIVE group ends, no
  *    leading zero, device memory.  Group e spans rows [start_e, end_e) with
