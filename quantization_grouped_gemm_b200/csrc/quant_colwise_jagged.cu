@@ -10,24 +10,26 @@
 // "AMD Boosts PyTorch FP8 Training on Instinct GPUs", third paragraph.
 //
 // B200 design.  A unit is one (group, 64-column tile): 128-byte row segments.
-// One block per SM; one producer warp streams rows with TMA into a ring of six
-// 240-row slots (30 KB); each of fifteen consumer warps owns 16 rows of every
-// slot and works on them alone (absmax, cast, store straight from registers),
-// meeting the other warps only once per unit to combine the column absmax.
+// Two blocks per SM; in each, one producer warp streams rows with TMA into a
+// ring of six 112-row slots (14 KB) and each of seven consumer warps owns 16
+// rows of every slot and works on them alone (absmax, cast, store straight
+// from registers), meeting the other warps only once per task to combine the
+// column absmax.
 //
 // Work is a list of tasks taken from an atomic counter:
-//  - a unit whose rows fit in three slots (720 rows) is one "whole" task:
+//  - a unit whose rows fit in four slots (448 rows) is one "whole" task:
 //    every lane keeps its part of the rows in registers between the absmax and
 //    the cast (one HBM read) and frees each slot at once, so the ring keeps
 //    streaming;
-//  - a taller unit is cut into chunks of equal height (at most three slots),
-//    and every chunk gives two tasks:
-//    an "amax" task (column absmax of the chunk, merged into the unit's
-//    absmax in global memory with atomic max, then counted in the unit's
-//    arrival counter) and a "cast" task (waits for the unit's count, derives
-//    the scales, re-reads the chunk and casts it).  A cast task is placed in
-//    the list after every amax task of its unit and about two grid-widths of
-//    tasks later, so the chunk it re-reads is still in L2 and the wait is
+//  - a taller unit is cut into chunks of equal height (at most four slots),
+//    and every chunk gives two tasks: an "amax" task (column absmax of the
+//    chunk, merged into the unit's absmax in global memory with atomic max,
+//    then counted in the unit's arrival counter by one warp) and a "cast"
+//    task (the producer waits for the unit's count and copies the unit's
+//    absmax into the task's first slot; the consumers derive the scales,
+//    read the chunk again and cast it).  A cast task is placed in the list
+//    after every amax task of its unit and about 1.5 grid-widths of tasks
+//    later, so the chunk it reads again is still in L2 and the wait is
 //    short.  Chunks of one tall group are spread over many SMs, so a skewed
 //    routing (one expert with many tokens) keeps every SM busy.
 // Tall units come first, largest group first, then whole units largest first.
@@ -42,30 +44,32 @@
 
 namespace fp8qgg {
 
-#ifndef FP8QGG_COLWISE_CHUNK_BOXES
-#define FP8QGG_COLWISE_CHUNK_BOXES 4
-#endif
+// Build-time shape of the kernel.  The defaults are the best of the variants
+// measured on B200 (the others were slower or spilled registers).
 #ifndef FP8QGG_COLWISE_CONSUMER_WARPS
-#define FP8QGG_COLWISE_CONSUMER_WARPS 7
+#define FP8QGG_COLWISE_CONSUMER_WARPS 7   // consumer warps per block (+ the producer)
 #endif
 #ifndef FP8QGG_COLWISE_BLOCKS_PER_SM
 #define FP8QGG_COLWISE_BLOCKS_PER_SM 2
 #endif
+#ifndef FP8QGG_COLWISE_SUB_ROWS
+#define FP8QGG_COLWISE_SUB_ROWS 16        // rows of a slot owned by one consumer warp
+#endif
+#ifndef FP8QGG_COLWISE_SLOTS
+#define FP8QGG_COLWISE_SLOTS 6            // ring depth
+#endif
+#ifndef FP8QGG_COLWISE_CHUNK_BOXES
+#define FP8QGG_COLWISE_CHUNK_BOXES 4      // slots of a whole unit / of a chunk
+#endif
 #ifndef FP8QGG_COLWISE_LAG_HALF_GRIDS
-#define FP8QGG_COLWISE_LAG_HALF_GRIDS 3
+#define FP8QGG_COLWISE_LAG_HALF_GRIDS 3   // cast task lag, in half grid-widths of tasks
 #endif
 
 constexpr int kCW = 64;                 // columns per unit: 128 bytes of bf16 per row
 constexpr int kWords = kCW / 2;         // 32-bit words (column pairs) per row
-#ifndef FP8QGG_COLWISE_SUB_ROWS
-#define FP8QGG_COLWISE_SUB_ROWS 16
-#endif
-#ifndef FP8QGG_COLWISE_SLOTS
-#define FP8QGG_COLWISE_SLOTS 6
-#endif
-constexpr int kSubRows = FP8QGG_COLWISE_SUB_ROWS;  // rows of a slot owned by one consumer warp
+constexpr int kSubRows = FP8QGG_COLWISE_SUB_ROWS;
 constexpr int kLaneRows = kSubRows / 4; // rows of a lane's block
-constexpr int kConsumerWarps = FP8QGG_COLWISE_CONSUMER_WARPS;  // + the producer warp
+constexpr int kConsumerWarps = FP8QGG_COLWISE_CONSUMER_WARPS;
 constexpr int kBlocksPerSM = FP8QGG_COLWISE_BLOCKS_PER_SM;
 constexpr int kBoxRows = kSubRows * kConsumerWarps;  // rows per ring slot (112: 14 KB)
 constexpr int kSlots = FP8QGG_COLWISE_SLOTS;
@@ -73,10 +77,7 @@ constexpr int kChunkBoxes = FP8QGG_COLWISE_CHUNK_BOXES;
 constexpr int kChunkRows = kChunkBoxes * kBoxRows;   // rows of a whole unit / of a chunk
 constexpr int kConsumers = 32 * kConsumerWarps;
 constexpr int kColThreads = kConsumers + 32;         // + one producer warp
-#ifndef FP8QGG_COLWISE_MAX_GROUPS
-#define FP8QGG_COLWISE_MAX_GROUPS 1024
-#endif
-constexpr int kMaxGroups = FP8QGG_COLWISE_MAX_GROUPS;
+constexpr int kMaxGroups = 1024;
 constexpr uint32_t kSubBytes = kSubRows * kCW * 2;
 constexpr uint32_t kBoxBytes = kBoxRows * kCW * 2;
 constexpr int kUnitAmaxWords = kCW;     // global absmax of a tall unit: one word per column
