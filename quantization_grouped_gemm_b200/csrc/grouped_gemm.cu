@@ -1007,8 +1007,7 @@ extern "C" int fp8_scaled_grouped_gemm(int mode, const uint8_t *a, int64_t ld_a,
     auto kern2 = out_dtype == FP8QGG_OUT_F32 ? grouped_gemm_2sm_kernel<FP8QGG_OUT_F32>
                                              : grouped_gemm_2sm_kernel<FP8QGG_OUT_BF16>;
     const int smem2 = static_cast<int>(sizeof(Gemm2Smem)) + 1024;
-    if (cudaFuncSetAttribute(kern2, cudaFuncAttributeMaxDynamicSharedMemorySize, smem2) !=
-        cudaSuccess)
+    if (!set_max_dynamic_smem(reinterpret_cast<const void *>(kern2), smem2))
       return FP8QGG_ERR_CUDA;
     const int64_t pair_tiles =
         ((m_total + kPairRows - 1) / kPairRows + num_groups) * ((n + BN - 1) / BN);
@@ -1021,8 +1020,7 @@ extern "C" int fp8_scaled_grouped_gemm(int mode, const uint8_t *a, int64_t ld_a,
 
   GemmKernel kern = gemm_kernel(mode, out_dtype);
   const int smem = static_cast<int>(sizeof(GemmSmem)) + 1024;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
-      cudaSuccess)
+  if (!set_max_dynamic_smem(reinterpret_cast<const void *>(kern), smem))
     return FP8QGG_ERR_CUDA;
   int64_t max_tiles;
   if (mode == FP8QGG_M_JAGGED)

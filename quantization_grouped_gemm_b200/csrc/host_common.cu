@@ -53,6 +53,38 @@ bool device_info(DeviceInfo *out) {
   return true;
 }
 
+namespace {
+struct SmemAttr {
+  int device;
+  const void *kernel;
+  int bytes;
+};
+constexpr int kMaxSmemAttrs = 256;
+SmemAttr g_smem_attr[kMaxSmemAttrs];
+int g_smem_attr_n = 0;
+std::mutex g_smem_mutex;
+}  // namespace
+
+bool set_max_dynamic_smem(const void *kernel, int bytes) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  std::lock_guard<std::mutex> lock(g_smem_mutex);
+  for (int i = 0; i < g_smem_attr_n; ++i)
+    if (g_smem_attr[i].device == dev && g_smem_attr[i].kernel == kernel &&
+        g_smem_attr[i].bytes >= bytes)
+      return true;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) !=
+      cudaSuccess)
+    return false;
+  for (int i = 0; i < g_smem_attr_n; ++i)
+    if (g_smem_attr[i].device == dev && g_smem_attr[i].kernel == kernel) {
+      g_smem_attr[i].bytes = bytes;
+      return true;
+    }
+  if (g_smem_attr_n < kMaxSmemAttrs) g_smem_attr[g_smem_attr_n++] = SmemAttr{dev, kernel, bytes};
+  return true;
+}
+
 bool encode_tensor_map(CUtensorMap *map, CUtensorMapDataType dtype, uint32_t rank, void *base,
                        const uint64_t *dims, const uint64_t *strides_bytes, const uint32_t *box,
                        CUtensorMapSwizzle swizzle) {

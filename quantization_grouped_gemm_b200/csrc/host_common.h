@@ -27,6 +27,11 @@ struct DeviceInfo {
 // Properties of the current device (cached per device ordinal).
 bool device_info(DeviceInfo *out);
 
+// cudaFuncSetAttribute(kernel, MaxDynamicSharedMemorySize, bytes) on the
+// current device, once per (device, kernel): later calls with no larger size
+// skip the runtime call.
+bool set_max_dynamic_smem(const void *kernel, int bytes);
+
 // Largest finite magnitude of the encoding.
 inline float format_max(int fmt) { return fmt == FP8QGG_E4M3FNUZ ? 240.0f : 448.0f; }
 

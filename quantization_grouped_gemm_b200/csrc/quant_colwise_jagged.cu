@@ -878,8 +878,7 @@ int colwise_launch(const void *x, int64_t rows_total, int64_t cols, int64_t ld_x
   const float smax = effective_scale_max(fmt, scale_max);
   ColKernel kern = col_kernel(fmt, layout, sat_count == nullptr && smax >= format_max(fmt));
   const int smem = static_cast<int>(sizeof(ColSmem)) + 1024;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
-      cudaSuccess)
+  if (!set_max_dynamic_smem(reinterpret_cast<const void *>(kern), smem))
     return FP8QGG_ERR_CUDA;
   // at most this many tasks: the grid never exceeds the work
   const int64_t n_ct = (cols + kCW - 1) / kCW;
