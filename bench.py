@@ -207,8 +207,8 @@ def config_dict(w, Step=None):
     d = dict(workload=w.name, M=m, K=k, E=w.num_groups, fmt="e4m3fn", gemm_out="fp32")
     if w.grad_out is not None and Step is not None and Step.__name__ == "BackwardDwStep":
         d.update(N=w.grad_out.shape[1],
-                 step=("jagged column-wise quant + transpose of grad_out and of X + "
-                       "contraction-jagged FP8 grouped GEMM (dW)"))
+                 step=("jagged column-wise quant + transpose of grad_out and of X, groups "
+                       "at 128-token boundaries + contraction-jagged FP8 grouped GEMM (dW)"))
     else:
         d.update(N=w.w.shape[1],
                  step=("rowwise quant X + rowwise quant W (per expert output channel) + "
@@ -241,6 +241,7 @@ class ForwardStep:
         rows = int(np.asarray(w.offsets)[-1]) if len(w.offsets) else 0
         self.flops = 2.0 * rows * n * k
         self.names = ["quant_rowwise_x", "quant_rowwise_w", "grouped_gemm"]
+        self.launches = 3  # this library's kernels per step
         self.bytes = [m * k * 3 + m * 4, e * n * k * 3 + e * n * 4, None]
         self.host_inputs = [(self.x, w.x), (self.wt, w.w.reshape(e * n, k))]
         self.result = self.out
@@ -272,7 +273,9 @@ class BackwardDwStep:
         self.g = w.grad_out.cuda()
         self.x = w.x.cuda()
         self.off = torch.from_numpy(w.offsets).cuda()
-        ld = (m + 127) // 128 * 128  # 128-token aligned rows for the GEMM's copies
+        # padded transposed codes: every group starts on a 128-token block of
+        # the GEMM's copies and is zero-filled to the next one
+        ld = (m + 128 * e + 127) // 128 * 128
         self.qg = torch.empty((n, ld), dtype=torch.uint8, device="cuda")
         self.qx = torch.empty((k, ld), dtype=torch.uint8, device="cuda")
         self.sg = torch.empty((e, n), dtype=torch.float32, device="cuda")
@@ -284,20 +287,21 @@ class BackwardDwStep:
         self.out = torch.empty((e, n, k), dtype=torch.float32, device="cuda")
         self.flops = 2.0 * m * n * k
         self.names = ["quant_colwise_t_grad_out", "quant_colwise_t_x", "grouped_gemm"]
+        self.launches = 5  # each colwise call: the quantisation and the gap fill
         self.bytes = [m * n * 3 + e * n * 4 + e * 4, m * k * 3 + e * k * 4 + e * 4, None]
         self.host_inputs = [(self.g, w.grad_out), (self.x, w.x)]
         self.result = self.out
 
     def kernels(self):
         q = self.qgg
-        T = q.LAYOUT_TRANSPOSED
+        T = q.LAYOUT_TRANSPOSED_PADDED
         return [
             lambda: q.fp8_quant_colwise_jagged(self.g, self.off, T, q=self.qg, scales=self.sg,
                                                workspace=self.wsg),
             lambda: q.fp8_quant_colwise_jagged(self.x, self.off, T, q=self.qx, scales=self.sx,
                                                workspace=self.wsx),
-            lambda: q.fp8_scaled_grouped_gemm(q.K_JAGGED, self.qg, self.sg, self.qx, self.sx,
-                                              self.off, m_total=self.m, out=self.out),
+            lambda: q.fp8_scaled_grouped_gemm(q.K_JAGGED_PADDED, self.qg, self.sg, self.qx,
+                                              self.sx, self.off, m_total=self.m, out=self.out),
         ]
 
 
@@ -404,7 +408,7 @@ def run_gpu(args, world, rank, local):
         e2e=dict(value=flops * world / (e2e_ms * 1e-3) / 1e12, unit="TFLOP/s",
                  h2d_bytes_per_step=int(sum(h.numel() * h.element_size() for _, h in pinned)),
                  d2h_bytes_per_step=int(hout.numel() * hout.element_size()), ms_per_step=e2e_ms),
-        gpu_launches=nk * args.steps,
+        gpu_launches=st.launches * args.steps,
         clocks=clocks,
     )
     if rank == 0 and world == 1 and Step is ForwardStep and not args.no_cpu_baseline:
@@ -425,7 +429,6 @@ def run_gpu(args, world, rank, local):
 # is absent until the current kernel has been captured on it.
 TRAFFIC = {
     "llama3_8b_up_proj": 269102336 + 422105344,     # grouped_gemm_2sm_kernel<0>
-    "deepseek_moe16b_bwd": 400662528 + 680892928,   # grouped_gemm_kernel<1, 0>
 }
 
 

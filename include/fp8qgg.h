@@ -75,10 +75,12 @@ extern "C" {
 /* output layouts of the jagged column-wise quantisation */
 #define FP8QGG_LAYOUT_SAME 0
 #define FP8QGG_LAYOUT_TRANSPOSED 1
+#define FP8QGG_LAYOUT_TRANSPOSED_PADDED 2 /* transposed, groups at 128-token boundaries */
 
 /* grouped GEMM modes */
 #define FP8QGG_M_JAGGED 0 /* groups split the rows of A and of the output */
 #define FP8QGG_K_JAGGED 1 /* groups split the contraction axis */
+#define FP8QGG_K_JAGGED_PADDED 2 /* the same, on FP8QGG_LAYOUT_TRANSPOSED_PADDED operands */
 
 /* grouped GEMM output types */
 #define FP8QGG_OUT_F32 0
@@ -148,6 +150,15 @@ size_t fp8_quant_colwise_jagged_workspace_size(int64_t rows_total, int64_t cols,
  *            every output row: the contraction axis of the weight-gradient
  *            GEMM comes out contiguous, with no separate transposed copy
  *            (the pages remove a .t().contiguous().t() round trip).
+ *            FP8QGG_LAYOUT_TRANSPOSED_PADDED: as TRANSPOSED, but group e
+ *            starts at column P_e = sum_{j<e} round_up(size_j, 128) of every
+ *            output row and is followed by zero codes up to P_e +
+ *            round_up(size_e, 128): the weight-gradient GEMM then meets no
+ *            group edge inside a 128-token block (mode
+ *            FP8QGG_K_JAGGED_PADDED).  ld_q >= rows_total + 128 * num_groups,
+ *            ld_q % 16 == 0; columns past the last padded group are not
+ *            written.  This layout is this library's choice: the pages do
+ *            not describe one.
  *   scales   fp32 [num_groups, cols]; an empty group gets Fmax / 1e-12 in
  *            every column and no codes.
  *   workspace, workspace_bytes: device scratch of at least
@@ -227,6 +238,10 @@ int fp8_quant_colwise_jagged_noalloc(const void *x, int64_t rows_total, int64_t 
  *   out      [num_groups, n, ld_out] with group stride out_group_stride
  *            (>= n * ld_out); an empty group's matrix is written as zeros.
  *   b_group_stride unused.
+ * mode FP8QGG_K_JAGGED_PADDED: the same product on operands in
+ * FP8QGG_LAYOUT_TRANSPOSED_PADDED (group e at tokens [P_e, P_e +
+ * round_up(size_e, 128)), zeros past its size); m_total is the unpadded token
+ * count, ld_a and ld_b >= m_total + 128 * num_groups.
  * Requirements: fmt == FP8QGG_E4M3FN (the tensor cores have no e4m3fnuz
  * input); m_total >= 0, n >= 1, k >= 1; num_groups in [1, 1024];
  * a, b 16-byte aligned; ld_a, ld_b, b_group_stride multiples of 16;

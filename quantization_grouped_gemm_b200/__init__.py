@@ -17,8 +17,10 @@ E4M3FN = 0
 E4M3FNUZ = 1
 LAYOUT_SAME = 0
 LAYOUT_TRANSPOSED = 1
+LAYOUT_TRANSPOSED_PADDED = 2
 M_JAGGED = 0
 K_JAGGED = 1
+K_JAGGED_PADDED = 2
 OUT_F32 = 0
 OUT_BF16 = 1
 STATUS_BAD_OFFSETS = 1
@@ -142,8 +144,8 @@ def fp8_quant_colwise_jagged(x, offsets, layout=LAYOUT_SAME, fmt=E4M3FN, scale_m
     """Per-(group, column) quantisation of a bf16 [rows_total, cols] CUDA tensor.
 
     offsets: int32 CUDA tensor of cumulative group ends.  Returns (q, scales)
-    with q [rows_total, cols] (SAME) or [cols, ld_q] (TRANSPOSED), scales
-    fp32 [num_groups, cols]."""
+    with q [rows_total, cols] (SAME) or [cols, ld_q] (TRANSPOSED and
+    TRANSPOSED_PADDED), scales fp32 [num_groups, cols]."""
     _need_cuda(x, offsets)
     assert x.dtype == torch.bfloat16 and x.dim() == 2
     assert offsets.dtype == torch.int32
@@ -154,6 +156,10 @@ def fp8_quant_colwise_jagged(x, offsets, layout=LAYOUT_SAME, fmt=E4M3FN, scale_m
             # default row pitch: a multiple of 128 tokens, so that every
             # 128-token block the contraction-jagged GEMM copies is aligned
             ld = ld_q if ld_q is not None else (rows + 127) // 128 * 128
+            q = torch.empty((cols, ld), dtype=torch.uint8, device=x.device)
+        elif layout == LAYOUT_TRANSPOSED_PADDED:
+            # room for every group rounded up to 128 tokens
+            ld = ld_q if ld_q is not None else (rows + 128 * e + 127) // 128 * 128
             q = torch.empty((cols, ld), dtype=torch.uint8, device=x.device)
         else:
             q = torch.empty((rows, cols), dtype=torch.uint8, device=x.device)
@@ -179,7 +185,9 @@ def fp8_scaled_grouped_gemm(mode, a, scale_a, b, scale_b, offsets, m_total=None,
     M_JAGGED: a uint8 [m_total, K], scale_a [m_total], b uint8 [E, N, K] (or any
     layout with b_group_stride), scale_b [E, N] -> out [m_total, N].
     K_JAGGED: a uint8 [N, ld_a], b uint8 [K, ld_b] (token axis contiguous),
-    scale_a [E, N], scale_b [E, K], m_total tokens -> out [E, N, K]."""
+    scale_a [E, N], scale_b [E, K], m_total tokens -> out [E, N, K].
+    K_JAGGED_PADDED: as K_JAGGED, on operands in LAYOUT_TRANSPOSED_PADDED;
+    m_total is the unpadded token count."""
     _need_cuda(a, scale_a, b, scale_b, offsets)
     assert a.dtype == torch.uint8 and b.dtype == torch.uint8 and offsets.dtype == torch.int32
     e = offsets.numel()

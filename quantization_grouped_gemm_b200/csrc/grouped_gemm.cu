@@ -79,6 +79,7 @@ struct GemmParams {
   int64_t ld_out;
   int64_t out_gs;  // output group stride (contraction-jagged mode)
   int32_t *status;
+  int padded;      // contraction-jagged operands with groups at 128-token boundaries
 };
 
 struct TileInfo {
@@ -170,7 +171,7 @@ __device__ void build_tile_table(Smem &sm, const GemmParams &p, int lane) {
   const int32_t nt_m = static_cast<int32_t>((p.n + BN - 1) / BN);
   const int32_t tiles_k_mode =
       static_cast<int32_t>(((p.n + BM - 1) / BM) * ((p.k + BN - 1) / BN));
-  int32_t carry_end = 0, carry_tiles = 0;
+  int32_t carry_end = 0, carry_tiles = 0, carry_pend = 0;
   bool bad = false;
   for (int base = 0; base < p.num_groups; base += 32) {
     const int e = base + lane;
@@ -195,8 +196,22 @@ __device__ void build_tile_table(Smem &sm, const GemmParams &p, int lane) {
       const int32_t o = __shfl_up_sync(0xFFFFFFFFu, tiles, d);
       if (lane >= d) tiles += o;
     }
+    // padded contraction-jagged operands: group e's tokens sit at
+    // [P_e, P_e + round_up(size_e, BK)), P_e the earlier groups' padded sizes
+    int32_t pend = endv;
+    if constexpr (MODE == FP8QGG_K_JAGGED) {
+      if (p.padded) {
+        int32_t psz = e < p.num_groups ? (endv - prev + BK - 1) & ~(BK - 1) : 0;
+        for (int d = 1; d < 32; d <<= 1) {
+          const int32_t o = __shfl_up_sync(0xFFFFFFFFu, psz, d);
+          if (lane >= d) psz += o;
+        }
+        pend = carry_pend + psz;
+        carry_pend += __shfl_sync(0xFFFFFFFFu, psz, 31);
+      }
+    }
     if (e < p.num_groups) {
-      sm.end[e] = endv;
+      sm.end[e] = pend;
       sm.tile_prefix[e + 1] = carry_tiles + tiles;
     }
     carry_end = __shfl_sync(0xFFFFFFFFu, endv, 31);
@@ -890,7 +905,10 @@ extern "C" int fp8_scaled_grouped_gemm(int mode, const uint8_t *a, int64_t ld_a,
                                        int64_t m_total, int64_t n, int64_t k, void *out,
                                        int64_t ld_out, int64_t out_group_stride, int out_dtype,
                                        int fmt, int32_t *dev_status, void *stream) {
-  if (mode != FP8QGG_M_JAGGED && mode != FP8QGG_K_JAGGED) return FP8QGG_ERR_UNSUPPORTED;
+  if (mode != FP8QGG_M_JAGGED && mode != FP8QGG_K_JAGGED && mode != FP8QGG_K_JAGGED_PADDED)
+    return FP8QGG_ERR_UNSUPPORTED;
+  const bool padded = mode == FP8QGG_K_JAGGED_PADDED;
+  if (padded) mode = FP8QGG_K_JAGGED;
   if (out_dtype != FP8QGG_OUT_F32 && out_dtype != FP8QGG_OUT_BF16) return FP8QGG_ERR_UNSUPPORTED;
   if (fmt != FP8QGG_E4M3FN) return FP8QGG_ERR_UNSUPPORTED;
   if (num_groups < 1 || num_groups > kMaxGemmGroups) return FP8QGG_ERR_SHAPE;
@@ -902,7 +920,10 @@ extern "C" int fp8_scaled_grouped_gemm(int mode, const uint8_t *a, int64_t ld_a,
     if (ld_a < k || ld_b < k || ld_out < n || scale_b_group_stride < n) return FP8QGG_ERR_SHAPE;
     if (num_groups > 1 && b_group_stride < n * ld_b) return FP8QGG_ERR_SHAPE;
   } else {
-    if (ld_a < m_total || ld_b < m_total || ld_out < k) return FP8QGG_ERR_SHAPE;
+    // padded operands hold up to 128 * num_groups more token columns
+    const int64_t tok = m_total + (padded ? int64_t(BK) * num_groups : 0);
+    if (tok > INT32_MAX - 2 * BK) return FP8QGG_ERR_SHAPE;
+    if (ld_a < tok || ld_b < tok || ld_out < k) return FP8QGG_ERR_SHAPE;
     if (scale_a_group_stride < n || scale_b_group_stride < k) return FP8QGG_ERR_SHAPE;
     if (num_groups > 1 && out_group_stride < n * ld_out) return FP8QGG_ERR_SHAPE;
   }
@@ -934,7 +955,8 @@ extern "C" int fp8_scaled_grouped_gemm(int mode, const uint8_t *a, int64_t ld_a,
                            bdims, bstr, bbox, CU_TENSOR_MAP_SWIZZLE_128B))
       return FP8QGG_ERR_CUDA;
   } else {
-    const uint64_t mt = static_cast<uint64_t>(std::max<int64_t>(m_total, 1));
+    const uint64_t mt = static_cast<uint64_t>(
+        std::max<int64_t>(m_total + (padded ? int64_t(BK) * num_groups : 0), 1));
     const uint64_t adims[2] = {mt, static_cast<uint64_t>(n)};
     const uint64_t astr[1] = {static_cast<uint64_t>(ld_a)};
     const uint64_t bdims[2] = {mt, static_cast<uint64_t>(k)};
@@ -990,6 +1012,7 @@ extern "C" int fp8_scaled_grouped_gemm(int mode, const uint8_t *a, int64_t ld_a,
   prm.ld_out = ld_out;
   prm.out_gs = out_group_stride;
   prm.status = dev_status;
+  prm.padded = padded ? 1 : 0;
 
   // Token-jagged problems whose groups average at least one 256-row pair
   // tile run on SM pairs (half the operand stream per SM); smaller groups

@@ -113,6 +113,7 @@ struct ColSmem {
   int32_t end[kMaxGroups];
   int32_t order[kMaxGroups];                 // groups by row span, largest first
   int32_t prefix[kMaxGroups];                // tall groups: first amax task of the group
+  int32_t pstart[kMaxGroups];                // padded transposed layout: group's first token
   uint64_t full[kSlots];
   uint64_t empty[kSlots];
   uint64_t red_bar[kRedBufs];
@@ -155,12 +156,32 @@ __device__ __forceinline__ int32_t group_start(const ColSmem &sm, int e) {
   return e ? sm.end[e - 1] : 0;
 }
 
-// Rows a group's units cover: from the 16-aligned row at or below its first
-// row to its end (0 for an empty group).
-__device__ __forceinline__ int32_t group_span(const ColSmem &sm, int e) {
+// Rows a group's units cover: from their first row (the group's first row
+// rounded down with bmask: to 16 rows for the plain layouts, not at all for
+// the padded transposed one) to the group's end (0 for an empty group).
+__device__ __forceinline__ int32_t group_span(const ColSmem &sm, int e, int32_t bmask) {
   const int32_t s = group_start(sm, e);
   const int32_t g = sm.end[e];
-  return g > s ? g - (s & ~15) : 0;
+  return g > s ? g - (s & bmask) : 0;
+}
+
+// Base-row mask of a layout: the padded transposed layout starts a group's
+// units on its first row, so that token runs stay 4-byte aligned relative to
+// the group's 128-aligned padded start; the others on the 16-aligned row.
+template <int LAYOUT>
+constexpr int32_t base_mask() {
+  return LAYOUT == FP8QGG_LAYOUT_TRANSPOSED_PADDED ? ~0 : ~15;
+}
+
+// Offset from a row of group e to its token in the codes: the padded
+// transposed layout moves the group to its 128-aligned first token (never
+// below its first row, as every padded size is at least the size).
+template <int LAYOUT>
+__device__ __forceinline__ int64_t token_shift(const ColSmem &sm, int e) {
+  if constexpr (LAYOUT == FP8QGG_LAYOUT_TRANSPOSED_PADDED)
+    return static_cast<int64_t>(sm.pstart[e]) - group_start(sm, e);
+  else
+    return 0;
 }
 
 struct Task {
@@ -173,7 +194,7 @@ struct Task {
 // stream B (same order); the list opens with L = min(lag, |A|) tasks of A,
 // then alternates A, B, and ends with the rest of B, so cast task j follows
 // amax task j + L.  Whole units follow.
-__device__ Task decode_task(const ColSmem &sm, int32_t t, int n_ct) {
+__device__ Task decode_task(const ColSmem &sm, int32_t t, int n_ct, int32_t bmask) {
   Task r;
   const int32_t NA = sm.na;
   if (t < 2 * NA) {
@@ -199,7 +220,7 @@ __device__ Task decode_task(const ColSmem &sm, int32_t t, int n_ct) {
     r.e = sm.order[lo];
     r.gstart = group_start(sm, r.e);
     const int32_t gend = sm.end[r.e];
-    const int32_t a = r.gstart & ~15;
+    const int32_t a = r.gstart & bmask;
     r.C = (gend - a + kChunkRows - 1) / kChunkRows;
     // chunks of equal height (a multiple of 16, at most kChunkRows)
     const int32_t ch = ((gend - a + r.C - 1) / r.C + 15) & ~15;
@@ -217,7 +238,7 @@ __device__ Task decode_task(const ColSmem &sm, int32_t t, int n_ct) {
     r.e = sm.order[i];
     r.gstart = group_start(sm, r.e);
     const int32_t gend = sm.end[r.e];
-    r.r0 = r.gstart & ~15;
+    r.r0 = r.gstart & bmask;
     r.r1 = gend > r.gstart ? gend : r.r0;
     r.k = 0;
     r.C = 1;
@@ -438,10 +459,10 @@ __global__ void __launch_bounds__(kColThreads, kBlocksPerSM)
   __syncthreads();
   // groups ranked by row span, largest first (ties by index)
   for (int e = tid; e < num_groups; e += kColThreads) {
-    const int32_t se = group_span(sm, e);
+    const int32_t se = group_span(sm, e, base_mask<LAYOUT>());
     int rank = 0;
     for (int f = 0; f < num_groups; ++f) {
-      const int32_t sf = group_span(sm, f);
+      const int32_t sf = group_span(sm, f, base_mask<LAYOUT>());
       rank += (sf > se) || (sf == se && f < e);
     }
     sm.order[rank] = e;
@@ -456,7 +477,7 @@ __global__ void __launch_bounds__(kColThreads, kBlocksPerSM)
       const int i = base + lane;
       int32_t c = 0;
       if (i < num_groups) {
-        const int32_t sp = group_span(sm, sm.order[i]);
+        const int32_t sp = group_span(sm, sm.order[i], base_mask<LAYOUT>());
         if (sp > kChunkRows) c = n_ct * ((sp + kChunkRows - 1) / kChunkRows);
       }
       int32_t incl = c;
@@ -472,9 +493,25 @@ __global__ void __launch_bounds__(kColThreads, kBlocksPerSM)
       sm.n_tall = n_tall;
       sm.na = carry;
       const int32_t c_max =
-          n_tall ? (group_span(sm, sm.order[0]) + kChunkRows - 1) / kChunkRows : 0;
+          n_tall ? (group_span(sm, sm.order[0], base_mask<LAYOUT>()) + kChunkRows - 1) / kChunkRows : 0;
       sm.lag = max(FP8QGG_COLWISE_LAG_HALF_GRIDS * static_cast<int32_t>(gridDim.x) / 2, c_max);
       sm.total = 2 * carry + (num_groups - n_tall) * n_ct;
+    }
+    if constexpr (LAYOUT == FP8QGG_LAYOUT_TRANSPOSED_PADDED) {
+      // first token of each group: the previous groups' sizes rounded up to 128
+      int32_t pc = 0;
+      for (int base = 0; base < num_groups; base += 32) {
+        const int e = base + lane;
+        const int32_t sz = e < num_groups ? sm.end[e] - group_start(sm, e) : 0;
+        const int32_t ps = (sz + 127) & ~127;
+        int32_t incl = ps;
+        for (int d = 1; d < 32; d <<= 1) {
+          const int32_t o = __shfl_up_sync(0xFFFFFFFFu, incl, d);
+          if (lane >= d) incl += o;
+        }
+        if (e < num_groups) sm.pstart[e] = pc + incl - ps;
+        pc += __shfl_sync(0xFFFFFFFFu, incl, 31);
+      }
     }
   }
   __syncthreads();
@@ -563,7 +600,7 @@ __global__ void __launch_bounds__(kColThreads, kBlocksPerSM)
       int32_t next = static_cast<int32_t>(atomicAdd(work_counter, 1u));
       while (ok && t < total) {
         const int32_t next2 = static_cast<int32_t>(atomicAdd(work_counter, 1u));
-        const Task tk = decode_task(sm, t, n_ct);
+        const Task tk = decode_task(sm, t, n_ct, base_mask<LAYOUT>());
         SlotMeta m;
         m.c0 = tk.ct * kCW;
         m.e = tk.e;
@@ -694,10 +731,11 @@ __global__ void __launch_bounds__(kColThreads, kBlocksPerSM)
         split_bits(a, mm);
         scales_from_bits<LAYOUT>(sc, a, smax, lane);
         if (w == 0) write_scales<LAYOUT>(sc, scales, m.e, m.c0, cols, lane);
+        uint8_t *const qe = q + token_shift<LAYOUT>(sm, m.e);
 #pragma unroll
         for (int b = 0; b < kChunkBoxes; ++b)
           if (b < nb)
-            cast_block<FMT, LAYOUT, FAST>(blk[b], ysb[b], r0b[b], r1b[b], m.c0, cols, q, ld_q, sc,
+            cast_block<FMT, LAYOUT, FAST>(blk[b], ysb[b], r0b[b], r1b[b], m.c0, cols, qe, ld_q, sc,
                                           smax, sat_thr, sat, lane);
       } else {
         const int32_t ys = m.y + w * kSubRows;
@@ -716,8 +754,9 @@ __global__ void __launch_bounds__(kColThreads, kBlocksPerSM)
         if (m.kind == kTaskCast) {
           if ((m.flags & kFirstBox) && (m.flags & kWriteScales) && w == 0)
             write_scales<LAYOUT>(sc, scales, m.e, m.c0, cols, lane);
-          cast_block<FMT, LAYOUT, FAST>(blk, ys, r0, r1, m.c0, cols, q, ld_q, sc, smax, sat_thr,
-                                        sat, lane);
+          cast_block<FMT, LAYOUT, FAST>(blk, ys, r0, r1, m.c0, cols,
+                                        q + token_shift<LAYOUT>(sm, m.e), ld_q, sc, smax,
+                                        sat_thr, sat, lane);
         } else {
           uint4 &am = chunk_am;
           amax_block(am, blk);
@@ -773,6 +812,61 @@ __global__ void __launch_bounds__(kColThreads, kBlocksPerSM)
   }
 }
 
+// Zero codes of the padded transposed layout: for every group e and column c,
+// tokens [P_e + size_e, P_e + round_up(size_e, 128)) of row c of the codes.
+// The run ends on a 16-byte boundary (P_e is a multiple of 128 and ld_q of
+// 16), so it takes byte stores up to the first boundary, then 16-byte stores.
+// Every block rebuilds the clamped ends and padded starts (warp 0 scans).
+__global__ void __launch_bounds__(256) pad_transposed_kernel(const int32_t *__restrict__ offsets,
+                                                             int num_groups, int64_t rows_total,
+                                                             int cols, uint8_t *__restrict__ q,
+                                                             int64_t ld_q) {
+  __shared__ int32_t s_start[kMaxGroups], s_size[kMaxGroups];
+  if (threadIdx.x < 32) {
+    const int lane = threadIdx.x;
+    const int32_t R = static_cast<int32_t>(rows_total);
+    int32_t carry_end = 0, carry_pad = 0;
+    for (int base = 0; base < num_groups; base += 32) {
+      const int e = base + lane;
+      int32_t run = e < num_groups ? max(__ldg(offsets + e), 0) : 0;
+      for (int d = 1; d < 32; d <<= 1) {
+        const int32_t o = __shfl_up_sync(0xFFFFFFFFu, run, d);
+        if (lane >= d) run = max(run, o);
+      }
+      const int32_t endv = min(R, max(carry_end, run));
+      int32_t prev = __shfl_up_sync(0xFFFFFFFFu, endv, 1);
+      if (lane == 0) prev = carry_end;
+      const int32_t sz = e < num_groups ? endv - prev : 0;
+      const int32_t ps = (sz + 127) & ~127;
+      int32_t incl = ps;
+      for (int d = 1; d < 32; d <<= 1) {
+        const int32_t o = __shfl_up_sync(0xFFFFFFFFu, incl, d);
+        if (lane >= d) incl += o;
+      }
+      if (e < num_groups) {
+        s_start[e] = carry_pad + incl - ps;
+        s_size[e] = sz;
+      }
+      carry_end = __shfl_sync(0xFFFFFFFFu, endv, 31);
+      carry_pad += __shfl_sync(0xFFFFFFFFu, incl, 31);
+    }
+  }
+  __syncthreads();
+  const int64_t pairs = static_cast<int64_t>(num_groups) * cols;
+  for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < pairs;
+       i += int64_t(gridDim.x) * blockDim.x) {
+    const int e = static_cast<int>(i / cols);
+    const int64_t c = i - int64_t(e) * cols;
+    const int32_t sz = s_size[e];
+    const int64_t lo = s_start[e] + int64_t(sz);
+    const int64_t hi = s_start[e] + int64_t((sz + 127) & ~127);
+    uint8_t *row = q + c * ld_q;
+    const int64_t mid = min(hi, (lo + 15) & ~int64_t(15));
+    for (int64_t t = lo; t < mid; ++t) row[t] = 0;
+    for (int64_t t = mid; t < hi; t += 16) *reinterpret_cast<uint4 *>(row + t) = make_uint4(0, 0, 0, 0);
+  }
+}
+
 namespace {
 
 using ColKernel = void (*)(const CUtensorMap, const CUtensorMap, int64_t, int, const int32_t *,
@@ -783,7 +877,9 @@ template <int FMT, bool FAST>
 ColKernel col_kernel_fmt(int layout) {
   return layout == FP8QGG_LAYOUT_SAME
              ? quant_colwise_jagged_kernel<FMT, FP8QGG_LAYOUT_SAME, FAST>
-             : quant_colwise_jagged_kernel<FMT, FP8QGG_LAYOUT_TRANSPOSED, FAST>;
+         : layout == FP8QGG_LAYOUT_TRANSPOSED
+             ? quant_colwise_jagged_kernel<FMT, FP8QGG_LAYOUT_TRANSPOSED, FAST>
+             : quant_colwise_jagged_kernel<FMT, FP8QGG_LAYOUT_TRANSPOSED_PADDED, FAST>;
 }
 
 // The fast kernels skip the clamp and the saturation count (see quant_pair_fast).
@@ -828,16 +924,21 @@ int colwise_check(const void *x, int64_t rows_total, int64_t cols, int64_t ld_x,
   if (cols < 1 || cols > INT32_MAX / 2 || ld_x < cols) return FP8QGG_ERR_SHAPE;
   if (num_groups < 1 || num_groups > kMaxGroups) return FP8QGG_ERR_SHAPE;
   if (fmt != FP8QGG_E4M3FN && fmt != FP8QGG_E4M3FNUZ) return FP8QGG_ERR_UNSUPPORTED;
-  if (layout != FP8QGG_LAYOUT_SAME && layout != FP8QGG_LAYOUT_TRANSPOSED)
+  if (layout != FP8QGG_LAYOUT_SAME && layout != FP8QGG_LAYOUT_TRANSPOSED &&
+      layout != FP8QGG_LAYOUT_TRANSPOSED_PADDED)
     return FP8QGG_ERR_UNSUPPORTED;
   if (!(scale_max >= 0.0f) || scale_max > 3.0e38f) return FP8QGG_ERR_UNSUPPORTED;
   if (layout == FP8QGG_LAYOUT_SAME && ld_q < cols) return FP8QGG_ERR_SHAPE;
   if (layout == FP8QGG_LAYOUT_TRANSPOSED && ld_q < rows_total) return FP8QGG_ERR_SHAPE;
+  if (layout == FP8QGG_LAYOUT_TRANSPOSED_PADDED &&
+      (ld_q < rows_total + 128 * int64_t(num_groups) ||
+       rows_total + 128 * int64_t(num_groups) > INT32_MAX - 4 * kChunkRows))
+    return FP8QGG_ERR_SHAPE;
   if (!offsets || !scales) return FP8QGG_ERR_NULL;
   if (rows_total > 0 && (!x || !q)) return FP8QGG_ERR_NULL;
   if (cols % 8 || ld_x % 8) return FP8QGG_ERR_ALIGN;
   if (layout == FP8QGG_LAYOUT_SAME && ld_q % 8) return FP8QGG_ERR_ALIGN;
-  if (layout == FP8QGG_LAYOUT_TRANSPOSED && ld_q % 16) return FP8QGG_ERR_ALIGN;
+  if (layout != FP8QGG_LAYOUT_SAME && ld_q % 16) return FP8QGG_ERR_ALIGN;
   if ((x && !aligned(x, 16)) || (q && !aligned(q, 16)) || !aligned(scales, 4) ||
       !aligned(offsets, 4))
     return FP8QGG_ERR_ALIGN;
@@ -895,6 +996,13 @@ int colwise_launch(const void *x, int64_t rows_total, int64_t cols, int64_t ld_x
       reinterpret_cast<unsigned long long *>(sat_count), dev_status,
       reinterpret_cast<uint32_t *>(base), reinterpret_cast<uint32_t *>(base + sl.arrive_off),
       reinterpret_cast<uint32_t *>(base + sl.amax_off), static_cast<int32_t>(sl.units_cap));
+  if (layout == FP8QGG_LAYOUT_TRANSPOSED_PADDED && rows_total > 0) {
+    const int64_t pairs = int64_t(num_groups) * cols;
+    const int pgrid = static_cast<int>(
+        std::max<int64_t>(1, std::min<int64_t>((pairs + 255) / 256, int64_t(dev.sm_count) * 4)));
+    pad_transposed_kernel<<<pgrid, 256, 0, stream>>>(offsets, static_cast<int>(num_groups),
+                                                     rows_total, static_cast<int>(cols), q, ld_q);
+  }
   return cudaGetLastError() == cudaSuccess ? FP8QGG_OK : FP8QGG_ERR_CUDA;
 }
 

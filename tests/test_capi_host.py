@@ -112,6 +112,10 @@ def test_colwise_argument_checks(lib):
     assert call(layout=1, ld_q=64) == -2       # transposed needs ld_q >= rows_total
     assert call(layout=1, ld_q=104) == -3      # and ld_q % 16 == 0
     assert call(cols=60, ld_x=64) == -3
+    # padded transposed: room for every group rounded up to 128 tokens
+    assert call(layout=2, ld_q=112) == -2
+    assert call(layout=2, ld_q=100 + 128 * 4 - 16) == -2
+    assert call(layout=2, ld_q=100 + 128 * 4 + 8) == -3
     assert call(layout=5) == -4
     assert call(fmt=3) == -4
 
@@ -128,7 +132,7 @@ def test_gemm_argument_checks(lib):
                  a["ogs"], a["odt"], a["fmt"], None, None)
 
     assert call(fmt=1) == -4           # no e4m3fnuz input on the tensor cores
-    assert call(mode=2) == -4
+    assert call(mode=3) == -4
     assert call(odt=3) == -4
     assert call(e=0) == -2
     assert call(e=1025) == -2
@@ -141,6 +145,9 @@ def test_gemm_argument_checks(lib):
     # K-jagged: token axis is the leading dimension of both operands
     assert call(mode=1, lda=64, ldb=64, m=100, sas=32, sbs=64, ldo=64, ogs=32 * 64) == -2
     assert call(mode=1, lda=112, ldb=112, m=100, sas=32, sbs=64, ldo=64, ogs=16) == -2
+    # padded operands: the token axis holds up to 128 more columns per group
+    assert call(mode=2, lda=112, ldb=112, m=100, sas=32, sbs=64, ldo=64, ogs=32 * 64) == -2
+    assert call(mode=2, lda=352, ldb=368, m=100, sas=32, sbs=64, ldo=64, ogs=32 * 64) == -2
 
 
 def test_cast_argument_checks(lib):

@@ -111,12 +111,24 @@ def test_deepseek_moe16b_backward_full_size_sampled():
     m = st.m
     ld = st.qg.shape[1]
     checked = []
+    # the step writes the padded transposed layout: group e at tokens
+    # [P_e, P_e + size_e), P_e the earlier sizes rounded up to 128, zero codes
+    # up to the next multiple of 128
+    starts = np.concatenate([[0], w.offsets[:-1]]).astype(np.int64)
+    sizes = w.offsets.astype(np.int64) - starts
+    padded = (sizes + 127) // 128 * 128
+    p_start = np.concatenate([[0], np.cumsum(padded)[:-1]])
+    p_end = int(p_start[-1] + padded[-1])
+    assert ld >= p_end
     for src, q_dev, s_dev in ((w.grad_out, st.qg, st.sg), (w.x, st.qx, st.sx)):
         cols = sample(g, src.shape[1], 24, must=[0, src.shape[1] - 1])
         xb = wl.bf16_bits(src[:, torch.from_numpy(cols)])
-        q_ref, s_ref, _ = orc.quant_colwise_jagged(xb, w.offsets, orc.TRANSPOSED, ld_q=ld)
-        got_q = q_dev[torch.from_numpy(cols).cuda(), :m].cpu().numpy()
-        assert (got_q == q_ref[:, :m]).all()
+        q_ref, s_ref, _ = orc.quant_colwise_jagged(xb, w.offsets, orc.TRANSPOSED)
+        expect = np.zeros((len(cols), p_end), np.uint8)
+        for e in range(len(sizes)):
+            expect[:, p_start[e]:p_start[e] + sizes[e]] = q_ref[:, starts[e]:starts[e] + sizes[e]]
+        got_q = q_dev[torch.from_numpy(cols).cuda(), :p_end].cpu().numpy()
+        assert (got_q == expect).all()
         got_s = s_dev[:, torch.from_numpy(cols).cuda()].cpu().numpy()
         assert (got_s.view(np.uint32) == s_ref.view(np.uint32)).all()
         checked.append((cols, q_ref, s_ref))

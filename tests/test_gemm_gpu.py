@@ -211,6 +211,40 @@ def test_k_jagged_every_element(sizes, n, k):
             assert (out[e] == 0).all()
 
 
+@pytest.mark.parametrize("sizes,n,k", [
+    ([0, 5, 17, 130, 1, 250], 200, 136),
+    ([3, 700, 0, 44, 128, 256], 72, 264),
+])
+def test_k_jagged_padded_operands_every_element(sizes, n, k):
+    """Operands in the padded transposed layout (groups at 128-token
+    boundaries, zeros in the gaps) give the oracle's products on the plain
+    operands.  The code buffers start filled with NaN codes, so a token the
+    GEMM read outside the groups' padded ranges, or a gap left unwritten,
+    would turn outputs into NaN."""
+    m = int(sum(sizes))
+    e = len(sizes)
+    seed = 5 * m + n
+    dh = rand_bf16(seed, (m, n), 1e-3)
+    x = rand_bf16(seed + 1, (m, k))
+    off = wl.offsets_from_sizes(sizes)
+    offd = torch.from_numpy(off).cuda()
+    ld = (m + 128 * e + 127) // 128 * 128
+    qa = torch.full((n, ld), 0x7F, dtype=torch.uint8, device="cuda")
+    qb = torch.full((k, ld), 0x7F, dtype=torch.uint8, device="cuda")
+    qa, sa = qgg.fp8_quant_colwise_jagged(dh.cuda(), offd, qgg.LAYOUT_TRANSPOSED_PADDED, q=qa)
+    qb, sb = qgg.fp8_quant_colwise_jagged(x.cuda(), offd, qgg.LAYOUT_TRANSPOSED_PADDED, q=qb)
+    out = torch.full((e, n, k), float("nan"), device="cuda")
+    qgg.fp8_scaled_grouped_gemm(qgg.K_JAGGED_PADDED, qa, sa, qb, sb, offd, m_total=m, out=out)
+    torch.cuda.synchronize()
+    oa, osa, _ = orc.quant_colwise_jagged(bits(dh), off, orc.TRANSPOSED)
+    ob, osb, _ = orc.quant_colwise_jagged(bits(x), off, orc.TRANSPOSED)
+    out = out.cpu().numpy()
+    check_k_all(out, (oa, osa, ob, osb, off, m))
+    for g, sz in enumerate(sizes):
+        if sz == 0:
+            assert (out[g] == 0).all()
+
+
 def test_k_jagged_group_starts_at_every_residue_of_a_block():
     """Groups whose starts fall at every position inside a 128-token block (and
     whose ends too), so that every pattern of skipped 32-token steps and

@@ -335,6 +335,52 @@ def test_colwise_format_mismatch_is_counted_like_the_oracle(fmt, smax):
     assert int(sat.item()) == sat_ref
 
 
+def padded_placement(q_t, off, ld_p, fill):
+    """The oracle's transposed codes at the padded layout's positions: group e
+    at tokens [P_e, P_e + size_e) with P_e the sum of the earlier sizes rounded
+    up to 128, zero codes up to P_e + round_up(size_e, 128), `fill` after."""
+    out = np.full((q_t.shape[0], ld_p), fill, np.uint8)
+    start, p = 0, 0
+    for end in np.asarray(off, np.int64):
+        sz = int(end) - start
+        out[:, p:p + sz] = q_t[:, start:int(end)]
+        r = (sz + 127) // 128 * 128
+        out[:, p + sz:p + r] = 0
+        start, p = int(end), p + r
+    return out
+
+
+@pytest.mark.parametrize("sizes,cols,fmt", [
+    ([5, 0, 19, 8], 16, qgg.E4M3FN),
+    ([0, 1, 15, 17, 0, 33, 128, 129, 255], 72, qgg.E4M3FNUZ),
+    ([20011, 3, 9000, 0, 385], 136, qgg.E4M3FN),
+    ([3000, 70, 700], 1408, qgg.E4M3FN),
+    ([1] * 17, 128, qgg.E4M3FN),
+    ([0, 0, 0], 64, qgg.E4M3FN),
+])
+def test_colwise_padded_transposed_layout(sizes, cols, fmt):
+    """Every group at a 128-token boundary, zero codes to the next boundary and
+    nothing written past the last group; codes and scales bit-exact with the
+    oracle's plain transposed layout moved to those positions.  The tall groups
+    go through the chunked path, whose rows then start at the group's first row."""
+    m = int(sum(sizes))
+    e = len(sizes)
+    x = rand_bf16(7 * m + cols, m, cols, outliers=0.002)
+    off = wl.offsets_from_sizes(sizes)
+    ld = (m + 128 * e + 16 + 15) // 16 * 16
+    q_t, s_ref, _ = orc.quant_colwise_jagged(bits(x), off, orc.TRANSPOSED, fmt)
+    expect = padded_placement(q_t, off, ld, 0xAB)
+    qbuf = torch.full((cols, ld), 0xAB, dtype=torch.uint8, device="cuda")
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    q, s = qgg.fp8_quant_colwise_jagged(dev(x), torch.from_numpy(off).cuda(),
+                                        qgg.LAYOUT_TRANSPOSED_PADDED, fmt, q=qbuf, status=st)
+    qn = q.cpu().numpy()
+    bad = np.argwhere(qn != expect)
+    assert bad.size == 0, (bad.shape, bad[:10])
+    assert (s.cpu().numpy().view(np.uint32) == s_ref.view(np.uint32)).all()
+    assert int(st.item()) == 0
+
+
 @pytest.mark.parametrize("layout", [qgg.LAYOUT_SAME, qgg.LAYOUT_TRANSPOSED])
 def test_colwise_tall_groups_split_over_many_blocks(layout):
     """Groups of 20k and 9k rows: cut into 45 and 21 chunks per 64-column tile,
