@@ -814,16 +814,20 @@ __global__ void __launch_bounds__(kColThreads, kBlocksPerSM)
 
 // Zero codes of the padded transposed layout: for every group e and column c,
 // tokens [P_e + size_e, P_e + round_up(size_e, 128)) of row c of the codes.
-// The run ends on a 16-byte boundary (P_e is a multiple of 128 and ld_q of
-// 16), so it takes byte stores up to the first boundary, then 16-byte stores.
-// Every block rebuilds the clamped ends and padded starts (warp 0 scans).
+// The run is shorter than 128 tokens and ends on a multiple of 128 (P_e is
+// one, and ld_q a multiple of 16), so it lies in the 128-byte window that
+// ends there: a warp takes four columns, eight lanes per column, one 16-byte
+// piece of the window per lane.  The lane holding the run's first token
+// clears the bytes up to its piece's end with naturally aligned 1, 2, 4 and
+// 8-byte stores.  Every block rebuilds the clamped ends and padded starts
+// (warp 0 scans).
 __global__ void __launch_bounds__(256) pad_transposed_kernel(const int32_t *__restrict__ offsets,
                                                              int num_groups, int64_t rows_total,
                                                              int cols, uint8_t *__restrict__ q,
                                                              int64_t ld_q) {
   __shared__ int32_t s_start[kMaxGroups], s_size[kMaxGroups];
+  const int lane = threadIdx.x & 31;
   if (threadIdx.x < 32) {
-    const int lane = threadIdx.x;
     const int32_t R = static_cast<int32_t>(rows_total);
     int32_t carry_end = 0, carry_pad = 0;
     for (int base = 0; base < num_groups; base += 32) {
@@ -852,18 +856,29 @@ __global__ void __launch_bounds__(256) pad_transposed_kernel(const int32_t *__re
     }
   }
   __syncthreads();
-  const int64_t pairs = static_cast<int64_t>(num_groups) * cols;
-  for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < pairs;
-       i += int64_t(gridDim.x) * blockDim.x) {
-    const int e = static_cast<int>(i / cols);
-    const int64_t c = i - int64_t(e) * cols;
+  const int64_t quads = (cols + 3) / 4;
+  const int64_t items = static_cast<int64_t>(num_groups) * quads;
+  const int64_t nwarps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
+  for (int64_t it = blockIdx.x * int64_t(blockDim.x >> 5) + (threadIdx.x >> 5); it < items;
+       it += nwarps) {
+    const int e = static_cast<int>(it / quads);
+    const int64_t c = (it - int64_t(e) * quads) * 4 + (lane >> 3);
     const int32_t sz = s_size[e];
     const int64_t lo = s_start[e] + int64_t(sz);
     const int64_t hi = s_start[e] + int64_t((sz + 127) & ~127);
+    if (c >= cols || lo >= hi) continue;
+    const int64_t t0 = hi - 16 * (8 - (lane & 7));  // this lane's piece [t0, t0 + 16)
+    if (t0 + 16 <= lo) continue;
     uint8_t *row = q + c * ld_q;
-    const int64_t mid = min(hi, (lo + 15) & ~int64_t(15));
-    for (int64_t t = lo; t < mid; ++t) row[t] = 0;
-    for (int64_t t = mid; t < hi; t += 16) *reinterpret_cast<uint4 *>(row + t) = make_uint4(0, 0, 0, 0);
+    if (t0 >= lo) {
+      *reinterpret_cast<uint4 *>(row + t0) = make_uint4(0u, 0u, 0u, 0u);
+    } else {
+      int64_t t = lo;  // up to the next 16-byte boundary, t0 + 16
+      if (t & 1) { row[t] = 0; t += 1; }
+      if (t & 2) { *reinterpret_cast<uint16_t *>(row + t) = 0; t += 2; }
+      if (t & 4) { *reinterpret_cast<uint32_t *>(row + t) = 0u; t += 4; }
+      if (t & 8) { *reinterpret_cast<uint2 *>(row + t) = make_uint2(0u, 0u); }
+    }
   }
 }
 
@@ -997,9 +1012,9 @@ int colwise_launch(const void *x, int64_t rows_total, int64_t cols, int64_t ld_x
       reinterpret_cast<uint32_t *>(base), reinterpret_cast<uint32_t *>(base + sl.arrive_off),
       reinterpret_cast<uint32_t *>(base + sl.amax_off), static_cast<int32_t>(sl.units_cap));
   if (layout == FP8QGG_LAYOUT_TRANSPOSED_PADDED && rows_total > 0) {
-    const int64_t pairs = int64_t(num_groups) * cols;
+    const int64_t warps = int64_t(num_groups) * ((cols + 3) / 4);
     const int pgrid = static_cast<int>(
-        std::max<int64_t>(1, std::min<int64_t>((pairs + 255) / 256, int64_t(dev.sm_count) * 4)));
+        std::max<int64_t>(1, std::min<int64_t>((warps + 7) / 8, int64_t(dev.sm_count) * 8)));
     pad_transposed_kernel<<<pgrid, 256, 0, stream>>>(offsets, static_cast<int>(num_groups),
                                                      rows_total, static_cast<int>(cols), q, ld_q);
   }
