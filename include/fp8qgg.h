@@ -157,8 +157,9 @@ size_t fp8_quant_colwise_jagged_workspace_size(int64_t rows_total, int64_t cols,
  *            group edge inside a 128-token block (mode
  *            FP8QGG_K_JAGGED_PADDED).  ld_q >= rows_total + 128 * num_groups,
  *            ld_q % 16 == 0; columns past the last padded group are not
- *            written.  This layout is this library's choice: the pages do
- *            not describe one.
+ *            written.  The zero codes come from a second, small kernel the
+ *            call enqueues on `stream` after the quantisation.  This layout
+ *            is this library's choice: the pages do not describe one.
  *   scales   fp32 [num_groups, cols]; an empty group gets Fmax / 1e-12 in
  *            every column and no codes.
  *   workspace, workspace_bytes: device scratch of at least
