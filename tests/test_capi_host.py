@@ -156,3 +156,26 @@ def test_cast_argument_checks(lib):
     assert f(FAKE, 4, FAKE, 2, None) == -4
     assert f(None, 4, FAKE, 0, None) == -1
     assert f(FAKE, 0, FAKE, 0, None) == 0
+
+
+def test_binding_refuses_host_tensors_instead_of_computing_on_the_cpu():
+    """There is no CPU or torch fallback: every entry point of the binding
+    raises on host tensors before anything is computed."""
+    import torch
+    x = torch.zeros((4, 8), dtype=torch.bfloat16)
+    off = torch.tensor([4], dtype=torch.int32)
+    q8 = torch.zeros((4, 8), dtype=torch.uint8)
+    s = torch.ones(4, dtype=torch.float32)
+    calls = [
+        lambda: qgg.fp8_quant_rowwise(x),
+        lambda: qgg.fp8_quant_colwise_jagged(x, off),
+        lambda: qgg.fp8_quant_colwise_jagged(x, off, qgg.LAYOUT_TRANSPOSED_PADDED),
+        lambda: qgg.fp8_scaled_grouped_gemm(qgg.M_JAGGED, q8, s, q8.view(1, 4, 8),
+                                            s.view(1, 4), off),
+        lambda: qgg.fp8_scaled_grouped_gemm(qgg.K_JAGGED_PADDED, q8, s.view(1, 4), q8,
+                                            s.view(1, 4), off, m_total=4),
+        lambda: qgg.fp8_cast_f32(torch.zeros(8)),
+    ]
+    for f in calls:
+        with pytest.raises(ValueError, match="CUDA tensors only"):
+            f()
