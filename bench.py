@@ -169,6 +169,14 @@ def oracle_sample(w, rows_x, rows_w, n_elem, seed=0):
     return t3 - t0, full, dict(rows_x=rows_x, rows_w=rows_w, gemm_outputs=n_elem)
 
 
+def host_cores():
+    """CPU cores this process may run on (the oracle itself uses one thread)."""
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count()
+
+
 def run_reference(args, world, rank):
     if rank != 0:
         return 0
@@ -191,11 +199,14 @@ def run_reference(args, world, rank):
               f"{n_elem} fp64 GEMM outputs; time extrapolated to the full step by rows and "
               f"outputs")
     line = dict(metric=METRIC, value=value, unit="TFLOP/s", n_gpus=args.gpus, steps=args.steps,
-                warmup=args.warmup, ms_per_step=t_step * 1e3, higher_is_better=True,
+                warmup=args.warmup, ms_per_step=t_step * 1e3,
+                ms_per_step_kind="extrapolated from the timed sample to one full step",
+                sample_ms_per_step=t_sample / args.steps * 1e3, higher_is_better=True,
                 scaling="weak", vs_baseline=None, dtype="f32 quantisation / f64 GEMM",
                 data="synthetic", impl="reference", config=config_dict(w),
-                cpu_baseline=dict(value=value, unit="TFLOP/s", cores=1, kind="oracle",
-                                  sample=sample),
+                cpu_baseline=dict(value=value, unit="TFLOP/s", cores=1,
+                                  host_cores=host_cores(), kind="oracle", sample=sample,
+                                  extrapolated=True),
                 e2e=dict(value=value, unit="TFLOP/s", h2d_bytes_per_step=0,
                          d2h_bytes_per_step=0))
     print(json.dumps(line))
@@ -244,6 +255,7 @@ class ForwardStep:
         self.launches = 3  # this library's kernels per step
         self.bytes = [m * k * 3 + m * 4, e * n * k * 3 + e * n * 4, None]
         self.host_inputs = [(self.x, w.x), (self.wt, w.w.reshape(e * n, k))]
+        self.input_bytes = 2 * (m * k + e * n * k)
         self.result = self.out
 
     def kernels(self):
@@ -290,6 +302,7 @@ class BackwardDwStep:
         self.launches = 5  # each colwise call: the quantisation and the gap fill
         self.bytes = [m * n * 3 + e * n * 4 + e * 4, m * k * 3 + e * k * 4 + e * 4, None]
         self.host_inputs = [(self.g, w.grad_out), (self.x, w.x)]
+        self.input_bytes = 2 * (m * n + m * k)
         self.result = self.out
 
     def kernels(self):
@@ -315,11 +328,11 @@ WORKLOADS = {
 }
 
 
-def run_gpu(args, world, rank, local):
-    pk = peaks()
-    make, Step = WORKLOADS[args.workload]
-    w = make()
-    st = Step(w)
+def time_steps(st, steps, warmup, flush=None):
+    """Runs `warmup` untimed steps, then `steps` timed ones with CUDA events on
+    the current stream around every kernel call.  `flush` (optional) runs
+    between steps, outside the events.  Returns (total ms of the timed region,
+    per-kernel mean ms, events)."""
     ks = st.kernels()
     nk = len(ks)
 
@@ -331,25 +344,92 @@ def run_gpu(args, world, rank, local):
         if ev is not None:
             ev[nk].record()
 
-    for _ in range(max(args.warmup, 3)):
+    for _ in range(max(warmup, 3)):
+        if flush is not None:
+            flush()
         step()
     torch.cuda.synchronize()
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nk + 1)]
-           for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nk + 1)] for _ in range(steps)]
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record()
+    for i in range(steps):
+        if flush is not None:
+            flush()
+        step(evs[i])
+    t_end.record()
+    torch.cuda.synchronize()
+    k_ms = [statistics.mean(e[i].elapsed_time(e[i + 1]) for e in evs) for i in range(nk)]
+    return t_start.elapsed_time(t_end), k_ms, step
+
+
+def kernel_table(st, k_ms, pk):
+    """Per-kernel figures of a step: GB/s and fraction of the HBM peak for the
+    quantisations (algorithmic bytes), TFLOP/s and fraction of the FP8 peak for
+    the GEMM."""
+    fp8_peak = 2.0 * pk["bf16"]
+    kern = {}
+    for name, b, t in zip(st.names, st.bytes, k_ms):
+        if b:
+            gbs = b / (t * 1e-3) / 1e9
+            kern[name] = dict(us=t * 1e3, gbs=gbs, frac_hbm=gbs / pk["hbm_gbs"],
+                              algorithmic_bytes=b)
+        else:
+            tf = st.flops / (t * 1e-3) / 1e12
+            kern[name] = dict(us=t * 1e3, tflops=tf, frac_fp8=tf / fp8_peak, flops=st.flops)
+    q = [(b, t) for b, t in zip(st.bytes, k_ms) if b]
+    if q:
+        q_gbs = sum(b for b, _ in q) / (sum(t for _, t in q) * 1e-3) / 1e9
+        kern.update(quant_gbs=q_gbs, quant_frac_hbm=q_gbs / pk["hbm_gbs"])
+    return kern
+
+
+def extra_workload(name, steps, warmup, pk):
+    """Times one more workload in the same run: the step's kernels with L2
+    flushed between steps (a 256 MB write outside the timed kernels) when its
+    inputs fit in L2.  Returns the per-kernel figures; the step time is the sum
+    of the kernels' event times."""
+    make, Step = WORKLOADS[name]
+    w = make()
+    st = Step(w)
+    small = st.input_bytes < 2 * L2_BYTES
+    flush = None
+    if small:
+        buf = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device="cuda")
+        flush = lambda: buf.fill_(1)  # noqa: E731
+    _, k_ms, _ = time_steps(st, steps, warmup, flush)
+    step_ms = sum(k_ms)
+    d = dict(config=config_dict(w, Step), ms_per_step=step_ms,
+             gemm_equivalent_tflops=st.flops / (step_ms * 1e-3) / 1e12,
+             kernels=kernel_table(st, k_ms, pk), gpu_launches_per_step=st.launches,
+             l2=("flushed between steps (256 MB write, not timed)" if small else
+                 "no flush: the step reads and writes more than the 126 MB L2"))
+    tr = TRAFFIC.get(name)
+    if tr:
+        d["traffic"] = tr
+    del st, w
+    torch.cuda.empty_cache()
+    return d
+
+
+# Workloads timed in the default run beside the headline one: the tiny MoE
+# layer (launch-bound) and the DeepSeek-MoE-16B backward weight-gradient step.
+EXTRA_WORKLOADS = ("tiny_moe", "deepseek_moe16b_bwd")
+
+
+def run_gpu(args, world, rank, local):
+    pk = peaks()
+    make, Step = WORKLOADS[args.workload]
+    w = make()
+    st = Step(w)
+
     barrier(world)
     torch.cuda.synchronize()
     with ClockSampler(torch.cuda.current_device()) as clk:
-        t_start.record()
-        for i in range(args.steps):
-            step(evs[i])
-        t_end.record()
-        torch.cuda.synchronize()
+        total_ms, k_ms, step = time_steps(st, args.steps, args.warmup)
     barrier(world)
-    total_ms = max_over_ranks(t_start.elapsed_time(t_end), world)
+    total_ms = max_over_ranks(total_ms, world)
     ms_step = total_ms / args.steps
-    k_ms = [statistics.mean(e[i].elapsed_time(e[i + 1]) for e in evs) for i in range(nk)]
     clocks = clk.summary()
 
     # end to end through the public API with host buffers: pinned H2D of the
@@ -379,23 +459,10 @@ def run_gpu(args, world, rank, local):
 
     flops = st.flops
     value = flops * world / (ms_step * 1e-3) / 1e12
-    gm_ms = k_ms[-1]
-    gemm_tflops = flops / (gm_ms * 1e-3) / 1e12
     fp8_peak = 2.0 * pk["bf16"]
-    q_bytes = sum(b for b in st.bytes if b)
-    q_ms = sum(k_ms[:-1])
-    quant_gbs = q_bytes / (q_ms * 1e-3) / 1e9
-    kern = {}
-    for name, b, t in zip(st.names, st.bytes, k_ms):
-        if b:
-            gbs = b / (t * 1e-3) / 1e9
-            kern[name] = dict(us=t * 1e3, gbs=gbs, frac_hbm=gbs / pk["hbm_gbs"],
-                              algorithmic_bytes=b)
-        else:
-            kern[name] = dict(us=t * 1e3, tflops=gemm_tflops, frac_fp8=gemm_tflops / fp8_peak,
-                              flops=flops)
-    kern.update(quant_gbs=quant_gbs, quant_frac_hbm=quant_gbs / pk["hbm_gbs"],
-                hbm_peak_gbs=pk["hbm_gbs"], fp8_peak_tflops=fp8_peak)
+    kern = kernel_table(st, k_ms, pk)
+    gemm_tflops = kern["grouped_gemm"]["tflops"]
+    kern.update(hbm_peak_gbs=pk["hbm_gbs"], fp8_peak_tflops=fp8_peak)
     line = dict(
         metric=METRIC, value=value, unit="TFLOP/s", n_gpus=world, steps=args.steps,
         warmup=args.warmup, ms_per_step=ms_step, higher_is_better=True, scaling="weak",
@@ -411,14 +478,23 @@ def run_gpu(args, world, rank, local):
         gpu_launches=st.launches * args.steps,
         clocks=clocks,
     )
+    del pinned, hout
     if rank == 0 and world == 1 and Step is ForwardStep and not args.no_cpu_baseline:
         _, full, desc = oracle_sample(w, min(8192, st.m), min(8192, st.e * st.n), 120000)
         cpu_v = flops / full / 1e12
         line["cpu_baseline"] = dict(
-            value=cpu_v, unit="TFLOP/s", cores=1, kind="oracle",
+            value=cpu_v, unit="TFLOP/s", cores=1, host_cores=host_cores(), kind="oracle",
+            extrapolated=True,
             sample=(f"oracle (1 thread) rowwise quantisation of {desc['rows_x']} X rows and "
                     f"{desc['rows_w']} W rows plus {desc['gemm_outputs']} fp64 GEMM outputs, "
                     "extrapolated to one full step"))
+    if args.workload == "llama3_8b_up_proj" and not args.no_extra:
+        # the other workloads the targets name, timed in the same run (not in
+        # `value`, which stays the headline workload's)
+        del st, w
+        torch.cuda.empty_cache()
+        line["configs"] = {name: extra_workload(name, args.steps, args.warmup, pk)
+                           for name in EXTRA_WORKLOADS}
     if rank == 0:
         print(json.dumps(line))
     return 0
@@ -440,6 +516,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="llama3_8b_up_proj", choices=sorted(WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="time only --workload (skip the extra workloads of the default run)")
     args = ap.parse_args()
     if args.impl == "reference":
         # the CPU oracle runs on rank 0 alone; no process group is needed
@@ -447,10 +525,9 @@ def main():
         return run_reference(args, int(os.environ.get("WORLD_SIZE", "1")), rank)
     world, rank, local = dist_setup(args)
     try:
-        if True:
-            if not torch.cuda.is_available():
-                raise RuntimeError("bench.py needs a CUDA device for the GPU arm")
-            rc = run_gpu(args, world, rank, local)
+        if not torch.cuda.is_available():
+            raise RuntimeError("bench.py needs a CUDA device for the GPU arm")
+        rc = run_gpu(args, world, rank, local)
     finally:
         if world > 1 and torch.distributed.is_initialized():
             torch.distributed.destroy_process_group()

@@ -89,7 +89,6 @@ extern "C" {
 /* bits OR-ed into *dev_status */
 #define FP8QGG_STATUS_BAD_OFFSETS 1  /* offsets had to be clamped */
 #define FP8QGG_STATUS_TIMEOUT 2      /* a bounded device-side wait gave up */
-#define FP8QGG_STATUS_GROUP_TOO_TALL 4 /* reserved (no current kernel sets it) */
 
 /* The FP8 variant this device's tensor cores consume.  The pages add
  * automatic detection of the format because the wrong maximum corrupts
@@ -199,8 +198,14 @@ int fp8_quant_colwise_jagged(const void *x, int64_t rows_total, int64_t cols, in
  *    tensor (1,733,632 bytes); it does not cover 64 groups of a 98304 x 8192
  *    tensor (2,130,176 bytes).
  *  - Set-up: the first call on each device looks up the array's device
- *    address with that device current (cudaGetSymbolAddress).  Make that
- *    first call before any stream capture on the device.
+ *    address with that device current (cudaGetSymbolAddress) and keeps it
+ *    with the device's current context.  Make that first call before any
+ *    stream capture on the device.  A later call made under another context
+ *    (for instance after cudaDeviceReset, which unloads the library's device
+ *    code with the old context) looks the address up again.
+ *  - Errors: FP8QGG_ERR_CUDA when the current device ordinal is 64 or above
+ *    (the set-up keeps one address per device for ordinals 0..63), when the
+ *    address lookup fails, or when the clearing memset or the launch fails.
  *  - Sharing: every call uses the same array and clears the part it needs on
  *    `stream` first.  Calls on one device whose executions could overlap on
  *    the GPU race; order them (one stream, or events).
@@ -213,6 +218,21 @@ int fp8_quant_colwise_jagged_noalloc(const void *x, int64_t rows_total, int64_t 
                                      uint8_t *q, int64_t ld_q, int layout, float *scales,
                                      int fmt, float scale_max, uint64_t *sat_count,
                                      int32_t *dev_status, void *stream);
+
+/*
+ * Test hook of the failure detection, not for production use.  Every device
+ * wait of the library gives up after a time limit and ORs
+ * FP8QGG_STATUS_TIMEOUT into *dev_status instead of spinning for ever.  This
+ * call changes one of them, for the jagged column-wise calls that follow it in
+ * the process: the wait of a tall unit's cast for the unit's merged absmax
+ * also needs `extra_arrivals` chunk arrivals that never come, and gives up
+ * after `limit_ns` nanoseconds (0 restores the normal limit of 2 s; at most
+ * 2e9).  With extra_arrivals > 0 a call with a group taller than one chunk
+ * therefore returns FP8QGG_OK, leaves FP8QGG_STATUS_TIMEOUT in *dev_status
+ * and undefined codes and scales, and the device stays usable.  The waits for
+ * copies in flight keep their normal limit.  (0, 0) restores normal calls.
+ */
+int fp8qgg_test_unit_wait(uint32_t extra_arrivals, uint64_t limit_ns);
 
 /*
  * FP8 scaled grouped GEMM on the 5th-generation tensor cores (the pages run

@@ -25,7 +25,6 @@ OUT_F32 = 0
 OUT_BF16 = 1
 STATUS_BAD_OFFSETS = 1
 STATUS_TIMEOUT = 2
-STATUS_GROUP_TOO_TALL = 4
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libfp8qgg.so")
@@ -52,6 +51,7 @@ _SIGNATURES = {
     "fp8_cast_f32": (_INT, [_P, _I64, _P, _INT, _P]),
     "fp8_quant_colwise_jagged_noalloc": (_INT, [_P, _I64, _I64, _I64, _P, _I32, _P, _I64, _INT,
                                                 _P, _INT, _F32, _P, _P, _P]),
+    "fp8qgg_test_unit_wait": (_INT, [ctypes.c_uint32, ctypes.c_uint64]),
 }
 
 

@@ -102,6 +102,14 @@ struct SlotMeta {
 };
 static_assert(sizeof(SlotMeta) == 32, "slot metadata is two 16-byte words");
 
+// The wait of a cast task for its tall unit's absmax: the chunk count it
+// needs beyond the unit's own chunks (0 in every normal call) and its time
+// limit.  Only the failure-detection test changes them (fp8qgg_test_unit_wait).
+struct UnitWait {
+  uint32_t extra_arrivals;
+  uint64_t limit_ns;
+};
+
 struct ColSmem {
   uint32_t ring[kSlots][kBoxRows * kWords];  // [row][32 words]; word = 2 bf16 columns
   // per-warp column absmax of a whole or amax task, one buffer per task that
@@ -436,7 +444,8 @@ __global__ void __launch_bounds__(kColThreads, kBlocksPerSM)
                                 float *__restrict__ scales, float smax, float sat_thr,
                                 unsigned long long *sat_count, int32_t *status,
                                 uint32_t *__restrict__ work_counter, uint32_t *__restrict__ arrive,
-                                uint32_t *__restrict__ unit_amax, int32_t units_cap) {
+                                uint32_t *__restrict__ unit_amax, int32_t units_cap,
+                                UnitWait uw) {
   extern __shared__ uint8_t smem_raw[];
   ColSmem &sm = *align_smem_1024<ColSmem>(smem_raw);
   const int tid = threadIdx.x;
@@ -537,13 +546,14 @@ __global__ void __launch_bounds__(kColThreads, kBlocksPerSM)
         const uint32_t *cnt = arrive + m.tu;
         uint32_t v;
         asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(cnt) : "memory");
-        if (v < static_cast<uint32_t>(m.target)) {
+        const uint32_t target = static_cast<uint32_t>(m.target) + uw.extra_arrivals;
+        if (v < target) {
           const uint64_t t0 = global_timer_ns();
           while (true) {
             __nanosleep(256);
             asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(cnt) : "memory");
-            if (v >= static_cast<uint32_t>(m.target)) break;
-            if (*abort || global_timer_ns() - t0 > kWaitLimitNs) return false;
+            if (v >= target) break;
+            if (*abort || global_timer_ns() - t0 > uw.limit_ns) return false;
           }
         }
         const uint4 *src =
@@ -886,7 +896,15 @@ namespace {
 
 using ColKernel = void (*)(const CUtensorMap, const CUtensorMap, int64_t, int, const int32_t *,
                            int, uint8_t *, int64_t, float *, float, float, unsigned long long *,
-                           int32_t *, uint32_t *, uint32_t *, uint32_t *, int32_t);
+                           int32_t *, uint32_t *, uint32_t *, uint32_t *, int32_t, UnitWait);
+
+std::mutex g_unit_wait_mutex;
+UnitWait g_unit_wait{0u, kWaitLimitNs};
+
+UnitWait current_unit_wait() {
+  std::lock_guard<std::mutex> lock(g_unit_wait_mutex);
+  return g_unit_wait;
+}
 
 template <int FMT, bool FAST>
 ColKernel col_kernel_fmt(int layout) {
@@ -1010,7 +1028,8 @@ int colwise_launch(const void *x, int64_t rows_total, int64_t cols, int64_t ld_x
       static_cast<int>(num_groups), q, ld_q, scales, smax, sat_thr,
       reinterpret_cast<unsigned long long *>(sat_count), dev_status,
       reinterpret_cast<uint32_t *>(base), reinterpret_cast<uint32_t *>(base + sl.arrive_off),
-      reinterpret_cast<uint32_t *>(base + sl.amax_off), static_cast<int32_t>(sl.units_cap));
+      reinterpret_cast<uint32_t *>(base + sl.amax_off), static_cast<int32_t>(sl.units_cap),
+      current_unit_wait());
   if (layout == FP8QGG_LAYOUT_TRANSPOSED_PADDED && rows_total > 0) {
     const int64_t warps = int64_t(num_groups) * ((cols + 3) / 4);
     const int pgrid = static_cast<int>(
@@ -1024,6 +1043,14 @@ int colwise_launch(const void *x, int64_t rows_total, int64_t cols, int64_t ld_x
 }  // namespace fp8qgg
 
 using namespace fp8qgg;
+
+extern "C" int fp8qgg_test_unit_wait(uint32_t extra_arrivals, uint64_t limit_ns) {
+  if (limit_ns > kWaitLimitNs) return FP8QGG_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_unit_wait_mutex);
+  g_unit_wait.extra_arrivals = extra_arrivals;
+  g_unit_wait.limit_ns = limit_ns ? limit_ns : kWaitLimitNs;
+  return FP8QGG_OK;
+}
 
 extern "C" size_t fp8_quant_colwise_jagged_workspace_size(int64_t rows_total, int64_t cols,
                                                           int32_t num_groups) {
@@ -1070,23 +1097,51 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratch
 
 namespace {
 constexpr int kMaxScratchDevices = 64;
-void *g_scratch_addr[kMaxScratchDevices];
+struct ScratchAddr {
+  CUcontext ctx;  // the context the address belongs to
+  void *addr;
+};
+ScratchAddr g_scratch_addr[kMaxScratchDevices];
 std::mutex g_scratch_mutex;
+
+using CtxGetCurrentFn = CUresult (*)(CUcontext *);
+
+// The calling thread's current context (nullptr when none is current or the
+// driver entry point is missing).
+CUcontext current_context() {
+  static CtxGetCurrentFn fn = [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return static_cast<CtxGetCurrentFn>(nullptr);
+    return reinterpret_cast<CtxGetCurrentFn>(p);
+  }();
+  CUcontext c = nullptr;
+  if (fn && fn(&c) != CUDA_SUCCESS) c = nullptr;
+  return c;
+}
 }  // namespace
 
 // Device address of the fixed scratch array on the current device.  In host
 // code `g_noalloc_scratch` only names a host-side stand-in, so the address is
-// looked up once per device (with that device current) and cached.
+// looked up with the device current and kept per device together with the
+// context it belongs to; a call under another context (after
+// cudaDeviceReset, for instance, the library's device code is loaded again)
+// looks it up again.
 static bool noalloc_scratch(void **out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxScratchDevices) return false;
   std::lock_guard<std::mutex> lock(g_scratch_mutex);
-  if (!g_scratch_addr[dev]) {
+  ScratchAddr &c = g_scratch_addr[dev];
+  const CUcontext ctx = current_context();
+  if (!c.addr || !ctx || c.ctx != ctx) {
     void *p = nullptr;
     if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return false;
-    g_scratch_addr[dev] = p;
+    c.addr = p;
+    c.ctx = current_context();  // the lookup makes the primary context current if none was
   }
-  *out = g_scratch_addr[dev];
+  *out = c.addr;
   return true;
 }
 

