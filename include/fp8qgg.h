@@ -126,11 +126,13 @@ int fp8_quant_rowwise(const void *x, int64_t rows, int64_t cols, int64_t ld_x,
                       int fmt, float scale_max, uint64_t *sat_count, void *stream);
 
 /*
- * Bytes of device workspace fp8_quant_colwise_jagged needs: a work counter
- * shared by the blocks (256 bytes), plus, for every (group, 64-column) unit
- * that may be taller than 448 rows, an arrival counter and 64 absmax words
- * (260 bytes per unit; at most min(num_groups, rows_total / 432) groups can be
- * that tall).  Always > 0 and a multiple of 256.
+ * Bytes of device workspace fp8_quant_colwise_jagged needs, for every layout:
+ * the larger of (a) the plain layouts' kernel: a task counter (256 bytes),
+ * plus, for every (group, 64-column) unit that may be taller than 448 rows,
+ * an arrival counter and 64 absmax words (at most min(num_groups,
+ * rows_total / 432) groups can be that tall), and (b) the padded layout's
+ * kernel: a task counter, one arrival counter per (group, 256-column panel)
+ * and one absmax word per (group, column).  Always > 0 and a multiple of 256.
  */
 size_t fp8_quant_colwise_jagged_workspace_size(int64_t rows_total, int64_t cols,
                                                int32_t num_groups);
@@ -156,9 +158,10 @@ size_t fp8_quant_colwise_jagged_workspace_size(int64_t rows_total, int64_t cols,
  *            group edge inside a 128-token block (mode
  *            FP8QGG_K_JAGGED_PADDED).  ld_q >= rows_total + 128 * num_groups,
  *            ld_q % 16 == 0; columns past the last padded group are not
- *            written.  The zero codes come from a second, small kernel the
- *            call enqueues on `stream` after the quantisation.  This layout
- *            is this library's choice: the pages do not describe one.
+ *            written.  The codes of each 128-token block (zeros past the
+ *            group's end included) leave the chip as one bulk tensor store.
+ *            This layout is this library's choice: the pages do not
+ *            describe one.
  *   scales   fp32 [num_groups, cols]; an empty group gets Fmax / 1e-12 in
  *            every column and no codes.
  *   workspace, workspace_bytes: device scratch of at least
@@ -182,6 +185,52 @@ int fp8_quant_colwise_jagged(const void *x, int64_t rows_total, int64_t cols, in
                              void *stream);
 
 /*
+ * Bytes of device workspace fp8_quant_dual_jagged needs: a task counter (256
+ * bytes), one arrival counter per group, the column absmax words
+ * [num_groups, cols] and one row absmax word per row, each part rounded up to
+ * 256 bytes.
+ */
+size_t fp8_quant_dual_jagged_workspace_size(int64_t rows_total, int64_t cols,
+                                            int32_t num_groups);
+
+/*
+ * Dual-output quantisation for the backward pass: ONE read of x gives both
+ * FP8 copies the two backward GEMMs of an expert layer need ([AIR] "Il
+ * guadagno vero è nel movimento dei dati", second paragraph: the backward's
+ * scale-and-cast fused and its transposed copy removed; [ABP] second
+ * paragraph):
+ *  - the rowwise quantisation (one scale per row) of every row of the groups,
+ *    for the input-gradient GEMM (token-jagged, FP8QGG_M_JAGGED);
+ *  - the jagged column-wise quantisation in FP8QGG_LAYOUT_TRANSPOSED_PADDED
+ *    (one scale per (group, column)), for the weight-gradient GEMM
+ *    (FP8QGG_K_JAGGED_PADDED).
+ * The codes and scales are those of fp8_quant_rowwise on each row of a group
+ * and of fp8_quant_colwise_jagged with the padded layout, bit for bit.
+ *   x          bf16 [rows_total, ld_x], read once from HBM (each 128-row
+ *              block is read a second time for the casts, from L2).
+ *   offsets    int32 [num_groups] cumulative group ends (device).
+ *   q_row      uint8 [rows_total, ld_qr]: columns [0, cols) of every row of
+ *              a group; rows past the last group end are not written.
+ *   scales_row fp32 [rows_total], written for the rows of the groups.
+ *   q_col      uint8 [cols, ld_qc] in the padded transposed layout,
+ *              ld_qc >= rows_total + 128 * num_groups, ld_qc % 16 == 0.
+ *   scales_col fp32 [num_groups, cols]; an empty group gets Fmax / 1e-12.
+ *   sat_count  (nullable) adds the saturated elements of both quantisations.
+ *   workspace  at least fp8_quant_dual_jagged_workspace_size(...) bytes,
+ *              16-byte aligned, cleared by the call on `stream`; calls that
+ *              share one workspace must be ordered on the device.
+ * Requirements: those of fp8_quant_colwise_jagged with the padded layout,
+ * plus ld_qr >= cols, ld_qr % 8 == 0, q_row 16-byte aligned, scales_row
+ * 4-byte aligned.
+ */
+int fp8_quant_dual_jagged(const void *x, int64_t rows_total, int64_t cols, int64_t ld_x,
+                          const int32_t *offsets, int32_t num_groups,
+                          uint8_t *q_row, int64_t ld_qr, float *scales_row,
+                          uint8_t *q_col, int64_t ld_qc, float *scales_col,
+                          int fmt, float scale_max, uint64_t *sat_count, int32_t *dev_status,
+                          void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * Same computation as fp8_quant_colwise_jagged, for callers that cannot
  * allocate device memory or supply a workspace (for example a runtime that
  * fixes its memory budget at start-up and forbids cudaMalloc later, or a
@@ -194,8 +243,8 @@ int fp8_quant_colwise_jagged(const void *x, int64_t rows_total, int64_t cols, in
  *  - Size limit: problems whose fp8_quant_colwise_jagged_workspace_size(...)
  *    exceeds FP8QGG_NOALLOC_SCRATCH_BYTES are rejected with FP8QGG_ERR_SHAPE
  *    before anything is enqueued.  2 MiB covers, for instance, 64 groups of
- *    a 98304 x 2048 tensor (532,736 bytes) or 1024 groups of a 131072 x 1408
- *    tensor (1,733,632 bytes); it does not cover 64 groups of a 98304 x 8192
+ *    a 98304 x 2048 tensor (532,736 bytes) or 256 groups of a 131072 x 1408
+ *    tensor (1,464,576 bytes); it does not cover 64 groups of a 98304 x 8192
  *    tensor (2,130,176 bytes).
  *  - Set-up: the first call on each device looks up the array's device
  *    address with that device current (cudaGetSymbolAddress) and keeps it

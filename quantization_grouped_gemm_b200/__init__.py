@@ -52,6 +52,9 @@ _SIGNATURES = {
     "fp8_quant_colwise_jagged_noalloc": (_INT, [_P, _I64, _I64, _I64, _P, _I32, _P, _I64, _INT,
                                                 _P, _INT, _F32, _P, _P, _P]),
     "fp8qgg_test_unit_wait": (_INT, [ctypes.c_uint32, ctypes.c_uint64]),
+    "fp8_quant_dual_jagged_workspace_size": (_SZ, [_I64, _I64, _I32]),
+    "fp8_quant_dual_jagged": (_INT, [_P, _I64, _I64, _I64, _P, _I32, _P, _I64, _P, _P, _I64, _P,
+                                     _INT, _F32, _P, _P, _P, _SZ, _P]),
 }
 
 
@@ -175,6 +178,46 @@ def fp8_quant_colwise_jagged(x, offsets, layout=LAYOUT_SAME, fmt=E4M3FN, scale_m
         workspace.numel() * workspace.element_size(), _stream(stream))
     _check(rc, "fp8_quant_colwise_jagged")
     return q, scales
+
+
+def dual_workspace_bytes(rows_total, cols, num_groups) -> int:
+    return int(lib().fp8_quant_dual_jagged_workspace_size(rows_total, cols, num_groups))
+
+
+def fp8_quant_dual_jagged(x, offsets, fmt=E4M3FN, scale_max=0.0, q_row=None, scales_row=None,
+                          q_col=None, ld_qc=None, scales_col=None, workspace=None,
+                          sat_count=None, status=None, stream=None):
+    """One read of a bf16 [rows_total, cols] CUDA tensor gives its rowwise
+    quantisation (q_row [rows_total, cols], scales_row [rows_total], rows of the
+    groups) and its jagged column-wise quantisation in LAYOUT_TRANSPOSED_PADDED
+    (q_col [cols, ld_qc], scales_col [num_groups, cols]).
+
+    Returns (q_row, scales_row, q_col, scales_col)."""
+    _need_cuda(x, offsets)
+    assert x.dtype == torch.bfloat16 and x.dim() == 2
+    assert offsets.dtype == torch.int32
+    rows, cols = x.shape
+    e = offsets.numel()
+    if q_row is None:
+        q_row = torch.empty((rows, cols), dtype=torch.uint8, device=x.device)
+    if scales_row is None:
+        scales_row = torch.empty((rows,), dtype=torch.float32, device=x.device)
+    if q_col is None:
+        ld = ld_qc if ld_qc is not None else (rows + 128 * e + 127) // 128 * 128
+        q_col = torch.empty((cols, ld), dtype=torch.uint8, device=x.device)
+    if scales_col is None:
+        scales_col = torch.empty((e, cols), dtype=torch.float32, device=x.device)
+    if workspace is None:
+        workspace = torch.empty(dual_workspace_bytes(rows, cols, e), dtype=torch.uint8,
+                                device=x.device)
+    _need_cuda(q_row, scales_row, q_col, scales_col, workspace, sat_count, status)
+    rc = lib().fp8_quant_dual_jagged(
+        _ptr(x), rows, cols, _ld(x), _ptr(offsets), e, _ptr(q_row), _ld(q_row),
+        _ptr(scales_row), _ptr(q_col), _ld(q_col), _ptr(scales_col), fmt, float(scale_max),
+        _ptr(sat_count), _ptr(status), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(rc, "fp8_quant_dual_jagged")
+    return q_row, scales_row, q_col, scales_col
 
 
 def fp8_scaled_grouped_gemm(mode, a, scale_a, b, scale_b, offsets, m_total=None, n=None, k=None,

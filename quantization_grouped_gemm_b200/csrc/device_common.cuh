@@ -19,6 +19,15 @@ namespace fp8qgg {
 // A bounded device wait gives up after this many nanoseconds of global time.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
 
+// The wait of a cast for its unit's merged absmax (jagged column-wise
+// kernels): the arrivals it needs beyond the unit's own (0 in every normal
+// call) and its time limit.  Only the failure-detection test changes them
+// (fp8qgg_test_unit_wait).
+struct UnitWait {
+  uint32_t extra_arrivals;
+  uint64_t limit_ns;
+};
+
 __device__ __forceinline__ uint32_t smem_addr(const void *p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }

@@ -41,6 +41,7 @@
 
 #include "device_common.cuh"
 #include "host_common.h"
+#include "quant_panels.h"
 
 namespace fp8qgg {
 
@@ -102,13 +103,6 @@ struct SlotMeta {
 };
 static_assert(sizeof(SlotMeta) == 32, "slot metadata is two 16-byte words");
 
-// The wait of a cast task for its tall unit's absmax: the chunk count it
-// needs beyond the unit's own chunks (0 in every normal call) and its time
-// limit.  Only the failure-detection test changes them (fp8qgg_test_unit_wait).
-struct UnitWait {
-  uint32_t extra_arrivals;
-  uint64_t limit_ns;
-};
 
 struct ColSmem {
   uint32_t ring[kSlots][kBoxRows * kWords];  // [row][32 words]; word = 2 bf16 columns
@@ -901,11 +895,6 @@ using ColKernel = void (*)(const CUtensorMap, const CUtensorMap, int64_t, int, c
 std::mutex g_unit_wait_mutex;
 UnitWait g_unit_wait{0u, kWaitLimitNs};
 
-UnitWait current_unit_wait() {
-  std::lock_guard<std::mutex> lock(g_unit_wait_mutex);
-  return g_unit_wait;
-}
-
 template <int FMT, bool FAST>
 ColKernel col_kernel_fmt(int layout) {
   return layout == FP8QGG_LAYOUT_SAME
@@ -946,6 +935,11 @@ ColScratch colwise_scratch(int64_t rows_total, int64_t cols, int32_t num_groups)
 }
 
 }  // namespace
+
+UnitWait current_unit_wait() {
+  std::lock_guard<std::mutex> lock(g_unit_wait_mutex);
+  return g_unit_wait;
+}
 
 // Validates the arguments of a jagged column-wise call; returns FP8QGG_OK or
 // the error code.
@@ -991,6 +985,11 @@ int colwise_launch(const void *x, int64_t rows_total, int64_t cols, int64_t ld_x
                    const int32_t *offsets, int32_t num_groups, uint8_t *q, int64_t ld_q,
                    int layout, float *scales, int fmt, float scale_max, uint64_t *sat_count,
                    int32_t *dev_status, void *scratch, cudaStream_t stream) {
+  // the padded transposed layout runs on the panel kernel (quant_panels.cu)
+  if (layout == FP8QGG_LAYOUT_TRANSPOSED_PADDED)
+    return panel_launch(x, rows_total, cols, ld_x, offsets, num_groups, q, ld_q, scales,
+                        nullptr, 0, nullptr, fmt, scale_max, sat_count, dev_status, scratch,
+                        current_unit_wait(), stream);
   // With no rows no copy is ever issued, so the maps may stay empty.
   CUtensorMap xmap_box, xmap_sub;
   memset(&xmap_box, 0, sizeof xmap_box);
@@ -1054,7 +1053,9 @@ extern "C" int fp8qgg_test_unit_wait(uint32_t extra_arrivals, uint64_t limit_ns)
 
 extern "C" size_t fp8_quant_colwise_jagged_workspace_size(int64_t rows_total, int64_t cols,
                                                           int32_t num_groups) {
-  return colwise_scratch(rows_total, cols, num_groups).bytes;
+  // one workspace size serves every layout: the larger of the two kernels' needs
+  return std::max(colwise_scratch(rows_total, cols, num_groups).bytes,
+                  panel_scratch(rows_total, cols, num_groups, false).bytes);
 }
 
 extern "C" int fp8_quant_colwise_jagged(const void *x, int64_t rows_total, int64_t cols,

@@ -92,13 +92,30 @@ def test_colwise_argument_checks(lib):
     f = lib.fp8_quant_colwise_jagged
     ws = lib.fp8_quant_colwise_jagged_workspace_size(100, 64, 4)
     assert ws > 0 and ws % 256 == 0
-    # tall units (over 448 rows) each need an arrival counter and 64 absmax
-    # words; at most min(groups, rows / 432) groups can be that tall
+    # the larger of the two kernels' needs.  Plain layouts: tall units (over
+    # 448 rows) each need an arrival counter and 64 absmax words; at most
+    # min(groups, rows / 432) groups can be that tall.  Padded layout: one
+    # arrival counter per (group, 256-column panel) and one absmax word per
+    # (group, column).  Each part is rounded up to 256 bytes.
     g = lib.fp8_quant_colwise_jagged_workspace_size
-    assert g(431, 64, 4) == 256
-    assert g(432, 64, 4) == 256 + 256 + 256
-    assert g(98304, 2048, 64) == 256 + 2048 * 4 + 2048 * 256
-    assert g(98304, 2048, 1000) == g(98304, 2048, 227) > g(98304, 2048, 64)
+
+    def r256(b):
+        return (b + 255) // 256 * 256
+
+    def plain(rows, cols, e):
+        units = min(e, rows // 432) * ((cols + 63) // 64)
+        return 256 + r256(4 * units) + 256 * units
+
+    def padded(rows, cols, e):
+        return 256 + r256(4 * e * ((cols + 255) // 256)) + r256(4 * e * cols)
+
+    for args in ((431, 64, 4), (432, 64, 4), (98304, 2048, 64), (98304, 2048, 1000),
+                 (98304, 1408, 64), (5, 8, 1)):
+        assert g(*args) == max(plain(*args), padded(*args)), args
+    assert g(98304, 2048, 64) == 256 + 2048 * 4 + 2048 * 256  # the plain kernel's need
+    assert g(431, 64, 4) == 256 + 256 + 4 * 4 * 64          # the padded kernel's need
+    d = lib.fp8_quant_dual_jagged_workspace_size
+    assert d(98304, 1408, 64) == padded(98304, 1408, 64) + r256(4 * 98304)
 
     def call(**kw):
         a = dict(x=FAKE, rows=100, cols=64, ld_x=64, off=FAKE, e=4, q=FAKE, ld_q=64, layout=0,
