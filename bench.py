@@ -214,9 +214,14 @@ def run_reference(args, world, rank):
 
 
 def config_dict(w, Step=None):
-    m, k = w.x.shape
+    src = w.x if w.x is not None else w.grad_out
+    m, k = src.shape
     d = dict(workload=w.name, M=m, K=k, E=w.num_groups, fmt="e4m3fn", gemm_out="fp32")
-    if w.grad_out is not None and Step is not None and Step.__name__ == "BackwardDwStep":
+    if Step is not None and Step.__name__ == "DualCompareStep":
+        d.update(K=None, N=w.grad_out.shape[1], gemm_out=None,
+                 step=("grad_out quantised for both backward GEMMs: rowwise + padded transposed "
+                       "jagged column-wise as two calls, then as one dual-output call"))
+    elif w.grad_out is not None and Step is not None and Step.__name__ == "BackwardDwStep":
         d.update(N=w.grad_out.shape[1],
                  step=("jagged column-wise quant + transpose of grad_out and of X, groups "
                        "at 128-token boundaries + contraction-jagged FP8 grouped GEMM (dW)"))
@@ -318,10 +323,65 @@ class BackwardDwStep:
         ]
 
 
+class DualCompareStep:
+    """The backward quantisation of grad_out [M, N] for both backward GEMMs:
+    the two separate calls (rowwise codes for the input gradient, padded
+    transposed jagged column-wise codes for the weight gradient), then the
+    dual-output call that writes both from one read.  The step runs all three
+    so that each is timed on the same data; the comparison is the sum of the
+    first two against the third."""
+
+    def __init__(self, w):
+        import quantization_grouped_gemm_b200 as qgg
+        self.qgg = qgg
+        self.w = w
+        m, n = w.grad_out.shape
+        e = w.num_groups
+        self.m, self.n, self.e = m, n, e
+        self.g = w.grad_out.cuda()
+        self.off = torch.from_numpy(w.offsets).cuda()
+        ld = (m + 128 * e + 127) // 128 * 128
+        self.qr = torch.empty((m, n), dtype=torch.uint8, device="cuda")
+        self.sr = torch.empty((m,), dtype=torch.float32, device="cuda")
+        self.qc = torch.empty((n, ld), dtype=torch.uint8, device="cuda")
+        self.sc = torch.empty((e, n), dtype=torch.float32, device="cuda")
+        self.qr2 = torch.empty_like(self.qr)
+        self.sr2 = torch.empty_like(self.sr)
+        self.qc2 = torch.empty_like(self.qc)
+        self.sc2 = torch.empty_like(self.sc)
+        self.ws = torch.empty(qgg.colwise_workspace_bytes(m, n, e), dtype=torch.uint8,
+                              device="cuda")
+        self.wsd = torch.empty(qgg.dual_workspace_bytes(m, n, e), dtype=torch.uint8,
+                               device="cuda")
+        self.flops = 0.0
+        self.names = ["quant_rowwise_grad_out", "quant_colwise_t_grad_out", "quant_dual_grad_out"]
+        self.launches = 3
+        rows = m * n * 3 + m * 4
+        cols = m * n * 3 + e * n * 4 + e * 4
+        self.bytes = [rows, cols, m * n * 4 + m * 4 + e * n * 4 + e * 4]
+        self.host_inputs = [(self.g, w.grad_out)]
+        self.input_bytes = 2 * m * n
+        self.result = self.qc2
+
+    def kernels(self):
+        q = self.qgg
+        T = q.LAYOUT_TRANSPOSED_PADDED
+        return [
+            lambda: q.fp8_quant_rowwise(self.g, q=self.qr, scales=self.sr),
+            lambda: q.fp8_quant_colwise_jagged(self.g, self.off, T, q=self.qc, scales=self.sc,
+                                               workspace=self.ws),
+            lambda: q.fp8_quant_dual_jagged(self.g, self.off, q_row=self.qr2, scales_row=self.sr2,
+                                            q_col=self.qc2, scales_col=self.sc2,
+                                            workspace=self.wsd),
+        ]
+
+
 WORKLOADS = {
     "llama3_8b_up_proj": (lambda: wl.llama3_8b_up_proj(), ForwardStep),
     "tiny_moe": (lambda: wl.tiny_moe(), ForwardStep),
     "deepseek_moe16b_bwd": (lambda: wl.deepseek_moe_16b_backward(), BackwardDwStep),
+    "deepseek_moe16b_bwd_dual": (lambda: wl.deepseek_moe_16b_backward(with_x=False),
+                                 DualCompareStep),
     "deepseek_v3_fwd": (lambda: wl.deepseek_v3_local_experts(), ForwardStep),
     "llama4_m8192_zipf": (lambda: wl.llama4_sweep(8192, "zipf"), ForwardStep),
     "llama4_m131072_uniform": (lambda: wl.llama4_sweep(131072, "uniform"), ForwardStep),
@@ -400,7 +460,7 @@ def extra_workload(name, steps, warmup, pk):
     _, k_ms, _ = time_steps(st, steps, warmup, flush)
     step_ms = sum(k_ms)
     d = dict(config=config_dict(w, Step), ms_per_step=step_ms,
-             gemm_equivalent_tflops=st.flops / (step_ms * 1e-3) / 1e12,
+             gemm_equivalent_tflops=st.flops / (step_ms * 1e-3) / 1e12 if st.flops else None,
              kernels=kernel_table(st, k_ms, pk), gpu_launches_per_step=st.launches,
              l2=("flushed between steps (256 MB write, not timed)" if small else
                  "no flush: the step reads and writes more than the 126 MB L2"))
@@ -414,7 +474,7 @@ def extra_workload(name, steps, warmup, pk):
 
 # Workloads timed in the default run beside the headline one: the tiny MoE
 # layer (launch-bound) and the DeepSeek-MoE-16B backward weight-gradient step.
-EXTRA_WORKLOADS = ("tiny_moe", "deepseek_moe16b_bwd")
+EXTRA_WORKLOADS = ("tiny_moe", "deepseek_moe16b_bwd", "deepseek_moe16b_bwd_dual")
 
 
 def run_gpu(args, world, rank, local):
