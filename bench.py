@@ -518,21 +518,36 @@ def run_gpu(args, world, rank, local):
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world) / e2e_steps
 
     flops = st.flops
-    value = flops * world / (ms_step * 1e-3) / 1e12
     fp8_peak = 2.0 * pk["bf16"]
     kern = kernel_table(st, k_ms, pk)
-    gemm_tflops = kern["grouped_gemm"]["tflops"]
     kern.update(hbm_peak_gbs=pk["hbm_gbs"], fp8_peak_tflops=fp8_peak)
+    if flops:
+        # GEMM-equivalent TFLOP/s of the whole step; the roofline is the GEMM's
+        value = flops * world / (ms_step * 1e-3) / 1e12
+        unit = "TFLOP/s"
+        e2e_value = flops * world / (e2e_ms * 1e-3) / 1e12
+        gemm_tflops = kern["grouped_gemm"]["tflops"]
+        roof = dict(bound="tensor", achieved=gemm_tflops, peak=fp8_peak, unit="TFLOP/s",
+                    frac=gemm_tflops / fp8_peak, traffic=TRAFFIC.get(args.workload),
+                    peak_note=(f"{pk['source']} bf16 burst {pk['bf16']} TFLOP/s x 2 "
+                               "(nominal fp8:bf16 dense ratio)"))
+    else:
+        # a quantisation-only step: algorithmic GB/s; the roofline is its last kernel's
+        qbytes = sum(st.bytes)
+        value = qbytes * world / (ms_step * 1e-3) / 1e9
+        unit = "GB/s"
+        e2e_value = qbytes * world / (e2e_ms * 1e-3) / 1e9
+        last = kern[st.names[-1]]
+        roof = dict(bound="hbm", achieved=last["gbs"], peak=pk["hbm_gbs"], unit="GB/s",
+                    frac=last["frac_hbm"], traffic=TRAFFIC.get(args.workload),
+                    peak_note=f"{pk['source']} HBM copy bandwidth")
     line = dict(
-        metric=METRIC, value=value, unit="TFLOP/s", n_gpus=world, steps=args.steps,
+        metric=METRIC, value=value, unit=unit, n_gpus=world, steps=args.steps,
         warmup=args.warmup, ms_per_step=ms_step, higher_is_better=True, scaling="weak",
         vs_baseline=None, dtype="fp8_e4m3", data="synthetic", config=config_dict(w, Step),
-        roofline=dict(bound="tensor", achieved=gemm_tflops, peak=fp8_peak, unit="TFLOP/s",
-                      frac=gemm_tflops / fp8_peak, traffic=TRAFFIC.get(args.workload),
-                      peak_note=(f"{pk['source']} bf16 burst {pk['bf16']} TFLOP/s x 2 "
-                                 "(nominal fp8:bf16 dense ratio)")),
+        roofline=roof,
         kernels=kern,
-        e2e=dict(value=flops * world / (e2e_ms * 1e-3) / 1e12, unit="TFLOP/s",
+        e2e=dict(value=e2e_value, unit=unit,
                  h2d_bytes_per_step=int(sum(h.numel() * h.element_size() for _, h in pinned)),
                  d2h_bytes_per_step=int(hout.numel() * hout.element_size()), ms_per_step=e2e_ms),
         gpu_launches=st.launches * args.steps,

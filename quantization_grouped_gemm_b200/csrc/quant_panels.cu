@@ -6,40 +6,41 @@
 // activation row, one per column of each expert's weights, an offsets tensor
 // routing tokens to experts), section "Il guadagno vero è nel movimento dei
 // dati" (absmax -> scale -> clamp -> cast fused; the backward's
-// .t().contiguous().t() copy removed; the output tile of the column-scales
-// kernel transposed on chip so that its stores coalesce; relaxed atomics for
-// the cross-block reduction).  "AMD Boosts PyTorch FP8 Training on Instinct
-// GPUs", second and third paragraphs (the backward fusion).
+// .t().contiguous().t() copy removed; the column-scales kernel's output
+// transposed on chip so that its stores coalesce; relaxed atomics for the
+// cross-block reduction).  "AMD Boosts PyTorch FP8 Training on Instinct GPUs",
+// second and third paragraphs (the backward fusion).
 //
-// B200 design.  The input is cut into blocks of 128 rows of one group and
-// panels of 256 columns (512-byte row segments: every warp load instruction
-// reads one whole segment).  A block of a group with more than one block is
-// visited twice:
-//  - an "absmax" task: each of the eight warps loads its 16 rows straight into
-//    registers (16 loads of 16 bytes in flight per lane), reduces the column
-//    absmax, the warps meet in shared memory and the block's partial is merged
-//    into the unit's column absmax in global memory with relaxed atomic max
-//    (dual form: also every row's partial absmax over the panel); the block
-//    is then counted in the unit's arrival counter;
+// B200 design.  Every warp works alone: no block-wide barrier anywhere after
+// the set-up.  The input is cut into panels of 256 columns (one warp load
+// instruction reads a whole 512-byte row segment; lane l owns columns
+// 8l .. 8l + 7) and chunks of 32 rows of one group.  A chunk is visited twice:
+//  - an "absmax" task: the warp loads 16 rows at a time straight into
+//    registers (16 loads of 16 bytes in flight per lane), keeps the running
+//    column absmax of its lane's 8 columns, then merges the chunk's 256
+//    column maxima into the unit's absmax words in global memory with relaxed
+//    atomic max (transposed through 1 KB of shared memory, so that each
+//    atomic instruction covers 32 consecutive words) and counts the chunk in
+//    the unit's arrival counter; the dual form also merges every row's
+//    partial absmax over the panel;
 //  - a "cast" task, later in the task list, once the unit's count is full:
-//    the scales are derived, the rows are read again (from L2: the list
-//    keeps the two visits about one grid-width of tasks apart), cast, and the
-//    codes are written transposed into a 32 KB shared-memory tile (256
-//    columns x 128 tokens, 128-byte swizzle) that one bulk tensor store sends
-//    to the group's 128-token block of the padded layout.  Rows past the
-//    group's end are zeros in the tile, so the same store writes the zero
-//    codes of the padding.  The dual form also casts every row with its own
-//    scale (from the merged row absmax) and stores it in place.
-// A single-block unit of the column-wise form is one "whole" task (its
-// absmax stays in shared memory).  The unit a cast waits for is one (group,
+//    the lane derives its 8 scales, reads the rows again (from L2: the list
+//    keeps the two visits about one grid-width of warps apart), encodes two
+//    rows of a column per conversion, and writes the 16 tokens of each of its
+//    columns as one 16-byte store into the group's block of the padded
+//    layout; chunks past the group's rows write the zero codes of the
+//    padding.  The dual form also encodes every row with its own scale (from
+//    the merged row absmax) and stores it in place, 8 bytes per lane.
+// A (group, panel) unit of at most 16 rows is one "whole" task whose absmax
+// never leaves the registers.  The unit a cast waits for is one (group,
 // panel) in the column-wise form and the whole group in the dual form (a
 // row's scale needs every panel).  Tasks come from an atomic counter; the
-// absmax tasks run largest group first, and the cast tasks of a unit are
-// placed about one grid-width of tasks after the unit's last absmax task, so
-// that a cast only waits for a task handed out earlier (to a running block).
+// absmax tasks run largest group first, and the casts of a unit are placed
+// about one grid-width of warps after its last absmax task, so that a cast
+// only waits for tasks handed out earlier (to running warps).  The task of a
+// list position is found by a 32-way search (one candidate per lane).
 #include <algorithm>
 #include <cstring>
-#include <mutex>
 
 #include "device_common.cuh"
 #include "host_common.h"
@@ -47,32 +48,28 @@
 
 namespace fp8qgg {
 
-constexpr int kPW = 256;                 // columns per panel
-constexpr int kPWords = kPW / 2;         // bf16 pairs per panel row
-constexpr int kRB = 128;                 // rows per block = tokens per store tile
-constexpr int kPWarps = 8;
+constexpr int kPW = 256;               // columns per panel
+constexpr int kCR = 32;                // rows per chunk (task)
+constexpr int kWR = 16;                // rows in registers at a time
+constexpr int kPadTok = 128;           // padded layout: groups on 128-token boundaries
+constexpr int kPWarps = 4;             // warps per block
 constexpr int kPThreads = 32 * kPWarps;
-constexpr int kWR = kRB / kPWarps;       // rows per warp: 16
+constexpr int kPBlocksPerSM = 4;
 constexpr int kPMaxGroups = 1024;
-constexpr uint32_t kTileBytes = kPW * kRB;  // [256 columns][128 tokens] codes
-static_assert(kWR == 16, "a lane's tokens of one column fill one 16-byte piece");
 
 enum : int { kTaskAbs = 0, kTaskCast = 1, kTaskWhole = 2 };
 
 struct PanelSmem {
-  uint8_t tile[2][kTileBytes];      // transposed code tiles (1024-byte aligned)
-  uint32_t red[kPWarps][kPWords];   // per-warp column absmax, bf16 magnitude pairs
-  uint32_t colmax[kPWords];         // whole tasks: the unit's column absmax
-  float sc[kPW];                    // the panel's column scales
-  int32_t end[kPMaxGroups];         // clamped group ends (by group index)
-  int32_t pstart[kPMaxGroups];      // padded first token (by group index)
-  int32_t order[kPMaxGroups];       // groups by size, largest first
-  int32_t nb[kPMaxGroups];          // blocks of ordered group i
-  int32_t gpre[kPMaxGroups + 1];    // ordered multi-block groups: blocks before group i
-  int32_t n_multi, n_nonempty, a_total, s_total, total, npu;
-  int32_t task, flag;
+  uint32_t xch[kPWarps][kPW];      // per-warp transpose of the column absmax
+  int32_t end[kPMaxGroups];        // clamped group ends (by group index)
+  int32_t pstart[kPMaxGroups];     // padded first token (by group index)
+  int32_t order[kPMaxGroups];      // groups by size, largest first
+  int32_t nc[kPMaxGroups];         // ordered group i: chunks holding rows
+  int32_t npc[kPMaxGroups];        // ordered group i: chunks of its padded span
+  int32_t apre[kPMaxGroups + 1];   // multi-chunk groups: absmax chunks before group i
+  int32_t cpre[kPMaxGroups + 1];   // multi-chunk groups: cast chunks before group i
+  int32_t n_multi, n_nonempty, a_total, s_total, total;
 };
-static_assert(offsetof(PanelSmem, tile) == 0, "tiles first (1024-byte aligned)");
 
 struct PanelParams {
   const uint4 *x;        // bf16 rows as 16-byte vectors
@@ -81,6 +78,8 @@ struct PanelParams {
   int cols;
   const int32_t *offsets;
   int num_groups;
+  uint8_t *q_col;        // [cols, ld_qc] padded transposed codes
+  int64_t ld_qc;
   float *scales_col;     // [num_groups, cols]
   uint8_t *q_row;        // dual form: [rows_total, ld_qr] codes
   int64_t ld_qr;
@@ -90,11 +89,19 @@ struct PanelParams {
   int32_t *status;
   uint32_t *work;        // task counter
   uint32_t *arrive;      // per unit
-  uint32_t *amax;        // [num_groups (ordered), cols] column absmax bits
+  uint32_t *amax;        // [ordered group, cols] column absmax bits
   uint32_t *rowmax;      // dual form: [rows_total] row absmax bits
-  int32_t delay;         // tasks between a unit's last absmax task and its casts
+  int32_t delay;         // list positions between a unit's last absmax task and its casts
   UnitWait uw;
 };
+
+__device__ __forceinline__ int32_t warp_scan_incl(int32_t v, int lane) {
+  for (int d = 1; d < 32; d <<= 1) {
+    const int32_t o = __shfl_up_sync(0xFFFFFFFFu, v, d);
+    if (lane >= d) v += o;
+  }
+  return v;
+}
 
 // Clamped group ends, padded starts, the size order and the task counts.
 template <bool DUAL>
@@ -117,12 +124,8 @@ __device__ void panel_prologue(PanelSmem &sm, const PanelParams &p, int np) {
       int32_t prev = __shfl_up_sync(0xFFFFFFFFu, endv, 1);
       if (lane == 0) prev = carry_end;
       if (e < G && (raw < prev || raw > R)) bad = true;
-      const int32_t ps = e < G ? ((endv - prev + kRB - 1) / kRB) * kRB : 0;
-      int32_t incl = ps;
-      for (int d = 1; d < 32; d <<= 1) {
-        const int32_t o = __shfl_up_sync(0xFFFFFFFFu, incl, d);
-        if (lane >= d) incl += o;
-      }
+      const int32_t ps = e < G ? ((endv - prev + kPadTok - 1) / kPadTok) * kPadTok : 0;
+      const int32_t incl = warp_scan_incl(ps, lane);
       if (e < G) {
         sm.end[e] = endv;
         sm.pstart[e] = carry_pad + incl - ps;
@@ -145,42 +148,40 @@ __device__ void panel_prologue(PanelSmem &sm, const PanelParams &p, int np) {
   }
   __syncthreads();
   if (tid < 32) {
-    // multi-block groups are a prefix of the order (sizes decrease)
-    int32_t carry = 0, n_multi = 0, n_ne = 0;
+    // groups with absmax and cast tasks ("multi") are a prefix of the order:
+    // every non-empty group in the dual form, groups of more than 16 rows in
+    // the column-wise form (smaller ones are whole tasks)
+    int32_t ca = 0, cc = 0, n_multi = 0, n_ne = 0;
     for (int base = 0; base < G; base += 32) {
       const int i = base + lane;
-      int32_t nbv = 0;
+      int32_t sz = 0;
       if (i < G) {
         const int e = sm.order[i];
-        const int32_t sz = sm.end[e] - (e ? sm.end[e - 1] : 0);
-        nbv = (sz + kRB - 1) / kRB;
-        sm.nb[i] = nbv;
+        sz = sm.end[e] - (e ? sm.end[e - 1] : 0);
+        sm.nc[i] = (sz + kCR - 1) / kCR;
+        sm.npc[i] = ((sz + kPadTok - 1) / kPadTok) * (kPadTok / kCR);
       }
-      // absmax tasks exist for multi-block groups (every non-empty group in
-      // the dual form)
-      const bool multi = DUAL ? nbv >= 1 : nbv >= 2;
-      int32_t c = multi ? nbv : 0;
-      int32_t incl = c;
-      for (int d = 1; d < 32; d <<= 1) {
-        const int32_t o = __shfl_up_sync(0xFFFFFFFFu, incl, d);
-        if (lane >= d) incl += o;
+      const bool multi = DUAL ? sz >= 1 : sz > kWR;
+      const int32_t a = multi ? (sz + kCR - 1) / kCR : 0;
+      const int32_t c = multi ? ((sz + kPadTok - 1) / kPadTok) * (kPadTok / kCR) : 0;
+      const int32_t ia = warp_scan_incl(a, lane), ic = warp_scan_incl(c, lane);
+      if (i < G) {
+        sm.apre[i] = ca + ia - a;
+        sm.cpre[i] = cc + ic - c;
       }
-      if (i < G) sm.gpre[i] = carry + incl - c;
-      carry += __shfl_sync(0xFFFFFFFFu, incl, 31);
+      ca += __shfl_sync(0xFFFFFFFFu, ia, 31);
+      cc += __shfl_sync(0xFFFFFFFFu, ic, 31);
       n_multi += __popc(__ballot_sync(0xFFFFFFFFu, multi));
-      n_ne += __popc(__ballot_sync(0xFFFFFFFFu, nbv >= 1));
+      n_ne += __popc(__ballot_sync(0xFFFFFFFFu, sz >= 1));
     }
     if (lane == 0) {
-      sm.gpre[G] = carry;
+      sm.apre[G] = ca;
+      sm.cpre[G] = cc;
       sm.n_multi = n_multi;
       sm.n_nonempty = n_ne;
-      const int32_t npu = DUAL ? 1 : np;  // units per group
-      sm.npu = npu;
-      // absmax tasks: every (multi group, panel, block); whole tasks: every
-      // (single-block group, panel) of the column-wise form
-      sm.a_total = carry * np;
+      sm.a_total = ca * np;
       sm.s_total = sm.a_total + (DUAL ? 0 : (n_ne - n_multi) * np);
-      sm.total = sm.s_total + sm.a_total;  // + one cast task per absmax task
+      sm.total = sm.s_total + cc * np;
     }
   }
   __syncthreads();
@@ -188,103 +189,120 @@ __device__ void panel_prologue(PanelSmem &sm, const PanelParams &p, int np) {
 
 struct PTask {
   int kind;
-  int i;      // ordered group
-  int e;      // group index
-  int p0, p1; // panels
-  int b;      // block
+  int i, e;   // ordered group, group index
+  int q;      // panel
+  int k;      // chunk of the group
   int u;      // unit (arrival counter)
   int32_t need;  // arrivals that complete the unit
 };
 
-// Position t of the task list.  The "A stream" holds the absmax tasks of the
-// multi-block units (unit-major: group i, then panel p for the column-wise
-// form, then block b), then the whole tasks.  The cast block of unit u
-// (nbu tasks, same order) is inserted after A-stream index
-// d_u = min(first_u + nbu + delay, S); first_u = the unit's first absmax index.
-// Since the cast tasks before unit u number first_u as well, the cast block
-// starts at list position d_u + first_u.
-__device__ PTask decode_panel_task(const PanelSmem &sm, int32_t t, int np, int32_t delay) {
-  const int npu = sm.npu;
+// Unit u of the list: first absmax index and count, first cast index and count.
+template <bool DUAL>
+__device__ __forceinline__ void unit_span(const PanelSmem &sm, int np, int u, int32_t &fa,
+                                          int32_t &na, int32_t &fc, int32_t &nc) {
+  if constexpr (DUAL) {
+    fa = sm.apre[u] * np;
+    na = sm.nc[u] * np;
+    fc = sm.cpre[u] * np;
+    nc = sm.npc[u] * np;
+  } else {
+    const int i = u / np, q = u - (u / np) * np;
+    fa = sm.apre[i] * np + q * sm.nc[i];
+    na = sm.nc[i];
+    fc = sm.cpre[i] * np + q * sm.npc[i];
+    nc = sm.npc[i];
+  }
+}
+
+// Position t of the task list (called by the whole warp; every lane gets the
+// same task).  The "A stream" holds the absmax tasks of the multi units
+// (group i in size order, then panel q, then chunk k), then the whole tasks.
+// The cast block of unit u (chunks of its padded span, in the same order) is
+// inserted after A-stream index d_u = min(fa_u + na_u + delay, S); the casts
+// before it number fc_u, so the block starts at list position d_u + fc_u.
+template <bool DUAL>
+__device__ PTask decode_panel_task(const PanelSmem &sm, int32_t t, int np, int32_t delay,
+                                   int lane) {
   const int32_t S = sm.s_total;
-  const int n_units = sm.n_multi * npu;
-  // unit u = i * npu + q: first absmax index and block count
-  auto unit_first = [&](int u, int32_t &first, int32_t &nbu) {
-    const int i = u / npu, q = u - (u / npu) * npu;
-    const int32_t nbi = sm.nb[i];
-    nbu = npu == 1 ? nbi * np : nbi;
-    first = sm.gpre[i] * np + q * nbi;
+  const int U = DUAL ? sm.n_multi : sm.n_multi * np;
+  auto pos_of = [&](int u) -> int32_t {
+    int32_t fa, na, fc, nc;
+    unit_span<DUAL>(sm, np, u, fa, na, fc, nc);
+    return min(fa + na + delay, S) + fc;
   };
-  // largest unit whose cast block starts at or before t
-  int lo = -1, hi = n_units - 1;
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    int32_t f, n;
-    unit_first(mid, f, n);
-    const int32_t pos = min(f + n + delay, S) + f;
-    if (pos <= t) lo = mid; else hi = mid - 1;
+  // largest unit whose cast block starts at or before t (32 candidates a round)
+  int best = -1;
+  if (U > 0 && pos_of(0) <= t) {
+    int lo = 0, hi = U;  // pos(lo) <= t; the answer lies in [lo, hi)
+    while (hi - lo > 1) {
+      const int step = (hi - lo + 31) / 32;
+      const int c = lo + lane * step;
+      const bool ok = c < hi && pos_of(c) <= t;
+      const int n = __popc(__ballot_sync(0xFFFFFFFFu, ok));  // lanes 0 .. n-1
+      const int nlo = lo + (n - 1) * step;
+      hi = min(hi, nlo + step);
+      lo = nlo;
+    }
+    best = lo;
   }
   PTask r;
   int32_t a = t;  // A-stream index, if t is not a cast
-  if (lo >= 0) {
-    int32_t f, n;
-    unit_first(lo, f, n);
-    const int32_t pos = min(f + n + delay, S) + f;
-    if (t < pos + n) {
-      // cast task: block (t - pos) of unit lo, in the unit's absmax order
+  if (best >= 0) {
+    int32_t fa, na, fc, nc;
+    unit_span<DUAL>(sm, np, best, fa, na, fc, nc);
+    const int32_t pos = min(fa + na + delay, S) + fc;
+    if (t < pos + nc) {
       const int32_t k = t - pos;
-      const int i = lo / npu;
-      const int32_t nbi = sm.nb[i];
       r.kind = kTaskCast;
-      r.i = i;
-      r.u = lo;
-      r.need = n;
-      if (npu == 1) {
-        r.p0 = k / nbi;
-        r.b = k - r.p0 * nbi;
+      r.u = best;
+      r.need = na;
+      if constexpr (DUAL) {
+        r.i = best;
+        const int32_t per = sm.npc[best];
+        r.q = k / per;
+        r.k = k - r.q * per;
       } else {
-        r.p0 = lo - i * npu;
-        r.b = k;
+        r.i = best / np;
+        r.q = best - r.i * np;
+        r.k = k;
       }
-      r.p1 = r.p0 + 1;
-      r.e = sm.order[i];
+      r.e = sm.order[r.i];
       return r;
     }
-    a = t - (f + n);  // every cast before t belongs to units 0..lo
+    a = t - (fc + nc);  // every cast before t belongs to units 0 .. best
   }
   if (a < sm.a_total) {
-    // absmax task: ordered group by binary search over the block prefix
-    int glo = 0, ghi = sm.n_multi - 1;
-    while (glo < ghi) {
-      const int mid = (glo + ghi + 1) >> 1;
-      if (sm.gpre[mid] * np <= a) glo = mid; else ghi = mid - 1;
+    // absmax task: the multi group whose absmax span holds a (32-way search)
+    int lo = 0, hi = sm.n_multi;  // apre[lo] * np <= a
+    while (hi - lo > 1) {
+      const int step = (hi - lo + 31) / 32;
+      const int c = lo + lane * step;
+      const bool ok = c < hi && sm.apre[c] * np <= a;
+      const int n = __popc(__ballot_sync(0xFFFFFFFFu, ok));
+      const int nlo = lo + (n - 1) * step;
+      hi = min(hi, nlo + step);
+      lo = nlo;
     }
-    const int32_t nbi = sm.nb[glo];
-    const int32_t k = a - sm.gpre[glo] * np;
+    const int32_t nci = sm.nc[lo];
+    const int32_t rr = a - sm.apre[lo] * np;
     r.kind = kTaskAbs;
-    r.i = glo;
-    r.p0 = k / nbi;
-    r.p1 = r.p0 + 1;
-    r.b = k - r.p0 * nbi;
-    r.u = glo * npu + (npu == 1 ? 0 : r.p0);
-    r.need = npu == 1 ? nbi * np : nbi;
+    r.i = lo;
+    r.q = rr / nci;
+    r.k = rr - r.q * nci;
+    r.u = DUAL ? lo : lo * np + r.q;
+    r.need = DUAL ? nci * np : nci;
   } else {
-    // whole task (column-wise form only): single-block group, one panel
+    // whole task (column-wise form only): a group of at most 16 rows, one panel
     const int32_t w = a - sm.a_total;
     r.kind = kTaskWhole;
     r.i = sm.n_multi + w / np;
-    r.p0 = w - (w / np) * np;
-    r.p1 = r.p0 + 1;
-    r.b = 0;
+    r.q = w - (w / np) * np;
+    r.k = 0;
     r.u = -1;
     r.need = 0;
   }
   r.e = sm.order[r.i];
   return r;
-}
-
-__device__ __forceinline__ uint32_t hmax_bits(uint32_t acc) {
-  const uint32_t m = absmax_bits(acc);
-  return max(m & 0xFFFFu, m >> 16);
 }
 
 template <int FMT, bool FAST>
@@ -314,8 +332,8 @@ __device__ __forceinline__ uint32_t word(const uint4 &v, int j) {
   return j == 0 ? v.x : j == 1 ? v.y : j == 2 ? v.z : v.w;
 }
 
-// Loads the lane's 16 rows x 8 columns (rows [r0, r1) of the block; the rest
-// read as zero).  EVICT: the cast's second read, last use of the data.
+// The lane's 16 rows x 8 columns from row rw0 (rows at or past r1 read as
+// zero).  SECOND: the cast's re-read, the data's last use.
 template <bool SECOND>
 __device__ __forceinline__ void load_rows(uint4 (&v)[kWR], const PanelParams &p, int32_t rw0,
                                           int32_t r1, int64_t cvec, bool lane_ok) {
@@ -331,14 +349,91 @@ __device__ __forceinline__ void load_rows(uint4 (&v)[kWR], const PanelParams &p,
   }
 }
 
+// Running absmax of the lane's 8 columns (bf16 pairs).
+__device__ __forceinline__ void fold_amax(uint4 &am, const uint4 (&v)[kWR]) {
+#pragma unroll
+  for (int k = 0; k < kWR; ++k) {
+    am.x = absmax_acc(am.x, v[k].x);
+    am.y = absmax_acc(am.y, v[k].y);
+    am.z = absmax_acc(am.z, v[k].z);
+    am.w = absmax_acc(am.w, v[k].w);
+  }
+}
+
+// Dual form: every row's absmax over the lane's 8 columns, reduced over the
+// warp (16 values over 32 lanes: halve four times, then pair lanes), merged
+// into the row's absmax word.
+__device__ __forceinline__ void merge_row_amax(const uint4 (&v)[kWR], uint32_t *rowmax,
+                                               int32_t rw0, int32_t r1, int lane) {
+  uint32_t rm[kWR];
+#pragma unroll
+  for (int k = 0; k < kWR; ++k) {
+    uint32_t a2 = absmax_acc(absmax_acc(0u, v[k].x), v[k].y);
+    a2 = absmax_acc(absmax_acc(a2, v[k].z), v[k].w);
+    const uint32_t m = absmax_bits(a2);
+    rm[k] = max(m & 0xFFFFu, m >> 16);
+  }
+#pragma unroll
+  for (int h = 8; h >= 1; h >>= 1) {
+    const bool upper = (lane & (2 * h)) != 0;
+#pragma unroll
+    for (int k = 0; k < h; ++k) {
+      const uint32_t send = upper ? rm[k] : rm[k + h];
+      const uint32_t got = __shfl_xor_sync(0xFFFFFFFFu, send, 2 * h);
+      rm[k] = max(upper ? rm[k + h] : rm[k], got);
+    }
+  }
+  const uint32_t rmax = max(rm[0], __shfl_xor_sync(0xFFFFFFFFu, rm[0], 1));
+  const int32_t row = rw0 + ((lane >> 1) & 15);  // lanes 2j, 2j+1 hold row rw0 + j
+  if (!(lane & 1) && row < r1) atomicMax(rowmax + row, rmax);
+}
+
+// Column-wise codes of the lane's 16 rows: column 8*lane + j as one 16-byte
+// piece of tokens (adjacent rows of a column share one conversion).  Rows past
+// the group's end are zeros, whose codes are the padding.
+template <int FMT, bool FAST>
+__device__ __forceinline__ void store_col_codes(const uint4 (&v)[kWR], const float (&s)[8],
+                                                uint8_t *dst, int64_t ld_qc, bool lane_ok,
+                                                float smax, float sat_thr, uint32_t &sat) {
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const int wj = j >> 1;
+    uint32_t c2[8];
+#pragma unroll
+    for (int m = 0; m < 8; ++m) {
+      const uint32_t w0 = word(v[2 * m], wj), w1 = word(v[2 * m + 1], wj);
+      const float x0 = (j & 1) ? hi_f(w0) : lo_f(w0);
+      const float x1 = (j & 1) ? hi_f(w1) : lo_f(w1);
+      c2[m] = enc_pair<FMT, FAST>(x0, x1, s[j], s[j], smax, sat_thr, sat);
+    }
+    const uint4 tok = make_uint4(c2[0] | (c2[1] << 16), c2[2] | (c2[3] << 16),
+                                 c2[4] | (c2[5] << 16), c2[6] | (c2[7] << 16));
+    if (lane_ok) *reinterpret_cast<uint4 *>(dst + j * ld_qc) = tok;
+  }
+}
+
+// The lane's 8 column scales (16-byte stores when the address allows).
+__device__ __forceinline__ void store_scales8(float *d, const float (&s)[8]) {
+  if ((reinterpret_cast<uintptr_t>(d) & 15) == 0) {
+    reinterpret_cast<float4 *>(d)[0] = make_float4(s[0], s[1], s[2], s[3]);
+    reinterpret_cast<float4 *>(d)[1] = make_float4(s[4], s[5], s[6], s[7]);
+  } else {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) d[j] = s[j];
+  }
+}
+
+// the dual form holds more in registers: three blocks per SM
+template <bool DUAL>
+constexpr int blocks_per_sm() { return DUAL ? 3 : kPBlocksPerSM; }
+
 template <int FMT, bool FAST, bool DUAL>
-__global__ void __launch_bounds__(kPThreads, 2)
-    quant_panel_kernel(const __grid_constant__ CUtensorMap qmap, const PanelParams p) {
+__global__ void __launch_bounds__(kPThreads, blocks_per_sm<DUAL>())
+    quant_panel_kernel(const PanelParams p) {
   extern __shared__ uint8_t smem_raw[];
-  PanelSmem &sm = *align_smem_1024<PanelSmem>(smem_raw);
+  PanelSmem &sm = *reinterpret_cast<PanelSmem *>(smem_raw);
   const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
   const int np = (p.cols + kPW - 1) / kPW;
-  if (tid == 0 && p.rows_total > 0) prefetch_tensormap(&qmap);
   panel_prologue<DUAL>(sm, p, np);
 
   // empty groups: scales only (Fmax / 1e-12 in every column), no codes
@@ -346,165 +441,155 @@ __global__ void __launch_bounds__(kPThreads, 2)
        i += static_cast<int>(gridDim.x)) {
     const int e = sm.order[i];
     const float s = scale_from_amax(0.0f, p.smax);
-    for (int c = tid; c < p.cols; c += kPThreads) p.scales_col[static_cast<int64_t>(e) * p.cols + c] = s;
+    for (int c = tid; c < p.cols; c += kPThreads)
+      p.scales_col[static_cast<int64_t>(e) * p.cols + c] = s;
   }
 
   uint32_t sat = 0;
-  uint32_t tile_parity = 0;
   const int32_t total = sm.total;
+  uint32_t *xch = sm.xch[w];
   int32_t next = 0;
-  if (tid == 0) next = static_cast<int32_t>(atomicAdd(p.work, 1u));
+  if (lane == 0) next = static_cast<int32_t>(atomicAdd(p.work, 1u));
   while (true) {
-    if (tid == 0) {
-      const int32_t t = next;
+    int32_t t = 0;
+    if (lane == 0) {
+      t = next;
       if (t < total) next = static_cast<int32_t>(atomicAdd(p.work, 1u));
-      sm.task = t;
     }
-    __syncthreads();
-    const int32_t t = sm.task;
+    t = __shfl_sync(0xFFFFFFFFu, t, 0);
     if (t >= total) break;
-    const PTask tk = decode_panel_task(sm, t, np, p.delay);
+    const PTask tk = decode_panel_task<DUAL>(sm, t, np, p.delay, lane);
     const int e = tk.e;
     const int32_t gs = e ? sm.end[e - 1] : 0;
     const int32_t ge = sm.end[e];
-    const int32_t r0 = gs + tk.b * kRB;
-    const int32_t r1 = min(ge, r0 + kRB);
-    const int32_t rw0 = r0 + kWR * w;
-    const int64_t amax_base = static_cast<int64_t>(tk.i) * p.cols;
+    const int32_t r0 = gs + tk.k * kCR;
+    const int32_t r1 = min(ge, r0 + kCR);
+    const int c0 = tk.q * kPW;
+    const bool lane_ok = c0 + 8 * lane < p.cols;
+    const int64_t cvec = (c0 >> 3) + lane;
+    const int64_t amax_base = static_cast<int64_t>(tk.i) * p.cols + c0;
 
-    if (tk.kind != kTaskCast) {
+    if (tk.kind == kTaskAbs) {
       // ------------------------------------------------------------ absmax
-      for (int pp = tk.p0; pp < tk.p1; ++pp) {
-        const int c0 = pp * kPW;
-        const bool lane_ok = c0 + 8 * lane < p.cols;
+      uint4 am = make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll 1
+      for (int32_t rw0 = r0; rw0 < r1; rw0 += kWR) {
         uint4 v[kWR];
-        load_rows<false>(v, p, rw0, r1, (c0 >> 3) + lane, lane_ok);
-        uint4 am = make_uint4(0u, 0u, 0u, 0u);
-#pragma unroll
-        for (int k = 0; k < kWR; ++k) {
-          am.x = absmax_acc(am.x, v[k].x);
-          am.y = absmax_acc(am.y, v[k].y);
-          am.z = absmax_acc(am.z, v[k].z);
-          am.w = absmax_acc(am.w, v[k].w);
-        }
-        if constexpr (DUAL) {
-          // the row's partial absmax over this panel, merged per row
-          uint32_t rm[kWR];
-#pragma unroll
-          for (int k = 0; k < kWR; ++k) {
-            uint32_t a2 = absmax_acc(absmax_acc(0u, v[k].x), v[k].y);
-            a2 = absmax_acc(absmax_acc(a2, v[k].z), v[k].w);
-            rm[k] = hmax_bits(a2);
-          }
-          // 16 values over 32 lanes: halve four times, then pair lanes
-#pragma unroll
-          for (int h = 8; h >= 1; h >>= 1) {
-            const bool upper = (lane & (2 * h)) != 0;  // partner bits 16, 8, 4, 2
-#pragma unroll
-            for (int k = 0; k < h; ++k) {
-              const uint32_t send = upper ? rm[k] : rm[k + h];
-              const uint32_t got = __shfl_xor_sync(0xFFFFFFFFu, send, 2 * h);
-              rm[k] = max(upper ? rm[k + h] : rm[k], got);
-            }
-          }
-          const uint32_t rmax = max(rm[0], __shfl_xor_sync(0xFFFFFFFFu, rm[0], 1));
-          const int32_t row = rw0 + ((lane >> 1) & 15);
-          if (!(lane & 1) && row < r1) atomicMax(p.rowmax + row, rmax);
-        }
-        am = make_uint4(absmax_bits(am.x), absmax_bits(am.y), absmax_bits(am.z),
-                        absmax_bits(am.w));
-        *reinterpret_cast<uint4 *>(&sm.red[w][4 * lane]) = am;
-        __syncthreads();
-        if (tid < kPWords) {
-          uint32_t m = 0;
-#pragma unroll
-          for (int ww = 0; ww < kPWarps; ++ww) m = __vmaxu2(m, sm.red[ww][tid]);
-          const int c = c0 + 2 * tid;
-          if (tk.kind == kTaskWhole) {
-            sm.colmax[tid] = m;
-          } else if (c < p.cols) {
-            atomicMax(p.amax + amax_base + c, m & 0xFFFFu);
-            atomicMax(p.amax + amax_base + c + 1, m >> 16);
-          }
-        }
-        __syncthreads();
+        load_rows<false>(v, p, rw0, r1, cvec, lane_ok);
+        fold_amax(am, v);
+        if constexpr (DUAL) merge_row_amax(v, p.rowmax, rw0, r1, lane);
       }
-      if (tk.kind == kTaskAbs) {
-        __threadfence();  // this thread's merges are visible before the count
-        __syncthreads();
-        if (tid == 0) atomicAdd(p.arrive + tk.u, 1u);
-        continue;
+      // the lane's 8 column words, transposed so that lane l merges columns
+      // 32m + l (one 128-byte run per atomic instruction)
+      am = make_uint4(absmax_bits(am.x), absmax_bits(am.y), absmax_bits(am.z),
+                      absmax_bits(am.w));
+      *reinterpret_cast<uint4 *>(xch + 8 * lane) =
+          make_uint4(am.x & 0xFFFFu, am.x >> 16, am.y & 0xFFFFu, am.y >> 16);
+      *reinterpret_cast<uint4 *>(xch + 8 * lane + 4) =
+          make_uint4(am.z & 0xFFFFu, am.z >> 16, am.w & 0xFFFFu, am.w >> 16);
+      __syncwarp();
+#pragma unroll
+      for (int m = 0; m < 8; ++m) {
+        const int cc = 32 * m + lane;
+        if (c0 + cc < p.cols) atomicMax(p.amax + amax_base + cc, xch[cc]);
       }
+      __threadfence();  // every lane's merges are visible before the count
+      __syncwarp();     // (and xch is free again)
+      if (lane == 0) atomicAdd(p.arrive + tk.u, 1u);
+      continue;
     }
 
     // ------------------------------------------------------------ cast
-    if (tk.kind == kTaskCast) {
-      if (tid == 0) {
+    float s[8];
+    if (tk.kind == kTaskWhole) {
+      // at most 16 rows: the absmax comes from the same registers
+      uint4 v[kWR];
+      load_rows<false>(v, p, r0, r1, cvec, lane_ok);
+      uint4 am = make_uint4(0u, 0u, 0u, 0u);
+      fold_amax(am, v);
+      am = make_uint4(absmax_bits(am.x), absmax_bits(am.y), absmax_bits(am.z),
+                      absmax_bits(am.w));
+      const uint32_t a[8] = {am.x & 0xFFFFu, am.x >> 16, am.y & 0xFFFFu, am.y >> 16,
+                             am.z & 0xFFFFu, am.z >> 16, am.w & 0xFFFFu, am.w >> 16};
+#pragma unroll
+      for (int j = 0; j < 8; ++j) s[j] = scale_from_amax(bf16_bits_to_float(a[j]), p.smax);
+      if (lane_ok) store_scales8(p.scales_col + static_cast<int64_t>(e) * p.cols + c0 + 8 * lane, s);
+      uint8_t *dst = p.q_col + static_cast<int64_t>(c0 + 8 * lane) * p.ld_qc + sm.pstart[e];
+      store_col_codes<FMT, FAST>(v, s, dst, p.ld_qc, lane_ok, p.smax, p.sat_thr, sat);
+      // the rest of the 128-token block: zero codes
+      if (lane_ok) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+#pragma unroll
+          for (int z = 1; z < kPadTok / 16; ++z)
+            *reinterpret_cast<uint4 *>(dst + j * p.ld_qc + 16 * z) = make_uint4(0u, 0u, 0u, 0u);
+      }
+      continue;
+    }
+
+    {  // wait (bounded) until every absmax task of the unit has been counted
+      int ok = 1;
+      if (lane == 0) {
         const uint32_t *cnt = p.arrive + tk.u;
         const uint32_t target = static_cast<uint32_t>(tk.need) + p.uw.extra_arrivals;
-        uint32_t v;
-        asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(cnt) : "memory");
-        int ok = 1;
-        if (v < target) {
+        uint32_t c;
+        asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(c) : "l"(cnt) : "memory");
+        if (c < target) {
           const uint64_t t0 = global_timer_ns();
           while (true) {
-            __nanosleep(128);
-            asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(cnt) : "memory");
-            if (v >= target) break;
+            __nanosleep(100);
+            asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(c) : "l"(cnt) : "memory");
+            if (c >= target) break;
             if (global_timer_ns() - t0 > p.uw.limit_ns) { ok = 0; break; }
           }
         }
-        sm.flag = ok;
       }
-      __syncthreads();
-      if (!sm.flag) {
-        if (tid == 0) status_or(p.status, FP8QGG_STATUS_TIMEOUT);
-        break;  // this block takes no more tasks; earlier stores complete below
+      ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+      if (ok) {  // every lane acquires the count it is about to rely on
+        uint32_t c;
+        asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(c) : "l"(p.arrive + tk.u)
+                     : "memory");
+        (void)c;
+      }
+      __syncwarp();
+      if (!ok) {
+        if (lane == 0) status_or(p.status, FP8QGG_STATUS_TIMEOUT);
+        break;  // this warp takes no more tasks
       }
     }
-    float rs_lane = 0.0f;  // dual form: the scale of row rw0 + lane (lanes 0..15)
+    {  // the lane's 8 column scales from the unit's merged absmax
+      uint4 a0 = make_uint4(0u, 0u, 0u, 0u), a1 = a0;
+      if (lane_ok) {
+        const uint4 *src = reinterpret_cast<const uint4 *>(p.amax + amax_base + 8 * lane);
+        a0 = __ldcg(src);
+        a1 = __ldcg(src + 1);
+      }
+      const uint32_t a[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+#pragma unroll
+      for (int j = 0; j < 8; ++j) s[j] = scale_from_amax(bf16_bits_to_float(a[j]), p.smax);
+      if (tk.k == 0 && lane_ok)
+        store_scales8(p.scales_col + static_cast<int64_t>(e) * p.cols + c0 + 8 * lane, s);
+    }
+    float rs_lane = 0.0f;  // dual form: the scale of row r0 + lane
     if constexpr (DUAL) {
-      const int32_t row = rw0 + lane;
-      if (lane < kWR && row < r1) {
-        const uint32_t bits = __ldcg(p.rowmax + row);
-        rs_lane = scale_from_amax(bf16_bits_to_float(bits), p.smax);
-        if (tk.p0 == 0) p.scales_row[row] = rs_lane;
+      const int32_t row = r0 + lane;
+      if (row < r1) {
+        rs_lane = scale_from_amax(bf16_bits_to_float(__ldcg(p.rowmax + row)), p.smax);
+        if (tk.q == 0) p.scales_row[row] = rs_lane;
       }
     }
-    for (int pp = tk.p0; pp < tk.p1; ++pp) {
-      const int c0 = pp * kPW;
-      const bool lane_ok = c0 + 8 * lane < p.cols;
-      {  // the panel's column scales, one column per thread
-        const int c = c0 + tid;
-        if (c < p.cols) {
-          uint32_t bits;
-          if (tk.kind == kTaskWhole)
-            bits = (tid & 1) ? sm.colmax[tid >> 1] >> 16 : sm.colmax[tid >> 1] & 0xFFFFu;
-          else
-            bits = __ldcg(p.amax + amax_base + c);
-          const float s = scale_from_amax(bf16_bits_to_float(bits), p.smax);
-          sm.sc[tid] = s;
-          if (tk.b == 0) p.scales_col[static_cast<int64_t>(e) * p.cols + c] = s;
-        }
-        // the tile about to be written was sent two stores ago: its store must
-        // have read it
-        if (tid == 0) bulk_wait_read<1>();
-      }
-      __syncthreads();
-      float s[8];
-      {
-        const float4 a = *reinterpret_cast<const float4 *>(&sm.sc[8 * lane]);
-        const float4 b = *reinterpret_cast<const float4 *>(&sm.sc[8 * lane + 4]);
-        s[0] = a.x; s[1] = a.y; s[2] = a.z; s[3] = a.w;
-        s[4] = b.x; s[5] = b.y; s[6] = b.z; s[7] = b.w;
-      }
+    uint8_t *dst0 = p.q_col + static_cast<int64_t>(c0 + 8 * lane) * p.ld_qc + sm.pstart[e] +
+                    tk.k * kCR;
+#pragma unroll 1
+    for (int h = 0; h < kCR / kWR; ++h) {
+      const int32_t rw0 = r0 + h * kWR;
       uint4 v[kWR];
-      load_rows<true>(v, p, rw0, r1, (c0 >> 3) + lane, lane_ok);
+      load_rows<true>(v, p, rw0, r1, cvec, lane_ok);
       if constexpr (DUAL) {
-        // rowwise codes in place: 8 columns of each row, one 8-byte store
+        // rowwise codes in place: 8 columns of a row per lane, one 8-byte store
 #pragma unroll
         for (int k = 0; k < kWR; ++k) {
-          const float rs = __shfl_sync(0xFFFFFFFFu, rs_lane, k);
+          const float rs = __shfl_sync(0xFFFFFFFFu, rs_lane, h * kWR + k);
           const int32_t row = rw0 + k;
           uint32_t c2[4];
 #pragma unroll
@@ -518,54 +603,9 @@ __global__ void __launch_bounds__(kPThreads, 2)
                 make_uint2(c2[0] | (c2[1] << 16), c2[2] | (c2[3] << 16));
         }
       }
-      // column-wise codes: column 8*lane + j, tokens rw0 .. rw0 + 15 as one
-      // 16-byte piece
-      uint4 tok[8];
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const int wj = j >> 1;
-        uint32_t c2[8];
-#pragma unroll
-        for (int m = 0; m < 8; ++m) {
-          const uint32_t w0 = word(v[2 * m], wj), w1 = word(v[2 * m + 1], wj);
-          const float x0 = (j & 1) ? hi_f(w0) : lo_f(w0);
-          const float x1 = (j & 1) ? hi_f(w1) : lo_f(w1);
-          // rows past the group's end are zero: their codes are the padding
-          c2[m] = enc_pair<FMT, FAST>(x0, x1, s[j], s[j], p.smax, p.sat_thr, sat);
-        }
-        tok[j] = make_uint4(c2[0] | (c2[1] << 16), c2[2] | (c2[3] << 16),
-                            c2[4] | (c2[5] << 16), c2[6] | (c2[7] << 16));
-      }
-      // rotate by lane % 8, so that the eight lanes of a shared-memory phase
-      // write eight different 16-byte bank groups of the swizzled tile
-      const int rot = lane & 7;
-#pragma unroll
-      for (int st = 1; st < 8; st <<= 1) {
-        if (rot & st) {
-          uint4 tmp[8];
-#pragma unroll
-          for (int j = 0; j < 8; ++j) tmp[j] = tok[(j + st) & 7];
-#pragma unroll
-          for (int j = 0; j < 8; ++j) tok[j] = tmp[j];
-        }
-      }
-      uint8_t *tile = sm.tile[tile_parity];
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const int cc = 8 * lane + ((j + rot) & 7);  // tile row = column of the panel
-        // 128-byte swizzle: 16-byte piece w of row cc sits at piece w ^ (cc % 8)
-        *reinterpret_cast<uint4 *>(tile + cc * kRB + 16 * (w ^ (cc & 7))) = tok[j];
-      }
-      fence_proxy_async_smem();
-      __syncthreads();
-      if (tid == 0) {
-        tma_store_2d(&qmap, tile, sm.pstart[e] + tk.b * kRB, c0);
-        bulk_commit();
-      }
-      tile_parity ^= 1;
+      store_col_codes<FMT, FAST>(v, s, dst0 + h * kWR, p.ld_qc, lane_ok, p.smax, p.sat_thr, sat);
     }
   }
-  if (tid == 0) bulk_wait_all();  // the tiles stay valid until their stores have read them
   if (!FAST && p.sat_count) {
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) sat += __shfl_xor_sync(0xFFFFFFFFu, sat, off);
@@ -575,7 +615,7 @@ __global__ void __launch_bounds__(kPThreads, 2)
 
 namespace {
 
-using PanelKernel = void (*)(const CUtensorMap, const PanelParams);
+using PanelKernel = void (*)(const PanelParams);
 
 template <bool DUAL>
 PanelKernel panel_kernel(int fmt, bool fast) {
@@ -608,24 +648,12 @@ int panel_launch(const void *x, int64_t rows_total, int64_t cols, int64_t ld_x,
                  float scale_max, uint64_t *sat_count, int32_t *dev_status, void *scratch,
                  UnitWait uw, cudaStream_t stream) {
   const bool dual = q_row != nullptr;
-  CUtensorMap qmap;
-  memset(&qmap, 0, sizeof qmap);
-  if (rows_total > 0) {
-    // codes [cols][ld_qc tokens]; boxes of 128 tokens x 256 columns (fewer
-    // columns when the tensor has fewer), 128-byte swizzle
-    const uint64_t dims[2] = {static_cast<uint64_t>(ld_qc), static_cast<uint64_t>(cols)};
-    const uint64_t strides[1] = {static_cast<uint64_t>(ld_qc)};
-    const uint32_t box[2] = {kRB, static_cast<uint32_t>(std::min<int64_t>(kPW, cols))};
-    if (!encode_tensor_map(&qmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, q_col, dims, strides, box,
-                           CU_TENSOR_MAP_SWIZZLE_128B))
-      return FP8QGG_ERR_CUDA;
-  }
   DeviceInfo dev;
   if (!device_info(&dev)) return FP8QGG_ERR_CUDA;
   const float smax = effective_scale_max(fmt, scale_max);
   const bool fast = sat_count == nullptr && smax >= format_max(fmt);
   PanelKernel kern = dual ? panel_kernel<true>(fmt, fast) : panel_kernel<false>(fmt, fast);
-  const int smem = static_cast<int>(sizeof(PanelSmem)) + 1024;
+  const int smem = static_cast<int>(sizeof(PanelSmem));
   if (!set_max_dynamic_smem(reinterpret_cast<const void *>(kern), smem)) return FP8QGG_ERR_CUDA;
   const PanelScratch sl = panel_scratch(rows_total, cols, num_groups, dual);
   uint8_t *base = static_cast<uint8_t *>(scratch);
@@ -636,6 +664,8 @@ int panel_launch(const void *x, int64_t rows_total, int64_t cols, int64_t ld_x,
   prm.cols = static_cast<int>(cols);
   prm.offsets = offsets;
   prm.num_groups = num_groups;
+  prm.q_col = q_col;
+  prm.ld_qc = ld_qc;
   prm.scales_col = scales_col;
   prm.q_row = q_row;
   prm.ld_qr = ld_qr;
@@ -649,14 +679,16 @@ int panel_launch(const void *x, int64_t rows_total, int64_t cols, int64_t ld_x,
   prm.amax = reinterpret_cast<uint32_t *>(base + sl.amax_off);
   prm.rowmax = reinterpret_cast<uint32_t *>(base + sl.rowmax_off);
   prm.uw = uw;
-  // blocks: two per SM, never more than the tasks (at least one, for the
-  // scales of empty groups)
+  // blocks: kPBlocksPerSM per SM, never more than the tasks need (at least
+  // one, for the scales of empty groups)
   const int64_t np = (cols + kPW - 1) / kPW;
-  const int64_t blocks_max = (rows_total + int64_t(kRB) * num_groups) / kRB * np;
-  const int grid = static_cast<int>(
-      std::max<int64_t>(1, std::min<int64_t>(2 * blocks_max, int64_t(dev.sm_count) * 2)));
-  prm.delay = grid;
-  kern<<<grid, kPThreads, smem, stream>>>(qmap, prm);
+  const int64_t chunks = (rows_total + int64_t(kPadTok) * num_groups) / kCR * np;
+  const int per_sm = dual ? blocks_per_sm<true>() : blocks_per_sm<false>();
+  const int grid = static_cast<int>(std::max<int64_t>(
+      1, std::min<int64_t>((2 * chunks + kPWarps - 1) / kPWarps, int64_t(dev.sm_count) * per_sm)));
+  // a cast waits for absmax tasks that every running warp has taken by then
+  prm.delay = grid * kPWarps;
+  kern<<<grid, kPThreads, smem, stream>>>(prm);
   return cudaGetLastError() == cudaSuccess ? FP8QGG_OK : FP8QGG_ERR_CUDA;
 }
 
@@ -690,7 +722,7 @@ extern "C" int fp8_quant_dual_jagged(const void *x, int64_t rows_total, int64_t 
   if (workspace_bytes < need) return FP8QGG_ERR_SHAPE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (cudaMemsetAsync(workspace, 0, need, s) != cudaSuccess) return FP8QGG_ERR_CUDA;
-  // a row pointer is needed to select the dual form even when no row exists
+  // a row pointer selects the dual form even when no row exists
   uint8_t *qr = q_row ? q_row : reinterpret_cast<uint8_t *>(workspace);
   return panel_launch(x, rows_total, cols, ld_x, offsets, num_groups, q_col, ld_qc, scales_col,
                       qr, ld_qr, scales_row, fmt, scale_max, sat_count, dev_status, workspace,

@@ -257,3 +257,40 @@ def test_k_jagged_group_starts_at_every_residue_of_a_block():
     assert len(set(starts.tolist())) > 40
     out, ref = k_jagged_case(4242, sizes, 40, 72, ld_pad=100)
     check_k_all(out, ref)
+
+
+@pytest.mark.parametrize("sizes,n,k,odt", [
+    ([300, 0, 1, 1000], 1408, 2048, torch.float32),
+    ([129, 5, 260], 24, 40, torch.float32),
+    ([700, 33] * 20, 96, 520, torch.float32),
+    ([257, 0, 90], 200, 136, torch.bfloat16),
+])
+def test_k_jagged_padded_pair_kernel_shapes(sizes, n, k, odt):
+    """The padded contraction-jagged GEMM (SM pairs, tiles of 256 x nt) on
+    shapes whose n and k are not tile multiples, with many groups (more tiles
+    than pairs), an empty group and bf16 output; every element against the
+    oracle (bf16 output: within the bound plus the bf16 rounding of the
+    output, 2^-8 relative)."""
+    m = int(sum(sizes))
+    e = len(sizes)
+    dh = rand_bf16(3 * m + n, (m, n), 1e-3)
+    x = rand_bf16(3 * m + n + 1, (m, k))
+    off = wl.offsets_from_sizes(sizes)
+    offd = torch.from_numpy(off).cuda()
+    P = qgg.LAYOUT_TRANSPOSED_PADDED
+    qa, sa = qgg.fp8_quant_colwise_jagged(dh.cuda(), offd, P)
+    qb, sb = qgg.fp8_quant_colwise_jagged(x.cuda(), offd, P)
+    out = torch.full((e, n, k), float("nan"), dtype=odt, device="cuda")
+    qgg.fp8_scaled_grouped_gemm(qgg.K_JAGGED_PADDED, qa, sa, qb, sb, offd, m_total=m, out=out)
+    torch.cuda.synchronize()
+    oa, osa, _ = orc.quant_colwise_jagged(bits(dh), off, orc.TRANSPOSED)
+    ob, osb, _ = orc.quant_colwise_jagged(bits(x), off, orc.TRANSPOSED)
+    ee, ii, jj = np.meshgrid(np.arange(e), np.arange(n), np.arange(k), indexing="ij")
+    c, b = orc.gemm_k_jagged_sample(oa, osa, ob, osb, off, m, ee.ravel(), ii.ravel(), jj.ravel())
+    got = out.float().cpu().numpy().ravel()
+    tol = b + (np.abs(c) * 2.0 ** -8 if odt == torch.bfloat16 else 0.0)
+    bad = np.nonzero(~(np.abs(got - c) <= tol))[0]
+    assert bad.size == 0, (bad.size, got[bad[:5]], c[bad[:5]], tol[bad[:5]])
+    for g, sz in enumerate(sizes):
+        if sz == 0:
+            assert (out[g] == 0).all()
