@@ -894,11 +894,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
 // the 32 lanes of a warp store 32 consecutive j of one i, a full 128-byte
 // line (fp32) per instruction.  Tiles are listed group by group, largest
 // group first, taken by the pairs in alternating directions.
-constexpr int kStagesK2 = 6;
+constexpr int kStagesK2 = 5;
 
 struct GemmK2Smem {
   uint8_t b[kStagesK2][128 * BK];  // this CTA's 128 rows of B (MMA rows)
   uint8_t a[kStagesK2][128 * BK];  // this CTA's nt / 2 rows of A (MMA columns)
+  float stg[kEpiWarps][2][16 * 32];  // per epilogue warp: two 16 (i) x 32 (j) output units
   float inv_sa[2][BN];             // 1 / scale_a of the tile's i columns
   int32_t pend[kMaxGemmGroups];    // padded group ends (tokens)
   int32_t order[kMaxGemmGroups];   // groups by size, largest first
@@ -939,7 +940,8 @@ __device__ __forceinline__ int32_t k2_position(int32_t i, int32_t c, int32_t nc)
 template <int OUT>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     grouped_gemm_k2_kernel(const __grid_constant__ CUtensorMap amap,
-                           const __grid_constant__ CUtensorMap bmap, const GemmParams p,
+                           const __grid_constant__ CUtensorMap bmap,
+                           const __grid_constant__ CUtensorMap omap, const GemmParams p,
                            int nt) {
   extern __shared__ uint8_t smem_raw[];
   GemmK2Smem &sm = *align_smem_1024<GemmK2Smem>(smem_raw);
@@ -956,6 +958,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   if (warp == 0 && lane == 0) {
     prefetch_tensormap(&amap);
     prefetch_tensormap(&bmap);
+    prefetch_tensormap(&omap);
     for (int s2 = 0; s2 < kStagesK2; ++s2) {
       mbar_init(&sm.full[s2], 1);
       mbar_init(&sm.empty[s2], 1);
@@ -1116,7 +1119,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue (both CTAs)
-    constexpr int kOutBytes = OUT == FP8QGG_OUT_F32 ? 4 : 2;
+    // A unit is 16 columns i (one 16-column TMEM load) x the warp's 32 lanes j:
+    // lane j writes its 16 scaled values into row i of a 16 x 32 staging
+    // buffer (consecutive lanes, consecutive words), and one bulk tensor store
+    // sends the buffer to out[e, i0 .. i0 + 15, j0 .. j0 + 31] (clipped at the
+    // tensor's edges).  The stores are asynchronous, so releasing the
+    // accumulator never waits for them.
     const int et = threadIdx.x - 64;
     const int ew = warp - 2;
     const int quarter = warp & 3;   // TMEM lanes [32 * quarter, +32)
@@ -1124,6 +1132,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     uint32_t tempty0[2];
     for (int b = 0; b < 2; ++b) tempty0[b] = mapa_shared(smem_addr(&sm.tempty[b]), 0);
     uint32_t acc = 0, acc_phase = 0;
+    int sb = 0;  // staging buffer of the next unit
     for (int32_t i = 0, t = k2_position(0, cid, ncl); t < total;
          t = k2_position(++i, cid, ncl)) {
       const K2Tile ti = k2_tile(sm, t, tj_n, ti_n);
@@ -1133,10 +1142,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         sm.inv_sa[acc][et] =
             col < p.n ? __frcp_rn(__ldg(p.scale_a + ti.e * p.sas + col)) : 0.0f;
       }
-      const int64_t j = static_cast<int64_t>(ti.tj) * 256 + 128 * static_cast<int64_t>(rank) +
-                        32 * quarter + lane;
-      const bool j_ok = j < p.k;
-      const float inv_b = j_ok ? __frcp_rn(__ldg(p.scale_b + ti.e * p.sbs + j)) : 0.0f;
+      const int32_t j0 = ti.tj * 256 + 128 * static_cast<int32_t>(rank) + 32 * quarter;
+      const int64_t j = j0 + lane;
+      const float inv_b = j < p.k ? __frcp_rn(__ldg(p.scale_b + ti.e * p.sbs + j)) : 0.0f;
       const bool got = mbar_wait(&sm.tfull[acc], acc_phase, abort);
       if (!epi_bar_and(got)) {
         *abort = 1;
@@ -1144,8 +1152,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         break;
       }
       tc_fence_after_sync();
-      char *obase = static_cast<char *>(p.out) +
-                    (static_cast<int64_t>(ti.e) * p.out_gs + i0 * p.ld_out + j) * kOutBytes;
       const uint32_t taddr =
           tmem_base + (static_cast<uint32_t>(32 * quarter) << 16) + acc * BN;
 #pragma unroll 1
@@ -1158,23 +1164,32 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
           for (int q = 0; q < 16; ++q) r[q] = 0u;
         }
+        float *buf = sm.stg[ew][sb];
+        if (lane == 0) bulk_wait_read<1>();  // the store that last read this buffer is done
+        __syncwarp();
 #pragma unroll
         for (int q = 0; q < 16; ++q) {
-          const int ii = 16 * c + q;
-          if (j_ok && i0 + ii < p.n) {
-            const float v = __fmul_rn(__fmul_rn(__uint_as_float(r[q]), sm.inv_sa[acc][ii]), inv_b);
-            char *dst = obase + static_cast<int64_t>(ii) * p.ld_out * kOutBytes;
-            if constexpr (OUT == FP8QGG_OUT_F32)
-              __stcs(reinterpret_cast<float *>(dst), v);
-            else
-              *reinterpret_cast<__nv_bfloat16 *>(dst) = __float2bfloat16_rn(v);
-          }
+          const float v = __fmul_rn(__fmul_rn(__uint_as_float(r[q]), sm.inv_sa[acc][16 * c + q]),
+                                    inv_b);
+          if constexpr (OUT == FP8QGG_OUT_F32)
+            buf[q * 32 + lane] = v;
+          else
+            reinterpret_cast<__nv_bfloat16 *>(buf)[q * 32 + lane] = __float2bfloat16_rn(v);
         }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_3d(&omap, buf, j0, static_cast<int32_t>(i0 + 16 * c), ti.e);
+          bulk_commit();
+        }
+        sb ^= 1;
       }
       tc_fence_before_sync();
       mbar_arrive_cluster(tempty0[acc]);
       if (++acc == 2) { acc = 0; acc_phase ^= 1; }
     }
+    if (lane == 0) bulk_wait_all();
+    __syncwarp();
   }
 
   tc_fence_before_sync();
@@ -1381,10 +1396,26 @@ extern "C" int fp8_scaled_grouped_gemm(int mode, const uint8_t *a, int64_t ld_a,
       return FP8QGG_ERR_CUDA;
     const int64_t pair_tiles = int64_t(num_groups) * ((k + 255) / 256) * ((n + nt - 1) / nt);
     if (pair_tiles > INT32_MAX) return FP8QGG_ERR_SHAPE;
+    // output units of 32 (j) x 16 (i) elements, no swizzle
+    CUtensorMap omap2;
+    {
+      const CUtensorMapDataType odt = out_dtype == FP8QGG_OUT_F32
+                                          ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
+                                          : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+      const uint64_t esz = out_dtype == FP8QGG_OUT_F32 ? 4 : 2;
+      const uint64_t dims[3] = {static_cast<uint64_t>(k), static_cast<uint64_t>(n),
+                                static_cast<uint64_t>(num_groups)};
+      const uint64_t gs = num_groups > 1 ? static_cast<uint64_t>(out_group_stride)
+                                         : static_cast<uint64_t>(n * ld_out);
+      const uint64_t str[2] = {static_cast<uint64_t>(ld_out) * esz, gs * esz};
+      const uint32_t box[3] = {32, 16, 1};
+      if (!encode_tensor_map(&omap2, odt, 3, out, dims, str, box, CU_TENSOR_MAP_SWIZZLE_NONE))
+        return FP8QGG_ERR_CUDA;
+    }
     const int clusters =
         static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(pair_tiles, dev.sm_count / 2)));
-    kern2<<<2 * clusters, kGemmThreads, smem2, static_cast<cudaStream_t>(stream)>>>(amap2, bmap2,
-                                                                                  prm, nt);
+    kern2<<<2 * clusters, kGemmThreads, smem2, static_cast<cudaStream_t>(stream)>>>(
+        amap2, bmap2, omap2, prm, nt);
     return cudaGetLastError() == cudaSuccess ? FP8QGG_OK : FP8QGG_ERR_CUDA;
   }
 

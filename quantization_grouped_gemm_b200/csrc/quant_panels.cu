@@ -11,34 +11,36 @@
 // cross-block reduction).  "AMD Boosts PyTorch FP8 Training on Instinct GPUs",
 // second and third paragraphs (the backward fusion).
 //
-// B200 design.  Every warp works alone: no block-wide barrier anywhere after
-// the set-up.  The input is cut into panels of 256 columns (one warp load
+// B200 design.  The input is cut into panels of 256 columns (one warp load
 // instruction reads a whole 512-byte row segment; lane l owns columns
-// 8l .. 8l + 7) and chunks of 32 rows of one group.  A chunk is visited twice:
-//  - an "absmax" task: the warp loads 16 rows at a time straight into
-//    registers (16 loads of 16 bytes in flight per lane), keeps the running
-//    column absmax of its lane's 8 columns, then merges the chunk's 256
-//    column maxima into the unit's absmax words in global memory with relaxed
-//    atomic max (transposed through 1 KB of shared memory, so that each
-//    atomic instruction covers 32 consecutive words) and counts the chunk in
-//    the unit's arrival counter; the dual form also merges every row's
-//    partial absmax over the panel;
+// 8l .. 8l + 7) and blocks of 128 rows of one group; a block of a panel is
+// one task of a block of eight warps, each warp owning 16 rows.  A block of a
+// group with more than one block is visited twice:
+//  - an "absmax" task: every warp loads its 16 rows straight into registers
+//    (16 loads of 16 bytes in flight per lane) and reduces its column absmax;
+//    the warps meet in shared memory, then each warp merges 32 of the
+//    panel's columns into the unit's absmax words in global memory with
+//    relaxed atomic max and counts itself in the unit's arrival counter (the
+//    dual form also merges every row's absmax over the panel);
 //  - a "cast" task, later in the task list, once the unit's count is full:
-//    the lane derives its 8 scales, reads the rows again (from L2: the list
-//    keeps the two visits about one grid-width of warps apart), encodes two
-//    rows of a column per conversion, and writes the 16 tokens of each of its
-//    columns as one 16-byte store into the group's block of the padded
-//    layout; chunks past the group's rows write the zero codes of the
-//    padding.  The dual form also encodes every row with its own scale (from
-//    the merged row absmax) and stores it in place, 8 bytes per lane.
-// A (group, panel) unit of at most 16 rows is one "whole" task whose absmax
-// never leaves the registers.  The unit a cast waits for is one (group,
-// panel) in the column-wise form and the whole group in the dual form (a
-// row's scale needs every panel).  Tasks come from an atomic counter; the
-// absmax tasks run largest group first, and the casts of a unit are placed
-// about one grid-width of warps after its last absmax task, so that a cast
-// only waits for tasks handed out earlier (to running warps).  The task of a
-// list position is found by a 32-way search (one candidate per lane).
+//    every lane derives its 8 scales, reads its rows again (from L2: the
+//    list keeps the two visits about one grid-width of tasks apart), encodes
+//    two rows of a column per conversion and writes each column's 16 tokens
+//    into a 32 KB shared-memory tile (256 columns x 128 tokens, 128-byte
+//    swizzle), which one bulk tensor store sends to the group's 128-token
+//    block of the padded layout: whole 128-byte lines, zero codes of the
+//    padding included (rows past the group's end are zeros).  The dual form
+//    also encodes every row with its own scale and stores it in place.
+// A single-block unit of the column-wise form is one "whole" task (absmax
+// and cast from the same registers).  The unit a cast waits for is one
+// (group, panel) in the column-wise form and the whole group in the dual
+// form (a row's scale needs every panel).  Tasks come from an atomic counter
+// read by warp 0, which also finds the next task (a 32-way search, one
+// candidate per lane) while the block works on the current one; each task
+// ends with the block's only barrier.  The absmax tasks run largest group
+// first, and the casts of a unit are placed about one grid-width of tasks
+// after its last absmax task, so that a cast only waits for tasks handed out
+// earlier (to running blocks).
 #include <algorithm>
 #include <cstring>
 
@@ -49,27 +51,40 @@
 namespace fp8qgg {
 
 constexpr int kPW = 256;               // columns per panel
-constexpr int kCR = 32;                // rows per chunk (task)
-constexpr int kWR = 16;                // rows in registers at a time
-constexpr int kPadTok = 128;           // padded layout: groups on 128-token boundaries
-constexpr int kPWarps = 4;             // warps per block
+constexpr int kPWords = kPW / 2;       // bf16 pairs per panel row
+constexpr int kRB = 128;               // rows per block = tokens per store tile
+constexpr int kPWarps = 8;
 constexpr int kPThreads = 32 * kPWarps;
-constexpr int kPBlocksPerSM = 4;
+constexpr int kWR = kRB / kPWarps;     // rows per warp: 16
+constexpr int kPBlocksPerSM = 2;
 constexpr int kPMaxGroups = 1024;
+constexpr uint32_t kTileBytes = kPW * kRB;
+static_assert(kWR == 16, "a lane's tokens of one column fill one 16-byte piece");
 
-enum : int { kTaskAbs = 0, kTaskCast = 1, kTaskWhole = 2 };
+enum : int { kTaskAbs = 0, kTaskCast = 1, kTaskWhole = 2, kTaskEnd = 3 };
+
+struct PTask {
+  int32_t kind;
+  int32_t i, e;   // ordered group, group index
+  int32_t q;      // panel
+  int32_t b;      // block of the group
+  int32_t u;      // unit (arrival counter)
+  int32_t need;   // arrivals that complete the unit
+  int32_t pad;
+};
 
 struct PanelSmem {
-  uint32_t xch[kPWarps][kPW];      // per-warp transpose of the column absmax
-  int32_t end[kPMaxGroups];        // clamped group ends (by group index)
-  int32_t pstart[kPMaxGroups];     // padded first token (by group index)
-  int32_t order[kPMaxGroups];      // groups by size, largest first
-  int32_t nc[kPMaxGroups];         // ordered group i: chunks holding rows
-  int32_t npc[kPMaxGroups];        // ordered group i: chunks of its padded span
-  int32_t apre[kPMaxGroups + 1];   // multi-chunk groups: absmax chunks before group i
-  int32_t cpre[kPMaxGroups + 1];   // multi-chunk groups: cast chunks before group i
+  uint8_t tile[2][kTileBytes];          // transposed code tiles (1024-byte aligned)
+  uint32_t red[2][kPWarps][kPWords];    // per-warp column absmax (bf16 magnitude pairs)
+  PTask tk[2];                          // the current and the next task
+  int32_t end[kPMaxGroups];             // clamped group ends (by group index)
+  int32_t pstart[kPMaxGroups];          // padded first token (by group index)
+  int32_t order[kPMaxGroups];           // groups by size, largest first
+  int32_t nb[kPMaxGroups];              // ordered group i: 128-row blocks
+  int32_t apre[kPMaxGroups + 1];        // multi-block groups: blocks before group i
   int32_t n_multi, n_nonempty, a_total, s_total, total;
 };
+static_assert(offsetof(PanelSmem, tile) == 0, "tiles first (1024-byte aligned)");
 
 struct PanelParams {
   const uint4 *x;        // bf16 rows as 16-byte vectors
@@ -78,8 +93,6 @@ struct PanelParams {
   int cols;
   const int32_t *offsets;
   int num_groups;
-  uint8_t *q_col;        // [cols, ld_qc] padded transposed codes
-  int64_t ld_qc;
   float *scales_col;     // [num_groups, cols]
   uint8_t *q_row;        // dual form: [rows_total, ld_qr] codes
   int64_t ld_qr;
@@ -124,7 +137,7 @@ __device__ void panel_prologue(PanelSmem &sm, const PanelParams &p, int np) {
       int32_t prev = __shfl_up_sync(0xFFFFFFFFu, endv, 1);
       if (lane == 0) prev = carry_end;
       if (e < G && (raw < prev || raw > R)) bad = true;
-      const int32_t ps = e < G ? ((endv - prev + kPadTok - 1) / kPadTok) * kPadTok : 0;
+      const int32_t ps = e < G ? ((endv - prev + kRB - 1) / kRB) * kRB : 0;
       const int32_t incl = warp_scan_incl(ps, lane);
       if (e < G) {
         sm.end[e] = endv;
@@ -149,88 +162,74 @@ __device__ void panel_prologue(PanelSmem &sm, const PanelParams &p, int np) {
   __syncthreads();
   if (tid < 32) {
     // groups with absmax and cast tasks ("multi") are a prefix of the order:
-    // every non-empty group in the dual form, groups of more than 16 rows in
-    // the column-wise form (smaller ones are whole tasks)
-    int32_t ca = 0, cc = 0, n_multi = 0, n_ne = 0;
+    // every non-empty group in the dual form, groups of more than one block
+    // in the column-wise form (single-block ones are whole tasks)
+    int32_t carry = 0, n_multi = 0, n_ne = 0;
     for (int base = 0; base < G; base += 32) {
       const int i = base + lane;
-      int32_t sz = 0;
+      int32_t nbv = 0;
       if (i < G) {
         const int e = sm.order[i];
-        sz = sm.end[e] - (e ? sm.end[e - 1] : 0);
-        sm.nc[i] = (sz + kCR - 1) / kCR;
-        sm.npc[i] = ((sz + kPadTok - 1) / kPadTok) * (kPadTok / kCR);
+        nbv = (sm.end[e] - (e ? sm.end[e - 1] : 0) + kRB - 1) / kRB;
+        sm.nb[i] = nbv;
       }
-      const bool multi = DUAL ? sz >= 1 : sz > kWR;
-      const int32_t a = multi ? (sz + kCR - 1) / kCR : 0;
-      const int32_t c = multi ? ((sz + kPadTok - 1) / kPadTok) * (kPadTok / kCR) : 0;
-      const int32_t ia = warp_scan_incl(a, lane), ic = warp_scan_incl(c, lane);
-      if (i < G) {
-        sm.apre[i] = ca + ia - a;
-        sm.cpre[i] = cc + ic - c;
-      }
-      ca += __shfl_sync(0xFFFFFFFFu, ia, 31);
-      cc += __shfl_sync(0xFFFFFFFFu, ic, 31);
+      const bool multi = DUAL ? nbv >= 1 : nbv >= 2;
+      const int32_t c = multi ? nbv : 0;
+      const int32_t incl = warp_scan_incl(c, lane);
+      if (i < G) sm.apre[i] = carry + incl - c;
+      carry += __shfl_sync(0xFFFFFFFFu, incl, 31);
       n_multi += __popc(__ballot_sync(0xFFFFFFFFu, multi));
-      n_ne += __popc(__ballot_sync(0xFFFFFFFFu, sz >= 1));
+      n_ne += __popc(__ballot_sync(0xFFFFFFFFu, nbv >= 1));
     }
     if (lane == 0) {
-      sm.apre[G] = ca;
-      sm.cpre[G] = cc;
+      sm.apre[G] = carry;
       sm.n_multi = n_multi;
       sm.n_nonempty = n_ne;
-      sm.a_total = ca * np;
+      sm.a_total = carry * np;
       sm.s_total = sm.a_total + (DUAL ? 0 : (n_ne - n_multi) * np);
-      sm.total = sm.s_total + cc * np;
+      sm.total = sm.s_total + sm.a_total;  // one cast per absmax task
     }
   }
   __syncthreads();
 }
 
-struct PTask {
-  int kind;
-  int i, e;   // ordered group, group index
-  int q;      // panel
-  int k;      // chunk of the group
-  int u;      // unit (arrival counter)
-  int32_t need;  // arrivals that complete the unit
-};
-
-// Unit u of the list: first absmax index and count, first cast index and count.
+// Unit u: first absmax index (= cast tasks before its cast block) and count.
 template <bool DUAL>
 __device__ __forceinline__ void unit_span(const PanelSmem &sm, int np, int u, int32_t &fa,
-                                          int32_t &na, int32_t &fc, int32_t &nc) {
+                                          int32_t &na) {
   if constexpr (DUAL) {
     fa = sm.apre[u] * np;
-    na = sm.nc[u] * np;
-    fc = sm.cpre[u] * np;
-    nc = sm.npc[u] * np;
+    na = sm.nb[u] * np;
   } else {
     const int i = u / np, q = u - (u / np) * np;
-    fa = sm.apre[i] * np + q * sm.nc[i];
-    na = sm.nc[i];
-    fc = sm.cpre[i] * np + q * sm.npc[i];
-    nc = sm.npc[i];
+    fa = sm.apre[i] * np + q * sm.nb[i];
+    na = sm.nb[i];
   }
 }
 
-// Position t of the task list (called by the whole warp; every lane gets the
+// Task at position t of the list (called by a whole warp; every lane gets the
 // same task).  The "A stream" holds the absmax tasks of the multi units
-// (group i in size order, then panel q, then chunk k), then the whole tasks.
-// The cast block of unit u (chunks of its padded span, in the same order) is
-// inserted after A-stream index d_u = min(fa_u + na_u + delay, S); the casts
-// before it number fc_u, so the block starts at list position d_u + fc_u.
+// (group i in size order, panel q, block b), then the whole tasks.  The cast
+// block of unit u (same blocks, same order) is inserted after A-stream index
+// d_u = min(fa_u + na_u + delay, S); the casts before it number fa_u, so it
+// starts at list position d_u + fa_u.
 template <bool DUAL>
 __device__ PTask decode_panel_task(const PanelSmem &sm, int32_t t, int np, int32_t delay,
                                    int lane) {
+  PTask r;
+  r.pad = 0;
+  if (t >= sm.total) {
+    r.kind = kTaskEnd;
+    r.i = r.e = r.q = r.b = r.u = r.need = 0;
+    return r;
+  }
   const int32_t S = sm.s_total;
   const int U = DUAL ? sm.n_multi : sm.n_multi * np;
   auto pos_of = [&](int u) -> int32_t {
-    int32_t fa, na, fc, nc;
-    unit_span<DUAL>(sm, np, u, fa, na, fc, nc);
-    return min(fa + na + delay, S) + fc;
+    int32_t fa, na;
+    unit_span<DUAL>(sm, np, u, fa, na);
+    return min(fa + na + delay, S) + fa;
   };
-  // largest unit whose cast block starts at or before t (32 candidates a round)
   int best = -1;
   if (U > 0 && pos_of(0) <= t) {
     int lo = 0, hi = U;  // pos(lo) <= t; the answer lies in [lo, hi)
@@ -245,34 +244,32 @@ __device__ PTask decode_panel_task(const PanelSmem &sm, int32_t t, int np, int32
     }
     best = lo;
   }
-  PTask r;
   int32_t a = t;  // A-stream index, if t is not a cast
   if (best >= 0) {
-    int32_t fa, na, fc, nc;
-    unit_span<DUAL>(sm, np, best, fa, na, fc, nc);
-    const int32_t pos = min(fa + na + delay, S) + fc;
-    if (t < pos + nc) {
+    int32_t fa, na;
+    unit_span<DUAL>(sm, np, best, fa, na);
+    const int32_t pos = min(fa + na + delay, S) + fa;
+    if (t < pos + na) {
       const int32_t k = t - pos;
       r.kind = kTaskCast;
       r.u = best;
-      r.need = na;
+      r.need = kPWarps * na;  // every warp of every absmax task arrives
       if constexpr (DUAL) {
         r.i = best;
-        const int32_t per = sm.npc[best];
+        const int32_t per = sm.nb[best];
         r.q = k / per;
-        r.k = k - r.q * per;
+        r.b = k - r.q * per;
       } else {
         r.i = best / np;
         r.q = best - r.i * np;
-        r.k = k;
+        r.b = k;
       }
       r.e = sm.order[r.i];
       return r;
     }
-    a = t - (fc + nc);  // every cast before t belongs to units 0 .. best
+    a = t - (fa + na);  // every cast before t belongs to units 0 .. best
   }
   if (a < sm.a_total) {
-    // absmax task: the multi group whose absmax span holds a (32-way search)
     int lo = 0, hi = sm.n_multi;  // apre[lo] * np <= a
     while (hi - lo > 1) {
       const int step = (hi - lo + 31) / 32;
@@ -283,21 +280,20 @@ __device__ PTask decode_panel_task(const PanelSmem &sm, int32_t t, int np, int32
       hi = min(hi, nlo + step);
       lo = nlo;
     }
-    const int32_t nci = sm.nc[lo];
+    const int32_t nbi = sm.nb[lo];
     const int32_t rr = a - sm.apre[lo] * np;
     r.kind = kTaskAbs;
     r.i = lo;
-    r.q = rr / nci;
-    r.k = rr - r.q * nci;
+    r.q = rr / nbi;
+    r.b = rr - r.q * nbi;
     r.u = DUAL ? lo : lo * np + r.q;
-    r.need = DUAL ? nci * np : nci;
+    r.need = 0;
   } else {
-    // whole task (column-wise form only): a group of at most 16 rows, one panel
-    const int32_t w = a - sm.a_total;
+    const int32_t w = a - sm.a_total;  // whole task: single-block group, one panel
     r.kind = kTaskWhole;
     r.i = sm.n_multi + w / np;
     r.q = w - (w / np) * np;
-    r.k = 0;
+    r.b = 0;
     r.u = -1;
     r.need = 0;
   }
@@ -349,17 +345,6 @@ __device__ __forceinline__ void load_rows(uint4 (&v)[kWR], const PanelParams &p,
   }
 }
 
-// Running absmax of the lane's 8 columns (bf16 pairs).
-__device__ __forceinline__ void fold_amax(uint4 &am, const uint4 (&v)[kWR]) {
-#pragma unroll
-  for (int k = 0; k < kWR; ++k) {
-    am.x = absmax_acc(am.x, v[k].x);
-    am.y = absmax_acc(am.y, v[k].y);
-    am.z = absmax_acc(am.z, v[k].z);
-    am.w = absmax_acc(am.w, v[k].w);
-  }
-}
-
 // Dual form: every row's absmax over the lane's 8 columns, reduced over the
 // warp (16 values over 32 lanes: halve four times, then pair lanes), merged
 // into the row's absmax word.
@@ -388,30 +373,6 @@ __device__ __forceinline__ void merge_row_amax(const uint4 (&v)[kWR], uint32_t *
   if (!(lane & 1) && row < r1) atomicMax(rowmax + row, rmax);
 }
 
-// Column-wise codes of the lane's 16 rows: column 8*lane + j as one 16-byte
-// piece of tokens (adjacent rows of a column share one conversion).  Rows past
-// the group's end are zeros, whose codes are the padding.
-template <int FMT, bool FAST>
-__device__ __forceinline__ void store_col_codes(const uint4 (&v)[kWR], const float (&s)[8],
-                                                uint8_t *dst, int64_t ld_qc, bool lane_ok,
-                                                float smax, float sat_thr, uint32_t &sat) {
-#pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    const int wj = j >> 1;
-    uint32_t c2[8];
-#pragma unroll
-    for (int m = 0; m < 8; ++m) {
-      const uint32_t w0 = word(v[2 * m], wj), w1 = word(v[2 * m + 1], wj);
-      const float x0 = (j & 1) ? hi_f(w0) : lo_f(w0);
-      const float x1 = (j & 1) ? hi_f(w1) : lo_f(w1);
-      c2[m] = enc_pair<FMT, FAST>(x0, x1, s[j], s[j], smax, sat_thr, sat);
-    }
-    const uint4 tok = make_uint4(c2[0] | (c2[1] << 16), c2[2] | (c2[3] << 16),
-                                 c2[4] | (c2[5] << 16), c2[6] | (c2[7] << 16));
-    if (lane_ok) *reinterpret_cast<uint4 *>(dst + j * ld_qc) = tok;
-  }
-}
-
 // The lane's 8 column scales (16-byte stores when the address allows).
 __device__ __forceinline__ void store_scales8(float *d, const float (&s)[8]) {
   if ((reinterpret_cast<uintptr_t>(d) & 15) == 0) {
@@ -423,17 +384,56 @@ __device__ __forceinline__ void store_scales8(float *d, const float (&s)[8]) {
   }
 }
 
-// the dual form holds more in registers: three blocks per SM
-template <bool DUAL>
-constexpr int blocks_per_sm() { return DUAL ? 3 : kPBlocksPerSM; }
+// Column-wise codes of the lane's 16 rows into the tile: column 8*lane + j as
+// one 16-byte piece (adjacent rows of a column share one conversion), at tile
+// row 8*lane + j, piece w ^ (row % 8) (128-byte swizzle).  The pieces are
+// stored in rotated order (lane % 8 steps), so that the 8 lanes of a
+// shared-memory phase hit 8 different 16-byte bank groups.
+template <int FMT, bool FAST>
+__device__ __forceinline__ void tile_col_codes(const uint4 (&v)[kWR], const float (&s)[8],
+                                               uint8_t *tile, int w, int lane, float smax,
+                                               float sat_thr, uint32_t &sat) {
+  uint4 tok[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const int wj = j >> 1;
+    uint32_t c2[8];
+#pragma unroll
+    for (int m = 0; m < 8; ++m) {
+      const uint32_t w0 = word(v[2 * m], wj), w1 = word(v[2 * m + 1], wj);
+      const float x0 = (j & 1) ? hi_f(w0) : lo_f(w0);
+      const float x1 = (j & 1) ? hi_f(w1) : lo_f(w1);
+      c2[m] = enc_pair<FMT, FAST>(x0, x1, s[j], s[j], smax, sat_thr, sat);
+    }
+    tok[j] = make_uint4(c2[0] | (c2[1] << 16), c2[2] | (c2[3] << 16), c2[4] | (c2[5] << 16),
+                        c2[6] | (c2[7] << 16));
+  }
+  const int rot = lane & 7;
+#pragma unroll
+  for (int st = 1; st < 8; st <<= 1) {
+    if (rot & st) {
+      uint4 tmp[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) tmp[j] = tok[(j + st) & 7];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) tok[j] = tmp[j];
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const int cc = 8 * lane + ((j + rot) & 7);
+    *reinterpret_cast<uint4 *>(tile + cc * kRB + 16 * (w ^ (cc & 7))) = tok[j];
+  }
+}
 
 template <int FMT, bool FAST, bool DUAL>
-__global__ void __launch_bounds__(kPThreads, blocks_per_sm<DUAL>())
-    quant_panel_kernel(const PanelParams p) {
+__global__ void __launch_bounds__(kPThreads, kPBlocksPerSM)
+    quant_panel_kernel(const __grid_constant__ CUtensorMap qmap, const PanelParams p) {
   extern __shared__ uint8_t smem_raw[];
-  PanelSmem &sm = *reinterpret_cast<PanelSmem *>(smem_raw);
+  PanelSmem &sm = *align_smem_1024<PanelSmem>(smem_raw);
   const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
   const int np = (p.cols + kPW - 1) / kPW;
+  if (tid == 0 && p.rows_total > 0) prefetch_tensormap(&qmap);
   panel_prologue<DUAL>(sm, p, np);
 
   // empty groups: scales only (Fmax / 1e-12 in every column), no codes
@@ -445,91 +445,81 @@ __global__ void __launch_bounds__(kPThreads, blocks_per_sm<DUAL>())
       p.scales_col[static_cast<int64_t>(e) * p.cols + c] = s;
   }
 
-  uint32_t sat = 0;
-  const int32_t total = sm.total;
-  uint32_t *xch = sm.xch[w];
+  // warp 0 fetches and decodes the tasks, one ahead of the block
   int32_t next = 0;
-  if (lane == 0) next = static_cast<int32_t>(atomicAdd(p.work, 1u));
-  while (true) {
+  if (w == 0) {
     int32_t t = 0;
     if (lane == 0) {
-      t = next;
-      if (t < total) next = static_cast<int32_t>(atomicAdd(p.work, 1u));
+      t = static_cast<int32_t>(atomicAdd(p.work, 1u));
+      next = static_cast<int32_t>(atomicAdd(p.work, 1u));
     }
     t = __shfl_sync(0xFFFFFFFFu, t, 0);
-    if (t >= total) break;
     const PTask tk = decode_panel_task<DUAL>(sm, t, np, p.delay, lane);
+    if (lane == 0) sm.tk[0] = tk;
+  }
+  __syncthreads();
+
+  uint32_t sat = 0;
+  bool failed = false;
+  for (int n = 0;; ++n) {
+    const int cur = n & 1;
+    const PTask tk = sm.tk[cur];
+    if (tk.kind == kTaskEnd) break;
     const int e = tk.e;
     const int32_t gs = e ? sm.end[e - 1] : 0;
     const int32_t ge = sm.end[e];
-    const int32_t r0 = gs + tk.k * kCR;
-    const int32_t r1 = min(ge, r0 + kCR);
+    const int32_t r0 = gs + tk.b * kRB;
+    const int32_t r1 = min(ge, r0 + kRB);
+    const int32_t rw0 = r0 + kWR * w;
     const int c0 = tk.q * kPW;
     const bool lane_ok = c0 + 8 * lane < p.cols;
     const int64_t cvec = (c0 >> 3) + lane;
     const int64_t amax_base = static_cast<int64_t>(tk.i) * p.cols + c0;
+    uint8_t *tile = sm.tile[cur];
 
-    if (tk.kind == kTaskAbs) {
-      // ------------------------------------------------------------ absmax
-      uint4 am = make_uint4(0u, 0u, 0u, 0u);
-#pragma unroll 1
-      for (int32_t rw0 = r0; rw0 < r1; rw0 += kWR) {
-        uint4 v[kWR];
-        load_rows<false>(v, p, rw0, r1, cvec, lane_ok);
-        fold_amax(am, v);
-        if constexpr (DUAL) merge_row_amax(v, p.rowmax, rw0, r1, lane);
-      }
-      // the lane's 8 column words, transposed so that lane l merges columns
-      // 32m + l (one 128-byte run per atomic instruction)
-      am = make_uint4(absmax_bits(am.x), absmax_bits(am.y), absmax_bits(am.z),
-                      absmax_bits(am.w));
-      *reinterpret_cast<uint4 *>(xch + 8 * lane) =
-          make_uint4(am.x & 0xFFFFu, am.x >> 16, am.y & 0xFFFFu, am.y >> 16);
-      *reinterpret_cast<uint4 *>(xch + 8 * lane + 4) =
-          make_uint4(am.z & 0xFFFFu, am.z >> 16, am.w & 0xFFFFu, am.w >> 16);
-      __syncwarp();
-#pragma unroll
-      for (int m = 0; m < 8; ++m) {
-        const int cc = 32 * m + lane;
-        if (c0 + cc < p.cols) atomicMax(p.amax + amax_base + cc, xch[cc]);
-      }
-      __threadfence();  // every lane's merges are visible before the count
-      __syncwarp();     // (and xch is free again)
-      if (lane == 0) atomicAdd(p.arrive + tk.u, 1u);
-      continue;
-    }
-
-    // ------------------------------------------------------------ cast
+    uint4 v[kWR];
     float s[8];
-    if (tk.kind == kTaskWhole) {
-      // at most 16 rows: the absmax comes from the same registers
-      uint4 v[kWR];
-      load_rows<false>(v, p, r0, r1, cvec, lane_ok);
+    if (tk.kind != kTaskCast) {
+      // ---------------------------------------------------------- absmax
+      load_rows<false>(v, p, rw0, r1, cvec, lane_ok);
       uint4 am = make_uint4(0u, 0u, 0u, 0u);
-      fold_amax(am, v);
-      am = make_uint4(absmax_bits(am.x), absmax_bits(am.y), absmax_bits(am.z),
-                      absmax_bits(am.w));
-      const uint32_t a[8] = {am.x & 0xFFFFu, am.x >> 16, am.y & 0xFFFFu, am.y >> 16,
-                             am.z & 0xFFFFu, am.z >> 16, am.w & 0xFFFFu, am.w >> 16};
 #pragma unroll
-      for (int j = 0; j < 8; ++j) s[j] = scale_from_amax(bf16_bits_to_float(a[j]), p.smax);
-      if (lane_ok) store_scales8(p.scales_col + static_cast<int64_t>(e) * p.cols + c0 + 8 * lane, s);
-      uint8_t *dst = p.q_col + static_cast<int64_t>(c0 + 8 * lane) * p.ld_qc + sm.pstart[e];
-      store_col_codes<FMT, FAST>(v, s, dst, p.ld_qc, lane_ok, p.smax, p.sat_thr, sat);
-      // the rest of the 128-token block: zero codes
-      if (lane_ok) {
-#pragma unroll
-        for (int j = 0; j < 8; ++j)
-#pragma unroll
-          for (int z = 1; z < kPadTok / 16; ++z)
-            *reinterpret_cast<uint4 *>(dst + j * p.ld_qc + 16 * z) = make_uint4(0u, 0u, 0u, 0u);
+      for (int k = 0; k < kWR; ++k) {
+        am.x = absmax_acc(am.x, v[k].x);
+        am.y = absmax_acc(am.y, v[k].y);
+        am.z = absmax_acc(am.z, v[k].z);
+        am.w = absmax_acc(am.w, v[k].w);
       }
-      continue;
-    }
-
-    {  // wait (bounded) until every absmax task of the unit has been counted
+      if constexpr (DUAL) merge_row_amax(v, p.rowmax, rw0, r1, lane);
+      *reinterpret_cast<uint4 *>(&sm.red[cur][w][4 * lane]) =
+          make_uint4(absmax_bits(am.x), absmax_bits(am.y), absmax_bits(am.z),
+                     absmax_bits(am.w));
+      if (tk.kind == kTaskWhole) {
+        // single block: the block's column absmax is the unit's; its scales
+        // and codes come from the same registers
+        __syncthreads();
+        uint4 mm = make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+        for (int ww = 0; ww < kPWarps; ++ww) {
+          const uint4 o = *reinterpret_cast<const uint4 *>(&sm.red[cur][ww][4 * lane]);
+          mm.x = __vmaxu2(mm.x, o.x);
+          mm.y = __vmaxu2(mm.y, o.y);
+          mm.z = __vmaxu2(mm.z, o.z);
+          mm.w = __vmaxu2(mm.w, o.w);
+        }
+        const uint32_t a[8] = {mm.x & 0xFFFFu, mm.x >> 16, mm.y & 0xFFFFu, mm.y >> 16,
+                               mm.z & 0xFFFFu, mm.z >> 16, mm.w & 0xFFFFu, mm.w >> 16};
+#pragma unroll
+        for (int j = 0; j < 8; ++j) s[j] = scale_from_amax(bf16_bits_to_float(a[j]), p.smax);
+        if (w == 0 && lane_ok)
+          store_scales8(p.scales_col + static_cast<int64_t>(e) * p.cols + c0 + 8 * lane, s);
+        tile_col_codes<FMT, FAST>(v, s, tile, w, lane, p.smax, p.sat_thr, sat);
+        fence_proxy_async_smem();
+      }
+    } else {
+      // ---------------------------------------------------------- cast
       int ok = 1;
-      if (lane == 0) {
+      if (lane == 0) {  // every warp waits (bounded) for the unit's count
         const uint32_t *cnt = p.arrive + tk.u;
         const uint32_t target = static_cast<uint32_t>(tk.need) + p.uw.extra_arrivals;
         uint32_t c;
@@ -537,7 +527,7 @@ __global__ void __launch_bounds__(kPThreads, blocks_per_sm<DUAL>())
         if (c < target) {
           const uint64_t t0 = global_timer_ns();
           while (true) {
-            __nanosleep(100);
+            __nanosleep(64);
             asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(c) : "l"(cnt) : "memory");
             if (c >= target) break;
             if (global_timer_ns() - t0 > p.uw.limit_ns) { ok = 0; break; }
@@ -545,67 +535,95 @@ __global__ void __launch_bounds__(kPThreads, blocks_per_sm<DUAL>())
         }
       }
       ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
-      if (ok) {  // every lane acquires the count it is about to rely on
+      if (ok) {  // every lane acquires the count it relies on
         uint32_t c;
         asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(c) : "l"(p.arrive + tk.u)
                      : "memory");
         (void)c;
+      } else {
+        failed = true;
       }
-      __syncwarp();
-      if (!ok) {
-        if (lane == 0) status_or(p.status, FP8QGG_STATUS_TIMEOUT);
-        break;  // this warp takes no more tasks
-      }
-    }
-    {  // the lane's 8 column scales from the unit's merged absmax
-      uint4 a0 = make_uint4(0u, 0u, 0u, 0u), a1 = a0;
-      if (lane_ok) {
-        const uint4 *src = reinterpret_cast<const uint4 *>(p.amax + amax_base + 8 * lane);
-        a0 = __ldcg(src);
-        a1 = __ldcg(src + 1);
-      }
-      const uint32_t a[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
-#pragma unroll
-      for (int j = 0; j < 8; ++j) s[j] = scale_from_amax(bf16_bits_to_float(a[j]), p.smax);
-      if (tk.k == 0 && lane_ok)
-        store_scales8(p.scales_col + static_cast<int64_t>(e) * p.cols + c0 + 8 * lane, s);
-    }
-    float rs_lane = 0.0f;  // dual form: the scale of row r0 + lane
-    if constexpr (DUAL) {
-      const int32_t row = r0 + lane;
-      if (row < r1) {
-        rs_lane = scale_from_amax(bf16_bits_to_float(__ldcg(p.rowmax + row)), p.smax);
-        if (tk.q == 0) p.scales_row[row] = rs_lane;
-      }
-    }
-    uint8_t *dst0 = p.q_col + static_cast<int64_t>(c0 + 8 * lane) * p.ld_qc + sm.pstart[e] +
-                    tk.k * kCR;
-#pragma unroll 1
-    for (int h = 0; h < kCR / kWR; ++h) {
-      const int32_t rw0 = r0 + h * kWR;
-      uint4 v[kWR];
-      load_rows<true>(v, p, rw0, r1, cvec, lane_ok);
-      if constexpr (DUAL) {
-        // rowwise codes in place: 8 columns of a row per lane, one 8-byte store
-#pragma unroll
-        for (int k = 0; k < kWR; ++k) {
-          const float rs = __shfl_sync(0xFFFFFFFFu, rs_lane, h * kWR + k);
-          const int32_t row = rw0 + k;
-          uint32_t c2[4];
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const uint32_t wd = word(v[k], j);
-            c2[j] = enc_pair<FMT, FAST>(lo_f(wd), hi_f(wd), rs, rs, p.smax, p.sat_thr, sat);
-          }
-          if (lane_ok && row < r1)
-            *reinterpret_cast<uint2 *>(p.q_row + static_cast<int64_t>(row) * p.ld_qr + c0 +
-                                       8 * lane) =
-                make_uint2(c2[0] | (c2[1] << 16), c2[2] | (c2[3] << 16));
+      if (!failed) {
+        uint4 a0 = make_uint4(0u, 0u, 0u, 0u), a1 = a0;
+        if (lane_ok) {
+          const uint4 *src = reinterpret_cast<const uint4 *>(p.amax + amax_base + 8 * lane);
+          a0 = __ldcg(src);
+          a1 = __ldcg(src + 1);
         }
+        const uint32_t a[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+#pragma unroll
+        for (int j = 0; j < 8; ++j) s[j] = scale_from_amax(bf16_bits_to_float(a[j]), p.smax);
+        if (tk.b == 0 && w == 0 && lane_ok)
+          store_scales8(p.scales_col + static_cast<int64_t>(e) * p.cols + c0 + 8 * lane, s);
+        float rs_lane = 0.0f;  // dual form: the scale of row rw0 + lane (lanes 0..15)
+        if constexpr (DUAL) {
+          const int32_t row = rw0 + lane;
+          if (lane < kWR && row < r1) {
+            rs_lane = scale_from_amax(bf16_bits_to_float(__ldcg(p.rowmax + row)), p.smax);
+            if (tk.q == 0) p.scales_row[row] = rs_lane;
+          }
+        }
+        load_rows<true>(v, p, rw0, r1, cvec, lane_ok);
+        if constexpr (DUAL) {
+          // rowwise codes in place: 8 columns of a row per lane, one 8-byte store
+#pragma unroll
+          for (int k = 0; k < kWR; ++k) {
+            const float rs = __shfl_sync(0xFFFFFFFFu, rs_lane, k);
+            const int32_t row = rw0 + k;
+            uint32_t c2[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const uint32_t wd = word(v[k], j);
+              c2[j] = enc_pair<FMT, FAST>(lo_f(wd), hi_f(wd), rs, rs, p.smax, p.sat_thr, sat);
+            }
+            if (lane_ok && row < r1)
+              *reinterpret_cast<uint2 *>(p.q_row + static_cast<int64_t>(row) * p.ld_qr + c0 +
+                                         8 * lane) =
+                  make_uint2(c2[0] | (c2[1] << 16), c2[2] | (c2[3] << 16));
+          }
+        }
+        tile_col_codes<FMT, FAST>(v, s, tile, w, lane, p.smax, p.sat_thr, sat);
+        fence_proxy_async_smem();
       }
-      store_col_codes<FMT, FAST>(v, s, dst0 + h * kWR, p.ld_qc, lane_ok, p.smax, p.sat_thr, sat);
+    }
+
+    // warp 0: the next task; the tile written above may only be reused once
+    // the store that read it two tasks ago has finished reading
+    if (w == 0) {
+      int32_t t = 0;
+      if (lane == 0) {
+        t = next;
+        if (t < sm.total) next = static_cast<int32_t>(atomicAdd(p.work, 1u));
+        bulk_wait_read<0>();
+      }
+      t = __shfl_sync(0xFFFFFFFFu, t, 0);
+      const PTask nt = decode_panel_task<DUAL>(sm, t, np, p.delay, lane);
+      if (lane == 0) sm.tk[cur ^ 1] = nt;
+    }
+    // a warp that gave up on its wait stops the block after this task
+    if (__syncthreads_or(failed)) {
+      if (tid == 0) status_or(p.status, FP8QGG_STATUS_TIMEOUT);
+      break;
+    }
+
+    if (tk.kind == kTaskAbs) {
+      // each warp merges 32 of the panel's columns into the unit's absmax and
+      // counts itself: column 32w + lane is half (lane & 1) of word 16w + lane / 2
+      const int wd = 16 * w + (lane >> 1);
+      uint32_t m = 0;
+#pragma unroll
+      for (int ww = 0; ww < kPWarps; ++ww) m = __vmaxu2(m, sm.red[cur][ww][wd]);
+      const int cc = 32 * w + lane;
+      if (c0 + cc < p.cols) atomicMax(p.amax + amax_base + cc, (lane & 1) ? m >> 16 : m & 0xFFFFu);
+      __threadfence();
+      __syncwarp();
+      if (lane == 0) atomicAdd(p.arrive + tk.u, 1u);
+    } else if (tid == 0) {
+      tma_store_2d(&qmap, tile, sm.pstart[e] + tk.b * kRB, c0);
+      bulk_commit();
     }
   }
+  if (tid == 0) bulk_wait_all();  // the tiles stay valid until their stores have read them
   if (!FAST && p.sat_count) {
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) sat += __shfl_xor_sync(0xFFFFFFFFu, sat, off);
@@ -615,7 +633,7 @@ __global__ void __launch_bounds__(kPThreads, blocks_per_sm<DUAL>())
 
 namespace {
 
-using PanelKernel = void (*)(const PanelParams);
+using PanelKernel = void (*)(const CUtensorMap, const PanelParams);
 
 template <bool DUAL>
 PanelKernel panel_kernel(int fmt, bool fast) {
@@ -648,12 +666,24 @@ int panel_launch(const void *x, int64_t rows_total, int64_t cols, int64_t ld_x,
                  float scale_max, uint64_t *sat_count, int32_t *dev_status, void *scratch,
                  UnitWait uw, cudaStream_t stream) {
   const bool dual = q_row != nullptr;
+  CUtensorMap qmap;
+  memset(&qmap, 0, sizeof qmap);
+  if (rows_total > 0) {
+    // codes [cols][ld_qc tokens]; boxes of 128 tokens x 256 columns (fewer
+    // columns when the tensor has fewer), 128-byte swizzle
+    const uint64_t dims[2] = {static_cast<uint64_t>(ld_qc), static_cast<uint64_t>(cols)};
+    const uint64_t strides[1] = {static_cast<uint64_t>(ld_qc)};
+    const uint32_t box[2] = {kRB, static_cast<uint32_t>(std::min<int64_t>(kPW, cols))};
+    if (!encode_tensor_map(&qmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, q_col, dims, strides, box,
+                           CU_TENSOR_MAP_SWIZZLE_128B))
+      return FP8QGG_ERR_CUDA;
+  }
   DeviceInfo dev;
   if (!device_info(&dev)) return FP8QGG_ERR_CUDA;
   const float smax = effective_scale_max(fmt, scale_max);
   const bool fast = sat_count == nullptr && smax >= format_max(fmt);
   PanelKernel kern = dual ? panel_kernel<true>(fmt, fast) : panel_kernel<false>(fmt, fast);
-  const int smem = static_cast<int>(sizeof(PanelSmem));
+  const int smem = static_cast<int>(sizeof(PanelSmem)) + 1024;
   if (!set_max_dynamic_smem(reinterpret_cast<const void *>(kern), smem)) return FP8QGG_ERR_CUDA;
   const PanelScratch sl = panel_scratch(rows_total, cols, num_groups, dual);
   uint8_t *base = static_cast<uint8_t *>(scratch);
@@ -664,8 +694,6 @@ int panel_launch(const void *x, int64_t rows_total, int64_t cols, int64_t ld_x,
   prm.cols = static_cast<int>(cols);
   prm.offsets = offsets;
   prm.num_groups = num_groups;
-  prm.q_col = q_col;
-  prm.ld_qc = ld_qc;
   prm.scales_col = scales_col;
   prm.q_row = q_row;
   prm.ld_qr = ld_qr;
@@ -682,13 +710,12 @@ int panel_launch(const void *x, int64_t rows_total, int64_t cols, int64_t ld_x,
   // blocks: kPBlocksPerSM per SM, never more than the tasks need (at least
   // one, for the scales of empty groups)
   const int64_t np = (cols + kPW - 1) / kPW;
-  const int64_t chunks = (rows_total + int64_t(kPadTok) * num_groups) / kCR * np;
-  const int per_sm = dual ? blocks_per_sm<true>() : blocks_per_sm<false>();
+  const int64_t blocks = (rows_total + int64_t(kRB) * num_groups) / kRB * np;
   const int grid = static_cast<int>(std::max<int64_t>(
-      1, std::min<int64_t>((2 * chunks + kPWarps - 1) / kPWarps, int64_t(dev.sm_count) * per_sm)));
-  // a cast waits for absmax tasks that every running warp has taken by then
-  prm.delay = grid * kPWarps;
-  kern<<<grid, kPThreads, smem, stream>>>(prm);
+      1, std::min<int64_t>(2 * blocks, int64_t(dev.sm_count) * kPBlocksPerSM)));
+  // a cast waits for absmax tasks that the running blocks have taken by then
+  prm.delay = grid;
+  kern<<<grid, kPThreads, smem, stream>>>(qmap, prm);
   return cudaGetLastError() == cudaSuccess ? FP8QGG_OK : FP8QGG_ERR_CUDA;
 }
 
