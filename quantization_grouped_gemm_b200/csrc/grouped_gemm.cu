@@ -880,327 +880,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   }
 }
 
-// ---------------------------------------------------------------------------
-// Contraction-jagged mode on padded operands, on SM pairs (cta_group::2).
-// The weight gradient dW_e[i, j] = sum over group e's tokens of A[i, t] B[j, t]
-// is computed transposed: the pair's MMA rows (M = 256, 128 per CTA) run over
-// j (B's rows) and its N columns over i (A's rows, nt of them: a multiple of
-// 16 that divides the i range into equal tiles when it can).  Per 128-token
-// k-block each CTA loads 128 rows of B and nt / 2 rows of A (half the operand
-// bytes per SM of the one-CTA kernel for the same tensor work), the first CTA
-// issues tcgen05.mma.cta_group::2 and commits to both CTAs' barriers.  In the
-// padded layout every k-block lies inside one group, so nothing is masked.
-// The epilogue reads TMEM lane j, columns i, and writes out[e, i, j] directly:
-// the 32 lanes of a warp store 32 consecutive j of one i, a full 128-byte
-// line (fp32) per instruction.  Tiles are listed group by group, largest
-// group first, taken by the pairs in alternating directions.
-constexpr int kStagesK2 = 5;
-
-struct GemmK2Smem {
-  uint8_t b[kStagesK2][128 * BK];  // this CTA's 128 rows of B (MMA rows)
-  uint8_t a[kStagesK2][128 * BK];  // this CTA's nt / 2 rows of A (MMA columns)
-  float stg[kEpiWarps][2][16 * 32];  // per epilogue warp: two 16 (i) x 32 (j) output units
-  float inv_sa[2][BN];             // 1 / scale_a of the tile's i columns
-  int32_t pend[kMaxGemmGroups];    // padded group ends (tokens)
-  int32_t order[kMaxGemmGroups];   // groups by size, largest first
-  uint64_t full[kStagesK2];
-  uint64_t empty[kStagesK2];
-  uint64_t tfull[2];
-  uint64_t tempty[2];
-  uint64_t drain;
-  uint32_t tmem_base;
-  int abort;
-};
-
-struct K2Tile {
-  int e;
-  int tj, ti;     // tile of j (MMA rows) and of i (MMA columns)
-  int32_t kx0;    // first token of the group in the padded layout
-  int nk;         // 128-token k-blocks
-};
-
-__device__ __forceinline__ K2Tile k2_tile(const GemmK2Smem &sm, int32_t pos, int tj_n,
-                                          int ti_n) {
-  const int32_t tpg = tj_n * ti_n;
-  K2Tile t;
-  t.e = sm.order[pos / tpg];
-  const int32_t local = pos - (pos / tpg) * tpg;
-  t.tj = local / ti_n;
-  t.ti = local - t.tj * ti_n;
-  t.kx0 = t.e ? sm.pend[t.e - 1] : 0;
-  t.nk = (sm.pend[t.e] - t.kx0) / BK;
-  return t;
-}
-
-// The i-th tile position of cluster c among nc clusters (alternating rounds).
-__device__ __forceinline__ int32_t k2_position(int32_t i, int32_t c, int32_t nc) {
-  return i * nc + ((i & 1) ? (nc - 1 - c) : c);
-}
-
-template <int OUT>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
-    grouped_gemm_k2_kernel(const __grid_constant__ CUtensorMap amap,
-                           const __grid_constant__ CUtensorMap bmap,
-                           const __grid_constant__ CUtensorMap omap, const GemmParams p,
-                           int nt) {
-  extern __shared__ uint8_t smem_raw[];
-  GemmK2Smem &sm = *align_smem_1024<GemmK2Smem>(smem_raw);
-  const int warp = threadIdx.x >> 5;
-  const int lane = threadIdx.x & 31;
-  const uint32_t rank = cluster_ctarank();
-  const bool first = rank == 0;
-  const int tj_n = static_cast<int>((p.k + 255) / 256);
-  const int ti_n = static_cast<int>((p.n + nt - 1) / nt);
-  const uint32_t a_half_bytes = static_cast<uint32_t>(nt / 2) * BK;
-  const uint32_t stage_bytes = 2u * (128u * BK + a_half_bytes);  // both CTAs' copies
-  const uint32_t idesc = idesc_e4m3_f32(256, static_cast<uint32_t>(nt));
-
-  if (warp == 0 && lane == 0) {
-    prefetch_tensormap(&amap);
-    prefetch_tensormap(&bmap);
-    prefetch_tensormap(&omap);
-    for (int s2 = 0; s2 < kStagesK2; ++s2) {
-      mbar_init(&sm.full[s2], 1);
-      mbar_init(&sm.empty[s2], 1);
-    }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&sm.tfull[b], 1);
-      mbar_init(&sm.tempty[b], 2 * kEpiThreads);
-    }
-    mbar_init(&sm.drain, 1);
-    sm.abort = 0;
-    fence_mbarrier_init();
-  }
-  if (warp == 1) {
-    tmem_alloc_2sm(&sm.tmem_base, kTmemCols);
-    tmem_relinquish_2sm();
-  }
-  if (warp == 2) {
-    // padded group ends: each group rounded up to 128 tokens (clamped ends as
-    // everywhere else)
-    const int32_t R = static_cast<int32_t>(p.m_total);
-    int32_t carry_end = 0, carry_pend = 0;
-    bool bad = false;
-    for (int base = 0; base < p.num_groups; base += 32) {
-      const int e = base + lane;
-      const int32_t raw = e < p.num_groups ? __ldg(p.offsets + e) : INT32_MIN;
-      int32_t run = max(raw, 0);
-      for (int d = 1; d < 32; d <<= 1) {
-        const int32_t o = __shfl_up_sync(0xFFFFFFFFu, run, d);
-        if (lane >= d) run = max(run, o);
-      }
-      const int32_t endv = min(R, max(carry_end, run));
-      int32_t prev = __shfl_up_sync(0xFFFFFFFFu, endv, 1);
-      if (lane == 0) prev = carry_end;
-      if (e < p.num_groups && (raw < prev || raw > R)) bad = true;
-      int32_t psz = e < p.num_groups ? (endv - prev + BK - 1) & ~(BK - 1) : 0;
-      for (int d = 1; d < 32; d <<= 1) {
-        const int32_t o = __shfl_up_sync(0xFFFFFFFFu, psz, d);
-        if (lane >= d) psz += o;
-      }
-      if (e < p.num_groups) sm.pend[e] = carry_pend + psz;
-      carry_end = __shfl_sync(0xFFFFFFFFu, endv, 31);
-      carry_pend += __shfl_sync(0xFFFFFFFFu, psz, 31);
-    }
-    bad = __any_sync(0xFFFFFFFFu, bad);
-    if (bad && lane == 0 && blockIdx.x == 0) status_or(p.status, FP8QGG_STATUS_BAD_OFFSETS);
-  }
-  tc_fence_before_sync();
-  __syncthreads();
-  // groups ranked by padded size, largest first (ties by index)
-  for (int e = threadIdx.x; e < p.num_groups; e += kGemmThreads) {
-    const int32_t se = sm.pend[e] - (e ? sm.pend[e - 1] : 0);
-    int rk = 0;
-    for (int f = 0; f < p.num_groups; ++f) {
-      const int32_t sf = sm.pend[f] - (f ? sm.pend[f - 1] : 0);
-      rk += (sf > se) || (sf == se && f < e);
-    }
-    sm.order[rk] = e;
-  }
-  __syncthreads();
-  cluster_sync();  // both CTAs' barriers exist before any copy or arrive crosses the pair
-  tc_fence_after_sync();
-
-  const int32_t total = p.num_groups * tj_n * ti_n;
-  const int32_t cid = static_cast<int32_t>(blockIdx.x) >> 1;
-  const int32_t ncl = static_cast<int32_t>(gridDim.x) >> 1;
-  volatile int *abort = &sm.abort;
-  const uint32_t tmem_base = sm.tmem_base;
-
-  if (warp == 0) {
-    // ------------------------------------------------------------ producer (both CTAs)
-    if (lane == 0) {
-      uint32_t stage = 0, phase = 0;
-      uint32_t armed = 0;
-      uint32_t last_par[kStagesK2];
-      bool ok = true;
-      for (int32_t i = 0, t = k2_position(0, cid, ncl); t < total && ok;
-           t = k2_position(++i, cid, ncl)) {
-        const K2Tile ti = k2_tile(sm, t, tj_n, ti_n);
-        const int32_t brow = ti.tj * 256 + 128 * static_cast<int32_t>(rank);
-        const int32_t arow = ti.ti * nt + (nt / 2) * static_cast<int32_t>(rank);
-        for (int kb = 0; kb < ti.nk; ++kb) {
-          if (!mbar_wait(&sm.empty[stage], phase ^ 1, abort)) { ok = false; break; }
-          const uint32_t full0 = mapa_shared(smem_addr(&sm.full[stage]), 0);
-          if (first) {
-            mbar_arrive_expect_tx(&sm.full[stage], stage_bytes);
-            armed |= 1u << stage;
-            last_par[stage] = phase;
-          }
-          const int32_t kx = ti.kx0 + kb * BK;
-          tma_load_2d_2sm(sm.b[stage], &bmap, full0, kx, brow);
-          tma_load_2d_2sm(sm.a[stage], &amap, full0, kx, arow);
-          if (++stage == kStagesK2) { stage = 0; phase ^= 1; }
-        }
-      }
-      if (!ok) {
-        *abort = 1;
-        status_or(p.status, FP8QGG_STATUS_TIMEOUT);
-        volatile int never = 0;
-        for (int s2 = 0; s2 < kStagesK2; ++s2)
-          if (armed & (1u << s2)) (void)mbar_wait(&sm.full[s2], last_par[s2], &never);
-      }
-    }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer (first CTA)
-    if (first) {
-      uint32_t stage = 0, phase = 0, acc = 0, acc_phase = 0;
-      bool ok = true;
-      uint32_t tfull_peer[2];
-      for (int b = 0; b < 2; ++b) tfull_peer[b] = mapa_shared(smem_addr(&sm.tfull[b]), 1);
-      for (int32_t i = 0, t = k2_position(0, cid, ncl); t < total && ok;
-           t = k2_position(++i, cid, ncl)) {
-        const K2Tile ti = k2_tile(sm, t, tj_n, ti_n);
-        if (!__all_sync(0xFFFFFFFFu, mbar_wait(&sm.tempty[acc], acc_phase ^ 1, abort))) {
-          ok = false;
-          break;
-        }
-        tc_fence_after_sync();
-        const uint32_t d_tmem = tmem_base + acc * BN;
-        for (int kb = 0; kb < ti.nk; ++kb) {
-          if (!__all_sync(0xFFFFFFFFu, mbar_wait(&sm.full[stage], phase, abort))) {
-            ok = false;
-            break;
-          }
-          tc_fence_after_sync();
-          if (lane == 0) {
-            const uint64_t bdesc = smem_desc_k_sw128(smem_addr(sm.b[stage]));
-            const uint64_t adesc = smem_desc_k_sw128(smem_addr(sm.a[stage]));
-#pragma unroll
-            for (int kk = 0; kk < BK / 32; ++kk)
-              mma_f8f6f4_2sm(d_tmem, bdesc + 2 * kk, adesc + 2 * kk, idesc, (kb | kk) != 0);
-            mma_commit_2sm_mc(&sm.empty[stage], 0x3);
-          }
-          __syncwarp();
-          if (++stage == kStagesK2) { stage = 0; phase ^= 1; }
-        }
-        if (!ok) break;
-        if (lane == 0) {
-          if (ti.nk > 0) {
-            mma_commit_2sm_mc(&sm.tfull[acc], 0x3);
-          } else {  // an empty group: nothing to wait for, zeros are written
-            mbar_arrive(&sm.tfull[acc]);
-            mbar_arrive_cluster(tfull_peer[acc]);
-          }
-        }
-        __syncwarp();
-        if (++acc == 2) { acc = 0; acc_phase ^= 1; }
-      }
-      if (!ok && lane == 0) {
-        *abort = 1;
-        status_or(p.status, FP8QGG_STATUS_TIMEOUT);
-      }
-      if (lane == 0) {
-        mma_commit_2sm(&sm.drain);
-        volatile int never = 0;
-        (void)mbar_wait(&sm.drain, 0, &never);
-      }
-      __syncwarp();
-    }
-  } else {
-    // ------------------------------------------------------------ epilogue (both CTAs)
-    // A unit is 16 columns i (one 16-column TMEM load) x the warp's 32 lanes j:
-    // lane j writes its 16 scaled values into row i of a 16 x 32 staging
-    // buffer (consecutive lanes, consecutive words), and one bulk tensor store
-    // sends the buffer to out[e, i0 .. i0 + 15, j0 .. j0 + 31] (clipped at the
-    // tensor's edges).  The stores are asynchronous, so releasing the
-    // accumulator never waits for them.
-    const int et = threadIdx.x - 64;
-    const int ew = warp - 2;
-    const int quarter = warp & 3;   // TMEM lanes [32 * quarter, +32)
-    const int half = ew >> 2;       // 16-column chunks half, half + 2, ...
-    uint32_t tempty0[2];
-    for (int b = 0; b < 2; ++b) tempty0[b] = mapa_shared(smem_addr(&sm.tempty[b]), 0);
-    uint32_t acc = 0, acc_phase = 0;
-    int sb = 0;  // staging buffer of the next unit
-    for (int32_t i = 0, t = k2_position(0, cid, ncl); t < total;
-         t = k2_position(++i, cid, ncl)) {
-      const K2Tile ti = k2_tile(sm, t, tj_n, ti_n);
-      const int64_t i0 = static_cast<int64_t>(ti.ti) * nt;
-      if (et < nt) {
-        const int64_t col = i0 + et;
-        sm.inv_sa[acc][et] =
-            col < p.n ? __frcp_rn(__ldg(p.scale_a + ti.e * p.sas + col)) : 0.0f;
-      }
-      const int32_t j0 = ti.tj * 256 + 128 * static_cast<int32_t>(rank) + 32 * quarter;
-      const int64_t j = j0 + lane;
-      const float inv_b = j < p.k ? __frcp_rn(__ldg(p.scale_b + ti.e * p.sbs + j)) : 0.0f;
-      const bool got = mbar_wait(&sm.tfull[acc], acc_phase, abort);
-      if (!epi_bar_and(got)) {
-        *abort = 1;
-        if (et == 0) status_or(p.status, FP8QGG_STATUS_TIMEOUT);
-        break;
-      }
-      tc_fence_after_sync();
-      const uint32_t taddr =
-          tmem_base + (static_cast<uint32_t>(32 * quarter) << 16) + acc * BN;
-#pragma unroll 1
-      for (int c = half; c < nt / 16; c += 2) {
-        uint32_t r[16];
-        if (ti.nk > 0) {
-          tmem_ld_32x32b_x16(taddr + 16 * c, r);
-          tmem_ld_wait();
-        } else {
-#pragma unroll
-          for (int q = 0; q < 16; ++q) r[q] = 0u;
-        }
-        float *buf = sm.stg[ew][sb];
-        if (lane == 0) bulk_wait_read<1>();  // the store that last read this buffer is done
-        __syncwarp();
-#pragma unroll
-        for (int q = 0; q < 16; ++q) {
-          const float v = __fmul_rn(__fmul_rn(__uint_as_float(r[q]), sm.inv_sa[acc][16 * c + q]),
-                                    inv_b);
-          if constexpr (OUT == FP8QGG_OUT_F32)
-            buf[q * 32 + lane] = v;
-          else
-            reinterpret_cast<__nv_bfloat16 *>(buf)[q * 32 + lane] = __float2bfloat16_rn(v);
-        }
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) {
-          tma_store_3d(&omap, buf, j0, static_cast<int32_t>(i0 + 16 * c), ti.e);
-          bulk_commit();
-        }
-        sb ^= 1;
-      }
-      tc_fence_before_sync();
-      mbar_arrive_cluster(tempty0[acc]);
-      if (++acc == 2) { acc = 0; acc_phase ^= 1; }
-    }
-    if (lane == 0) bulk_wait_all();
-    __syncwarp();
-  }
-
-  tc_fence_before_sync();
-  __syncthreads();
-  cluster_sync();  // the pair's MMAs are drained and no peer access is pending
-  if (warp == 1) {
-    tc_fence_after_sync();
-    tmem_dealloc_2sm(tmem_base, kTmemCols);
-  }
-}
-
 namespace {
 using GemmKernel = void (*)(const CUtensorMap, const CUtensorMap, const CUtensorMap,
                            const GemmParams);
@@ -1359,63 +1038,6 @@ extern "C" int fp8_scaled_grouped_gemm(int mode, const uint8_t *a, int64_t ld_a,
         static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(pair_tiles, dev.sm_count / 2)));
     kern2<<<2 * clusters, kGemmThreads, smem2, static_cast<cudaStream_t>(stream)>>>(amap, bmap2,
                                                                                   omap, prm);
-    return cudaGetLastError() == cudaSuccess ? FP8QGG_OK : FP8QGG_ERR_CUDA;
-  }
-
-  // Padded contraction-jagged problems run on SM pairs: the pair's MMA rows
-  // run over k (256 per tile), its columns over n in nt-wide tiles, nt the
-  // multiple of 16 that covers n with the least padding (ties: fewer tiles).
-  if (padded && dev.sm_count >= 2) {
-    int nt = 256;
-    int64_t best = INT64_MAX;
-    for (int64_t t = (n + 255) / 256; t <= (n + 255) / 256 + 8; ++t) {
-      const int64_t w = ((n + t - 1) / t + 15) / 16 * 16;
-      if (w > 256 || w < 16) continue;
-      if (t * w < best) {
-        best = t * w;
-        nt = static_cast<int>(w);
-      }
-    }
-    const uint64_t mt = static_cast<uint64_t>(std::max<int64_t>(m_total + int64_t(BK) * num_groups, 1));
-    CUtensorMap amap2, bmap2;
-    const uint64_t adims[2] = {mt, static_cast<uint64_t>(n)};
-    const uint64_t astr[1] = {static_cast<uint64_t>(ld_a)};
-    const uint32_t abox[2] = {BK, static_cast<uint32_t>(nt / 2)};
-    const uint64_t bdims[2] = {mt, static_cast<uint64_t>(k)};
-    const uint64_t bstr[1] = {static_cast<uint64_t>(ld_b)};
-    const uint32_t bbox[2] = {BK, 128};
-    if (!encode_tensor_map(&amap2, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t *>(a),
-                           adims, astr, abox, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !encode_tensor_map(&bmap2, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t *>(b),
-                           bdims, bstr, bbox, CU_TENSOR_MAP_SWIZZLE_128B))
-      return FP8QGG_ERR_CUDA;
-    auto kern2 = out_dtype == FP8QGG_OUT_F32 ? grouped_gemm_k2_kernel<FP8QGG_OUT_F32>
-                                             : grouped_gemm_k2_kernel<FP8QGG_OUT_BF16>;
-    const int smem2 = static_cast<int>(sizeof(GemmK2Smem)) + 1024;
-    if (!set_max_dynamic_smem(reinterpret_cast<const void *>(kern2), smem2))
-      return FP8QGG_ERR_CUDA;
-    const int64_t pair_tiles = int64_t(num_groups) * ((k + 255) / 256) * ((n + nt - 1) / nt);
-    if (pair_tiles > INT32_MAX) return FP8QGG_ERR_SHAPE;
-    // output units of 32 (j) x 16 (i) elements, no swizzle
-    CUtensorMap omap2;
-    {
-      const CUtensorMapDataType odt = out_dtype == FP8QGG_OUT_F32
-                                          ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
-                                          : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
-      const uint64_t esz = out_dtype == FP8QGG_OUT_F32 ? 4 : 2;
-      const uint64_t dims[3] = {static_cast<uint64_t>(k), static_cast<uint64_t>(n),
-                                static_cast<uint64_t>(num_groups)};
-      const uint64_t gs = num_groups > 1 ? static_cast<uint64_t>(out_group_stride)
-                                         : static_cast<uint64_t>(n * ld_out);
-      const uint64_t str[2] = {static_cast<uint64_t>(ld_out) * esz, gs * esz};
-      const uint32_t box[3] = {32, 16, 1};
-      if (!encode_tensor_map(&omap2, odt, 3, out, dims, str, box, CU_TENSOR_MAP_SWIZZLE_NONE))
-        return FP8QGG_ERR_CUDA;
-    }
-    const int clusters =
-        static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(pair_tiles, dev.sm_count / 2)));
-    kern2<<<2 * clusters, kGemmThreads, smem2, static_cast<cudaStream_t>(stream)>>>(
-        amap2, bmap2, omap2, prm, nt);
     return cudaGetLastError() == cudaSuccess ? FP8QGG_OK : FP8QGG_ERR_CUDA;
   }
 

@@ -265,12 +265,11 @@ def test_k_jagged_group_starts_at_every_residue_of_a_block():
     ([700, 33] * 20, 96, 520, torch.float32),
     ([257, 0, 90], 200, 136, torch.bfloat16),
 ])
-def test_k_jagged_padded_pair_kernel_shapes(sizes, n, k, odt):
-    """The padded contraction-jagged GEMM (SM pairs, tiles of 256 x nt) on
-    shapes whose n and k are not tile multiples, with many groups (more tiles
-    than pairs), an empty group and bf16 output; every element against the
-    oracle (bf16 output: within the bound plus the bf16 rounding of the
-    output, 2^-8 relative)."""
+def test_k_jagged_padded_odd_shapes(sizes, n, k, odt):
+    """The padded contraction-jagged GEMM on shapes whose n and k are not tile
+    multiples, with many groups (more tiles than SMs), an empty group and bf16
+    output; every element against the oracle (bf16 output: within the bound
+    plus the bf16 rounding of the output, 2^-8 relative)."""
     m = int(sum(sizes))
     e = len(sizes)
     dh = rand_bf16(3 * m + n, (m, n), 1e-3)
