@@ -13,34 +13,29 @@
 //
 // B200 design.  The input is cut into panels of 256 columns (one warp load
 // instruction reads a whole 512-byte row segment; lane l owns columns
-// 8l .. 8l + 7) and blocks of 128 rows of one group; a block of a panel is
-// one task of a block of eight warps, each warp owning 16 rows.  A block of a
-// group with more than one block is visited twice:
-//  - an "absmax" task: every warp loads its 16 rows straight into registers
-//    (16 loads of 16 bytes in flight per lane) and reduces its column absmax;
-//    the warps meet in shared memory, then each warp merges 32 of the
-//    panel's columns into the unit's absmax words in global memory with
-//    relaxed atomic max and counts itself in the unit's arrival counter (the
-//    dual form also merges every row's absmax over the panel);
-//  - a "cast" task, later in the task list, once the unit's count is full:
-//    every lane derives its 8 scales, reads its rows again (from L2: the
-//    list keeps the two visits about one grid-width of tasks apart), encodes
-//    two rows of a column per conversion and writes each column's 16 tokens
-//    into a 32 KB shared-memory tile (256 columns x 128 tokens, 128-byte
-//    swizzle), which one bulk tensor store sends to the group's 128-token
-//    block of the padded layout: whole 128-byte lines, zero codes of the
-//    padding included (rows past the group's end are zeros).  The dual form
-//    also encodes every row with its own scale and stores it in place.
-// A single-block unit of the column-wise form is one "whole" task (absmax
-// and cast from the same registers).  The unit a cast waits for is one
-// (group, panel) in the column-wise form and the whole group in the dual
-// form (a row's scale needs every panel).  Tasks come from an atomic counter
-// read by warp 0, which also finds the next task (a 32-way search, one
-// candidate per lane) while the block works on the current one; each task
-// ends with the block's only barrier.  The absmax tasks run largest group
-// first, and the casts of a unit are placed about one grid-width of tasks
-// after its last absmax task, so that a cast only waits for tasks handed out
-// earlier (to running blocks).
+// 8l .. 8l + 7) and blocks of 128 rows of one group (16 rows per warp of an
+// eight-warp thread block).  The blocks are listed unit by unit, largest
+// group first, where a unit is one (group, panel) in the column-wise form and
+// one group (all its panels) in the dual form.  The kernel is a software
+// pipeline over that list: the thread block that takes step s from an
+// atomic counter
+//  - reads block s (HBM), reduces its column absmax (the warps meet in
+//    shared memory) and merges it into the unit's absmax words in global
+//    memory with relaxed atomic max, then counts it in the unit's arrival
+//    counter (the dual form also merges every row's absmax);
+//  - reads block s - D again (from L2: D blocks ago is about one grid-width
+//    plus the longest unit, so the block is still there and its unit's count
+//    is normally full already; the block waits for it, bounded, otherwise),
+//    derives the scales from the unit's absmax, encodes two rows of a column
+//    per conversion and writes each column's 16 tokens into a 32 KB tile
+//    (256 columns x 128 tokens, 128-byte swizzle) that one bulk tensor store
+//    sends to the group's 128-token block of the padded layout: whole
+//    128-byte lines, zero codes of the padding included (rows past the
+//    group's end are zeros).  The dual form also encodes every row with its
+//    own scale and stores it in place.
+// Every block is read once from HBM.  A step only waits for steps handed out
+// earlier (to running thread blocks), so no thread block waits for one that
+// is not running.
 #include <algorithm>
 #include <cstring>
 
@@ -49,6 +44,12 @@
 #include "quant_panels.h"
 
 namespace fp8qgg {
+
+// Build-time knob: the pipeline delay beyond the longest unit, in quarters
+// of the grid (the default is the best of the values measured on B200).
+#ifndef FP8QGG_PANEL_DELAY_Q
+#define FP8QGG_PANEL_DELAY_Q 5
+#endif
 
 constexpr int kPW = 256;               // columns per panel
 constexpr int kPWords = kPW / 2;       // bf16 pairs per panel row
@@ -61,30 +62,18 @@ constexpr int kPMaxGroups = 1024;
 constexpr uint32_t kTileBytes = kPW * kRB;
 static_assert(kWR == 16, "a lane's tokens of one column fill one 16-byte piece");
 
-enum : int { kTaskAbs = 0, kTaskCast = 1, kTaskWhole = 2, kTaskEnd = 3 };
-
-struct PTask {
-  int32_t kind;
-  int32_t i, e;   // ordered group, group index
-  int32_t q;      // panel
-  int32_t b;      // block of the group
-  int32_t u;      // unit (arrival counter)
-  int32_t need;   // arrivals that complete the unit
-  int32_t pad;
-};
-
 struct PanelSmem {
-  uint8_t tile[2][kTileBytes];          // transposed code tiles (1024-byte aligned)
-  uint32_t red[2][kPWarps][kPWords];    // per-warp column absmax (bf16 magnitude pairs)
-  PTask tk[2];                          // the current and the next task
+  uint8_t tile[kTileBytes];             // transposed code tile (1024-byte aligned)
+  uint32_t red[kPWarps][kPWords];       // per-warp column absmax (bf16 magnitude pairs)
   int32_t end[kPMaxGroups];             // clamped group ends (by group index)
   int32_t pstart[kPMaxGroups];          // padded first token (by group index)
   int32_t order[kPMaxGroups];           // groups by size, largest first
   int32_t nb[kPMaxGroups];              // ordered group i: 128-row blocks
-  int32_t apre[kPMaxGroups + 1];        // multi-block groups: blocks before group i
-  int32_t n_multi, n_nonempty, a_total, s_total, total;
+  int32_t apre[kPMaxGroups + 1];        // blocks of the groups before ordered group i
+  int32_t n_nonempty, total, delay;
+  int32_t step;
 };
-static_assert(offsetof(PanelSmem, tile) == 0, "tiles first (1024-byte aligned)");
+static_assert(offsetof(PanelSmem, tile) == 0, "store tile 1024-byte aligned");
 
 struct PanelParams {
   const uint4 *x;        // bf16 rows as 16-byte vectors
@@ -100,11 +89,10 @@ struct PanelParams {
   float smax, sat_thr;
   unsigned long long *sat_count;
   int32_t *status;
-  uint32_t *work;        // task counter
+  uint32_t *work;        // step counter
   uint32_t *arrive;      // per unit
   uint32_t *amax;        // [ordered group, cols] column absmax bits
   uint32_t *rowmax;      // dual form: [rows_total] row absmax bits
-  int32_t delay;         // list positions between a unit's last absmax task and its casts
   UnitWait uw;
 };
 
@@ -116,7 +104,8 @@ __device__ __forceinline__ int32_t warp_scan_incl(int32_t v, int lane) {
   return v;
 }
 
-// Clamped group ends, padded starts, the size order and the task counts.
+// Clamped group ends, padded starts, the size order, the block list and the
+// pipeline delay.
 template <bool DUAL>
 __device__ void panel_prologue(PanelSmem &sm, const PanelParams &p, int np) {
   const int tid = threadIdx.x, lane = tid & 31;
@@ -161,10 +150,7 @@ __device__ void panel_prologue(PanelSmem &sm, const PanelParams &p, int np) {
   }
   __syncthreads();
   if (tid < 32) {
-    // groups with absmax and cast tasks ("multi") are a prefix of the order:
-    // every non-empty group in the dual form, groups of more than one block
-    // in the column-wise form (single-block ones are whole tasks)
-    int32_t carry = 0, n_multi = 0, n_ne = 0;
+    int32_t carry = 0, n_ne = 0, nb_max = 0;
     for (int base = 0; base < G; base += 32) {
       const int i = base + lane;
       int32_t nbv = 0;
@@ -173,131 +159,56 @@ __device__ void panel_prologue(PanelSmem &sm, const PanelParams &p, int np) {
         nbv = (sm.end[e] - (e ? sm.end[e - 1] : 0) + kRB - 1) / kRB;
         sm.nb[i] = nbv;
       }
-      const bool multi = DUAL ? nbv >= 1 : nbv >= 2;
-      const int32_t c = multi ? nbv : 0;
-      const int32_t incl = warp_scan_incl(c, lane);
-      if (i < G) sm.apre[i] = carry + incl - c;
+      const int32_t incl = warp_scan_incl(nbv, lane);
+      if (i < G) sm.apre[i] = carry + incl - nbv;
       carry += __shfl_sync(0xFFFFFFFFu, incl, 31);
-      n_multi += __popc(__ballot_sync(0xFFFFFFFFu, multi));
       n_ne += __popc(__ballot_sync(0xFFFFFFFFu, nbv >= 1));
+      nb_max = max(nb_max, nbv);
     }
+    for (int d = 16; d > 0; d >>= 1) nb_max = max(nb_max, __shfl_xor_sync(0xFFFFFFFFu, nb_max, d));
     if (lane == 0) {
       sm.apre[G] = carry;
-      sm.n_multi = n_multi;
       sm.n_nonempty = n_ne;
-      sm.a_total = carry * np;
-      sm.s_total = sm.a_total + (DUAL ? 0 : (n_ne - n_multi) * np);
-      sm.total = sm.s_total + sm.a_total;  // one cast per absmax task
+      sm.total = carry * np;
+      // a unit's blocks are consecutive: the delay covers the longest unit and
+      // the steps the running blocks hold, with a quarter of margin
+      const int32_t span = DUAL ? nb_max * np : nb_max;
+      sm.delay = min(sm.total, span + (FP8QGG_PANEL_DELAY_Q * static_cast<int32_t>(gridDim.x)) / 4);
     }
   }
   __syncthreads();
 }
 
-// Unit u: first absmax index (= cast tasks before its cast block) and count.
-template <bool DUAL>
-__device__ __forceinline__ void unit_span(const PanelSmem &sm, int np, int u, int32_t &fa,
-                                          int32_t &na) {
-  if constexpr (DUAL) {
-    fa = sm.apre[u] * np;
-    na = sm.nb[u] * np;
-  } else {
-    const int i = u / np, q = u - (u / np) * np;
-    fa = sm.apre[i] * np + q * sm.nb[i];
-    na = sm.nb[i];
-  }
-}
+struct PBlock {
+  int32_t i, e;   // ordered group, group index
+  int32_t q, b;   // panel, block of the group
+  int32_t u;      // unit (arrival counter)
+  int32_t need;   // arrivals that complete the unit
+};
 
-// Task at position t of the list (called by a whole warp; every lane gets the
-// same task).  The "A stream" holds the absmax tasks of the multi units
-// (group i in size order, panel q, block b), then the whole tasks.  The cast
-// block of unit u (same blocks, same order) is inserted after A-stream index
-// d_u = min(fa_u + na_u + delay, S); the casts before it number fa_u, so it
-// starts at list position d_u + fa_u.
+// Block a of the list (the whole warp calls it; every lane gets the same
+// answer): the ordered group by a 32-way search over the block prefix.
 template <bool DUAL>
-__device__ PTask decode_panel_task(const PanelSmem &sm, int32_t t, int np, int32_t delay,
-                                   int lane) {
-  PTask r;
-  r.pad = 0;
-  if (t >= sm.total) {
-    r.kind = kTaskEnd;
-    r.i = r.e = r.q = r.b = r.u = r.need = 0;
-    return r;
+__device__ PBlock decode_block(const PanelSmem &sm, int32_t a, int np, int lane) {
+  int lo = 0, hi = sm.n_nonempty;  // apre[lo] * np <= a
+  while (hi - lo > 1) {
+    const int step = (hi - lo + 31) / 32;
+    const int c = lo + lane * step;
+    const bool ok = c < hi && sm.apre[c] * np <= a;
+    const int n = __popc(__ballot_sync(0xFFFFFFFFu, ok));  // lanes 0 .. n-1
+    const int nlo = lo + (n - 1) * step;
+    hi = min(hi, nlo + step);
+    lo = nlo;
   }
-  const int32_t S = sm.s_total;
-  const int U = DUAL ? sm.n_multi : sm.n_multi * np;
-  auto pos_of = [&](int u) -> int32_t {
-    int32_t fa, na;
-    unit_span<DUAL>(sm, np, u, fa, na);
-    return min(fa + na + delay, S) + fa;
-  };
-  int best = -1;
-  if (U > 0 && pos_of(0) <= t) {
-    int lo = 0, hi = U;  // pos(lo) <= t; the answer lies in [lo, hi)
-    while (hi - lo > 1) {
-      const int step = (hi - lo + 31) / 32;
-      const int c = lo + lane * step;
-      const bool ok = c < hi && pos_of(c) <= t;
-      const int n = __popc(__ballot_sync(0xFFFFFFFFu, ok));  // lanes 0 .. n-1
-      const int nlo = lo + (n - 1) * step;
-      hi = min(hi, nlo + step);
-      lo = nlo;
-    }
-    best = lo;
-  }
-  int32_t a = t;  // A-stream index, if t is not a cast
-  if (best >= 0) {
-    int32_t fa, na;
-    unit_span<DUAL>(sm, np, best, fa, na);
-    const int32_t pos = min(fa + na + delay, S) + fa;
-    if (t < pos + na) {
-      const int32_t k = t - pos;
-      r.kind = kTaskCast;
-      r.u = best;
-      r.need = kPWarps * na;  // every warp of every absmax task arrives
-      if constexpr (DUAL) {
-        r.i = best;
-        const int32_t per = sm.nb[best];
-        r.q = k / per;
-        r.b = k - r.q * per;
-      } else {
-        r.i = best / np;
-        r.q = best - r.i * np;
-        r.b = k;
-      }
-      r.e = sm.order[r.i];
-      return r;
-    }
-    a = t - (fa + na);  // every cast before t belongs to units 0 .. best
-  }
-  if (a < sm.a_total) {
-    int lo = 0, hi = sm.n_multi;  // apre[lo] * np <= a
-    while (hi - lo > 1) {
-      const int step = (hi - lo + 31) / 32;
-      const int c = lo + lane * step;
-      const bool ok = c < hi && sm.apre[c] * np <= a;
-      const int n = __popc(__ballot_sync(0xFFFFFFFFu, ok));
-      const int nlo = lo + (n - 1) * step;
-      hi = min(hi, nlo + step);
-      lo = nlo;
-    }
-    const int32_t nbi = sm.nb[lo];
-    const int32_t rr = a - sm.apre[lo] * np;
-    r.kind = kTaskAbs;
-    r.i = lo;
-    r.q = rr / nbi;
-    r.b = rr - r.q * nbi;
-    r.u = DUAL ? lo : lo * np + r.q;
-    r.need = 0;
-  } else {
-    const int32_t w = a - sm.a_total;  // whole task: single-block group, one panel
-    r.kind = kTaskWhole;
-    r.i = sm.n_multi + w / np;
-    r.q = w - (w / np) * np;
-    r.b = 0;
-    r.u = -1;
-    r.need = 0;
-  }
-  r.e = sm.order[r.i];
+  PBlock r;
+  const int32_t nbi = sm.nb[lo];
+  const int32_t rr = a - sm.apre[lo] * np;
+  r.i = lo;
+  r.e = sm.order[lo];
+  r.q = rr / nbi;
+  r.b = rr - r.q * nbi;
+  r.u = DUAL ? lo : lo * np + r.q;
+  r.need = kPWarps * (DUAL ? nbi * np : nbi);  // every warp of every block arrives
   return r;
 }
 
@@ -326,23 +237,6 @@ __device__ __forceinline__ float lo_f(uint32_t w) { return __uint_as_float(w << 
 __device__ __forceinline__ float hi_f(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 __device__ __forceinline__ uint32_t word(const uint4 &v, int j) {
   return j == 0 ? v.x : j == 1 ? v.y : j == 2 ? v.z : v.w;
-}
-
-// The lane's 16 rows x 8 columns from row rw0 (rows at or past r1 read as
-// zero).  SECOND: the cast's re-read, the data's last use.
-template <bool SECOND>
-__device__ __forceinline__ void load_rows(uint4 (&v)[kWR], const PanelParams &p, int32_t rw0,
-                                          int32_t r1, int64_t cvec, bool lane_ok) {
-#pragma unroll
-  for (int k = 0; k < kWR; ++k) {
-    const int32_t row = rw0 + k;
-    if (lane_ok && row < r1) {
-      const uint4 *src = p.x + static_cast<int64_t>(row) * p.ld_x16 + cvec;
-      v[k] = SECOND ? __ldcs(src) : __ldcg(src);
-    } else {
-      v[k] = make_uint4(0u, 0u, 0u, 0u);
-    }
-  }
 }
 
 // Dual form: every row's absmax over the lane's 8 columns, reduced over the
@@ -445,43 +339,69 @@ __global__ void __launch_bounds__(kPThreads, kPBlocksPerSM)
       p.scales_col[static_cast<int64_t>(e) * p.cols + c] = s;
   }
 
-  // warp 0 fetches and decodes the tasks, one ahead of the block
-  int32_t next = 0;
-  if (w == 0) {
-    int32_t t = 0;
-    if (lane == 0) {
-      t = static_cast<int32_t>(atomicAdd(p.work, 1u));
-      next = static_cast<int32_t>(atomicAdd(p.work, 1u));
-    }
-    t = __shfl_sync(0xFFFFFFFFu, t, 0);
-    const PTask tk = decode_panel_task<DUAL>(sm, t, np, p.delay, lane);
-    if (lane == 0) sm.tk[0] = tk;
-  }
-  __syncthreads();
-
+  const int32_t total = sm.total, delay = sm.delay;
+  const int32_t steps = total + delay;
   uint32_t sat = 0;
-  bool failed = false;
-  for (int n = 0;; ++n) {
-    const int cur = n & 1;
-    const PTask tk = sm.tk[cur];
-    if (tk.kind == kTaskEnd) break;
-    const int e = tk.e;
-    const int32_t gs = e ? sm.end[e - 1] : 0;
-    const int32_t ge = sm.end[e];
-    const int32_t r0 = gs + tk.b * kRB;
-    const int32_t r1 = min(ge, r0 + kRB);
-    const int32_t rw0 = r0 + kWR * w;
-    const int c0 = tk.q * kPW;
-    const bool lane_ok = c0 + 8 * lane < p.cols;
-    const int64_t cvec = (c0 >> 3) + lane;
-    const int64_t amax_base = static_cast<int64_t>(tk.i) * p.cols + c0;
-    uint8_t *tile = sm.tile[cur];
+  int32_t next = 0;
+  if (tid == 0) next = static_cast<int32_t>(atomicAdd(p.work, 1u));
+  while (true) {
+    if (tid == 0) {
+      sm.step = next;
+      if (next < steps) next = static_cast<int32_t>(atomicAdd(p.work, 1u));
+      bulk_wait_read<0>();  // the tile's previous store has read it
+    }
+    __syncthreads();
+    const int32_t st = sm.step;
+    if (st >= steps) break;
+    const bool has_a = st < total;
+    const bool has_c = st >= delay;
+    PBlock A{}, C{};
+    if (has_a) A = decode_block<DUAL>(sm, st, np, lane);
+    if (has_c) C = decode_block<DUAL>(sm, st - delay, np, lane);
 
-    uint4 v[kWR];
-    float s[8];
-    if (tk.kind != kTaskCast) {
-      // ---------------------------------------------------------- absmax
-      load_rows<false>(v, p, rw0, r1, cvec, lane_ok);
+    // the cast's scale words, early when the unit is complete already
+    bool c_ready = false;
+    uint4 ua0 = make_uint4(0u, 0u, 0u, 0u), ua1 = ua0;
+    uint32_t urow = 0;
+    const int cc0 = C.q * kPW;
+    const bool c_lane = has_c && cc0 + 8 * lane < p.cols;
+    if (has_c) {
+      uint32_t cnt = 0;
+      if (lane == 0)
+        asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(cnt) : "l"(p.arrive + C.u)
+                     : "memory");
+      c_ready = __shfl_sync(0xFFFFFFFFu, cnt, 0) >= static_cast<uint32_t>(C.need) +
+                                                     p.uw.extra_arrivals;
+    }
+    auto load_c_words = [&]() {
+      if (c_lane) {
+        const uint4 *src = reinterpret_cast<const uint4 *>(
+            p.amax + static_cast<int64_t>(C.i) * p.cols + cc0 + 8 * lane);
+        ua0 = __ldcg(src);
+        ua1 = __ldcg(src + 1);
+      }
+      if constexpr (DUAL) {
+        const int32_t cgs = C.e ? sm.end[C.e - 1] : 0;
+        const int32_t row = cgs + C.b * kRB + kWR * w + lane;
+        const int32_t r1 = min(sm.end[C.e], cgs + C.b * kRB + kRB);
+        urow = (lane < kWR && row < r1) ? __ldcg(p.rowmax + row) : 0u;
+      }
+    };
+    if (c_ready) load_c_words();
+
+    // ---------------------------------------------------------- absmax of block s
+    if (has_a) {
+      const int32_t gs = A.e ? sm.end[A.e - 1] : 0;
+      const int32_t r0 = gs + A.b * kRB;
+      const int32_t r1 = min(sm.end[A.e], r0 + kRB);
+      const int32_t rw0 = r0 + kWR * w;
+      const int c0 = A.q * kPW;
+      const bool lane_ok = c0 + 8 * lane < p.cols;
+      const uint4 *src = p.x + static_cast<int64_t>(rw0) * p.ld_x16 + (c0 >> 3) + lane;
+      uint4 v[kWR];
+#pragma unroll
+      for (int k = 0; k < kWR; ++k)
+        v[k] = (lane_ok && rw0 + k < r1) ? __ldcg(src + k * p.ld_x16) : make_uint4(0u, 0u, 0u, 0u);
       uint4 am = make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
       for (int k = 0; k < kWR; ++k) {
@@ -491,139 +411,119 @@ __global__ void __launch_bounds__(kPThreads, kPBlocksPerSM)
         am.w = absmax_acc(am.w, v[k].w);
       }
       if constexpr (DUAL) merge_row_amax(v, p.rowmax, rw0, r1, lane);
-      *reinterpret_cast<uint4 *>(&sm.red[cur][w][4 * lane]) =
+      *reinterpret_cast<uint4 *>(&sm.red[w][4 * lane]) =
           make_uint4(absmax_bits(am.x), absmax_bits(am.y), absmax_bits(am.z),
                      absmax_bits(am.w));
-      if (tk.kind == kTaskWhole) {
-        // single block: the block's column absmax is the unit's; its scales
-        // and codes come from the same registers
-        __syncthreads();
-        uint4 mm = make_uint4(0u, 0u, 0u, 0u);
+    }
+    __syncthreads();
+    if (has_a) {
+      // each warp merges 32 of the panel's columns into the unit's absmax:
+      // column 32w + lane is half (lane & 1) of word 16w + lane / 2
+      const int wd = 16 * w + (lane >> 1);
+      uint32_t m = 0;
 #pragma unroll
-        for (int ww = 0; ww < kPWarps; ++ww) {
-          const uint4 o = *reinterpret_cast<const uint4 *>(&sm.red[cur][ww][4 * lane]);
-          mm.x = __vmaxu2(mm.x, o.x);
-          mm.y = __vmaxu2(mm.y, o.y);
-          mm.z = __vmaxu2(mm.z, o.z);
-          mm.w = __vmaxu2(mm.w, o.w);
-        }
-        const uint32_t a[8] = {mm.x & 0xFFFFu, mm.x >> 16, mm.y & 0xFFFFu, mm.y >> 16,
-                               mm.z & 0xFFFFu, mm.z >> 16, mm.w & 0xFFFFu, mm.w >> 16};
-#pragma unroll
-        for (int j = 0; j < 8; ++j) s[j] = scale_from_amax(bf16_bits_to_float(a[j]), p.smax);
-        if (w == 0 && lane_ok)
-          store_scales8(p.scales_col + static_cast<int64_t>(e) * p.cols + c0 + 8 * lane, s);
-        tile_col_codes<FMT, FAST>(v, s, tile, w, lane, p.smax, p.sat_thr, sat);
-        fence_proxy_async_smem();
-      }
-    } else {
-      // ---------------------------------------------------------- cast
-      int ok = 1;
-      if (lane == 0) {  // every warp waits (bounded) for the unit's count
-        const uint32_t *cnt = p.arrive + tk.u;
-        const uint32_t target = static_cast<uint32_t>(tk.need) + p.uw.extra_arrivals;
-        uint32_t c;
-        asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(c) : "l"(cnt) : "memory");
-        if (c < target) {
+      for (int ww = 0; ww < kPWarps; ++ww) m = __vmaxu2(m, sm.red[ww][wd]);
+      const int c0 = A.q * kPW;
+      const int cc = 32 * w + lane;
+      if (c0 + cc < p.cols)
+        atomicMax(p.amax + static_cast<int64_t>(A.i) * p.cols + c0 + cc,
+                  (lane & 1) ? m >> 16 : m & 0xFFFFu);
+    }
+    // (the warp counts its merge below, after the fence, which then overlaps
+    // the cast's loads)
+
+    // ---------------------------------------------------------- cast of block s - D
+    bool failed = false;
+    if (has_c && !c_ready) {  // wait (bounded) until every block of the unit is counted
+        int ok = 1;
+        if (lane == 0) {
+          const uint32_t target = static_cast<uint32_t>(C.need) + p.uw.extra_arrivals;
           const uint64_t t0 = global_timer_ns();
           while (true) {
-            __nanosleep(64);
-            asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(c) : "l"(cnt) : "memory");
+            uint32_t c;
+            asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(c) : "l"(p.arrive + C.u)
+                         : "memory");
             if (c >= target) break;
             if (global_timer_ns() - t0 > p.uw.limit_ns) { ok = 0; break; }
+            __nanosleep(64);
           }
         }
-      }
-      ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
-      if (ok) {  // every lane acquires the count it relies on
-        uint32_t c;
-        asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(c) : "l"(p.arrive + tk.u)
-                     : "memory");
-        (void)c;
-      } else {
-        failed = true;
-      }
-      if (!failed) {
-        uint4 a0 = make_uint4(0u, 0u, 0u, 0u), a1 = a0;
-        if (lane_ok) {
-          const uint4 *src = reinterpret_cast<const uint4 *>(p.amax + amax_base + 8 * lane);
-          a0 = __ldcg(src);
-          a1 = __ldcg(src + 1);
+        ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+        if (ok) {
+          uint32_t c;  // every lane acquires the count it relies on
+          asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(c) : "l"(p.arrive + C.u)
+                       : "memory");
+          (void)c;
+          load_c_words();
+        } else {
+          failed = true;
         }
-        const uint32_t a[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+    }
+    uint4 v[kWR];
+    int32_t c_r1 = 0, c_rw0 = 0;
+    if (has_c && !failed) {
+      const int32_t gs = C.e ? sm.end[C.e - 1] : 0;
+      const int32_t r0 = gs + C.b * kRB;
+      c_r1 = min(sm.end[C.e], r0 + kRB);
+      c_rw0 = r0 + kWR * w;
+      const uint4 *src = p.x + static_cast<int64_t>(c_rw0) * p.ld_x16 + (cc0 >> 3) + lane;
+#pragma unroll
+      for (int k = 0; k < kWR; ++k)
+        v[k] = (c_lane && c_rw0 + k < c_r1) ? __ldcs(src + k * p.ld_x16)
+                                            : make_uint4(0u, 0u, 0u, 0u);
+    }
+    if (has_a) {
+      __threadfence();  // every lane's merge is visible before the count
+      __syncwarp();
+      if (lane == 0) atomicAdd(p.arrive + A.u, 1u);
+    }
+    if (has_c) {
+      if (!failed) {
+        const int e = C.e;
+        const int32_t r1 = c_r1, rw0 = c_rw0;
+        float s[8];
+        const uint32_t a[8] = {ua0.x, ua0.y, ua0.z, ua0.w, ua1.x, ua1.y, ua1.z, ua1.w};
 #pragma unroll
         for (int j = 0; j < 8; ++j) s[j] = scale_from_amax(bf16_bits_to_float(a[j]), p.smax);
-        if (tk.b == 0 && w == 0 && lane_ok)
-          store_scales8(p.scales_col + static_cast<int64_t>(e) * p.cols + c0 + 8 * lane, s);
-        float rs_lane = 0.0f;  // dual form: the scale of row rw0 + lane (lanes 0..15)
+        if (C.b == 0 && w == 0 && c_lane)
+          store_scales8(p.scales_col + static_cast<int64_t>(e) * p.cols + cc0 + 8 * lane, s);
         if constexpr (DUAL) {
-          const int32_t row = rw0 + lane;
-          if (lane < kWR && row < r1) {
-            rs_lane = scale_from_amax(bf16_bits_to_float(__ldcg(p.rowmax + row)), p.smax);
-            if (tk.q == 0) p.scales_row[row] = rs_lane;
+          float rs_lane = 0.0f;  // the scale of row rw0 + lane (lanes 0..15)
+          if (lane < kWR && rw0 + lane < r1) {
+            rs_lane = scale_from_amax(bf16_bits_to_float(urow), p.smax);
+            if (C.q == 0) p.scales_row[rw0 + lane] = rs_lane;
           }
-        }
-        load_rows<true>(v, p, rw0, r1, cvec, lane_ok);
-        if constexpr (DUAL) {
           // rowwise codes in place: 8 columns of a row per lane, one 8-byte store
 #pragma unroll
           for (int k = 0; k < kWR; ++k) {
             const float rs = __shfl_sync(0xFFFFFFFFu, rs_lane, k);
-            const int32_t row = rw0 + k;
             uint32_t c2[4];
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
               const uint32_t wd = word(v[k], j);
               c2[j] = enc_pair<FMT, FAST>(lo_f(wd), hi_f(wd), rs, rs, p.smax, p.sat_thr, sat);
             }
-            if (lane_ok && row < r1)
-              *reinterpret_cast<uint2 *>(p.q_row + static_cast<int64_t>(row) * p.ld_qr + c0 +
-                                         8 * lane) =
+            if (c_lane && rw0 + k < r1)
+              *reinterpret_cast<uint2 *>(p.q_row + static_cast<int64_t>(rw0 + k) * p.ld_qr +
+                                         cc0 + 8 * lane) =
                   make_uint2(c2[0] | (c2[1] << 16), c2[2] | (c2[3] << 16));
           }
         }
-        tile_col_codes<FMT, FAST>(v, s, tile, w, lane, p.smax, p.sat_thr, sat);
+        tile_col_codes<FMT, FAST>(v, s, sm.tile, w, lane, p.smax, p.sat_thr, sat);
         fence_proxy_async_smem();
       }
     }
-
-    // warp 0: the next task; the tile written above may only be reused once
-    // the store that read it two tasks ago has finished reading
-    if (w == 0) {
-      int32_t t = 0;
-      if (lane == 0) {
-        t = next;
-        if (t < sm.total) next = static_cast<int32_t>(atomicAdd(p.work, 1u));
-        bulk_wait_read<0>();
-      }
-      t = __shfl_sync(0xFFFFFFFFu, t, 0);
-      const PTask nt = decode_panel_task<DUAL>(sm, t, np, p.delay, lane);
-      if (lane == 0) sm.tk[cur ^ 1] = nt;
-    }
-    // a warp that gave up on its wait stops the block after this task
     if (__syncthreads_or(failed)) {
       if (tid == 0) status_or(p.status, FP8QGG_STATUS_TIMEOUT);
-      break;
+      break;  // this block takes no more steps
     }
-
-    if (tk.kind == kTaskAbs) {
-      // each warp merges 32 of the panel's columns into the unit's absmax and
-      // counts itself: column 32w + lane is half (lane & 1) of word 16w + lane / 2
-      const int wd = 16 * w + (lane >> 1);
-      uint32_t m = 0;
-#pragma unroll
-      for (int ww = 0; ww < kPWarps; ++ww) m = __vmaxu2(m, sm.red[cur][ww][wd]);
-      const int cc = 32 * w + lane;
-      if (c0 + cc < p.cols) atomicMax(p.amax + amax_base + cc, (lane & 1) ? m >> 16 : m & 0xFFFFu);
-      __threadfence();
-      __syncwarp();
-      if (lane == 0) atomicAdd(p.arrive + tk.u, 1u);
-    } else if (tid == 0) {
-      tma_store_2d(&qmap, tile, sm.pstart[e] + tk.b * kRB, c0);
+    if (has_c && tid == 0) {
+      const int32_t ps = sm.pstart[C.e] + C.b * kRB;
+      tma_store_2d(&qmap, sm.tile, ps, cc0);
       bulk_commit();
     }
   }
-  if (tid == 0) bulk_wait_all();  // the tiles stay valid until their stores have read them
+  if (tid == 0) bulk_wait_all();  // the tile stays valid until its stores have read it
   if (!FAST && p.sat_count) {
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) sat += __shfl_xor_sync(0xFFFFFFFFu, sat, off);
@@ -707,14 +607,12 @@ int panel_launch(const void *x, int64_t rows_total, int64_t cols, int64_t ld_x,
   prm.amax = reinterpret_cast<uint32_t *>(base + sl.amax_off);
   prm.rowmax = reinterpret_cast<uint32_t *>(base + sl.rowmax_off);
   prm.uw = uw;
-  // blocks: kPBlocksPerSM per SM, never more than the tasks need (at least
-  // one, for the scales of empty groups)
+  // thread blocks: kPBlocksPerSM per SM, never more than the steps need (at
+  // least one, for the scales of empty groups)
   const int64_t np = (cols + kPW - 1) / kPW;
   const int64_t blocks = (rows_total + int64_t(kRB) * num_groups) / kRB * np;
   const int grid = static_cast<int>(std::max<int64_t>(
-      1, std::min<int64_t>(2 * blocks, int64_t(dev.sm_count) * kPBlocksPerSM)));
-  // a cast waits for absmax tasks that the running blocks have taken by then
-  prm.delay = grid;
+      1, std::min<int64_t>(blocks, int64_t(dev.sm_count) * kPBlocksPerSM)));
   kern<<<grid, kPThreads, smem, stream>>>(qmap, prm);
   return cudaGetLastError() == cudaSuccess ? FP8QGG_OK : FP8QGG_ERR_CUDA;
 }
