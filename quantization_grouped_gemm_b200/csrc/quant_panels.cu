@@ -428,36 +428,37 @@ __global__ void __launch_bounds__(kPThreads, kPBlocksPerSM)
       if (c0 + cc < p.cols)
         atomicMax(p.amax + static_cast<int64_t>(A.i) * p.cols + c0 + cc,
                   (lane & 1) ? m >> 16 : m & 0xFFFFu);
+      __threadfence();  // every lane's merge is visible before the count
+      __syncwarp();
+      if (lane == 0) atomicAdd(p.arrive + A.u, 1u);
     }
-    // (the warp counts its merge below, after the fence, which then overlaps
-    // the cast's loads)
 
     // ---------------------------------------------------------- cast of block s - D
     bool failed = false;
     if (has_c && !c_ready) {  // wait (bounded) until every block of the unit is counted
-        int ok = 1;
-        if (lane == 0) {
-          const uint32_t target = static_cast<uint32_t>(C.need) + p.uw.extra_arrivals;
-          const uint64_t t0 = global_timer_ns();
-          while (true) {
-            uint32_t c;
-            asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(c) : "l"(p.arrive + C.u)
-                         : "memory");
-            if (c >= target) break;
-            if (global_timer_ns() - t0 > p.uw.limit_ns) { ok = 0; break; }
-            __nanosleep(64);
-          }
-        }
-        ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
-        if (ok) {
-          uint32_t c;  // every lane acquires the count it relies on
+      int ok = 1;
+      if (lane == 0) {
+        const uint32_t target = static_cast<uint32_t>(C.need) + p.uw.extra_arrivals;
+        const uint64_t t0 = global_timer_ns();
+        while (true) {
+          uint32_t c;
           asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(c) : "l"(p.arrive + C.u)
                        : "memory");
-          (void)c;
-          load_c_words();
-        } else {
-          failed = true;
+          if (c >= target) break;
+          if (global_timer_ns() - t0 > p.uw.limit_ns) { ok = 0; break; }
+          __nanosleep(64);
         }
+      }
+      ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+      if (ok) {
+        uint32_t c;  // every lane acquires the count it relies on
+        asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(c) : "l"(p.arrive + C.u)
+                     : "memory");
+        (void)c;
+        load_c_words();
+      } else {
+        failed = true;
+      }
     }
     uint4 v[kWR];
     int32_t c_r1 = 0, c_rw0 = 0;
@@ -471,11 +472,6 @@ __global__ void __launch_bounds__(kPThreads, kPBlocksPerSM)
       for (int k = 0; k < kWR; ++k)
         v[k] = (c_lane && c_rw0 + k < c_r1) ? __ldcs(src + k * p.ld_x16)
                                             : make_uint4(0u, 0u, 0u, 0u);
-    }
-    if (has_a) {
-      __threadfence();  // every lane's merge is visible before the count
-      __syncwarp();
-      if (lane == 0) atomicAdd(p.arrive + A.u, 1u);
     }
     if (has_c) {
       if (!failed) {
