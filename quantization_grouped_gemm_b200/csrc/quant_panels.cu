@@ -428,9 +428,10 @@ __global__ void __launch_bounds__(kPThreads, kPBlocksPerSM)
       if (c0 + cc < p.cols)
         atomicMax(p.amax + static_cast<int64_t>(A.i) * p.cols + c0 + cc,
                   (lane & 1) ? m >> 16 : m & 0xFFFFu);
-      __threadfence();  // every lane's merge is visible before the count
+      // the lanes' merges happen before lane 0's release of the count
       __syncwarp();
-      if (lane == 0) atomicAdd(p.arrive + A.u, 1u);
+      if (lane == 0)
+        asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(p.arrive + A.u) : "memory");
     }
 
     // ---------------------------------------------------------- cast of block s - D
