@@ -281,3 +281,70 @@ def fp8_cast_f32(y, fmt=E4M3FN, q=None, sat_count=None, stream=None):
     rc = lib().fp8_cast_f32(_ptr(y), y.numel(), _ptr(q), fmt, _stream(stream))
     _check(rc, "fp8_cast_f32")
     return q
+
+
+class Fp8WeightCache:
+    """FP8 codes and scales of weights kept between calls.
+
+    Expert weights change only at optimizer steps, while the forward and
+    backward passes of every micro-batch in between need their FP8 copies
+    ("AMD Primus adds FP8/MXFP8 kernels ...", "What Primus adds for MoE
+    training on MI355X": FP8 weight caching).  A cached copy is reused while
+    the weight is the same tensor (storage, shape, strides) at the same
+    in-place version (torch bumps ``tensor._version`` on every in-place
+    update, which is how optimizers write parameters), and the quantisation
+    is re-run, into the same buffers, when it changed.  This class only
+    decides whether to call the library; every code and scale comes from the
+    library's kernels.
+
+    ``quantize`` is the function that fills (q, scales); it defaults to the
+    library call and can be replaced (for instance by a counting wrapper).
+    """
+
+    def __init__(self, quantize=None):
+        self._quantize = quantize
+        self._entries = {}
+        self.hits = 0
+        self.misses = 0
+
+    def _key(self, w, kind, args):
+        return (kind, w.data_ptr(), tuple(w.shape), tuple(w.stride()), w.dtype, args)
+
+    def rowwise(self, w, fmt=E4M3FN, scale_max=0.0):
+        """(q, scales) of fp8_quant_rowwise(w), reused while w is unchanged."""
+        q_fn = self._quantize or fp8_quant_rowwise
+        key = self._key(w, "rowwise", (fmt, float(scale_max)))
+        ent = self._entries.get(key)
+        if ent is not None and ent[0] == w._version:
+            self.hits += 1
+            return ent[1], ent[2]
+        self.misses += 1
+        if ent is None:
+            q, s = q_fn(w, fmt=fmt, scale_max=scale_max)
+        else:
+            q, s = q_fn(w, fmt=fmt, scale_max=scale_max, q=ent[1], scales=ent[2])
+        self._entries[key] = (w._version, q, s)
+        return q, s
+
+    def colwise_jagged(self, w, offsets, layout=LAYOUT_SAME, fmt=E4M3FN, scale_max=0.0):
+        """(q, scales) of fp8_quant_colwise_jagged(w, offsets, layout), reused
+        while w and offsets are unchanged."""
+        q_fn = self._quantize or fp8_quant_colwise_jagged
+        key = self._key(w, "colwise", (layout, fmt, float(scale_max), offsets.data_ptr(),
+                                       offsets.numel()))
+        ent = self._entries.get(key)
+        ver = (w._version, offsets._version)
+        if ent is not None and ent[0] == ver:
+            self.hits += 1
+            return ent[1], ent[2]
+        self.misses += 1
+        if ent is None:
+            q, s = q_fn(w, offsets, layout, fmt=fmt, scale_max=scale_max)
+        else:
+            q, s = q_fn(w, offsets, layout, fmt=fmt, scale_max=scale_max, q=ent[1],
+                        scales=ent[2])
+        self._entries[key] = (ver, q, s)
+        return q, s
+
+    def clear(self):
+        self._entries.clear()
