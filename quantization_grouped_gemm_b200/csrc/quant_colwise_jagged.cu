@@ -1,6 +1,9 @@
 // Jagged column-wise FP8 quantisation: for every expert group (rows given by
 // the int32 offsets tensor) and every column, absmax -> scale -> clamp -> RNE
-// e4m3 cast, with an optional fused transpose.
+// e4m3 cast, in the same layout or with a fused transpose (tokens at their
+// original positions).  The padded transposed layout and the dual-output form
+// run on the panel kernel (quant_panels.cu); this file also holds the entry
+// points, the argument checks and the no-allocation variant for all layouts.
 //
 // Sources: "FP8 su GPU AMD: ..." (ai-radar.it) — introduction (one scale per
 // column of each expert's weights, an offsets tensor routing tokens), section
@@ -115,7 +118,6 @@ struct ColSmem {
   int32_t end[kMaxGroups];
   int32_t order[kMaxGroups];                 // groups by row span, largest first
   int32_t prefix[kMaxGroups];                // tall groups: first amax task of the group
-  int32_t pstart[kMaxGroups];                // padded transposed layout: group's first token
   uint64_t full[kSlots];
   uint64_t empty[kSlots];
   uint64_t red_bar[kRedBufs];
@@ -159,32 +161,16 @@ __device__ __forceinline__ int32_t group_start(const ColSmem &sm, int e) {
 }
 
 // Rows a group's units cover: from their first row (the group's first row
-// rounded down with bmask: to 16 rows for the plain layouts, not at all for
-// the padded transposed one) to the group's end (0 for an empty group).
+// rounded down with bmask, to 16 rows) to the group's end (0 for an empty
+// group).
 __device__ __forceinline__ int32_t group_span(const ColSmem &sm, int e, int32_t bmask) {
   const int32_t s = group_start(sm, e);
   const int32_t g = sm.end[e];
   return g > s ? g - (s & bmask) : 0;
 }
 
-// Base-row mask of a layout: the padded transposed layout starts a group's
-// units on its first row, so that token runs stay 4-byte aligned relative to
-// the group's 128-aligned padded start; the others on the 16-aligned row.
-template <int LAYOUT>
-constexpr int32_t base_mask() {
-  return LAYOUT == FP8QGG_LAYOUT_TRANSPOSED_PADDED ? ~0 : ~15;
-}
-
-// Offset from a row of group e to its token in the codes: the padded
-// transposed layout moves the group to its 128-aligned first token (never
-// below its first row, as every padded size is at least the size).
-template <int LAYOUT>
-__device__ __forceinline__ int64_t token_shift(const ColSmem &sm, int e) {
-  if constexpr (LAYOUT == FP8QGG_LAYOUT_TRANSPOSED_PADDED)
-    return static_cast<int64_t>(sm.pstart[e]) - group_start(sm, e);
-  else
-    return 0;
-}
+// Units start on the 16-aligned row at or below a group's first row.
+constexpr int32_t kBaseMask = ~15;
 
 struct Task {
   int16_t kind;
@@ -462,10 +448,10 @@ __global__ void __launch_bounds__(kColThreads, kBlocksPerSM)
   __syncthreads();
   // groups ranked by row span, largest first (ties by index)
   for (int e = tid; e < num_groups; e += kColThreads) {
-    const int32_t se = group_span(sm, e, base_mask<LAYOUT>());
+    const int32_t se = group_span(sm, e, kBaseMask);
     int rank = 0;
     for (int f = 0; f < num_groups; ++f) {
-      const int32_t sf = group_span(sm, f, base_mask<LAYOUT>());
+      const int32_t sf = group_span(sm, f, kBaseMask);
       rank += (sf > se) || (sf == se && f < e);
     }
     sm.order[rank] = e;
@@ -480,7 +466,7 @@ __global__ void __launch_bounds__(kColThreads, kBlocksPerSM)
       const int i = base + lane;
       int32_t c = 0;
       if (i < num_groups) {
-        const int32_t sp = group_span(sm, sm.order[i], base_mask<LAYOUT>());
+        const int32_t sp = group_span(sm, sm.order[i], kBaseMask);
         if (sp > kChunkRows) c = n_ct * ((sp + kChunkRows - 1) / kChunkRows);
       }
       int32_t incl = c;
@@ -496,25 +482,9 @@ __global__ void __launch_bounds__(kColThreads, kBlocksPerSM)
       sm.n_tall = n_tall;
       sm.na = carry;
       const int32_t c_max =
-          n_tall ? (group_span(sm, sm.order[0], base_mask<LAYOUT>()) + kChunkRows - 1) / kChunkRows : 0;
+          n_tall ? (group_span(sm, sm.order[0], kBaseMask) + kChunkRows - 1) / kChunkRows : 0;
       sm.lag = max(FP8QGG_COLWISE_LAG_HALF_GRIDS * static_cast<int32_t>(gridDim.x) / 2, c_max);
       sm.total = 2 * carry + (num_groups - n_tall) * n_ct;
-    }
-    if constexpr (LAYOUT == FP8QGG_LAYOUT_TRANSPOSED_PADDED) {
-      // first token of each group: the previous groups' sizes rounded up to 128
-      int32_t pc = 0;
-      for (int base = 0; base < num_groups; base += 32) {
-        const int e = base + lane;
-        const int32_t sz = e < num_groups ? sm.end[e] - group_start(sm, e) : 0;
-        const int32_t ps = (sz + 127) & ~127;
-        int32_t incl = ps;
-        for (int d = 1; d < 32; d <<= 1) {
-          const int32_t o = __shfl_up_sync(0xFFFFFFFFu, incl, d);
-          if (lane >= d) incl += o;
-        }
-        if (e < num_groups) sm.pstart[e] = pc + incl - ps;
-        pc += __shfl_sync(0xFFFFFFFFu, incl, 31);
-      }
     }
   }
   __syncthreads();
@@ -604,7 +574,7 @@ __global__ void __launch_bounds__(kColThreads, kBlocksPerSM)
       int32_t next = static_cast<int32_t>(atomicAdd(work_counter, 1u));
       while (ok && t < total) {
         const int32_t next2 = static_cast<int32_t>(atomicAdd(work_counter, 1u));
-        const Task tk = decode_task(sm, t, n_ct, base_mask<LAYOUT>());
+        const Task tk = decode_task(sm, t, n_ct, kBaseMask);
         SlotMeta m;
         m.c0 = tk.ct * kCW;
         m.e = tk.e;
@@ -735,7 +705,7 @@ __global__ void __launch_bounds__(kColThreads, kBlocksPerSM)
         split_bits(a, mm);
         scales_from_bits<LAYOUT>(sc, a, smax, lane);
         if (w == 0) write_scales<LAYOUT>(sc, scales, m.e, m.c0, cols, lane);
-        uint8_t *const qe = q + token_shift<LAYOUT>(sm, m.e);
+        uint8_t *const qe = q;
 #pragma unroll
         for (int b = 0; b < kChunkBoxes; ++b)
           if (b < nb)
@@ -759,7 +729,7 @@ __global__ void __launch_bounds__(kColThreads, kBlocksPerSM)
           if ((m.flags & kFirstBox) && (m.flags & kWriteScales) && w == 0)
             write_scales<LAYOUT>(sc, scales, m.e, m.c0, cols, lane);
           cast_block<FMT, LAYOUT, FAST>(blk, ys, r0, r1, m.c0, cols,
-                                        q + token_shift<LAYOUT>(sm, m.e), ld_q, sc, smax,
+                                        q, ld_q, sc, smax,
                                         sat_thr, sat, lane);
         } else {
           uint4 &am = chunk_am;
@@ -816,76 +786,6 @@ __global__ void __launch_bounds__(kColThreads, kBlocksPerSM)
   }
 }
 
-// Zero codes of the padded transposed layout: for every group e and column c,
-// tokens [P_e + size_e, P_e + round_up(size_e, 128)) of row c of the codes.
-// The run is shorter than 128 tokens and ends on a multiple of 128 (P_e is
-// one, and ld_q a multiple of 16), so it lies in the 128-byte window that
-// ends there: a warp takes four columns, eight lanes per column, one 16-byte
-// piece of the window per lane.  The lane holding the run's first token
-// clears the bytes up to its piece's end with naturally aligned 1, 2, 4 and
-// 8-byte stores.  Every block rebuilds the clamped ends and padded starts
-// (warp 0 scans).
-__global__ void __launch_bounds__(256) pad_transposed_kernel(const int32_t *__restrict__ offsets,
-                                                             int num_groups, int64_t rows_total,
-                                                             int cols, uint8_t *__restrict__ q,
-                                                             int64_t ld_q) {
-  __shared__ int32_t s_start[kMaxGroups], s_size[kMaxGroups];
-  const int lane = threadIdx.x & 31;
-  if (threadIdx.x < 32) {
-    const int32_t R = static_cast<int32_t>(rows_total);
-    int32_t carry_end = 0, carry_pad = 0;
-    for (int base = 0; base < num_groups; base += 32) {
-      const int e = base + lane;
-      int32_t run = e < num_groups ? max(__ldg(offsets + e), 0) : 0;
-      for (int d = 1; d < 32; d <<= 1) {
-        const int32_t o = __shfl_up_sync(0xFFFFFFFFu, run, d);
-        if (lane >= d) run = max(run, o);
-      }
-      const int32_t endv = min(R, max(carry_end, run));
-      int32_t prev = __shfl_up_sync(0xFFFFFFFFu, endv, 1);
-      if (lane == 0) prev = carry_end;
-      const int32_t sz = e < num_groups ? endv - prev : 0;
-      const int32_t ps = (sz + 127) & ~127;
-      int32_t incl = ps;
-      for (int d = 1; d < 32; d <<= 1) {
-        const int32_t o = __shfl_up_sync(0xFFFFFFFFu, incl, d);
-        if (lane >= d) incl += o;
-      }
-      if (e < num_groups) {
-        s_start[e] = carry_pad + incl - ps;
-        s_size[e] = sz;
-      }
-      carry_end = __shfl_sync(0xFFFFFFFFu, endv, 31);
-      carry_pad += __shfl_sync(0xFFFFFFFFu, incl, 31);
-    }
-  }
-  __syncthreads();
-  const int64_t quads = (cols + 3) / 4;
-  const int64_t items = static_cast<int64_t>(num_groups) * quads;
-  const int64_t nwarps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
-  for (int64_t it = blockIdx.x * int64_t(blockDim.x >> 5) + (threadIdx.x >> 5); it < items;
-       it += nwarps) {
-    const int e = static_cast<int>(it / quads);
-    const int64_t c = (it - int64_t(e) * quads) * 4 + (lane >> 3);
-    const int32_t sz = s_size[e];
-    const int64_t lo = s_start[e] + int64_t(sz);
-    const int64_t hi = s_start[e] + int64_t((sz + 127) & ~127);
-    if (c >= cols || lo >= hi) continue;
-    const int64_t t0 = hi - 16 * (8 - (lane & 7));  // this lane's piece [t0, t0 + 16)
-    if (t0 + 16 <= lo) continue;
-    uint8_t *row = q + c * ld_q;
-    if (t0 >= lo) {
-      *reinterpret_cast<uint4 *>(row + t0) = make_uint4(0u, 0u, 0u, 0u);
-    } else {
-      int64_t t = lo;  // up to the next 16-byte boundary, t0 + 16
-      if (t & 1) { row[t] = 0; t += 1; }
-      if (t & 2) { *reinterpret_cast<uint16_t *>(row + t) = 0; t += 2; }
-      if (t & 4) { *reinterpret_cast<uint32_t *>(row + t) = 0u; t += 4; }
-      if (t & 8) { *reinterpret_cast<uint2 *>(row + t) = make_uint2(0u, 0u); }
-    }
-  }
-}
-
 namespace {
 
 using ColKernel = void (*)(const CUtensorMap, const CUtensorMap, int64_t, int, const int32_t *,
@@ -899,9 +799,7 @@ template <int FMT, bool FAST>
 ColKernel col_kernel_fmt(int layout) {
   return layout == FP8QGG_LAYOUT_SAME
              ? quant_colwise_jagged_kernel<FMT, FP8QGG_LAYOUT_SAME, FAST>
-         : layout == FP8QGG_LAYOUT_TRANSPOSED
-             ? quant_colwise_jagged_kernel<FMT, FP8QGG_LAYOUT_TRANSPOSED, FAST>
-             : quant_colwise_jagged_kernel<FMT, FP8QGG_LAYOUT_TRANSPOSED_PADDED, FAST>;
+             : quant_colwise_jagged_kernel<FMT, FP8QGG_LAYOUT_TRANSPOSED, FAST>;
 }
 
 // The fast kernels skip the clamp and the saturation count (see quant_pair_fast).
@@ -1029,13 +927,6 @@ int colwise_launch(const void *x, int64_t rows_total, int64_t cols, int64_t ld_x
       reinterpret_cast<uint32_t *>(base), reinterpret_cast<uint32_t *>(base + sl.arrive_off),
       reinterpret_cast<uint32_t *>(base + sl.amax_off), static_cast<int32_t>(sl.units_cap),
       current_unit_wait());
-  if (layout == FP8QGG_LAYOUT_TRANSPOSED_PADDED && rows_total > 0) {
-    const int64_t warps = int64_t(num_groups) * ((cols + 3) / 4);
-    const int pgrid = static_cast<int>(
-        std::max<int64_t>(1, std::min<int64_t>((warps + 7) / 8, int64_t(dev.sm_count) * 8)));
-    pad_transposed_kernel<<<pgrid, 256, 0, stream>>>(offsets, static_cast<int>(num_groups),
-                                                     rows_total, static_cast<int>(cols), q, ld_q);
-  }
   return cudaGetLastError() == cudaSuccess ? FP8QGG_OK : FP8QGG_ERR_CUDA;
 }
 
