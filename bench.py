@@ -580,6 +580,7 @@ def run_gpu(args, world, rank, local):
 # is absent until the current kernel has been captured on it.
 TRAFFIC = {
     "llama3_8b_up_proj": 269102336 + 422105344,     # grouped_gemm_2sm_kernel<0>
+    "deepseek_moe16b_bwd": 389194752 + 680884992,   # grouped_gemm_kernel<1, 0>, padded operands
 }
 
 
