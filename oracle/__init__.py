@@ -54,6 +54,18 @@ def lib():
         L.oracle_gemm_k_jagged_sample.restype = None
         L.oracle_gemm_k_jagged_sample.argtypes = [P, i64, P, i64, P, i64, P, i64, P, i32, i64,
                                                   ci, P, P, P, i64, P, P, P, P]
+        L.oracle_mx_quant_rowwise.restype = None
+        L.oracle_mx_quant_rowwise.argtypes = [P, i64, i64, i64, P, i64, P, i64]
+        L.oracle_mx_quant_colwise_padded.restype = None
+        L.oracle_mx_quant_colwise_padded.argtypes = [P, i64, i64, i64, P, i32, P, i64, P, i64,
+                                                     P, P, P]
+        L.oracle_mx_gemm_m_jagged_sample.restype = None
+        L.oracle_mx_gemm_m_jagged_sample.argtypes = [P, i64, P, i64, P, i64, i64, P, i64, i64,
+                                                     P, i32, i64, i64, P, P, i64, P, P, P, P]
+        L.oracle_mx_gemm_k_jagged_padded_sample.restype = None
+        L.oracle_mx_gemm_k_jagged_padded_sample.argtypes = [P, i64, P, i64, P, i64, P, i64, P,
+                                                            i32, i64, P, P, P, i64, P, P, P, P,
+                                                            P]
         _lib = L
     return _lib
 
@@ -193,4 +205,107 @@ def gemm_k_jagged_sample(qa_t, sa, qb_t, sb, offsets, m_total, grp, rows, cols,
     lib().oracle_gemm_k_jagged_sample(_p(qa_t), ld_a, _p(sa), n, _p(qb_t), ld_b, _p(sb), k,
                                       _p(off), e, m_total, fmt, _p(grp), _p(rows), _p(cols), ns,
                                       _p(c), _p(b), _p(start), _p(end))
+    return c, b
+
+
+# ---------------------------------------------------------------- MXFP8
+# The OCP MX v1.0 reading of MXFP8 (32-element blocks, E8M0 scale
+# 2^(floor(log2 amax) - 8), e4m3fn elements); see the MX section of
+# fp8_oracle.c.
+
+
+def padded_len(sizes) -> int:
+    """Tokens of the padded transposed layout: sum of round_up(size, 128)."""
+    return int(sum((int(s) + 127) // 128 * 128 for s in sizes))
+
+
+def mx_quant_rowwise(x_bits):
+    """MX quantisation along rows.  x_bits: uint16 [rows, cols], cols % 32 == 0.
+
+    Returns (codes uint8 [rows, cols], scales uint8 [rows, cols // 32])."""
+    x = _c(x_bits, np.uint16)
+    rows, cols = x.shape
+    assert cols % 32 == 0
+    q = np.zeros((rows, cols), np.uint8)
+    s = np.zeros((rows, cols // 32), np.uint8)
+    lib().oracle_mx_quant_rowwise(_p(x), rows, cols, cols, _p(q), cols, _p(s), cols // 32)
+    return q, s
+
+
+def mx_quant_colwise_padded(x_bits, offsets, ld_q: int = None, fill: int = 0,
+                            scale_fill: int = 0):
+    """MX quantisation along each group's tokens, transposed into the padded
+    layout.  x_bits: uint16 [rows_total, cols]; offsets: int32 group ends.
+
+    Returns (codes uint8 [cols, ld_q], scales uint8 [cols, ld_q // 32]);
+    entries past the last padded group keep ``fill`` / ``scale_fill``."""
+    x = _c(x_bits, np.uint16)
+    rows, cols = x.shape
+    off = _c(offsets, np.int32)
+    e = off.shape[0]
+    start, end = group_bounds(off, rows) if e else (np.zeros(0, np.int64),) * 2
+    need = padded_len(end - start)
+    ld = need if ld_q is None else ld_q
+    assert ld >= need and ld % 32 == 0
+    q = np.full((cols, ld), fill, np.uint8)
+    s = np.full((cols, ld // 32), scale_fill, np.uint8)
+    st = np.zeros(max(e, 1), np.int64)
+    en = np.zeros(max(e, 1), np.int64)
+    ps = np.zeros(max(e, 1), np.int64)
+    lib().oracle_mx_quant_colwise_padded(_p(x), rows, cols, cols, _p(off), e, _p(q), ld, _p(s),
+                                         ld // 32, _p(st), _p(en), _p(ps))
+    return q, s
+
+
+def mx_gemm_m_jagged_sample(qa, sa, qb, sb, offsets, rows, cols):
+    """Sampled fp64 reference of the MX token-jagged grouped GEMM.
+
+    qa: uint8 [m_total, k]; sa: uint8 [m_total, k // 32]; qb: uint8 [E, n, k];
+    sb: uint8 [E, n, k // 32].  Returns (c_ref, bound)."""
+    qa = _c(qa, np.uint8)
+    qb = _c(qb, np.uint8)
+    sa = _c(sa, np.uint8)
+    sb = _c(sb, np.uint8)
+    off = _c(offsets, np.int32)
+    m_total, k = qa.shape
+    e, n, k2 = qb.shape
+    assert k2 == k and sa.shape == (m_total, k // 32) and sb.shape == (e, n, k // 32)
+    rows = _c(rows, np.int64)
+    cols = _c(cols, np.int64)
+    ns = rows.shape[0]
+    c = np.zeros(ns, np.float64)
+    b = np.zeros(ns, np.float64)
+    start = np.zeros(max(e, 1), np.int64)
+    end = np.zeros(max(e, 1), np.int64)
+    lib().oracle_mx_gemm_m_jagged_sample(_p(qa), k, _p(sa), k // 32, _p(qb), k, n * k, _p(sb),
+                                         k // 32, n * (k // 32), _p(off), off.shape[0], m_total,
+                                         k, _p(rows), _p(cols), ns, _p(c), _p(b), _p(start),
+                                         _p(end))
+    return c, b
+
+
+def mx_gemm_k_jagged_padded_sample(qa_t, sa_t, qb_t, sb_t, offsets, m_total, grp, rows, cols):
+    """Sampled fp64 reference of the MX contraction-jagged grouped GEMM on
+    the padded transposed layout.  qa_t: uint8 [n, ld_a]; sa_t: uint8
+    [n, ld_a // 32]; qb_t / sb_t likewise for the second operand.
+    Returns (c_ref, bound) at (grp[i], rows[i], cols[i])."""
+    qa_t = _c(qa_t, np.uint8)
+    qb_t = _c(qb_t, np.uint8)
+    sa_t = _c(sa_t, np.uint8)
+    sb_t = _c(sb_t, np.uint8)
+    off = _c(offsets, np.int32)
+    e = off.shape[0]
+    grp = _c(grp, np.int64)
+    rows = _c(rows, np.int64)
+    cols = _c(cols, np.int64)
+    ns = rows.shape[0]
+    c = np.zeros(ns, np.float64)
+    b = np.zeros(ns, np.float64)
+    st = np.zeros(max(e, 1), np.int64)
+    en = np.zeros(max(e, 1), np.int64)
+    ps = np.zeros(max(e, 1), np.int64)
+    lib().oracle_mx_gemm_k_jagged_padded_sample(
+        _p(qa_t), qa_t.shape[1], _p(sa_t), sa_t.shape[1], _p(qb_t), qb_t.shape[1], _p(sb_t),
+        sb_t.shape[1], _p(off), e, m_total, _p(grp), _p(rows), _p(cols), ns, _p(c), _p(b),
+        _p(st), _p(en), _p(ps))
     return c, b

@@ -314,3 +314,199 @@ void oracle_fp8_encode_array(const float *y, int64_t n, uint8_t *q, int fmt)
 {
     for (int64_t i = 0; i < n; ++i) q[i] = oracle_fp8_encode(y[i], fmt);
 }
+
+/* ------------------------------------------------------------------------
+ * MXFP8: microscaled FP8 ("AMD Primus adds FP8/MXFP8 kernels ...", section
+ * "What Primus adds for MoE training on MI355X": MXFP8 grouped GEMM and
+ * quantisation kernels; "AMD Boosts PyTorch FP8 Training on Instinct GPUs",
+ * last paragraph; "FP8 su GPU AMD ...", section "Cosa significa per chi
+ * gestisce cluster locali": MXFP8 as the next, finer-grained format).
+ * The pages name the format and do not define it; the reading taken is the
+ * OCP Microscaling Formats (MX) v1.0 definition of MXFP8 with e4m3 elements:
+ *  - a block is 32 consecutive elements along the contraction axis;
+ *  - its shared scale is X = 2^E, E = floor(log2(amax)) - 8 (8 = the
+ *    exponent of e4m3fn's largest normal binade), stored as the E8M0 byte
+ *    E + 127, E clamped to [-127, 127];
+ *  - element code = encode(x / X): the quotient is clamped to +-448 and
+ *    rounded to nearest even (the e4m3fn encoder above);
+ *  - value = decode(code) * X.
+ * Readings for the cases the definition leaves open (same as the per-row
+ * path where they overlap): amax skips NaN; an all-zero (or all-NaN) block
+ * takes E = -127; an infinite amax takes E = 127.
+ * ------------------------------------------------------------------------ */
+
+/* E of a block from its absmax (an exact fp32 value). */
+static int mx_exponent(float amax)
+{
+    if (!(amax > 0.0f)) return -127;
+    if (isinf(amax)) return 127;
+    int ex;
+    (void)frexp((double)amax, &ex); /* amax = f * 2^ex, f in [0.5, 1): floor(log2) = ex - 1 */
+    int e = ex - 1 - 8;
+    if (e < -127) e = -127;
+    if (e > 127) e = 127;
+    return e;
+}
+
+/* Code of one element of a block with exponent e: x / 2^e is exact in
+ * double; as an fp32 value it is exact too wherever it can reach a nonzero
+ * code (a bf16 value times a power of two keeps its 8 significant bits, and
+ * magnitudes from 2^-10 up lie in fp32's normal range). */
+static uint8_t mx_encode_one(float x, int e)
+{
+    double y = ldexp((double)x, -e);
+    if (y > 448.0) y = 448.0;
+    if (y < -448.0) y = -448.0;
+    return oracle_fp8_encode((float)y, ORC_FMT_E4M3FN);
+}
+
+/* Scale byte of the block x[0], x[stride], ... (n <= 32 elements; the
+ * missing ones of a partial block count as zeros). */
+static uint8_t mx_block_scale(const uint16_t *x, int64_t stride, int64_t n, int *e_out)
+{
+    float amax = 0.0f;
+    for (int64_t i = 0; i < n; ++i) {
+        float v = fabsf(bf16_to_f32(x[i * stride]));
+        if (v > amax) amax = v;
+    }
+    int e = mx_exponent(amax);
+    *e_out = e;
+    return (uint8_t)(e + 127);
+}
+
+/* MX quantisation along rows: blocks of 32 consecutive columns.
+ * x: bf16 bits [rows, ld_x], cols a multiple of 32; q: codes [rows, ld_q];
+ * sc: E8M0 bytes [rows, ld_s], sc[r, b] for columns [32b, 32b + 32). */
+void oracle_mx_quant_rowwise(const uint16_t *x, int64_t rows, int64_t cols, int64_t ld_x,
+                             uint8_t *q, int64_t ld_q, uint8_t *sc, int64_t ld_s)
+{
+    for (int64_t r = 0; r < rows; ++r) {
+        for (int64_t b = 0; b < cols / 32; ++b) {
+            const uint16_t *xb = x + r * ld_x + 32 * b;
+            int e;
+            sc[r * ld_s + b] = mx_block_scale(xb, 1, 32, &e);
+            for (int64_t i = 0; i < 32; ++i)
+                q[r * ld_q + 32 * b + i] = mx_encode_one(bf16_to_f32(xb[i]), e);
+        }
+    }
+}
+
+/* Padded start of each group: P_0 = 0, P_e = sum_{j<e} round_up(size_j, 128). */
+static void padded_starts(const int64_t *start, const int64_t *end, int32_t num_groups,
+                          int64_t *pstart)
+{
+    int64_t p = 0;
+    for (int32_t e = 0; e < num_groups; ++e) {
+        pstart[e] = p;
+        p += (end[e] - start[e] + 127) / 128 * 128;
+    }
+}
+
+/* MX quantisation along the tokens of each expert group, written transposed
+ * in the padded layout: column c, token t of group e (t < size_e) goes to
+ * q[c, P_e + t]; the tokens [size_e, round_up(size_e, 128)) hold zero codes.
+ * Blocks are 32 consecutive tokens from the group's start; a group's last
+ * block may be partial (its missing tokens are the zero padding).  Scales:
+ * sc[c, P_e / 32 + b] for the group's blocks b < round_up(size_e, 128) / 32
+ * (padding-only blocks: amax 0, E = -127).  Tokens past the last group are
+ * not written.  start/end/pstart: caller scratch of num_groups. */
+void oracle_mx_quant_colwise_padded(const uint16_t *x, int64_t rows_total, int64_t cols,
+                                    int64_t ld_x, const int32_t *offsets, int32_t num_groups,
+                                    uint8_t *q, int64_t ld_q, uint8_t *sc, int64_t ld_s,
+                                    int64_t *start, int64_t *end, int64_t *pstart)
+{
+    oracle_group_bounds(offsets, num_groups, rows_total, start, end);
+    padded_starts(start, end, num_groups, pstart);
+    for (int32_t g = 0; g < num_groups; ++g) {
+        int64_t size = end[g] - start[g];
+        int64_t padded = (size + 127) / 128 * 128;
+        for (int64_t c = 0; c < cols; ++c) {
+            for (int64_t b = 0; b < padded / 32; ++b) {
+                int64_t t0 = 32 * b;
+                int64_t n = size - t0;
+                if (n > 32) n = 32;
+                if (n < 0) n = 0;
+                int e;
+                sc[c * ld_s + pstart[g] / 32 + b] =
+                    mx_block_scale(x + (start[g] + t0) * ld_x + c, ld_x, n, &e);
+                for (int64_t i = 0; i < 32; ++i) {
+                    int64_t t = t0 + i;
+                    q[c * ld_q + pstart[g] + t] =
+                        t < size ? mx_encode_one(bf16_to_f32(x[(start[g] + t) * ld_x + c]), e)
+                                 : (uint8_t)0;
+                }
+            }
+        }
+    }
+}
+
+/* Value of an MX element: decode(code) * 2^(scale byte - 127). */
+static double mx_value(uint8_t code, uint8_t scale)
+{
+    return ldexp(oracle_fp8_decode(code, ORC_FMT_E4M3FN), (int)scale - 127);
+}
+
+/* MX grouped GEMM, token-jagged form:
+ *   C[m, n] = sum_k value(qa[m,k], sa[m, k/32]) * value(qb_e[n,k], sb_e[n, k/32])
+ * with e the group of row m; fp64 at the sample points; rows outside every
+ * group give NaN.  bound[i] = 1e-3 * sum |a||b|. */
+void oracle_mx_gemm_m_jagged_sample(const uint8_t *qa, int64_t ld_a, const uint8_t *sa,
+                                    int64_t ld_sa, const uint8_t *qb, int64_t ld_b,
+                                    int64_t b_group_stride, const uint8_t *sb, int64_t ld_sb,
+                                    int64_t sb_group_stride, const int32_t *offsets,
+                                    int32_t num_groups, int64_t m_total, int64_t k,
+                                    const int64_t *rows, const int64_t *cols, int64_t n_samples,
+                                    double *c_ref, double *bound, int64_t *start, int64_t *end)
+{
+    oracle_group_bounds(offsets, num_groups, m_total, start, end);
+    for (int64_t i = 0; i < n_samples; ++i) {
+        int64_t m = rows[i], n = cols[i];
+        int32_t g = -1;
+        for (int32_t e = 0; e < num_groups; ++e)
+            if (m >= start[e] && m < end[e]) { g = e; break; }
+        if (g < 0) { c_ref[i] = NAN; bound[i] = 0.0; continue; }
+        const uint8_t *arow = qa + m * ld_a;
+        const uint8_t *asc = sa + m * ld_sa;
+        const uint8_t *brow = qb + (int64_t)g * b_group_stride + n * ld_b;
+        const uint8_t *bsc = sb + (int64_t)g * sb_group_stride + n * ld_sb;
+        double acc = 0.0, mag = 0.0;
+        for (int64_t kk = 0; kk < k; ++kk) {
+            double a = mx_value(arow[kk], asc[kk / 32]);
+            double b = mx_value(brow[kk], bsc[kk / 32]);
+            acc += a * b;
+            mag += fabs(a * b);
+        }
+        c_ref[i] = acc;
+        bound[i] = 1e-3 * mag;
+    }
+}
+
+/* MX grouped GEMM, contraction-jagged form on the padded transposed layout
+ * (weight gradient):
+ *   C[e, i, j] = sum_{t < size_e} value(qa[i, P_e + t], sa[i, (P_e + t)/32])
+ *                                 * value(qb[j, P_e + t], sb[j, (P_e + t)/32])
+ * Sample points (grp[s], rows[s], cols[s]); an empty group gives 0. */
+void oracle_mx_gemm_k_jagged_padded_sample(const uint8_t *qa, int64_t ld_a, const uint8_t *sa,
+                                           int64_t ld_sa, const uint8_t *qb, int64_t ld_b,
+                                           const uint8_t *sb, int64_t ld_sb,
+                                           const int32_t *offsets, int32_t num_groups,
+                                           int64_t m_total, const int64_t *grp,
+                                           const int64_t *rows, const int64_t *cols,
+                                           int64_t n_samples, double *c_ref, double *bound,
+                                           int64_t *start, int64_t *end, int64_t *pstart)
+{
+    oracle_group_bounds(offsets, num_groups, m_total, start, end);
+    padded_starts(start, end, num_groups, pstart);
+    for (int64_t s = 0; s < n_samples; ++s) {
+        int64_t e = grp[s], i = rows[s], j = cols[s];
+        double acc = 0.0, mag = 0.0;
+        for (int64_t t = pstart[e]; t < pstart[e] + (end[e] - start[e]); ++t) {
+            double a = mx_value(qa[i * ld_a + t], sa[i * ld_sa + t / 32]);
+            double b = mx_value(qb[j * ld_b + t], sb[j * ld_sb + t / 32]);
+            acc += a * b;
+            mag += fabs(a * b);
+        }
+        c_ref[s] = acc;
+        bound[s] = 1e-3 * mag;
+    }
+}
