@@ -55,6 +55,11 @@ _SIGNATURES = {
     "fp8_quant_dual_jagged_workspace_size": (_SZ, [_I64, _I64, _I32]),
     "fp8_quant_dual_jagged": (_INT, [_P, _I64, _I64, _I64, _P, _I32, _P, _I64, _P, _P, _I64, _P,
                                      _INT, _F32, _P, _P, _P, _SZ, _P]),
+    "fp8_mx_quant_rowwise": (_INT, [_P, _I64, _I64, _I64, _P, _I64, _P, _I64, _P]),
+    "fp8_mx_quant_colwise_padded": (_INT, [_P, _I64, _I64, _I64, _P, _I32, _P, _I64, _P, _I64,
+                                           _P, _P]),
+    "fp8_mx_grouped_gemm": (_INT, [_INT, _P, _I64, _P, _I64, _P, _I64, _I64, _P, _I64, _I64, _P,
+                                   _I32, _I64, _I64, _I64, _P, _I64, _I64, _INT, _P, _P]),
 }
 
 
@@ -281,6 +286,102 @@ def fp8_cast_f32(y, fmt=E4M3FN, q=None, sat_count=None, stream=None):
     rc = lib().fp8_cast_f32(_ptr(y), y.numel(), _ptr(q), fmt, _stream(stream))
     _check(rc, "fp8_cast_f32")
     return q
+
+
+# ------------------------------------------------------------------ MXFP8
+def mx_scale_ld(cols: int) -> int:
+    """Scale bytes per row the MX grouped GEMM reads: 4 per 128 columns."""
+    return 4 * ((cols + 127) // 128)
+
+
+def fp8_mx_quant_rowwise(x, q=None, scales=None, stream=None):
+    """MXFP8 quantisation along the rows of a bf16 [rows, cols] CUDA tensor
+    (cols % 32 == 0): one E8M0 scale byte per 32 consecutive columns.
+
+    Returns (q uint8 [rows, cols], scales uint8 [rows, mx_scale_ld(cols)]);
+    scale columns [0, cols // 32) are written."""
+    _need_cuda(x)
+    assert x.dtype == torch.bfloat16 and x.dim() == 2
+    rows, cols = x.shape
+    if q is None:
+        q = torch.empty((rows, cols), dtype=torch.uint8, device=x.device)
+    if scales is None:
+        scales = torch.empty((rows, mx_scale_ld(cols)), dtype=torch.uint8, device=x.device)
+    _need_cuda(q, scales)
+    rc = lib().fp8_mx_quant_rowwise(_ptr(x), rows, cols, _ld(x), _ptr(q), _ld(q), _ptr(scales),
+                                    _ld(scales), _stream(stream))
+    _check(rc, "fp8_mx_quant_rowwise")
+    return q, scales
+
+
+def fp8_mx_quant_colwise_padded(x, offsets, q=None, ld_q=None, scales=None, status=None,
+                                stream=None):
+    """MXFP8 quantisation along each expert group's tokens of a bf16
+    [rows_total, cols] CUDA tensor, written transposed in the padded layout
+    (group e from token P_e, zero codes up to a 128-token boundary).
+
+    Returns (q uint8 [cols, ld_q], scales uint8 [cols, ld_q // 32])."""
+    _need_cuda(x, offsets)
+    assert x.dtype == torch.bfloat16 and x.dim() == 2 and offsets.dtype == torch.int32
+    rows, cols = x.shape
+    e = offsets.numel()
+    if q is None:
+        ld = ld_q if ld_q is not None else (rows + 128 * e + 127) // 128 * 128
+        q = torch.empty((cols, ld), dtype=torch.uint8, device=x.device)
+    if scales is None:
+        scales = torch.empty((cols, (q.shape[1] + 127) // 128 * 4), dtype=torch.uint8,
+                             device=x.device)
+    _need_cuda(q, scales, status)
+    rc = lib().fp8_mx_quant_colwise_padded(_ptr(x), rows, cols, _ld(x), _ptr(offsets), e,
+                                           _ptr(q), _ld(q), _ptr(scales), _ld(scales),
+                                           _ptr(status), _stream(stream))
+    _check(rc, "fp8_mx_quant_colwise_padded")
+    return q, scales
+
+
+def fp8_mx_grouped_gemm(mode, a, scale_a, b, scale_b, offsets, m_total=None, n=None, k=None,
+                        out=None, out_dtype=torch.float32, status=None, stream=None):
+    """MXFP8 grouped GEMM (see the C header).
+
+    M_JAGGED: a uint8 [m_total, K], scale_a uint8 [m_total, ld_sa],
+    b uint8 [E, N, K], scale_b uint8 [E, N, ld_sb] -> out [m_total, N].
+    K_JAGGED_PADDED: a uint8 [N, ld_a], scale_a uint8 [N, ld_sa], b uint8
+    [K, ld_b], scale_b uint8 [K, ld_sb] (outputs of fp8_mx_quant_colwise_padded),
+    m_total unpadded tokens -> out [E, N, K]."""
+    _need_cuda(a, scale_a, b, scale_b, offsets)
+    assert a.dtype == torch.uint8 and b.dtype == torch.uint8 and offsets.dtype == torch.int32
+    assert scale_a.dtype == torch.uint8 and scale_b.dtype == torch.uint8
+    e = offsets.numel()
+    if out is not None:
+        out_dtype = out.dtype
+    assert out_dtype in (torch.float32, torch.bfloat16)
+    odt = OUT_F32 if out_dtype == torch.float32 else OUT_BF16
+    if mode == M_JAGGED:
+        m_total = a.shape[0] if m_total is None else m_total
+        k = a.shape[1] if k is None else k
+        assert b.dim() == 3 and scale_b.dim() == 3
+        n = b.shape[1] if n is None else n
+        ld_b, bgs = b.stride(1), b.stride(0)
+        ld_sb, sbgs = scale_b.stride(1), scale_b.stride(0)
+        if out is None:
+            out = torch.empty((m_total, n), dtype=out_dtype, device=a.device)
+        ld_out, ogs = _ld(out), 0
+    else:
+        n = a.shape[0] if n is None else n
+        k = b.shape[0] if k is None else k
+        assert m_total is not None
+        ld_b, bgs = _ld(b), 0
+        ld_sb, sbgs = _ld(scale_b), 0
+        if out is None:
+            out = torch.empty((e, n, k), dtype=out_dtype, device=a.device)
+        ld_out, ogs = out.stride(-2), out.stride(0)
+    _need_cuda(out, status)
+    rc = lib().fp8_mx_grouped_gemm(
+        mode, _ptr(a), _ld(a), _ptr(scale_a), _ld(scale_a), _ptr(b), ld_b, bgs, _ptr(scale_b),
+        ld_sb, sbgs, _ptr(offsets), e, m_total, n, k, _ptr(out), ld_out, ogs, odt, _ptr(status),
+        _stream(stream))
+    _check(rc, "fp8_mx_grouped_gemm")
+    return out
 
 
 class Fp8WeightCache:
