@@ -217,7 +217,11 @@ def config_dict(w, Step=None):
     src = w.x if w.x is not None else w.grad_out
     m, k = src.shape
     d = dict(workload=w.name, M=m, K=k, E=w.num_groups, fmt="e4m3fn", gemm_out="fp32")
-    if Step is not None and Step.__name__ == "DualCompareStep":
+    if Step is not None and getattr(Step, "STEP", None):
+        d.update(N=(w.grad_out if w.grad_out is not None and Step.BACKWARD else w.w).shape[1],
+                 step=Step.STEP, fmt=Step.FMT)
+        d.update(workload=w.name + "_mxfp8")
+    elif Step is not None and Step.__name__ == "DualCompareStep":
         d.update(K=None, N=w.grad_out.shape[1], gemm_out=None,
                  step=("grad_out quantised for both backward GEMMs: rowwise + padded transposed "
                        "jagged column-wise as two calls, then as one dual-output call"))
@@ -304,7 +308,7 @@ class BackwardDwStep:
         self.out = torch.empty((e, n, k), dtype=torch.float32, device="cuda")
         self.flops = 2.0 * m * n * k
         self.names = ["quant_colwise_t_grad_out", "quant_colwise_t_x", "grouped_gemm"]
-        self.launches = 5  # each colwise call: the quantisation and the gap fill
+        self.launches = 3
         self.bytes = [m * n * 3 + e * n * 4 + e * 4, m * k * 3 + e * k * 4 + e * 4, None]
         self.host_inputs = [(self.g, w.grad_out), (self.x, w.x)]
         self.input_bytes = 2 * (m * n + m * k)
@@ -376,6 +380,97 @@ class DualCompareStep:
         ]
 
 
+class MxForwardStep:
+    """MXFP8 token-jagged forward: MX rowwise quantisation of X and of W viewed
+    [E*N, K] (one E8M0 scale per 32 elements along K), block-scaled grouped
+    GEMM (fp32 out)."""
+    STEP = ("MX rowwise quant X + MX rowwise quant W (32-element blocks along K) + "
+            "block-scaled token-jagged MXFP8 grouped GEMM")
+    FMT = "mxfp8 (e4m3fn elements, E8M0 scales per 32 elements)"
+    BACKWARD = False
+
+    def __init__(self, w):
+        import quantization_grouped_gemm_b200 as qgg
+        self.qgg = qgg
+        self.w = w
+        m, k = w.x.shape
+        e, n = w.w.shape[0], w.w.shape[1]
+        self.m, self.n, self.k, self.e = m, n, k, e
+        self.x = w.x.cuda()
+        self.wt = w.w.reshape(e * n, k).cuda()
+        self.off = torch.from_numpy(w.offsets).cuda()
+        gk = qgg.mx_scale_groups(k)
+        self.qa = torch.empty((m, k), dtype=torch.uint8, device="cuda")
+        self.sa = torch.empty((gk, m), dtype=torch.int32, device="cuda")
+        self.qb = torch.empty((e * n, k), dtype=torch.uint8, device="cuda")
+        self.sb = torch.empty((gk, e * n), dtype=torch.int32, device="cuda")
+        self.out = torch.empty((m, n), dtype=torch.float32, device="cuda")
+        rows = int(np.asarray(w.offsets)[-1]) if len(w.offsets) else 0
+        self.flops = 2.0 * rows * n * k
+        self.names = ["mx_quant_rowwise_x", "mx_quant_rowwise_w", "mx_grouped_gemm"]
+        self.launches = 3
+        self.bytes = [m * k * 3 + m * k // 32, e * n * k * 3 + e * n * k // 32, None]
+        self.host_inputs = [(self.x, w.x), (self.wt, w.w.reshape(e * n, k))]
+        self.input_bytes = 2 * (m * k + e * n * k)
+        self.result = self.out
+
+    def kernels(self):
+        q = self.qgg
+        e, n = self.e, self.n
+        return [
+            lambda: q.fp8_mx_quant_rowwise(self.x, q=self.qa, scales=self.sa),
+            lambda: q.fp8_mx_quant_rowwise(self.wt, q=self.qb, scales=self.sb),
+            lambda: q.fp8_mx_grouped_gemm(q.M_JAGGED, self.qa, self.sa, self.qb.view(e, n, -1),
+                                          self.sb, self.off, out=self.out),
+        ]
+
+
+class MxBackwardDwStep:
+    """MXFP8 contraction-jagged weight gradient: MX quantisation of grad_out
+    [M, N] and of X [M, K] along each group's tokens (32-token blocks),
+    transposed into the padded layout, then the block-scaled
+    dW_e = dH_e^T X_e."""
+    STEP = ("MX quant + transpose of grad_out and of X along each group's tokens "
+            "(32-token blocks, groups at 128-token boundaries) + block-scaled "
+            "contraction-jagged MXFP8 grouped GEMM (dW)")
+    FMT = "mxfp8 (e4m3fn elements, E8M0 scales per 32 tokens)"
+    BACKWARD = True
+
+    def __init__(self, w):
+        import quantization_grouped_gemm_b200 as qgg
+        self.qgg = qgg
+        self.w = w
+        m, k = w.x.shape
+        n = w.grad_out.shape[1]
+        e = w.num_groups
+        self.m, self.n, self.k, self.e = m, n, k, e
+        self.g = w.grad_out.cuda()
+        self.x = w.x.cuda()
+        self.off = torch.from_numpy(w.offsets).cuda()
+        ld = (m + 128 * e + 127) // 128 * 128
+        self.qg = torch.empty((n, ld), dtype=torch.uint8, device="cuda")
+        self.qx = torch.empty((k, ld), dtype=torch.uint8, device="cuda")
+        self.sg = torch.empty((ld // 128, n), dtype=torch.int32, device="cuda")
+        self.sx = torch.empty((ld // 128, k), dtype=torch.int32, device="cuda")
+        self.out = torch.empty((e, n, k), dtype=torch.float32, device="cuda")
+        self.flops = 2.0 * m * n * k
+        self.names = ["mx_quant_colwise_t_grad_out", "mx_quant_colwise_t_x", "mx_grouped_gemm"]
+        self.launches = 3
+        self.bytes = [m * n * 3 + m * n // 32, m * k * 3 + m * k // 32, None]
+        self.host_inputs = [(self.g, w.grad_out), (self.x, w.x)]
+        self.input_bytes = 2 * (m * n + m * k)
+        self.result = self.out
+
+    def kernels(self):
+        q = self.qgg
+        return [
+            lambda: q.fp8_mx_quant_colwise_padded(self.g, self.off, q=self.qg, scales=self.sg),
+            lambda: q.fp8_mx_quant_colwise_padded(self.x, self.off, q=self.qx, scales=self.sx),
+            lambda: q.fp8_mx_grouped_gemm(q.K_JAGGED_PADDED, self.qg, self.sg, self.qx, self.sx,
+                                          self.off, m_total=self.m, out=self.out),
+        ]
+
+
 WORKLOADS = {
     "llama3_8b_up_proj": (lambda: wl.llama3_8b_up_proj(), ForwardStep),
     "tiny_moe": (lambda: wl.tiny_moe(), ForwardStep),
@@ -385,6 +480,8 @@ WORKLOADS = {
     "deepseek_v3_fwd": (lambda: wl.deepseek_v3_local_experts(), ForwardStep),
     "llama4_m8192_zipf": (lambda: wl.llama4_sweep(8192, "zipf"), ForwardStep),
     "llama4_m131072_uniform": (lambda: wl.llama4_sweep(131072, "uniform"), ForwardStep),
+    "llama3_8b_up_proj_mxfp8": (lambda: wl.llama3_8b_up_proj(), MxForwardStep),
+    "deepseek_moe16b_bwd_mxfp8": (lambda: wl.deepseek_moe_16b_backward(), MxBackwardDwStep),
 }
 
 
@@ -473,8 +570,10 @@ def extra_workload(name, steps, warmup, pk):
 
 
 # Workloads timed in the default run beside the headline one: the tiny MoE
-# layer (launch-bound) and the DeepSeek-MoE-16B backward weight-gradient step.
-EXTRA_WORKLOADS = ("tiny_moe", "deepseek_moe16b_bwd", "deepseek_moe16b_bwd_dual")
+# layer (launch-bound), the DeepSeek-MoE-16B backward weight-gradient step,
+# the dual-output comparison, and the MXFP8 forward and weight-gradient steps.
+EXTRA_WORKLOADS = ("tiny_moe", "deepseek_moe16b_bwd", "deepseek_moe16b_bwd_dual",
+                   "llama3_8b_up_proj_mxfp8", "deepseek_moe16b_bwd_mxfp8")
 
 
 def run_gpu(args, world, rank, local):

@@ -344,8 +344,12 @@ int fp8_scaled_grouped_gemm(int mode,
  *        scale byte (E8M0) = E + 127
  *        q    = e4m3fn(x / 2^E)  round to nearest even, saturating at 448
  *        value = decode(q) * 2^E
- * Scales are bytes, row-major: the scale of block b of row r is
- * scales[r * ld_s + b].  Only e4m3fn exists in this format.
+ * Scale layout (packed for the grouped GEMM): the contraction axis is cut
+ * into groups of 128 elements (four blocks); one uint32 word per (group g,
+ * row r) holds the four scale bytes, byte j = block 4g + j (bytes of blocks
+ * past the end of the axis are 0), and the words of one group are
+ * contiguous over the rows: scales[g * ld_sw + r].  Only e4m3fn exists in
+ * this format.
  */
 
 /*
@@ -353,13 +357,11 @@ int fp8_scaled_grouped_gemm(int mode,
  * [E*N, K]): blocks of 32 consecutive columns.
  *   x       bf16 [rows, ld_x], 16-byte aligned, ld_x % 8 == 0.
  *   q       uint8 [rows, ld_q], 8-byte aligned, ld_q % 8 == 0.
- *   scales  uint8 [rows, ld_s], ld_s >= cols / 32.
+ *   scales  uint32 [ceil(cols / 128), ld_sw], ld_sw >= rows, 4-byte aligned.
  * Requirements: cols >= 1, cols % 32 == 0 (FP8QGG_ERR_SHAPE otherwise).
- * For the MX grouped GEMM, ld_s must be a multiple of 4 covering
- * 4 * ceil(cols / 128) bytes (the GEMM reads the scales 4 blocks at a time).
  */
 int fp8_mx_quant_rowwise(const void *x, int64_t rows, int64_t cols, int64_t ld_x,
-                         uint8_t *q, int64_t ld_q, uint8_t *scales, int64_t ld_s,
+                         uint8_t *q, int64_t ld_q, uint32_t *scales, int64_t ld_sw,
                          void *stream);
 
 /*
@@ -369,42 +371,45 @@ int fp8_mx_quant_rowwise(const void *x, int64_t rows, int64_t cols, int64_t ld_x
  * to q[c * ld_q + P_e + t], P_e = sum_{j<e} round_up(size_j, 128); the tokens
  * [size_e, round_up(size_e, 128)) of the group hold zero codes.  Blocks are
  * 32 consecutive tokens from the group's start (a group's last block may be
- * partial; its padding counts as zeros), so no block holds two groups; the
- * scale of block b of group e, column c is scales[c * ld_s + P_e / 32 + b]
- * for b < round_up(size_e, 128) / 32 (padding-only blocks: amax 0, byte 0).
- * Tokens past the last padded group are not written.
+ * partial; its padding counts as zeros), so no block holds two groups.  The
+ * scales follow the packed layout with the columns as rows and the padded
+ * token axis as contraction axis: word (P_e / 128 + b, c) for the group's
+ * 128-token groups b < round_up(size_e, 128) / 128 (padding-only blocks:
+ * amax 0, byte 0).  Tokens past the last padded group are not written.
  *   x        bf16 [rows_total, ld_x], read once.
  *   offsets  int32 [num_groups] cumulative group ends (device).
  *   q        uint8 [cols, ld_q], ld_q >= rows_total + 128 * num_groups,
  *            ld_q % 16 == 0, 16-byte aligned.
- *   scales   uint8 [cols, ld_s], ld_s >= ceil((rows_total + 128 * num_groups) / 32),
- *            ld_s % 4 == 0, 4-byte aligned.
+ *   scales   uint32 [ld_q / 128, ld_sw], ld_sw >= cols, 4-byte aligned.
  * Requirements: cols % 8 == 0, ld_x % 8 == 0, x 16-byte aligned,
  * num_groups in [1, 1024].
  */
 int fp8_mx_quant_colwise_padded(const void *x, int64_t rows_total, int64_t cols, int64_t ld_x,
                                 const int32_t *offsets, int32_t num_groups,
-                                uint8_t *q, int64_t ld_q, uint8_t *scales, int64_t ld_s,
+                                uint8_t *q, int64_t ld_q, uint32_t *scales, int64_t ld_sw,
                                 int32_t *dev_status, void *stream);
 
 /*
  * MXFP8 grouped GEMM: block-scaled tensor-core products (each 32-element
- * block's partial sum times 2^(Ea + Eb)), fp32 accumulation.
+ * block's partial sum times 2^(Ea + Eb)), fp32 accumulation.  Scales in the
+ * packed layout above (ld_sa, ld_sb: words per 128-element group).
  * mode FP8QGG_M_JAGGED (forward, input gradient):
  *   out[m, n] = sum_k value_a[m, k] * value_b_e[n, k], e the group of row m
- *   a        e4m3 [m_total, ld_a];  scale_a uint8 [m_total, ld_sa]
- *   b        B_e[n, k] at b[e*b_group_stride + n*ld_b + k];
- *            scale_b at scale_b[e*scale_b_group_stride + n*ld_sb + k/32]
+ *   a        e4m3 [m_total, ld_a]; scale_a word (g, m) at scale_a[g * ld_sa + m],
+ *            ld_sa >= m_total
+ *   b        B_e[n, k] at b[e*b_group_stride + n*ld_b + k]; scale_b word
+ *            (g, e, n) at scale_b[g * ld_sb + e * scale_b_group_stride + n]
+ *            (B quantised as one [E*N, K] matrix: scale_b_group_stride = n).
  *   out      [m_total, ld_out]; rows outside every group are not written.
- *   Requirements: k % 32 == 0; ld_sa, ld_sb >= 4 * ceil(k / 128) and
- *   multiples of 4; scale_b_group_stride >= n * ld_sb and a multiple of 4.
+ *   Requirements: k % 32 == 0; scale_b_group_stride >= n;
+ *   ld_sb >= (num_groups - 1) * scale_b_group_stride + n.
  * mode FP8QGG_K_JAGGED_PADDED (weight gradient, outputs of
  * fp8_mx_quant_colwise_padded):
  *   out[e, i, j] = sum_{t < size_e} value_a[i, P_e + t] * value_b[j, P_e + t]
- *   a        e4m3 [n, ld_a], scale_a uint8 [n, ld_sa];
- *   b        e4m3 [k, ld_b], scale_b uint8 [k, ld_sb];
+ *   a        e4m3 [n, ld_a], scale_a words [.., ld_sa >= n];
+ *   b        e4m3 [k, ld_b], scale_b words [.., ld_sb >= k];
  *            ld_a, ld_b >= m_total + 128 * num_groups (m_total: unpadded
- *            tokens); ld_sa, ld_sb >= (m_total + 128 * num_groups) / 32.
+ *            tokens).
  *   out      [num_groups, n, ld_out], group stride out_group_stride; an empty
  *            group's matrix is written as zeros.
  * (The plain K_JAGGED mode does not exist here: a 32-token block may not
@@ -414,9 +419,9 @@ int fp8_mx_quant_colwise_padded(const void *x, int64_t rows_total, int64_t cols,
  * aligned.  Returns FP8QGG_ERR_UNSUPPORTED for another mode or out_dtype.
  */
 int fp8_mx_grouped_gemm(int mode,
-                        const uint8_t *a, int64_t ld_a, const uint8_t *scale_a, int64_t ld_sa,
+                        const uint8_t *a, int64_t ld_a, const uint32_t *scale_a, int64_t ld_sa,
                         const uint8_t *b, int64_t ld_b, int64_t b_group_stride,
-                        const uint8_t *scale_b, int64_t ld_sb, int64_t scale_b_group_stride,
+                        const uint32_t *scale_b, int64_t ld_sb, int64_t scale_b_group_stride,
                         const int32_t *offsets, int32_t num_groups,
                         int64_t m_total, int64_t n, int64_t k,
                         void *out, int64_t ld_out, int64_t out_group_stride, int out_dtype,

@@ -289,25 +289,35 @@ def fp8_cast_f32(y, fmt=E4M3FN, q=None, sat_count=None, stream=None):
 
 
 # ------------------------------------------------------------------ MXFP8
-def mx_scale_ld(cols: int) -> int:
-    """Scale bytes per row the MX grouped GEMM reads: 4 per 128 columns."""
-    return 4 * ((cols + 127) // 128)
+def mx_scale_groups(length: int) -> int:
+    """Scale words per row: one per 128 elements of the contraction axis."""
+    return (length + 127) // 128
+
+
+def mx_scales_to_blocks(words, nblocks: int):
+    """The packed scale words [groups, ld_sw] (torch int32 / uint32 storage)
+    as plain E8M0 bytes [rows, nblocks] for the first ld_sw rows: byte j of
+    word (g, r) is the scale of block 4g + j of row r.  (A view change and a
+    transpose, for reading results; the kernels never need it.)"""
+    w = words.contiguous().view(torch.uint8).view(words.shape[0], words.shape[1], 4)
+    return w.permute(1, 0, 2).reshape(words.shape[1], -1)[:, :nblocks]
 
 
 def fp8_mx_quant_rowwise(x, q=None, scales=None, stream=None):
     """MXFP8 quantisation along the rows of a bf16 [rows, cols] CUDA tensor
-    (cols % 32 == 0): one E8M0 scale byte per 32 consecutive columns.
+    (cols % 32 == 0): one E8M0 scale byte per 32 consecutive columns, packed
+    four to a word per 128 columns.
 
-    Returns (q uint8 [rows, cols], scales uint8 [rows, mx_scale_ld(cols)]);
-    scale columns [0, cols // 32) are written."""
+    Returns (q uint8 [rows, cols], scales int32 [ceil(cols / 128), rows])."""
     _need_cuda(x)
     assert x.dtype == torch.bfloat16 and x.dim() == 2
     rows, cols = x.shape
     if q is None:
         q = torch.empty((rows, cols), dtype=torch.uint8, device=x.device)
     if scales is None:
-        scales = torch.empty((rows, mx_scale_ld(cols)), dtype=torch.uint8, device=x.device)
+        scales = torch.empty((mx_scale_groups(cols), rows), dtype=torch.int32, device=x.device)
     _need_cuda(q, scales)
+    assert scales.dtype == torch.int32
     rc = lib().fp8_mx_quant_rowwise(_ptr(x), rows, cols, _ld(x), _ptr(q), _ld(q), _ptr(scales),
                                     _ld(scales), _stream(stream))
     _check(rc, "fp8_mx_quant_rowwise")
@@ -320,7 +330,7 @@ def fp8_mx_quant_colwise_padded(x, offsets, q=None, ld_q=None, scales=None, stat
     [rows_total, cols] CUDA tensor, written transposed in the padded layout
     (group e from token P_e, zero codes up to a 128-token boundary).
 
-    Returns (q uint8 [cols, ld_q], scales uint8 [cols, ld_q // 32])."""
+    Returns (q uint8 [cols, ld_q], scales int32 [ld_q // 128, cols])."""
     _need_cuda(x, offsets)
     assert x.dtype == torch.bfloat16 and x.dim() == 2 and offsets.dtype == torch.int32
     rows, cols = x.shape
@@ -329,9 +339,10 @@ def fp8_mx_quant_colwise_padded(x, offsets, q=None, ld_q=None, scales=None, stat
         ld = ld_q if ld_q is not None else (rows + 128 * e + 127) // 128 * 128
         q = torch.empty((cols, ld), dtype=torch.uint8, device=x.device)
     if scales is None:
-        scales = torch.empty((cols, (q.shape[1] + 127) // 128 * 4), dtype=torch.uint8,
+        scales = torch.empty((mx_scale_groups(q.shape[1]), cols), dtype=torch.int32,
                              device=x.device)
     _need_cuda(q, scales, status)
+    assert scales.dtype == torch.int32
     rc = lib().fp8_mx_quant_colwise_padded(_ptr(x), rows, cols, _ld(x), _ptr(offsets), e,
                                            _ptr(q), _ld(q), _ptr(scales), _ld(scales),
                                            _ptr(status), _stream(stream))
@@ -340,17 +351,19 @@ def fp8_mx_quant_colwise_padded(x, offsets, q=None, ld_q=None, scales=None, stat
 
 
 def fp8_mx_grouped_gemm(mode, a, scale_a, b, scale_b, offsets, m_total=None, n=None, k=None,
-                        out=None, out_dtype=torch.float32, status=None, stream=None):
-    """MXFP8 grouped GEMM (see the C header).
+                        out=None, out_dtype=torch.float32, status=None, b_group_stride=None,
+                        scale_b_group_stride=None, stream=None):
+    """MXFP8 grouped GEMM (see the C header); scales as returned by the MX
+    quantisation calls (int32 words [groups, rows]).
 
-    M_JAGGED: a uint8 [m_total, K], scale_a uint8 [m_total, ld_sa],
-    b uint8 [E, N, K], scale_b uint8 [E, N, ld_sb] -> out [m_total, N].
-    K_JAGGED_PADDED: a uint8 [N, ld_a], scale_a uint8 [N, ld_sa], b uint8
-    [K, ld_b], scale_b uint8 [K, ld_sb] (outputs of fp8_mx_quant_colwise_padded),
-    m_total unpadded tokens -> out [E, N, K]."""
+    M_JAGGED: a uint8 [m_total, K], scale_a [K/128, m_total], b uint8 [E, N, K]
+    (or [E*N, K]), scale_b [K/128, E*N] -> out [m_total, N].
+    K_JAGGED_PADDED: a uint8 [N, ld_a], scale_a [ld_a/128, N], b uint8 [K, ld_b],
+    scale_b [ld_b/128, K] (outputs of fp8_mx_quant_colwise_padded), m_total
+    unpadded tokens -> out [E, N, K]."""
     _need_cuda(a, scale_a, b, scale_b, offsets)
     assert a.dtype == torch.uint8 and b.dtype == torch.uint8 and offsets.dtype == torch.int32
-    assert scale_a.dtype == torch.uint8 and scale_b.dtype == torch.uint8
+    assert scale_a.dtype == torch.int32 and scale_b.dtype == torch.int32
     e = offsets.numel()
     if out is not None:
         out_dtype = out.dtype
@@ -359,10 +372,15 @@ def fp8_mx_grouped_gemm(mode, a, scale_a, b, scale_b, offsets, m_total=None, n=N
     if mode == M_JAGGED:
         m_total = a.shape[0] if m_total is None else m_total
         k = a.shape[1] if k is None else k
-        assert b.dim() == 3 and scale_b.dim() == 3
-        n = b.shape[1] if n is None else n
-        ld_b, bgs = b.stride(1), b.stride(0)
-        ld_sb, sbgs = scale_b.stride(1), scale_b.stride(0)
+        if b.dim() == 3:
+            n = b.shape[1] if n is None else n
+            ld_b = b.stride(1)
+            bgs = b.stride(0) if b_group_stride is None else b_group_stride
+        else:
+            n = b.shape[0] // e if n is None else n
+            ld_b = b.stride(0)
+            bgs = n * ld_b if b_group_stride is None else b_group_stride
+        sbgs = n if scale_b_group_stride is None else scale_b_group_stride
         if out is None:
             out = torch.empty((m_total, n), dtype=out_dtype, device=a.device)
         ld_out, ogs = _ld(out), 0
@@ -370,16 +388,15 @@ def fp8_mx_grouped_gemm(mode, a, scale_a, b, scale_b, offsets, m_total=None, n=N
         n = a.shape[0] if n is None else n
         k = b.shape[0] if k is None else k
         assert m_total is not None
-        ld_b, bgs = _ld(b), 0
-        ld_sb, sbgs = _ld(scale_b), 0
+        ld_b, bgs, sbgs = _ld(b), 0, 0
         if out is None:
             out = torch.empty((e, n, k), dtype=out_dtype, device=a.device)
         ld_out, ogs = out.stride(-2), out.stride(0)
     _need_cuda(out, status)
     rc = lib().fp8_mx_grouped_gemm(
         mode, _ptr(a), _ld(a), _ptr(scale_a), _ld(scale_a), _ptr(b), ld_b, bgs, _ptr(scale_b),
-        ld_sb, sbgs, _ptr(offsets), e, m_total, n, k, _ptr(out), ld_out, ogs, odt, _ptr(status),
-        _stream(stream))
+        _ld(scale_b), sbgs, _ptr(offsets), e, m_total, n, k, _ptr(out), ld_out, ogs, odt,
+        _ptr(status), _stream(stream))
     _check(rc, "fp8_mx_grouped_gemm")
     return out
 

@@ -22,10 +22,14 @@
 // Structure (one persistent CTA per SM, 10 warps):
 //   warp 0     producer: lane 0 issues the TMA copies of the A and B tiles
 //              (128 bytes of K per row, 128-byte swizzle) into a 4-stage ring;
-//              all 32 lanes copy the stage's scale bytes with 4-byte cp.async
-//              straight into the layout tcgen05.cp reads (row i + 32j of a
-//              128-row chunk at word 4i + j), whatever row the tile starts on,
-//              and the stage's full barrier completes when both have landed.
+//              all 32 lanes copy the stage's scale words (one 32-bit word per
+//              row holds the four block scales of the stage; the words of a
+//              stage are contiguous over the rows) with 4-byte cp.async,
+//              lane i taking rows i, i + 32, i + 64, i + 96 (each instruction
+//              reads one 128-byte line) straight into the layout tcgen05.cp
+//              reads (row i + 32j of a 128-row chunk at word 4i + j), whatever
+//              row the tile starts on; the stage's full barrier completes when
+//              both have landed.
 //   warp 1     MMA issuer: per stage, tcgen05.cp moves the scale chunks into
 //              TMEM (32x128b, replicated to the four lane quarters), then four
 //              block-scaled MMAs (M128 N bn K32), each selecting its block's
@@ -78,11 +82,11 @@ struct MxGemmSmem {
 };
 
 struct MxGemmParams {
-  const uint8_t *sfa;
+  const uint32_t *sfa;  // scale words [stage group, ld_sa]
   int64_t ld_sa;
-  const uint8_t *sfb;
+  const uint32_t *sfb;
   int64_t ld_sb;
-  int64_t sbs;  // scale_b group stride (token-jagged mode)
+  int64_t sbs;  // token-jagged mode: words between the experts' rows of B
   const int32_t *offsets;
   int num_groups;
   int64_t m_total, n, k;
@@ -342,7 +346,10 @@ __global__ void __launch_bounds__(kMxGemmThreads, 1)
           }
         }
         // scale words: row i + 32j of a chunk -> word 4i + j (lane = i)
-        const int64_t kw = ka / 32;  // the stage's first block
+        const int64_t kg = ka / kMxBK;  // the stage's group of four blocks
+        const uint32_t *sa_src = p.sfa + kg * p.ld_sa;
+        const uint32_t *sb_src = p.sfb + kg * p.ld_sb +
+                                 (MODE == FP8QGG_M_JAGGED ? int64_t(ti.e) * p.sbs : int64_t(0));
         const uint32_t sa_dst = smem_addr(sm.sfa[stage]) + 16 * lane;
         const uint32_t sb_dst = smem_addr(sm.sfb[stage]) + 16 * lane;
 #pragma unroll
@@ -356,7 +363,7 @@ __global__ void __launch_bounds__(kMxGemmThreads, 1)
             r = int64_t(ti.tm) * kMxBM + lane + 32 * j;
             lim = p.n;
           }
-          if (r < lim) cp_async_4(sa_dst + 4 * j, p.sfa + r * p.ld_sa + kw);
+          if (r < lim) cp_async_4(sa_dst + 4 * j, sa_src + r);
         }
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
@@ -364,12 +371,8 @@ __global__ void __launch_bounds__(kMxGemmThreads, 1)
           for (int j = 0; j < 4; ++j) {
             const int rr = 128 * c + lane + 32 * j;  // row of the B tile
             const int64_t nrow = int64_t(ti.tn) * bn + rr;
-            if (rr < bn && nrow < (MODE == FP8QGG_M_JAGGED ? p.n : p.k)) {
-              const uint8_t *src = MODE == FP8QGG_M_JAGGED
-                                       ? p.sfb + int64_t(ti.e) * p.sbs + nrow * p.ld_sb + kw
-                                       : p.sfb + nrow * p.ld_sb + kw;
-              cp_async_4(sb_dst + 512 * c + 4 * j, src);
-            }
+            if (rr < bn && nrow < (MODE == FP8QGG_M_JAGGED ? p.n : p.k))
+              cp_async_4(sb_dst + 512 * c + 4 * j, sb_src + nrow);
           }
         }
         cp_async_arrive_noinc(&sm.full[stage]);
@@ -564,8 +567,8 @@ int mx_pick_bn(int64_t n) {
 using namespace fp8qgg;
 
 extern "C" int fp8_mx_grouped_gemm(int mode, const uint8_t *a, int64_t ld_a,
-                                   const uint8_t *scale_a, int64_t ld_sa, const uint8_t *b,
-                                   int64_t ld_b, int64_t b_group_stride, const uint8_t *scale_b,
+                                   const uint32_t *scale_a, int64_t ld_sa, const uint8_t *b,
+                                   int64_t ld_b, int64_t b_group_stride, const uint32_t *scale_b,
                                    int64_t ld_sb, int64_t scale_b_group_stride,
                                    const int32_t *offsets, int32_t num_groups, int64_t m_total,
                                    int64_t n, int64_t k, void *out, int64_t ld_out,
@@ -581,24 +584,20 @@ extern "C" int fp8_mx_grouped_gemm(int mode, const uint8_t *a, int64_t ld_a,
   const int64_t ocols = kmode == FP8QGG_M_JAGGED ? n : k;
   if (kmode == FP8QGG_M_JAGGED) {
     if (k % 32) return FP8QGG_ERR_SHAPE;
-    const int64_t words = 4 * ((k + kMxBK - 1) / kMxBK);  // scale bytes read per row
-    if (ld_a < k || ld_b < k || ld_out < n || ld_sa < words || ld_sb < words)
+    if (ld_a < k || ld_b < k || ld_out < n || ld_sa < m_total) return FP8QGG_ERR_SHAPE;
+    if (num_groups > 1 && (b_group_stride < n * ld_b || scale_b_group_stride < n))
       return FP8QGG_ERR_SHAPE;
-    if (num_groups > 1 && (b_group_stride < n * ld_b || scale_b_group_stride < n * ld_sb))
-      return FP8QGG_ERR_SHAPE;
+    const int64_t brows = (num_groups > 1 ? (num_groups - 1) * scale_b_group_stride : 0) + n;
+    if (ld_sb < brows) return FP8QGG_ERR_SHAPE;
   } else {
     const int64_t tok = m_total + int64_t(kMxBK) * num_groups;
     if (tok > INT32_MAX / 2) return FP8QGG_ERR_SHAPE;
-    if (ld_a < tok || ld_b < tok || ld_out < k || ld_sa < tok / 32 || ld_sb < tok / 32)
-      return FP8QGG_ERR_SHAPE;
+    if (ld_a < tok || ld_b < tok || ld_out < k || ld_sa < n || ld_sb < k) return FP8QGG_ERR_SHAPE;
     if (num_groups > 1 && out_group_stride < n * ld_out) return FP8QGG_ERR_SHAPE;
   }
   if (!a || !b || !scale_a || !scale_b || !offsets || !out) return FP8QGG_ERR_NULL;
   if (!aligned(a, 16) || !aligned(b, 16) || !aligned(out, 16)) return FP8QGG_ERR_ALIGN;
   if (!aligned(scale_a, 4) || !aligned(scale_b, 4) || !aligned(offsets, 4)) return FP8QGG_ERR_ALIGN;
-  if (ld_sa % 4 || ld_sb % 4) return FP8QGG_ERR_ALIGN;
-  if (kmode == FP8QGG_M_JAGGED && num_groups > 1 && scale_b_group_stride % 4)
-    return FP8QGG_ERR_ALIGN;
   if (dev_status && !aligned(dev_status, 4)) return FP8QGG_ERR_ALIGN;
   if (ld_a % 16 || ld_b % 16) return FP8QGG_ERR_ALIGN;
   if (kmode == FP8QGG_M_JAGGED && b_group_stride % 16) return FP8QGG_ERR_ALIGN;

@@ -15,16 +15,23 @@
 //
 // The scale of a block depends on its 32 elements only, so each kernel reads
 // its input once and needs no cross-block reduction:
+// Scales are stored packed for the grouped GEMM: one 32-bit word per (row,
+// group of four blocks = 128 elements of the contraction axis), byte j the
+// scale of block 4g + j, and the words of one group g contiguous over the
+// rows (word g * ld_sw + r).  The GEMM then reads, per 128-deep stage, one
+// contiguous run of words for the rows of its tile.
 //  - rowwise: a lane owns 8 consecutive columns (one 16-byte load), four
-//    lanes one block; the block absmax is two shuffles away;
+//    lanes one block; the block absmax is two shuffles away, and four
+//    shuffles gather a group's four scale bytes into one word;
 //  - column-wise along each expert group's tokens, written transposed in the
 //    padded layout (group e from token P_e = sum_{j<e} round_up(size_j, 128),
 //    zero codes up to P_e + round_up(size_e, 128)): a thread block takes a
 //    tile of 128 tokens x 256 columns, eight warps of 16 tokens; the two warps
 //    of a 32-token block meet in shared memory for its column absmax; the
 //    codes go through a 128-byte-swizzled shared-memory tile to one bulk
-//    tensor store (whole 128-byte lines, padding zeros included), and each
-//    column's four scale bytes of the tile leave as one 4-byte store.
+//    tensor store (whole 128-byte lines, padding zeros included); a tile is
+//    one 128-token group, so its 256 scale words are contiguous (one 1 KB
+//    store).
 #include <algorithm>
 #include <cstring>
 
@@ -70,6 +77,10 @@ __device__ __forceinline__ uint32_t absmax8(const uint4 &v) {
 
 // ------------------------------------------------------------------ rowwise
 constexpr int kMxRowThreads = 256;
+
+__device__ __forceinline__ int64_t id_of(int64_t base, int u, int64_t nwarps) {
+  return base + u * nwarps;
+}
 constexpr int kMxRowUnroll = 4;  // 256-column segments in flight per warp
 
 struct MxRowParams {
@@ -78,10 +89,11 @@ struct MxRowParams {
   int64_t rows;
   int64_t segs;    // 256-column segments per row
   int cols;
+  int ngroups;     // 128-column groups (scale words per row)
   uint8_t *q;
   int64_t ld_q;
-  uint8_t *sc;
-  int64_t ld_s;
+  uint32_t *sw;    // scale words [ngroups, ld_sw]
+  int64_t ld_sw;
 };
 
 __global__ void __launch_bounds__(kMxRowThreads) mx_rowwise_kernel(const MxRowParams p) {
@@ -96,7 +108,7 @@ __global__ void __launch_bounds__(kMxRowThreads) mx_rowwise_kernel(const MxRowPa
     bool ok[kMxRowUnroll];
 #pragma unroll
     for (int u = 0; u < kMxRowUnroll; ++u) {
-      const int64_t id = base + u * nwarps;
+      const int64_t id = id_of(base, u, nwarps);
       row[u] = id / p.segs;
       col[u] = static_cast<int>(id - row[u] * p.segs) * 256 + 8 * lane;
       ok[u] = id < units && col[u] < p.cols;
@@ -109,10 +121,18 @@ __global__ void __launch_bounds__(kMxRowThreads) mx_rowwise_kernel(const MxRowPa
       m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
       const int e = mx_exponent(m);
       const uint2 c = mx_encode8(v[u], mx_multiplier(e));
-      if (ok[u]) {
-        __stcs(reinterpret_cast<uint2 *>(p.q + row[u] * p.ld_q + col[u]), c);
-        if ((lane & 3) == 0) p.sc[row[u] * p.ld_s + col[u] / 32] = static_cast<uint8_t>(e + 127);
-      }
+      // the word of 128-column group (lane >> 4): the bytes of lanes l0, l0 + 4,
+      // l0 + 8, l0 + 12 (columns past the row's end give byte 0)
+      const uint32_t byte = static_cast<uint32_t>(e + 127);
+      const int l0 = lane & 16;
+      const uint32_t word = __shfl_sync(0xFFFFFFFFu, byte, l0) |
+                            (__shfl_sync(0xFFFFFFFFu, byte, l0 + 4) << 8) |
+                            (__shfl_sync(0xFFFFFFFFu, byte, l0 + 8) << 16) |
+                            (__shfl_sync(0xFFFFFFFFu, byte, l0 + 12) << 24);
+      if (ok[u]) __stcs(reinterpret_cast<uint2 *>(p.q + row[u] * p.ld_q + col[u]), c);
+      const int64_t g = (id_of(base, u, nwarps) - row[u] * p.segs) * 2 + (lane >> 4);
+      if ((lane & 15) == 0 && id_of(base, u, nwarps) < units && g < p.ngroups)
+        p.sw[g * p.ld_sw + row[u]] = word;
     }
   }
 }
@@ -128,7 +148,7 @@ static_assert(kMxColWarps * kTileRowsPerWarp == kTileTokens, "eight warps of 16 
 struct MxColSmem {
   uint8_t tile[2][kMxTileBytes];           // transposed code tiles (1024-byte aligned)
   uint32_t red[kMxColWarps][kMxColWidth / 2];  // per-warp column absmax (bf16 pairs)
-  uint32_t sbytes[kMxColWidth];            // per column: the tile's four scale bytes
+  uint32_t sbytes[kMxColWidth];            // per column: the tile's scale word
   int32_t start[kMxMaxGroups];
   int32_t end[kMxMaxGroups];
   int32_t pstart[kMxMaxGroups];
@@ -143,8 +163,8 @@ struct MxColParams {
   int np;  // 256-column panels
   const int32_t *offsets;
   int num_groups;
-  uint8_t *sc;
-  int64_t ld_s;
+  uint32_t *sw;    // scale words [tokens / 128, ld_sw]
+  int64_t ld_sw;
   int32_t *status;
 };
 
@@ -263,9 +283,7 @@ __global__ void __launch_bounds__(kMxColThreads, 2)
       tma_store_2d(&qmap, tile, tok, c0);
       bulk_commit();
     }
-    if (c0 + tid < p.cols)
-      *reinterpret_cast<uint32_t *>(p.sc + static_cast<int64_t>(c0 + tid) * p.ld_s + tok / 32) =
-          sm.sbytes[tid];
+    if (c0 + tid < p.cols) p.sw[static_cast<int64_t>(tok / kTileTokens) * p.ld_sw + c0 + tid] = sm.sbytes[tid];
   }
   if (tid == 0) bulk_wait_all();  // the tiles stay valid until their stores have read them
 }
@@ -275,13 +293,14 @@ __global__ void __launch_bounds__(kMxColThreads, 2)
 using namespace fp8qgg;
 
 extern "C" int fp8_mx_quant_rowwise(const void *x, int64_t rows, int64_t cols, int64_t ld_x,
-                                    uint8_t *q, int64_t ld_q, uint8_t *scales, int64_t ld_s,
+                                    uint8_t *q, int64_t ld_q, uint32_t *scales, int64_t ld_sw,
                                     void *stream) {
   if (rows < 0 || cols < 1 || cols % 32 || cols > INT32_MAX / 2) return FP8QGG_ERR_SHAPE;
-  if (ld_x < cols || ld_q < cols || ld_s < cols / 32) return FP8QGG_ERR_SHAPE;
+  if (ld_x < cols || ld_q < cols || ld_sw < rows) return FP8QGG_ERR_SHAPE;
   if (rows == 0) return FP8QGG_OK;
   if (!x || !q || !scales) return FP8QGG_ERR_NULL;
   if (!aligned(x, 16) || ld_x % 8 || !aligned(q, 8) || ld_q % 8) return FP8QGG_ERR_ALIGN;
+  if (!aligned(scales, 4)) return FP8QGG_ERR_ALIGN;
   DeviceInfo dev;
   if (!device_info(&dev)) return FP8QGG_ERR_CUDA;
   MxRowParams prm;
@@ -290,10 +309,11 @@ extern "C" int fp8_mx_quant_rowwise(const void *x, int64_t rows, int64_t cols, i
   prm.rows = rows;
   prm.segs = (cols + 255) / 256;
   prm.cols = static_cast<int>(cols);
+  prm.ngroups = static_cast<int>((cols + 127) / 128);
   prm.q = q;
   prm.ld_q = ld_q;
-  prm.sc = scales;
-  prm.ld_s = ld_s;
+  prm.sw = scales;
+  prm.ld_sw = ld_sw;
   const int64_t warps = (rows * prm.segs + kMxRowUnroll - 1) / kMxRowUnroll;
   const int64_t want = (warps + kMxRowThreads / 32 - 1) / (kMxRowThreads / 32);
   const int grid = static_cast<int>(
@@ -305,16 +325,15 @@ extern "C" int fp8_mx_quant_rowwise(const void *x, int64_t rows, int64_t cols, i
 extern "C" int fp8_mx_quant_colwise_padded(const void *x, int64_t rows_total, int64_t cols,
                                            int64_t ld_x, const int32_t *offsets,
                                            int32_t num_groups, uint8_t *q, int64_t ld_q,
-                                           uint8_t *scales, int64_t ld_s, int32_t *dev_status,
+                                           uint32_t *scales, int64_t ld_sw, int32_t *dev_status,
                                            void *stream) {
   if (rows_total < 0 || cols < 1 || cols > INT32_MAX / 2 || ld_x < cols) return FP8QGG_ERR_SHAPE;
   if (num_groups < 1 || num_groups > kMxMaxGroups) return FP8QGG_ERR_SHAPE;
   const int64_t tokens = rows_total + int64_t(kTileTokens) * num_groups;
-  if (tokens > INT32_MAX / 2 || ld_q < tokens || ld_s < (tokens + 31) / 32)
-    return FP8QGG_ERR_SHAPE;
+  if (tokens > INT32_MAX / 2 || ld_q < tokens || ld_sw < cols) return FP8QGG_ERR_SHAPE;
   if (!offsets || !scales) return FP8QGG_ERR_NULL;
   if (rows_total > 0 && (!x || !q)) return FP8QGG_ERR_NULL;
-  if (cols % 8 || ld_x % 8 || ld_q % 16 || ld_s % 4) return FP8QGG_ERR_ALIGN;
+  if (cols % 8 || ld_x % 8 || ld_q % 16) return FP8QGG_ERR_ALIGN;
   if ((x && !aligned(x, 16)) || (q && !aligned(q, 16)) || !aligned(scales, 4) ||
       !aligned(offsets, 4))
     return FP8QGG_ERR_ALIGN;
@@ -349,8 +368,8 @@ extern "C" int fp8_mx_quant_colwise_padded(const void *x, int64_t rows_total, in
   prm.np = np;
   prm.offsets = offsets;
   prm.num_groups = num_groups;
-  prm.sc = scales;
-  prm.ld_s = ld_s;
+  prm.sw = scales;
+  prm.ld_sw = ld_sw;
   prm.status = dev_status;
   const int grid = static_cast<int>(
       std::max<int64_t>(1, std::min<int64_t>(tiles, int64_t(dev.sm_count) * 2)));

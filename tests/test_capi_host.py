@@ -211,44 +211,46 @@ def test_mx_quant_argument_checks(lib):
     r = lib.fp8_mx_quant_rowwise
 
     def row(**kw):
-        a = dict(x=FAKE, rows=10, cols=64, ldx=64, q=FAKE, ldq=64, s=FAKE, lds=4)
+        a = dict(x=FAKE, rows=10, cols=64, ldx=64, q=FAKE, ldq=64, s=FAKE, ldsw=10)
         a.update(kw)
-        return r(a["x"], a["rows"], a["cols"], a["ldx"], a["q"], a["ldq"], a["s"], a["lds"], None)
+        return r(a["x"], a["rows"], a["cols"], a["ldx"], a["q"], a["ldq"], a["s"], a["ldsw"],
+                 None)
 
     assert row(cols=48, ldx=48, ldq=48) == -2   # not whole 32-element blocks
-    assert row(lds=1) == -2                     # two blocks per row need two scale bytes
+    assert row(ldsw=9) == -2                    # one scale word per row and group
     assert row(ldx=32) == -2
     assert row(x=None) == -1
+    assert row(s=None) == -1
     assert row(ldx=68) == -3                    # 16-byte rows
     assert row(q=ODD) == -3
+    assert row(s=ctypes.c_void_p((1 << 20) + 2)) == -3
     assert row(rows=0) == 0                     # nothing to do
     c = lib.fp8_mx_quant_colwise_padded
 
     def col(**kw):
         a = dict(x=FAKE, rows=100, cols=64, ldx=64, off=FAKE, e=2, q=FAKE, ldq=368, s=FAKE,
-                 lds=12)
+                 ldsw=64)
         a.update(kw)
         return c(a["x"], a["rows"], a["cols"], a["ldx"], a["off"], a["e"], a["q"], a["ldq"],
-                 a["s"], a["lds"], None, None)
+                 a["s"], a["ldsw"], None, None)
 
     assert col(ldq=352) == -2                   # rows + 128 per group = 356 tokens
-    assert col(lds=8) == -2                     # 356 tokens = 12 blocks
+    assert col(ldsw=63) == -2                   # one word per column and token group
     assert col(ldq=360) == -3                   # 16-byte token rows
-    assert col(lds=13) == -3
-    assert col(lds=14) == -3                    # 4-byte scale words
     assert col(e=0) == -2
     assert col(e=1025) == -2
-    assert col(cols=60, ldx=64) == -3
+    assert col(cols=60, ldx=64, ldsw=64) == -3
     assert col(off=None) == -1
+    assert col(s=ctypes.c_void_p((1 << 20) + 2)) == -3
 
 
 def test_mx_gemm_argument_checks(lib):
     f = lib.fp8_mx_grouped_gemm
 
     def call(**kw):
-        a = dict(mode=0, a=FAKE, lda=256, sa=FAKE, ldsa=8, b=FAKE, ldb=256, bgs=256 * 32, sb=FAKE,
-                 ldsb=8, sbgs=8 * 32, off=FAKE, e=2, m=100, n=32, k=256, out=FAKE, ldo=32, ogs=0,
-                 odt=0)
+        a = dict(mode=0, a=FAKE, lda=256, sa=FAKE, ldsa=100, b=FAKE, ldb=256, bgs=256 * 32,
+                 sb=FAKE, ldsb=64, sbgs=32, off=FAKE, e=2, m=100, n=32, k=256, out=FAKE, ldo=32,
+                 ogs=0, odt=0)
         a.update(kw)
         return f(a["mode"], a["a"], a["lda"], a["sa"], a["ldsa"], a["b"], a["ldb"], a["bgs"],
                  a["sb"], a["ldsb"], a["sbgs"], a["off"], a["e"], a["m"], a["n"], a["k"],
@@ -257,16 +259,17 @@ def test_mx_gemm_argument_checks(lib):
     assert call(mode=1) == -4          # plain contraction-jagged: blocks could hold two groups
     assert call(odt=3) == -4
     assert call(k=240, lda=256, ldb=256) == -2   # whole 32-element blocks only
-    assert call(ldsa=4) == -2          # 256 columns: 8 scale bytes per row are read
-    assert call(ldsa=10) == -3         # scale rows of whole 4-byte words
-    assert call(sbgs=8 * 31) == -2     # scale groups of B overlap
+    assert call(ldsa=99) == -2         # one scale word per row of A and group
+    assert call(sbgs=31) == -2         # the experts' scale rows of B overlap
+    assert call(ldsb=63) == -2         # two experts of 32 rows
     assert call(bgs=256 * 31) == -2
     assert call(e=0) == -2
     assert call(sa=None) == -1
     assert call(sa=ctypes.c_void_p((1 << 20) + 2)) == -3
     assert call(m=0) == 0              # token-jagged with no rows: nothing to write
-    # padded contraction-jagged: tokens + 128 per group on both operands and scales
-    kw = dict(mode=2, lda=368, ldb=368, ldsa=12, ldsb=12, n=32, k=64, ldo=64, ogs=32 * 64)
+    # padded contraction-jagged: tokens + 128 per group on both operands
+    kw = dict(mode=2, lda=368, ldb=368, ldsa=32, ldsb=64, n=32, k=64, ldo=64, ogs=32 * 64)
     assert call(**dict(kw, lda=352)) == -2
-    assert call(**dict(kw, ldsa=8)) == -2
+    assert call(**dict(kw, ldsa=31)) == -2
+    assert call(**dict(kw, ldsb=63)) == -2
     assert call(**dict(kw, ogs=16)) == -2

@@ -19,6 +19,7 @@ import pytest
 import torch
 
 import oracle as orc
+import quantization_grouped_gemm_b200 as qgg
 from quantization_grouped_gemm_b200 import workloads as wl
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
@@ -237,3 +238,74 @@ def test_deepseek_moe16b_dual_output_full_size():
     assert (got == expect).all()
     got_s = st.sc2[:, torch.from_numpy(cols).cuda()].cpu().numpy()
     assert (got_s.view(np.uint32) == cs_ref.view(np.uint32)).all()
+
+
+def test_llama3_8b_up_projection_mxfp8_full_size_sampled():
+    """MXFP8 forward at full size (the benchmark's MxForwardStep): MX rowwise X
+    and W on sampled rows, bit-exact with every block scale; the block-scaled
+    GEMM on sampled outputs from the oracle's own MX quantisation."""
+    w = wl.llama3_8b_up_proj()
+    st = bench.MxForwardStep(w)
+    run_step(st)
+    g = np.random.default_rng(21)
+    m, k = w.x.shape
+    e, n = w.w.shape[0], w.w.shape[1]
+    rows = sample(g, m, 32, must=[0, m - 1])
+    qa_ref, sa_ref = orc.mx_quant_rowwise(wl.bf16_bits(w.x[torch.from_numpy(rows)]))
+    assert (st.qa[torch.from_numpy(rows).cuda()].cpu().numpy() == qa_ref).all()
+    sa_blocks = qgg.mx_scales_to_blocks(st.sa, k // 32)
+    assert (sa_blocks[torch.from_numpy(rows).cuda()].cpu().numpy() == sa_ref).all()
+    cols = sample(g, n, 32, must=[0, n - 1])
+    wsel = w.w[:, torch.from_numpy(cols), :].reshape(e * len(cols), k)
+    qb_ref, sb_ref = orc.mx_quant_rowwise(wl.bf16_bits(wsel))
+    qb = st.qb.view(e, n, k)[:, torch.from_numpy(cols).cuda(), :].reshape(e * len(cols), k)
+    assert (qb.cpu().numpy() == qb_ref).all()
+    sb = qgg.mx_scales_to_blocks(st.sb, k // 32).view(e, n, -1)[:, torch.from_numpy(cols).cuda()]
+    assert (sb.reshape(e * len(cols), -1).cpu().numpy() == sb_ref).all()
+    ns = 2000
+    li = g.integers(0, len(rows), ns)
+    lj = g.integers(0, len(cols), ns)
+    c, b = orc.mx_gemm_m_jagged_sample(qa_ref, sa_ref, qb_ref.reshape(e, len(cols), k),
+                                       sb_ref.reshape(e, len(cols), k // 32),
+                                       np.array([len(rows)], np.int32), li, lj)
+    out = st.out[torch.from_numpy(rows[li]).cuda(), torch.from_numpy(cols[lj]).cuda()]
+    got = out.cpu().numpy().astype(np.float64)
+    bad = np.nonzero(~(np.abs(got - c) <= b))[0]
+    assert bad.size == 0, (bad.size, got[bad[:4]], c[bad[:4]], b[bad[:4]])
+
+
+def test_deepseek_moe16b_backward_mxfp8_full_size_sampled():
+    """MXFP8 weight gradient at full size (the benchmark's MxBackwardDwStep):
+    MX quantisation of grad_out and X along each group's tokens on sampled
+    columns over all 98304 rows (codes of the whole padded range, gaps
+    included, and every scale byte), then the block-scaled contraction-jagged
+    dW on sampled (expert, row, column) outputs."""
+    w = wl.deepseek_moe_16b_backward()
+    st = bench.MxBackwardDwStep(w)
+    run_step(st)
+    g = np.random.default_rng(22)
+    m = st.m
+    p_end = orc.padded_len(np.diff(np.concatenate([[0], w.offsets])))
+    checked = []
+    for src, q_dev, s_dev in ((w.grad_out, st.qg, st.sg), (w.x, st.qx, st.sx)):
+        cols = sample(g, src.shape[1], 16, must=[0, src.shape[1] - 1])
+        q_ref, s_ref = orc.mx_quant_colwise_padded(wl.bf16_bits(src[:, torch.from_numpy(cols)]),
+                                                   w.offsets)
+        assert q_ref.shape[1] == p_end
+        got_q = q_dev[torch.from_numpy(cols).cuda(), :p_end].cpu().numpy()
+        assert (got_q == q_ref).all()
+        blocks = qgg.mx_scales_to_blocks(s_dev, p_end // 32)
+        got_s = blocks[torch.from_numpy(cols).cuda()].cpu().numpy()
+        assert (got_s == s_ref).all()
+        checked.append((cols, q_ref, s_ref))
+    (ci, qa_t, sa_t), (cj, qb_t, sb_t) = checked
+    ns = 3000
+    grp = g.integers(0, st.e, ns)
+    li = g.integers(0, len(ci), ns)
+    lj = g.integers(0, len(cj), ns)
+    c, b = orc.mx_gemm_k_jagged_padded_sample(qa_t, sa_t, qb_t, sb_t, w.offsets, m, grp, li, lj)
+    out = st.out[torch.from_numpy(grp).cuda(), torch.from_numpy(ci[li]).cuda(),
+                 torch.from_numpy(cj[lj]).cuda()]
+    got = out.cpu().numpy().astype(np.float64)
+    bad = np.nonzero(~(np.abs(got - c) <= b))[0]
+    assert bad.size == 0, (bad.size, got[bad[:4]], c[bad[:4]], b[bad[:4]])

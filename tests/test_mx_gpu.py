@@ -36,6 +36,9 @@ def spread_bf16(seed, shape, block_axis=-1, spread=12.0, outliers=0.0):
     return wl.to_bf16(a.astype(np.float32))
 
 
+CANARY = -842150451  # 0xCDCDCDCD
+
+
 def bits(x):
     return wl.bf16_bits(x)
 
@@ -49,7 +52,9 @@ def test_mx_rowwise_bit_exact(rows, cols):
     torch.cuda.synchronize()
     q_ref, s_ref = orc.mx_quant_rowwise(bits(x))
     assert (q.cpu().numpy() == q_ref).all()
-    assert (s.cpu().numpy()[:, :cols // 32] == s_ref).all()
+    blocks = qgg.mx_scales_to_blocks(s, 4 * s.shape[0]).cpu().numpy()
+    assert (blocks[:, :cols // 32] == s_ref).all()
+    assert (blocks[:, cols // 32:] == 0).all()  # bytes past the row's last block
 
 
 def test_mx_rowwise_special_values():
@@ -76,7 +81,7 @@ def test_mx_rowwise_special_values():
     q_ref, s_ref = orc.mx_quant_rowwise(bits(x))
     qd = q.cpu().numpy()
     nan = np.isnan(x.float().numpy())
-    assert (s.cpu().numpy()[:, :2] == s_ref).all()
+    assert (qgg.mx_scales_to_blocks(s, 2).cpu().numpy() == s_ref).all()
     assert (qd[~nan] == q_ref[~nan]).all()
     # a NaN input gives a NaN code (0x7F or 0xFF)
     assert ((qd[nan] & 0x7F) == 0x7F).all()
@@ -86,14 +91,14 @@ def test_mx_rowwise_strided_input_and_untouched_padding():
     base = spread_bf16(5, (40, 200))
     x = base[:, 8:168]  # 160 columns, row stride 200
     q = torch.full((40, 168), 0xAB, dtype=torch.uint8, device="cuda")
-    s = torch.full((40, 8), 0xCD, dtype=torch.uint8, device="cuda")
-    qgg.fp8_mx_quant_rowwise(x.cuda(), q=q[:, :160], scales=s)
+    s = torch.full((3, 44), CANARY, dtype=torch.int32, device="cuda")  # 2 groups, ld_sw 44
+    qgg.fp8_mx_quant_rowwise(x.cuda(), q=q[:, :160], scales=s[:2])
     torch.cuda.synchronize()
     q_ref, s_ref = orc.mx_quant_rowwise(bits(x.contiguous()))
     assert (q.cpu().numpy()[:, :160] == q_ref).all()
     assert (q.cpu().numpy()[:, 160:] == 0xAB).all()
-    assert (s.cpu().numpy()[:, :5] == s_ref).all()
-    assert (s.cpu().numpy()[:, 5:] == 0xCD).all()
+    assert (qgg.mx_scales_to_blocks(s[:2, :40], 5).cpu().numpy() == s_ref).all()
+    assert (s[:2, 40:] == CANARY).all() and (s[2] == CANARY).all()
 
 
 # --------------------------------------------------------------------------- colwise
@@ -114,7 +119,7 @@ def test_mx_colwise_padded_bit_exact(sizes, cols):
     e = len(sizes)
     ld_q = (m + extra + 128 * e + 127) // 128 * 128
     q = torch.full((cols, ld_q), 0xAB, dtype=torch.uint8, device="cuda")
-    s = torch.full((cols, ld_q // 32), 0xCD, dtype=torch.uint8, device="cuda")
+    s = torch.full((ld_q // 128, cols), CANARY, dtype=torch.int32, device="cuda")
     st = torch.zeros(1, dtype=torch.int32, device="cuda")
     qgg.fp8_mx_quant_colwise_padded(x.cuda(), torch.from_numpy(off).cuda(), q=q, scales=s,
                                     status=st)
@@ -123,7 +128,7 @@ def test_mx_colwise_padded_bit_exact(sizes, cols):
                                                scale_fill=0xCD)
     bad = np.argwhere(q.cpu().numpy() != q_ref)
     assert bad.size == 0, (bad.shape, bad[:8])
-    assert (s.cpu().numpy() == s_ref).all()
+    assert (qgg.mx_scales_to_blocks(s, ld_q // 32).cpu().numpy() == s_ref).all()
     assert int(st.item()) == 0
 
 
@@ -145,7 +150,7 @@ def check_m_jagged(sizes, n, k, out_dtype=torch.float32, seed=1, full=True):
     qb, sb = qgg.fp8_mx_quant_rowwise(w.cuda())
     out = torch.full((m + 5, n), float("nan"), dtype=out_dtype, device="cuda")
     st = torch.zeros(1, dtype=torch.int32, device="cuda")
-    qgg.fp8_mx_grouped_gemm(qgg.M_JAGGED, qa, sa, qb.view(e, n, k), sb.view(e, n, -1),
+    qgg.fp8_mx_grouped_gemm(qgg.M_JAGGED, qa, sa, qb.view(e, n, k), sb,
                             torch.from_numpy(off).cuda(), out=out[:m], status=st)
     torch.cuda.synchronize()
     assert int(st.item()) == 0
