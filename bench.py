@@ -625,7 +625,8 @@ def run_gpu(args, world, rank, local):
         value = flops * world / (ms_step * 1e-3) / 1e12
         unit = "TFLOP/s"
         e2e_value = flops * world / (e2e_ms * 1e-3) / 1e12
-        gemm_tflops = kern["grouped_gemm"]["tflops"]
+        gemm_name = next(nm for nm in st.names if nm.endswith("grouped_gemm"))
+        gemm_tflops = kern[gemm_name]["tflops"]
         roof = dict(bound="tensor", achieved=gemm_tflops, peak=fp8_peak, unit="TFLOP/s",
                     frac=gemm_tflops / fp8_peak, traffic=TRAFFIC.get(args.workload),
                     peak_note=(f"{pk['source']} bf16 burst {pk['bf16']} TFLOP/s x 2 "

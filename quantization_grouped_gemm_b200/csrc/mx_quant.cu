@@ -20,13 +20,16 @@
 // scale of block 4g + j, and the words of one group g contiguous over the
 // rows (word g * ld_sw + r).  The GEMM then reads, per 128-deep stage, one
 // contiguous run of words for the rows of its tile.
-//  - rowwise: a lane owns 8 consecutive columns (one 16-byte load), four
-//    lanes one block; the block absmax is two shuffles away, and four
-//    shuffles gather a group's four scale bytes into one word;
+//  - rowwise: a warp takes 32 rows x one 128-column group; a lane owns 8
+//    consecutive columns of a row (one 16-byte load), four lanes one block;
+//    the block absmax is two shuffles away, four shuffles gather a row's
+//    four scale bytes into its word, and the group's 32 words leave as one
+//    128-byte store;
 //  - column-wise along each expert group's tokens, written transposed in the
 //    padded layout (group e from token P_e = sum_{j<e} round_up(size_j, 128),
-//    zero codes up to P_e + round_up(size_e, 128)): a thread block takes a
-//    tile of 128 tokens x 256 columns, eight warps of 16 tokens; the two warps
+//    zero codes up to P_e + round_up(size_e, 128)): tiles of 128 tokens x 256
+//    columns stream in by TMA through a two-stage shared-memory ring; eight
+//    consumer warps of 16 tokens reduce and encode a tile; the two warps
 //    of a 32-token block meet in shared memory for its column absmax; the
 //    codes go through a 128-byte-swizzled shared-memory tile to one bulk
 //    tensor store (whole 128-byte lines, padding zeros included); a tile is
@@ -76,107 +79,172 @@ __device__ __forceinline__ uint32_t absmax8(const uint4 &v) {
 }
 
 // ------------------------------------------------------------------ rowwise
+// A warp takes 32 rows x one 128-column group: sixteen lanes per row (8
+// columns each, one 16-byte load), two rows per load instruction, sixteen
+// loads in flight per lane.  A block's four lanes meet by two shuffles; the
+// group's scale words of the 32 rows end up one per lane and leave as one
+// 128-byte store.
 constexpr int kMxRowThreads = 256;
-
-__device__ __forceinline__ int64_t id_of(int64_t base, int u, int64_t nwarps) {
-  return base + u * nwarps;
-}
-constexpr int kMxRowUnroll = 4;  // 256-column segments in flight per warp
+constexpr int kMxRowsPerWarp = 32;
 
 struct MxRowParams {
   const uint4 *x;
   int64_t ld_x16;  // row pitch in 16-byte vectors
   int64_t rows;
-  int64_t segs;    // 256-column segments per row
   int cols;
   int ngroups;     // 128-column groups (scale words per row)
+  int64_t units;   // ceil(rows / 32) * ngroups
   uint8_t *q;
   int64_t ld_q;
   uint32_t *sw;    // scale words [ngroups, ld_sw]
   int64_t ld_sw;
 };
 
-__global__ void __launch_bounds__(kMxRowThreads) mx_rowwise_kernel(const MxRowParams p) {
+__global__ void __launch_bounds__(kMxRowThreads, 2) mx_rowwise_kernel(const MxRowParams p) {
   const int lane = threadIdx.x & 31;
-  const int64_t units = p.rows * p.segs;
+  const int half = lane >> 4;          // which of the two rows of a load
+  const int c16 = lane & 15;           // 8-column slot within the group
   const int64_t nwarps = static_cast<int64_t>(gridDim.x) * (kMxRowThreads / 32);
-  const int64_t warp0 = (static_cast<int64_t>(blockIdx.x) * kMxRowThreads + threadIdx.x) >> 5;
-  for (int64_t base = warp0; base < units; base += nwarps * kMxRowUnroll) {
-    uint4 v[kMxRowUnroll];
-    int64_t row[kMxRowUnroll];
-    int col[kMxRowUnroll];
-    bool ok[kMxRowUnroll];
+  for (int64_t u = (static_cast<int64_t>(blockIdx.x) * kMxRowThreads + threadIdx.x) >> 5;
+       u < p.units; u += nwarps) {
+    const int64_t rb = u / p.ngroups;  // once per 32 x 128 unit
+    const int g = static_cast<int>(u - rb * p.ngroups);
+    const int64_t r0 = rb * kMxRowsPerWarp;
+    const int col = 128 * g + 8 * c16;
+    const bool c_ok = col < p.cols;
+    uint4 v[kMxRowsPerWarp / 2];
 #pragma unroll
-    for (int u = 0; u < kMxRowUnroll; ++u) {
-      const int64_t id = id_of(base, u, nwarps);
-      row[u] = id / p.segs;
-      col[u] = static_cast<int>(id - row[u] * p.segs) * 256 + 8 * lane;
-      ok[u] = id < units && col[u] < p.cols;
-      v[u] = ok[u] ? __ldcs(p.x + row[u] * p.ld_x16 + col[u] / 8) : make_uint4(0u, 0u, 0u, 0u);
+    for (int i = 0; i < kMxRowsPerWarp / 2; ++i) {
+      const int64_t r = r0 + 2 * i + half;
+      v[i] = (c_ok && r < p.rows) ? __ldcs(p.x + r * p.ld_x16 + col / 8)
+                                  : make_uint4(0u, 0u, 0u, 0u);
     }
+    uint32_t myword = 0;  // lane j: the scale word of row r0 + j
 #pragma unroll
-    for (int u = 0; u < kMxRowUnroll; ++u) {
-      uint32_t m = absmax8(v[u]);
+    for (int i = 0; i < kMxRowsPerWarp / 2; ++i) {
+      uint32_t m = absmax8(v[i]);
       m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
       m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
       const int e = mx_exponent(m);
-      const uint2 c = mx_encode8(v[u], mx_multiplier(e));
-      // the word of 128-column group (lane >> 4): the bytes of lanes l0, l0 + 4,
-      // l0 + 8, l0 + 12 (columns past the row's end give byte 0)
+      const uint2 c = mx_encode8(v[i], mx_multiplier(e));
+      const int64_t r = r0 + 2 * i + half;
+      if (c_ok && r < p.rows) __stcs(reinterpret_cast<uint2 *>(p.q + r * p.ld_q + col), c);
+      // the row's word: bytes of the lanes 16h, 16h + 4, 16h + 8, 16h + 12
+      // (columns past the row's end give byte 0)
       const uint32_t byte = static_cast<uint32_t>(e + 127);
       const int l0 = lane & 16;
       const uint32_t word = __shfl_sync(0xFFFFFFFFu, byte, l0) |
                             (__shfl_sync(0xFFFFFFFFu, byte, l0 + 4) << 8) |
                             (__shfl_sync(0xFFFFFFFFu, byte, l0 + 8) << 16) |
                             (__shfl_sync(0xFFFFFFFFu, byte, l0 + 12) << 24);
-      if (ok[u]) __stcs(reinterpret_cast<uint2 *>(p.q + row[u] * p.ld_q + col[u]), c);
-      const int64_t g = (id_of(base, u, nwarps) - row[u] * p.segs) * 2 + (lane >> 4);
-      if ((lane & 15) == 0 && id_of(base, u, nwarps) < units && g < p.ngroups)
-        p.sw[g * p.ld_sw + row[u]] = word;
+      const uint32_t w0 = __shfl_sync(0xFFFFFFFFu, word, 0);
+      const uint32_t w1 = __shfl_sync(0xFFFFFFFFu, word, 16);
+      if (lane == 2 * i) myword = w0;
+      if (lane == 2 * i + 1) myword = w1;
     }
+    if (r0 + lane < p.rows) p.sw[static_cast<int64_t>(g) * p.ld_sw + r0 + lane] = myword;
   }
 }
 
 // ------------------------------------------------------- column-wise, padded
-constexpr int kMxColWarps = 8;
-constexpr int kMxColThreads = 32 * kMxColWarps;
+// One persistent thread block per SM: a producer warp copies the input tiles
+// (128 rows x 256 columns of bf16, 64 KB) with TMA into a two-stage ring in
+// shared memory, so that the next tile streams in while eight consumer warps
+// (16 rows each) reduce, encode and store the current one.
+constexpr int kMxColWarps = 8;                       // consumers
+constexpr int kMxColThreads = 32 * kMxColWarps + 32;  // + the producer warp
+constexpr int kMxColConsumers = 32 * kMxColWarps;
 constexpr int kMxColWidth = 256;  // columns per tile
 constexpr int kMxMaxGroups = 1024;
+constexpr int kMxColStages = 2;
 constexpr uint32_t kMxTileBytes = kMxColWidth * kTileTokens;
+constexpr uint32_t kMxInBytes = kTileTokens * kMxColWidth * 2;
 static_assert(kMxColWarps * kTileRowsPerWarp == kTileTokens, "eight warps of 16 tokens");
 
 struct MxColSmem {
-  uint8_t tile[2][kMxTileBytes];           // transposed code tiles (1024-byte aligned)
+  uint8_t in[kMxColStages][kMxInBytes];    // input tiles, row-major (1024-byte aligned)
+  uint8_t tile[2][kMxTileBytes];           // transposed code tiles
   uint32_t red[kMxColWarps][kMxColWidth / 2];  // per-warp column absmax (bf16 pairs)
   uint32_t sbytes[kMxColWidth];            // per column: the tile's scale word
   int32_t start[kMxMaxGroups];
   int32_t end[kMxMaxGroups];
   int32_t pstart[kMxMaxGroups];
   int32_t tpre[kMxMaxGroups + 1];          // tiles of the groups before group e
+  uint64_t full[kMxColStages];
+  uint64_t empty[kMxColStages];
+  int abort;
 };
 
 struct MxColParams {
-  const uint4 *x;
-  int64_t ld_x16;
   int64_t rows_total;
   int cols;
-  int np;  // 256-column panels
+  int box_cols;  // columns of an input tile (min(256, cols))
+  int np;        // 256-column panels
   const int32_t *offsets;
   int num_groups;
-  uint32_t *sw;    // scale words [tokens / 128, ld_sw]
+  uint32_t *sw;  // scale words [tokens / 128, ld_sw]
   int64_t ld_sw;
   int32_t *status;
 };
 
-__global__ void __launch_bounds__(kMxColThreads, 2)
-    mx_colwise_kernel(const __grid_constant__ CUtensorMap qmap, const MxColParams p) {
+struct MxColTile {
+  int e, q;
+  int32_t b;
+};
+
+__device__ __forceinline__ MxColTile mx_col_tile(const MxColSmem &sm, int G, int32_t t) {
+  // tile t -> group e (last group whose prefix is <= t), panel, block
+  int lo = 0, hi = G - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (sm.tpre[mid] <= t) lo = mid; else hi = mid - 1;
+  }
+  MxColTile r;
+  r.e = lo;
+  const int32_t nb = (sm.end[lo] - sm.start[lo] + kTileTokens - 1) / kTileTokens;
+  const int32_t local = t - sm.tpre[lo];
+  r.q = local / nb;
+  r.b = local - r.q * nb;
+  return r;
+}
+
+// Named barrier over the consumer warps that also ANDs a flag across them.
+__device__ __forceinline__ bool consumers_and(bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 q, %1, 0;\n\t"
+      "bar.red.and.pred p, 1, %2, q;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(r)
+      : "r"(static_cast<uint32_t>(v)), "n"(kMxColConsumers)
+      : "memory");
+  return r != 0;
+}
+
+__device__ __forceinline__ void consumers_sync() {
+  asm volatile("bar.sync 1, %0;" ::"n"(kMxColConsumers) : "memory");
+}
+
+__global__ void __launch_bounds__(kMxColThreads, 1)
+    mx_colwise_kernel(const __grid_constant__ CUtensorMap xmap,
+                      const __grid_constant__ CUtensorMap qmap, const MxColParams p) {
   extern __shared__ uint8_t smem_raw[];
   MxColSmem &sm = *align_smem_1024<MxColSmem>(smem_raw);
   const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
   const int G = p.num_groups;
-  if (tid == 0) prefetch_tensormap(&qmap);
+  if (tid == 0) {
+    prefetch_tensormap(&xmap);
+    prefetch_tensormap(&qmap);
+    for (int s = 0; s < kMxColStages; ++s) {
+      mbar_init(&sm.full[s], 1);
+      mbar_init(&sm.empty[s], kMxColWarps);
+    }
+    sm.abort = 0;
+    fence_mbarrier_init();
+  }
   // clamped group bounds, padded starts and tile prefix (one warp)
-  if (tid < 32) {
+  if (w == kMxColWarps) {
     const int32_t R = static_cast<int32_t>(p.rows_total);
     int32_t carry_end = 0, carry_pad = 0, carry_t = 0;
     bool bad = false;
@@ -218,74 +286,111 @@ __global__ void __launch_bounds__(kMxColThreads, 2)
   }
   __syncthreads();
   const int32_t total = sm.tpre[G];
-  uint8_t *sb8 = reinterpret_cast<uint8_t *>(sm.sbytes);
-  int it = 0;
-  for (int32_t t = blockIdx.x; t < total; t += gridDim.x, ++it) {
-    // tile t -> group e (last group whose prefix is <= t), panel, block
-    int lo = 0, hi = G - 1;
-    while (lo < hi) {
-      const int mid = (lo + hi + 1) >> 1;
-      if (sm.tpre[mid] <= t) lo = mid; else hi = mid - 1;
+  volatile int *abort = &sm.abort;
+  const uint32_t in_bytes = static_cast<uint32_t>(kTileTokens * p.box_cols * 2);
+
+  if (w == kMxColWarps) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      uint32_t armed = 0, last_par[kMxColStages] = {0, 0};
+      int i = 0;
+      bool ok = true;
+      for (int32_t t = blockIdx.x; t < total; t += gridDim.x, ++i) {
+        const int st = i % kMxColStages;
+        const uint32_t ph = (i / kMxColStages) & 1;
+        if (!mbar_wait(&sm.empty[st], ph ^ 1, abort)) {
+          ok = false;
+          break;
+        }
+        const MxColTile tl = mx_col_tile(sm, G, t);
+        mbar_arrive_expect_tx(&sm.full[st], in_bytes);
+        tma_load_2d(sm.in[st], &xmap, &sm.full[st], tl.q * kMxColWidth,
+                    sm.start[tl.e] + tl.b * kTileTokens);
+        armed |= 1u << st;
+        last_par[st] = ph;
+      }
+      if (!ok) {
+        *abort = 1;
+        status_or(p.status, FP8QGG_STATUS_TIMEOUT);
+      }
+      // copies in flight land before the block can exit
+      volatile int never = 0;
+      for (int s = 0; s < kMxColStages; ++s)
+        if (armed & (1u << s)) (void)mbar_wait(&sm.full[s], last_par[s], &never);
     }
-    const int e = lo;
-    const int32_t nb = (sm.end[e] - sm.start[e] + kTileTokens - 1) / kTileTokens;
-    const int32_t local = t - sm.tpre[e];
-    const int q = local / nb;
-    const int32_t b = local - q * nb;
-    const int c0 = q * kMxColWidth;
-    const int col = c0 + 8 * lane;
-    const bool c_ok = col < p.cols;
-    const int32_t r0 = sm.start[e] + b * kTileTokens + kTileRowsPerWarp * w;
-    const int32_t r1 = sm.end[e];
-    uint4 v[kTileRowsPerWarp];
-    const uint4 *src = p.x + static_cast<int64_t>(r0) * p.ld_x16 + col / 8;
+  } else {
+    // ------------------------------------------------------------ consumers
+    uint8_t *sb8 = reinterpret_cast<uint8_t *>(sm.sbytes);
+    const int row_bytes = p.box_cols * 2;
+    int i = 0;
+    for (int32_t t = blockIdx.x; t < total; t += gridDim.x, ++i) {
+      const int st = i % kMxColStages;
+      const uint32_t ph = (i / kMxColStages) & 1;
+      const MxColTile tl = mx_col_tile(sm, G, t);
+      const int c0 = tl.q * kMxColWidth;
+      const bool c_ok = c0 + 8 * lane < p.cols;
+      const int32_t rw0 = sm.start[tl.e] + tl.b * kTileTokens + kTileRowsPerWarp * w;
+      const int32_t r1 = sm.end[tl.e];
+      const bool got = mbar_wait(&sm.full[st], ph, abort);
+      uint4 v[kTileRowsPerWarp];
+      const uint8_t *src = sm.in[st] + (kTileRowsPerWarp * w) * row_bytes + 16 * lane;
 #pragma unroll
-    for (int k = 0; k < kTileRowsPerWarp; ++k)
-      v[k] = (c_ok && r0 + k < r1) ? __ldcs(src + k * p.ld_x16) : make_uint4(0u, 0u, 0u, 0u);
-    // the warp's 16-row column absmax, as bf16 magnitude pairs
-    uint32_t acc[4] = {0u, 0u, 0u, 0u};
+      for (int k = 0; k < kTileRowsPerWarp; ++k)
+        v[k] = (got && c_ok && rw0 + k < r1) ? *reinterpret_cast<const uint4 *>(src + k * row_bytes)
+                                             : make_uint4(0u, 0u, 0u, 0u);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.empty[st]);  // the stage may be refilled
+      uint32_t acc[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
-    for (int k = 0; k < kTileRowsPerWarp; ++k) {
-      acc[0] = absmax_acc(acc[0], v[k].x);
-      acc[1] = absmax_acc(acc[1], v[k].y);
-      acc[2] = absmax_acc(acc[2], v[k].z);
-      acc[3] = absmax_acc(acc[3], v[k].w);
-    }
-    *reinterpret_cast<uint4 *>(&sm.red[w][4 * lane]) =
-        make_uint4(absmax_bits(acc[0]), absmax_bits(acc[1]), absmax_bits(acc[2]),
-                   absmax_bits(acc[3]));
-    uint8_t *tile = sm.tile[it & 1];
-    // the store issued from this tile buffer two tiles ago has read it
-    if (tid == 0) bulk_wait_read<1>();
-    __syncthreads();
-    // the 32-token block of warps 2k, 2k+1: its column absmax and scale
-    const uint4 mine = *reinterpret_cast<const uint4 *>(&sm.red[w][4 * lane]);
-    const uint4 other = *reinterpret_cast<const uint4 *>(&sm.red[w ^ 1][4 * lane]);
-    // per-half max of magnitude bits (non-NaN bf16 magnitudes order like
-    // unsigned 16-bit integers)
-    const uint32_t m2[4] = {__vmaxu2(mine.x, other.x), __vmaxu2(mine.y, other.y),
-                            __vmaxu2(mine.z, other.z), __vmaxu2(mine.w, other.w)};
-    float s[8];
+      for (int k = 0; k < kTileRowsPerWarp; ++k) {
+        acc[0] = absmax_acc(acc[0], v[k].x);
+        acc[1] = absmax_acc(acc[1], v[k].y);
+        acc[2] = absmax_acc(acc[2], v[k].z);
+        acc[3] = absmax_acc(acc[3], v[k].w);
+      }
+      *reinterpret_cast<uint4 *>(&sm.red[w][4 * lane]) =
+          make_uint4(absmax_bits(acc[0]), absmax_bits(acc[1]), absmax_bits(acc[2]),
+                     absmax_bits(acc[3]));
+      uint8_t *tile = sm.tile[i & 1];
+      // the store issued from this code tile two tiles ago has read it
+      if (tid == 0) bulk_wait_read<1>();
+      if (!consumers_and(got)) {
+        if (tid == 0) {
+          *abort = 1;
+          status_or(p.status, FP8QGG_STATUS_TIMEOUT);
+        }
+        break;
+      }
+      // the 32-token block of warps 2k, 2k+1: per-half max of the magnitude
+      // bits (non-NaN bf16 magnitudes order like unsigned 16-bit integers)
+      const uint4 mine = *reinterpret_cast<const uint4 *>(&sm.red[w][4 * lane]);
+      const uint4 other = *reinterpret_cast<const uint4 *>(&sm.red[w ^ 1][4 * lane]);
+      const uint32_t m2[4] = {__vmaxu2(mine.x, other.x), __vmaxu2(mine.y, other.y),
+                              __vmaxu2(mine.z, other.z), __vmaxu2(mine.w, other.w)};
+      float s[8];
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const uint32_t pair = m2[j >> 1];
-      const uint32_t m = (j & 1) ? (pair >> 16) : (pair & 0xFFFFu);
-      const int ex = mx_exponent(m);
-      s[j] = mx_multiplier(ex);
-      if (!(w & 1)) sb8[4 * (8 * lane + j) + (w >> 1)] = static_cast<uint8_t>(ex + 127);
+      for (int j = 0; j < 8; ++j) {
+        const uint32_t pair = m2[j >> 1];
+        const uint32_t m = (j & 1) ? (pair >> 16) : (pair & 0xFFFFu);
+        const int ex = mx_exponent(m);
+        s[j] = mx_multiplier(ex);
+        if (!(w & 1)) sb8[4 * (8 * lane + j) + (w >> 1)] = static_cast<uint8_t>(ex + 127);
+      }
+      uint32_t sat = 0;
+      tile_col_codes<FP8QGG_E4M3FN, true>(v, s, tile, w, lane, 0.f, 0.f, sat);
+      fence_proxy_async_smem();
+      consumers_sync();
+      const int32_t tok = sm.pstart[tl.e] + tl.b * kTileTokens;
+      if (tid == 0) {
+        tma_store_2d(&qmap, tile, tok, c0);
+        bulk_commit();
+      }
+      if (c0 + tid < p.cols)
+        p.sw[static_cast<int64_t>(tok / kTileTokens) * p.ld_sw + c0 + tid] = sm.sbytes[tid];
+      // sbytes and red are rewritten only after the next tile's first barrier
     }
-    uint32_t sat = 0;
-    tile_col_codes<FP8QGG_E4M3FN, true>(v, s, tile, w, lane, 0.f, 0.f, sat);
-    fence_proxy_async_smem();
-    __syncthreads();
-    const int32_t tok = sm.pstart[e] + b * kTileTokens;
-    if (tid == 0) {
-      tma_store_2d(&qmap, tile, tok, c0);
-      bulk_commit();
-    }
-    if (c0 + tid < p.cols) p.sw[static_cast<int64_t>(tok / kTileTokens) * p.ld_sw + c0 + tid] = sm.sbytes[tid];
+    if (tid == 0) bulk_wait_all();  // the code tiles stay valid until their stores have read them
   }
-  if (tid == 0) bulk_wait_all();  // the tiles stay valid until their stores have read them
 }
 
 }  // namespace fp8qgg
@@ -307,17 +412,16 @@ extern "C" int fp8_mx_quant_rowwise(const void *x, int64_t rows, int64_t cols, i
   prm.x = static_cast<const uint4 *>(x);
   prm.ld_x16 = ld_x / 8;
   prm.rows = rows;
-  prm.segs = (cols + 255) / 256;
   prm.cols = static_cast<int>(cols);
   prm.ngroups = static_cast<int>((cols + 127) / 128);
+  prm.units = (rows + kMxRowsPerWarp - 1) / kMxRowsPerWarp * prm.ngroups;
   prm.q = q;
   prm.ld_q = ld_q;
   prm.sw = scales;
   prm.ld_sw = ld_sw;
-  const int64_t warps = (rows * prm.segs + kMxRowUnroll - 1) / kMxRowUnroll;
-  const int64_t want = (warps + kMxRowThreads / 32 - 1) / (kMxRowThreads / 32);
+  const int64_t want = (prm.units + kMxRowThreads / 32 - 1) / (kMxRowThreads / 32);
   const int grid = static_cast<int>(
-      std::max<int64_t>(1, std::min<int64_t>(want, int64_t(dev.sm_count) * 8)));
+      std::max<int64_t>(1, std::min<int64_t>(want, int64_t(dev.sm_count) * 4)));
   mx_rowwise_kernel<<<grid, kMxRowThreads, 0, static_cast<cudaStream_t>(stream)>>>(prm);
   return cudaGetLastError() == cudaSuccess ? FP8QGG_OK : FP8QGG_ERR_CUDA;
 }
@@ -342,15 +446,25 @@ extern "C" int fp8_mx_quant_colwise_padded(const void *x, int64_t rows_total, in
   const int np = static_cast<int>((cols + kMxColWidth - 1) / kMxColWidth);
   const int64_t tiles = (rows_total / kTileTokens + num_groups) * int64_t(np);
   if (tiles > INT32_MAX / 2) return FP8QGG_ERR_SHAPE;
-  CUtensorMap qmap;
+  const int box_cols = static_cast<int>(std::min<int64_t>(kMxColWidth, cols));
+  CUtensorMap xmap, qmap;
+  memset(&xmap, 0, sizeof xmap);
   memset(&qmap, 0, sizeof qmap);
+  {
+    // input [rows_total][ld_x] bf16; boxes of 128 rows x 256 columns, no swizzle
+    const uint64_t dims[2] = {static_cast<uint64_t>(cols), static_cast<uint64_t>(rows_total)};
+    const uint64_t strides[1] = {static_cast<uint64_t>(ld_x) * 2};
+    const uint32_t box[2] = {static_cast<uint32_t>(box_cols), static_cast<uint32_t>(kTileTokens)};
+    if (!encode_tensor_map(&xmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(x), dims,
+                           strides, box, CU_TENSOR_MAP_SWIZZLE_NONE))
+      return FP8QGG_ERR_CUDA;
+  }
   {
     // codes [cols][ld_q tokens]; boxes of 128 tokens x 256 columns (fewer
     // columns when the tensor has fewer), 128-byte swizzle
     const uint64_t dims[2] = {static_cast<uint64_t>(ld_q), static_cast<uint64_t>(cols)};
     const uint64_t strides[1] = {static_cast<uint64_t>(ld_q)};
-    const uint32_t box[2] = {static_cast<uint32_t>(kTileTokens),
-                             static_cast<uint32_t>(std::min<int64_t>(kMxColWidth, cols))};
+    const uint32_t box[2] = {static_cast<uint32_t>(kTileTokens), static_cast<uint32_t>(box_cols)};
     if (!encode_tensor_map(&qmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, q, dims, strides, box,
                            CU_TENSOR_MAP_SWIZZLE_128B))
       return FP8QGG_ERR_CUDA;
@@ -361,18 +475,18 @@ extern "C" int fp8_mx_quant_colwise_padded(const void *x, int64_t rows_total, in
   if (!set_max_dynamic_smem(reinterpret_cast<const void *>(mx_colwise_kernel), smem))
     return FP8QGG_ERR_CUDA;
   MxColParams prm;
-  prm.x = static_cast<const uint4 *>(x);
-  prm.ld_x16 = ld_x / 8;
   prm.rows_total = rows_total;
   prm.cols = static_cast<int>(cols);
+  prm.box_cols = box_cols;
   prm.np = np;
   prm.offsets = offsets;
   prm.num_groups = num_groups;
   prm.sw = scales;
   prm.ld_sw = ld_sw;
   prm.status = dev_status;
-  const int grid = static_cast<int>(
-      std::max<int64_t>(1, std::min<int64_t>(tiles, int64_t(dev.sm_count) * 2)));
-  mx_colwise_kernel<<<grid, kMxColThreads, smem, static_cast<cudaStream_t>(stream)>>>(qmap, prm);
+  const int grid =
+      static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(tiles, int64_t(dev.sm_count))));
+  mx_colwise_kernel<<<grid, kMxColThreads, smem, static_cast<cudaStream_t>(stream)>>>(xmap, qmap,
+                                                                                     prm);
   return cudaGetLastError() == cudaSuccess ? FP8QGG_OK : FP8QGG_ERR_CUDA;
 }
