@@ -681,6 +681,7 @@ def run_gpu(args, world, rank, local):
 TRAFFIC = {
     "llama3_8b_up_proj": 269102336 + 422105344,     # grouped_gemm_2sm_kernel<0>
     "deepseek_moe16b_bwd": 389194752 + 680884992,   # grouped_gemm_kernel<1, 0>, padded operands
+    "deepseek_moe16b_bwd_mxfp8": 410045952 + 684758016,  # mx_grouped_gemm_kernel<1, 0>
 }
 
 
