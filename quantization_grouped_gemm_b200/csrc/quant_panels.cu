@@ -22,7 +22,8 @@
 //  - reads block s (HBM), reduces its column absmax (the warps meet in
 //    shared memory) and merges it into the unit's absmax words in global
 //    memory with relaxed atomic max, then counts it in the unit's arrival
-//    counter (the dual form also merges every row's absmax);
+//    counter with one release reduction by the first warp once every warp
+//    has merged (the dual form also merges every row's absmax);
 //  - reads block s - D again (from L2: D blocks ago is about one grid-width
 //    plus the longest unit, so the block is still there and its unit's count
 //    is normally full already; the block waits for it, bounded, otherwise),
@@ -209,7 +210,7 @@ __device__ PBlock decode_block(const PanelSmem &sm, int32_t a, int np, int lane)
   r.q = rr / nbi;
   r.b = rr - r.q * nbi;
   r.u = DUAL ? lo : lo * np + r.q;
-  r.need = kPWarps * (DUAL ? nbi * np : nbi);  // every warp of every block arrives
+  r.need = kPWarps * (DUAL ? nbi * np : nbi);  // each block of the unit adds kPWarps
   return r;
 }
 
@@ -360,10 +361,20 @@ __global__ void __launch_bounds__(kPThreads, kPBlocksPerSM)
       if (c0 + cc < p.cols)
         atomicMax(p.amax + static_cast<int64_t>(A.i) * p.cols + c0 + cc,
                   (lane & 1) ? m >> 16 : m & 0xFFFFu);
-      // the lanes' merges happen before lane 0's release of the count
+      // every warp's merges happen before warp 0's one release of the count
+      // (a named barrier: the other warps arrive without waiting and go on to
+      // the cast; the release orders their merges too, being cumulative over
+      // the barrier)
       __syncwarp();
-      if (lane == 0)
-        asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(p.arrive + A.u) : "memory");
+      if (w != 0) {
+        asm volatile("bar.arrive 2, %0;" ::"n"(kPThreads) : "memory");
+      } else {
+        asm volatile("bar.sync 2, %0;" ::"n"(kPThreads) : "memory");
+        if (lane == 0)
+          asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p.arrive + A.u),
+                       "n"(kPWarps)
+                       : "memory");
+      }
     }
 
     // ---------------------------------------------------------- cast of block s - D
