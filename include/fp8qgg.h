@@ -400,9 +400,18 @@ int fp8_mx_quant_colwise_padded(const void *x, int64_t rows_total, int64_t cols,
  *   b        B_e[n, k] at b[e*b_group_stride + n*ld_b + k]; scale_b word
  *            (g, e, n) at scale_b[g * ld_sb + e * scale_b_group_stride + n]
  *            (B quantised as one [E*N, K] matrix: scale_b_group_stride = n).
+ *            The experts' matrices may be stacked (b_group_stride >= n*ld_b,
+ *            ld_b >= k) or interleaved in the rows of one matrix (ld_b >=
+ *            (E-1)*b_group_stride + k, b_group_stride >= k): the input
+ *            gradient's B = W_e^T as fp8_mx_quant_colwise_padded writes it for
+ *            W viewed [E*N, K] with groups of N rows (N % 128 == 0), where
+ *            b_group_stride = N, ld_b = ld_q, and the scale words of expert e
+ *            start at group e*N/128 (scale_b_group_stride = (N/128)*ld_sb).
+ *            Their scale words: stacked (scale_b_group_stride >= n, ld_sb >=
+ *            (E-1)*scale_b_group_stride + n) or in per-expert blocks (ld_sb >=
+ *            n, scale_b_group_stride >= ceil(k/128) * ld_sb).
  *   out      [m_total, ld_out]; rows outside every group are not written.
- *   Requirements: k % 32 == 0; scale_b_group_stride >= n;
- *   ld_sb >= (num_groups - 1) * scale_b_group_stride + n.
+ *   Requirements: k % 32 == 0; ld_sa >= m_total.
  * mode FP8QGG_K_JAGGED_PADDED (weight gradient, outputs of
  * fp8_mx_quant_colwise_padded):
  *   out[e, i, j] = sum_{t < size_e} value_a[i, P_e + t] * value_b[j, P_e + t]

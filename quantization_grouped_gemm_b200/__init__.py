@@ -464,5 +464,41 @@ class Fp8WeightCache:
         self._entries[key] = (ver, q, s)
         return q, s
 
+    def mx_rowwise(self, w):
+        """(q, scales) of fp8_mx_quant_rowwise(w) (MXFP8, the forward's B),
+        reused while w is unchanged."""
+        q_fn = self._quantize or fp8_mx_quant_rowwise
+        key = self._key(w, "mx_rowwise", ())
+        ent = self._entries.get(key)
+        if ent is not None and ent[0] == w._version:
+            self.hits += 1
+            return ent[1], ent[2]
+        self.misses += 1
+        if ent is None:
+            q, s = q_fn(w)
+        else:
+            q, s = q_fn(w, q=ent[1], scales=ent[2])
+        self._entries[key] = (w._version, q, s)
+        return q, s
+
+    def mx_colwise_padded(self, w, offsets):
+        """(q, scales) of fp8_mx_quant_colwise_padded(w, offsets) (MXFP8,
+        W^T for the input gradient with groups of each expert's rows), reused
+        while w and offsets are unchanged."""
+        q_fn = self._quantize or fp8_mx_quant_colwise_padded
+        key = self._key(w, "mx_colwise", (offsets.data_ptr(), offsets.numel()))
+        ent = self._entries.get(key)
+        ver = (w._version, offsets._version)
+        if ent is not None and ent[0] == ver:
+            self.hits += 1
+            return ent[1], ent[2]
+        self.misses += 1
+        if ent is None:
+            q, s = q_fn(w, offsets)
+        else:
+            q, s = q_fn(w, offsets, q=ent[1], scales=ent[2])
+        self._entries[key] = (ver, q, s)
+        return q, s
+
     def clear(self):
         self._entries.clear()

@@ -91,6 +91,7 @@ struct MxGemmParams {
   int num_groups;
   int64_t m_total, n, k;
   int bn;
+  int b_inter;  // token-jagged: B's experts interleaved in its rows (map dims k, expert, row)
   void *out;
   int64_t ld_out;
   int64_t out_gs;
@@ -339,7 +340,10 @@ __global__ void __launch_bounds__(kMxGemmThreads, 1)
           mbar_arrive_expect_tx(&sm.full[stage], stage_bytes);
           if constexpr (MODE == FP8QGG_M_JAGGED) {
             tma_load_2d(sm.a[stage], &amap, &sm.full[stage], ka, ti.gstart + ti.tm * kMxBM);
-            tma_load_3d(sm.b[stage], &bmap, &sm.full[stage], ka, ti.tn * bn, ti.e);
+            if (p.b_inter)
+              tma_load_3d(sm.b[stage], &bmap, &sm.full[stage], ka, ti.e, ti.tn * bn);
+            else
+              tma_load_3d(sm.b[stage], &bmap, &sm.full[stage], ka, ti.tn * bn, ti.e);
           } else {
             tma_load_2d(sm.a[stage], &amap, &sm.full[stage], ka, ti.tm * kMxBM);
             tma_load_2d(sm.b[stage], &bmap, &sm.full[stage], ka, ti.tn * bn);
@@ -582,13 +586,27 @@ extern "C" int fp8_mx_grouped_gemm(int mode, const uint8_t *a, int64_t ld_a,
   if (n > INT32_MAX / 2 || k > INT32_MAX / 2) return FP8QGG_ERR_SHAPE;
   const int vec = out_dtype == FP8QGG_OUT_F32 ? 4 : 8;
   const int64_t ocols = kmode == FP8QGG_M_JAGGED ? n : k;
+  bool interleaved = false;
   if (kmode == FP8QGG_M_JAGGED) {
     if (k % 32) return FP8QGG_ERR_SHAPE;
-    if (ld_a < k || ld_b < k || ld_out < n || ld_sa < m_total) return FP8QGG_ERR_SHAPE;
-    if (num_groups > 1 && (b_group_stride < n * ld_b || scale_b_group_stride < n))
-      return FP8QGG_ERR_SHAPE;
-    const int64_t brows = (num_groups > 1 ? (num_groups - 1) * scale_b_group_stride : 0) + n;
-    if (ld_sb < brows) return FP8QGG_ERR_SHAPE;
+    if (ld_a < k || ld_out < n || ld_sa < m_total) return FP8QGG_ERR_SHAPE;
+    // the experts' B matrices may be stacked (B_e after B_{e-1}) or
+    // interleaved (row i of every B_e in row i of one matrix, as the
+    // column-wise quantisation of W writes W^T); either way they must not
+    // overlap
+    const int64_t E = num_groups;
+    const bool b_stacked = ld_b >= k && (E == 1 || b_group_stride >= n * ld_b);
+    const bool b_inter = E > 1 && b_group_stride >= k && ld_b >= (E - 1) * b_group_stride + k;
+    if (!b_stacked && !b_inter) return FP8QGG_ERR_SHAPE;
+    interleaved = !b_stacked;
+    // scale words likewise: the experts' rows stacked within a 128-column
+    // group, or each expert's groups in a block of its own
+    const int64_t kgroups = (k + kMxBK - 1) / kMxBK;
+    const bool s_stacked = E == 1 ? ld_sb >= n
+                                  : scale_b_group_stride >= n &&
+                                        ld_sb >= (E - 1) * scale_b_group_stride + n;
+    const bool s_blocked = E > 1 && ld_sb >= n && scale_b_group_stride >= kgroups * ld_sb;
+    if (!s_stacked && !s_blocked) return FP8QGG_ERR_SHAPE;
   } else {
     const int64_t tok = m_total + int64_t(kMxBK) * num_groups;
     if (tok > INT32_MAX / 2) return FP8QGG_ERR_SHAPE;
@@ -612,11 +630,18 @@ extern "C" int fp8_mx_grouped_gemm(int mode, const uint8_t *a, int64_t ld_a,
   if (kmode == FP8QGG_M_JAGGED) {
     const uint64_t adims[2] = {static_cast<uint64_t>(k), static_cast<uint64_t>(m_total)};
     const uint64_t astr[1] = {static_cast<uint64_t>(ld_a)};
-    const uint64_t bdims[3] = {static_cast<uint64_t>(k), static_cast<uint64_t>(n),
-                               static_cast<uint64_t>(num_groups)};
-    const uint64_t bstr[2] = {static_cast<uint64_t>(ld_b),
-                              static_cast<uint64_t>(num_groups > 1 ? b_group_stride : n * ld_b)};
-    const uint32_t bbox[3] = {kMxBK, static_cast<uint32_t>(bn), 1};
+    // stacked experts: dims (k, row, expert); interleaved: (k, expert, row),
+    // so that the strides grow with the dimension either way
+    const uint64_t bdims[3] = {
+        static_cast<uint64_t>(k),
+        static_cast<uint64_t>(interleaved ? num_groups : n),
+        static_cast<uint64_t>(interleaved ? n : num_groups)};
+    const uint64_t bstr[2] = {
+        static_cast<uint64_t>(interleaved ? b_group_stride : ld_b),
+        static_cast<uint64_t>(interleaved ? ld_b
+                                          : (num_groups > 1 ? b_group_stride : n * ld_b))};
+    const uint32_t bbox[3] = {kMxBK, interleaved ? 1u : static_cast<uint32_t>(bn),
+                              interleaved ? static_cast<uint32_t>(bn) : 1u};
     if (!encode_tensor_map(&amap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t *>(a),
                            adims, astr, abox, CU_TENSOR_MAP_SWIZZLE_128B) ||
         !encode_tensor_map(&bmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<uint8_t *>(b),
@@ -673,6 +698,7 @@ extern "C" int fp8_mx_grouped_gemm(int mode, const uint8_t *a, int64_t ld_a,
   prm.n = n;
   prm.k = k;
   prm.bn = bn;
+  prm.b_inter = interleaved ? 1 : 0;
   prm.out = out;
   prm.ld_out = ld_out;
   prm.out_gs = out_group_stride;

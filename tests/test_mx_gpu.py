@@ -236,3 +236,36 @@ def test_mx_gemm_k_jagged_padded_every_element(sizes, n1, n2):
 
 def test_mx_gemm_k_jagged_padded_bf16_output():
     check_k_jagged([100, 0, 257], 64, 128, out_dtype=torch.bfloat16)
+
+
+@pytest.mark.parametrize("sizes,n_w,k_w", [([70, 0, 200], 256, 192), ([33, 300], 128, 96)])
+def test_mx_input_gradient_path(sizes, n_w, k_w):
+    """dX = grad_out W_e in MXFP8: grad_out quantised along its N columns
+    (rowwise), W [E*N, K] quantised along each expert's N rows by the
+    column-wise kernel with groups of N rows (W_e^T codes, experts side by
+    side in every row, scale words of expert e from group e*N/128), then the
+    token-jagged block-scaled GEMM with B interleaved."""
+    e = len(sizes)
+    m = int(sum(sizes))
+    go = spread_bf16(17 + m, (m, n_w), spread=8.0)
+    wt = spread_bf16(19 + m, (e * n_w, k_w), block_axis=0, spread=8.0)
+    off = wl.offsets_from_sizes(sizes)
+    off_w = wl.offsets_from_sizes([n_w] * e)
+    qg, sg = qgg.fp8_mx_quant_rowwise(go.cuda())
+    qwt, swt = qgg.fp8_mx_quant_colwise_padded(wt.cuda(), torch.from_numpy(off_w).cuda())
+    ld_q = qwt.shape[1]
+    b = qwt.as_strided((e, k_w, n_w), (n_w, ld_q, 1))
+    out = torch.full((m, k_w), float("nan"), device="cuda")
+    qgg.fp8_mx_grouped_gemm(qgg.M_JAGGED, qg, sg, b, swt, torch.from_numpy(off).cuda(), out=out,
+                            scale_b_group_stride=(n_w // 128) * swt.stride(0))
+    torch.cuda.synchronize()
+    oqg, osg = orc.mx_quant_rowwise(bits(go))
+    oqw, osw = orc.mx_quant_colwise_padded(bits(wt), off_w)
+    qb = np.stack([oqw[:, i * n_w:(i + 1) * n_w] for i in range(e)])               # [E, K, N]
+    sb = np.stack([osw[:, i * n_w // 32:(i + 1) * n_w // 32] for i in range(e)])   # [E, K, N/32]
+    rows = np.repeat(np.arange(m), k_w)
+    cols = np.tile(np.arange(k_w), m)
+    ref, bound = orc.mx_gemm_m_jagged_sample(oqg, osg, qb, sb, off, rows, cols)
+    got = out.cpu().numpy()[rows, cols].astype(np.float64)
+    err = np.abs(got - ref)
+    assert (err <= bound).all(), (err.max(), np.argmax(err - bound))

@@ -50,3 +50,45 @@ def test_cached_codes_are_reused_and_refreshed_after_an_update():
     ref_q3, ref_s3, _ = orc.quant_rowwise(wl.bf16_bits(w.cpu()))
     assert (q3.cpu().numpy() == ref_q3).all()
     assert (s3.cpu().numpy().view(np.uint32) == ref_s3.view(np.uint32)).all()
+
+
+def test_mx_cache_decides_on_version_without_a_gpu():
+    calls = []
+
+    def fake(w, *rest, q=None, scales=None):
+        calls.append(w._version)
+        return (q if q is not None else torch.zeros(w.shape, dtype=torch.uint8),
+                scales if scales is not None else torch.zeros(1, dtype=torch.int32))
+
+    c = qgg.Fp8WeightCache(quantize=fake)
+    w = torch.ones(4, 64, dtype=torch.bfloat16)
+    off = torch.tensor([2, 4], dtype=torch.int32)
+    q1, _ = c.mx_rowwise(w)
+    assert c.mx_rowwise(w)[0] is q1 and len(calls) == 1
+    c.mx_colwise_padded(w, off)
+    c.mx_colwise_padded(w, off)
+    assert len(calls) == 2 and c.hits == 2
+    w.add_(1)
+    assert c.mx_rowwise(w)[0] is q1 and len(calls) == 3
+    off.add_(0)  # the offsets' in-place version counts too
+    c.mx_colwise_padded(w, off)
+    assert len(calls) == 4
+
+
+@pytest.mark.gpu
+def test_mx_cached_codes_match_the_oracle_and_refresh():
+    w = wl.normal_bf16(78, 2, (2 * 128, 96), 0.02).cuda()
+    c = qgg.Fp8WeightCache()
+    q, s = c.mx_rowwise(w)
+    torch.cuda.synchronize()
+    ref_q, ref_s = orc.mx_quant_rowwise(wl.bf16_bits(w.cpu()))
+    assert (q.cpu().numpy() == ref_q).all()
+    assert (qgg.mx_scales_to_blocks(s, 3).cpu().numpy() == ref_s).all()
+    q.fill_(0xAB)
+    assert (c.mx_rowwise(w)[0] == 0xAB).all()
+    w.mul_(5)
+    q2, s2 = c.mx_rowwise(w)
+    torch.cuda.synchronize()
+    ref_q2, ref_s2 = orc.mx_quant_rowwise(wl.bf16_bits(w.cpu()))
+    assert (q2.cpu().numpy() == ref_q2).all()
+    assert (qgg.mx_scales_to_blocks(s2, 3).cpu().numpy() == ref_s2).all()
