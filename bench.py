@@ -221,6 +221,8 @@ def config_dict(w, Step=None):
         d.update(N=(w.grad_out if w.grad_out is not None and Step.BACKWARD else w.w).shape[1],
                  step=Step.STEP, fmt=Step.FMT)
         d.update(workload=w.name + "_mxfp8")
+        if Step.__name__ == "MxDualCompareStep":
+            d.update(K=None, gemm_out=None)
     elif Step is not None and Step.__name__ == "DualCompareStep":
         d.update(K=None, N=w.grad_out.shape[1], gemm_out=None,
                  step=("grad_out quantised for both backward GEMMs: rowwise + padded transposed "
@@ -471,6 +473,56 @@ class MxBackwardDwStep:
         ]
 
 
+
+class MxDualCompareStep:
+    """The MXFP8 backward quantisation of grad_out [M, N] for both backward
+    GEMMs: the MX rowwise call and the MX padded column-wise call, then the
+    dual-output call that writes both from one read."""
+    STEP = ("grad_out quantised in MXFP8 for both backward GEMMs: MX rowwise + MX padded "
+            "column-wise as two calls, then as one dual-output call")
+    FMT = "mxfp8 (e4m3fn elements, E8M0 scales per 32 elements)"
+    BACKWARD = True
+
+    def __init__(self, w):
+        import quantization_grouped_gemm_b200 as qgg
+        self.qgg = qgg
+        self.w = w
+        m, n = w.grad_out.shape
+        e = w.num_groups
+        self.m, self.n, self.e = m, n, e
+        self.g = w.grad_out.cuda()
+        self.off = torch.from_numpy(w.offsets).cuda()
+        ld = (m + 128 * e + 127) // 128 * 128
+        gn = qgg.mx_scale_groups(n)
+        self.qr = torch.empty((m, n), dtype=torch.uint8, device="cuda")
+        self.sr = torch.empty((gn, m), dtype=torch.int32, device="cuda")
+        self.qc = torch.empty((n, ld), dtype=torch.uint8, device="cuda")
+        self.sc = torch.empty((ld // 128, n), dtype=torch.int32, device="cuda")
+        self.qr2 = torch.empty_like(self.qr)
+        self.sr2 = torch.empty_like(self.sr)
+        self.qc2 = torch.empty_like(self.qc)
+        self.sc2 = torch.empty_like(self.sc)
+        self.flops = 0.0
+        self.names = ["mx_quant_rowwise_grad_out", "mx_quant_colwise_t_grad_out",
+                      "mx_quant_dual_grad_out"]
+        self.launches = 3
+        one = m * n * 3 + m * n // 32
+        self.bytes = [one, one, m * n * 4 + 2 * (m * n // 32)]
+        self.host_inputs = [(self.g, w.grad_out)]
+        self.input_bytes = 2 * m * n
+        self.result = self.qc2
+
+    def kernels(self):
+        q = self.qgg
+        return [
+            lambda: q.fp8_mx_quant_rowwise(self.g, q=self.qr, scales=self.sr),
+            lambda: q.fp8_mx_quant_colwise_padded(self.g, self.off, q=self.qc, scales=self.sc),
+            lambda: q.fp8_mx_quant_dual_padded(self.g, self.off, q_row=self.qr2,
+                                               scales_row=self.sr2, q_col=self.qc2,
+                                               scales_col=self.sc2),
+        ]
+
+
 WORKLOADS = {
     "llama3_8b_up_proj": (lambda: wl.llama3_8b_up_proj(), ForwardStep),
     "tiny_moe": (lambda: wl.tiny_moe(), ForwardStep),
@@ -482,6 +534,8 @@ WORKLOADS = {
     "llama4_m131072_uniform": (lambda: wl.llama4_sweep(131072, "uniform"), ForwardStep),
     "llama3_8b_up_proj_mxfp8": (lambda: wl.llama3_8b_up_proj(), MxForwardStep),
     "deepseek_moe16b_bwd_mxfp8": (lambda: wl.deepseek_moe_16b_backward(), MxBackwardDwStep),
+    "deepseek_moe16b_bwd_dual_mxfp8": (lambda: wl.deepseek_moe_16b_backward(with_x=False),
+                                       MxDualCompareStep),
 }
 
 
@@ -573,7 +627,8 @@ def extra_workload(name, steps, warmup, pk):
 # layer (launch-bound), the DeepSeek-MoE-16B backward weight-gradient step,
 # the dual-output comparison, and the MXFP8 forward and weight-gradient steps.
 EXTRA_WORKLOADS = ("tiny_moe", "deepseek_moe16b_bwd", "deepseek_moe16b_bwd_dual",
-                   "llama3_8b_up_proj_mxfp8", "deepseek_moe16b_bwd_mxfp8")
+                   "llama3_8b_up_proj_mxfp8", "deepseek_moe16b_bwd_mxfp8",
+                   "deepseek_moe16b_bwd_dual_mxfp8")
 
 
 def run_gpu(args, world, rank, local):

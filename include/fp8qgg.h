@@ -390,6 +390,30 @@ int fp8_mx_quant_colwise_padded(const void *x, int64_t rows_total, int64_t cols,
                                 int32_t *dev_status, void *stream);
 
 /*
+ * Dual-output MX quantisation for the backward pass: ONE read of x gives the
+ * MX rowwise quantisation of every row of the groups (blocks along the
+ * columns, for the input-gradient GEMM) and the MX column-wise quantisation
+ * in the padded transposed layout (blocks along each group's tokens, for the
+ * weight-gradient GEMM): the codes and scale words of
+ * fp8_mx_quant_rowwise on each grouped row and of
+ * fp8_mx_quant_colwise_padded, bit for bit ([AIR] "Il guadagno vero è nel
+ * movimento dei dati", second paragraph: the backward's quantisations fused;
+ * [PRI] "What Primus adds…": MXFP8 kernels).  Rows past the last group end
+ * are not written.
+ *   q_row      uint8 [rows_total, ld_qr], ld_qr >= cols, ld_qr % 8 == 0,
+ *              8-byte aligned.
+ *   scales_row uint32 [cols / 128 rounded up, ld_swr], ld_swr >= rows_total.
+ *   q_col, scales_col, ld_qc, ld_swc: as q, scales, ld_q, ld_sw of
+ *              fp8_mx_quant_colwise_padded.
+ * Requirements: those of fp8_mx_quant_colwise_padded, plus cols % 32 == 0.
+ */
+int fp8_mx_quant_dual_padded(const void *x, int64_t rows_total, int64_t cols, int64_t ld_x,
+                             const int32_t *offsets, int32_t num_groups,
+                             uint8_t *q_row, int64_t ld_qr, uint32_t *scales_row, int64_t ld_swr,
+                             uint8_t *q_col, int64_t ld_qc, uint32_t *scales_col, int64_t ld_swc,
+                             int32_t *dev_status, void *stream);
+
+/*
  * MXFP8 grouped GEMM: block-scaled tensor-core products (each 32-element
  * block's partial sum times 2^(Ea + Eb)), fp32 accumulation.  Scales in the
  * packed layout above (ld_sa, ld_sb: words per 128-element group).

@@ -60,6 +60,8 @@ _SIGNATURES = {
                                            _P, _P]),
     "fp8_mx_grouped_gemm": (_INT, [_INT, _P, _I64, _P, _I64, _P, _I64, _I64, _P, _I64, _I64, _P,
                                    _I32, _I64, _I64, _I64, _P, _I64, _I64, _INT, _P, _P]),
+    "fp8_mx_quant_dual_padded": (_INT, [_P, _I64, _I64, _I64, _P, _I32, _P, _I64, _P, _I64, _P,
+                                        _I64, _P, _I64, _P, _P]),
 }
 
 
@@ -348,6 +350,38 @@ def fp8_mx_quant_colwise_padded(x, offsets, q=None, ld_q=None, scales=None, stat
                                            _ptr(status), _stream(stream))
     _check(rc, "fp8_mx_quant_colwise_padded")
     return q, scales
+
+
+def fp8_mx_quant_dual_padded(x, offsets, q_row=None, scales_row=None, q_col=None, ld_qc=None,
+                             scales_col=None, status=None, stream=None):
+    """One read of a bf16 [rows_total, cols] CUDA tensor (cols % 32 == 0) gives
+    its MX rowwise quantisation (rows of the groups) and its MX column-wise
+    quantisation in the padded transposed layout.
+
+    Returns (q_row [rows_total, cols], scales_row int32 [cols/128, rows_total],
+    q_col [cols, ld_qc], scales_col int32 [ld_qc/128, cols])."""
+    _need_cuda(x, offsets)
+    assert x.dtype == torch.bfloat16 and x.dim() == 2 and offsets.dtype == torch.int32
+    rows, cols = x.shape
+    e = offsets.numel()
+    if q_row is None:
+        q_row = torch.empty((rows, cols), dtype=torch.uint8, device=x.device)
+    if scales_row is None:
+        scales_row = torch.empty((mx_scale_groups(cols), rows), dtype=torch.int32,
+                                 device=x.device)
+    if q_col is None:
+        ld = ld_qc if ld_qc is not None else (rows + 128 * e + 127) // 128 * 128
+        q_col = torch.empty((cols, ld), dtype=torch.uint8, device=x.device)
+    if scales_col is None:
+        scales_col = torch.empty((mx_scale_groups(q_col.shape[1]), cols), dtype=torch.int32,
+                                 device=x.device)
+    _need_cuda(q_row, scales_row, q_col, scales_col, status)
+    rc = lib().fp8_mx_quant_dual_padded(
+        _ptr(x), rows, cols, _ld(x), _ptr(offsets), e, _ptr(q_row), _ld(q_row), _ptr(scales_row),
+        _ld(scales_row), _ptr(q_col), _ld(q_col), _ptr(scales_col), _ld(scales_col),
+        _ptr(status), _stream(stream))
+    _check(rc, "fp8_mx_quant_dual_padded")
+    return q_row, scales_row, q_col, scales_col
 
 
 def fp8_mx_grouped_gemm(mode, a, scale_a, b, scale_b, offsets, m_total=None, n=None, k=None,

@@ -166,6 +166,7 @@ struct MxColSmem {
   uint8_t tile[2][kMxTileBytes];           // transposed code tiles
   uint32_t red[kMxColWarps][kMxColWidth / 2];  // per-warp column absmax (bf16 pairs)
   uint32_t sbytes[kMxColWidth];            // per column: the tile's scale word
+  uint32_t rowsb[kMxColWarps][2 * kTileRowsPerWarp];  // dual form: row scale bytes of a warp
   int32_t start[kMxMaxGroups];
   int32_t end[kMxMaxGroups];
   int32_t pstart[kMxMaxGroups];
@@ -185,6 +186,11 @@ struct MxColParams {
   uint32_t *sw;  // scale words [tokens / 128, ld_sw]
   int64_t ld_sw;
   int32_t *status;
+  // dual form: rowwise codes [rows_total, ld_qr] and scale words [cols / 128, ld_swr]
+  uint8_t *q_row;
+  int64_t ld_qr;
+  uint32_t *swr;
+  int64_t ld_swr;
 };
 
 struct MxColTile {
@@ -226,6 +232,9 @@ __device__ __forceinline__ void consumers_sync() {
   asm volatile("bar.sync 1, %0;" ::"n"(kMxColConsumers) : "memory");
 }
 
+// One thread block of nine warps per SM: a sub-partition holds three of them,
+// which caps a thread at 168 registers.
+template <bool DUAL>
 __global__ void __launch_bounds__(kMxColThreads, 1)
     mx_colwise_kernel(const __grid_constant__ CUtensorMap xmap,
                       const __grid_constant__ CUtensorMap qmap, const MxColParams p) {
@@ -338,8 +347,10 @@ __global__ void __launch_bounds__(kMxColThreads, 1)
       for (int k = 0; k < kTileRowsPerWarp; ++k)
         v[k] = (got && c_ok && rw0 + k < r1) ? *reinterpret_cast<const uint4 *>(src + k * row_bytes)
                                              : make_uint4(0u, 0u, 0u, 0u);
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&sm.empty[st]);  // the stage may be refilled
+      if constexpr (!DUAL) {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.empty[st]);  // the stage may be refilled
+      }
       uint32_t acc[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
       for (int k = 0; k < kTileRowsPerWarp; ++k) {
@@ -379,6 +390,40 @@ __global__ void __launch_bounds__(kMxColThreads, 1)
       uint32_t sat = 0;
       tile_col_codes<FP8QGG_E4M3FN, true>(v, s, tile, w, lane, 0.f, 0.f, sat);
       fence_proxy_async_smem();
+      if constexpr (DUAL) {
+        // the rowwise MX quantisation of the same rows, re-read from the
+        // stage (the column-wise registers are free now): a 32-column block is
+        // four lanes; the row's scale word of a 128-column group (lanes
+        // 16h .. 16h + 15) is gathered by four shuffles, and lane 16h + j
+        // keeps the word of row rw0 + j for one coalesced store
+        // block scale bytes [16 rows][8 blocks] of the warp; a lane's row word
+        // is then one 4-byte read
+        uint8_t *rb = reinterpret_cast<uint8_t *>(&sm.rowsb[w][0]);
+#pragma unroll
+        for (int k = 0; k < kTileRowsPerWarp; ++k) {
+          const uint4 vk = (c_ok && rw0 + k < r1)
+                               ? *reinterpret_cast<const uint4 *>(src + k * row_bytes)
+                               : make_uint4(0u, 0u, 0u, 0u);
+          uint32_t m = absmax8(vk);
+          m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
+          m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
+          const int ex = mx_exponent(m);
+          const uint2 c = mx_encode8(vk, mx_multiplier(ex));
+          if (c_ok && rw0 + k < r1)
+            __stcs(reinterpret_cast<uint2 *>(p.q_row + static_cast<int64_t>(rw0 + k) * p.ld_qr +
+                                             c0 + 8 * lane),
+                   c);
+          if ((lane & 3) == 0) rb[8 * k + (lane >> 2)] = static_cast<uint8_t>(ex + 127);
+        }
+        __syncwarp();
+        // lane 16h + j: row rw0 + j, blocks 4h .. 4h + 3 (the 128-column group 2q + h)
+        const uint32_t myword = sm.rowsb[w][2 * (lane & 15) + (lane >> 4)];
+        const int g = 2 * tl.q + (lane >> 4);
+        if (rw0 + (lane & 15) < r1 && 128 * g < p.cols)
+          p.swr[static_cast<int64_t>(g) * p.ld_swr + rw0 + (lane & 15)] = myword;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.empty[st]);  // the stage may be refilled
+      }
       consumers_sync();
       const int32_t tok = sm.pstart[tl.e] + tl.b * kTileTokens;
       if (tid == 0) {
@@ -426,21 +471,27 @@ extern "C" int fp8_mx_quant_rowwise(const void *x, int64_t rows, int64_t cols, i
   return cudaGetLastError() == cudaSuccess ? FP8QGG_OK : FP8QGG_ERR_CUDA;
 }
 
-extern "C" int fp8_mx_quant_colwise_padded(const void *x, int64_t rows_total, int64_t cols,
-                                           int64_t ld_x, const int32_t *offsets,
-                                           int32_t num_groups, uint8_t *q, int64_t ld_q,
-                                           uint32_t *scales, int64_t ld_sw, int32_t *dev_status,
-                                           void *stream) {
+namespace fp8qgg {
+
+// Checks and launch shared by the column-wise MX call and its dual form
+// (q_row non-null).
+int mx_colwise_launch(const void *x, int64_t rows_total, int64_t cols, int64_t ld_x,
+                      const int32_t *offsets, int32_t num_groups, uint8_t *q, int64_t ld_q,
+                      uint32_t *scales, int64_t ld_sw, uint8_t *q_row, int64_t ld_qr,
+                      uint32_t *scales_row, int64_t ld_swr, int32_t *dev_status, void *stream) {
+  const bool dual = q_row != nullptr;
   if (rows_total < 0 || cols < 1 || cols > INT32_MAX / 2 || ld_x < cols) return FP8QGG_ERR_SHAPE;
   if (num_groups < 1 || num_groups > kMxMaxGroups) return FP8QGG_ERR_SHAPE;
   const int64_t tokens = rows_total + int64_t(kTileTokens) * num_groups;
   if (tokens > INT32_MAX / 2 || ld_q < tokens || ld_sw < cols) return FP8QGG_ERR_SHAPE;
-  if (!offsets || !scales) return FP8QGG_ERR_NULL;
+  if (dual && (cols % 32 || ld_qr < cols || ld_swr < rows_total)) return FP8QGG_ERR_SHAPE;
+  if (!offsets || !scales || (dual && !scales_row)) return FP8QGG_ERR_NULL;
   if (rows_total > 0 && (!x || !q)) return FP8QGG_ERR_NULL;
   if (cols % 8 || ld_x % 8 || ld_q % 16) return FP8QGG_ERR_ALIGN;
   if ((x && !aligned(x, 16)) || (q && !aligned(q, 16)) || !aligned(scales, 4) ||
       !aligned(offsets, 4))
     return FP8QGG_ERR_ALIGN;
+  if (dual && (!aligned(q_row, 8) || ld_qr % 8 || !aligned(scales_row, 4))) return FP8QGG_ERR_ALIGN;
   if (dev_status && !aligned(dev_status, 4)) return FP8QGG_ERR_ALIGN;
   if (rows_total == 0) return FP8QGG_OK;  // every group is empty: nothing is written
   const int np = static_cast<int>((cols + kMxColWidth - 1) / kMxColWidth);
@@ -471,9 +522,9 @@ extern "C" int fp8_mx_quant_colwise_padded(const void *x, int64_t rows_total, in
   }
   DeviceInfo dev;
   if (!device_info(&dev)) return FP8QGG_ERR_CUDA;
+  auto kern = dual ? mx_colwise_kernel<true> : mx_colwise_kernel<false>;
   const int smem = static_cast<int>(sizeof(MxColSmem)) + 1024;
-  if (!set_max_dynamic_smem(reinterpret_cast<const void *>(mx_colwise_kernel), smem))
-    return FP8QGG_ERR_CUDA;
+  if (!set_max_dynamic_smem(reinterpret_cast<const void *>(kern), smem)) return FP8QGG_ERR_CUDA;
   MxColParams prm;
   prm.rows_total = rows_total;
   prm.cols = static_cast<int>(cols);
@@ -484,9 +535,35 @@ extern "C" int fp8_mx_quant_colwise_padded(const void *x, int64_t rows_total, in
   prm.sw = scales;
   prm.ld_sw = ld_sw;
   prm.status = dev_status;
+  prm.q_row = q_row;
+  prm.ld_qr = ld_qr;
+  prm.swr = scales_row;
+  prm.ld_swr = ld_swr;
   const int grid =
       static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(tiles, int64_t(dev.sm_count))));
-  mx_colwise_kernel<<<grid, kMxColThreads, smem, static_cast<cudaStream_t>(stream)>>>(xmap, qmap,
-                                                                                     prm);
+  kern<<<grid, kMxColThreads, smem, static_cast<cudaStream_t>(stream)>>>(xmap, qmap, prm);
   return cudaGetLastError() == cudaSuccess ? FP8QGG_OK : FP8QGG_ERR_CUDA;
+}
+
+}  // namespace fp8qgg
+
+extern "C" int fp8_mx_quant_colwise_padded(const void *x, int64_t rows_total, int64_t cols,
+                                           int64_t ld_x, const int32_t *offsets,
+                                           int32_t num_groups, uint8_t *q, int64_t ld_q,
+                                           uint32_t *scales, int64_t ld_sw, int32_t *dev_status,
+                                           void *stream) {
+  return mx_colwise_launch(x, rows_total, cols, ld_x, offsets, num_groups, q, ld_q, scales, ld_sw,
+                           nullptr, 0, nullptr, 0, dev_status, stream);
+}
+
+extern "C" int fp8_mx_quant_dual_padded(const void *x, int64_t rows_total, int64_t cols,
+                                        int64_t ld_x, const int32_t *offsets, int32_t num_groups,
+                                        uint8_t *q_row, int64_t ld_qr, uint32_t *scales_row,
+                                        int64_t ld_swr, uint8_t *q_col, int64_t ld_qc,
+                                        uint32_t *scales_col, int64_t ld_swc, int32_t *dev_status,
+                                        void *stream) {
+  if (!q_row) return FP8QGG_ERR_NULL;
+  return mx_colwise_launch(x, rows_total, cols, ld_x, offsets, num_groups, q_col, ld_qc,
+                           scales_col, ld_swc, q_row, ld_qr, scales_row, ld_swr, dev_status,
+                           stream);
 }

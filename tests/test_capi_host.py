@@ -199,6 +199,7 @@ def test_binding_refuses_host_tensors_instead_of_computing_on_the_cpu():
         lambda: qgg.fp8_cast_f32(torch.zeros(8)),
         lambda: qgg.fp8_mx_quant_rowwise(torch.zeros((4, 32), dtype=torch.bfloat16)),
         lambda: qgg.fp8_mx_quant_colwise_padded(x, off),
+        lambda: qgg.fp8_mx_quant_dual_padded(torch.zeros((4, 32), dtype=torch.bfloat16), off),
         lambda: qgg.fp8_mx_grouped_gemm(qgg.M_JAGGED, q8, q8, q8.view(1, 4, 8),
                                         q8.view(1, 4, 8), off),
     ]
@@ -273,3 +274,24 @@ def test_mx_gemm_argument_checks(lib):
     assert call(**dict(kw, ldsa=31)) == -2
     assert call(**dict(kw, ldsb=63)) == -2
     assert call(**dict(kw, ogs=16)) == -2
+
+
+def test_mx_dual_argument_checks(lib):
+    f = lib.fp8_mx_quant_dual_padded
+
+    def call(**kw):
+        a = dict(x=FAKE, rows=100, cols=64, ldx=64, off=FAKE, e=2, qr=FAKE, ldqr=64, sr=FAKE,
+                 ldswr=100, qc=FAKE, ldqc=368, sc=FAKE, ldswc=64)
+        a.update(kw)
+        return f(a["x"], a["rows"], a["cols"], a["ldx"], a["off"], a["e"], a["qr"], a["ldqr"],
+                 a["sr"], a["ldswr"], a["qc"], a["ldqc"], a["sc"], a["ldswc"], None, None)
+
+    assert call(qr=None) == -1
+    assert call(sr=None) == -1
+    assert call(cols=48, ldx=48, ldqr=48, ldswc=48) == -2   # rowwise blocks of 32 columns
+    assert call(ldswr=99) == -2                              # one scale word per row
+    assert call(ldqr=56) == -2
+    assert call(ldqr=68) == -3
+    assert call(qr=ctypes.c_void_p((1 << 20) + 4)) == -3
+    assert call(ldqc=352) == -2                              # as the column-wise call
+    assert call(rows=0, ldswr=0) == 0

@@ -269,3 +269,42 @@ def test_mx_input_gradient_path(sizes, n_w, k_w):
     got = out.cpu().numpy()[rows, cols].astype(np.float64)
     err = np.abs(got - ref)
     assert (err <= bound).all(), (err.max(), np.argmax(err - bound))
+
+
+@pytest.mark.parametrize("sizes,cols", [
+    ([5, 0, 19, 8], 32),
+    ([0, 1, 31, 32, 33, 0, 129, 255, 256], 96),
+    ([3000, 70, 700], 288),
+    ([20011, 3, 385], 128),
+    ([0, 0, 0], 64),
+])
+def test_mx_dual_matches_rowwise_and_padded_colwise(sizes, cols):
+    """One read gives the MX rowwise codes of every grouped row and the MX
+    padded column-wise codes, each bit-exact against the oracle; rows past
+    the last group are not written."""
+    m = int(sum(sizes))
+    extra = 21
+    x = spread_bf16(7 * m + cols, (m + extra, cols), block_axis=0, outliers=0.002)
+    off = wl.offsets_from_sizes(sizes)
+    e = len(sizes)
+    ld_q = (m + extra + 128 * e + 127) // 128 * 128
+    q_row = torch.full((m + extra, cols), 0xAB, dtype=torch.uint8, device="cuda")
+    s_row = torch.full(((cols + 127) // 128, m + extra), CANARY, dtype=torch.int32, device="cuda")
+    q_col = torch.full((cols, ld_q), 0xAB, dtype=torch.uint8, device="cuda")
+    s_col = torch.full((ld_q // 128, cols), CANARY, dtype=torch.int32, device="cuda")
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    qgg.fp8_mx_quant_dual_padded(x.cuda(), torch.from_numpy(off).cuda(), q_row=q_row,
+                                 scales_row=s_row, q_col=q_col, scales_col=s_col, status=st)
+    torch.cuda.synchronize()
+    xb = bits(x)
+    r_q, r_s = orc.mx_quant_rowwise(xb[:m])
+    c_q, c_s = orc.mx_quant_colwise_padded(xb, off, ld_q=ld_q, fill=0xAB, scale_fill=0xCD)
+    qr = q_row.cpu().numpy()
+    assert (qr[:m] == r_q).all()
+    assert (qr[m:] == 0xAB).all()
+    blocks = qgg.mx_scales_to_blocks(s_row, 4 * s_row.shape[0]).cpu().numpy()
+    assert (blocks[:m, :cols // 32] == r_s).all()
+    assert (s_row[:, m:] == CANARY).all()
+    assert (q_col.cpu().numpy() == c_q).all()
+    assert (qgg.mx_scales_to_blocks(s_col, ld_q // 32).cpu().numpy() == c_s).all()
+    assert int(st.item()) == 0
