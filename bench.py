@@ -646,30 +646,60 @@ def run_gpu(args, world, rank, local):
     ms_step = total_ms / args.steps
     clocks = clk.summary()
 
-    # end to end through the public API with host buffers: pinned H2D of the
-    # step's inputs, the step's calls, D2H of the result, every step
-    pinned = [(d, h.contiguous().pin_memory()) for d, h in st.host_inputs]
-    hout = torch.empty(st.result.shape, dtype=st.result.dtype).pin_memory()
-    e2e_steps = max(2, min(args.steps, 5))
+    # end to end through the public API with host buffers: every step copies
+    # its inputs from pinned host memory to the device, runs the step's calls
+    # and copies its result back to pinned host memory.  Two sets of device
+    # buffers and three streams (upload, compute, download) let step i + 1's
+    # upload run while step i computes and downloads (PCIe is full duplex);
+    # events order each buffer's reuse.
+    sts = [st, Step(w)]
+    pinned = [[(d, h.contiguous().pin_memory()) for d, h in t.host_inputs] for t in sts]
+    houts = [torch.empty(t.result.shape, dtype=t.result.dtype).pin_memory() for t in sts]
+    e2e_steps = max(3, min(args.steps, 6))
+    comp = torch.cuda.current_stream()
+    up, down = torch.cuda.Stream(), torch.cuda.Stream()
+    ev = {key: [torch.cuda.Event() for _ in sts] for key in ("up", "comp", "down")}
+    calls = [t.kernels() for t in sts]
+    first = [True, True]
 
-    def e2e_step():
-        for d, h in pinned:
-            d.copy_(h.view(d.shape), non_blocking=True)
-        step()
-        hout.copy_(st.result, non_blocking=True)
+    def e2e_step(i):
+        b = i % 2
+        with torch.cuda.stream(up):
+            if not first[b]:
+                up.wait_event(ev["comp"][b])  # the step two back has read these inputs
+            for d, h in pinned[b]:
+                d.copy_(h.view(d.shape), non_blocking=True)
+            ev["up"][b].record(up)
+        comp.wait_event(ev["up"][b])
+        if not first[b]:
+            comp.wait_event(ev["down"][b])  # the result two back has been read
+        for f in calls[b]:
+            f()
+        ev["comp"][b].record(comp)
+        with torch.cuda.stream(down):
+            down.wait_event(ev["comp"][b])
+            houts[b].copy_(sts[b].result, non_blocking=True)
+            ev["down"][b].record(down)
+        first[b] = False
 
-    e2e_step()
+    e2e_step(0)
+    e2e_step(1)
     torch.cuda.synchronize()
     barrier(world)
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for _ in range(e2e_steps):
-        e2e_step()
-    e1.record()
+    e0.record(comp)
+    up.wait_event(e0)
+    for i in range(e2e_steps):
+        e2e_step(i)
+    for b in range(2):
+        comp.wait_event(ev["down"][b])
+    e1.record(comp)
     torch.cuda.synchronize()
     barrier(world)
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world) / e2e_steps
+    hout = houts[0]
+    pinned = pinned[0]
 
     flops = st.flops
     fp8_peak = 2.0 * pk["bf16"]
@@ -708,7 +738,7 @@ def run_gpu(args, world, rank, local):
         gpu_launches=st.launches * args.steps,
         clocks=clocks,
     )
-    del pinned, hout
+    del pinned, hout, houts, sts
     if rank == 0 and world == 1 and Step is ForwardStep and not args.no_cpu_baseline:
         _, full, desc = oracle_sample(w, min(8192, st.m), min(8192, st.e * st.n), 120000)
         cpu_v = flops / full / 1e12
