@@ -22,8 +22,8 @@
 // contiguous run of words for the rows of its tile.
 //  - rowwise: a warp takes 32 rows x one 128-column group; a lane owns 8
 //    consecutive columns of a row (one 16-byte load), four lanes one block;
-//    the block absmax is two shuffles away, four shuffles gather a row's
-//    four scale bytes into its word, and the group's 32 words leave as one
+//    the block absmax is two shuffles away, the block bytes go to a per-warp
+//    table in shared memory, and the group's 32 row words leave as one
 //    128-byte store;
 //  - column-wise along each expert group's tokens, written transposed in the
 //    padded layout (group e from token P_e = sum_{j<e} round_up(size_j, 128),
@@ -82,8 +82,8 @@ __device__ __forceinline__ uint32_t absmax8(const uint4 &v) {
 // A warp takes 32 rows x one 128-column group: sixteen lanes per row (8
 // columns each, one 16-byte load), two rows per load instruction, sixteen
 // loads in flight per lane.  A block's four lanes meet by two shuffles; the
-// group's scale words of the 32 rows end up one per lane and leave as one
-// 128-byte store.
+// block bytes of the 32 rows go to a per-warp table, so that the group's
+// scale words end up one per lane and leave as one 128-byte store.
 constexpr int kMxRowThreads = 256;
 constexpr int kMxRowsPerWarp = 32;
 
@@ -101,15 +101,19 @@ struct MxRowParams {
 };
 
 __global__ void __launch_bounds__(kMxRowThreads, 2) mx_rowwise_kernel(const MxRowParams p) {
+  // per warp: the scale bytes [32 rows][4 blocks] of its unit; row j's word
+  // is then one 4-byte read
+  __shared__ uint32_t rowsb[kMxRowThreads / 32][kMxRowsPerWarp];
   const int lane = threadIdx.x & 31;
   const int half = lane >> 4;          // which of the two rows of a load
   const int c16 = lane & 15;           // 8-column slot within the group
+  uint8_t *rb = reinterpret_cast<uint8_t *>(rowsb[threadIdx.x >> 5]);
   const int64_t nwarps = static_cast<int64_t>(gridDim.x) * (kMxRowThreads / 32);
   for (int64_t u = (static_cast<int64_t>(blockIdx.x) * kMxRowThreads + threadIdx.x) >> 5;
        u < p.units; u += nwarps) {
-    const int64_t rb = u / p.ngroups;  // once per 32 x 128 unit
-    const int g = static_cast<int>(u - rb * p.ngroups);
-    const int64_t r0 = rb * kMxRowsPerWarp;
+    const int64_t rb_i = u / p.ngroups;  // once per 32 x 128 unit
+    const int g = static_cast<int>(u - rb_i * p.ngroups);
+    const int64_t r0 = rb_i * kMxRowsPerWarp;
     const int col = 128 * g + 8 * c16;
     const bool c_ok = col < p.cols;
     uint4 v[kMxRowsPerWarp / 2];
@@ -119,7 +123,6 @@ __global__ void __launch_bounds__(kMxRowThreads, 2) mx_rowwise_kernel(const MxRo
       v[i] = (c_ok && r < p.rows) ? __ldcs(p.x + r * p.ld_x16 + col / 8)
                                   : make_uint4(0u, 0u, 0u, 0u);
     }
-    uint32_t myword = 0;  // lane j: the scale word of row r0 + j
 #pragma unroll
     for (int i = 0; i < kMxRowsPerWarp / 2; ++i) {
       uint32_t m = absmax8(v[i]);
@@ -129,20 +132,13 @@ __global__ void __launch_bounds__(kMxRowThreads, 2) mx_rowwise_kernel(const MxRo
       const uint2 c = mx_encode8(v[i], mx_multiplier(e));
       const int64_t r = r0 + 2 * i + half;
       if (c_ok && r < p.rows) __stcs(reinterpret_cast<uint2 *>(p.q + r * p.ld_q + col), c);
-      // the row's word: bytes of the lanes 16h, 16h + 4, 16h + 8, 16h + 12
-      // (columns past the row's end give byte 0)
-      const uint32_t byte = static_cast<uint32_t>(e + 127);
-      const int l0 = lane & 16;
-      const uint32_t word = __shfl_sync(0xFFFFFFFFu, byte, l0) |
-                            (__shfl_sync(0xFFFFFFFFu, byte, l0 + 4) << 8) |
-                            (__shfl_sync(0xFFFFFFFFu, byte, l0 + 8) << 16) |
-                            (__shfl_sync(0xFFFFFFFFu, byte, l0 + 12) << 24);
-      const uint32_t w0 = __shfl_sync(0xFFFFFFFFu, word, 0);
-      const uint32_t w1 = __shfl_sync(0xFFFFFFFFu, word, 16);
-      if (lane == 2 * i) myword = w0;
-      if (lane == 2 * i + 1) myword = w1;
+      // the block's byte (columns past the row's end give byte 0)
+      if ((c16 & 3) == 0) rb[4 * (2 * i + half) + (c16 >> 2)] = static_cast<uint8_t>(e + 127);
     }
-    if (r0 + lane < p.rows) p.sw[static_cast<int64_t>(g) * p.ld_sw + r0 + lane] = myword;
+    __syncwarp();
+    if (r0 + lane < p.rows)
+      p.sw[static_cast<int64_t>(g) * p.ld_sw + r0 + lane] = rowsb[threadIdx.x >> 5][lane];
+    __syncwarp();  // the table is rewritten by the warp's next unit
   }
 }
 
