@@ -72,10 +72,16 @@ struct PanelSmem {
   int32_t order[kPMaxGroups];           // groups by size, largest first
   int32_t nb[kPMaxGroups];              // ordered group i: 128-row blocks
   int32_t apre[kPMaxGroups + 1];        // blocks of the groups before ordered group i
+  alignas(16) float cscale[kPW];        // the cast's column scales (read as float4)
   int32_t n_nonempty, total, delay;
-  int32_t step;
+  int32_t nstep;                        // the step decoded during the current one
+  int32_t sidx[2];                      // step index, by parity
+  int32_t dA[2][6], dC[2][6];           // its decoded blocks (PBlock), by parity
 };
 static_assert(offsetof(PanelSmem, tile) == 0, "store tile 1024-byte aligned");
+static_assert(kPWarps >= 3, "warps 1 and 2 decode the next step");
+static_assert(offsetof(PanelSmem, cscale) % 16 == 0 && offsetof(PanelSmem, red) % 16 == 0,
+              "16-byte shared-memory accesses");
 
 struct PanelParams {
   const uint4 *x;        // bf16 rows as 16-byte vectors
@@ -187,6 +193,7 @@ struct PBlock {
   int32_t u;      // unit (arrival counter)
   int32_t need;   // arrivals that complete the unit
 };
+static_assert(sizeof(PBlock) == sizeof(PanelSmem::dA[0]), "decoded blocks are kept as six words");
 
 // Block a of the list (the whole warp calls it; every lane gets the same
 // answer): the ordered group by a 32-way search over the block prefix.
@@ -212,6 +219,26 @@ __device__ PBlock decode_block(const PanelSmem &sm, int32_t a, int np, int lane)
   r.u = DUAL ? lo : lo * np + r.q;
   r.need = kPWarps * (DUAL ? nbi * np : nbi);  // each block of the unit adds kPWarps
   return r;
+}
+
+// The blocks of step sm.nstep, decoded one step ahead into parity slot par:
+// warp 1 takes the absmax block (and the index), warp 2 the cast block.
+template <bool DUAL>
+__device__ __forceinline__ void decode_ahead(PanelSmem &sm, int par, int np, int w, int lane,
+                                             int32_t total, int32_t delay, int32_t steps) {
+  const int32_t ns = sm.nstep;
+  if (w == 1) {
+    if (ns < total) {
+      const PBlock b = decode_block<DUAL>(sm, ns, np, lane);
+      if (lane == 0) memcpy(sm.dA[par], &b, sizeof b);
+    }
+    if (lane == 0) sm.sidx[par] = ns;
+  } else if (w == 2) {
+    if (ns >= delay && ns < steps) {
+      const PBlock b = decode_block<DUAL>(sm, ns - delay, np, lane);
+      if (lane == 0) memcpy(sm.dC[par], &b, sizeof b);
+    }
+  }
 }
 
 // Dual form: every row's absmax over the lane's 8 columns, reduced over the
@@ -275,29 +302,35 @@ __global__ void __launch_bounds__(kPThreads, kPBlocksPerSM)
   const int32_t total = sm.total, delay = sm.delay;
   const int32_t steps = total + delay;
   uint32_t sat = 0;
-  int32_t next = 0;
-  if (tid == 0) next = static_cast<int32_t>(atomicAdd(p.work, 1u));
-  while (true) {
-    if (tid == 0) {
-      sm.step = next;
-      if (next < steps) next = static_cast<int32_t>(atomicAdd(p.work, 1u));
-      bulk_wait_read<0>();  // the tile's previous store has read it
-    }
-    __syncthreads();
-    const int32_t st = sm.step;
+  int32_t next = 0;  // thread 0: the step after the one being decoded
+  if (tid == 0) sm.nstep = static_cast<int32_t>(atomicAdd(p.work, 1u));
+  __syncthreads();
+  decode_ahead<DUAL>(sm, 0, np, w, lane, total, delay, steps);
+  if (tid == 0 && sm.nstep < steps) next = static_cast<int32_t>(atomicAdd(p.work, 1u));
+  __syncthreads();
+  for (int par = 0;; par ^= 1) {
+    // a step is bracketed by two block barriers: the one after the absmax
+    // (which also publishes the cast's column scales and the next step's
+    // index) and the one before the tile's store
+    const int32_t st = sm.sidx[par];
     if (st >= steps) break;
+    if (tid == 0) {
+      sm.nstep = next;
+      if (next < steps) next = static_cast<int32_t>(atomicAdd(p.work, 1u));
+    }
     const bool has_a = st < total;
     const bool has_c = st >= delay;
     PBlock A{}, C{};
-    if (has_a) A = decode_block<DUAL>(sm, st, np, lane);
-    if (has_c) C = decode_block<DUAL>(sm, st - delay, np, lane);
+    if (has_a) memcpy(&A, sm.dA[par], sizeof A);
+    if (has_c) memcpy(&C, sm.dC[par], sizeof C);
 
-    // the cast's scale words, early when the unit is complete already
+    // the cast's scale words, early when the unit is complete already: each
+    // warp derives the scales of 32 of the panel's columns
     bool c_ready = false;
-    uint4 ua0 = make_uint4(0u, 0u, 0u, 0u), ua1 = ua0;
-    uint32_t urow = 0;
+    uint32_t uword = 0, urow = 0;
     const int cc0 = C.q * kPW;
     const bool c_lane = has_c && cc0 + 8 * lane < p.cols;
+    const int ccol = cc0 + 32 * w + lane;  // this lane's scale column
     if (has_c) {
       uint32_t cnt = 0;
       if (lane == 0)
@@ -306,13 +339,7 @@ __global__ void __launch_bounds__(kPThreads, kPBlocksPerSM)
       c_ready = __shfl_sync(0xFFFFFFFFu, cnt, 0) >= static_cast<uint32_t>(C.need) +
                                                      p.uw.extra_arrivals;
     }
-    auto load_c_words = [&]() {
-      if (c_lane) {
-        const uint4 *src = reinterpret_cast<const uint4 *>(
-            p.amax + static_cast<int64_t>(C.i) * p.cols + cc0 + 8 * lane);
-        ua0 = __ldcg(src);
-        ua1 = __ldcg(src + 1);
-      }
+    auto load_row_word = [&]() {
       if constexpr (DUAL) {
         const int32_t cgs = C.e ? sm.end[C.e - 1] : 0;
         const int32_t row = cgs + C.b * kRB + kWR * w + lane;
@@ -320,7 +347,10 @@ __global__ void __launch_bounds__(kPThreads, kPBlocksPerSM)
         urow = (lane < kWR && row < r1) ? __ldcg(p.rowmax + row) : 0u;
       }
     };
-    if (c_ready) load_c_words();
+    if (c_ready) {
+      uword = ccol < p.cols ? __ldcg(p.amax + static_cast<int64_t>(C.i) * p.cols + ccol) : 0u;
+      load_row_word();
+    }
 
     // ---------------------------------------------------------- absmax of block s
     if (has_a) {
@@ -348,7 +378,13 @@ __global__ void __launch_bounds__(kPThreads, kPBlocksPerSM)
           make_uint4(absmax_bits(am.x), absmax_bits(am.y), absmax_bits(am.z),
                      absmax_bits(am.w));
     }
-    __syncthreads();
+    if (c_ready) {
+      const float sc = scale_from_amax(bf16_bits_to_float(uword), p.smax);
+      sm.cscale[32 * w + lane] = sc;
+      if (C.b == 0 && ccol < p.cols) p.scales_col[static_cast<int64_t>(C.e) * p.cols + ccol] = sc;
+    }
+    if (tid == 0) bulk_wait_read<0>();  // the previous store has read the tile
+    const bool all_ready = __syncthreads_and(!has_c || c_ready) != 0;
     if (has_a) {
       // each warp merges 32 of the panel's columns into the unit's absmax:
       // column 32w + lane is half (lane & 1) of word 16w + lane / 2
@@ -376,10 +412,17 @@ __global__ void __launch_bounds__(kPThreads, kPBlocksPerSM)
                        : "memory");
       }
     }
+    decode_ahead<DUAL>(sm, par ^ 1, np, w, lane, total, delay, steps);
 
     // ---------------------------------------------------------- cast of block s - D
     bool failed = false;
-    if (has_c && !c_ready) {  // wait (bounded) until every block of the unit is counted
+    float s[8];
+    if (has_c && all_ready) {
+      const float4 s0 = *reinterpret_cast<const float4 *>(&sm.cscale[8 * lane]);
+      const float4 s1 = *reinterpret_cast<const float4 *>(&sm.cscale[8 * lane + 4]);
+      s[0] = s0.x; s[1] = s0.y; s[2] = s0.z; s[3] = s0.w;
+      s[4] = s1.x; s[5] = s1.y; s[6] = s1.z; s[7] = s1.w;
+    } else if (has_c) {  // wait (bounded) until every block of the unit is counted
       int ok = 1;
       if (lane == 0) {
         const uint32_t target = static_cast<uint32_t>(C.need) + p.uw.extra_arrivals;
@@ -399,7 +442,19 @@ __global__ void __launch_bounds__(kPThreads, kPBlocksPerSM)
         asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(c) : "l"(p.arrive + C.u)
                      : "memory");
         (void)c;
-        load_c_words();
+        uint4 ua0 = make_uint4(0u, 0u, 0u, 0u), ua1 = ua0;
+        if (c_lane) {
+          const uint4 *src = reinterpret_cast<const uint4 *>(
+              p.amax + static_cast<int64_t>(C.i) * p.cols + cc0 + 8 * lane);
+          ua0 = __ldcg(src);
+          ua1 = __ldcg(src + 1);
+        }
+        load_row_word();
+        const uint32_t a[8] = {ua0.x, ua0.y, ua0.z, ua0.w, ua1.x, ua1.y, ua1.z, ua1.w};
+#pragma unroll
+        for (int j = 0; j < 8; ++j) s[j] = scale_from_amax(bf16_bits_to_float(a[j]), p.smax);
+        if (C.b == 0 && w == 0 && c_lane)
+          store_scales8(p.scales_col + static_cast<int64_t>(C.e) * p.cols + cc0 + 8 * lane, s);
       } else {
         failed = true;
       }
@@ -417,41 +472,32 @@ __global__ void __launch_bounds__(kPThreads, kPBlocksPerSM)
         v[k] = (c_lane && c_rw0 + k < c_r1) ? __ldcs(src + k * p.ld_x16)
                                             : make_uint4(0u, 0u, 0u, 0u);
     }
-    if (has_c) {
-      if (!failed) {
-        const int e = C.e;
-        const int32_t r1 = c_r1, rw0 = c_rw0;
-        float s[8];
-        const uint32_t a[8] = {ua0.x, ua0.y, ua0.z, ua0.w, ua1.x, ua1.y, ua1.z, ua1.w};
-#pragma unroll
-        for (int j = 0; j < 8; ++j) s[j] = scale_from_amax(bf16_bits_to_float(a[j]), p.smax);
-        if (C.b == 0 && w == 0 && c_lane)
-          store_scales8(p.scales_col + static_cast<int64_t>(e) * p.cols + cc0 + 8 * lane, s);
-        if constexpr (DUAL) {
-          float rs_lane = 0.0f;  // the scale of row rw0 + lane (lanes 0..15)
-          if (lane < kWR && rw0 + lane < r1) {
-            rs_lane = scale_from_amax(bf16_bits_to_float(urow), p.smax);
-            if (C.q == 0) p.scales_row[rw0 + lane] = rs_lane;
-          }
-          // rowwise codes in place: 8 columns of a row per lane, one 8-byte store
-#pragma unroll
-          for (int k = 0; k < kWR; ++k) {
-            const float rs = __shfl_sync(0xFFFFFFFFu, rs_lane, k);
-            uint32_t c2[4];
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              const uint32_t wd = word(v[k], j);
-              c2[j] = enc_pair<FMT, FAST>(lo_f(wd), hi_f(wd), rs, rs, p.smax, p.sat_thr, sat);
-            }
-            if (c_lane && rw0 + k < r1)
-              *reinterpret_cast<uint2 *>(p.q_row + static_cast<int64_t>(rw0 + k) * p.ld_qr +
-                                         cc0 + 8 * lane) =
-                  make_uint2(c2[0] | (c2[1] << 16), c2[2] | (c2[3] << 16));
-          }
+    if (has_c && !failed) {
+      const int32_t r1 = c_r1, rw0 = c_rw0;
+      if constexpr (DUAL) {
+        float rs_lane = 0.0f;  // the scale of row rw0 + lane (lanes 0..15)
+        if (lane < kWR && rw0 + lane < r1) {
+          rs_lane = scale_from_amax(bf16_bits_to_float(urow), p.smax);
+          if (C.q == 0) p.scales_row[rw0 + lane] = rs_lane;
         }
-        tile_col_codes<FMT, FAST>(v, s, sm.tile, w, lane, p.smax, p.sat_thr, sat);
-        fence_proxy_async_smem();
+        // rowwise codes in place: 8 columns of a row per lane, one 8-byte store
+#pragma unroll
+        for (int k = 0; k < kWR; ++k) {
+          const float rs = __shfl_sync(0xFFFFFFFFu, rs_lane, k);
+          uint32_t c2[4];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const uint32_t wd = word(v[k], j);
+            c2[j] = enc_pair<FMT, FAST>(lo_f(wd), hi_f(wd), rs, rs, p.smax, p.sat_thr, sat);
+          }
+          if (c_lane && rw0 + k < r1)
+            *reinterpret_cast<uint2 *>(p.q_row + static_cast<int64_t>(rw0 + k) * p.ld_qr +
+                                       cc0 + 8 * lane) =
+                make_uint2(c2[0] | (c2[1] << 16), c2[2] | (c2[3] << 16));
+        }
       }
+      tile_col_codes<FMT, FAST>(v, s, sm.tile, w, lane, p.smax, p.sat_thr, sat);
+      fence_proxy_async_smem();
     }
     if (__syncthreads_or(failed)) {
       if (tid == 0) status_or(p.status, FP8QGG_STATUS_TIMEOUT);
