@@ -75,8 +75,8 @@ struct PanelSmem {
   alignas(16) float cscale[kPW];        // the cast's column scales (read as float4)
   int32_t n_nonempty, total, delay;
   int32_t nstep;                        // the step decoded during the current one
-  int32_t sidx[2];                      // step index, by parity
-  int32_t dA[2][6], dC[2][6];           // its decoded blocks (PBlock), by parity
+  int32_t sidx[3];                      // step index, by slot (step number mod 3)
+  int32_t dA[3][6], dC[3][6];           // its decoded blocks (PBlock), by slot
 };
 static_assert(offsetof(PanelSmem, tile) == 0, "store tile 1024-byte aligned");
 static_assert(kPWarps >= 3, "warps 1 and 2 decode the next step");
@@ -221,8 +221,8 @@ __device__ PBlock decode_block(const PanelSmem &sm, int32_t a, int np, int lane)
   return r;
 }
 
-// The blocks of step sm.nstep, decoded one step ahead into parity slot par:
-// warp 1 takes the absmax block (and the index), warp 2 the cast block.
+// The blocks of step sm.nstep, decoded ahead into slot par: warp 1 takes the
+// absmax block (and the index), warp 2 the cast block.
 template <bool DUAL>
 __device__ __forceinline__ void decode_ahead(PanelSmem &sm, int par, int np, int w, int lane,
                                              int32_t total, int32_t delay, int32_t steps) {
@@ -302,27 +302,82 @@ __global__ void __launch_bounds__(kPThreads, kPBlocksPerSM)
   const int32_t total = sm.total, delay = sm.delay;
   const int32_t steps = total + delay;
   uint32_t sat = 0;
-  int32_t next = 0;  // thread 0: the step after the one being decoded
-  if (tid == 0) sm.nstep = static_cast<int32_t>(atomicAdd(p.work, 1u));
+  // The dual form loads each block early: the absmax block's rows at the end
+  // of the previous step (under the end-of-step barrier and the store), the
+  // cast block's as soon as the absmax has read them (under the mid-step
+  // barrier); its longer step gains from the overlap (185 -> 177 us on the
+  // DeepSeek-MoE-16B grad_out), while the column-wise form measured 2%
+  // slower that way and loads each block where the step needs it.  Early
+  // loads need the next step's blocks a step in advance: they are decoded
+  // two steps ahead (three slots) instead of one (two slots).
+  constexpr bool kEarly = DUAL;
+  constexpr int kSlots = kEarly ? 3 : 2;
+  // thread 0 claims this block's steps from the counter, in increasing order;
+  // each is published in sm.nstep and decoded kSlots - 1 steps before it runs
+  int32_t next = 0;
+  auto claim = [&]() {
+    sm.nstep = next;
+    if (next < steps) next = static_cast<int32_t>(atomicAdd(p.work, 1u));
+  };
+  if (tid == 0) {
+    next = static_cast<int32_t>(atomicAdd(p.work, 1u));
+    claim();
+  }
   __syncthreads();
   decode_ahead<DUAL>(sm, 0, np, w, lane, total, delay, steps);
-  if (tid == 0 && sm.nstep < steps) next = static_cast<int32_t>(atomicAdd(p.work, 1u));
   __syncthreads();
-  for (int par = 0;; par ^= 1) {
-    // a step is bracketed by two block barriers: the one after the absmax
-    // (which also publishes the cast's column scales and the next step's
-    // index) and the one before the tile's store
-    const int32_t st = sm.sidx[par];
-    if (st >= steps) break;
-    if (tid == 0) {
-      sm.nstep = next;
-      if (next < steps) next = static_cast<int32_t>(atomicAdd(p.work, 1u));
+  if constexpr (kSlots == 3) {
+    if (tid == 0) claim();
+    __syncthreads();
+    decode_ahead<DUAL>(sm, 1, np, w, lane, total, delay, steps);
+    __syncthreads();
+  }
+
+  // The block's rows, 16 per warp (the dual form's v lives across steps).
+  uint4 v[kWR];
+  // (every call defines all of v, zeros when there is no block, so that no
+  // earlier contents stay live)
+  auto load_rows = [&](uint4 (&dst)[kWR], const PBlock &B, bool has, bool streaming) {
+    const int32_t gs = B.e ? sm.end[B.e - 1] : 0;
+    const int32_t r0 = gs + B.b * kRB;
+    const int32_t r1 = has ? min(sm.end[B.e], r0 + kRB) : 0;
+    const int32_t rw0 = r0 + kWR * w;
+    const int c0 = B.q * kPW;
+    const bool lane_ok = c0 + 8 * lane < p.cols;
+    const uint4 *src = p.x + static_cast<int64_t>(rw0) * p.ld_x16 + (c0 >> 3) + lane;
+#pragma unroll
+    for (int k = 0; k < kWR; ++k) {
+      const bool ok = lane_ok && rw0 + k < r1;
+      dst[k] = !ok ? make_uint4(0u, 0u, 0u, 0u)
+                   : streaming ? __ldcs(src + k * p.ld_x16) : __ldcg(src + k * p.ld_x16);
     }
+  };
+  auto load_a = [&](int slot) {  // the absmax block of the step in this slot
+    PBlock B{};
+    const bool has = sm.sidx[slot] < total;
+    if (has) memcpy(&B, sm.dA[slot], sizeof B);
+    load_rows(v, B, has, false);
+  };
+  if constexpr (kEarly) load_a(0);
+  for (int slot = 0;; slot = slot == kSlots - 1 ? 0 : slot + 1) {
+    // a step is bracketed by two block barriers: the one after the absmax
+    // (which also publishes the cast's column scales and the index of the
+    // step decoded next) and the one before the tile's store
+    const int slot1 = slot == kSlots - 1 ? 0 : slot + 1;
+    const int slot_dec = kSlots == 3 ? (slot1 == 2 ? 0 : slot1 + 1) : slot1;
+    const int32_t st = sm.sidx[slot];
+    if (st >= steps) break;
+    if (tid == 0) claim();
     const bool has_a = st < total;
     const bool has_c = st >= delay;
     PBlock A{}, C{};
-    if (has_a) memcpy(&A, sm.dA[par], sizeof A);
-    if (has_c) memcpy(&C, sm.dC[par], sizeof C);
+    if (has_a) memcpy(&A, sm.dA[slot], sizeof A);
+    if (has_c) memcpy(&C, sm.dC[slot], sizeof C);
+    // (the column-wise form: the step's own arrays, as it loads them in place)
+    uint4 va[kWR], vc[kWR];
+    uint4 (&vA)[kWR] = kEarly ? v : va;
+    uint4 (&vC)[kWR] = kEarly ? v : vc;
+    if constexpr (!kEarly) load_rows(vA, A, has_a, false);
 
     // the cast's scale words, early when the unit is complete already: each
     // warp derives the scales of 32 of the panel's columns
@@ -358,26 +413,22 @@ __global__ void __launch_bounds__(kPThreads, kPBlocksPerSM)
       const int32_t r0 = gs + A.b * kRB;
       const int32_t r1 = min(sm.end[A.e], r0 + kRB);
       const int32_t rw0 = r0 + kWR * w;
-      const int c0 = A.q * kPW;
-      const bool lane_ok = c0 + 8 * lane < p.cols;
-      const uint4 *src = p.x + static_cast<int64_t>(rw0) * p.ld_x16 + (c0 >> 3) + lane;
-      uint4 v[kWR];
-#pragma unroll
-      for (int k = 0; k < kWR; ++k)
-        v[k] = (lane_ok && rw0 + k < r1) ? __ldcg(src + k * p.ld_x16) : make_uint4(0u, 0u, 0u, 0u);
       uint4 am = make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
       for (int k = 0; k < kWR; ++k) {
-        am.x = absmax_acc(am.x, v[k].x);
-        am.y = absmax_acc(am.y, v[k].y);
-        am.z = absmax_acc(am.z, v[k].z);
-        am.w = absmax_acc(am.w, v[k].w);
+        am.x = absmax_acc(am.x, vA[k].x);
+        am.y = absmax_acc(am.y, vA[k].y);
+        am.z = absmax_acc(am.z, vA[k].z);
+        am.w = absmax_acc(am.w, vA[k].w);
       }
-      if constexpr (DUAL) merge_row_amax(v, p.rowmax, rw0, r1, lane);
+      if constexpr (DUAL) merge_row_amax(vA, p.rowmax, rw0, r1, lane);
       *reinterpret_cast<uint4 *>(&sm.red[w][4 * lane]) =
           make_uint4(absmax_bits(am.x), absmax_bits(am.y), absmax_bits(am.z),
                      absmax_bits(am.w));
     }
+    // the cast block's rows (read-only input: no need to wait for its unit)
+    auto load_c = [&]() { load_rows(vC, C, has_c, true); };
+    if constexpr (kEarly) load_c();
     if (c_ready) {
       const float sc = scale_from_amax(bf16_bits_to_float(uword), p.smax);
       sm.cscale[32 * w + lane] = sc;
@@ -412,7 +463,7 @@ __global__ void __launch_bounds__(kPThreads, kPBlocksPerSM)
                        : "memory");
       }
     }
-    decode_ahead<DUAL>(sm, par ^ 1, np, w, lane, total, delay, steps);
+    decode_ahead<DUAL>(sm, slot_dec, np, w, lane, total, delay, steps);
 
     // ---------------------------------------------------------- cast of block s - D
     bool failed = false;
@@ -459,22 +510,12 @@ __global__ void __launch_bounds__(kPThreads, kPBlocksPerSM)
         failed = true;
       }
     }
-    uint4 v[kWR];
-    int32_t c_r1 = 0, c_rw0 = 0;
+    if constexpr (!kEarly) load_c();
     if (has_c && !failed) {
-      const int32_t gs = C.e ? sm.end[C.e - 1] : 0;
-      const int32_t r0 = gs + C.b * kRB;
-      c_r1 = min(sm.end[C.e], r0 + kRB);
-      c_rw0 = r0 + kWR * w;
-      const uint4 *src = p.x + static_cast<int64_t>(c_rw0) * p.ld_x16 + (cc0 >> 3) + lane;
-#pragma unroll
-      for (int k = 0; k < kWR; ++k)
-        v[k] = (c_lane && c_rw0 + k < c_r1) ? __ldcs(src + k * p.ld_x16)
-                                            : make_uint4(0u, 0u, 0u, 0u);
-    }
-    if (has_c && !failed) {
-      const int32_t r1 = c_r1, rw0 = c_rw0;
       if constexpr (DUAL) {
+        const int32_t cgs = C.e ? sm.end[C.e - 1] : 0;
+        const int32_t r1 = min(sm.end[C.e], cgs + C.b * kRB + kRB);
+        const int32_t rw0 = cgs + C.b * kRB + kWR * w;
         float rs_lane = 0.0f;  // the scale of row rw0 + lane (lanes 0..15)
         if (lane < kWR && rw0 + lane < r1) {
           rs_lane = scale_from_amax(bf16_bits_to_float(urow), p.smax);
@@ -487,7 +528,7 @@ __global__ void __launch_bounds__(kPThreads, kPBlocksPerSM)
           uint32_t c2[4];
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
-            const uint32_t wd = word(v[k], j);
+            const uint32_t wd = word(vC[k], j);
             c2[j] = enc_pair<FMT, FAST>(lo_f(wd), hi_f(wd), rs, rs, p.smax, p.sat_thr, sat);
           }
           if (c_lane && rw0 + k < r1)
@@ -496,8 +537,11 @@ __global__ void __launch_bounds__(kPThreads, kPBlocksPerSM)
                 make_uint2(c2[0] | (c2[1] << 16), c2[2] | (c2[3] << 16));
         }
       }
-      tile_col_codes<FMT, FAST>(v, s, sm.tile, w, lane, p.smax, p.sat_thr, sat);
+      tile_col_codes<FMT, FAST>(vC, s, sm.tile, w, lane, p.smax, p.sat_thr, sat);
       fence_proxy_async_smem();
+    }
+    if constexpr (kEarly) {
+      if (!failed) load_a(slot1);  // the next step's absmax block
     }
     if (__syncthreads_or(failed)) {
       if (tid == 0) status_or(p.status, FP8QGG_STATUS_TIMEOUT);
