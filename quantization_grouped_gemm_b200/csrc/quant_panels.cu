@@ -302,255 +302,420 @@ __global__ void __launch_bounds__(kPThreads, kPBlocksPerSM)
   const int32_t total = sm.total, delay = sm.delay;
   const int32_t steps = total + delay;
   uint32_t sat = 0;
-  // The dual form loads each block early: the absmax block's rows at the end
-  // of the previous step (under the end-of-step barrier and the store), the
-  // cast block's as soon as the absmax has read them (under the mid-step
-  // barrier); its longer step gains from the overlap (185 -> 177 us on the
-  // DeepSeek-MoE-16B grad_out), while the column-wise form measured 2%
-  // slower that way and loads each block where the step needs it.  Early
-  // loads need the next step's blocks a step in advance: they are decoded
-  // two steps ahead (three slots) instead of one (two slots).
-  constexpr bool kEarly = DUAL;
-  constexpr int kSlots = kEarly ? 3 : 2;
-  // thread 0 claims this block's steps from the counter, in increasing order;
-  // each is published in sm.nstep and decoded kSlots - 1 steps before it runs
-  int32_t next = 0;
-  auto claim = [&]() {
-    sm.nstep = next;
-    if (next < steps) next = static_cast<int32_t>(atomicAdd(p.work, 1u));
-  };
-  if (tid == 0) {
-    next = static_cast<int32_t>(atomicAdd(p.work, 1u));
-    claim();
-  }
-  __syncthreads();
-  decode_ahead<DUAL>(sm, 0, np, w, lane, total, delay, steps);
-  __syncthreads();
-  if constexpr (kSlots == 3) {
+  if constexpr (!DUAL) {
+    // The column-wise form loads each block where the step needs it (early
+    // loads, as in the dual form below, measured 2% slower here); the next
+    // step's blocks are decoded one step ahead (two slots).
+    int32_t next = 0;  // thread 0: the step after the one being decoded
+    if (tid == 0) sm.nstep = static_cast<int32_t>(atomicAdd(p.work, 1u));
+    __syncthreads();
+    decode_ahead<false>(sm, 0, np, w, lane, total, delay, steps);
+    if (tid == 0 && sm.nstep < steps) next = static_cast<int32_t>(atomicAdd(p.work, 1u));
+    __syncthreads();
+    for (int par = 0;; par ^= 1) {
+      // a step is bracketed by two block barriers: the one after the absmax
+      // (which also publishes the cast's column scales and the next step's
+      // index) and the one before the tile's store
+      const int32_t st = sm.sidx[par];
+      if (st >= steps) break;
+      if (tid == 0) {
+        sm.nstep = next;
+        if (next < steps) next = static_cast<int32_t>(atomicAdd(p.work, 1u));
+      }
+      const bool has_a = st < total;
+      const bool has_c = st >= delay;
+      PBlock A{}, C{};
+      if (has_a) memcpy(&A, sm.dA[par], sizeof A);
+      if (has_c) memcpy(&C, sm.dC[par], sizeof C);
+
+      // the cast's scale words, early when the unit is complete already: each
+      // warp derives the scales of 32 of the panel's columns
+      bool c_ready = false;
+      uint32_t uword = 0;
+      const int cc0 = C.q * kPW;
+      const bool c_lane = has_c && cc0 + 8 * lane < p.cols;
+      const int ccol = cc0 + 32 * w + lane;  // this lane's scale column
+      if (has_c) {
+        uint32_t cnt = 0;
+        if (lane == 0)
+          asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(cnt) : "l"(p.arrive + C.u)
+                       : "memory");
+        c_ready = __shfl_sync(0xFFFFFFFFu, cnt, 0) >= static_cast<uint32_t>(C.need) +
+                                                       p.uw.extra_arrivals;
+      }
+      if (c_ready)
+        uword = ccol < p.cols ? __ldcg(p.amax + static_cast<int64_t>(C.i) * p.cols + ccol) : 0u;
+
+      // ---------------------------------------------------------- absmax of block s
+      if (has_a) {
+        const int32_t gs = A.e ? sm.end[A.e - 1] : 0;
+        const int32_t r0 = gs + A.b * kRB;
+        const int32_t r1 = min(sm.end[A.e], r0 + kRB);
+        const int32_t rw0 = r0 + kWR * w;
+        const int c0 = A.q * kPW;
+        const bool lane_ok = c0 + 8 * lane < p.cols;
+        const uint4 *src = p.x + static_cast<int64_t>(rw0) * p.ld_x16 + (c0 >> 3) + lane;
+        uint4 v[kWR];
+  #pragma unroll
+        for (int k = 0; k < kWR; ++k)
+          v[k] = (lane_ok && rw0 + k < r1) ? __ldcg(src + k * p.ld_x16) : make_uint4(0u, 0u, 0u, 0u);
+        uint4 am = make_uint4(0u, 0u, 0u, 0u);
+  #pragma unroll
+        for (int k = 0; k < kWR; ++k) {
+          am.x = absmax_acc(am.x, v[k].x);
+          am.y = absmax_acc(am.y, v[k].y);
+          am.z = absmax_acc(am.z, v[k].z);
+          am.w = absmax_acc(am.w, v[k].w);
+        }
+        *reinterpret_cast<uint4 *>(&sm.red[w][4 * lane]) =
+            make_uint4(absmax_bits(am.x), absmax_bits(am.y), absmax_bits(am.z),
+                       absmax_bits(am.w));
+      }
+      if (c_ready) {
+        const float sc = scale_from_amax(bf16_bits_to_float(uword), p.smax);
+        sm.cscale[32 * w + lane] = sc;
+        if (C.b == 0 && ccol < p.cols) p.scales_col[static_cast<int64_t>(C.e) * p.cols + ccol] = sc;
+      }
+      if (tid == 0) bulk_wait_read<0>();  // the previous store has read the tile
+      const bool all_ready = __syncthreads_and(!has_c || c_ready) != 0;
+      if (has_a) {
+        // each warp merges 32 of the panel's columns into the unit's absmax:
+        // column 32w + lane is half (lane & 1) of word 16w + lane / 2
+        const int wd = 16 * w + (lane >> 1);
+        uint32_t m = 0;
+  #pragma unroll
+        for (int ww = 0; ww < kPWarps; ++ww) m = __vmaxu2(m, sm.red[ww][wd]);
+        const int c0 = A.q * kPW;
+        const int cc = 32 * w + lane;
+        if (c0 + cc < p.cols)
+          atomicMax(p.amax + static_cast<int64_t>(A.i) * p.cols + c0 + cc,
+                    (lane & 1) ? m >> 16 : m & 0xFFFFu);
+        // every warp's merges happen before warp 0's one release of the count
+        // (a named barrier: the other warps arrive without waiting and go on to
+        // the cast; the release orders their merges too, being cumulative over
+        // the barrier)
+        __syncwarp();
+        if (w != 0) {
+          asm volatile("bar.arrive 2, %0;" ::"n"(kPThreads) : "memory");
+        } else {
+          asm volatile("bar.sync 2, %0;" ::"n"(kPThreads) : "memory");
+          if (lane == 0)
+            asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p.arrive + A.u),
+                         "n"(kPWarps)
+                         : "memory");
+        }
+      }
+      decode_ahead<false>(sm, par ^ 1, np, w, lane, total, delay, steps);
+
+      // ---------------------------------------------------------- cast of block s - D
+      bool failed = false;
+      float s[8];
+      if (has_c && all_ready) {
+        const float4 s0 = *reinterpret_cast<const float4 *>(&sm.cscale[8 * lane]);
+        const float4 s1 = *reinterpret_cast<const float4 *>(&sm.cscale[8 * lane + 4]);
+        s[0] = s0.x; s[1] = s0.y; s[2] = s0.z; s[3] = s0.w;
+        s[4] = s1.x; s[5] = s1.y; s[6] = s1.z; s[7] = s1.w;
+      } else if (has_c) {  // wait (bounded) until every block of the unit is counted
+        int ok = 1;
+        if (lane == 0) {
+          const uint32_t target = static_cast<uint32_t>(C.need) + p.uw.extra_arrivals;
+          const uint64_t t0 = global_timer_ns();
+          while (true) {
+            uint32_t c;
+            asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(c) : "l"(p.arrive + C.u)
+                         : "memory");
+            if (c >= target) break;
+            if (global_timer_ns() - t0 > p.uw.limit_ns) { ok = 0; break; }
+            __nanosleep(64);
+          }
+        }
+        ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+        if (ok) {
+          uint32_t c;  // every lane acquires the count it relies on
+          asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(c) : "l"(p.arrive + C.u)
+                       : "memory");
+          (void)c;
+          uint4 ua0 = make_uint4(0u, 0u, 0u, 0u), ua1 = ua0;
+          if (c_lane) {
+            const uint4 *src = reinterpret_cast<const uint4 *>(
+                p.amax + static_cast<int64_t>(C.i) * p.cols + cc0 + 8 * lane);
+            ua0 = __ldcg(src);
+            ua1 = __ldcg(src + 1);
+          }
+          const uint32_t a[8] = {ua0.x, ua0.y, ua0.z, ua0.w, ua1.x, ua1.y, ua1.z, ua1.w};
+  #pragma unroll
+          for (int j = 0; j < 8; ++j) s[j] = scale_from_amax(bf16_bits_to_float(a[j]), p.smax);
+          if (C.b == 0 && w == 0 && c_lane)
+            store_scales8(p.scales_col + static_cast<int64_t>(C.e) * p.cols + cc0 + 8 * lane, s);
+        } else {
+          failed = true;
+        }
+      }
+      uint4 v[kWR];
+      int32_t c_r1 = 0, c_rw0 = 0;
+      if (has_c && !failed) {
+        const int32_t gs = C.e ? sm.end[C.e - 1] : 0;
+        const int32_t r0 = gs + C.b * kRB;
+        c_r1 = min(sm.end[C.e], r0 + kRB);
+        c_rw0 = r0 + kWR * w;
+        const uint4 *src = p.x + static_cast<int64_t>(c_rw0) * p.ld_x16 + (cc0 >> 3) + lane;
+  #pragma unroll
+        for (int k = 0; k < kWR; ++k)
+          v[k] = (c_lane && c_rw0 + k < c_r1) ? __ldcs(src + k * p.ld_x16)
+                                              : make_uint4(0u, 0u, 0u, 0u);
+      }
+      if (has_c && !failed) {
+        tile_col_codes<FMT, FAST>(v, s, sm.tile, w, lane, p.smax, p.sat_thr, sat);
+        fence_proxy_async_smem();
+      }
+      if (__syncthreads_or(failed)) {
+        if (tid == 0) status_or(p.status, FP8QGG_STATUS_TIMEOUT);
+        break;  // this block takes no more steps
+      }
+      if (has_c && tid == 0) {
+        const int32_t ps = sm.pstart[C.e] + C.b * kRB;
+        tma_store_2d(&qmap, sm.tile, ps, cc0);
+        bulk_commit();
+      }
+    }
+  } else {
+    // The dual form loads each block early: the absmax block's rows at the end
+    // of the previous step (under the end-of-step barrier and the store), the
+    // cast block's as soon as the absmax has read them (under the mid-step
+    // barrier); its longer step gains from the overlap (185 -> 177 us on the
+    // DeepSeek-MoE-16B grad_out).  Early loads need the next step's blocks a
+    // step in advance: they are decoded two steps ahead (three slots).
+    constexpr int kSlots = 3;
+    // thread 0 claims this block's steps from the counter, in increasing order;
+    // each is published in sm.nstep and decoded two steps before it runs
+    int32_t next = 0;
+    auto claim = [&]() {
+      sm.nstep = next;
+      if (next < steps) next = static_cast<int32_t>(atomicAdd(p.work, 1u));
+    };
+    if (tid == 0) {
+      next = static_cast<int32_t>(atomicAdd(p.work, 1u));
+      claim();
+    }
+    __syncthreads();
+    decode_ahead<DUAL>(sm, 0, np, w, lane, total, delay, steps);
+    __syncthreads();
     if (tid == 0) claim();
     __syncthreads();
     decode_ahead<DUAL>(sm, 1, np, w, lane, total, delay, steps);
     __syncthreads();
-  }
 
-  // The block's rows, 16 per warp (the dual form's v lives across steps).
-  uint4 v[kWR];
-  // (every call defines all of v, zeros when there is no block, so that no
-  // earlier contents stay live)
-  auto load_rows = [&](uint4 (&dst)[kWR], const PBlock &B, bool has, bool streaming) {
-    const int32_t gs = B.e ? sm.end[B.e - 1] : 0;
-    const int32_t r0 = gs + B.b * kRB;
-    const int32_t r1 = has ? min(sm.end[B.e], r0 + kRB) : 0;
-    const int32_t rw0 = r0 + kWR * w;
-    const int c0 = B.q * kPW;
-    const bool lane_ok = c0 + 8 * lane < p.cols;
-    const uint4 *src = p.x + static_cast<int64_t>(rw0) * p.ld_x16 + (c0 >> 3) + lane;
-#pragma unroll
-    for (int k = 0; k < kWR; ++k) {
-      const bool ok = lane_ok && rw0 + k < r1;
-      dst[k] = !ok ? make_uint4(0u, 0u, 0u, 0u)
-                   : streaming ? __ldcs(src + k * p.ld_x16) : __ldcg(src + k * p.ld_x16);
-    }
-  };
-  auto load_a = [&](int slot) {  // the absmax block of the step in this slot
-    PBlock B{};
-    const bool has = sm.sidx[slot] < total;
-    if (has) memcpy(&B, sm.dA[slot], sizeof B);
-    load_rows(v, B, has, false);
-  };
-  if constexpr (kEarly) load_a(0);
-  for (int slot = 0;; slot = slot == kSlots - 1 ? 0 : slot + 1) {
-    // a step is bracketed by two block barriers: the one after the absmax
-    // (which also publishes the cast's column scales and the index of the
-    // step decoded next) and the one before the tile's store
-    const int slot1 = slot == kSlots - 1 ? 0 : slot + 1;
-    const int slot_dec = kSlots == 3 ? (slot1 == 2 ? 0 : slot1 + 1) : slot1;
-    const int32_t st = sm.sidx[slot];
-    if (st >= steps) break;
-    if (tid == 0) claim();
-    const bool has_a = st < total;
-    const bool has_c = st >= delay;
-    PBlock A{}, C{};
-    if (has_a) memcpy(&A, sm.dA[slot], sizeof A);
-    if (has_c) memcpy(&C, sm.dC[slot], sizeof C);
-    // (the column-wise form: the step's own arrays, as it loads them in place)
-    uint4 va[kWR], vc[kWR];
-    uint4 (&vA)[kWR] = kEarly ? v : va;
-    uint4 (&vC)[kWR] = kEarly ? v : vc;
-    if constexpr (!kEarly) load_rows(vA, A, has_a, false);
-
-    // the cast's scale words, early when the unit is complete already: each
-    // warp derives the scales of 32 of the panel's columns
-    bool c_ready = false;
-    uint32_t uword = 0, urow = 0;
-    const int cc0 = C.q * kPW;
-    const bool c_lane = has_c && cc0 + 8 * lane < p.cols;
-    const int ccol = cc0 + 32 * w + lane;  // this lane's scale column
-    if (has_c) {
-      uint32_t cnt = 0;
-      if (lane == 0)
-        asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(cnt) : "l"(p.arrive + C.u)
-                     : "memory");
-      c_ready = __shfl_sync(0xFFFFFFFFu, cnt, 0) >= static_cast<uint32_t>(C.need) +
-                                                     p.uw.extra_arrivals;
-    }
-    auto load_row_word = [&]() {
-      if constexpr (DUAL) {
-        const int32_t cgs = C.e ? sm.end[C.e - 1] : 0;
-        const int32_t row = cgs + C.b * kRB + kWR * w + lane;
-        const int32_t r1 = min(sm.end[C.e], cgs + C.b * kRB + kRB);
-        urow = (lane < kWR && row < r1) ? __ldcg(p.rowmax + row) : 0u;
+    // The block's rows, 16 per warp (v lives across steps).
+    uint4 v[kWR];
+    // (every call defines all of v, zeros when there is no block, so that no
+    // earlier contents stay live)
+    auto load_rows = [&](uint4 (&dst)[kWR], const PBlock &B, bool has, bool streaming) {
+      const int32_t gs = B.e ? sm.end[B.e - 1] : 0;
+      const int32_t r0 = gs + B.b * kRB;
+      const int32_t r1 = has ? min(sm.end[B.e], r0 + kRB) : 0;
+      const int32_t rw0 = r0 + kWR * w;
+      const int c0 = B.q * kPW;
+      const bool lane_ok = c0 + 8 * lane < p.cols;
+      const uint4 *src = p.x + static_cast<int64_t>(rw0) * p.ld_x16 + (c0 >> 3) + lane;
+  #pragma unroll
+      for (int k = 0; k < kWR; ++k) {
+        const bool ok = lane_ok && rw0 + k < r1;
+        dst[k] = !ok ? make_uint4(0u, 0u, 0u, 0u)
+                     : streaming ? __ldcs(src + k * p.ld_x16) : __ldcg(src + k * p.ld_x16);
       }
     };
-    if (c_ready) {
-      uword = ccol < p.cols ? __ldcg(p.amax + static_cast<int64_t>(C.i) * p.cols + ccol) : 0u;
-      load_row_word();
-    }
+    auto load_a = [&](int slot) {  // the absmax block of the step in this slot
+      PBlock B{};
+      const bool has = sm.sidx[slot] < total;
+      if (has) memcpy(&B, sm.dA[slot], sizeof B);
+      load_rows(v, B, has, false);
+    };
+    load_a(0);
+    for (int slot = 0;; slot = slot == kSlots - 1 ? 0 : slot + 1) {
+      // a step is bracketed by two block barriers: the one after the absmax
+      // (which also publishes the cast's column scales and the index of the
+      // step decoded next) and the one before the tile's store
+      const int slot1 = slot == kSlots - 1 ? 0 : slot + 1;
+      const int slot_dec = slot1 == 2 ? 0 : slot1 + 1;
+      const int32_t st = sm.sidx[slot];
+      if (st >= steps) break;
+      if (tid == 0) claim();
+      const bool has_a = st < total;
+      const bool has_c = st >= delay;
+      PBlock A{}, C{};
+      if (has_a) memcpy(&A, sm.dA[slot], sizeof A);
+      if (has_c) memcpy(&C, sm.dC[slot], sizeof C);
 
-    // ---------------------------------------------------------- absmax of block s
-    if (has_a) {
-      const int32_t gs = A.e ? sm.end[A.e - 1] : 0;
-      const int32_t r0 = gs + A.b * kRB;
-      const int32_t r1 = min(sm.end[A.e], r0 + kRB);
-      const int32_t rw0 = r0 + kWR * w;
-      uint4 am = make_uint4(0u, 0u, 0u, 0u);
-#pragma unroll
-      for (int k = 0; k < kWR; ++k) {
-        am.x = absmax_acc(am.x, vA[k].x);
-        am.y = absmax_acc(am.y, vA[k].y);
-        am.z = absmax_acc(am.z, vA[k].z);
-        am.w = absmax_acc(am.w, vA[k].w);
-      }
-      if constexpr (DUAL) merge_row_amax(vA, p.rowmax, rw0, r1, lane);
-      *reinterpret_cast<uint4 *>(&sm.red[w][4 * lane]) =
-          make_uint4(absmax_bits(am.x), absmax_bits(am.y), absmax_bits(am.z),
-                     absmax_bits(am.w));
-    }
-    // the cast block's rows (read-only input: no need to wait for its unit)
-    auto load_c = [&]() { load_rows(vC, C, has_c, true); };
-    if constexpr (kEarly) load_c();
-    if (c_ready) {
-      const float sc = scale_from_amax(bf16_bits_to_float(uword), p.smax);
-      sm.cscale[32 * w + lane] = sc;
-      if (C.b == 0 && ccol < p.cols) p.scales_col[static_cast<int64_t>(C.e) * p.cols + ccol] = sc;
-    }
-    if (tid == 0) bulk_wait_read<0>();  // the previous store has read the tile
-    const bool all_ready = __syncthreads_and(!has_c || c_ready) != 0;
-    if (has_a) {
-      // each warp merges 32 of the panel's columns into the unit's absmax:
-      // column 32w + lane is half (lane & 1) of word 16w + lane / 2
-      const int wd = 16 * w + (lane >> 1);
-      uint32_t m = 0;
-#pragma unroll
-      for (int ww = 0; ww < kPWarps; ++ww) m = __vmaxu2(m, sm.red[ww][wd]);
-      const int c0 = A.q * kPW;
-      const int cc = 32 * w + lane;
-      if (c0 + cc < p.cols)
-        atomicMax(p.amax + static_cast<int64_t>(A.i) * p.cols + c0 + cc,
-                  (lane & 1) ? m >> 16 : m & 0xFFFFu);
-      // every warp's merges happen before warp 0's one release of the count
-      // (a named barrier: the other warps arrive without waiting and go on to
-      // the cast; the release orders their merges too, being cumulative over
-      // the barrier)
-      __syncwarp();
-      if (w != 0) {
-        asm volatile("bar.arrive 2, %0;" ::"n"(kPThreads) : "memory");
-      } else {
-        asm volatile("bar.sync 2, %0;" ::"n"(kPThreads) : "memory");
+      // the cast's scale words, early when the unit is complete already: each
+      // warp derives the scales of 32 of the panel's columns
+      bool c_ready = false;
+      uint32_t uword = 0, urow = 0;
+      const int cc0 = C.q * kPW;
+      const bool c_lane = has_c && cc0 + 8 * lane < p.cols;
+      const int ccol = cc0 + 32 * w + lane;  // this lane's scale column
+      if (has_c) {
+        uint32_t cnt = 0;
         if (lane == 0)
-          asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p.arrive + A.u),
-                       "n"(kPWarps)
+          asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(cnt) : "l"(p.arrive + C.u)
                        : "memory");
+        c_ready = __shfl_sync(0xFFFFFFFFu, cnt, 0) >= static_cast<uint32_t>(C.need) +
+                                                       p.uw.extra_arrivals;
       }
-    }
-    decode_ahead<DUAL>(sm, slot_dec, np, w, lane, total, delay, steps);
+      auto load_row_word = [&]() {
+        if constexpr (DUAL) {
+          const int32_t cgs = C.e ? sm.end[C.e - 1] : 0;
+          const int32_t row = cgs + C.b * kRB + kWR * w + lane;
+          const int32_t r1 = min(sm.end[C.e], cgs + C.b * kRB + kRB);
+          urow = (lane < kWR && row < r1) ? __ldcg(p.rowmax + row) : 0u;
+        }
+      };
+      if (c_ready) {
+        uword = ccol < p.cols ? __ldcg(p.amax + static_cast<int64_t>(C.i) * p.cols + ccol) : 0u;
+        load_row_word();
+      }
 
-    // ---------------------------------------------------------- cast of block s - D
-    bool failed = false;
-    float s[8];
-    if (has_c && all_ready) {
-      const float4 s0 = *reinterpret_cast<const float4 *>(&sm.cscale[8 * lane]);
-      const float4 s1 = *reinterpret_cast<const float4 *>(&sm.cscale[8 * lane + 4]);
-      s[0] = s0.x; s[1] = s0.y; s[2] = s0.z; s[3] = s0.w;
-      s[4] = s1.x; s[5] = s1.y; s[6] = s1.z; s[7] = s1.w;
-    } else if (has_c) {  // wait (bounded) until every block of the unit is counted
-      int ok = 1;
-      if (lane == 0) {
-        const uint32_t target = static_cast<uint32_t>(C.need) + p.uw.extra_arrivals;
-        const uint64_t t0 = global_timer_ns();
-        while (true) {
-          uint32_t c;
+      // ---------------------------------------------------------- absmax of block s
+      if (has_a) {
+        const int32_t gs = A.e ? sm.end[A.e - 1] : 0;
+        const int32_t r0 = gs + A.b * kRB;
+        const int32_t r1 = min(sm.end[A.e], r0 + kRB);
+        const int32_t rw0 = r0 + kWR * w;
+        uint4 am = make_uint4(0u, 0u, 0u, 0u);
+  #pragma unroll
+        for (int k = 0; k < kWR; ++k) {
+          am.x = absmax_acc(am.x, v[k].x);
+          am.y = absmax_acc(am.y, v[k].y);
+          am.z = absmax_acc(am.z, v[k].z);
+          am.w = absmax_acc(am.w, v[k].w);
+        }
+        if constexpr (DUAL) merge_row_amax(v, p.rowmax, rw0, r1, lane);
+        *reinterpret_cast<uint4 *>(&sm.red[w][4 * lane]) =
+            make_uint4(absmax_bits(am.x), absmax_bits(am.y), absmax_bits(am.z),
+                       absmax_bits(am.w));
+      }
+      // the cast block's rows (read-only input: no need to wait for its unit)
+      auto load_c = [&]() { load_rows(v, C, has_c, true); };
+      load_c();
+      if (c_ready) {
+        const float sc = scale_from_amax(bf16_bits_to_float(uword), p.smax);
+        sm.cscale[32 * w + lane] = sc;
+        if (C.b == 0 && ccol < p.cols) p.scales_col[static_cast<int64_t>(C.e) * p.cols + ccol] = sc;
+      }
+      if (tid == 0) bulk_wait_read<0>();  // the previous store has read the tile
+      const bool all_ready = __syncthreads_and(!has_c || c_ready) != 0;
+      if (has_a) {
+        // each warp merges 32 of the panel's columns into the unit's absmax:
+        // column 32w + lane is half (lane & 1) of word 16w + lane / 2
+        const int wd = 16 * w + (lane >> 1);
+        uint32_t m = 0;
+  #pragma unroll
+        for (int ww = 0; ww < kPWarps; ++ww) m = __vmaxu2(m, sm.red[ww][wd]);
+        const int c0 = A.q * kPW;
+        const int cc = 32 * w + lane;
+        if (c0 + cc < p.cols)
+          atomicMax(p.amax + static_cast<int64_t>(A.i) * p.cols + c0 + cc,
+                    (lane & 1) ? m >> 16 : m & 0xFFFFu);
+        // every warp's merges happen before warp 0's one release of the count
+        // (a named barrier: the other warps arrive without waiting and go on to
+        // the cast; the release orders their merges too, being cumulative over
+        // the barrier)
+        __syncwarp();
+        if (w != 0) {
+          asm volatile("bar.arrive 2, %0;" ::"n"(kPThreads) : "memory");
+        } else {
+          asm volatile("bar.sync 2, %0;" ::"n"(kPThreads) : "memory");
+          if (lane == 0)
+            asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p.arrive + A.u),
+                         "n"(kPWarps)
+                         : "memory");
+        }
+      }
+      decode_ahead<DUAL>(sm, slot_dec, np, w, lane, total, delay, steps);
+
+      // ---------------------------------------------------------- cast of block s - D
+      bool failed = false;
+      float s[8];
+      if (has_c && all_ready) {
+        const float4 s0 = *reinterpret_cast<const float4 *>(&sm.cscale[8 * lane]);
+        const float4 s1 = *reinterpret_cast<const float4 *>(&sm.cscale[8 * lane + 4]);
+        s[0] = s0.x; s[1] = s0.y; s[2] = s0.z; s[3] = s0.w;
+        s[4] = s1.x; s[5] = s1.y; s[6] = s1.z; s[7] = s1.w;
+      } else if (has_c) {  // wait (bounded) until every block of the unit is counted
+        int ok = 1;
+        if (lane == 0) {
+          const uint32_t target = static_cast<uint32_t>(C.need) + p.uw.extra_arrivals;
+          const uint64_t t0 = global_timer_ns();
+          while (true) {
+            uint32_t c;
+            asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(c) : "l"(p.arrive + C.u)
+                         : "memory");
+            if (c >= target) break;
+            if (global_timer_ns() - t0 > p.uw.limit_ns) { ok = 0; break; }
+            __nanosleep(64);
+          }
+        }
+        ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+        if (ok) {
+          uint32_t c;  // every lane acquires the count it relies on
           asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(c) : "l"(p.arrive + C.u)
                        : "memory");
-          if (c >= target) break;
-          if (global_timer_ns() - t0 > p.uw.limit_ns) { ok = 0; break; }
-          __nanosleep(64);
-        }
-      }
-      ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
-      if (ok) {
-        uint32_t c;  // every lane acquires the count it relies on
-        asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(c) : "l"(p.arrive + C.u)
-                     : "memory");
-        (void)c;
-        uint4 ua0 = make_uint4(0u, 0u, 0u, 0u), ua1 = ua0;
-        if (c_lane) {
-          const uint4 *src = reinterpret_cast<const uint4 *>(
-              p.amax + static_cast<int64_t>(C.i) * p.cols + cc0 + 8 * lane);
-          ua0 = __ldcg(src);
-          ua1 = __ldcg(src + 1);
-        }
-        load_row_word();
-        const uint32_t a[8] = {ua0.x, ua0.y, ua0.z, ua0.w, ua1.x, ua1.y, ua1.z, ua1.w};
-#pragma unroll
-        for (int j = 0; j < 8; ++j) s[j] = scale_from_amax(bf16_bits_to_float(a[j]), p.smax);
-        if (C.b == 0 && w == 0 && c_lane)
-          store_scales8(p.scales_col + static_cast<int64_t>(C.e) * p.cols + cc0 + 8 * lane, s);
-      } else {
-        failed = true;
-      }
-    }
-    if constexpr (!kEarly) load_c();
-    if (has_c && !failed) {
-      if constexpr (DUAL) {
-        const int32_t cgs = C.e ? sm.end[C.e - 1] : 0;
-        const int32_t r1 = min(sm.end[C.e], cgs + C.b * kRB + kRB);
-        const int32_t rw0 = cgs + C.b * kRB + kWR * w;
-        float rs_lane = 0.0f;  // the scale of row rw0 + lane (lanes 0..15)
-        if (lane < kWR && rw0 + lane < r1) {
-          rs_lane = scale_from_amax(bf16_bits_to_float(urow), p.smax);
-          if (C.q == 0) p.scales_row[rw0 + lane] = rs_lane;
-        }
-        // rowwise codes in place: 8 columns of a row per lane, one 8-byte store
-#pragma unroll
-        for (int k = 0; k < kWR; ++k) {
-          const float rs = __shfl_sync(0xFFFFFFFFu, rs_lane, k);
-          uint32_t c2[4];
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const uint32_t wd = word(vC[k], j);
-            c2[j] = enc_pair<FMT, FAST>(lo_f(wd), hi_f(wd), rs, rs, p.smax, p.sat_thr, sat);
+          (void)c;
+          uint4 ua0 = make_uint4(0u, 0u, 0u, 0u), ua1 = ua0;
+          if (c_lane) {
+            const uint4 *src = reinterpret_cast<const uint4 *>(
+                p.amax + static_cast<int64_t>(C.i) * p.cols + cc0 + 8 * lane);
+            ua0 = __ldcg(src);
+            ua1 = __ldcg(src + 1);
           }
-          if (c_lane && rw0 + k < r1)
-            *reinterpret_cast<uint2 *>(p.q_row + static_cast<int64_t>(rw0 + k) * p.ld_qr +
-                                       cc0 + 8 * lane) =
-                make_uint2(c2[0] | (c2[1] << 16), c2[2] | (c2[3] << 16));
+          load_row_word();
+          const uint32_t a[8] = {ua0.x, ua0.y, ua0.z, ua0.w, ua1.x, ua1.y, ua1.z, ua1.w};
+  #pragma unroll
+          for (int j = 0; j < 8; ++j) s[j] = scale_from_amax(bf16_bits_to_float(a[j]), p.smax);
+          if (C.b == 0 && w == 0 && c_lane)
+            store_scales8(p.scales_col + static_cast<int64_t>(C.e) * p.cols + cc0 + 8 * lane, s);
+        } else {
+          failed = true;
         }
       }
-      tile_col_codes<FMT, FAST>(vC, s, sm.tile, w, lane, p.smax, p.sat_thr, sat);
-      fence_proxy_async_smem();
-    }
-    if constexpr (kEarly) {
+      if (has_c && !failed) {
+        if constexpr (DUAL) {
+          const int32_t cgs = C.e ? sm.end[C.e - 1] : 0;
+          const int32_t r1 = min(sm.end[C.e], cgs + C.b * kRB + kRB);
+          const int32_t rw0 = cgs + C.b * kRB + kWR * w;
+          float rs_lane = 0.0f;  // the scale of row rw0 + lane (lanes 0..15)
+          if (lane < kWR && rw0 + lane < r1) {
+            rs_lane = scale_from_amax(bf16_bits_to_float(urow), p.smax);
+            if (C.q == 0) p.scales_row[rw0 + lane] = rs_lane;
+          }
+          // rowwise codes in place: 8 columns of a row per lane, one 8-byte store
+  #pragma unroll
+          for (int k = 0; k < kWR; ++k) {
+            const float rs = __shfl_sync(0xFFFFFFFFu, rs_lane, k);
+            uint32_t c2[4];
+  #pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const uint32_t wd = word(v[k], j);
+              c2[j] = enc_pair<FMT, FAST>(lo_f(wd), hi_f(wd), rs, rs, p.smax, p.sat_thr, sat);
+            }
+            if (c_lane && rw0 + k < r1)
+              *reinterpret_cast<uint2 *>(p.q_row + static_cast<int64_t>(rw0 + k) * p.ld_qr +
+                                         cc0 + 8 * lane) =
+                  make_uint2(c2[0] | (c2[1] << 16), c2[2] | (c2[3] << 16));
+          }
+        }
+        tile_col_codes<FMT, FAST>(v, s, sm.tile, w, lane, p.smax, p.sat_thr, sat);
+        fence_proxy_async_smem();
+      }
       if (!failed) load_a(slot1);  // the next step's absmax block
-    }
-    if (__syncthreads_or(failed)) {
-      if (tid == 0) status_or(p.status, FP8QGG_STATUS_TIMEOUT);
-      break;  // this block takes no more steps
-    }
-    if (has_c && tid == 0) {
-      const int32_t ps = sm.pstart[C.e] + C.b * kRB;
-      tma_store_2d(&qmap, sm.tile, ps, cc0);
-      bulk_commit();
+      if (__syncthreads_or(failed)) {
+        if (tid == 0) status_or(p.status, FP8QGG_STATUS_TIMEOUT);
+        break;  // this block takes no more steps
+      }
+      if (has_c && tid == 0) {
+        const int32_t ps = sm.pstart[C.e] + C.b * kRB;
+        tma_store_2d(&qmap, sm.tile, ps, cc0);
+        bulk_commit();
+      }
     }
   }
   if (tid == 0) bulk_wait_all();  // the tile stays valid until its stores have read it
