@@ -45,7 +45,7 @@ constexpr int kGemmThreads = 64 + kEpiThreads;
 constexpr int kMaskWarp = kGemmThreads / 32;
 constexpr int kGemm1Threads = kGemmThreads + 32;
 constexpr int kMaxGemmGroups = 1024;
-constexpr int kBandRows = 2048;  // rows per raster band of tiles (token-jagged mode)
+constexpr int kBandRows = 4096;  // rows per raster band of tiles (token-jagged mode)
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kStageBytes = (BM + BN) * BK;
 constexpr uint32_t kIdesc = idesc_e4m3_f32(BM, BN);

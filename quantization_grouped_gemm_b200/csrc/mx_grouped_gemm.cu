@@ -55,7 +55,7 @@ constexpr int kMxEpiWarps = 8;
 constexpr int kMxEpiThreads = 32 * kMxEpiWarps;
 constexpr int kMxGemmThreads = 64 + kMxEpiThreads;
 constexpr int kMxGemmMaxGroups = 1024;
-constexpr int kMxBandRows = 2048;
+constexpr int kMxBandRows = 4096;
 constexpr uint32_t kMxTmemCols = 512;
 constexpr uint32_t kMxAccStride = 256;
 constexpr uint32_t kMxSfaCol = 496;
