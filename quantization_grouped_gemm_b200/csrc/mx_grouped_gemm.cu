@@ -35,10 +35,11 @@
 //              block-scaled MMAs (M128 N bn K32), each selecting its block's
 //              scale byte through the instruction descriptor.
 //   warps 2-9  epilogue: tcgen05.ld of the accumulator, bulk tensor stores.
-// TMEM: two accumulators of up to 224 columns at columns 0 and 256, the A
-// scales at 496 (4 columns), the B scales at 504 (8 columns).  bn (<= 224, a
-// multiple of 32) is chosen per call so that the N tiles cover N with little
-// waste.
+// TMEM: two accumulators of up to 240 columns at columns 0 and 256, the A
+// scales at 496 (4 columns), the B scales at 504 (8 columns).  bn (<= 240, a
+// multiple of 16 for fp32 output; <= 224, a multiple of 32, for bf16 output,
+// whose 64-byte store units are 32 columns wide) is chosen per call for the
+// fewest tiles with little waste.
 #include <algorithm>
 
 #include "device_common.cuh"
@@ -49,7 +50,7 @@ namespace fp8qgg {
 
 constexpr int kMxBM = 128;
 constexpr int kMxBK = 128;       // K bytes per stage = four 32-element blocks
-constexpr int kMxMaxBN = 224;
+constexpr int kMxMaxBN = 240;
 constexpr int kMxStages = 4;
 constexpr int kMxEpiWarps = 8;
 constexpr int kMxEpiThreads = 32 * kMxEpiWarps;
@@ -64,7 +65,7 @@ constexpr uint32_t kMxFullCount = 1 + 32;  // lane 0's expect-tx arrive + one pe
 
 struct MxGemmSmem {
   uint8_t a[kMxStages][kMxBM * kMxBK];      // 16 KB each, 1024-aligned
-  uint8_t b[kMxStages][kMxMaxBN * kMxBK];   // 28 KB each
+  uint8_t b[kMxStages][kMxMaxBN * kMxBK];   // 30 KB each
   uint8_t sfa[kMxStages][512];              // one 128-row chunk
   uint8_t sfb[kMxStages][1024];             // two 128-row chunks
   float stg[kMxEpiWarps][512];
@@ -80,6 +81,9 @@ struct MxGemmSmem {
   uint32_t tmem_base;
   int abort;
 };
+
+static_assert(sizeof(MxGemmSmem) + 1024 <= 232448, "one thread block's shared memory on sm_100a");
+static_assert(kMxMaxBN + kMxAccStride <= kMxSfaCol, "the second accumulator ends below the A scales");
 
 struct MxGemmParams {
   const uint32_t *sfa;  // scale words [stage group, ld_sa]
@@ -497,9 +501,21 @@ __global__ void __launch_bounds__(kMxGemmThreads, 1)
       const uint32_t taddr =
           tmem_base + (static_cast<uint32_t>(32 * quarter) << 16) + acc * kMxAccStride;
       for (int u = half; 32 * u < bn; u += 2) {
+        // a 16-column last chunk (fp32 output only) is loaded and stored alone,
+        // so that nothing past the tile's bn columns is read or written
+        const bool whole = 32 * u + 32 <= bn;
         uint32_t r[32];
         if (ti.nk > 0) {
-          tmem_ld_32x32b_x32(taddr + 32 * u, r);
+          if (whole) {
+            tmem_ld_32x32b_x32(taddr + 32 * u, r);
+          } else {
+            uint32_t h[16];
+            tmem_ld_32x32b_x16(taddr + 32 * u, h);
+#pragma unroll
+            for (int c = 0; c < 16; ++c) r[c] = h[c];
+#pragma unroll
+            for (int c = 16; c < 32; ++c) r[c] = 0u;
+          }
           tmem_ld_wait();
         } else {
 #pragma unroll
@@ -512,7 +528,7 @@ __global__ void __launch_bounds__(kMxGemmThreads, 1)
                                     static_cast<int32_t>(row0), ti.e, tma, out_base, row_stride,
                                     valid_rows, ncols, lane);
         if constexpr (OUT == FP8QGG_OUT_F32) {
-          if (cc + 16 < ncols)
+          if (whole && cc + 16 < ncols)
             emit_unit<MODE, OUT, false>(stg, &omap, r + 16, 1.f, ones,
                                         static_cast<int32_t>(cc + 16), static_cast<int32_t>(row0),
                                         ti.e, tma, out_base, row_stride, valid_rows, ncols, lane);
@@ -546,18 +562,22 @@ MxGemmKernel mx_gemm_kernel(int mode, int out_dtype) {
                                      : mx_grouped_gemm_kernel<FP8QGG_K_JAGGED, FP8QGG_OUT_BF16>;
 }
 
-// N tile width: a multiple of 32 up to 224, for the tile count (between the
-// fewest possible and four more) that computes the fewest columns, counting
-// 16 columns of fixed cost per tile.
-int mx_pick_bn(int64_t n) {
-  const int64_t t0 = (n + kMxMaxBN - 1) / kMxMaxBN;
-  int best_bn = kMxMaxBN;
+// N tile width: a multiple of `gran` (16 for fp32 output, 32 for bf16) up to
+// the widest such width that fits (240 / 224), for the tile count (between the
+// fewest possible and four more) of the lowest cost, counting 256 columns of
+// fixed cost per tile: on B200 a 128-deep stage takes about the same time at
+// any width from 128 to 224 columns (481 us at 224 and 531 us at 192 on the
+// Llama3-8B up-projection fit a fixed cost of some 330 columns).
+int mx_pick_bn(int64_t n, int gran) {
+  const int max_bn = kMxMaxBN / gran * gran;
+  const int64_t t0 = (n + max_bn - 1) / max_bn;
+  int best_bn = max_bn;
   int64_t best_cost = INT64_MAX;
   for (int64_t t = t0; t <= t0 + 4; ++t) {
-    const int64_t w = ((n + t - 1) / t + 31) / 32 * 32;
-    if (w > kMxMaxBN || w < 32) continue;
+    const int64_t w = std::max<int64_t>(32, ((n + t - 1) / t + gran - 1) / gran * gran);
+    if (w > max_bn) continue;
     const int64_t tiles = (n + w - 1) / w;
-    const int64_t cost = tiles * (w + 16);
+    const int64_t cost = tiles * (w + 256);
     if (cost < best_cost) {
       best_cost = cost;
       best_bn = static_cast<int>(w);
@@ -624,7 +644,7 @@ extern "C" int fp8_mx_grouped_gemm(int mode, const uint8_t *a, int64_t ld_a,
     return FP8QGG_ERR_ALIGN;
   if (kmode == FP8QGG_M_JAGGED && m_total == 0) return FP8QGG_OK;  // no rows: nothing to write
 
-  const int bn = mx_pick_bn(kmode == FP8QGG_M_JAGGED ? n : k);
+  const int bn = mx_pick_bn(kmode == FP8QGG_M_JAGGED ? n : k, out_dtype == FP8QGG_OUT_F32 ? 16 : 32);
   CUtensorMap amap, bmap;
   const uint32_t abox[2] = {kMxBK, kMxBM};
   if (kmode == FP8QGG_M_JAGGED) {

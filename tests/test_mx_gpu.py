@@ -181,8 +181,10 @@ def check_m_jagged(sizes, n, k, out_dtype=torch.float32, seed=1, full=True):
     ([300, 1, 129], 96, 160),        # K tail: 160 = 128 + 32
     ([0, 257, 0, 64], 224, 256),
     ([200, 200], 448, 128),          # two full 224-column tiles
-    ([130, 7], 200, 96),             # N tail inside the tile
+    ([130, 7], 200, 96),             # N tail inside the tile (a 208-column tile)
     ([1000], 64, 512),
+    ([260, 0, 33], 240, 128),        # one 240-column tile: its last 16 columns loaded alone
+    ([64, 200], 480, 96),            # two 240-column tiles
 ])
 def test_mx_gemm_m_jagged_every_element(sizes, n, k):
     check_m_jagged(sizes, n, k)
@@ -229,6 +231,8 @@ def check_k_jagged(sizes, n1, n2, out_dtype=torch.float32, seed=3):
     ([0, 1, 31, 32, 33, 129, 255], 128, 96),
     ([700, 3000], 136, 224),
     ([300, 300], 256, 448),
+    ([300, 0, 129], 96, 200),        # a 208-column tile: its last 16 columns loaded alone
+    ([200, 70], 128, 464),           # two 240-column tiles, the second cut at the edge
 ])
 def test_mx_gemm_k_jagged_padded_every_element(sizes, n1, n2):
     check_k_jagged(sizes, n1, n2)
