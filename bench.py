@@ -765,9 +765,9 @@ def run_gpu(args, world, rank, local):
 # is absent until the current kernel has been captured on it.
 TRAFFIC = {
     "llama3_8b_up_proj": 161937152 + 426585088,     # grouped_gemm_2sm_kernel<0>
-    "llama3_8b_up_proj_mxfp8": 157975040 + 426478080,  # mx_grouped_gemm_kernel<0, 0>
+    "llama3_8b_up_proj_mxfp8": 158574592 + 426209536,  # mx_grouped_gemm_kernel<0, 0>
     "deepseek_moe16b_bwd": 389905920 + 683739136,   # grouped_gemm_kernel<1, 0>, padded operands
-    "deepseek_moe16b_bwd_mxfp8": 414630144 + 683563776,  # mx_grouped_gemm_kernel<1, 0>
+    "deepseek_moe16b_bwd_mxfp8": 401601792 + 683939072,  # mx_grouped_gemm_kernel<1, 0>
 }
 
 
