@@ -356,11 +356,11 @@ __global__ void __launch_bounds__(kPThreads, kPBlocksPerSM)
         const bool lane_ok = c0 + 8 * lane < p.cols;
         const uint4 *src = p.x + static_cast<int64_t>(rw0) * p.ld_x16 + (c0 >> 3) + lane;
         uint4 v[kWR];
-  #pragma unroll
+#pragma unroll
         for (int k = 0; k < kWR; ++k)
           v[k] = (lane_ok && rw0 + k < r1) ? __ldcg(src + k * p.ld_x16) : make_uint4(0u, 0u, 0u, 0u);
         uint4 am = make_uint4(0u, 0u, 0u, 0u);
-  #pragma unroll
+#pragma unroll
         for (int k = 0; k < kWR; ++k) {
           am.x = absmax_acc(am.x, v[k].x);
           am.y = absmax_acc(am.y, v[k].y);
@@ -383,7 +383,7 @@ __global__ void __launch_bounds__(kPThreads, kPBlocksPerSM)
         // column 32w + lane is half (lane & 1) of word 16w + lane / 2
         const int wd = 16 * w + (lane >> 1);
         uint32_t m = 0;
-  #pragma unroll
+#pragma unroll
         for (int ww = 0; ww < kPWarps; ++ww) m = __vmaxu2(m, sm.red[ww][wd]);
         const int c0 = A.q * kPW;
         const int cc = 32 * w + lane;
@@ -443,7 +443,7 @@ __global__ void __launch_bounds__(kPThreads, kPBlocksPerSM)
             ua1 = __ldcg(src + 1);
           }
           const uint32_t a[8] = {ua0.x, ua0.y, ua0.z, ua0.w, ua1.x, ua1.y, ua1.z, ua1.w};
-  #pragma unroll
+#pragma unroll
           for (int j = 0; j < 8; ++j) s[j] = scale_from_amax(bf16_bits_to_float(a[j]), p.smax);
           if (C.b == 0 && w == 0 && c_lane)
             store_scales8(p.scales_col + static_cast<int64_t>(C.e) * p.cols + cc0 + 8 * lane, s);
@@ -459,7 +459,7 @@ __global__ void __launch_bounds__(kPThreads, kPBlocksPerSM)
         c_r1 = min(sm.end[C.e], r0 + kRB);
         c_rw0 = r0 + kWR * w;
         const uint4 *src = p.x + static_cast<int64_t>(c_rw0) * p.ld_x16 + (cc0 >> 3) + lane;
-  #pragma unroll
+#pragma unroll
         for (int k = 0; k < kWR; ++k)
           v[k] = (c_lane && c_rw0 + k < c_r1) ? __ldcs(src + k * p.ld_x16)
                                               : make_uint4(0u, 0u, 0u, 0u);
@@ -517,7 +517,7 @@ __global__ void __launch_bounds__(kPThreads, kPBlocksPerSM)
       const int c0 = B.q * kPW;
       const bool lane_ok = c0 + 8 * lane < p.cols;
       const uint4 *src = p.x + static_cast<int64_t>(rw0) * p.ld_x16 + (c0 >> 3) + lane;
-  #pragma unroll
+#pragma unroll
       for (int k = 0; k < kWR; ++k) {
         const bool ok = lane_ok && rw0 + k < r1;
         dst[k] = !ok ? make_uint4(0u, 0u, 0u, 0u)
@@ -581,7 +581,7 @@ __global__ void __launch_bounds__(kPThreads, kPBlocksPerSM)
         const int32_t r1 = min(sm.end[A.e], r0 + kRB);
         const int32_t rw0 = r0 + kWR * w;
         uint4 am = make_uint4(0u, 0u, 0u, 0u);
-  #pragma unroll
+#pragma unroll
         for (int k = 0; k < kWR; ++k) {
           am.x = absmax_acc(am.x, v[k].x);
           am.y = absmax_acc(am.y, v[k].y);
@@ -608,7 +608,7 @@ __global__ void __launch_bounds__(kPThreads, kPBlocksPerSM)
         // column 32w + lane is half (lane & 1) of word 16w + lane / 2
         const int wd = 16 * w + (lane >> 1);
         uint32_t m = 0;
-  #pragma unroll
+#pragma unroll
         for (int ww = 0; ww < kPWarps; ++ww) m = __vmaxu2(m, sm.red[ww][wd]);
         const int c0 = A.q * kPW;
         const int cc = 32 * w + lane;
@@ -669,7 +669,7 @@ __global__ void __launch_bounds__(kPThreads, kPBlocksPerSM)
           }
           load_row_word();
           const uint32_t a[8] = {ua0.x, ua0.y, ua0.z, ua0.w, ua1.x, ua1.y, ua1.z, ua1.w};
-  #pragma unroll
+#pragma unroll
           for (int j = 0; j < 8; ++j) s[j] = scale_from_amax(bf16_bits_to_float(a[j]), p.smax);
           if (C.b == 0 && w == 0 && c_lane)
             store_scales8(p.scales_col + static_cast<int64_t>(C.e) * p.cols + cc0 + 8 * lane, s);
@@ -688,11 +688,11 @@ __global__ void __launch_bounds__(kPThreads, kPBlocksPerSM)
             if (C.q == 0) p.scales_row[rw0 + lane] = rs_lane;
           }
           // rowwise codes in place: 8 columns of a row per lane, one 8-byte store
-  #pragma unroll
+#pragma unroll
           for (int k = 0; k < kWR; ++k) {
             const float rs = __shfl_sync(0xFFFFFFFFu, rs_lane, k);
             uint32_t c2[4];
-  #pragma unroll
+#pragma unroll
             for (int j = 0; j < 4; ++j) {
               const uint32_t wd = word(v[k], j);
               c2[j] = enc_pair<FMT, FAST>(lo_f(wd), hi_f(wd), rs, rs, p.smax, p.sat_thr, sat);
