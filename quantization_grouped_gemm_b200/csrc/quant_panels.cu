@@ -561,13 +561,11 @@ __global__ void __launch_bounds__(kPThreads, kPBlocksPerSM)
         c_ready = __shfl_sync(0xFFFFFFFFu, cnt, 0) >= static_cast<uint32_t>(C.need) +
                                                        p.uw.extra_arrivals;
       }
-      auto load_row_word = [&]() {
-        if constexpr (DUAL) {
-          const int32_t cgs = C.e ? sm.end[C.e - 1] : 0;
-          const int32_t row = cgs + C.b * kRB + kWR * w + lane;
-          const int32_t r1 = min(sm.end[C.e], cgs + C.b * kRB + kRB);
-          urow = (lane < kWR && row < r1) ? __ldcg(p.rowmax + row) : 0u;
-        }
+      auto load_row_word = [&]() {  // the row absmax word of row rw0 + lane (lanes 0..15)
+        const int32_t cgs = C.e ? sm.end[C.e - 1] : 0;
+        const int32_t row = cgs + C.b * kRB + kWR * w + lane;
+        const int32_t r1 = min(sm.end[C.e], cgs + C.b * kRB + kRB);
+        urow = (lane < kWR && row < r1) ? __ldcg(p.rowmax + row) : 0u;
       };
       if (c_ready) {
         uword = ccol < p.cols ? __ldcg(p.amax + static_cast<int64_t>(C.i) * p.cols + ccol) : 0u;
@@ -588,14 +586,13 @@ __global__ void __launch_bounds__(kPThreads, kPBlocksPerSM)
           am.z = absmax_acc(am.z, v[k].z);
           am.w = absmax_acc(am.w, v[k].w);
         }
-        if constexpr (DUAL) merge_row_amax(v, p.rowmax, rw0, r1, lane);
+        merge_row_amax(v, p.rowmax, rw0, r1, lane);
         *reinterpret_cast<uint4 *>(&sm.red[w][4 * lane]) =
             make_uint4(absmax_bits(am.x), absmax_bits(am.y), absmax_bits(am.z),
                        absmax_bits(am.w));
       }
       // the cast block's rows (read-only input: no need to wait for its unit)
-      auto load_c = [&]() { load_rows(v, C, has_c, true); };
-      load_c();
+      load_rows(v, C, has_c, true);
       if (c_ready) {
         const float sc = scale_from_amax(bf16_bits_to_float(uword), p.smax);
         sm.cscale[32 * w + lane] = sc;
@@ -678,30 +675,28 @@ __global__ void __launch_bounds__(kPThreads, kPBlocksPerSM)
         }
       }
       if (has_c && !failed) {
-        if constexpr (DUAL) {
-          const int32_t cgs = C.e ? sm.end[C.e - 1] : 0;
-          const int32_t r1 = min(sm.end[C.e], cgs + C.b * kRB + kRB);
-          const int32_t rw0 = cgs + C.b * kRB + kWR * w;
-          float rs_lane = 0.0f;  // the scale of row rw0 + lane (lanes 0..15)
-          if (lane < kWR && rw0 + lane < r1) {
-            rs_lane = scale_from_amax(bf16_bits_to_float(urow), p.smax);
-            if (C.q == 0) p.scales_row[rw0 + lane] = rs_lane;
-          }
-          // rowwise codes in place: 8 columns of a row per lane, one 8-byte store
+        const int32_t cgs = C.e ? sm.end[C.e - 1] : 0;
+        const int32_t r1 = min(sm.end[C.e], cgs + C.b * kRB + kRB);
+        const int32_t rw0 = cgs + C.b * kRB + kWR * w;
+        float rs_lane = 0.0f;  // the scale of row rw0 + lane (lanes 0..15)
+        if (lane < kWR && rw0 + lane < r1) {
+          rs_lane = scale_from_amax(bf16_bits_to_float(urow), p.smax);
+          if (C.q == 0) p.scales_row[rw0 + lane] = rs_lane;
+        }
+        // rowwise codes in place: 8 columns of a row per lane, one 8-byte store
 #pragma unroll
-          for (int k = 0; k < kWR; ++k) {
-            const float rs = __shfl_sync(0xFFFFFFFFu, rs_lane, k);
-            uint32_t c2[4];
+        for (int k = 0; k < kWR; ++k) {
+          const float rs = __shfl_sync(0xFFFFFFFFu, rs_lane, k);
+          uint32_t c2[4];
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              const uint32_t wd = word(v[k], j);
-              c2[j] = enc_pair<FMT, FAST>(lo_f(wd), hi_f(wd), rs, rs, p.smax, p.sat_thr, sat);
-            }
-            if (c_lane && rw0 + k < r1)
-              *reinterpret_cast<uint2 *>(p.q_row + static_cast<int64_t>(rw0 + k) * p.ld_qr +
-                                         cc0 + 8 * lane) =
-                  make_uint2(c2[0] | (c2[1] << 16), c2[2] | (c2[3] << 16));
+          for (int j = 0; j < 4; ++j) {
+            const uint32_t wd = word(v[k], j);
+            c2[j] = enc_pair<FMT, FAST>(lo_f(wd), hi_f(wd), rs, rs, p.smax, p.sat_thr, sat);
           }
+          if (c_lane && rw0 + k < r1)
+            *reinterpret_cast<uint2 *>(p.q_row + static_cast<int64_t>(rw0 + k) * p.ld_qr +
+                                       cc0 + 8 * lane) =
+                make_uint2(c2[0] | (c2[1] << 16), c2[2] | (c2[3] << 16));
         }
         tile_col_codes<FMT, FAST>(v, s, sm.tile, w, lane, p.smax, p.sat_thr, sat);
         fence_proxy_async_smem();
