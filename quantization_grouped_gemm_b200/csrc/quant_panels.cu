@@ -50,7 +50,7 @@ namespace fp8qgg {
 // Build-time knob: the pipeline delay beyond the longest unit, in quarters
 // of the grid (the default is the best of the values measured on B200).
 #ifndef FP8QGG_PANEL_DELAY_Q
-#define FP8QGG_PANEL_DELAY_Q 5
+#define FP8QGG_PANEL_DELAY_Q 4
 #endif
 
 constexpr int kPW = 256;               // columns per panel
@@ -179,7 +179,7 @@ __device__ void panel_prologue(PanelSmem &sm, const PanelParams &p, int np) {
       sm.n_nonempty = n_ne;
       sm.total = carry * np;
       // a unit's blocks are consecutive: the delay covers the longest unit and
-      // the steps the running blocks hold, with a quarter of margin
+      // the steps the running blocks hold (one grid width at the default)
       const int32_t span = DUAL ? nb_max * np : nb_max;
       sm.delay = min(sm.total, span + (FP8QGG_PANEL_DELAY_Q * static_cast<int32_t>(gridDim.x)) / 4);
     }
