@@ -27,16 +27,20 @@
 //  - reads block s - D again (from L2: D blocks ago is about one grid-width
 //    plus the longest unit, so the block is still there and its unit's count
 //    is normally full already; the block waits for it, bounded, otherwise),
-//    derives the scales from the unit's absmax, encodes two rows of a column
-//    per conversion and writes each column's 16 tokens into a 32 KB tile
+//    derives the scales from the unit's absmax (once per thread block: each
+//    warp 32 of the 256 columns, shared through shared memory), encodes two
+//    rows of a column per conversion and writes each column's 16 tokens into
+//    a 32 KB tile
 //    (256 columns x 128 tokens, 128-byte swizzle) that one bulk tensor store
 //    sends to the group's 128-token block of the padded layout: whole
 //    128-byte lines, zero codes of the padding included (rows past the
 //    group's end are zeros).  The dual form also encodes every row with its
 //    own scale and stores it in place.
-// Every block is read once from HBM.  A step only waits for steps handed out
-// earlier (to running thread blocks), so no thread block waits for one that
-// is not running.
+// A step has two block barriers (after the absmax, which also publishes the
+// scales; before the tile's store), and warps 1 and 2 decode the blocks of a
+// later step into shared memory while it runs.  Every block is read once from
+// HBM.  A step only waits for steps handed out earlier (to running thread
+// blocks), so no thread block waits for one that is not running.
 #include <algorithm>
 #include <cstring>
 
